@@ -1,0 +1,209 @@
+/*
+ * bq.h -- C ABI of the block-quantised weight GEMV library for B200 (sm_100a).
+ *
+ * The operation is the decode step of an LLM inference runtime: block-quantised
+ * weight matrices are streamed from HBM once per token and multiplied against
+ * a small batch of activation vectors, with the dequantisation done inside the
+ * dot-product loop so dequantised weights never exist in memory (BaseRT:
+ * Best-in-Class LLM Inference on Apple Silicon via Native Metal, gist.science
+ * technical summary, "Methodologie" -> "Kernel Fusie en Specialisatie"; the
+ * same page's "De 'Big Model' Realiteit" paragraph states that decode is
+ * bound by memory bandwidth).
+ *
+ *   y[b][n] = sum_k deq(W)[n][k] * x[b][k],   0 <= b < B <= 8,  0 <= n < N
+ *
+ * Block formats (32 consecutive weights along K share one fp16 scale d):
+ *   Q8: int8 code q, weight = d * q,        d = fp16(absmax / 127)
+ *   Q4: 4-bit code q, weight = d * (q - 8), d = fp16(absmax / 7); byte i
+ *       (0..15) of a block holds element i in its low nibble and element
+ *       i + 16 in its high nibble.
+ *
+ * Physical layout of a quantised matrix (bq_qmat), "planes":
+ *   codes  : Q4 uint8 [N][K/2], Q8 int8 [N][K]; row n at codes + n*(K/2) (Q4)
+ *            or codes + n*K (Q8); block j of a row at byte offset 16*j (Q4) or
+ *            32*j (Q8).
+ *   scales : fp16 bit patterns, [N][ldS] with ldS = bq_scales_ld(K) =
+ *            roundup(K/32, 8); entry (n, j) is the scale of block j of row n;
+ *            entries j >= K/32 are padding (ignored by the GEMV, written as 0
+ *            by the quantisers).  Every scale row therefore starts on a
+ *            16-byte boundary.
+ *   Both planes must start on a 16-byte boundary; K must be a multiple of 32.
+ *   bq_planes_to_blocks_* converts planes to the interleaved per-block form
+ *   (fp16 scale followed by the 16 or 32 code bytes) and back, bit-exactly.
+ *
+ * Activations x are fp16 bit patterns, [B][K] row-major (row b at x + b*K),
+ * 16-byte aligned.  Outputs y are fp32 [B][N] row-major, 16-byte aligned, and
+ * are overwritten (never accumulated).
+ *
+ * Conventions for every call:
+ *   - Ownership: the caller owns every buffer.  The library never allocates
+ *     device or pinned memory (the zero-allocation decode loop: gist.science
+ *     technical summary, "Methodologie" -> "Zero-Allocation Decode Loop").
+ *   - Pointers marked "device" are CUDA device pointers of the current
+ *     device; "host" pointers are ordinary CPU memory.
+ *   - GPU calls are asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and return after the launch.
+ *   - Workspace: calls that take `ws` need ws_bytes >= the matching
+ *     bq_*_workspace_bytes() value.  The workspace must be zero-filled once
+ *     (e.g. cudaMemsetAsync) before its first use; every call that completes
+ *     leaves its counters at zero again, so one zero-fill suffices.  Two calls
+ *     that may run at the same time must not share a workspace.
+ *   - Errors: the return code covers everything the host can check before
+ *     launching (null pointers, shapes, alignment, batch range, workspace
+ *     size) and launch failures; nothing is launched when it is not BQ_OK.
+ *     Errors the device detects (an expert index outside [0, E), a bounded
+ *     wait that ran out) are OR-ed as (1 << code) into *dev_status when
+ *     dev_status is not NULL; the caller reads it after synchronising.  The
+ *     device never traps.
+ *   - Results are deterministic for a given device, shape and batch: every
+ *     split sum is combined in a fixed order.
+ */
+#ifndef BQ_H
+#define BQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BQ_OK = 0,
+    BQ_ERR_NULL = 1,         /* a required pointer is NULL */
+    BQ_ERR_SHAPE = 2,        /* N < 1, K < 32, K % 32 != 0, topk/E out of range */
+    BQ_ERR_ALIGN = 3,        /* a pointer or stride is not 16-byte aligned */
+    BQ_ERR_BATCH = 4,        /* B outside [1, 8] (or B*topk > 64 for MoE) */
+    BQ_ERR_EXPERT_INDEX = 5, /* device: an expert index outside [0, E) */
+    BQ_ERR_CUDA = 6,         /* a CUDA runtime call or launch failed */
+    BQ_ERR_TIMEOUT = 7,      /* device: a bounded wait ran out */
+    BQ_ERR_WORKSPACE = 8,    /* ws NULL or smaller than required */
+    BQ_ERR_RANGE = 9         /* quantiser input not finite or scale overflows fp16 */
+} bq_status;
+
+/* A quantised matrix: N output rows, K inputs, in the plane layout above.
+ * codes and scales are device pointers for the GEMV calls and host pointers
+ * for the host-side pack/unpack calls. */
+typedef struct bq_qmat {
+    const void *codes;
+    const uint16_t *scales;
+    int32_t N;
+    int32_t K;
+} bq_qmat;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *bq_status_string(int32_t status);
+
+/* Entries per scale-plane row for a K-column matrix: roundup(K/32, 8).
+ * Returns 0 when K is not a positive multiple of 32. */
+int32_t bq_scales_ld(int32_t K);
+
+/* ---------------------------------------------------------------- GEMV --- */
+
+/* Bytes of workspace bq_gemv_q4 / bq_gemv_q8 need for an N x K matrix
+ * (independent of B and of the format).  0 on a bad shape. */
+size_t bq_gemv_workspace_bytes(int32_t N, int32_t K);
+
+/* Q4 decode GEMV: y[b][n] = sum_k d(n,k/32) * (q(n,k) - 8) * x[b][k].
+ * The operation is the per-format decode GEMV with dequantisation in the
+ * inner loop (gist.science technical summary, "Kernel Fusie en
+ * Specialisatie").
+ *   W          host pointer to a bq_qmat whose planes are device pointers
+ *   x          device, fp16 bits [B][K]
+ *   B          batch, 1..8
+ *   y          device, fp32 [B][N], overwritten
+ *   ws         device workspace, ws_bytes >= bq_gemv_workspace_bytes(N, K)
+ *   dev_status device int32 or NULL (see conventions)
+ *   stream     cudaStream_t
+ * The launch uses programmatic dependent launch: its weight prefetch may
+ * start while the previous kernel on the stream drains; x, y and ws are only
+ * touched after that kernel has completed. */
+int32_t bq_gemv_q4(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
+                   void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* Q8 decode GEMV: y[b][n] = sum_k d(n,k/32) * q(n,k) * x[b][k].
+ * Arguments as bq_gemv_q4. */
+int32_t bq_gemv_q8(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
+                   void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------ routed experts --- */
+
+/* Bytes of workspace bq_moe_gemv_q4 needs.  0 on a bad shape. */
+size_t bq_moe_workspace_bytes(int32_t N, int32_t K, int32_t B, int32_t topk, int32_t E);
+
+/* Grouped Q4 GEMV over routed experts (decode step of a mixture-of-experts
+ * layer; the pages discuss expert GEMMs in the technical summary's
+ * "Prefill Throughput" results for Qwen3-30B-A3B and in the follow-up
+ * paper's method paragraph).  Each routed expert's weights are streamed
+ * once and applied to every token routed to it.
+ *   Wstack        host pointer to a bq_qmat describing expert 0 (device
+ *                 planes); expert e's planes start at codes + e*codes_stride
+ *                 bytes and scales + e*scales_stride fp16 entries.
+ *                 codes_stride must be >= N*K/2 and a multiple of 16;
+ *                 scales_stride >= N*ldS and a multiple of 8.
+ *   E             number of experts (1..65535)
+ *   x             device fp16 bits: [B][K] (x_per_slot == 0, a token's input
+ *                 is shared by its experts) or [B][topk][K] (x_per_slot == 1)
+ *   expert_idx    device int32 [B][topk]
+ *   route_w       device fp32 [B][topk] or NULL
+ *   y             device fp32: route_w == NULL -> [B][topk][N] per-slot
+ *                 outputs y[b][s] = W_{idx[b][s]} x_{b,s};
+ *                 otherwise [B][N], y[b] = sum_s route_w[b][s] * W_{idx[b][s]} x_{b,s}
+ *                 summed in fp32 in slot order.
+ *   B, topk       1 <= B <= 8, 1 <= topk, B*topk <= 64
+ * A slot whose index lies outside [0, E) contributes zero (its per-slot
+ * output is zero) and sets bit BQ_ERR_EXPERT_INDEX in *dev_status. */
+int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t codes_stride,
+                       int64_t scales_stride, const uint16_t *x, int32_t x_per_slot,
+                       const int32_t *expert_idx, const float *route_w, int32_t B,
+                       int32_t topk, float *y, void *ws, size_t ws_bytes,
+                       int32_t *dev_status, void *stream);
+
+/* ---------------------------------------------- host-side pack / unpack --- */
+/* All host pointers; no CUDA call is made.  Bit-exact by construction. */
+
+/* Quantise fp32 weights [N][K] (row-major) into planes.  Per 32-block:
+ * a = max|w| (fp32), d = fp16_rne(a / 127) (Q8) or fp16_rne(a / 7) (Q4),
+ * q = round-half-away(w / d) clamped to [-127, 127] (Q8), or
+ * clamp(round-half-away(w / d) + 8, 0, 15) (Q4); a block whose fp16 scale is
+ * zero gets code 0 (Q8) or 8 (Q4).  codes: Q8 int8 [N][K], Q4 uint8 [N][K/2];
+ * scales: uint16 [N][bq_scales_ld(K)], padding written as 0.
+ * BQ_ERR_RANGE if an input is not finite or a scale overflows fp16. */
+int32_t bq_quantize_q8(const float *w, int32_t N, int32_t K, int8_t *codes, uint16_t *scales);
+int32_t bq_quantize_q4(const float *w, int32_t N, int32_t K, uint8_t *codes, uint16_t *scales);
+
+/* Dequantise planes into fp32 weights [N][K] (exact: d * q fits fp32). */
+int32_t bq_dequantize_q8(const int8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
+                         float *w);
+int32_t bq_dequantize_q4(const uint8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
+                         float *w);
+
+/* Planes <-> interleaved blocks.  blocks: N*(K/32) records, row-major over
+ * (n, j); each record is the fp16 scale (2 bytes, little-endian) followed by
+ * 16 code bytes (Q4, 18-byte records) or 32 code bytes (Q8, 34-byte records). */
+int32_t bq_planes_to_blocks_q4(const uint8_t *codes, const uint16_t *scales, int32_t N,
+                               int32_t K, uint8_t *blocks);
+int32_t bq_planes_to_blocks_q8(const int8_t *codes, const uint16_t *scales, int32_t N,
+                               int32_t K, uint8_t *blocks);
+int32_t bq_blocks_to_planes_q4(const uint8_t *blocks, int32_t N, int32_t K, uint8_t *codes,
+                               uint16_t *scales);
+int32_t bq_blocks_to_planes_q8(const uint8_t *blocks, int32_t N, int32_t K, int8_t *codes,
+                               uint16_t *scales);
+
+/* ------------------------------------------------ device-side quantiser --- */
+
+/* Same arithmetic as bq_quantize_q4 / _q8, on the GPU (for building large
+ * resident weight sets without a host round trip).  w: device fp32 [N][K];
+ * codes / scales: device planes.  Non-finite inputs or fp16-overflowing
+ * scales set bit BQ_ERR_RANGE in *dev_status (if not NULL) and produce the
+ * zero-point codes for that block. */
+int32_t bq_quantize_q4_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
+                           uint16_t *scales, int32_t *dev_status, void *stream);
+int32_t bq_quantize_q8_dev(const float *w, int32_t N, int32_t K, int8_t *codes,
+                           uint16_t *scales, int32_t *dev_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BQ_H */

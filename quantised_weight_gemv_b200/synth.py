@@ -1,0 +1,183 @@
+"""Seeded synthetic inputs and workload shapes.
+
+This module only draws random numbers and describes shapes.  It holds none of
+the GEMV's arithmetic (no quantisation, no packing, no dot products), so both
+the oracle side and the CUDA side of the tests, and the benchmark, may take
+their inputs from it.
+
+Distributions (stated with the workloads): weights w ~ N(0, 0.02) (0.02 is the
+standard deviation) drawn in fp32; activations x ~ N(0, 1) drawn in fp32 and
+rounded to fp16 (nearest-even); routed-expert indices drawn uniformly without
+replacement per token; routing weights are a softmax (fp64, stored as fp32) of
+N(0, 1) logits.  Every stream is keyed by
+``(seed, workload id, layer, matrix id, kind)``.
+
+Two generators: numpy ``default_rng`` for anything the CPU handles in
+seconds, and torch's CUDA Philox generator (seeded from the same key) for the
+multi-GB weight sets, which are then quantised on the device.
+"""
+from __future__ import annotations
+
+import dataclasses
+import hashlib
+from typing import List, Optional, Sequence, Tuple
+
+import numpy as np
+
+KIND_W, KIND_X, KIND_IDX, KIND_LOGIT, KIND_H = 0, 1, 2, 3, 4
+W_STD = 0.02
+
+
+def key(seed: int, workload: int, layer: int, matrix: int, kind: int) -> List[int]:
+    return [int(seed), int(workload), int(layer), int(matrix), int(kind)]
+
+
+def rng(k: Sequence[int]) -> np.random.Generator:
+    return np.random.default_rng(list(k))
+
+
+def torch_seed(k: Sequence[int]) -> int:
+    """63-bit seed for torch.Generator derived from the same key."""
+    h = hashlib.sha256((",".join(str(int(v)) for v in k)).encode()).digest()
+    return int.from_bytes(h[:8], "little") & ((1 << 63) - 1)
+
+
+# ------------------------------------------------------------- numpy side ----
+def weights_f32(k: Sequence[int], N: int, K: int) -> np.ndarray:
+    """fp32 [N, K], N(0, 0.02)."""
+    return (rng(k).standard_normal((N, K), dtype=np.float32) * np.float32(W_STD)).astype(np.float32)
+
+
+def activations_f16_bits(k: Sequence[int], *shape: int) -> np.ndarray:
+    """fp16 bit patterns (uint16) of N(0,1) fp32 draws rounded to nearest-even."""
+    x = rng(k).standard_normal(shape, dtype=np.float32)
+    return x.astype(np.float16).view(np.uint16)
+
+
+def routing(k_idx: Sequence[int], k_logit: Sequence[int], B: int, E: int, topk: int
+            ) -> Tuple[np.ndarray, np.ndarray]:
+    """(expert_idx int32 [B, topk], route_w float32 [B, topk]).
+
+    Indices: per token a uniform sample without replacement of topk of E.
+    Weights: softmax (fp64) over that token's topk N(0,1) logits, stored fp32.
+    """
+    r = rng(k_idx)
+    idx = np.stack([r.choice(E, size=topk, replace=False) for _ in range(B)]).astype(np.int32)
+    logits = rng(k_logit).standard_normal((B, topk))
+    ex = np.exp(logits - logits.max(axis=1, keepdims=True))
+    w = (ex / ex.sum(axis=1, keepdims=True)).astype(np.float32)
+    return idx, w
+
+
+# ------------------------------------------------------------- torch side ----
+def weights_f32_torch(k: Sequence[int], N: int, K: int, device):
+    """fp32 [N, K] N(0, 0.02) on `device`, from torch's generator for that device."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(torch_seed(k))
+    return torch.randn((N, K), generator=g, device=device, dtype=torch.float32).mul_(W_STD)
+
+
+def activations_f16_torch(k: Sequence[int], shape, device):
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(torch_seed(k))
+    return torch.randn(tuple(shape), generator=g, device=device, dtype=torch.float32).to(torch.float16)
+
+
+# -------------------------------------------------------------- workloads ----
+@dataclasses.dataclass(frozen=True)
+class Mat:
+    """One weight matrix of a decode step: N outputs x K inputs."""
+    name: str
+    N: int
+    K: int
+    stage: int          # stages run in order; matrices of one stage are independent
+
+
+@dataclasses.dataclass(frozen=True)
+class DenseWorkload:
+    wid: int            # workload id, part of every seed key
+    name: str
+    fmt: int            # 4 or 8
+    layers: int
+    mats: Tuple[Mat, ...]   # per-layer matrices, in model order
+    B: int = 1
+
+    def layer_weights(self) -> int:
+        return sum(m.N * m.K for m in self.mats)
+
+    def step_mats(self) -> List[Tuple[int, Mat]]:
+        """(layer, matrix) for a whole decode step, stage by stage in model order."""
+        n_st = 1 + max(m.stage for m in self.mats)
+        out = []
+        for l in range(self.layers):
+            for m in self.mats:
+                out.append((l, dataclasses.replace(m, stage=l * n_st + m.stage)))
+        return out
+
+
+def packed_bytes(fmt: int, N: int, K: int) -> int:
+    """Algorithmic bytes of one packed matrix: codes + scales (no padding)."""
+    codes = N * K // 2 if fmt == 4 else N * K
+    return codes + N * (K // 32) * 2
+
+
+# A single 2048 x 2048 Q8 matrix at batch 1 (the small case).
+SINGLE_Q8 = DenseWorkload(1, "q8-2048x2048", 8, 1, (Mat("w", 2048, 2048, 0),))
+
+# 16-layer dense decoder, hidden 2048, FFN 8192, Q4, batch 1.  q|k|v share an
+# input, as do gate|up; each group forms one stage.
+DENSE_H2048 = DenseWorkload(2, "dense16L-h2048-ffn8192-q4", 4, 16, (
+    Mat("q", 2048, 2048, 0), Mat("k", 512, 2048, 0), Mat("v", 512, 2048, 0),
+    Mat("o", 2048, 2048, 1),
+    Mat("gate", 8192, 2048, 2), Mat("up", 8192, 2048, 2),
+    Mat("down", 2048, 8192, 3),
+))
+
+
+def dense_h4096(fmt: int, B: int) -> DenseWorkload:
+    """One layer of a dense decoder, hidden 4096, FFN 12288 (qkv and gate|up
+    fused), streamed 36 times as distinct copies."""
+    return DenseWorkload(3, f"dense36L-h4096-ffn12288-q{fmt}-b{B}", fmt, 36, (
+        Mat("qkv", 6144, 4096, 0), Mat("o", 4096, 4096, 1),
+        Mat("gateup", 24576, 4096, 2), Mat("down", 4096, 12288, 3),
+    ), B)
+
+
+# 64-layer dense decoder, hidden 5120, FFN 25600, Q4, batch 1 (~16 GB packed).
+# Attention shapes: q, o 5120 x 5120; k, v 1024 x 5120 (8 KV heads x 128).
+DENSE_H5120 = DenseWorkload(5, "dense64L-h5120-ffn25600-q4", 4, 64, (
+    Mat("q", 5120, 5120, 0), Mat("k", 1024, 5120, 0), Mat("v", 1024, 5120, 0),
+    Mat("o", 5120, 5120, 1),
+    Mat("gate", 25600, 5120, 2), Mat("up", 25600, 5120, 2),
+    Mat("down", 5120, 25600, 3),
+))
+
+# Matrix-shape sweep (N x K) for achieved bandwidth against matrix size.
+SWEEP_SHAPES = ((512, 512), (1024, 1024), (2048, 2048), (4096, 4096), (5120, 5120),
+                (1024, 5120), (8192, 5120), (25600, 5120), (5120, 25600))
+
+
+@dataclasses.dataclass(frozen=True)
+class MoEWorkload:
+    wid: int
+    name: str
+    layers: int
+    E: int
+    topk: int
+    hidden: int
+    ffn: int
+    B: int
+
+    def gateup(self) -> Tuple[int, int]:
+        return 2 * self.ffn, self.hidden      # gate|up of one expert fused: N, K
+
+    def down(self) -> Tuple[int, int]:
+        return self.hidden, self.ffn
+
+
+def moe_h2048(B: int) -> MoEWorkload:
+    """48 layers, hidden 2048, 128 experts (gate/up 768 x 2048, down 2048 x 768),
+    top-8 routing."""
+    return MoEWorkload(4, f"moe48L-e128-top8-h2048-b{B}", 48, 128, 8, 2048, 768, B)

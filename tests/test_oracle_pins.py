@@ -1,0 +1,348 @@
+"""Pins of the fp64 oracle to things other than itself.
+
+Each test ties an oracle function to something the definition or mathematics
+fixes: numpy's IEEE binary16 conversions (library routines), exhaustive
+enumeration of the Q4 nibble positions, exactly representable quantiser
+inputs, hand-derived worked blocks (tests/golden), closed forms (one-hot and
+all-ones activations) and exact rational brute force on tiny matrices.  A
+plausible slip in the oracle (swapped nibbles, a transposed operand, a dropped
+-8 offset, a wrong rounding rule, a mis-strided scale plane) fails at least
+one of them.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from quantised_weight_gemv_b200 import synth
+from tests.conftest import read_golden
+
+
+# ------------------------------------------------------------------ fp16 ----
+def test_half_to_double_exhaustive_vs_numpy():
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.half_to_double(bits)
+    ref = bits.view(np.float16).astype(np.float64)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+
+
+def test_double_to_half_vs_numpy_rne():
+    r = np.random.default_rng(7)
+    vals = np.concatenate([
+        r.standard_normal(20000) * 10.0 ** r.integers(-9, 6, 20000),
+        # exact midpoints between neighbouring fp16 values (ties to even)
+        (np.arange(0, 4096, dtype=np.float64) + 0.5) * 2.0 ** -24,          # subnormal ties
+        (1024 + np.arange(0, 1024, dtype=np.float64) + 0.5) * 2.0 ** -10,  # [1, 2) ties
+        [65504.0, 65519.99, 65520.0, 70000.0, 2.0 ** -25, 2.0 ** -25 * 1.0000001,
+         2.0 ** -14, 2.0 ** -14 * (1 - 2.0 ** -12), 0.0, -0.0, 1e-30, -65520.0],
+    ])
+    vals = np.concatenate([vals, -vals])
+    ours = oracle.double_to_half(vals)
+    ref = vals.astype(np.float16).view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+# ------------------------------------------------------------ quantisers ----
+def _expect_exact(fmt, N, nb, e, seed):
+    """w = d*v with d = 2^-e and one element per block at +-levels."""
+    r = np.random.default_rng(seed)
+    lv = 7 if fmt == 4 else 127
+    v = r.integers(-lv, lv + 1, size=(N, nb, 32))
+    pin = r.integers(0, 32, size=(N, nb))
+    sgn = r.choice([-1, 1], size=(N, nb))
+    for n in range(N):
+        for j in range(nb):
+            v[n, j, pin[n, j]] = sgn[n, j] * lv
+    d = 2.0 ** -e
+    w = (v * d).astype(np.float32).reshape(N, nb * 32)
+    assert np.array_equal(w.astype(np.float64), (v * d).reshape(N, nb * 32))
+    return v, w, d
+
+
+@pytest.mark.parametrize("e", [4, 7, 10, 15, 18, 24])
+def test_quantize_q4_exact_representable(e):
+    N, nb = 5, 9                       # K = 288: ldS = 16 (padded from 9)
+    v, w, d = _expect_exact(4, N, nb, e, 100 + e)
+    codes, scales = oracle.quantize_q4(w)
+    assert scales.shape == (N, 16)
+    # fp16 bits of 2^-e: normal (e <= 14) or subnormal, from the format definition
+    dbits = ((15 - e) << 10) if e <= 14 else (1 << (24 - e))
+    assert np.all(scales[:, :nb] == dbits) and np.all(scales[:, nb:] == 0)
+    q = v + 8
+    lo, hi = q[..., :16], q[..., 16:]
+    assert np.array_equal(codes.reshape(N, nb, 16), (lo | (hi << 4)).astype(np.uint8))
+    assert np.array_equal(oracle.dequantize_q4(codes, scales), w.astype(np.float64))
+
+
+@pytest.mark.parametrize("e", [4, 7, 10, 16, 24])
+def test_quantize_q8_exact_representable(e):
+    N, nb = 3, 8
+    v, w, d = _expect_exact(8, N, nb, e, 200 + e)
+    # the scale a/127 = d is exact only when d*127 is exact in fp32 (always here)
+    codes, scales = oracle.quantize_q8(w)
+    dbits = ((15 - e) << 10) if e <= 14 else (1 << (24 - e))
+    assert np.all(scales[:, :nb] == dbits)
+    assert np.array_equal(codes.reshape(N, nb, 32), v.astype(np.int8))
+    assert np.array_equal(oracle.dequantize_q8(codes, scales), w.astype(np.float64))
+
+
+def test_quantize_zero_block_and_tiny_scale():
+    w = np.zeros((2, 64), dtype=np.float32)
+    w[1, 32:] = 1e-9                      # a/7 rounds to fp16 zero
+    c4, s4 = oracle.quantize_q4(w)
+    assert np.all(s4 == 0) and np.all(c4 == 0x88)
+    c8, s8 = oracle.quantize_q8(w)
+    assert np.all(s8 == 0) and np.all(c8 == 0)
+
+
+def test_quantize_round_half_away_and_ties():
+    d = 2.0 ** -6
+    w = np.zeros((1, 32), dtype=np.float32)
+    w[0, 0] = 7 * d                       # absmax -> d exactly
+    w[0, 1] = -7 * d                      # the symmetric tie of the absmax
+    w[0, 2] = 2.5 * d                     # half: away from zero -> 3 (even rule: 2)
+    w[0, 3] = -2.5 * d                    # -> -3
+    w[0, 4] = 0.5 * d                     # -> 1
+    w[0, 5] = -0.5 * d                    # -> -1
+    w[0, 6] = 1.49 * d                    # -> 1
+    codes, scales = oracle.quantize_q4(w)
+    q = [(codes[0, i % 16] >> (4 * (i // 16))) & 15 for i in range(32)]
+    assert q[:7] == [15, 1, 11, 5, 9, 7, 9]
+    assert scales[0, 0] == (15 - 6) << 10
+
+
+def test_quantize_rejects_overflow_and_nonfinite():
+    w = np.zeros((1, 32), dtype=np.float32)
+    w[0, 0] = 7 * 65600.0                 # a/7 > 65504 -> fp16 overflow
+    with pytest.raises(ValueError):
+        oracle.quantize_q4(w)
+    w[0, 0] = np.inf
+    with pytest.raises(ValueError):
+        oracle.quantize_q8(w)
+
+
+def test_quantize_nearest_grid_point():
+    """Away from ties, every dequantised weight is the nearest point of its
+    block's grid d*{-8..7} (Q4) / d*{-127..127} (Q8) to w."""
+    w = synth.weights_f32(synth.key(0, 90, 0, 0, 0), 16, 256)
+    c4, s4 = oracle.quantize_q4(w)
+    c8, s8 = oracle.quantize_q8(w)
+    for fmt, codes, scales, lv in ((4, c4, s4, (-8, 7)), (8, c8, s8, (-127, 127))):
+        deq = oracle.dequantize_q4(codes, scales) if fmt == 4 else oracle.dequantize_q8(codes, scales)
+        d = oracle.half_to_double(scales[:, :8]).repeat(32, axis=1)
+        grid = np.arange(lv[0], lv[1] + 1)[None, None, :] * d[..., None]
+        nearest = np.abs(grid - w.astype(np.float64)[..., None]).min(axis=-1)
+        assert np.all(np.abs(deq - w) <= nearest + 1e-18)
+
+
+# ---------------------------------------------------------- golden files ----
+@pytest.mark.parametrize("name,fmt", [("q4_block_worked.txt", 4), ("q8_block_worked.txt", 8)])
+def test_golden_worked_block(name, fmt):
+    g = read_golden(name)
+    v = np.array([int(t) for t in g["w_over_d"]])
+    d = 2.0 ** int(g["d_log2"][0])
+    w = (v * d).astype(np.float32)[None, :]
+    x = np.array([float(t) for t in g["x"]], dtype=np.float16).view(np.uint16)[None, :]
+    if fmt == 4:
+        codes, scales = oracle.quantize_q4(w)
+        assert [int(b) for b in codes[0]] == [int(t, 16) for t in g["packed"]]
+        q = [(codes[0, i % 16] >> (4 * (i // 16))) & 15 for i in range(32)]
+        y, a = oracle.gemv_q4(codes, scales, x)
+    else:
+        codes, scales = oracle.quantize_q8(w)
+        q = [int(c) for c in codes[0]]
+        y, a = oracle.gemv_q8(codes, scales, x)
+    assert q == [int(t) for t in g["codes"]]
+    assert scales[0, 0] == int(g["scale_bits"][0], 16)
+    assert y[0, 0] == float(g["y"][0])
+    assert a[0, 0] == float(g["abs_sum"][0])
+
+
+# ---------------------------------------------------------- nibble order ----
+def test_q4_nibble_order_exhaustive():
+    """Every (position, code) of a 1x32 block: element i < 16 lives in the low
+    nibble of byte i, element i >= 16 in the high nibble of byte i-16."""
+    one = np.array([0x3C00], dtype=np.uint16)          # fp16 1.0
+    scales = np.zeros((1, 8), dtype=np.uint16)
+    scales[0, 0] = one[0]
+    for p in range(32):
+        xo = np.zeros((1, 32), dtype=np.uint16)
+        xo[0, p] = one[0]
+        for c in range(16):
+            q = [8] * 32
+            q[p] = c
+            packed = np.array([[q[i] | (q[i + 16] << 4) for i in range(16)]], dtype=np.uint8)
+            deq = oracle.dequantize_q4(packed, scales)
+            expect = np.zeros((1, 32))
+            expect[0, p] = c - 8
+            assert np.array_equal(deq, expect), (p, c)
+            y, _ = oracle.gemv_q4(packed, scales, xo)
+            assert y[0, 0] == c - 8
+
+
+def test_scale_plane_stride_and_block_index():
+    """Scale (n, j) scales exactly block j of row n, with rows ldS apart."""
+    N, K = 3, 96                                       # ldS = 8 > K/32 = 3
+    codes = np.full((N, K // 2), 0x99, dtype=np.uint8)  # every code 9 -> v = 1
+    scales = np.zeros((N, 8), dtype=np.uint16)
+    for n in range(N):
+        for j in range(3):
+            scales[n, j] = oracle.double_to_half(float(10 * n + j + 1))
+        scales[n, 3:] = 0x7C00                          # padding must be ignored (inf)
+    deq = oracle.dequantize_q4(codes, scales)
+    for n in range(N):
+        for k in range(K):
+            assert deq[n, k] == 10 * n + k // 32 + 1
+    c8 = np.ones((N, K), dtype=np.int8)
+    deq8 = oracle.dequantize_q8(c8, scales)
+    assert np.array_equal(deq8, deq)
+
+
+# ------------------------------------------------------------------ GEMV ----
+def _rand_planes(fmt, N, K, seed):
+    w = synth.weights_f32(synth.key(seed, 91, 0, 0, 0), N, K)
+    return oracle.quantize_q4(w) if fmt == 4 else oracle.quantize_q8(w)
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+def test_gemv_one_hot_returns_columns(fmt):
+    N, K = 7, 96
+    codes, scales = _rand_planes(fmt, N, K, 1)
+    deq = oracle.dequantize_q4(codes, scales) if fmt == 4 else oracle.dequantize_q8(codes, scales)
+    gemv = oracle.gemv_q4 if fmt == 4 else oracle.gemv_q8
+    one = np.float16(1.0).view(np.uint16)
+    x = np.zeros((K, K), dtype=np.uint16)
+    x[np.arange(K), np.arange(K)] = one                 # B = K one-hot rows, 8 at a time
+    for b0 in range(0, K, 8):
+        y, _ = gemv(codes, scales, x[b0:b0 + 8])
+        assert np.array_equal(y, deq[:, b0:b0 + 8].T)
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+def test_gemv_all_ones_returns_row_sums(fmt):
+    import math
+    N, K = 11, 160
+    codes, scales = _rand_planes(fmt, N, K, 2)
+    deq = oracle.dequantize_q4(codes, scales) if fmt == 4 else oracle.dequantize_q8(codes, scales)
+    gemv = oracle.gemv_q4 if fmt == 4 else oracle.gemv_q8
+    x = np.full((2, K), np.float16(1.0).view(np.uint16), dtype=np.uint16)
+    y, a = gemv(codes, scales, x)
+    for n in range(N):
+        assert y[0, n] == y[1, n] == math.fsum(deq[n])
+        assert a[0, n] == math.fsum(np.abs(deq[n]))
+
+
+def _unpack_fraction(fmt, codes, scales, n, k):
+    """Independent unpack straight from the format text, as an exact Fraction."""
+    bits = int(scales[n, k // 32])
+    d = Fraction(np.uint16(bits).view(np.float16).item())
+    if fmt == 8:
+        return d * int(codes[n, k])
+    i = k % 32
+    byte = int(codes[n, (k // 32) * 16 + i % 16])
+    q = byte & 15 if i < 16 else byte >> 4
+    return d * (q - 8)
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+@pytest.mark.parametrize("N,K,B", [(1, 32, 1), (3, 64, 2), (8, 96, 8), (5, 32, 3), (2, 96, 5)])
+def test_gemv_brute_force_exact(fmt, N, K, B):
+    codes, scales = _rand_planes(fmt, N, K, 10 * N + K + B)
+    x = synth.activations_f16_bits(synth.key(3, 91, N, K, 1), B, K)
+    gemv = oracle.gemv_q4 if fmt == 4 else oracle.gemv_q8
+    y, a = gemv(codes, scales, x)
+    xf = x.view(np.float16)
+    for b in range(B):
+        for n in range(N):
+            terms = [_unpack_fraction(fmt, codes, scales, n, k) * Fraction(xf[b, k].item())
+                     for k in range(K)]
+            exact = sum(terms)
+            exact_abs = sum(abs(t) for t in terms)
+            assert abs(Fraction(y[b, n]) - exact) <= exact_abs * Fraction(1, 2 ** 50)
+            assert abs(Fraction(a[b, n]) - exact_abs) <= exact_abs * Fraction(1, 2 ** 50)
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+def test_gemv_batch_rows_independent_and_threads(fmt):
+    N, K, B = 37, 256, 6
+    codes, scales = _rand_planes(fmt, N, K, 5)
+    x = synth.activations_f16_bits(synth.key(4, 91, 0, 0, 1), B, K)
+    gemv = oracle.gemv_q4 if fmt == 4 else oracle.gemv_q8
+    y, a = gemv(codes, scales, x)
+    y4, a4 = gemv(codes, scales, x, nthreads=4)
+    assert np.array_equal(y, y4) and np.array_equal(a, a4)
+    for b in range(B):
+        yb, _ = gemv(codes, scales, x[b:b + 1])
+        assert np.array_equal(yb[0], y[b])
+
+
+# ------------------------------------------------------------------- MoE ----
+def _moe_stack(E, N, K, seed):
+    cs, ss = [], []
+    for e in range(E):
+        c, s = oracle.quantize_q4(synth.weights_f32(synth.key(seed, 92, 0, e, 0), N, K))
+        cs.append(c)
+        ss.append(s)
+    return np.stack(cs), np.stack(ss)
+
+
+def test_moe_identical_experts_uniform_weights_is_dense():
+    E, N, K, B, topk = 6, 24, 64, 3, 4
+    c, s = oracle.quantize_q4(synth.weights_f32(synth.key(1, 92, 0, 0, 0), N, K))
+    codes, scales = np.stack([c] * E), np.stack([s] * E)
+    x = synth.activations_f16_bits(synth.key(1, 92, 0, 0, 1), B, K)
+    idx = np.array([[0, 2, 3, 5], [1, 2, 4, 0], [5, 4, 3, 2]], dtype=np.int32)
+    r = np.full((B, topk), 0.25, dtype=np.float32)
+    y, _, bad = oracle.moe_gemv_q4(codes, scales, x, False, idx, r)
+    yd, _ = oracle.gemv_q4(c, s, x)
+    assert not bad
+    np.testing.assert_allclose(y, yd, rtol=1e-14, atol=1e-15)
+
+
+def test_moe_slot_permutation_invariance_and_combine():
+    E, N, K, B, topk = 9, 16, 96, 4, 3
+    codes, scales = _moe_stack(E, N, K, 2)
+    x = synth.activations_f16_bits(synth.key(2, 92, 0, 0, 1), B, topk, K)
+    idx, r = synth.routing(synth.key(2, 92, 0, 0, 2), synth.key(2, 92, 0, 0, 3), B, E, topk)
+    y, a, _ = oracle.moe_gemv_q4(codes, scales, x, True, idx, r)
+    perm = np.array([2, 0, 1])
+    yp, ap, _ = oracle.moe_gemv_q4(codes, scales, x[:, perm], True, idx[:, perm], r[:, perm])
+    np.testing.assert_allclose(yp, y, rtol=1e-13, atol=1e-15)
+    per, aper, _ = oracle.moe_gemv_q4(codes, scales, x, True, idx, None)
+    assert per.shape == (B, topk, N)
+    comb = (r.astype(np.float64)[..., None] * per).sum(axis=1)
+    np.testing.assert_allclose(comb, y, rtol=1e-13, atol=1e-15)
+    # each per-slot output is the dense GEMV of the routed expert
+    for b in range(B):
+        for t in range(topk):
+            yd, _ = oracle.gemv_q4(codes[idx[b, t]], scales[idx[b, t]], x[b, t][None])
+            assert np.array_equal(per[b, t], yd[0])
+
+
+def test_moe_single_expert_is_dense_batch():
+    E, N, K, B = 4, 20, 64, 5
+    codes, scales = _moe_stack(E, N, K, 3)
+    x = synth.activations_f16_bits(synth.key(3, 92, 0, 0, 1), B, K)
+    idx = np.full((B, 1), 2, dtype=np.int32)
+    per, _, _ = oracle.moe_gemv_q4(codes, scales, x, False, idx, None)
+    yd, _ = oracle.gemv_q4(codes[2], scales[2], x)
+    assert np.array_equal(per[:, 0], yd)
+
+
+def test_moe_out_of_range_index_flags_and_skips():
+    E, N, K, B, topk = 3, 8, 32, 2, 2
+    codes, scales = _moe_stack(E, N, K, 4)
+    x = synth.activations_f16_bits(synth.key(4, 92, 0, 0, 1), B, K)
+    idx = np.array([[0, 3], [-1, 1]], dtype=np.int32)
+    r = np.array([[0.5, 0.5], [0.25, 0.75]], dtype=np.float32)
+    y, _, bad = oracle.moe_gemv_q4(codes, scales, x, False, idx, r)
+    assert bad
+    y0, _ = oracle.gemv_q4(codes[0], scales[0], x[0:1])
+    y1, _ = oracle.gemv_q4(codes[1], scales[1], x[1:2])
+    np.testing.assert_allclose(y[0], 0.5 * y0[0], rtol=1e-15)
+    np.testing.assert_allclose(y[1], np.float64(np.float32(0.75)) * y1[0], rtol=1e-15)
+    per, _, bad = oracle.moe_gemv_q4(codes, scales, x, False, idx, None)
+    assert bad and np.all(per[0, 1] == 0) and np.all(per[1, 0] == 0)
