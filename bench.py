@@ -1,0 +1,445 @@
+"""Decode-step benchmark of the block-quantised weight GEMV on B200.
+
+One step = one decode token through the whole weight stream of the workload:
+every layer's projections in model order (q|k|v, o, gate|up, down), each a Q4
+GEMV with dequantisation in the inner loop.  Default workload: 16-layer dense
+decoder, hidden 2048, FFN 8192, Q4, batch 1 (547 MB of packed weights per step,
+> L2, so no L2 flush is needed).  Weights and activations are synthetic
+(seeded N(0, 0.02) weights, N(0, 1) fp16 activations), generated and quantised
+on the device.
+
+Prints ONE JSON line (rank 0).  `value` = algorithmic bytes (packed codes +
+scales + x + y) of all ranks per second of the slowest rank; tokens/s-equiv =
+B / step time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bq|reference]
+                  [--workload NAME] [--engine graph|step]
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantised_weight_gemv_b200 import synth  # noqa: E402
+
+METRIC = "weight-stream HBM GB/s (decode step, algorithmic bytes)"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return dict(PEAKS_FALLBACK)
+
+
+WORKLOADS = {
+    synth.DENSE_H2048.name: synth.DENSE_H2048,
+    synth.SINGLE_Q8.name: synth.SINGLE_Q8,
+    synth.DENSE_H5120.name: synth.DENSE_H5120,
+}
+for _f in (4, 8):
+    for _b in (1, 2, 4, 8):
+        _w = synth.dense_h4096(_f, _b)
+        WORKLOADS[_w.name] = _w
+
+
+def fused_stages(wl: synth.DenseWorkload):
+    """Per layer: list of (stage, [Mat...]) -- matrices sharing a stage share x
+    and are stored as one row-concatenated matrix."""
+    st = {}
+    for m in wl.mats:
+        st.setdefault(m.stage, []).append(m)
+    return [(s, st[s]) for s in sorted(st)]
+
+
+# ------------------------------------------------------------- clocks ----
+class ClockSampler:
+    """nvidia-smi sampling of SM clock / throttle reasons during a region."""
+
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, phys_index: int):
+        self.idx = phys_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="bq_clocks_", suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-i", str(self.idx), "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        self.t0 = time.time()
+
+    def mark(self):
+        return time.time()
+
+    def stop(self, t_begin, t_end):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [s.strip() for s in line.split(",")]
+                if len(p) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(p[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    ts += float("0." + p[0].split(".")[1]) if "." in p[0] else 0.0
+                    rows.append((ts, float(p[2]), float(p[3]), p[6:10]))
+                except Exception:
+                    continue
+        os.unlink(self.path)
+        inside = [r for r in rows if t_begin - 0.25 <= r[0] <= t_end + 0.25] or rows
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "samples": len(inside)}
+
+
+def phys_gpu_index(local_rank: int) -> int:
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [s for s in cvd.split(",") if s.strip()]
+    if ids and all(s.strip().isdigit() for s in ids) and local_rank < len(ids):
+        return int(ids[local_rank])
+    return local_rank
+
+
+# ------------------------------------------------------ device workload ----
+class DenseStep:
+    """All matrices of one decode step resident in HBM, plus x / y buffers."""
+
+    def __init__(self, wl: synth.DenseWorkload, device, seed: int = 0):
+        import torch
+        from quantised_weight_gemv_b200 import bq
+        self.wl, self.device, self.bq = wl, device, bq
+        self.B = wl.B
+        self.fmt = wl.fmt
+        self.launches = []      # (qmat, x, y, label)
+        self.bytes_alg = 0
+        self.bytes_by_label = {}
+        self._keep = []
+        st = torch.zeros(1, dtype=torch.int32, device=device)
+        ws_max = 0
+        stages = fused_stages(wl)
+        for layer in range(wl.layers):
+            for s, mats in stages:
+                K = mats[0].K
+                Ntot = sum(m.N for m in mats)
+                ldS = bq.scales_ld(K)
+                codes = torch.empty((Ntot, K // 2 if wl.fmt == 4 else K), dtype=torch.uint8, device=device)
+                scales = torch.empty((Ntot, ldS), dtype=torch.int16, device=device)
+                r0 = 0
+                for mi, m in enumerate(mats):
+                    w = synth.weights_f32_torch(synth.key(seed, wl.wid, layer, wl.mats.index(m),
+                                                          synth.KIND_W), m.N, K, device)
+                    bq.quantize_dev(wl.fmt, w, codes[r0:r0 + m.N], scales[r0:r0 + m.N], st)
+                    r0 += m.N
+                    del w
+                x = synth.activations_f16_torch(synth.key(seed, wl.wid, layer, s, synth.KIND_X),
+                                                (self.B, K), device)
+                y = torch.empty((self.B, Ntot), dtype=torch.float32, device=device)
+                label = "+".join(m.name for m in mats)
+                q = bq.qmat(codes, scales, Ntot, K)
+                self.launches.append((q, x, y, label))
+                self._keep += [codes, scales]
+                nb = synth.packed_bytes(wl.fmt, Ntot, K) + self.B * K * 2 + self.B * Ntot * 4
+                self.bytes_alg += nb
+                self.bytes_by_label[label] = self.bytes_by_label.get(label, 0) + nb
+                ws_max = max(ws_max, bq.lib().bq_gemv_workspace_bytes(Ntot, K))
+        torch.cuda.synchronize()
+        if int(st.item()) != 0:
+            raise RuntimeError(f"device quantiser status {int(st.item()):#x}")
+        self.ws = bq.workspace(ws_max, device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def launch(self, stream, only=None):
+        import ctypes
+        L = self.bq.lib()
+        fn = L.bq_gemv_q4 if self.fmt == 4 else L.bq_gemv_q8
+        sp = stream.cuda_stream
+        wsp, wsb, stp = self.ws.data_ptr(), self.ws.numel(), self.status.data_ptr()
+        n = 0
+        for q, x, y, label in self.launches:
+            if only is not None and label != only:
+                continue
+            rc = fn(ctypes.byref(q), x.data_ptr(), self.B, y.data_ptr(), wsp, wsb, stp, sp)
+            if rc != 0:
+                raise RuntimeError(f"bq_gemv_q{self.fmt}: {self.bq.bq_status_string(rc)}")
+            n += 1
+        return n
+
+    def io_tensors(self):
+        return [x for _, x, _, _ in self.launches], [y for _, _, y, _ in self.launches]
+
+
+# ---------------------------------------------------------- CPU oracle ----
+def oracle_sample(wl: synth.DenseWorkload, seed: int = 0):
+    """Packed planes (oracle quantiser) + x for one layer of the workload."""
+    import numpy as np
+    import oracle
+    mats = []
+    for s, group in fused_stages(wl):
+        K = group[0].K
+        parts = [synth.weights_f32(synth.key(seed, wl.wid, 0, wl.mats.index(m), synth.KIND_W), m.N, K)
+                 for m in group]
+        w = np.concatenate(parts, axis=0)
+        codes, scales = oracle.quantize_q4(w) if wl.fmt == 4 else oracle.quantize_q8(w)
+        x = synth.activations_f16_bits(synth.key(seed, wl.wid, 0, s, synth.KIND_X), wl.B, K)
+        nbytes = synth.packed_bytes(wl.fmt, w.shape[0], K) + wl.B * K * 2 + wl.B * w.shape[0] * 4
+        mats.append((codes, scales, x, nbytes))
+    return mats
+
+
+def time_oracle_once(wl, mats, threads):
+    import oracle
+    t0 = time.perf_counter()
+    for codes, scales, x, _ in mats:
+        (oracle.gemv_q4 if wl.fmt == 4 else oracle.gemv_q8)(codes, scales, x, nthreads=threads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, budget_s=10.0):
+    threads = os.cpu_count() or 1
+    mats = oracle_sample(wl)
+    nbytes = sum(m[3] for m in mats)
+    reps, total = 0, 0.0
+    while total < budget_s or reps == 0:
+        total += time_oracle_once(wl, mats, threads)
+        reps += 1
+    return {"value": round(nbytes * reps / total / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"layer 0 of {wl.layers} ({nbytes/1e6:.1f} MB algorithmic), {reps} pass(es), "
+                      f"fp64 oracle, {threads} threads"}
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return
+    threads = os.cpu_count() or 1
+    mats = oracle_sample(wl)
+    nbytes = sum(m[3] for m in mats)
+    for _ in range(args.warmup):
+        time_oracle_once(wl, mats, threads)
+    t = 0.0
+    for _ in range(args.steps):
+        t += time_oracle_once(wl, mats, threads)
+    val = nbytes * args.steps / t / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.B, "layers": wl.layers,
+                   "sample": "one layer per step"},
+        "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"layer 0 of {wl.layers} per step ({nbytes/1e6:.1f} MB)"},
+        "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- main ----
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="bq", choices=["bq", "reference"])
+    ap.add_argument("--workload", default=synth.DENSE_H2048.name, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    wl = WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    step = DenseStep(wl, device)
+    stream = torch.cuda.Stream(device)
+    peaks = load_peaks()
+
+    # warm the kernels (attributes, module load) before capture
+    with torch.cuda.stream(stream):
+        n_launch = step.launch(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        step.launch(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(phys_gpu_index(local_rank))
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            g.replay()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_begin = time.time()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t_end = time.time()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop(t_begin, t_end)
+    t_dev = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        tt = torch.tensor([t_dev], dtype=torch.float64, device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_dev = float(tt.item())
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {int(step.status.item()):#x}")
+
+    # dominant kernel: its launches timed one by one with events on its stream
+    dom = max(step.bytes_by_label, key=step.bytes_by_label.get)
+    durs = []
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            for q, x, y, label in step.launches:
+                if label != dom:
+                    continue
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                import ctypes
+                fn = step.bq.lib().bq_gemv_q4 if step.fmt == 4 else step.bq.lib().bq_gemv_q8
+                fn(ctypes.byref(q), x.data_ptr(), step.B, y.data_ptr(), step.ws.data_ptr(),
+                   step.ws.numel(), step.status.data_ptr(), stream.cuda_stream)
+                b.record(stream)
+                durs.append((a, b))
+    torch.cuda.synchronize()
+    n_dom = sum(1 for l in step.launches if l[3] == dom)
+    dom_s = statistics.mean(a.elapsed_time(b) for a, b in durs) / 1e3
+    dom_bytes = step.bytes_by_label[dom] / n_dom
+    achieved = dom_bytes / dom_s / 1e9
+
+    # end to end: pinned host x -> device, step, y -> pinned host, every step
+    xs, ys = step.io_tensors()
+    hx = [x.cpu().pin_memory() for x in xs]
+    hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys]
+    e2e_steps = max(1, min(args.steps, 500))
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            for h, d in zip(hx, xs):
+                d.copy_(h, non_blocking=True)
+            g.replay()
+            for h, d in zip(hy, ys):
+                h.copy_(d, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            for h, d in zip(hx, xs):
+                d.copy_(h, non_blocking=True)
+            g.replay()
+            for h, d in zip(hy, ys):
+                h.copy_(d, non_blocking=True)
+        f1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = f0.elapsed_time(f1) / 1e3
+    if world > 1:
+        tt = torch.tensor([t_e2e], dtype=torch.float64, device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_e2e = float(tt.item())
+    h2d = sum(x.numel() * x.element_size() for x in xs)
+    d2h = sum(y.numel() * y.element_size() for y in ys)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
+
+    if rank == 0:
+        value = world * step.bytes_alg * args.steps / t_dev / 1e9
+        ms = t_dev / args.steps * 1e3
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": f"q{wl.fmt} weights, f16 x, f16 mma operands, f32 accumulate",
+            "data": "synthetic (seeded N(0,0.02) weights, N(0,1) fp16 activations)",
+            "config": {"workload": wl.name, "batch": wl.B, "layers": wl.layers,
+                       "launches_per_step": n_launch, "bytes_per_step": step.bytes_alg,
+                       "engine": "cuda-graph of per-matrix launches",
+                       "l2": "inputs larger than L2 (no flush)",
+                       "parallelism": f"replicas x{world}"},
+            "tokens_per_s_equiv": round(world * wl.B / (t_dev / args.steps), 1),
+            "frac_of_measured_hbm": round(value / world / peaks["hbm_gbs"], 4),
+            "frac_of_8TBps": round(value / world / 8000.0, 4),
+            "roofline": {"bound": "hbm", "kernel": f"stream_gemv q{wl.fmt} ({dom})",
+                         "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                         "peak_source": peaks["source"], "unit": "GB/s",
+                         "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                         "bytes_per_launch": int(dom_bytes),
+                         "launch_us": round(dom_s * 1e6, 3)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(world * step.bytes_alg * e2e_steps / t_e2e / 1e9, 2),
+                    "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps},
+            "gpu_launches": n_launch * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    del g
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

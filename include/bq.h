@@ -64,6 +64,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define BQ_API __attribute__((visibility("default")))
+#else
+#define BQ_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -92,17 +98,17 @@ typedef struct bq_qmat {
 } bq_qmat;
 
 /* Human-readable name of a status code (static string, never NULL). */
-const char *bq_status_string(int32_t status);
+BQ_API const char *bq_status_string(int32_t status);
 
 /* Entries per scale-plane row for a K-column matrix: roundup(K/32, 8).
  * Returns 0 when K is not a positive multiple of 32. */
-int32_t bq_scales_ld(int32_t K);
+BQ_API int32_t bq_scales_ld(int32_t K);
 
 /* ---------------------------------------------------------------- GEMV --- */
 
 /* Bytes of workspace bq_gemv_q4 / bq_gemv_q8 need for an N x K matrix
  * (independent of B and of the format).  0 on a bad shape. */
-size_t bq_gemv_workspace_bytes(int32_t N, int32_t K);
+BQ_API size_t bq_gemv_workspace_bytes(int32_t N, int32_t K);
 
 /* Q4 decode GEMV: y[b][n] = sum_k d(n,k/32) * (q(n,k) - 8) * x[b][k].
  * The operation is the per-format decode GEMV with dequantisation in the
@@ -115,21 +121,21 @@ size_t bq_gemv_workspace_bytes(int32_t N, int32_t K);
  *   ws         device workspace, ws_bytes >= bq_gemv_workspace_bytes(N, K)
  *   dev_status device int32 or NULL (see conventions)
  *   stream     cudaStream_t
- * The launch uses programmatic dependent launch: its weight prefetch may
- * start while the previous kernel on the stream drains; x, y and ws are only
- * touched after that kernel has completed. */
-int32_t bq_gemv_q4(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
+ * The launch carries the programmatic-dependent-launch attribute: its CTAs
+ * may become resident while the previous kernel on the stream drains, and
+ * they read or write no memory before that kernel has completed. */
+BQ_API int32_t bq_gemv_q4(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
                    void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
 
 /* Q8 decode GEMV: y[b][n] = sum_k d(n,k/32) * q(n,k) * x[b][k].
  * Arguments as bq_gemv_q4. */
-int32_t bq_gemv_q8(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
+BQ_API int32_t bq_gemv_q8(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
                    void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
 
 /* ------------------------------------------------------ routed experts --- */
 
 /* Bytes of workspace bq_moe_gemv_q4 needs.  0 on a bad shape. */
-size_t bq_moe_workspace_bytes(int32_t N, int32_t K, int32_t B, int32_t topk, int32_t E);
+BQ_API size_t bq_moe_workspace_bytes(int32_t N, int32_t K, int32_t B, int32_t topk, int32_t E);
 
 /* Grouped Q4 GEMV over routed experts (decode step of a mixture-of-experts
  * layer; the pages discuss expert GEMMs in the technical summary's
@@ -153,7 +159,7 @@ size_t bq_moe_workspace_bytes(int32_t N, int32_t K, int32_t B, int32_t topk, int
  *   B, topk       1 <= B <= 8, 1 <= topk, B*topk <= 64
  * A slot whose index lies outside [0, E) contributes zero (its per-slot
  * output is zero) and sets bit BQ_ERR_EXPERT_INDEX in *dev_status. */
-int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t codes_stride,
+BQ_API int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t codes_stride,
                        int64_t scales_stride, const uint16_t *x, int32_t x_per_slot,
                        const int32_t *expert_idx, const float *route_w, int32_t B,
                        int32_t topk, float *y, void *ws, size_t ws_bytes,
@@ -169,25 +175,25 @@ int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t codes_stride,
  * zero gets code 0 (Q8) or 8 (Q4).  codes: Q8 int8 [N][K], Q4 uint8 [N][K/2];
  * scales: uint16 [N][bq_scales_ld(K)], padding written as 0.
  * BQ_ERR_RANGE if an input is not finite or a scale overflows fp16. */
-int32_t bq_quantize_q8(const float *w, int32_t N, int32_t K, int8_t *codes, uint16_t *scales);
-int32_t bq_quantize_q4(const float *w, int32_t N, int32_t K, uint8_t *codes, uint16_t *scales);
+BQ_API int32_t bq_quantize_q8(const float *w, int32_t N, int32_t K, int8_t *codes, uint16_t *scales);
+BQ_API int32_t bq_quantize_q4(const float *w, int32_t N, int32_t K, uint8_t *codes, uint16_t *scales);
 
 /* Dequantise planes into fp32 weights [N][K] (exact: d * q fits fp32). */
-int32_t bq_dequantize_q8(const int8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
+BQ_API int32_t bq_dequantize_q8(const int8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
                          float *w);
-int32_t bq_dequantize_q4(const uint8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
+BQ_API int32_t bq_dequantize_q4(const uint8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
                          float *w);
 
 /* Planes <-> interleaved blocks.  blocks: N*(K/32) records, row-major over
  * (n, j); each record is the fp16 scale (2 bytes, little-endian) followed by
  * 16 code bytes (Q4, 18-byte records) or 32 code bytes (Q8, 34-byte records). */
-int32_t bq_planes_to_blocks_q4(const uint8_t *codes, const uint16_t *scales, int32_t N,
+BQ_API int32_t bq_planes_to_blocks_q4(const uint8_t *codes, const uint16_t *scales, int32_t N,
                                int32_t K, uint8_t *blocks);
-int32_t bq_planes_to_blocks_q8(const int8_t *codes, const uint16_t *scales, int32_t N,
+BQ_API int32_t bq_planes_to_blocks_q8(const int8_t *codes, const uint16_t *scales, int32_t N,
                                int32_t K, uint8_t *blocks);
-int32_t bq_blocks_to_planes_q4(const uint8_t *blocks, int32_t N, int32_t K, uint8_t *codes,
+BQ_API int32_t bq_blocks_to_planes_q4(const uint8_t *blocks, int32_t N, int32_t K, uint8_t *codes,
                                uint16_t *scales);
-int32_t bq_blocks_to_planes_q8(const uint8_t *blocks, int32_t N, int32_t K, int8_t *codes,
+BQ_API int32_t bq_blocks_to_planes_q8(const uint8_t *blocks, int32_t N, int32_t K, int8_t *codes,
                                uint16_t *scales);
 
 /* ------------------------------------------------ device-side quantiser --- */
@@ -197,9 +203,9 @@ int32_t bq_blocks_to_planes_q8(const uint8_t *blocks, int32_t N, int32_t K, int8
  * codes / scales: device planes.  Non-finite inputs or fp16-overflowing
  * scales set bit BQ_ERR_RANGE in *dev_status (if not NULL) and produce the
  * zero-point codes for that block. */
-int32_t bq_quantize_q4_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
+BQ_API int32_t bq_quantize_q4_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
                            uint16_t *scales, int32_t *dev_status, void *stream);
-int32_t bq_quantize_q8_dev(const float *w, int32_t N, int32_t K, int8_t *codes,
+BQ_API int32_t bq_quantize_q8_dev(const float *w, int32_t N, int32_t K, int8_t *codes,
                            uint16_t *scales, int32_t *dev_status, void *stream);
 
 #ifdef __cplusplus

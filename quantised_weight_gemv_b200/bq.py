@@ -1,0 +1,142 @@
+"""ctypes binding of libbq.so -- same names as the C ABI in include/bq.h.
+
+Argument marshalling only: every step of the GEMV runs in the CUDA library.
+The raw functions take integer addresses (device or host, as the header says)
+and return the bq_status code.  The helpers at the bottom accept torch tensors
+(torch is used for device memory and streams only) and raise on a non-zero
+status.  There is no fallback: if the library is missing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbq.so")
+
+BQ_OK, BQ_ERR_NULL, BQ_ERR_SHAPE, BQ_ERR_ALIGN, BQ_ERR_BATCH = 0, 1, 2, 3, 4
+BQ_ERR_EXPERT_INDEX, BQ_ERR_CUDA, BQ_ERR_TIMEOUT, BQ_ERR_WORKSPACE, BQ_ERR_RANGE = 5, 6, 7, 8, 9
+
+
+class bq_qmat(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("N", ctypes.c_int32), ("K", ctypes.c_int32)]
+
+
+class BQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {bq_status_string(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_QP = ctypes.POINTER(bq_qmat)
+
+# name -> (restype, argtypes); mirrors include/bq.h
+_SIGS = {
+    "bq_status_string": (ctypes.c_char_p, [_i32]),
+    "bq_scales_ld": (_i32, [_i32]),
+    "bq_gemv_workspace_bytes": (_sz, [_i32, _i32]),
+    "bq_gemv_q4": (_i32, [_QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
+    "bq_gemv_q8": (_i32, [_QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
+    "bq_moe_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
+    "bq_moe_gemv_q4": (_i32, [_QP, _i32, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _i32, _vp,
+                              _vp, _sz, _vp, _vp]),
+    "bq_quantize_q8": (_i32, [_vp, _i32, _i32, _vp, _vp]),
+    "bq_quantize_q4": (_i32, [_vp, _i32, _i32, _vp, _vp]),
+    "bq_dequantize_q8": (_i32, [_vp, _vp, _i32, _i32, _vp]),
+    "bq_dequantize_q4": (_i32, [_vp, _vp, _i32, _i32, _vp]),
+    "bq_planes_to_blocks_q4": (_i32, [_vp, _vp, _i32, _i32, _vp]),
+    "bq_planes_to_blocks_q8": (_i32, [_vp, _vp, _i32, _i32, _vp]),
+    "bq_blocks_to_planes_q4": (_i32, [_vp, _i32, _i32, _vp, _vp]),
+    "bq_blocks_to_planes_q8": (_i32, [_vp, _i32, _i32, _vp, _vp]),
+    "bq_quantize_q4_dev": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "bq_quantize_q8_dev": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbq.so; raises if it has not been built (no fallback path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m quantised_weight_gemv_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def __getattr__(name):
+    # module-level access to the raw C functions: bq.bq_gemv_q4(...)
+    if name in _SIGS:
+        return getattr(lib(), name)
+    raise AttributeError(name)
+
+
+def bq_status_string(status: int) -> str:
+    return lib().bq_status_string(int(status)).decode()
+
+
+def check(fn: str, status: int) -> None:
+    if status != BQ_OK:
+        raise BQError(fn, status)
+
+
+# ------------------------------------------------------- torch helpers ----
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def qmat(codes, scales, N: int, K: int) -> bq_qmat:
+    """bq_qmat over two tensors (device planes for GEMV, host for pack calls)."""
+    return bq_qmat(codes.data_ptr(), scales.data_ptr(), int(N), int(K))
+
+
+def scales_ld(K: int) -> int:
+    return int(lib().bq_scales_ld(int(K)))
+
+
+def workspace(nbytes: int, device):
+    """A zero-filled caller-owned workspace of nbytes (torch allocation)."""
+    import torch
+    return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def gemv(fmt: int, W: bq_qmat, x, y, ws, status=None, stream=None) -> None:
+    """y[B, N] (fp32) = deq(W) . x[B, K] (fp16), through bq_gemv_q4 / bq_gemv_q8."""
+    fn = lib().bq_gemv_q4 if fmt == 4 else lib().bq_gemv_q8
+    B = x.shape[0]
+    rc = fn(ctypes.byref(W), x.data_ptr(), B, y.data_ptr(), ws.data_ptr(),
+            ws.numel() * ws.element_size(), _ptr(status), _stream_ptr(stream))
+    check(f"bq_gemv_q{fmt}", rc)
+
+
+def moe_gemv_q4(Wstack: bq_qmat, E: int, codes_stride: int, scales_stride: int, x,
+                x_per_slot: bool, expert_idx, route_w, y, ws, status=None, stream=None) -> None:
+    B, topk = expert_idx.shape
+    rc = lib().bq_moe_gemv_q4(ctypes.byref(Wstack), int(E), int(codes_stride), int(scales_stride),
+                              x.data_ptr(), 1 if x_per_slot else 0, expert_idx.data_ptr(),
+                              _ptr(route_w), B, topk, y.data_ptr(), ws.data_ptr(),
+                              ws.numel() * ws.element_size(), _ptr(status), _stream_ptr(stream))
+    check("bq_moe_gemv_q4", rc)
+
+
+def quantize_dev(fmt: int, w, codes, scales, status=None, stream=None) -> None:
+    N, K = w.shape
+    fn = lib().bq_quantize_q4_dev if fmt == 4 else lib().bq_quantize_q8_dev
+    check(f"bq_quantize_q{fmt}_dev",
+          fn(w.data_ptr(), N, K, codes.data_ptr(), scales.data_ptr(), _ptr(status),
+             _stream_ptr(stream)))

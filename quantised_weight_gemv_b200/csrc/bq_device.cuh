@@ -1,0 +1,339 @@
+// bq_device.cuh -- device building blocks of the streamed block-quantised GEMV
+// for sm_100a: PTX wrappers (mbarrier, TMA tensor loads, mma.sync,
+// programmatic dependent launch), in-register Q4/Q8 dequantisation and the
+// per-chunk dot product.
+//
+// Work unit ("chunk"): 16 weight rows x 256 weights along K (8 blocks of 32).
+// A chunk's codes arrive in shared memory through one (Q4) or two (Q8) 2-D TMA
+// boxes of 16 rows x 128 bytes with the 128-byte swizzle, its scales through
+// one 16 rows x 8 fp16 box.  A warp reads them with 32-bit shared loads that
+// the swizzle makes bank-conflict free, dequantises each 4-byte group into
+// fp16 pairs in registers (the codes are small integers, exact in fp16), and
+// forms the block's partial dot products with two m16n8k16 mma.sync (fp16 in,
+// fp32 accumulate): M = the 16 weight rows, N = the batch (B <= 8; absent
+// columns are zero), K = 16 elements of one block.  Each block's partial sum
+// is scaled by its fp32-converted scale once (y += d * sum(q * x)), so the
+// only roundings are fp32 ones.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace bq {
+
+constexpr int kBlock = 32;          // weights per quantisation block
+constexpr int kChunkK = 256;        // weights along K per chunk
+constexpr int kChunkRows = 16;      // weight rows per chunk (mma M)
+constexpr int kWarps = 8;           // worker warps per CTA
+constexpr int kThreads = kWarps * 32;
+constexpr int kScaleBytes = kChunkRows * 16;   // 16 rows x 8 fp16 scales
+constexpr int kBoxBytes = kChunkRows * 128;    // one 16 x 128-byte code box
+
+// Status bits OR-ed into the caller's device status word (1 << bq_status).
+constexpr int kStatusExpertIndex = 1 << 5;
+constexpr int kStatusTimeout = 1 << 7;
+constexpr int kStatusRange = 1 << 9;
+
+// A bounded mbarrier wait gives up after this many SM clock cycles (~2 s).
+constexpr long long kWaitCycles = 4000000000LL;
+
+template <int FMT> struct Fmt;
+template <> struct Fmt<4> {
+    static constexpr int kCodeBytes = kBoxBytes;       // 16 rows x 128 B
+    static constexpr int kBoxes = 1;
+    static constexpr int kStages = 5;
+};
+template <> struct Fmt<8> {
+    static constexpr int kCodeBytes = 2 * kBoxBytes;   // 16 rows x 256 B
+    static constexpr int kBoxes = 2;
+    static constexpr int kStages = 3;
+};
+
+template <int FMT>
+constexpr int smem_bytes()
+{
+    return kWarps * Fmt<FMT>::kStages * (Fmt<FMT>::kCodeBytes + kScaleBytes) +
+           kWarps * Fmt<FMT>::kStages * 8 + 1024;
+}
+
+// ------------------------------------------------------------------ PTX ----
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after kWaitCycles.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kWaitCycles)
+            return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int x, int y, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int x, int y, int z, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Programmatic dependent launch: let the next kernel on the stream be
+// scheduled, and wait until the previous one has completed and its writes are
+// visible.  Both are no-ops when the launch carries no PDL attribute.
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+// 8 bytes of x through the read-only path; zero when !pred.
+__device__ __forceinline__ uint2 ldg64_pred(const void *p, bool pred)
+{
+    uint2 v = make_uint2(0u, 0u);
+    if (pred)
+        v = __ldg(reinterpret_cast<const uint2 *>(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t hsub2u(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t hfma2u(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// D = A(16x16 f16) * B(16x8 f16) + C, fp32 accumulators.
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1, const float (&c)[4])
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]),
+          "f"(c[2]), "f"(c[3]));
+}
+
+// ------------------------------------------------------------- dequant ----
+// The mma fragment of a block half: lane (g = lane/4, t = lane%4) supplies
+// for its rows g and g+8 the k-slots {2t, 2t+1} and {2t+8, 2t+9}.  We map
+// slot pair {2t, 2t+1} -> elements {4t, 4t+1} and {2t+8, 2t+9} -> {4t+2, 4t+3}
+// of the half (a bijection of the 16 slots), so a lane's four elements are
+// the 4 consecutive code bytes 4t..4t+3 it loads, and its x fragment is the
+// 4 consecutive x values at the same k -- one 8-byte load, no shuffles.
+//
+// Q4: bytes b0..b3 of a word hold elements e..e+3 (low nibbles) and
+// e+16..e+19 (high nibbles).  fp16 0x6400 | n is 1024 + n exactly.
+struct Q4Pairs {
+    uint32_t lo01, lo23, hi01, hi23;   // f16x2 of (q - 8)
+};
+
+__device__ __forceinline__ Q4Pairs dequant_q4(uint32_t w)
+{
+    const uint32_t p01 = prmt(w, 0u, 0x4140u);    // [b0, 0, b1, 0]
+    const uint32_t p23 = prmt(w, 0u, 0x4342u);    // [b2, 0, b3, 0]
+    Q4Pairs r;
+    // low nibble n: (1024 + n) - 1032 = n - 8
+    r.lo01 = hsub2u((p01 & 0x000F000Fu) | 0x64006400u, 0x64086408u);
+    r.lo23 = hsub2u((p23 & 0x000F000Fu) | 0x64006400u, 0x64086408u);
+    // high nibble n (in place): (1024 + 16 n) / 16 - 72 = n - 8
+    r.hi01 = hfma2u((p01 & 0x00F000F0u) | 0x64006400u, 0x2C002C00u, 0xD480D480u);
+    r.hi23 = hfma2u((p23 & 0x00F000F0u) | 0x64006400u, 0x2C002C00u, 0xD480D480u);
+    return r;
+}
+
+// Q8: int8 q -> byte q ^ 0x80 = q + 128 in [0, 255]; (1024 + q + 128) - 1152 = q.
+struct Q8Pairs {
+    uint32_t p01, p23;                 // f16x2 of q
+};
+
+__device__ __forceinline__ Q8Pairs dequant_q8(uint32_t w)
+{
+    const uint32_t u = w ^ 0x80808080u;
+    Q8Pairs r;
+    r.p01 = hsub2u(prmt(u, 0x64646464u, 0x4140u), 0x64806480u);
+    r.p23 = hsub2u(prmt(u, 0x64646464u, 0x4342u), 0x64806480u);
+    return r;
+}
+
+__device__ __forceinline__ float half_lo(uint32_t v)
+{
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xffffu)));
+}
+__device__ __forceinline__ float half_hi(uint32_t v)
+{
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
+}
+__device__ __forceinline__ uint32_t pick_u32(const uint4 &v, int i)
+{
+    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// One block (32 weights along K) of the chunk for the lane's rows g and g+8.
+// `xa` holds x at k..k+3 and `xb` at k+16..k+19 (k = block start + 4t) for
+// batch column g (zero if the column is absent).
+template <int FMT>
+__device__ __forceinline__ void block_mma(uint32_t codes_s, int jb, int g, int t, uint2 xa,
+                                          uint2 xb, float dg, float dg8, float (&acc)[4])
+{
+    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+    float c[4];
+    if constexpr (FMT == 4) {
+        const uint32_t off = (uint32_t)(g * 128 + (((jb ^ g) & 7) << 4) + 4 * t);
+        const Q4Pairs r0 = dequant_q4(lds32(codes_s + off));          // row g
+        const Q4Pairs r8 = dequant_q4(lds32(codes_s + off + 1024));   // row g + 8
+        mma16816(c, r0.lo01, r8.lo01, r0.lo23, r8.lo23, xa.x, xa.y, zero);
+        mma16816(c, r0.hi01, r8.hi01, r0.hi23, r8.hi23, xb.x, xb.y, c);
+    } else {
+        const int box = jb >> 2, jj = jb & 3;
+        const uint32_t base = codes_s + (uint32_t)(box * kBoxBytes + g * 128 + 4 * t);
+        const uint32_t oa = (uint32_t)((((2 * jj) ^ g) & 7) << 4);
+        const uint32_t ob = (uint32_t)((((2 * jj + 1) ^ g) & 7) << 4);
+        const Q8Pairs a0 = dequant_q8(lds32(base + oa));
+        const Q8Pairs a8 = dequant_q8(lds32(base + oa + 1024));
+        const Q8Pairs b0 = dequant_q8(lds32(base + ob));
+        const Q8Pairs b8 = dequant_q8(lds32(base + ob + 1024));
+        mma16816(c, a0.p01, a8.p01, a0.p23, a8.p23, xa.x, xa.y, zero);
+        mma16816(c, b0.p01, b8.p01, b0.p23, b8.p23, xb.x, xb.y, c);
+    }
+    acc[0] = fmaf(dg, c[0], acc[0]);
+    acc[1] = fmaf(dg, c[1], acc[1]);
+    acc[2] = fmaf(dg8, c[2], acc[2]);
+    acc[3] = fmaf(dg8, c[3], acc[3]);
+}
+
+// A whole chunk: blocks kb0 .. kb0+7 (k0 = 32*kb0 along K), nblk of them valid.
+// xrow points at x[column g][0] or is null when the column is absent.
+template <int FMT>
+__device__ __forceinline__ void chunk_mma(uint32_t codes_s, uint32_t scales_s,
+                                          const __half *xrow, int k0, int nblk, int g, int t,
+                                          float (&acc)[4])
+{
+    const uint4 sg = lds128(scales_s + g * 16);
+    const uint4 sg8 = lds128(scales_s + (g + 8) * 16);
+    const bool has_x = xrow != nullptr;
+    const __half *xp = has_x ? xrow + k0 + 4 * t : nullptr;
+    if (nblk == 8) {
+        uint2 xa[8], xb[8];
+#pragma unroll
+        for (int jb = 0; jb < 8; jb++) {
+            xa[jb] = ldg64_pred(xp + 32 * jb, has_x);
+            xb[jb] = ldg64_pred(xp + 32 * jb + 16, has_x);
+        }
+#pragma unroll
+        for (int jb = 0; jb < 8; jb++) {
+            const uint32_t wg = pick_u32(sg, jb >> 1), wg8 = pick_u32(sg8, jb >> 1);
+            const float dg = (jb & 1) ? half_hi(wg) : half_lo(wg);
+            const float dg8 = (jb & 1) ? half_hi(wg8) : half_lo(wg8);
+            block_mma<FMT>(codes_s, jb, g, t, xa[jb], xb[jb], dg, dg8, acc);
+        }
+    } else {
+#pragma unroll
+        for (int jb = 0; jb < 8; jb++) {
+            if (jb < nblk) {
+                const uint2 xa = ldg64_pred(xp + 32 * jb, has_x);
+                const uint2 xb = ldg64_pred(xp + 32 * jb + 16, has_x);
+                const uint32_t wg = pick_u32(sg, jb >> 1), wg8 = pick_u32(sg8, jb >> 1);
+                const float dg = (jb & 1) ? half_hi(wg) : half_lo(wg);
+                const float dg8 = (jb & 1) ? half_hi(wg8) : half_lo(wg8);
+                block_mma<FMT>(codes_s, jb, g, t, xa, xb, dg, dg8, acc);
+            }
+        }
+    }
+}
+
+}  // namespace bq

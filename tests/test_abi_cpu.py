@@ -1,0 +1,189 @@
+"""C ABI checks that need no GPU: the library loads and exports every entry
+point include/bq.h declares, the host-side quantiser and unpacker agree
+bit-for-bit with the oracle, the plane <-> block converters round-trip, and
+every GPU entry point rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from quantised_weight_gemv_b200 import bq, synth
+from tests.conftest import ROOT, read_golden
+
+FAKE = 0x7f0000000000          # a 16-byte aligned address that is never dereferenced
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "bq.h")) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"BQ_API[^;(]*?\b(bq_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 17
+    L = bq.lib()
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in bq._SIGS, f"binding lacks {n}"
+
+
+def test_status_strings_and_scales_ld():
+    assert bq.bq_status_string(0) == "ok"
+    assert bq.bq_status_string(bq.BQ_ERR_TIMEOUT) == "bounded wait timed out"
+    for K in (32, 64, 96, 256, 288, 768, 2048, 25600):
+        assert bq.scales_ld(K) == oracle.scales_ld(K) == -(-(K // 32) // 8) * 8
+    assert bq.scales_ld(33) == 0 and bq.scales_ld(0) == 0
+
+
+def _host_quantize(fmt, w):
+    N, K = w.shape
+    codes = np.zeros((N, K // 2 if fmt == 4 else K), dtype=np.uint8 if fmt == 4 else np.int8)
+    scales = np.zeros((N, bq.scales_ld(K)), dtype=np.uint16)
+    fn = bq.lib().bq_quantize_q4 if fmt == 4 else bq.lib().bq_quantize_q8
+    rc = fn(w.ctypes.data, N, K, codes.ctypes.data, scales.ctypes.data)
+    return rc, codes, scales
+
+
+def _edge_weights():
+    w = synth.weights_f32(synth.key(0, 93, 0, 0, 0), 24, 320)
+    w[0, :32] = 0.0                                   # zero block
+    w[1, :32] = 1e-9                                  # scale rounds to zero
+    w[2, :32] = np.float32(2.0 ** -20)                # subnormal fp16 scale
+    w[3, 0], w[3, 1] = 0.7, -0.7                      # symmetric absmax tie
+    d = np.float32(0.1) / np.float32(7.0)
+    w[4, 32:64] = np.float32(2.5) * np.float32(2.0 ** -6)
+    w[4, 32] = 7 * 2.0 ** -6                          # exact half-way codes
+    w[5] *= 1000.0                                    # large but finite scales
+    return w
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+def test_host_quantiser_bit_exact_vs_oracle(fmt):
+    w = _edge_weights()
+    rc, codes, scales = _host_quantize(fmt, w)
+    assert rc == 0
+    oc, os_ = oracle.quantize_q4(w) if fmt == 4 else oracle.quantize_q8(w)
+    assert np.array_equal(codes.view(np.uint8), oc.view(np.uint8))
+    assert np.array_equal(scales, os_)
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+def test_host_quantiser_rejects_out_of_range(fmt):
+    w = np.zeros((1, 32), dtype=np.float32)
+    w[0, 3] = np.nan
+    assert _host_quantize(fmt, w)[0] == bq.BQ_ERR_RANGE
+    w[0, 3] = 1.0e7                                    # absmax/levels overflows fp16
+    assert _host_quantize(fmt, w)[0] == bq.BQ_ERR_RANGE
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+def test_host_dequantize_matches_oracle(fmt):
+    w = synth.weights_f32(synth.key(1, 93, 0, 0, 0), 9, 96)
+    codes, scales = oracle.quantize_q4(w) if fmt == 4 else oracle.quantize_q8(w)
+    out = np.zeros(w.shape, dtype=np.float32)
+    fn = bq.lib().bq_dequantize_q4 if fmt == 4 else bq.lib().bq_dequantize_q8
+    assert fn(codes.ctypes.data, scales.ctypes.data, 9, 96, out.ctypes.data) == 0
+    ref = oracle.dequantize_q4(codes, scales) if fmt == 4 else oracle.dequantize_q8(codes, scales)
+    assert np.array_equal(out.astype(np.float64), ref)
+
+
+def test_blocks_layout_matches_golden_and_round_trips():
+    g = read_golden("q4_block_worked.txt")
+    codes = np.array([[int(t, 16) for t in g["packed"]]], dtype=np.uint8)
+    scales = np.zeros((1, 8), dtype=np.uint16)
+    scales[0, 0] = int(g["scale_bits"][0], 16)
+    blk = np.zeros(18, dtype=np.uint8)
+    assert bq.lib().bq_planes_to_blocks_q4(codes.ctypes.data, scales.ctypes.data, 1, 32,
+                                           blk.ctypes.data) == 0
+    assert list(blk[:2]) == [0x00, 0x20]              # little-endian fp16 scale first
+    assert np.array_equal(blk[2:], codes[0])
+    r = np.random.default_rng(5)
+    for fmt, rec in ((4, 18), (8, 34)):
+        N, K = 7, 160
+        blocks = r.integers(0, 256, size=N * (K // 32) * rec, dtype=np.uint8)
+        c = np.zeros((N, K // 2 if fmt == 4 else K), dtype=np.uint8)
+        s = np.zeros((N, bq.scales_ld(K)), dtype=np.uint16)
+        to_p = bq.lib().bq_blocks_to_planes_q4 if fmt == 4 else bq.lib().bq_blocks_to_planes_q8
+        to_b = bq.lib().bq_planes_to_blocks_q4 if fmt == 4 else bq.lib().bq_planes_to_blocks_q8
+        assert to_p(blocks.ctypes.data, N, K, c.ctypes.data, s.ctypes.data) == 0
+        back = np.zeros_like(blocks)
+        assert to_b(c.ctypes.data, s.ctypes.data, N, K, back.ctypes.data) == 0
+        assert np.array_equal(back, blocks)
+        assert np.all(s[:, K // 32:] == 0)
+
+
+def test_workspace_sizes():
+    assert bq.lib().bq_gemv_workspace_bytes(0, 32) == 0
+    assert bq.lib().bq_gemv_workspace_bytes(16, 48) == 0
+    a = bq.lib().bq_gemv_workspace_bytes(2048, 2048)
+    b = bq.lib().bq_gemv_workspace_bytes(51200, 5120)
+    assert 0 < a < b < (64 << 20)
+    assert bq.lib().bq_moe_workspace_bytes(2048, 768, 8, 8, 128) > 0
+    assert bq.lib().bq_moe_workspace_bytes(2048, 768, 9, 8, 128) == 0
+    assert bq.lib().bq_moe_workspace_bytes(2048, 768, 8, 9, 128) == 0
+
+
+def _gemv_rc(fmt=4, W=None, x=FAKE, B=1, y=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    W = W if W is not None else bq.bq_qmat(FAKE, FAKE, 64, 256)
+    fn = bq.lib().bq_gemv_q4 if fmt == 4 else bq.lib().bq_gemv_q8
+    return fn(ctypes.byref(W), x, B, y, ws, ws_bytes, None, None)
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+def test_gemv_argument_validation_before_launch(fmt):
+    assert bq.lib().bq_gemv_q4(None, FAKE, 1, FAKE, FAKE, 1 << 30, None, None) == bq.BQ_ERR_NULL
+    assert _gemv_rc(fmt, W=bq.bq_qmat(None, FAKE, 64, 256)) == bq.BQ_ERR_NULL
+    assert _gemv_rc(fmt, x=None) == bq.BQ_ERR_NULL
+    assert _gemv_rc(fmt, ws=None) == bq.BQ_ERR_NULL
+    assert _gemv_rc(fmt, W=bq.bq_qmat(FAKE, FAKE, 64, 48)) == bq.BQ_ERR_SHAPE
+    assert _gemv_rc(fmt, W=bq.bq_qmat(FAKE, FAKE, 0, 256)) == bq.BQ_ERR_SHAPE
+    assert _gemv_rc(fmt, B=0) == bq.BQ_ERR_BATCH
+    assert _gemv_rc(fmt, B=9) == bq.BQ_ERR_BATCH
+    assert _gemv_rc(fmt, x=FAKE + 8) == bq.BQ_ERR_ALIGN
+    assert _gemv_rc(fmt, W=bq.bq_qmat(FAKE + 4, FAKE, 64, 256)) == bq.BQ_ERR_ALIGN
+    assert _gemv_rc(fmt, ws_bytes=1024) == bq.BQ_ERR_WORKSPACE
+
+
+def test_moe_argument_validation_before_launch():
+    W = bq.bq_qmat(FAKE, FAKE, 64, 256)
+    f = bq.lib().bq_moe_gemv_q4
+    cs, ss = 64 * 128, 64 * 8
+
+    def rc(**kw):
+        a = dict(W=W, E=16, cs=cs, ss=ss, x=FAKE, xps=0, idx=FAKE, rw=None, B=2, topk=4, y=FAKE,
+                 ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return f(ctypes.byref(a["W"]), a["E"], a["cs"], a["ss"], a["x"], a["xps"], a["idx"],
+                 a["rw"], a["B"], a["topk"], a["y"], a["ws"], a["wsb"], None, None)
+
+    assert rc(idx=None) == bq.BQ_ERR_NULL
+    assert rc(B=9) == bq.BQ_ERR_BATCH
+    assert rc(B=8, topk=9) == bq.BQ_ERR_BATCH
+    assert rc(E=0) == bq.BQ_ERR_SHAPE
+    assert rc(cs=cs - 16) == bq.BQ_ERR_SHAPE
+    assert rc(ss=ss + 4) == bq.BQ_ERR_ALIGN
+    assert rc(wsb=4096) == bq.BQ_ERR_WORKSPACE
+
+
+def test_device_quantiser_argument_validation():
+    f = bq.lib().bq_quantize_q4_dev
+    assert f(None, 4, 64, FAKE, FAKE, None, None) == bq.BQ_ERR_NULL
+    assert f(FAKE, 4, 60, FAKE, FAKE, None, None) == bq.BQ_ERR_SHAPE
+    assert f(FAKE + 4, 4, 64, FAKE, FAKE, None, None) == bq.BQ_ERR_ALIGN
+
+
+def test_product_path_has_no_oracle_or_fallback():
+    """The library and its binding never reference the oracle, and the binding
+    raises instead of falling back when the library is absent."""
+    pkg = os.path.join(ROOT, "quantised_weight_gemv_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                with open(os.path.join(dirpath, fn)) as f:
+                    src = f.read()
+                assert "import oracle" not in src and "from oracle" not in src, fn
+                assert "oracle.c" not in src and "liboracle" not in src, fn

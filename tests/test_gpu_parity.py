@@ -1,0 +1,203 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Inputs come from the seeded generators in quantised_weight_gemv_b200.synth;
+packed planes for the small cases come from the oracle's own quantiser, so no
+oracle input is produced by the CUDA path.  Tolerance per output element:
+|y - y_ref| <= 1e-3 * sum_k |deq(w) x| + 1e-5; packing is bit-exact.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from quantised_weight_gemv_b200 import bq, synth
+from tests.gpu_helpers import DEV, check_tol, dev, gpu_gemv, new_status, oracle_gemv, quantize
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(1, 32), (15, 32), (16, 256), (17, 288), (33, 800), (100, 2048), (257, 4128),
+          (1000, 96), (4, 25600), (48, 768)]
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+@pytest.mark.parametrize("N,K", SHAPES)
+@pytest.mark.parametrize("B", [1, 2, 3, 8])
+def test_gemv_parity_small(fmt, N, K, B):
+    w = synth.weights_f32(synth.key(0, 80, N, K, synth.KIND_W), N, K)
+    codes, scales = quantize(fmt, w)
+    x = synth.activations_f16_bits(synth.key(0, 80, N, K, synth.KIND_X), B, K)
+    y = gpu_gemv(fmt, codes, scales, x)
+    y_ref, absy = oracle_gemv(fmt, codes, scales, x)
+    check_tol(y, y_ref, absy)
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+def test_gemv_one_hot_is_correctly_rounded(fmt):
+    """x = e_k returns column k of deq(W); the only rounding is fp32's."""
+    N, K = 40, 512
+    w = synth.weights_f32(synth.key(1, 80, 0, 0, synth.KIND_W), N, K)
+    codes, scales = quantize(fmt, w)
+    for k0 in (0, 17, 255, 256, 500):
+        x = np.zeros((8, K), dtype=np.float16)
+        for b in range(8):
+            x[b, (k0 + 3 * b) % K] = np.float16(1.5 - 0.25 * b)
+        xb = x.view(np.uint16)
+        y = gpu_gemv(fmt, codes, scales, xb)
+        y_ref, _ = oracle_gemv(fmt, codes, scales, xb)
+        assert np.array_equal(y, y_ref.astype(np.float32))
+
+
+def test_q4_nibble_order_exhaustive_on_gpu():
+    """Row r = 32*c + p holds code c at element p (all other codes 8, d = 1):
+    with x = e_p the GPU must return c - 8 exactly at row 32*c + p."""
+    N, K = 512, 32
+    codes = np.full((N, 16), 0x88, dtype=np.uint8)
+    for c in range(16):
+        for p in range(32):
+            r = 32 * c + p
+            i = p % 16
+            codes[r, i] = (codes[r, i] & 0xF0) | c if p < 16 else (codes[r, i] & 0x0F) | (c << 4)
+    scales = np.zeros((N, 8), dtype=np.uint16)
+    scales[:, 0] = 0x3C00
+    for p0 in range(0, 32, 8):
+        x = np.zeros((8, K), dtype=np.float16)
+        for b in range(8):
+            x[b, p0 + b] = 1.0
+        y = gpu_gemv(4, codes, scales, x.view(np.uint16))
+        for b in range(8):
+            p = p0 + b
+            expect = np.zeros(N, dtype=np.float32)
+            for c in range(16):
+                expect[32 * c + p] = c - 8
+            assert np.array_equal(y[b], expect), p
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+def test_batch_columns_independent_and_deterministic(fmt):
+    N, K = 777, 3072
+    w = synth.weights_f32(synth.key(2, 80, 0, 0, synth.KIND_W), N, K)
+    codes, scales = quantize(fmt, w)
+    x = synth.activations_f16_bits(synth.key(2, 80, 0, 0, synth.KIND_X), 8, K)
+    y8 = gpu_gemv(fmt, codes, scales, x)
+    assert np.array_equal(y8, gpu_gemv(fmt, codes, scales, x))
+    for b in range(8):
+        assert np.array_equal(gpu_gemv(fmt, codes, scales, x[b:b + 1])[0], y8[b])
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+def test_device_quantiser_bit_exact(fmt):
+    import torch
+    from tests.test_abi_cpu import _edge_weights
+    w = _edge_weights()
+    N, K = w.shape
+    codes_ref, scales_ref = quantize(fmt, w)
+    c = torch.zeros((N, K // 2 if fmt == 4 else K), dtype=torch.uint8, device=DEV)
+    s = torch.full((N, bq.scales_ld(K)), 0x1234, dtype=torch.int16, device=DEV)
+    st = new_status()
+    bq.quantize_dev(fmt, dev(w), c, s, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(c.cpu().numpy(), codes_ref.view(np.uint8))
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), scales_ref)
+    wbad = w.copy()
+    wbad[7, 40] = np.inf
+    bq.quantize_dev(fmt, dev(wbad), c, s, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 1 << bq.BQ_ERR_RANGE
+
+
+def test_workspace_counters_return_to_zero():
+    import torch
+    N, K = 300, 5120
+    w = synth.weights_f32(synth.key(3, 80, 0, 0, synth.KIND_W), N, K)
+    codes, scales = quantize(4, w)
+    ws = bq.workspace(bq.lib().bq_gemv_workspace_bytes(N, K), DEV)
+    x = synth.activations_f16_bits(synth.key(3, 80, 0, 0, synth.KIND_X), 2, K)
+    y1 = gpu_gemv(4, codes, scales, x, ws=ws)
+    y2 = gpu_gemv(4, codes, scales, x, ws=ws)
+    assert np.array_equal(y1, y2)
+    nb = (N + 15) // 16
+    assert int(ws[: nb * 4].view(torch.int32).abs().sum().item()) == 0
+
+
+# ---------------------------------------------------------------- experts ----
+def _moe_inputs(E, N, K, B, topk, seed, x_per_slot):
+    cs, ss = [], []
+    for e in range(E):
+        c, s = oracle.quantize_q4(synth.weights_f32(synth.key(seed, 81, 0, e, synth.KIND_W), N, K))
+        cs.append(c)
+        ss.append(s)
+    codes, scales = np.stack(cs), np.stack(ss)
+    shape = (B, topk, K) if x_per_slot else (B, K)
+    x = synth.activations_f16_bits(synth.key(seed, 81, 0, 0, synth.KIND_X), *shape)
+    idx, r = synth.routing(synth.key(seed, 81, 0, 0, synth.KIND_IDX),
+                           synth.key(seed, 81, 0, 0, synth.KIND_LOGIT), B, E, topk)
+    return codes, scales, x, idx, r
+
+
+def gpu_moe(codes, scales, x, x_per_slot, idx, r):
+    import torch
+    E, N, K2 = codes.shape
+    K = 2 * K2
+    B, topk = idx.shape
+    c, s = dev(codes), dev(scales)
+    xt, it = dev(x), dev(idx)
+    rt = dev(r) if r is not None else None
+    y = torch.full((B, N) if r is not None else (B, topk, N), float("nan"),
+                   dtype=torch.float32, device=DEV)
+    ws = bq.workspace(bq.lib().bq_moe_workspace_bytes(N, K, B, topk, E), DEV)
+    st = new_status()
+    bq.moe_gemv_q4(bq.qmat(c, s, N, K), E, N * K2, N * scales.shape[2], xt, x_per_slot, it, rt,
+                   y, ws, st)
+    torch.cuda.synchronize()
+    return y.cpu().numpy(), int(st.item())
+
+
+@pytest.mark.parametrize("B,topk,E", [(1, 8, 32), (8, 8, 32), (3, 4, 5), (8, 2, 1)])
+@pytest.mark.parametrize("x_per_slot", [False, True])
+@pytest.mark.parametrize("combine", [False, True])
+def test_moe_parity(B, topk, E, x_per_slot, combine):
+    N, K = 96, 768
+    if E < topk:
+        pytest.skip("needs E >= topk for sampling without replacement")
+    codes, scales, x, idx, r = _moe_inputs(E, N, K, B, topk, B * 100 + topk, x_per_slot)
+    rr = r if combine else None
+    y, st = gpu_moe(codes, scales, x, x_per_slot, idx, rr)
+    assert st == 0
+    y_ref, absy, bad = oracle.moe_gemv_q4(codes, scales, x, x_per_slot, idx, rr, nthreads=8)
+    assert not bad
+    check_tol(y, y_ref, absy)
+
+
+def test_moe_repeated_expert_and_many_tokens():
+    """All 8 tokens route all slots to a few experts (pieces of > 8 slots are
+    split), including one token that lists the same expert twice."""
+    N, K, B, topk, E = 64, 512, 8, 4, 6
+    codes, scales, x, _, r = _moe_inputs(E, N, K, B, topk, 9, True)
+    idx = np.array([[0, 1, 2, 3]] * 7 + [[5, 5, 0, 1]], dtype=np.int32)
+    for rr in (None, r):
+        y, st = gpu_moe(codes, scales, x, True, idx, rr)
+        assert st == 0
+        y_ref, absy, _ = oracle.moe_gemv_q4(codes, scales, x, True, idx, rr)
+        check_tol(y, y_ref, absy)
+
+
+def test_moe_out_of_range_index_sets_status_no_trap():
+    N, K, B, topk, E = 32, 256, 2, 2, 4
+    codes, scales, x, _, r = _moe_inputs(E, N, K, B, topk, 11, False)
+    idx = np.array([[0, 4], [-3, 1]], dtype=np.int32)
+    for rr in (None, r):
+        y, st = gpu_moe(codes, scales, x, False, idx, rr)
+        assert st == 1 << bq.BQ_ERR_EXPERT_INDEX
+        y_ref, absy, bad = oracle.moe_gemv_q4(codes, scales, x, False, idx, rr)
+        assert bad
+        check_tol(y, y_ref, absy)
+
+
+def test_moe_single_expert_matches_dense():
+    N, K, B = 200, 1024, 6
+    codes, scales, x, _, _ = _moe_inputs(3, N, K, B, 1, 12, False)
+    idx = np.full((B, 1), 1, dtype=np.int32)
+    y, st = gpu_moe(codes, scales, x, False, idx, None)
+    assert st == 0
+    yd = gpu_gemv(4, codes[1], scales[1], x)
+    np.testing.assert_array_equal(y[:, 0], yd)
