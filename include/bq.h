@@ -132,6 +132,53 @@ BQ_API int32_t bq_gemv_q4(const bq_qmat *W, const uint16_t *x, int32_t B, float 
 BQ_API int32_t bq_gemv_q8(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
                    void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
 
+/* --------------------------------------------------------- decode step --- */
+
+/* One matrix of a decode step.  All planes and buffers are device memory. */
+typedef struct bq_step_mat {
+    bq_qmat W;            /* the quantised matrix (plane layout above) */
+    const uint16_t *x;    /* fp16 bits [B][K], 16-byte aligned */
+    float *y;             /* fp32 [B][N], 16-byte aligned, overwritten */
+    int32_t B;            /* 1..8 */
+    int32_t stage;        /* >= 0; stages run in increasing order */
+} bq_step_mat;
+
+/* Host-side description of a built plan (filled by bq_step_plan). */
+typedef struct bq_step_info {
+    int32_t fmt, n_mats, n_stages, grid, max_stage_bands, reserved;
+    uint64_t stages_off, mats_off;   /* byte offsets inside the device plan */
+    uint64_t ws_bytes;               /* workspace bq_step_run needs */
+} bq_step_info;
+
+/* Device bytes a plan of n_mats matrices needs (0 if n_mats < 1). */
+BQ_API size_t bq_step_plan_bytes(int32_t n_mats);
+
+/* Build, once (e.g. at model load), the plan of a whole decode step: every
+ * matrix of one token's forward pass, grouped in stages.  Matrices of one
+ * stage are independent; a later stage may read what an earlier one wrote,
+ * so stages are separated by a grid-wide barrier inside the single launch
+ * bq_step_run makes.  The launch-per-projection overhead that dominates
+ * small models at decode (gist.science technical summary, "Resultaten":
+ * the fixed per-token overhead; "Kernel Fusie": launch overhead matters
+ * because decode kernels are short) becomes one launch per token.
+ *   fmt        4 or 8 (every matrix of the plan has this format)
+ *   mats       host array of n_mats matrices (any order; stable by stage)
+ *   plan       device buffer, 64-byte aligned, >= bq_step_plan_bytes(n_mats);
+ *              written synchronously (cudaMemcpy) -- do not call during
+ *              stream capture
+ *   info       host struct filled on success
+ * The plan holds the planes' addresses and x / y pointers; those buffers
+ * must stay allocated while the plan is used. */
+BQ_API int32_t bq_step_plan(int32_t fmt, const bq_step_mat *mats, int32_t n_mats, void *plan,
+                            size_t plan_bytes, bq_step_info *info);
+
+/* Run one decode step of a plan: one cooperative launch (its grid is sized
+ * for co-residency on the device the plan was built on).
+ *   ws      device workspace, >= info->ws_bytes, zero-filled before first use
+ *           (left zero-filled on completion) */
+BQ_API int32_t bq_step_run(const bq_step_info *info, const void *plan, void *ws, size_t ws_bytes,
+                           int32_t *dev_status, void *stream);
+
 /* ------------------------------------------------------ routed experts --- */
 
 /* Bytes of workspace bq_moe_gemv_q4 needs.  0 on a bad shape. */

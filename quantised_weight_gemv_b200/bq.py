@@ -24,6 +24,19 @@ class bq_qmat(ctypes.Structure):
                 ("N", ctypes.c_int32), ("K", ctypes.c_int32)]
 
 
+class bq_step_mat(ctypes.Structure):
+    _fields_ = [("W", bq_qmat), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("B", ctypes.c_int32), ("stage", ctypes.c_int32)]
+
+
+class bq_step_info(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("n_mats", ctypes.c_int32),
+                ("n_stages", ctypes.c_int32), ("grid", ctypes.c_int32),
+                ("max_stage_bands", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("stages_off", ctypes.c_uint64), ("mats_off", ctypes.c_uint64),
+                ("ws_bytes", ctypes.c_uint64)]
+
+
 class BQError(RuntimeError):
     def __init__(self, fn: str, status: int):
         super().__init__(f"{fn}: {bq_status_string(status)} ({status})")
@@ -33,6 +46,8 @@ class BQError(RuntimeError):
 _lib = None
 _vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
 _QP = ctypes.POINTER(bq_qmat)
+_SMP = ctypes.POINTER(bq_step_mat)
+_SIP = ctypes.POINTER(bq_step_info)
 
 # name -> (restype, argtypes); mirrors include/bq.h
 _SIGS = {
@@ -41,6 +56,9 @@ _SIGS = {
     "bq_gemv_workspace_bytes": (_sz, [_i32, _i32]),
     "bq_gemv_q4": (_i32, [_QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
     "bq_gemv_q8": (_i32, [_QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
+    "bq_step_plan_bytes": (_sz, [_i32]),
+    "bq_step_plan": (_i32, [_i32, _SMP, _i32, _vp, _sz, _SIP]),
+    "bq_step_run": (_i32, [_SIP, _vp, _vp, _sz, _vp, _vp]),
     "bq_moe_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "bq_moe_gemv_q4": (_i32, [_QP, _i32, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _i32, _vp,
                               _vp, _sz, _vp, _vp]),
@@ -101,8 +119,13 @@ def _stream_ptr(stream) -> int:
 
 
 def qmat(codes, scales, N: int, K: int) -> bq_qmat:
-    """bq_qmat over two tensors (device planes for GEMV, host for pack calls)."""
-    return bq_qmat(codes.data_ptr(), scales.data_ptr(), int(N), int(K))
+    """bq_qmat over two tensors (device planes for GEMV, host for pack calls).
+
+    The struct keeps references to both tensors, so their memory stays
+    allocated for as long as the bq_qmat is alive."""
+    m = bq_qmat(codes.data_ptr(), scales.data_ptr(), int(N), int(K))
+    m._refs = (codes, scales)
+    return m
 
 
 def scales_ld(K: int) -> int:
@@ -132,6 +155,34 @@ def moe_gemv_q4(Wstack: bq_qmat, E: int, codes_stride: int, scales_stride: int, 
                               _ptr(route_w), B, topk, y.data_ptr(), ws.data_ptr(),
                               ws.numel() * ws.element_size(), _ptr(status), _stream_ptr(stream))
     check("bq_moe_gemv_q4", rc)
+
+
+class StepPlan:
+    """A decode-step plan: device plan buffer + host info + workspace (torch
+    allocations owned by this object), built once by bq_step_plan."""
+
+    def __init__(self, fmt: int, entries, device):
+        """entries: iterable of (bq_qmat, x, y, stage) with device tensors."""
+        import torch
+        entries = list(entries)
+        arr = (bq_step_mat * len(entries))()
+        self._refs = []
+        for i, (W, x, y, stage) in enumerate(entries):
+            arr[i] = bq_step_mat(W, x.data_ptr(), y.data_ptr(), int(x.shape[0]), int(stage))
+            self._refs += [W, x, y]
+        nbytes = lib().bq_step_plan_bytes(len(entries))
+        self.plan = torch.empty(nbytes + 64, dtype=torch.uint8, device=device)
+        off = (-self.plan.data_ptr()) % 64
+        self.plan_ptr = self.plan.data_ptr() + off
+        self.info = bq_step_info()
+        check("bq_step_plan", lib().bq_step_plan(int(fmt), arr, len(entries), self.plan_ptr,
+                                                 nbytes, ctypes.byref(self.info)))
+        self.ws = workspace(self.info.ws_bytes, device)
+
+    def run(self, status=None, stream=None) -> None:
+        check("bq_step_run", lib().bq_step_run(ctypes.byref(self.info), self.plan_ptr,
+                                               self.ws.data_ptr(), self.ws.numel(), _ptr(status),
+                                               _stream_ptr(stream)))
 
 
 def quantize_dev(fmt: int, w, codes, scales, status=None, stream=None) -> None:

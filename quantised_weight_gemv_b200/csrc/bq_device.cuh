@@ -42,7 +42,7 @@ template <int FMT> struct Fmt;
 template <> struct Fmt<4> {
     static constexpr int kCodeBytes = kBoxBytes;       // 16 rows x 128 B
     static constexpr int kBoxes = 1;
-    static constexpr int kStages = 5;
+    static constexpr int kStages = 4;
 };
 template <> struct Fmt<8> {
     static constexpr int kCodeBytes = 2 * kBoxBytes;   // 16 rows x 256 B
@@ -150,29 +150,23 @@ __device__ __forceinline__ void pdl_wait()
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t addr)
+// Shared-memory reads through ordinary pointers: the compiler sees them as
+// loads, so it can schedule them freely between the mbarrier waits (whose asm
+// carries a memory clobber) but never across one.
+__device__ __forceinline__ uint32_t lds32(const uint8_t *p)
 {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
+    return *reinterpret_cast<const uint32_t *>(p);
 }
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr)
+__device__ __forceinline__ uint4 lds128(const uint8_t *p)
 {
-    uint4 v;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr));
-    return v;
+    return *reinterpret_cast<const uint4 *>(p);
 }
 
-// 8 bytes of x through the read-only path; zero when !pred.
-__device__ __forceinline__ uint2 ldg64_pred(const void *p, bool pred)
+// 8 bytes of x through the read-only, L1-cached path.
+__device__ __forceinline__ uint2 ldg64(const void *p)
 {
-    uint2 v = make_uint2(0u, 0u);
-    if (pred)
-        v = __ldg(reinterpret_cast<const uint2 *>(p));
-    return v;
+    return __ldg(reinterpret_cast<const uint2 *>(p));
 }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
@@ -200,8 +194,7 @@ __device__ __forceinline__ uint32_t hfma2u(uint32_t a, uint32_t b, uint32_t c)
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1, const float (&c)[4])
 {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
         "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
         : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]),
@@ -267,22 +260,22 @@ __device__ __forceinline__ uint32_t pick_u32(const uint4 &v, int i)
 // `xa` holds x at k..k+3 and `xb` at k+16..k+19 (k = block start + 4t) for
 // batch column g (zero if the column is absent).
 template <int FMT>
-__device__ __forceinline__ void block_mma(uint32_t codes_s, int jb, int g, int t, uint2 xa,
+__device__ __forceinline__ void block_mma(const uint8_t *codes_s, int jb, int g, int t, uint2 xa,
                                           uint2 xb, float dg, float dg8, float (&acc)[4])
 {
     const float zero[4] = {0.f, 0.f, 0.f, 0.f};
     float c[4];
     if constexpr (FMT == 4) {
-        const uint32_t off = (uint32_t)(g * 128 + (((jb ^ g) & 7) << 4) + 4 * t);
+        const int off = g * 128 + (((jb ^ g) & 7) << 4) + 4 * t;
         const Q4Pairs r0 = dequant_q4(lds32(codes_s + off));          // row g
         const Q4Pairs r8 = dequant_q4(lds32(codes_s + off + 1024));   // row g + 8
         mma16816(c, r0.lo01, r8.lo01, r0.lo23, r8.lo23, xa.x, xa.y, zero);
         mma16816(c, r0.hi01, r8.hi01, r0.hi23, r8.hi23, xb.x, xb.y, c);
     } else {
         const int box = jb >> 2, jj = jb & 3;
-        const uint32_t base = codes_s + (uint32_t)(box * kBoxBytes + g * 128 + 4 * t);
-        const uint32_t oa = (uint32_t)((((2 * jj) ^ g) & 7) << 4);
-        const uint32_t ob = (uint32_t)((((2 * jj + 1) ^ g) & 7) << 4);
+        const uint8_t *base = codes_s + box * kBoxBytes + g * 128 + 4 * t;
+        const int oa = (((2 * jj) ^ g) & 7) << 4;
+        const int ob = (((2 * jj + 1) ^ g) & 7) << 4;
         const Q8Pairs a0 = dequant_q8(lds32(base + oa));
         const Q8Pairs a8 = dequant_q8(lds32(base + oa + 1024));
         const Q8Pairs b0 = dequant_q8(lds32(base + ob));
@@ -297,22 +290,23 @@ __device__ __forceinline__ void block_mma(uint32_t codes_s, int jb, int g, int t
 }
 
 // A whole chunk: blocks kb0 .. kb0+7 (k0 = 32*kb0 along K), nblk of them valid.
-// xrow points at x[column g][0] or is null when the column is absent.
+// xrow points at x[column g][0].  A lane whose column is absent (g >= B) reads
+// a valid row instead; its mma column is garbage and is never stored, which
+// keeps every load unconditional.
 template <int FMT>
-__device__ __forceinline__ void chunk_mma(uint32_t codes_s, uint32_t scales_s,
+__device__ __forceinline__ void chunk_mma(const uint8_t *codes_s, const uint8_t *scales_s,
                                           const __half *xrow, int k0, int nblk, int g, int t,
                                           float (&acc)[4])
 {
     const uint4 sg = lds128(scales_s + g * 16);
     const uint4 sg8 = lds128(scales_s + (g + 8) * 16);
-    const bool has_x = xrow != nullptr;
-    const __half *xp = has_x ? xrow + k0 + 4 * t : nullptr;
+    const __half *xp = xrow + k0 + 4 * t;
     if (nblk == 8) {
         uint2 xa[8], xb[8];
 #pragma unroll
         for (int jb = 0; jb < 8; jb++) {
-            xa[jb] = ldg64_pred(xp + 32 * jb, has_x);
-            xb[jb] = ldg64_pred(xp + 32 * jb + 16, has_x);
+            xa[jb] = ldg64(xp + 32 * jb);
+            xb[jb] = ldg64(xp + 32 * jb + 16);
         }
 #pragma unroll
         for (int jb = 0; jb < 8; jb++) {
@@ -325,8 +319,8 @@ __device__ __forceinline__ void chunk_mma(uint32_t codes_s, uint32_t scales_s,
 #pragma unroll
         for (int jb = 0; jb < 8; jb++) {
             if (jb < nblk) {
-                const uint2 xa = ldg64_pred(xp + 32 * jb, has_x);
-                const uint2 xb = ldg64_pred(xp + 32 * jb + 16, has_x);
+                const uint2 xa = ldg64(xp + 32 * jb);
+                const uint2 xb = ldg64(xp + 32 * jb + 16);
                 const uint32_t wg = pick_u32(sg, jb >> 1), wg8 = pick_u32(sg8, jb >> 1);
                 const float dg = (jb & 1) ? half_hi(wg) : half_lo(wg);
                 const float dg8 = (jb & 1) ? half_hi(wg8) : half_lo(wg8);

@@ -1,40 +1,51 @@
 // stream_gemv.cu -- the streamed decode GEMV over block-quantised weights
-// (dense Q4/Q8 and grouped routed-expert Q4), sm_100a.
+// (dense Q4/Q8, whole decode steps, grouped routed-expert Q4), sm_100a.
 //
 // The decode step is a GEMV per quantisation format with the dequantisation
 // inside the inner loop (BaseRT, gist.science technical summary,
 // "Methodologie" -> "Kernel Fusie en Specialisatie"), and it is bound by
-// memory bandwidth ("De 'Big Model' Realiteit"; the follow-up paper's
-// results paragraph says the same of its decode path).  So the design goal
-// here is one thing: keep HBM busy with the packed weight bytes and read each
-// of them exactly once.
+// memory bandwidth ("De 'Big Model' Realiteit"; the follow-up paper's results
+// paragraph says the same of its decode path).  The design goal is one thing:
+// keep HBM busy with the packed weight bytes and read each of them once.
 //
-// Work decomposition (stream-K over chunks).  A matrix is cut into bands of
-// 16 rows, a band into chunks of 256 weights along K; chunks are numbered
-// band-major (all chunks of band 0, then band 1, ...).  Every warp of the grid
-// is an independent worker that takes one contiguous range of that numbering
-// (ranges differ by at most one chunk, so every SM streams the same number of
-// bytes whatever the matrix shape).  A worker owns a ring of shared-memory
-// slots and its own mbarriers; its lane 0 keeps `stages - 1` chunks of TMA
-// loads in flight ahead of the chunk the warp is computing.
+// Work decomposition (stream-K over chunks).  A matrix is cut into bands of 16
+// rows and a band into chunks of 256 weights along K; chunks are numbered
+// band-major.  Every warp of the grid is an independent worker that owns a
+// ring of shared-memory slots with its own mbarriers; its lane 0 keeps
+// `stages - 1` chunks of TMA loads in flight ahead of the chunk the warp is
+// computing.  Worker w takes chunks [w*cpw, (w+1)*cpw) of a stage, where cpw =
+// ceil(chunks / workers), so every SM streams the same number of bytes
+// whatever the matrix shapes.
 //
-// A band that lies wholly inside one worker's range is written straight to y.
-// A band cut by range boundaries is summed deterministically: each worker that
-// touched it stores its fp32 partial (16 rows x 8 columns) in the workspace and
-// bumps the band's arrival counter; the last to arrive adds the partials in
-// worker order, writes y and resets the counter to zero.  No worker ever waits
-// for another.
+// A band wholly inside one worker's range is written straight to y.  A band
+// cut by range boundaries is summed deterministically: each worker that
+// touched it stores its fp32 partial (16 rows x 8 columns) in the workspace
+// and bumps the band's arrival counter; the last to arrive adds the partials
+// in worker order, writes y and resets the counter.  No worker waits for
+// another.
 //
-// Routed experts: every CTA sorts the (token, slot) -> expert list (at most 64
-// entries) in shared memory, which gives the same grouping on every CTA
-// without a separate kernel.  Each distinct expert (split into pieces of at
-// most 8 routed slots, the mma's N) becomes one "matrix" of the stream-K
-// numbering, so each routed expert's weights are read once and multiplied
-// with all of its tokens.  Per-slot outputs are written directly; the
-// routing-weighted combine runs as a second small kernel in slot order.
+// Three modes share that worker loop:
+//  - one matrix (bq_gemv_q4 / _q8): its descriptor is a kernel parameter;
+//  - a decode step (bq_step_run): a plan in device memory lists matrices in
+//    stages; stage s+1 may read what stage s wrote (in a model, the next
+//    projection's input), so the persistent, co-resident grid passes a grid
+//    barrier between stages.  Weight loads never wait for it: a worker's ring
+//    runs ahead across stage boundaries, so HBM keeps streaming the next
+//    stage's weights while the barrier settles.  The fixed per-token launch
+//    and dispatch cost the pages single out for small models (gist.science
+//    technical summary, "Resultaten" and "Kernel Fusie") becomes one launch
+//    per token;
+//  - routed experts (bq_moe_gemv_q4): every CTA sorts the (token, slot) ->
+//    expert list (at most 64 entries) in shared memory, which gives the same
+//    grouping on every CTA without a separate kernel; each distinct expert,
+//    cut into pieces of at most 8 routed slots (the mma's N), becomes one
+//    matrix of the numbering, so each routed expert's weights are read once
+//    for all of its tokens.
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <cstring>
+#include <vector>
 
 #include "bq_device.cuh"
 #include "bq_internal.h"
@@ -42,19 +53,46 @@
 namespace bq {
 
 constexpr int kMaxSlots = 64;   // B * topk
+constexpr int kModeMatrix = 0, kModePlan = 1, kModeMoE = 2;
+constexpr uint32_t kPlanMagic = 0x42515031u;   // "BQP1"
 
-struct GemvArgs {
+struct alignas(64) MatDesc {
     CUtensorMap tm_codes;
     CUtensorMap tm_scales;
-    const __half *x;
-    float *out;         // dense: y [B][N]; experts: per-slot [B*topk][N]
+    const __half *x;     // [B][K]
+    float *y;            // [B][N]
     int N, K, B;
-    int cpb;            // chunks per band
-    int nbands;         // bands per matrix (or per expert piece)
-    int wmax;           // gridDim.x * kWarps
-    int *counters;      // one per (piece, band), zero on entry and exit
-    float *partials;    // [wmax][2][128]
-    int *status;        // device status word or null
+    int cpb;             // chunks per band
+    int nbands;
+    int chunk_base;      // first chunk of this matrix within its stage
+    int band_base;       // first arrival counter of this matrix within its stage
+};
+
+struct StageDesc {
+    int mat_begin, mat_end;
+    int T;               // chunks in the stage
+    int cpw;             // chunks per worker
+    int W;               // workers with a non-empty range
+    int nbands;          // bands in the stage
+};
+
+struct PlanHeader {
+    uint32_t magic;
+    int fmt, n_mats, n_stages, grid, max_stage_bands;
+    uint64_t stages_off, mats_off;   // byte offsets from the plan base
+};
+
+struct KernelArgs {
+    MatDesc mat0;                    // matrix / routed-expert modes
+    StageDesc stage0;
+    const MatDesc *mats;             // plan mode (device memory)
+    const StageDesc *stages;
+    int n_stages;
+    int wmax;                        // gridDim.x * kWarps
+    int *counters;                   // per band of a stage; zero on entry and exit
+    float *partials;                 // [wmax][2][128]
+    int *status;                     // device status word or null
+    unsigned *sync;                  // plan mode: [0] barrier arrivals, [1] exits
     // routed experts
     int E, topk, x_per_slot;
     const int *idx;
@@ -72,10 +110,10 @@ struct ExpertGroups {
 
 // Sort the routed slots by (expert, slot) and cut them into pieces of at most
 // 8 slots of one expert.  Run by warp 0; invalid indices are left out.
-__device__ void group_experts(const GemvArgs &a, ExpertGroups &grp)
+__device__ void group_experts(const KernelArgs &a, ExpertGroups &grp)
 {
     const int lane = threadIdx.x & 31;
-    const int M = a.B * a.topk;
+    const int M = a.mat0.B * a.topk;
     for (int i = lane; i < M; i += 32) {
         const int e = a.idx[i];
         grp.key[i] = (e >= 0 && e < a.E) ? e * kMaxSlots + i : 0x7fffffff;
@@ -112,223 +150,351 @@ __device__ void group_experts(const GemvArgs &a, ExpertGroups &grp)
     __syncwarp();
 }
 
-// Index of the worker whose range holds chunk c (ranges: [w*T/W, (w+1)*T/W)).
-__device__ __forceinline__ long long worker_of(long long c, long long T, long long W)
+// Position of a chunk inside a stage: matrix (or expert piece) u, band, k-piece.
+struct Cursor {
+    int s;        // stage
+    int u;        // matrix index (plan: global; otherwise 0 / piece)
+    int band, kp;
+    int c, c_end; // chunk index within the stage and end of this worker's range
+};
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
 {
-    return ((c + 1) * W - 1) / T;
-}
-__device__ __forceinline__ long long range_start(long long w, long long T, long long W)
-{
-    return w * T / W;
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
-template <int FMT, bool MOE>
-__global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_constant__ GemvArgs a)
+template <int FMT, int MODE>
+__global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_constant__ KernelArgs a)
 {
     constexpr int D = Fmt<FMT>::kStages;
     constexpr int CB = Fmt<FMT>::kCodeBytes;
     constexpr uint32_t kTx = CB + kScaleBytes;
+    constexpr bool MOE = MODE == kModeMoE;
+    constexpr bool PLAN = MODE == kModePlan;
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ ExpertGroups grp;
+    __shared__ int cta_arrivals;
+    __shared__ alignas(8) uint64_t stage_bar;
 
-    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const uint32_t codes_ring = base + (uint32_t)(warp * D * CB);
-    const uint32_t scales_ring = base + (uint32_t)(kWarps * D * CB + warp * D * kScaleBytes);
-    const uint32_t bars = base + (uint32_t)(kWarps * D * (CB + kScaleBytes) + warp * D * 8);
+    uint8_t *codes_ring = sbase + warp * D * CB;
+    uint8_t *scales_ring = sbase + kWarps * D * CB + warp * D * kScaleBytes;
+    const uint32_t bars = smem_u32(sbase + kWarps * D * (CB + kScaleBytes) + warp * D * 8);
 
-    pdl_launch_dependents();
-    // Everything below reads x / idx or writes the outputs and the workspace,
-    // so it waits for the previous kernel on the stream.
-    pdl_wait();
-
-    long long units = 1;
-    if constexpr (MOE) {
-        if (warp == 0)
-            group_experts(a, grp);
-        __syncthreads();
-        units = grp.npieces;
-        // CTA 0 reports invalid indices and zeroes their per-slot outputs.
-        if (blockIdx.x == 0 && grp.nvalid < a.B * a.topk) {
-            if (threadIdx.x == 0 && a.status)
-                atomicOr(a.status, kStatusExpertIndex);
-            if (a.out) {
-                for (int i = 0; i < a.B * a.topk; i++) {
-                    if (grp.key[i] != 0x7fffffff)
-                        continue;
-                    for (int r = threadIdx.x; r < a.N; r += kThreads)
-                        a.out[(size_t)i * a.N + r] = 0.f;
-                }
-            }
-        }
-    }
-
-    const long long bands_total = units * a.nbands;
-    const long long T = bands_total * a.cpb;
-    const long long W = T < a.wmax ? T : a.wmax;
-    const long long w = (long long)warp * gridDim.x + blockIdx.x;
-    if (w >= W)
-        return;
+    const MatDesc *mats = PLAN ? a.mats : &a.mat0;
+    const StageDesc *stg = PLAN ? a.stages : &a.stage0;
+    const int n_stages = PLAN ? a.n_stages : 1;
 
     if (lane == 0) {
         for (int s = 0; s < D; s++)
             mbar_init(bars + 8 * s, 1);
-        fence_barrier_init();
-        prefetch_tensormap(&a.tm_codes);
-        prefetch_tensormap(&a.tm_scales);
     }
-    __syncwarp();
+    if (PLAN && threadIdx.x == 0) {
+        cta_arrivals = 0;
+        mbar_init(smem_u32(&stage_bar), 1);
+    }
+    if (lane == 0)
+        fence_barrier_init();
 
-    const long long c0 = range_start(w, T, W);
-    const long long c1 = range_start(w + 1, T, W);
-    const int n = (int)(c1 - c0);
-    const uint64_t pol = policy_evict_first();
-    const int nb32 = a.K / kBlock;
+    pdl_launch_dependents();
+    // Everything below reads inputs or writes outputs and the workspace, so it
+    // waits for the previous kernel on the stream to complete.
+    pdl_wait();
 
-    auto issue = [&](int i) {
-        if (lane != 0)
-            return;
-        const long long c = c0 + i;
-        const long long gb = c / a.cpb;
-        const int kp = (int)(c - gb * a.cpb);
-        const int unit = (int)(gb / a.nbands);
-        const int row = (int)(gb - (long long)unit * a.nbands) * kChunkRows;
-        const int slot = i % D;
-        const uint32_t bar = bars + 8 * slot;
-        const uint32_t cdst = codes_ring + (uint32_t)(slot * CB);
-        const uint32_t sdst = scales_ring + (uint32_t)(slot * kScaleBytes);
-        mbar_arrive_expect_tx(bar, kTx);
-        if constexpr (MOE) {
-            const int e = grp.piece_expert[unit];
-            tma_load_3d(cdst, &a.tm_codes, bar, kp * 128, row, e, pol);
-            tma_load_3d(sdst, &a.tm_scales, bar, kp * 8, row, e, pol);
-        } else {
-#pragma unroll
-            for (int bx = 0; bx < Fmt<FMT>::kBoxes; bx++)
-                tma_load_2d(cdst + bx * kBoxBytes, &a.tm_codes, bar,
-                            kp * 128 * Fmt<FMT>::kBoxes + bx * 128, row, pol);
-            tma_load_2d(sdst, &a.tm_scales, bar, kp * 8, row, pol);
+    StageDesc moe_stage;
+    if constexpr (MOE) {
+        if (warp == 0)
+            group_experts(a, grp);
+        __syncthreads();
+        // CTA 0 reports invalid indices and zeroes their per-slot outputs.
+        if (blockIdx.x == 0 && grp.nvalid < a.mat0.B * a.topk) {
+            if (threadIdx.x == 0 && a.status)
+                atomicOr(a.status, kStatusExpertIndex);
+            for (int i = 0; i < a.mat0.B * a.topk; i++) {
+                if (grp.key[i] != 0x7fffffff)
+                    continue;
+                for (int r = threadIdx.x; r < a.mat0.N; r += kThreads)
+                    a.mat0.y[(size_t)i * a.mat0.N + r] = 0.f;
+            }
         }
+        moe_stage = a.stage0;
+        moe_stage.nbands = grp.npieces * a.mat0.nbands;
+        moe_stage.T = moe_stage.nbands * a.mat0.cpb;
+        moe_stage.cpw = (moe_stage.T + a.wmax - 1) / a.wmax;
+        if (moe_stage.cpw < 1)
+            moe_stage.cpw = 1;
+        moe_stage.W = (moe_stage.T + moe_stage.cpw - 1) / moe_stage.cpw;
+        stg = &moe_stage;
+    } else {
+        __syncthreads();
+    }
+
+    const int w = warp * gridDim.x + blockIdx.x;
+    const uint64_t pol = policy_evict_first();
+
+    // Per-unit geometry (matrix, or expert piece in MoE mode).
+    auto unit_mat = [&](int u) -> const MatDesc & { return MOE ? a.mat0 : mats[u]; };
+    auto unit_cpb = [&](int u) { return unit_mat(u).cpb; };
+    auto unit_nbands = [&](int u) { return unit_mat(u).nbands; };
+    auto unit_chunk_base = [&](int u) {
+        return MOE ? u * a.mat0.nbands * a.mat0.cpb : mats[u].chunk_base;
     };
+    auto unit_band_base = [&](int u) { return MOE ? u * a.mat0.nbands : mats[u].band_base; };
+
+    // Place a cursor at the first chunk of this worker's range in stage s, or
+    // at the first later stage where the range is non-empty.  Returns false
+    // when no stage >= s has work for this worker.
+    auto seek = [&](Cursor &cu, int s) -> bool {
+        for (; s < n_stages; s++) {
+            const StageDesc &st = stg[s];
+            if (w >= st.W)
+                continue;
+            const int c0 = w * st.cpw;
+            const int c1 = min(c0 + st.cpw, st.T);
+            int u = MOE ? c0 / (a.mat0.nbands * a.mat0.cpb) : st.mat_begin;
+            if (!MOE)
+                while (u + 1 < st.mat_end && mats[u + 1].chunk_base <= c0)
+                    u++;
+            const int rel = c0 - unit_chunk_base(u);
+            cu.s = s;
+            cu.u = u;
+            cu.band = rel / unit_cpb(u);
+            cu.kp = rel - cu.band * unit_cpb(u);
+            cu.c = c0;
+            cu.c_end = c1;
+            return true;
+        }
+        cu.s = n_stages;
+        return false;
+    };
+    auto advance = [&](Cursor &cu) {
+        cu.c++;
+        if (++cu.kp == unit_cpb(cu.u)) {
+            cu.kp = 0;
+            if (++cu.band == unit_nbands(cu.u)) {
+                cu.band = 0;
+                cu.u++;
+            }
+        }
+        if (cu.c == cu.c_end)
+            seek(cu, cu.s + 1);
+    };
+
+    Cursor iss;
+    bool iss_live = seek(iss, 0);
+    int issued = 0;
+    auto issue_one = [&]() {
+        if (lane == 0) {
+            const int slot = issued % D;
+            const uint32_t bar = bars + 8 * slot;
+            const uint32_t cdst = smem_u32(codes_ring + slot * CB);
+            const uint32_t sdst = smem_u32(scales_ring + slot * kScaleBytes);
+            const int row = iss.band * kChunkRows;
+            mbar_arrive_expect_tx(bar, kTx);
+            if constexpr (MOE) {
+                const int e = grp.piece_expert[iss.u];
+                tma_load_3d(cdst, &a.mat0.tm_codes, bar, iss.kp * 128, row, e, pol);
+                tma_load_3d(sdst, &a.mat0.tm_scales, bar, iss.kp * 8, row, e, pol);
+            } else {
+                const MatDesc &m = mats[iss.u];
+#pragma unroll
+                for (int bx = 0; bx < Fmt<FMT>::kBoxes; bx++)
+                    tma_load_2d(cdst + bx * kBoxBytes, &m.tm_codes, bar,
+                                iss.kp * 128 * Fmt<FMT>::kBoxes + bx * 128, row, pol);
+                tma_load_2d(sdst, &m.tm_scales, bar, iss.kp * 8, row, pol);
+            }
+        }
+        issued++;
+        advance(iss);
+        iss_live = iss.s < n_stages;
+    };
+
+    // Fill the ring.
+    while (iss_live && issued < D - 1)
+        issue_one();
 
     // Output of one band: acc holds (row g, col 2t), (row g, col 2t+1),
     // (row g+8, col 2t), (row g+8, col 2t+1).
-    auto store_band = [&](long long gb, const float (&v)[4]) {
-        const int unit = (int)(gb / a.nbands);
-        const int r0 = (int)(gb - (long long)unit * a.nbands) * kChunkRows + g;
+    auto store_band = [&](int u, int band, const float (&v)[4]) {
+        const MatDesc &m = unit_mat(u);
+        const int r0 = band * kChunkRows + g;
 #pragma unroll
         for (int q = 0; q < 4; q++) {
             const int row = r0 + ((q & 2) ? 8 : 0);
             const int col = 2 * t + (q & 1);
-            if (row >= a.N)
+            if (row >= m.N)
                 continue;
             if constexpr (MOE) {
-                if (col < grp.piece_count[unit]) {
-                    const int slot = grp.sorted_slot[grp.piece_first[unit] + col];
-                    a.out[(size_t)slot * a.N + row] = v[q];
+                if (col < grp.piece_count[u]) {
+                    const int slot = grp.sorted_slot[grp.piece_first[u] + col];
+                    m.y[(size_t)slot * m.N + row] = v[q];
                 }
             } else {
-                if (col < a.B)
-                    a.out[(size_t)col * a.N + row] = v[q];
+                if (col < m.B)
+                    m.y[(size_t)col * m.N + row] = v[q];
             }
         }
     };
 
-    auto flush = [&](long long gb, const float (&acc)[4]) {
-        const long long bs = gb * a.cpb, be = bs + a.cpb;
+    auto flush = [&](int s, int u, int band, const float (&acc)[4]) {
+        const StageDesc &st = stg[s];
+        const int cpb = unit_cpb(u);
+        const int bs = unit_chunk_base(u) + band * cpb, be = bs + cpb;
+        const int c0 = w * st.cpw, c1 = min(c0 + st.cpw, st.T);
         if (bs >= c0 && be <= c1) {
-            store_band(gb, acc);
+            store_band(u, band, acc);
             return;
         }
-        const int myslot = (gb == c0 / a.cpb) ? 0 : 1;
-        float4 *mine = reinterpret_cast<float4 *>(a.partials) + ((size_t)w * 2 + myslot) * 32 + lane;
-        __stcg(mine, make_float4(acc[0], acc[1], acc[2], acc[3]));
+        const int myslot = (c0 >= bs) ? 0 : 1;
+        float4 *part = reinterpret_cast<float4 *>(a.partials);
+        __stcg(part + ((size_t)w * 2 + myslot) * 32 + lane, make_float4(acc[0], acc[1], acc[2], acc[3]));
         __threadfence();
         __syncwarp();
-        const long long wf = worker_of(bs, T, W), wl = worker_of(be - 1, T, W);
+        const int wf = bs / st.cpw, wl = (be - 1) / st.cpw;
+        int *ctr = a.counters + unit_band_base(u) + band;
         int old = 0;
         if (lane == 0)
-            old = atomicAdd(&a.counters[gb], 1);
+            old = atomicAdd(ctr, 1);
         old = __shfl_sync(0xffffffffu, old, 0);
-        if (old != (int)(wl - wf))
+        if (old != wl - wf)
             return;
         __threadfence();
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
-        for (long long v = wf; v <= wl; v++) {
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int v = wf; v <= wl; v++) {
             float4 p;
             if (v == w) {
                 p = make_float4(acc[0], acc[1], acc[2], acc[3]);
             } else {
-                const int sl = (gb == range_start(v, T, W) / a.cpb) ? 0 : 1;
-                p = __ldcg(reinterpret_cast<const float4 *>(a.partials) + ((size_t)v * 2 + sl) * 32 + lane);
+                const int sl = (v * st.cpw >= bs) ? 0 : 1;
+                p = __ldcg(part + ((size_t)v * 2 + sl) * 32 + lane);
             }
-            s[0] += p.x;
-            s[1] += p.y;
-            s[2] += p.z;
-            s[3] += p.w;
+            s4[0] += p.x;
+            s4[1] += p.y;
+            s4[2] += p.z;
+            s4[3] += p.w;
         }
-        store_band(gb, s);
+        store_band(u, band, s4);
         if (lane == 0)
-            a.counters[gb] = 0;
+            *ctr = 0;
     };
 
-    // Prologue: fill the ring.
-    const int pre = n < D - 1 ? n : D - 1;
-    for (int i = 0; i < pre; i++)
-        issue(i);
-
-    long long cur = -1;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const __half *xrow = nullptr;
-    if constexpr (!MOE)
-        xrow = (g < a.B) ? a.x + (size_t)g * a.K : nullptr;
-
-    int i = 0;
-    for (; i < n; i++) {
-        if (i + D - 1 < n) {
-            __syncwarp();
-            issue(i + D - 1);
-        }
-        const int slot = i % D;
-        if (!mbar_wait_bounded(bars + 8 * slot, (uint32_t)((i / D) & 1))) {
-            if (lane == 0 && a.status)
-                atomicOr(a.status, kStatusTimeout);
-            break;
-        }
-        const long long c = c0 + i;
-        const long long gb = c / a.cpb;
-        const int kp = (int)(c - gb * a.cpb);
-        if (gb != cur) {
-            if (cur >= 0)
-                flush(cur, acc);
-            cur = gb;
-            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-            if constexpr (MOE) {
-                const int unit = (int)(gb / a.nbands);
-                xrow = nullptr;
-                if (g < grp.piece_count[unit]) {
-                    const int sl = grp.sorted_slot[grp.piece_first[unit] + g];
-                    const int xr = a.x_per_slot ? sl : sl / a.topk;
-                    xrow = a.x + (size_t)xr * a.K;
+    // Grid barrier between stages (plan mode; the launch is cooperative, so
+    // every CTA is resident).  The last warp of a CTA to finish stage s bumps
+    // the grid counter, waits for all CTAs, then releases its CTA's warps
+    // through a shared mbarrier.  Every wait is bounded.
+    bool ok = true;
+    auto stage_arrive_and_wait = [&](int s) {
+        __syncwarp();
+        if (lane == 0) {
+            __threadfence();
+            const int old = atomicAdd(&cta_arrivals, 1);
+            if (old == kWarps * (s + 1) - 1) {
+                atomicAdd(&a.sync[0], 1u);
+                const unsigned target = gridDim.x * (unsigned)(s + 1);
+                const long long t0 = clock64();
+                while (ld_acquire_gpu(&a.sync[0]) < target) {
+                    if (clock64() - t0 > kWaitCycles) {
+                        if (a.status)
+                            atomicOr(a.status, kStatusTimeout);
+                        break;
+                    }
                 }
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&stage_bar))
+                             : "memory");
             }
         }
-        const int left = nb32 - kp * 8;
-        chunk_mma<FMT>(codes_ring + (uint32_t)(slot * CB), scales_ring + (uint32_t)(slot * kScaleBytes),
-                       xrow, kp * kChunkK, left < 8 ? left : 8, g, t, acc);
+        __syncwarp();
+        if (!mbar_wait_bounded(smem_u32(&stage_bar), (uint32_t)(s & 1))) {
+            if (lane == 0 && a.status)
+                atomicOr(a.status, kStatusTimeout);
+            ok = false;
+        }
+        __threadfence();
+    };
+
+    Cursor cur;
+    bool live = seek(cur, 0);
+    int done = 0;                  // chunks consumed (ring index)
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int acc_u = -1, acc_band = -1; // band the accumulators belong to
+    const __half *xrow = nullptr;
+    int nb32 = 0;
+
+    for (int s = 0; s < n_stages; s++) {
+        if (s > 0) {
+            stage_arrive_and_wait(s - 1);
+            if (!ok)
+                break;
+        }
+        while (live && cur.s == s) {
+            if (iss_live && issued < done + D) {
+                __syncwarp();
+                issue_one();
+            }
+            const int slot = done % D;
+            if (!mbar_wait_bounded(bars + 8 * slot, (uint32_t)((done / D) & 1))) {
+                if (lane == 0 && a.status)
+                    atomicOr(a.status, kStatusTimeout);
+                ok = false;
+                break;
+            }
+            if (cur.u != acc_u || cur.band != acc_band) {
+                if (acc_u >= 0)
+                    flush(s, acc_u, acc_band, acc);
+                acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+                if (cur.u != acc_u) {
+                    const MatDesc &m = unit_mat(cur.u);
+                    nb32 = m.K / kBlock;
+                    if constexpr (MOE) {
+                        const int col = min(g, grp.piece_count[cur.u] - 1);
+                        const int sl = grp.sorted_slot[grp.piece_first[cur.u] + col];
+                        xrow = m.x + (size_t)(a.x_per_slot ? sl : sl / a.topk) * m.K;
+                    } else {
+                        xrow = m.x + (size_t)min(g, m.B - 1) * m.K;
+                    }
+                }
+                acc_u = cur.u;
+                acc_band = cur.band;
+            }
+            const int left = nb32 - cur.kp * 8;
+            chunk_mma<FMT>(codes_ring + slot * CB, scales_ring + slot * kScaleBytes, xrow,
+                           cur.kp * kChunkK, left < 8 ? left : 8, g, t, acc);
+            done++;
+            advance(cur);
+            live = cur.s < n_stages;
+        }
+        if (!ok)
+            break;
+        if (acc_u >= 0) {
+            flush(s, acc_u, acc_band, acc);
+            acc_u = acc_band = -1;
+        }
     }
-    if (i == n) {
-        if (cur >= 0)
-            flush(cur, acc);
-        return;
+
+    if (!ok) {
+        // A wait ran out: drain the copies this worker still has in flight
+        // (bounded again) so none lands in shared memory after the CTA exits.
+        for (int j = done; j < issued; j++)
+            (void)mbar_wait_bounded(bars + 8 * (j % D), (uint32_t)((j / D) & 1));
     }
-    // A wait ran out: drain the copies this worker still has in flight
-    // (bounded again) so none lands in shared memory after the CTA exits.
-    const int issued = (n < i + D) ? n : i + D;
-    for (int j = i; j < issued; j++)
-        (void)mbar_wait_bounded(bars + 8 * (j % D), (uint32_t)((j / D) & 1));
+    if constexpr (PLAN) {
+        // The last CTA to leave resets the barrier counters for the next launch.
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            const unsigned old = atomicAdd(&a.sync[1], 1u);
+            if (old == gridDim.x - 1) {
+                a.sync[0] = 0;
+                a.sync[1] = 0;
+                __threadfence();
+            }
+        }
+    }
 }
 
 // y[b][n] = sum_s route_w[b][s] * slot_out[b*topk + s][n], in slot order, over
@@ -354,7 +520,7 @@ __global__ void moe_combine_kernel(const float *slot_out, const int *idx, const 
 // ------------------------------------------------------------------ host ----
 namespace {
 
-template <int FMT, bool MOE>
+template <int FMT, int MODE>
 int32_t prepare_kernel()
 {
     static bool done[64] = {};
@@ -363,7 +529,7 @@ int32_t prepare_kernel()
         return BQ_ERR_CUDA;
     if (dev >= 0 && dev < 64 && done[dev])
         return BQ_OK;
-    if (cudaFuncSetAttribute((const void *)stream_gemv_kernel<FMT, MOE>,
+    if (cudaFuncSetAttribute((const void *)stream_gemv_kernel<FMT, MODE>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem_bytes<FMT>()) != cudaSuccess)
         return BQ_ERR_CUDA;
@@ -372,20 +538,55 @@ int32_t prepare_kernel()
     return BQ_OK;
 }
 
-int grid_ctas(long long T)
+// CTAs of one launch: two per SM (the kernel's occupancy), capped.
+int max_ctas()
 {
     const int sms = device_sm_count();
     if (sms <= 0)
         return -1;
-    long long g = 2LL * sms;
-    if (g > kMaxCtas)
-        g = kMaxCtas;
-    if (T >= 0 && g > T)
-        g = T;
-    return (int)(g < 1 ? 1 : g);
+    return std::min(2 * sms, kMaxCtas);
 }
 
 size_t counters_bytes(long long n) { return align_up((size_t)n * sizeof(int), 256); }
+constexpr size_t kPartialsBytes = (size_t)kMaxWorkers * kPartialBytesPerWorker;
+constexpr size_t kSyncBytes = 256;
+
+bool fill_matdesc(int fmt, const bq_qmat *W, const uint16_t *x, int B, float *y, MatDesc *m)
+{
+    const int N = W->N, K = W->K;
+    const uint64_t cdims[2] = {(uint64_t)(fmt == 4 ? K / 2 : K), (uint64_t)N};
+    const uint64_t cstr[1] = {(uint64_t)(fmt == 4 ? K / 2 : K)};
+    const uint32_t cbox[2] = {128, (uint32_t)kChunkRows};
+    const int ldS = bq_scales_ld(K);
+    const uint64_t sdims[2] = {(uint64_t)(K / 32), (uint64_t)N};
+    const uint64_t sstr[1] = {(uint64_t)ldS * 2};
+    const uint32_t sbox[2] = {8, (uint32_t)kChunkRows};
+    if (!encode_tensor_map(&m->tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, cdims, cstr,
+                           cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tensor_map(&m->tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, W->scales, sdims, sstr,
+                           sbox, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return false;
+    m->x = reinterpret_cast<const __half *>(x);
+    m->y = y;
+    m->N = N;
+    m->K = K;
+    m->B = B;
+    m->cpb = (K + kChunkK - 1) / kChunkK;
+    m->nbands = (N + kChunkRows - 1) / kChunkRows;
+    m->chunk_base = 0;
+    m->band_base = 0;
+    return true;
+}
+
+void fill_stage(StageDesc *st, int mat_begin, int mat_end, long long T, int nbands, int wmax)
+{
+    st->mat_begin = mat_begin;
+    st->mat_end = mat_end;
+    st->T = (int)T;
+    st->cpw = (int)std::max<long long>(1, (T + wmax - 1) / wmax);
+    st->W = (int)((T + st->cpw - 1) / st->cpw);
+    st->nbands = nbands;
+}
 
 template <int FMT>
 int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void *ws,
@@ -402,43 +603,66 @@ int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void
         return BQ_ERR_ALIGN;
     if (ws_bytes < bq_gemv_workspace_bytes(W->N, W->K))
         return BQ_ERR_WORKSPACE;
-    st = prepare_kernel<FMT, false>();
+    const long long nbands = (W->N + kChunkRows - 1) / kChunkRows;
+    if (nbands * ((W->K + kChunkK - 1) / kChunkK) >= (1LL << 31))
+        return BQ_ERR_SHAPE;
+    st = prepare_kernel<FMT, kModeMatrix>();
     if (st != BQ_OK)
         return st;
 
-    GemvArgs a;
+    KernelArgs a;
     memset(&a, 0, sizeof(a));
-    const int N = W->N, K = W->K;
-    const uint64_t cdims[2] = {(uint64_t)(FMT == 4 ? K / 2 : K), (uint64_t)N};
-    const uint64_t cstr[1] = {(uint64_t)(FMT == 4 ? K / 2 : K)};
-    const uint32_t cbox[2] = {128, (uint32_t)kChunkRows};
-    const int ldS = bq_scales_ld(K);
-    const uint64_t sdims[2] = {(uint64_t)(K / 32), (uint64_t)N};
-    const uint64_t sstr[1] = {(uint64_t)ldS * 2};
-    const uint32_t sbox[2] = {8, (uint32_t)kChunkRows};
-    if (!encode_tensor_map(&a.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, cdims, cstr,
-                           cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tensor_map(&a.tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, W->scales, sdims,
-                           sstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!fill_matdesc(FMT, W, x, B, y, &a.mat0))
         return BQ_ERR_CUDA;
-    a.x = reinterpret_cast<const __half *>(x);
-    a.out = y;
-    a.N = N;
-    a.K = K;
-    a.B = B;
-    a.cpb = (K + kChunkK - 1) / kChunkK;
-    a.nbands = (N + kChunkRows - 1) / kChunkRows;
-    const long long T = (long long)a.cpb * a.nbands;
-    const int G = grid_ctas(T);
-    if (G < 0)
+    const long long T = (long long)a.mat0.cpb * a.mat0.nbands;
+    const int cap = max_ctas();
+    if (cap < 0)
         return BQ_ERR_CUDA;
+    const int G = (int)std::min<long long>(cap, T);
     a.wmax = G * kWarps;
+    fill_stage(&a.stage0, 0, 1, T, a.mat0.nbands, a.wmax);
+    a.n_stages = 1;
     a.counters = static_cast<int *>(ws);
-    a.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + counters_bytes(a.nbands));
+    a.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + counters_bytes(a.mat0.nbands));
     a.status = dev_status;
     void *args[] = {&a};
-    cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<FMT, false>, dim3(G), dim3(kThreads),
-                               smem_bytes<FMT>(), static_cast<cudaStream_t>(stream), args);
+    cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<FMT, kModeMatrix>, dim3(G),
+                               dim3(kThreads), smem_bytes<FMT>(), static_cast<cudaStream_t>(stream),
+                               args);
+    return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+template <int FMT>
+int32_t step_run_impl(const bq_step_info *info, const void *plan, void *ws, int32_t *dev_status,
+                      void *stream)
+{
+    int32_t st = prepare_kernel<FMT, kModePlan>();
+    if (st != BQ_OK)
+        return st;
+    KernelArgs a;
+    memset(&a, 0, sizeof(a));
+    const uint8_t *pb = static_cast<const uint8_t *>(plan);
+    a.stages = reinterpret_cast<const StageDesc *>(pb + info->stages_off);
+    a.mats = reinterpret_cast<const MatDesc *>(pb + info->mats_off);
+    a.n_stages = info->n_stages;
+    a.wmax = info->grid * kWarps;
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    a.sync = reinterpret_cast<unsigned *>(wsb);
+    a.counters = reinterpret_cast<int *>(wsb + kSyncBytes);
+    a.partials = reinterpret_cast<float *>(wsb + kSyncBytes + counters_bytes(info->max_stage_bands));
+    a.status = dev_status;
+    void *args[] = {&a};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(info->grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem_bytes<FMT>();
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelExC(&cfg, (const void *)stream_gemv_kernel<FMT, kModePlan>, args);
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
@@ -452,7 +676,7 @@ extern "C" size_t bq_gemv_workspace_bytes(int32_t N, int32_t K)
     if (N < 1 || K < 32 || K % 32 != 0)
         return 0;
     const long long nbands = (N + kChunkRows - 1) / kChunkRows;
-    return counters_bytes(nbands) + (size_t)kMaxWorkers * kPartialBytesPerWorker;
+    return counters_bytes(nbands) + kPartialsBytes;
 }
 
 extern "C" int32_t bq_gemv_q4(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void *ws,
@@ -467,13 +691,136 @@ extern "C" int32_t bq_gemv_q8(const bq_qmat *W, const uint16_t *x, int32_t B, fl
     return gemv_impl<8>(W, x, B, y, ws, ws_bytes, dev_status, stream);
 }
 
+// ------------------------------------------------------------ decode step --
+extern "C" size_t bq_step_plan_bytes(int32_t n_mats)
+{
+    if (n_mats < 1)
+        return 0;
+    return align_up(sizeof(PlanHeader), 64) + align_up((size_t)n_mats * sizeof(StageDesc), 64) +
+           (size_t)n_mats * sizeof(MatDesc);
+}
+
+extern "C" int32_t bq_step_plan(int32_t fmt, const bq_step_mat *mats, int32_t n_mats, void *plan,
+                                size_t plan_bytes, bq_step_info *info)
+{
+    if (!mats || !plan || !info)
+        return BQ_ERR_NULL;
+    if ((fmt != 4 && fmt != 8) || n_mats < 1)
+        return BQ_ERR_SHAPE;
+    if (plan_bytes < bq_step_plan_bytes(n_mats))
+        return BQ_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(plan) & 63u) != 0)
+        return BQ_ERR_ALIGN;
+    for (int i = 0; i < n_mats; i++) {
+        const int32_t st = check_qmat(&mats[i].W);
+        if (st != BQ_OK)
+            return st;
+        if (!mats[i].x || !mats[i].y)
+            return BQ_ERR_NULL;
+        if (mats[i].B < 1 || mats[i].B > 8)
+            return BQ_ERR_BATCH;
+        if (mats[i].stage < 0)
+            return BQ_ERR_SHAPE;
+        if (!aligned16(mats[i].x) || !aligned16(mats[i].y))
+            return BQ_ERR_ALIGN;
+    }
+    int32_t st = fmt == 4 ? prepare_kernel<4, kModePlan>() : prepare_kernel<8, kModePlan>();
+    if (st != BQ_OK)
+        return st;
+    // Co-residency: every CTA of the grid must fit on the device at once.
+    int occ = 0;
+    const void *kfn = fmt == 4 ? (const void *)stream_gemv_kernel<4, kModePlan>
+                               : (const void *)stream_gemv_kernel<8, kModePlan>;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &occ, kfn, kThreads, fmt == 4 ? smem_bytes<4>() : smem_bytes<8>()) != cudaSuccess ||
+        occ < 1)
+        return BQ_ERR_CUDA;
+    const int sms = device_sm_count();
+    if (sms <= 0)
+        return BQ_ERR_CUDA;
+    const int G = std::min(std::min(occ, 2) * sms, kMaxCtas);
+    const int wmax = G * kWarps;
+
+    std::vector<int> order(n_mats);
+    for (int i = 0; i < n_mats; i++)
+        order[i] = i;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int p, int q) { return mats[p].stage < mats[q].stage; });
+    std::vector<MatDesc> md(n_mats);
+    std::vector<StageDesc> sd;
+    long long max_bands = 1;
+    for (int i = 0; i < n_mats;) {
+        const int s = mats[order[i]].stage;
+        int j = i;
+        long long T = 0, bands = 0;
+        while (j < n_mats && mats[order[j]].stage == s) {
+            const bq_step_mat &m = mats[order[j]];
+            if (!fill_matdesc(fmt, &m.W, m.x, m.B, m.y, &md[j]))
+                return BQ_ERR_CUDA;
+            md[j].chunk_base = (int)T;
+            md[j].band_base = (int)bands;
+            T += (long long)md[j].cpb * md[j].nbands;
+            bands += md[j].nbands;
+            if (T >= (1LL << 31))
+                return BQ_ERR_SHAPE;
+            j++;
+        }
+        StageDesc sdesc;
+        fill_stage(&sdesc, i, j, T, (int)bands, wmax);
+        sd.push_back(sdesc);
+        max_bands = std::max(max_bands, bands);
+        i = j;
+    }
+    PlanHeader h;
+    memset(&h, 0, sizeof(h));
+    h.magic = kPlanMagic;
+    h.fmt = fmt;
+    h.n_mats = n_mats;
+    h.n_stages = (int)sd.size();
+    h.grid = G;
+    h.max_stage_bands = (int)max_bands;
+    h.stages_off = align_up(sizeof(PlanHeader), 64);
+    h.mats_off = h.stages_off + align_up((size_t)n_mats * sizeof(StageDesc), 64);
+    std::vector<uint8_t> host(h.mats_off + (size_t)n_mats * sizeof(MatDesc), 0);
+    memcpy(host.data(), &h, sizeof(h));
+    memcpy(host.data() + h.stages_off, sd.data(), sd.size() * sizeof(StageDesc));
+    memcpy(host.data() + h.mats_off, md.data(), (size_t)n_mats * sizeof(MatDesc));
+    if (cudaMemcpy(plan, host.data(), host.size(), cudaMemcpyHostToDevice) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    info->fmt = fmt;
+    info->n_mats = n_mats;
+    info->n_stages = h.n_stages;
+    info->grid = G;
+    info->max_stage_bands = (int)max_bands;
+    info->stages_off = h.stages_off;
+    info->mats_off = h.mats_off;
+    info->ws_bytes = kSyncBytes + counters_bytes(max_bands) + kPartialsBytes;
+    return BQ_OK;
+}
+
+extern "C" int32_t bq_step_run(const bq_step_info *info, const void *plan, void *ws,
+                               size_t ws_bytes, int32_t *dev_status, void *stream)
+{
+    if (!info || !plan || !ws)
+        return BQ_ERR_NULL;
+    if ((info->fmt != 4 && info->fmt != 8) || info->n_stages < 1 || info->grid < 1)
+        return BQ_ERR_SHAPE;
+    if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(plan) & 63u) != 0)
+        return BQ_ERR_ALIGN;
+    if (ws_bytes < info->ws_bytes)
+        return BQ_ERR_WORKSPACE;
+    return info->fmt == 4 ? step_run_impl<4>(info, plan, ws, dev_status, stream)
+                          : step_run_impl<8>(info, plan, ws, dev_status, stream);
+}
+
+// ------------------------------------------------------- routed experts --
 extern "C" size_t bq_moe_workspace_bytes(int32_t N, int32_t K, int32_t B, int32_t topk, int32_t E)
 {
     if (N < 1 || K < 32 || K % 32 != 0 || B < 1 || B > 8 || topk < 1 || B * topk > kMaxSlots ||
         E < 1 || E > 65535)
         return 0;
     const long long nbands = (N + kChunkRows - 1) / kChunkRows;
-    return counters_bytes(nbands * B * topk) + (size_t)kMaxWorkers * kPartialBytesPerWorker +
+    return counters_bytes(nbands * B * topk) + kPartialsBytes +
            align_up((size_t)B * topk * N * sizeof(float), 256);
 }
 
@@ -499,11 +846,15 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
         return BQ_ERR_ALIGN;
     if (ws_bytes < bq_moe_workspace_bytes(N, K, B, topk, E))
         return BQ_ERR_WORKSPACE;
-    st = prepare_kernel<4, true>();
+    const long long nbands = (N + kChunkRows - 1) / kChunkRows;
+    const long long cpb = (K + kChunkK - 1) / kChunkK;
+    if ((long long)B * topk * nbands * cpb >= (1LL << 31))
+        return BQ_ERR_SHAPE;
+    st = prepare_kernel<4, kModeMoE>();
     if (st != BQ_OK)
         return st;
 
-    GemvArgs a;
+    KernelArgs a;
     memset(&a, 0, sizeof(a));
     const uint64_t cdims[3] = {(uint64_t)(K / 2), (uint64_t)N, (uint64_t)E};
     const uint64_t cstr[2] = {(uint64_t)(K / 2), (uint64_t)codes_stride};
@@ -511,26 +862,25 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
     const uint64_t sdims[3] = {(uint64_t)(K / 32), (uint64_t)N, (uint64_t)E};
     const uint64_t sstr[2] = {(uint64_t)ldS * 2, (uint64_t)scales_stride * 2};
     const uint32_t sbox[3] = {8, (uint32_t)kChunkRows, 1};
-    if (!encode_tensor_map(&a.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, Wstack->codes, cdims,
-                           cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tensor_map(&a.tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, Wstack->scales, sdims,
-                           sstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!encode_tensor_map(&a.mat0.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, Wstack->codes,
+                           cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tensor_map(&a.mat0.tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, Wstack->scales,
+                           sdims, sstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE))
         return BQ_ERR_CUDA;
-    const long long nbands = (N + kChunkRows - 1) / kChunkRows;
     uint8_t *wsb = static_cast<uint8_t *>(ws);
-    float *slot_buf = reinterpret_cast<float *>(wsb + counters_bytes(nbands * B * topk) +
-                                                (size_t)kMaxWorkers * kPartialBytesPerWorker);
-    a.x = reinterpret_cast<const __half *>(x);
-    a.out = route_w ? slot_buf : y;
-    a.N = N;
-    a.K = K;
-    a.B = B;
-    a.cpb = (K + kChunkK - 1) / kChunkK;
-    a.nbands = (int)nbands;
-    const int G = grid_ctas(-1);
+    float *slot_buf = reinterpret_cast<float *>(wsb + counters_bytes(nbands * B * topk) + kPartialsBytes);
+    a.mat0.x = reinterpret_cast<const __half *>(x);
+    a.mat0.y = route_w ? slot_buf : y;
+    a.mat0.N = N;
+    a.mat0.K = K;
+    a.mat0.B = B;
+    a.mat0.cpb = (int)cpb;
+    a.mat0.nbands = (int)nbands;
+    const int G = max_ctas();
     if (G < 0)
         return BQ_ERR_CUDA;
     a.wmax = G * kWarps;
+    a.n_stages = 1;
     a.counters = reinterpret_cast<int *>(wsb);
     a.partials = reinterpret_cast<float *>(wsb + counters_bytes(nbands * B * topk));
     a.status = dev_status;
@@ -540,8 +890,8 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
     a.idx = expert_idx;
     void *args[] = {&a};
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<4, true>, dim3(G), dim3(kThreads),
-                               smem_bytes<4>(), s, args);
+    cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<4, kModeMoE>, dim3(G),
+                               dim3(kThreads), smem_bytes<4>(), s, args);
     if (e != cudaSuccess)
         return BQ_ERR_CUDA;
     if (route_w) {
@@ -549,8 +899,7 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
         int Bv = B, tk = topk, Nv = N, Ev = E;
         void *cargs[] = {(void *)&sb, (void *)&expert_idx, (void *)&route_w, &Bv, &tk, &Nv, &Ev, &y};
         int cg = (B * N + 255) / 256;
-        if (cg > 4 * device_sm_count())
-            cg = 4 * device_sm_count();
+        cg = std::max(1, std::min(cg, 4 * std::max(1, device_sm_count())));
         e = launch_pdl((const void *)moe_combine_kernel, dim3(cg), dim3(256), 0, s, cargs);
         if (e != cudaSuccess)
             return BQ_ERR_CUDA;

@@ -187,3 +187,30 @@ def test_product_path_has_no_oracle_or_fallback():
                     src = f.read()
                 assert "import oracle" not in src and "from oracle" not in src, fn
                 assert "oracle.c" not in src and "liboracle" not in src, fn
+
+
+def test_step_argument_validation_before_launch():
+    L = bq.lib()
+    assert L.bq_step_plan_bytes(0) == 0 and L.bq_step_plan_bytes(3) > 3 * 320
+    info = bq.bq_step_info()
+    arr = (bq.bq_step_mat * 2)()
+    for i in range(2):
+        arr[i] = bq.bq_step_mat(bq.bq_qmat(FAKE, FAKE, 64, 256), FAKE, FAKE, 1, i)
+    nb = L.bq_step_plan_bytes(2)
+    assert L.bq_step_plan(4, None, 2, FAKE, nb, ctypes.byref(info)) == bq.BQ_ERR_NULL
+    assert L.bq_step_plan(5, arr, 2, FAKE, nb, ctypes.byref(info)) == bq.BQ_ERR_SHAPE
+    assert L.bq_step_plan(4, arr, 0, FAKE, nb, ctypes.byref(info)) == bq.BQ_ERR_SHAPE
+    assert L.bq_step_plan(4, arr, 2, FAKE, nb - 1, ctypes.byref(info)) == bq.BQ_ERR_WORKSPACE
+    assert L.bq_step_plan(4, arr, 2, FAKE + 16, nb, ctypes.byref(info)) == bq.BQ_ERR_ALIGN
+    arr[1].B = 9
+    assert L.bq_step_plan(4, arr, 2, FAKE, nb, ctypes.byref(info)) == bq.BQ_ERR_BATCH
+    arr[1].B = 1
+    arr[1].stage = -1
+    assert L.bq_step_plan(4, arr, 2, FAKE, nb, ctypes.byref(info)) == bq.BQ_ERR_SHAPE
+    arr[1].stage = 1
+    arr[0].W.K = 40
+    assert L.bq_step_plan(4, arr, 2, FAKE, nb, ctypes.byref(info)) == bq.BQ_ERR_SHAPE
+    info = bq.bq_step_info(4, 2, 2, 296, 10, 0, 64, 128, 1 << 20)
+    assert L.bq_step_run(None, FAKE, FAKE, 1 << 20, None, None) == bq.BQ_ERR_NULL
+    assert L.bq_step_run(ctypes.byref(info), FAKE, FAKE, 1024, None, None) == bq.BQ_ERR_WORKSPACE
+    assert L.bq_step_run(ctypes.byref(info), FAKE + 16, FAKE, 1 << 20, None, None) == bq.BQ_ERR_ALIGN

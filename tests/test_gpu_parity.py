@@ -201,3 +201,90 @@ def test_moe_single_expert_matches_dense():
     assert st == 0
     yd = gpu_gemv(4, codes[1], scales[1], x)
     np.testing.assert_array_equal(y[:, 0], yd)
+
+
+# ------------------------------------------------------------ decode step ----
+def _step_entries(fmt, specs, seed):
+    """specs: list of (N, K, B, stage) -> (entries, numpy planes/x for the oracle)."""
+    import torch
+    entries, host = [], []
+    for i, (N, K, B, stage) in enumerate(specs):
+        w = synth.weights_f32(synth.key(seed, 82, i, 0, synth.KIND_W), N, K)
+        codes, scales = quantize(fmt, w)
+        x = synth.activations_f16_bits(synth.key(seed, 82, i, 0, synth.KIND_X), B, K)
+        c, s, xt = dev(codes.view(np.uint8)), dev(scales), dev(x)
+        y = torch.full((B, N), float("nan"), dtype=torch.float32, device=DEV)
+        entries.append((bq.qmat(c, s, N, K), xt, y, stage))
+        host.append((codes, scales, x))
+    return entries, host
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+def test_step_plan_parity_and_repeat(fmt):
+    import torch
+    specs = [(3072, 2048, 1, 0), (512, 2048, 1, 0), (2048, 2048, 1, 1), (16384, 2048, 1, 2),
+             (2048, 8192, 1, 3), (77, 288, 3, 3), (1000, 96, 8, 5), (16, 32, 2, 4),
+             (4096, 4096, 8, 7), (300, 5120, 2, 6)]
+    order = [5, 0, 9, 2, 7, 1, 4, 3, 8, 6]           # plan input order is irrelevant
+    entries, host = _step_entries(fmt, [specs[i] for i in order], 7 + fmt)
+    plan = bq.StepPlan(fmt, entries, DEV)
+    assert plan.info.n_stages == 8
+    st = new_status()
+    plan.run(st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    first = [e[2].cpu().numpy() for e in entries]
+    for (W, x, y, stage), (codes, scales, xb), yg in zip(entries, host, first):
+        y_ref, absy = oracle_gemv(fmt, codes, scales, xb)
+        check_tol(yg, y_ref, absy)
+    for _ in range(3):
+        for e in entries:
+            e[2].fill_(float("nan"))
+        plan.run(st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for e, y0 in zip(entries, first):
+        assert np.array_equal(e[2].cpu().numpy(), y0)
+    ws = plan.ws
+    assert int(ws.view(torch.int32).abs().sum().item()) == 0     # barrier + band counters reset
+
+
+def test_step_barrier_orders_dependent_stages():
+    """Stage 1 reads stage 0's output buffer (its fp32 bits as fp16 x).  Stage
+    0 returns small integers (one-hot x, unit scales), whose fp32 bits are
+    known, so stage 1's exact input is known; without the grid barrier stage 1
+    would read the NaN fill."""
+    import torch
+    N0, K0 = 256, 64
+    r = np.random.default_rng(3)
+    q0 = r.integers(0, 16, size=(N0, K0))
+    codes0 = np.zeros((N0, K0 // 2), dtype=np.uint8)
+    for j in range(K0 // 32):
+        for i in range(16):
+            codes0[:, 16 * j + i] = q0[:, 32 * j + i] | (q0[:, 32 * j + i + 16] << 4)
+    scales0 = np.zeros((N0, 8), dtype=np.uint16)
+    scales0[:, :2] = 0x3C00
+    x0 = np.zeros((1, K0), dtype=np.float16)
+    x0[0, 0] = 1.0
+    y0_expect = (q0[:, 0] - 8).astype(np.float32)
+    x1_expect = y0_expect.view(np.uint16).reshape(1, 2 * N0)    # little-endian halves
+    N1, K1 = 3000, 2 * N0
+    w1 = synth.weights_f32(synth.key(0, 83, 1, 0, synth.KIND_W), N1, K1)
+    codes1, scales1 = oracle.quantize_q4(w1)
+    c0, s0, xt0 = dev(codes0), dev(scales0), dev(x0.view(np.uint16))
+    y0 = torch.full((1, N0), float("nan"), dtype=torch.float32, device=DEV)
+    c1, s1 = dev(codes1), dev(scales1)
+    y1 = torch.full((1, N1), float("nan"), dtype=torch.float32, device=DEV)
+    x1_alias = y0.view(torch.int16)                             # [1, 2*N0] fp16 bits
+    plan = bq.StepPlan(4, [(bq.qmat(c0, s0, N0, K0), xt0, y0, 0),
+                           (bq.qmat(c1, s1, N1, K1), x1_alias, y1, 1)], DEV)
+    st = new_status()
+    for _ in range(3):
+        y0.fill_(float("nan"))
+        y1.fill_(float("nan"))
+        plan.run(st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        assert np.array_equal(y0.cpu().numpy()[0], y0_expect)
+        y_ref, absy = oracle.gemv_q4(codes1, scales1, x1_expect)
+        check_tol(y1.cpu().numpy(), y_ref, absy)
