@@ -3,15 +3,16 @@
 // programmatic dependent launch), in-register Q4/Q8 dequantisation and the
 // per-chunk dot product.
 //
-// Work unit ("chunk"): 16 weight rows x 256 weights along K (8 blocks of 32).
-// A chunk's codes arrive in shared memory through one (Q4) or two (Q8) 2-D TMA
-// boxes of 16 rows x 128 bytes with the 128-byte swizzle, its scales through
-// one 16 rows x 8 fp16 box.  A warp reads them with 32-bit shared loads that
+// Work unit ("chunk"): kRows weight rows (32 for Q4, 16 for Q8) x 256 weights
+// along K (8 blocks of 32).  A chunk's codes arrive in shared memory through
+// one (Q4: 32 rows x 128 bytes) or two (Q8: 16 rows x 128 bytes each) 2-D TMA
+// boxes with the 128-byte swizzle, its scales through one kRows x 8 fp16 box.  A warp reads them with 32-bit shared loads that
 // the swizzle makes bank-conflict free, dequantises each 4-byte group into
 // fp16 pairs in registers (the codes are small integers, exact in fp16), and
-// forms the block's partial dot products with two m16n8k16 mma.sync (fp16 in,
-// fp32 accumulate): M = the 16 weight rows, N = the batch (B <= 8; absent
-// columns are zero), K = 16 elements of one block.  Each block's partial sum
+// forms the block's partial dot products with m16n8k16 mma.sync (fp16 in,
+// fp32 accumulate): M = 16 weight rows (a Q4 chunk is two such m-tiles that
+// share every x fragment), N = the batch (B <= 8), K = 16 elements of one
+// block.  Each block's partial sum
 // is scaled by its fp32-converted scale once (y += d * sum(q * x)), so the
 // only roundings are fp32 ones.
 #pragma once
@@ -19,41 +20,45 @@
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
+#include <string.h>
 
 namespace bq {
 
 constexpr int kBlock = 32;          // weights per quantisation block
 constexpr int kChunkK = 256;        // weights along K per chunk
-constexpr int kChunkRows = 16;      // weight rows per chunk (mma M)
 constexpr int kWarps = 8;           // worker warps per CTA
 constexpr int kThreads = kWarps * 32;
-constexpr int kScaleBytes = kChunkRows * 16;   // 16 rows x 8 fp16 scales
-constexpr int kBoxBytes = kChunkRows * 128;    // one 16 x 128-byte code box
 
 // Status bits OR-ed into the caller's device status word (1 << bq_status).
 constexpr int kStatusExpertIndex = 1 << 5;
 constexpr int kStatusTimeout = 1 << 7;
 constexpr int kStatusRange = 1 << 9;
 
-// A bounded mbarrier wait gives up after this many SM clock cycles (~2 s).
+// A bounded wait gives up after this many SM clock cycles (~2 s).
 constexpr long long kWaitCycles = 4000000000LL;
 
 template <int FMT> struct Fmt;
 template <> struct Fmt<4> {
-    static constexpr int kCodeBytes = kBoxBytes;       // 16 rows x 128 B
-    static constexpr int kBoxes = 1;
-    static constexpr int kStages = 4;
+    static constexpr int kMT = 2;                       // m-tiles of 16 rows per chunk
+    static constexpr int kRows = 16 * kMT;              // rows per chunk / band
+    static constexpr int kBoxes = 1;                    // 128-byte-wide code boxes
+    static constexpr int kCodeBytes = kRows * 128;      // 4 KB
+    static constexpr int kScaleBytes = kRows * 16;      // kRows x 8 fp16
+    static constexpr int kStages = 3;
 };
 template <> struct Fmt<8> {
-    static constexpr int kCodeBytes = 2 * kBoxBytes;   // 16 rows x 256 B
+    static constexpr int kMT = 1;
+    static constexpr int kRows = 16;
     static constexpr int kBoxes = 2;
+    static constexpr int kCodeBytes = 2 * kRows * 128;  // 4 KB
+    static constexpr int kScaleBytes = kRows * 16;
     static constexpr int kStages = 3;
 };
 
 template <int FMT>
 constexpr int smem_bytes()
 {
-    return kWarps * Fmt<FMT>::kStages * (Fmt<FMT>::kCodeBytes + kScaleBytes) +
+    return kWarps * Fmt<FMT>::kStages * (Fmt<FMT>::kCodeBytes + Fmt<FMT>::kScaleBytes) +
            kWarps * Fmt<FMT>::kStages * 8 + 1024;
 }
 
@@ -245,37 +250,42 @@ __device__ __forceinline__ Q8Pairs dequant_q8(uint32_t w)
 
 __device__ __forceinline__ float half_lo(uint32_t v)
 {
-    return __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xffffu)));
+    __half2 h;
+    memcpy(&h, &v, 4);
+    return __low2float(h);
 }
 __device__ __forceinline__ float half_hi(uint32_t v)
 {
-    return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
+    __half2 h;
+    memcpy(&h, &v, 4);
+    return __high2float(h);
 }
 __device__ __forceinline__ uint32_t pick_u32(const uint4 &v, int i)
 {
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
 
-// One block (32 weights along K) of the chunk for the lane's rows g and g+8.
-// `xa` holds x at k..k+3 and `xb` at k+16..k+19 (k = block start + 4t) for
-// batch column g (zero if the column is absent).
+// One block (32 weights along K) of the chunk for m-tile mt (rows
+// 16*mt + g and 16*mt + g + 8).  `xa` holds x at k..k+3 and `xb` at
+// k+16..k+19 (k = block start + 4t) for batch column g; `sw` is this lane's
+// swizzled offset of block jb in a 128-byte code row.
 template <int FMT>
-__device__ __forceinline__ void block_mma(const uint8_t *codes_s, int jb, int g, int t, uint2 xa,
+__device__ __forceinline__ void block_mma(const uint8_t *lane_codes, int jb, int sw, uint2 xa,
                                           uint2 xb, float dg, float dg8, float (&acc)[4])
 {
     const float zero[4] = {0.f, 0.f, 0.f, 0.f};
     float c[4];
     if constexpr (FMT == 4) {
-        const int off = g * 128 + (((jb ^ g) & 7) << 4) + 4 * t;
-        const Q4Pairs r0 = dequant_q4(lds32(codes_s + off));          // row g
-        const Q4Pairs r8 = dequant_q4(lds32(codes_s + off + 1024));   // row g + 8
+        const uint8_t *p = lane_codes + sw;
+        const Q4Pairs r0 = dequant_q4(lds32(p));          // row g
+        const Q4Pairs r8 = dequant_q4(lds32(p + 1024));   // row g + 8
         mma16816(c, r0.lo01, r8.lo01, r0.lo23, r8.lo23, xa.x, xa.y, zero);
         mma16816(c, r0.hi01, r8.hi01, r0.hi23, r8.hi23, xb.x, xb.y, c);
     } else {
-        const int box = jb >> 2, jj = jb & 3;
-        const uint8_t *base = codes_s + box * kBoxBytes + g * 128 + 4 * t;
-        const int oa = (((2 * jj) ^ g) & 7) << 4;
-        const int ob = (((2 * jj + 1) ^ g) & 7) << 4;
+        // sw holds the offsets of the block's two 16-byte halves (granules
+        // 2jj and 2jj+1 of box jb/4) packed as two 16-bit values.
+        const uint8_t *base = lane_codes + (jb >> 2) * 2048;
+        const int oa = sw & 0xffff, ob = sw >> 16;
         const Q8Pairs a0 = dequant_q8(lds32(base + oa));
         const Q8Pairs a8 = dequant_q8(lds32(base + oa + 1024));
         const Q8Pairs b0 = dequant_q8(lds32(base + ob));
@@ -289,17 +299,40 @@ __device__ __forceinline__ void block_mma(const uint8_t *codes_s, int jb, int g,
     acc[3] = fmaf(dg8, c[3], acc[3]);
 }
 
-// A whole chunk: blocks kb0 .. kb0+7 (k0 = 32*kb0 along K), nblk of them valid.
-// xrow points at x[column g][0].  A lane whose column is absent (g >= B) reads
-// a valid row instead; its mma column is garbage and is never stored, which
-// keeps every load unconditional.
+// Per-lane swizzled offsets of the 8 blocks of a chunk row (constant for a
+// lane): TMA's 128-byte swizzle XORs the 16-byte granule index with the row
+// index mod 8, and row mod 8 == g for every row this lane reads.
+template <int FMT>
+__device__ __forceinline__ void lane_swizzle(int g, int (&sw)[8])
+{
+#pragma unroll
+    for (int jb = 0; jb < 8; jb++) {
+        if constexpr (FMT == 4) {
+            sw[jb] = ((jb ^ g) & 7) << 4;
+        } else {
+            const int jj = jb & 3;
+            sw[jb] = ((((2 * jj) ^ g) & 7) << 4) | (((((2 * jj + 1) ^ g) & 7) << 4) << 16);
+        }
+    }
+}
+
+// A whole chunk: 8 blocks (nblk of them valid) starting at k0 along K, for
+// the chunk's kMT m-tiles.  xrow points at x[column g][0]; a lane whose column
+// is absent (g >= B) reads a valid row instead -- its mma column is garbage
+// and is never stored, which keeps every load unconditional.
 template <int FMT>
 __device__ __forceinline__ void chunk_mma(const uint8_t *codes_s, const uint8_t *scales_s,
                                           const __half *xrow, int k0, int nblk, int g, int t,
-                                          float (&acc)[4])
+                                          const int (&sw)[8], float (&acc)[Fmt<FMT>::kMT][4])
 {
-    const uint4 sg = lds128(scales_s + g * 16);
-    const uint4 sg8 = lds128(scales_s + (g + 8) * 16);
+    constexpr int MT = Fmt<FMT>::kMT;
+    uint4 sc[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; mt++) {
+        sc[mt][0] = lds128(scales_s + (16 * mt + g) * 16);
+        sc[mt][1] = lds128(scales_s + (16 * mt + g + 8) * 16);
+    }
+    const uint8_t *lane_codes = codes_s + g * 128 + 4 * t;
     const __half *xp = xrow + k0 + 4 * t;
     if (nblk == 8) {
         uint2 xa[8], xb[8];
@@ -310,10 +343,13 @@ __device__ __forceinline__ void chunk_mma(const uint8_t *codes_s, const uint8_t 
         }
 #pragma unroll
         for (int jb = 0; jb < 8; jb++) {
-            const uint32_t wg = pick_u32(sg, jb >> 1), wg8 = pick_u32(sg8, jb >> 1);
-            const float dg = (jb & 1) ? half_hi(wg) : half_lo(wg);
-            const float dg8 = (jb & 1) ? half_hi(wg8) : half_lo(wg8);
-            block_mma<FMT>(codes_s, jb, g, t, xa[jb], xb[jb], dg, dg8, acc);
+#pragma unroll
+            for (int mt = 0; mt < MT; mt++) {
+                const uint32_t wg = pick_u32(sc[mt][0], jb >> 1), wg8 = pick_u32(sc[mt][1], jb >> 1);
+                const float dg = (jb & 1) ? half_hi(wg) : half_lo(wg);
+                const float dg8 = (jb & 1) ? half_hi(wg8) : half_lo(wg8);
+                block_mma<FMT>(lane_codes + mt * 2048, jb, sw[jb], xa[jb], xb[jb], dg, dg8, acc[mt]);
+            }
         }
     } else {
 #pragma unroll
@@ -321,10 +357,13 @@ __device__ __forceinline__ void chunk_mma(const uint8_t *codes_s, const uint8_t 
             if (jb < nblk) {
                 const uint2 xa = ldg64(xp + 32 * jb);
                 const uint2 xb = ldg64(xp + 32 * jb + 16);
-                const uint32_t wg = pick_u32(sg, jb >> 1), wg8 = pick_u32(sg8, jb >> 1);
-                const float dg = (jb & 1) ? half_hi(wg) : half_lo(wg);
-                const float dg8 = (jb & 1) ? half_hi(wg8) : half_lo(wg8);
-                block_mma<FMT>(codes_s, jb, g, t, xa, xb, dg, dg8, acc);
+#pragma unroll
+                for (int mt = 0; mt < MT; mt++) {
+                    const uint32_t wg = pick_u32(sc[mt][0], jb >> 1), wg8 = pick_u32(sc[mt][1], jb >> 1);
+                    const float dg = (jb & 1) ? half_hi(wg) : half_lo(wg);
+                    const float dg8 = (jb & 1) ? half_hi(wg8) : half_lo(wg8);
+                    block_mma<FMT>(lane_codes + mt * 2048, jb, sw[jb], xa, xb, dg, dg8, acc[mt]);
+                }
             }
         }
     }

@@ -8,9 +8,9 @@
 // paragraph says the same of its decode path).  The design goal is one thing:
 // keep HBM busy with the packed weight bytes and read each of them once.
 //
-// Work decomposition (stream-K over chunks).  A matrix is cut into bands of 16
-// rows and a band into chunks of 256 weights along K; chunks are numbered
-// band-major.  Every warp of the grid is an independent worker that owns a
+// Work decomposition (stream-K over chunks).  A matrix is cut into bands of
+// kRows rows (32 for Q4, 16 for Q8) and a band into chunks of 256 weights
+// along K; chunks are numbered band-major.  Every warp of the grid is an independent worker that owns a
 // ring of shared-memory slots with its own mbarriers; its lane 0 keeps
 // `stages - 1` chunks of TMA loads in flight ahead of the chunk the warp is
 // computing.  Worker w takes chunks [w*cpw, (w+1)*cpw) of a stage, where cpw =
@@ -19,7 +19,7 @@
 //
 // A band wholly inside one worker's range is written straight to y.  A band
 // cut by range boundaries is summed deterministically: each worker that
-// touched it stores its fp32 partial (16 rows x 8 columns) in the workspace
+// touched it stores its fp32 partial (kRows rows x 8 columns) in the workspace
 // and bumps the band's arrival counter; the last to arrive adds the partials
 // in worker order, writes y and resets the counter.  No worker waits for
 // another.
@@ -90,9 +90,10 @@ struct KernelArgs {
     int n_stages;
     int wmax;                        // gridDim.x * kWarps
     int *counters;                   // per band of a stage; zero on entry and exit
-    float *partials;                 // [wmax][2][128]
+    float *partials;                 // [wmax][2][kMT][32 lanes] float4
     int *status;                     // device status word or null
-    unsigned *sync;                  // plan mode: [0] barrier arrivals, [1] exits
+    unsigned *sync;                  // plan mode: [0] arrivals, [32] stage flag, [64] exits
+                                     // (separate 128-byte lines)
     // routed experts
     int E, topk, x_per_slot;
     const int *idx;
@@ -170,7 +171,10 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
 {
     constexpr int D = Fmt<FMT>::kStages;
     constexpr int CB = Fmt<FMT>::kCodeBytes;
-    constexpr uint32_t kTx = CB + kScaleBytes;
+    constexpr int SB = Fmt<FMT>::kScaleBytes;
+    constexpr int MT = Fmt<FMT>::kMT;
+    constexpr int ROWS = Fmt<FMT>::kRows;
+    constexpr uint32_t kTx = CB + SB;
     constexpr bool MOE = MODE == kModeMoE;
     constexpr bool PLAN = MODE == kModePlan;
 
@@ -183,8 +187,8 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     uint8_t *codes_ring = sbase + warp * D * CB;
-    uint8_t *scales_ring = sbase + kWarps * D * CB + warp * D * kScaleBytes;
-    const uint32_t bars = smem_u32(sbase + kWarps * D * (CB + kScaleBytes) + warp * D * 8);
+    uint8_t *scales_ring = sbase + kWarps * D * CB + warp * D * SB;
+    const uint32_t bars = smem_u32(sbase + kWarps * D * (CB + SB) + warp * D * 8);
 
     const MatDesc *mats = PLAN ? a.mats : &a.mat0;
     const StageDesc *stg = PLAN ? a.stages : &a.stage0;
@@ -293,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
             const int slot = issued % D;
             const uint32_t bar = bars + 8 * slot;
             const uint32_t cdst = smem_u32(codes_ring + slot * CB);
-            const uint32_t sdst = smem_u32(scales_ring + slot * kScaleBytes);
-            const int row = iss.band * kChunkRows;
+            const uint32_t sdst = smem_u32(scales_ring + slot * SB);
+            const int row = iss.band * ROWS;
             mbar_arrive_expect_tx(bar, kTx);
             if constexpr (MOE) {
                 const int e = grp.piece_expert[iss.u];
@@ -304,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
                 const MatDesc &m = mats[iss.u];
 #pragma unroll
                 for (int bx = 0; bx < Fmt<FMT>::kBoxes; bx++)
-                    tma_load_2d(cdst + bx * kBoxBytes, &m.tm_codes, bar,
+                    tma_load_2d(cdst + bx * (ROWS * 128), &m.tm_codes, bar,
                                 iss.kp * 128 * Fmt<FMT>::kBoxes + bx * 128, row, pol);
                 tma_load_2d(sdst, &m.tm_scales, bar, iss.kp * 8, row, pol);
             }
@@ -318,30 +322,36 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
     while (iss_live && issued < D - 1)
         issue_one();
 
-    // Output of one band: acc holds (row g, col 2t), (row g, col 2t+1),
-    // (row g+8, col 2t), (row g+8, col 2t+1).
-    auto store_band = [&](int u, int band, const float (&v)[4]) {
+    // Output of one band: acc[mt] holds (row 16mt+g, col 2t), (row 16mt+g,
+    // col 2t+1), (row 16mt+g+8, col 2t), (row 16mt+g+8, col 2t+1).
+    auto store_band = [&](int u, int band, const float (&v)[MT][4]) {
         const MatDesc &m = unit_mat(u);
-        const int r0 = band * kChunkRows + g;
 #pragma unroll
-        for (int q = 0; q < 4; q++) {
-            const int row = r0 + ((q & 2) ? 8 : 0);
-            const int col = 2 * t + (q & 1);
-            if (row >= m.N)
-                continue;
-            if constexpr (MOE) {
-                if (col < grp.piece_count[u]) {
-                    const int slot = grp.sorted_slot[grp.piece_first[u] + col];
-                    m.y[(size_t)slot * m.N + row] = v[q];
+        for (int mt = 0; mt < MT; mt++) {
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const int row = band * ROWS + 16 * mt + g + ((q & 2) ? 8 : 0);
+                const int col = 2 * t + (q & 1);
+                if (row >= m.N)
+                    continue;
+                if constexpr (MOE) {
+                    if (col < grp.piece_count[u]) {
+                        const int slot = grp.sorted_slot[grp.piece_first[u] + col];
+                        m.y[(size_t)slot * m.N + row] = v[mt][q];
+                    }
+                } else {
+                    if (col < m.B)
+                        m.y[(size_t)col * m.N + row] = v[mt][q];
                 }
-            } else {
-                if (col < m.B)
-                    m.y[(size_t)col * m.N + row] = v[q];
             }
         }
     };
 
-    auto flush = [&](int s, int u, int band, const float (&acc)[4]) {
+    // Partials: [worker][slot 0/1][mt][lane] float4.
+    auto part_at = [&](int v, int sl, int mt) {
+        return reinterpret_cast<float4 *>(a.partials) + (((size_t)v * 2 + sl) * MT + mt) * 32 + lane;
+    };
+    auto flush = [&](int s, int u, int band, const float (&acc)[MT][4]) {
         const StageDesc &st = stg[s];
         const int cpb = unit_cpb(u);
         const int bs = unit_chunk_base(u) + band * cpb, be = bs + cpb;
@@ -351,8 +361,9 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
             return;
         }
         const int myslot = (c0 >= bs) ? 0 : 1;
-        float4 *part = reinterpret_cast<float4 *>(a.partials);
-        __stcg(part + ((size_t)w * 2 + myslot) * 32 + lane, make_float4(acc[0], acc[1], acc[2], acc[3]));
+#pragma unroll
+        for (int mt = 0; mt < MT; mt++)
+            __stcg(part_at(w, myslot, mt), make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]));
         __threadfence();
         __syncwarp();
         const int wf = bs / st.cpw, wl = (be - 1) / st.cpw;
@@ -364,19 +375,21 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
         if (old != wl - wf)
             return;
         __threadfence();
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        float s4[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; mt++)
+            s4[mt][0] = s4[mt][1] = s4[mt][2] = s4[mt][3] = 0.f;
         for (int v = wf; v <= wl; v++) {
-            float4 p;
-            if (v == w) {
-                p = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            } else {
-                const int sl = (v * st.cpw >= bs) ? 0 : 1;
-                p = __ldcg(part + ((size_t)v * 2 + sl) * 32 + lane);
+            const int sl = (v * st.cpw >= bs) ? 0 : 1;
+#pragma unroll
+            for (int mt = 0; mt < MT; mt++) {
+                const float4 p = (v == w) ? make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3])
+                                          : __ldcg(part_at(v, sl, mt));
+                s4[mt][0] += p.x;
+                s4[mt][1] += p.y;
+                s4[mt][2] += p.z;
+                s4[mt][3] += p.w;
             }
-            s4[0] += p.x;
-            s4[1] += p.y;
-            s4[2] += p.z;
-            s4[3] += p.w;
         }
         store_band(u, band, s4);
         if (lane == 0)
@@ -384,9 +397,12 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
     };
 
     // Grid barrier between stages (plan mode; the launch is cooperative, so
-    // every CTA is resident).  The last warp of a CTA to finish stage s bumps
-    // the grid counter, waits for all CTAs, then releases its CTA's warps
-    // through a shared mbarrier.  Every wait is bounded.
+    // every CTA is resident).  The last warp of a CTA to finish stage s adds
+    // one arrival to the grid counter; the CTA whose arrival completes stage s
+    // publishes s+1 in a separate flag word, which every CTA's last warp polls
+    // (with back-off, so the pollers do not hammer the line the arrivals hit)
+    // before releasing its CTA's warps through a shared mbarrier.  Every wait
+    // is bounded.
     bool ok = true;
     auto stage_arrive_and_wait = [&](int s) {
         __syncwarp();
@@ -394,15 +410,21 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
             __threadfence();
             const int old = atomicAdd(&cta_arrivals, 1);
             if (old == kWarps * (s + 1) - 1) {
-                atomicAdd(&a.sync[0], 1u);
                 const unsigned target = gridDim.x * (unsigned)(s + 1);
+                if (atomicAdd(&a.sync[0], 1u) == target - 1) {
+                    __threadfence();
+                    atomicExch(&a.sync[32], (unsigned)(s + 1));
+                }
                 const long long t0 = clock64();
-                while (ld_acquire_gpu(&a.sync[0]) < target) {
+                unsigned ns = 32;
+                while (ld_acquire_gpu(&a.sync[32]) < (unsigned)(s + 1)) {
                     if (clock64() - t0 > kWaitCycles) {
                         if (a.status)
                             atomicOr(a.status, kStatusTimeout);
                         break;
                     }
+                    __nanosleep(ns);
+                    ns = ns < 256 ? 2 * ns : 256;
                 }
                 asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&stage_bar))
                              : "memory");
@@ -420,8 +442,10 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
     Cursor cur;
     bool live = seek(cur, 0);
     int done = 0;                  // chunks consumed (ring index)
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[MT][4];
     int acc_u = -1, acc_band = -1; // band the accumulators belong to
+    int sw[8];
+    lane_swizzle<FMT>(g, sw);
     const __half *xrow = nullptr;
     int nb32 = 0;
 
@@ -446,7 +470,9 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
             if (cur.u != acc_u || cur.band != acc_band) {
                 if (acc_u >= 0)
                     flush(s, acc_u, acc_band, acc);
-                acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+#pragma unroll
+                for (int mt = 0; mt < MT; mt++)
+                    acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
                 if (cur.u != acc_u) {
                     const MatDesc &m = unit_mat(cur.u);
                     nb32 = m.K / kBlock;
@@ -462,8 +488,8 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
                 acc_band = cur.band;
             }
             const int left = nb32 - cur.kp * 8;
-            chunk_mma<FMT>(codes_ring + slot * CB, scales_ring + slot * kScaleBytes, xrow,
-                           cur.kp * kChunkK, left < 8 ? left : 8, g, t, acc);
+            chunk_mma<FMT>(codes_ring + slot * CB, scales_ring + slot * SB, xrow,
+                           cur.kp * kChunkK, left < 8 ? left : 8, g, t, sw, acc);
             done++;
             advance(cur);
             live = cur.s < n_stages;
@@ -487,10 +513,11 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
         __syncthreads();
         if (threadIdx.x == 0) {
             __threadfence();
-            const unsigned old = atomicAdd(&a.sync[1], 1u);
+            const unsigned old = atomicAdd(&a.sync[64], 1u);
             if (old == gridDim.x - 1) {
                 a.sync[0] = 0;
-                a.sync[1] = 0;
+                a.sync[32] = 0;
+                a.sync[64] = 0;
                 __threadfence();
             }
         }
@@ -549,18 +576,20 @@ int max_ctas()
 
 size_t counters_bytes(long long n) { return align_up((size_t)n * sizeof(int), 256); }
 constexpr size_t kPartialsBytes = (size_t)kMaxWorkers * kPartialBytesPerWorker;
-constexpr size_t kSyncBytes = 256;
+constexpr size_t kSyncBytes = 512;
+
+int rows_of(int fmt) { return fmt == 4 ? Fmt<4>::kRows : Fmt<8>::kRows; }
 
 bool fill_matdesc(int fmt, const bq_qmat *W, const uint16_t *x, int B, float *y, MatDesc *m)
 {
-    const int N = W->N, K = W->K;
+    const int N = W->N, K = W->K, R = rows_of(fmt);
     const uint64_t cdims[2] = {(uint64_t)(fmt == 4 ? K / 2 : K), (uint64_t)N};
     const uint64_t cstr[1] = {(uint64_t)(fmt == 4 ? K / 2 : K)};
-    const uint32_t cbox[2] = {128, (uint32_t)kChunkRows};
+    const uint32_t cbox[2] = {128, (uint32_t)R};
     const int ldS = bq_scales_ld(K);
     const uint64_t sdims[2] = {(uint64_t)(K / 32), (uint64_t)N};
     const uint64_t sstr[1] = {(uint64_t)ldS * 2};
-    const uint32_t sbox[2] = {8, (uint32_t)kChunkRows};
+    const uint32_t sbox[2] = {8, (uint32_t)R};
     if (!encode_tensor_map(&m->tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, cdims, cstr,
                            cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_tensor_map(&m->tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, W->scales, sdims, sstr,
@@ -572,7 +601,7 @@ bool fill_matdesc(int fmt, const bq_qmat *W, const uint16_t *x, int B, float *y,
     m->K = K;
     m->B = B;
     m->cpb = (K + kChunkK - 1) / kChunkK;
-    m->nbands = (N + kChunkRows - 1) / kChunkRows;
+    m->nbands = (N + R - 1) / R;
     m->chunk_base = 0;
     m->band_base = 0;
     return true;
@@ -603,7 +632,7 @@ int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void
         return BQ_ERR_ALIGN;
     if (ws_bytes < bq_gemv_workspace_bytes(W->N, W->K))
         return BQ_ERR_WORKSPACE;
-    const long long nbands = (W->N + kChunkRows - 1) / kChunkRows;
+    const long long nbands = (W->N + 15) / 16;
     if (nbands * ((W->K + kChunkK - 1) / kChunkK) >= (1LL << 31))
         return BQ_ERR_SHAPE;
     st = prepare_kernel<FMT, kModeMatrix>();
@@ -675,7 +704,7 @@ extern "C" size_t bq_gemv_workspace_bytes(int32_t N, int32_t K)
 {
     if (N < 1 || K < 32 || K % 32 != 0)
         return 0;
-    const long long nbands = (N + kChunkRows - 1) / kChunkRows;
+    const long long nbands = (N + 15) / 16;   // the finest band height of any format
     return counters_bytes(nbands) + kPartialsBytes;
 }
 
@@ -819,7 +848,7 @@ extern "C" size_t bq_moe_workspace_bytes(int32_t N, int32_t K, int32_t B, int32_
     if (N < 1 || K < 32 || K % 32 != 0 || B < 1 || B > 8 || topk < 1 || B * topk > kMaxSlots ||
         E < 1 || E > 65535)
         return 0;
-    const long long nbands = (N + kChunkRows - 1) / kChunkRows;
+    const long long nbands = (N + Fmt<4>::kRows - 1) / Fmt<4>::kRows;
     return counters_bytes(nbands * B * topk) + kPartialsBytes +
            align_up((size_t)B * topk * N * sizeof(float), 256);
 }
@@ -846,7 +875,7 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
         return BQ_ERR_ALIGN;
     if (ws_bytes < bq_moe_workspace_bytes(N, K, B, topk, E))
         return BQ_ERR_WORKSPACE;
-    const long long nbands = (N + kChunkRows - 1) / kChunkRows;
+    const long long nbands = (N + Fmt<4>::kRows - 1) / Fmt<4>::kRows;
     const long long cpb = (K + kChunkK - 1) / kChunkK;
     if ((long long)B * topk * nbands * cpb >= (1LL << 31))
         return BQ_ERR_SHAPE;
@@ -858,10 +887,10 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
     memset(&a, 0, sizeof(a));
     const uint64_t cdims[3] = {(uint64_t)(K / 2), (uint64_t)N, (uint64_t)E};
     const uint64_t cstr[2] = {(uint64_t)(K / 2), (uint64_t)codes_stride};
-    const uint32_t cbox[3] = {128, (uint32_t)kChunkRows, 1};
+    const uint32_t cbox[3] = {128, (uint32_t)Fmt<4>::kRows, 1};
     const uint64_t sdims[3] = {(uint64_t)(K / 32), (uint64_t)N, (uint64_t)E};
     const uint64_t sstr[2] = {(uint64_t)ldS * 2, (uint64_t)scales_stride * 2};
-    const uint32_t sbox[3] = {8, (uint32_t)kChunkRows, 1};
+    const uint32_t sbox[3] = {8, (uint32_t)Fmt<4>::kRows, 1};
     if (!encode_tensor_map(&a.mat0.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, Wstack->codes,
                            cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_tensor_map(&a.mat0.tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, Wstack->scales,
