@@ -7,14 +7,12 @@
 // along K (8 blocks of 32).  A chunk's codes arrive in shared memory through
 // one (Q4: 32 rows x 128 bytes) or two (Q8: 16 rows x 128 bytes each) 2-D TMA
 // boxes with the 128-byte swizzle, its scales through one kRows x 8 fp16 box.  A warp reads them with 32-bit shared loads that
-// the swizzle makes bank-conflict free, dequantises each 4-byte group into
-// fp16 pairs in registers (the codes are small integers, exact in fp16), and
-// forms the block's partial dot products with m16n8k16 mma.sync (fp16 in,
-// fp32 accumulate): M = 16 weight rows (a Q4 chunk is two such m-tiles that
+// the swizzle makes bank-conflict free, turns each 4-byte group into fp16
+// pairs in registers (exact: see "dequant" below), and forms the block's
+// partial dot products with m16n8k16 mma.sync (fp16 in, fp32 accumulate): M = 16 weight rows (a Q4 chunk is two such m-tiles that
 // share every x fragment), N = the batch (B <= 8), K = 16 elements of one
-// block.  Each block's partial sum
-// is scaled by its fp32-converted scale once (y += d * sum(q * x)), so the
-// only roundings are fp32 ones.
+// block.  Each block's partial sum is scaled by its fp32-converted scale once
+// (y += d * sum((q - z) x)), so the only roundings are fp32 ones.
 #pragma once
 
 #include <cuda.h>
@@ -214,39 +212,53 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // the 4 consecutive code bytes 4t..4t+3 it loads, and its x fragment is the
 // 4 consecutive x values at the same k -- one 8-byte load, no shuffles.
 //
-// Q4: bytes b0..b3 of a word hold elements e..e+3 (low nibbles) and
-// e+16..e+19 (high nibbles).  fp16 0x6400 | n is 1024 + n exactly.
+// Codes enter the tensor core as fp16 *subnormals*: a 16-bit lane holding the
+// integer u (< 1024) in its low bits and zero elsewhere is exactly u * 2^-24,
+// so masking the code bits into place is the whole conversion.  The format's
+// zero point z (8 for Q4, 128 for the Q8 code biased by +128) is removed by a
+// second mma that starts each block's accumulator at -z * 2^-24 * sum(x)
+// (see block_mma).  Every product is exact; the 2^-24 is undone at the store.
 struct Q4Pairs {
-    uint32_t lo01, lo23, hi01, hi23;   // f16x2 of (q - 8)
+    uint32_t lo01, lo23, hi01, hi23;   // f16x2 of q * 2^-24, q in [0, 15]
 };
 
 __device__ __forceinline__ Q4Pairs dequant_q4(uint32_t w)
 {
+    // bytes b0..b3 of w hold elements e..e+3 (low nibbles) and e+16..e+19
+    // (high nibbles)
     const uint32_t p01 = prmt(w, 0u, 0x4140u);    // [b0, 0, b1, 0]
     const uint32_t p23 = prmt(w, 0u, 0x4342u);    // [b2, 0, b3, 0]
     Q4Pairs r;
-    // low nibble n: (1024 + n) - 1032 = n - 8
-    r.lo01 = hsub2u((p01 & 0x000F000Fu) | 0x64006400u, 0x64086408u);
-    r.lo23 = hsub2u((p23 & 0x000F000Fu) | 0x64006400u, 0x64086408u);
-    // high nibble n (in place): (1024 + 16 n) / 16 - 72 = n - 8
-    r.hi01 = hfma2u((p01 & 0x00F000F0u) | 0x64006400u, 0x2C002C00u, 0xD480D480u);
-    r.hi23 = hfma2u((p23 & 0x00F000F0u) | 0x64006400u, 0x2C002C00u, 0xD480D480u);
+    r.lo01 = p01 & 0x000F000Fu;
+    r.lo23 = p23 & 0x000F000Fu;
+    r.hi01 = (p01 >> 4) & 0x000F000Fu;
+    r.hi23 = (p23 >> 4) & 0x000F000Fu;
     return r;
 }
 
-// Q8: int8 q -> byte q ^ 0x80 = q + 128 in [0, 255]; (1024 + q + 128) - 1152 = q.
+// Q8: int8 q -> byte u = q ^ 0x80 = q + 128 in [0, 255], as u * 2^-24.
 struct Q8Pairs {
-    uint32_t p01, p23;                 // f16x2 of q
+    uint32_t p01, p23;                 // f16x2 of (q + 128) * 2^-24
 };
 
 __device__ __forceinline__ Q8Pairs dequant_q8(uint32_t w)
 {
     const uint32_t u = w ^ 0x80808080u;
     Q8Pairs r;
-    r.p01 = hsub2u(prmt(u, 0x64646464u, 0x4140u), 0x64806480u);
-    r.p23 = hsub2u(prmt(u, 0x64646464u, 0x4342u), 0x64806480u);
+    r.p01 = prmt(u, 0u, 0x4140u);
+    r.p23 = prmt(u, 0u, 0x4342u);
     return r;
 }
+
+// f16x2 of -z * 2^-24 (a subnormal): z = 8 -> 2^-21, z = 128 -> 2^-17.
+template <int FMT>
+__host__ __device__ constexpr uint32_t zero_point_pair()
+{
+    return FMT == 4 ? 0x80088008u : 0x80808080u;
+}
+
+// The y of a band is stored as acc * 2^24.
+constexpr float kUnscale = 16777216.0f;
 
 __device__ __forceinline__ float half_lo(uint32_t v)
 {
@@ -265,21 +277,33 @@ __device__ __forceinline__ uint32_t pick_u32(const uint4 &v, int i)
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
 
+// sum(x) of one block, pre-multiplied by -z * 2^-24, in the accumulator
+// layout (rows are all equal): the starting value of the block's mma chain.
+template <int FMT>
+__device__ __forceinline__ void block_offset(uint2 xa, uint2 xb, float (&s)[4])
+{
+    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t z = zero_point_pair<FMT>();
+    mma16816(s, z, z, z, z, xa.x, xa.y, zero);
+    mma16816(s, z, z, z, z, xb.x, xb.y, s);
+}
+
 // One block (32 weights along K) of the chunk for m-tile mt (rows
 // 16*mt + g and 16*mt + g + 8).  `xa` holds x at k..k+3 and `xb` at
 // k+16..k+19 (k = block start + 4t) for batch column g; `sw` is this lane's
-// swizzled offset of block jb in a 128-byte code row.
+// swizzled offset of block jb in a 128-byte code row; `off` the block's
+// zero-point term from block_offset.
 template <int FMT>
 __device__ __forceinline__ void block_mma(const uint8_t *lane_codes, int jb, int sw, uint2 xa,
-                                          uint2 xb, float dg, float dg8, float (&acc)[4])
+                                          uint2 xb, const float (&off)[4], float dg, float dg8,
+                                          float (&acc)[4])
 {
-    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
     float c[4];
     if constexpr (FMT == 4) {
         const uint8_t *p = lane_codes + sw;
         const Q4Pairs r0 = dequant_q4(lds32(p));          // row g
         const Q4Pairs r8 = dequant_q4(lds32(p + 1024));   // row g + 8
-        mma16816(c, r0.lo01, r8.lo01, r0.lo23, r8.lo23, xa.x, xa.y, zero);
+        mma16816(c, r0.lo01, r8.lo01, r0.lo23, r8.lo23, xa.x, xa.y, off);
         mma16816(c, r0.hi01, r8.hi01, r0.hi23, r8.hi23, xb.x, xb.y, c);
     } else {
         // sw holds the offsets of the block's two 16-byte halves (granules
@@ -290,7 +314,7 @@ __device__ __forceinline__ void block_mma(const uint8_t *lane_codes, int jb, int
         const Q8Pairs a8 = dequant_q8(lds32(base + oa + 1024));
         const Q8Pairs b0 = dequant_q8(lds32(base + ob));
         const Q8Pairs b8 = dequant_q8(lds32(base + ob + 1024));
-        mma16816(c, a0.p01, a8.p01, a0.p23, a8.p23, xa.x, xa.y, zero);
+        mma16816(c, a0.p01, a8.p01, a0.p23, a8.p23, xa.x, xa.y, off);
         mma16816(c, b0.p01, b8.p01, b0.p23, b8.p23, xb.x, xb.y, c);
     }
     acc[0] = fmaf(dg, c[0], acc[0]);
@@ -343,12 +367,15 @@ __device__ __forceinline__ void chunk_mma(const uint8_t *codes_s, const uint8_t 
         }
 #pragma unroll
         for (int jb = 0; jb < 8; jb++) {
+            float off[4];
+            block_offset<FMT>(xa[jb], xb[jb], off);
 #pragma unroll
             for (int mt = 0; mt < MT; mt++) {
                 const uint32_t wg = pick_u32(sc[mt][0], jb >> 1), wg8 = pick_u32(sc[mt][1], jb >> 1);
                 const float dg = (jb & 1) ? half_hi(wg) : half_lo(wg);
                 const float dg8 = (jb & 1) ? half_hi(wg8) : half_lo(wg8);
-                block_mma<FMT>(lane_codes + mt * 2048, jb, sw[jb], xa[jb], xb[jb], dg, dg8, acc[mt]);
+                block_mma<FMT>(lane_codes + mt * 2048, jb, sw[jb], xa[jb], xb[jb], off, dg, dg8,
+                               acc[mt]);
             }
         }
     } else {
@@ -357,12 +384,14 @@ __device__ __forceinline__ void chunk_mma(const uint8_t *codes_s, const uint8_t 
             if (jb < nblk) {
                 const uint2 xa = ldg64(xp + 32 * jb);
                 const uint2 xb = ldg64(xp + 32 * jb + 16);
+                float off[4];
+                block_offset<FMT>(xa, xb, off);
 #pragma unroll
                 for (int mt = 0; mt < MT; mt++) {
                     const uint32_t wg = pick_u32(sc[mt][0], jb >> 1), wg8 = pick_u32(sc[mt][1], jb >> 1);
                     const float dg = (jb & 1) ? half_hi(wg) : half_lo(wg);
                     const float dg8 = (jb & 1) ? half_hi(wg8) : half_lo(wg8);
-                    block_mma<FMT>(lane_codes + mt * 2048, jb, sw[jb], xa, xb, dg, dg8, acc[mt]);
+                    block_mma<FMT>(lane_codes + mt * 2048, jb, sw[jb], xa, xb, off, dg, dg8, acc[mt]);
                 }
             }
         }

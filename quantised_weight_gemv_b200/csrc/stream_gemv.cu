@@ -337,11 +337,11 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
                 if constexpr (MOE) {
                     if (col < grp.piece_count[u]) {
                         const int slot = grp.sorted_slot[grp.piece_first[u] + col];
-                        m.y[(size_t)slot * m.N + row] = v[mt][q];
+                        m.y[(size_t)slot * m.N + row] = v[mt][q] * kUnscale;
                     }
                 } else {
                     if (col < m.B)
-                        m.y[(size_t)col * m.N + row] = v[mt][q];
+                        m.y[(size_t)col * m.N + row] = v[mt][q] * kUnscale;
                 }
             }
         }
