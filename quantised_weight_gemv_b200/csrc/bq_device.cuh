@@ -35,14 +35,28 @@ constexpr int kStatusRange = 1 << 9;
 // A bounded wait gives up after this many SM clock cycles (~2 s).
 constexpr long long kWaitCycles = 4000000000LL;
 
+// Tuning knobs (compile-time; the defaults are the measured best on B200).
+#ifndef BQ_Q4_MT
+#define BQ_Q4_MT 2          // 16-row m-tiles per Q4 chunk
+#endif
+#ifndef BQ_STAGES
+#define BQ_STAGES 2         // ring slots per worker warp
+#endif
+#ifndef BQ_MIN_BLOCKS
+#define BQ_MIN_BLOCKS 2     // CTAs per SM the register budget is sized for
+#endif
+#ifndef BQ_Q4_HI_INPLACE
+#define BQ_Q4_HI_INPLACE 0  // 1: high nibbles stay in place (x scaled by 1/16)
+#endif
+
 template <int FMT> struct Fmt;
 template <> struct Fmt<4> {
-    static constexpr int kMT = 2;                       // m-tiles of 16 rows per chunk
+    static constexpr int kMT = BQ_Q4_MT;                // m-tiles of 16 rows per chunk
     static constexpr int kRows = 16 * kMT;              // rows per chunk / band
     static constexpr int kBoxes = 1;                    // 128-byte-wide code boxes
     static constexpr int kCodeBytes = kRows * 128;      // 4 KB
     static constexpr int kScaleBytes = kRows * 16;      // kRows x 8 fp16
-    static constexpr int kStages = 3;
+    static constexpr int kStages = BQ_STAGES;
 };
 template <> struct Fmt<8> {
     static constexpr int kMT = 1;
@@ -50,7 +64,7 @@ template <> struct Fmt<8> {
     static constexpr int kBoxes = 2;
     static constexpr int kCodeBytes = 2 * kRows * 128;  // 4 KB
     static constexpr int kScaleBytes = kRows * 16;
-    static constexpr int kStages = 3;
+    static constexpr int kStages = BQ_STAGES;
 };
 
 template <int FMT>
@@ -166,10 +180,27 @@ __device__ __forceinline__ uint4 lds128(const uint8_t *p)
     return *reinterpret_cast<const uint4 *>(p);
 }
 
-// 8 bytes of x through the read-only, L1-cached path.
+// 8 bytes of x through the read-only path, kept in L1 (every warp of the SM
+// re-reads the same activations for every band).
 __device__ __forceinline__ uint2 ldg64(const void *p)
 {
-    return __ldg(reinterpret_cast<const uint2 *>(p));
+    uint2 v;
+    asm("ld.global.nc.L1::evict_last.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+
+// Release / acquire read-modify-writes at GPU scope (no separate fence).
+__device__ __forceinline__ int atom_add_release_gpu(int *p, int v)
+{
+    int old;
+    asm volatile("atom.add.release.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int *p, int v)
+{
+    int old;
+    asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
 }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
@@ -183,6 +214,13 @@ __device__ __forceinline__ uint32_t hsub2u(uint32_t a, uint32_t b)
 {
     uint32_t d;
     asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
@@ -231,8 +269,13 @@ __device__ __forceinline__ Q4Pairs dequant_q4(uint32_t w)
     Q4Pairs r;
     r.lo01 = p01 & 0x000F000Fu;
     r.lo23 = p23 & 0x000F000Fu;
+#if BQ_Q4_HI_INPLACE
+    r.hi01 = p01 & 0x00F000F0u;       // 16 q * 2^-24: paired with x / 16
+    r.hi23 = p23 & 0x00F000F0u;
+#else
     r.hi01 = (p01 >> 4) & 0x000F000Fu;
     r.hi23 = (p23 >> 4) & 0x000F000Fu;
+#endif
     return r;
 }
 
@@ -304,7 +347,12 @@ __device__ __forceinline__ void block_mma(const uint8_t *lane_codes, int jb, int
         const Q4Pairs r0 = dequant_q4(lds32(p));          // row g
         const Q4Pairs r8 = dequant_q4(lds32(p + 1024));   // row g + 8
         mma16816(c, r0.lo01, r8.lo01, r0.lo23, r8.lo23, xa.x, xa.y, off);
+#if BQ_Q4_HI_INPLACE
+        const uint32_t xb0 = hmul2u(xb.x, 0x2C002C00u), xb1 = hmul2u(xb.y, 0x2C002C00u);
+        mma16816(c, r0.hi01, r8.hi01, r0.hi23, r8.hi23, xb0, xb1, c);
+#else
         mma16816(c, r0.hi01, r8.hi01, r0.hi23, r8.hi23, xb.x, xb.y, c);
+#endif
     } else {
         // sw holds the offsets of the block's two 16-byte halves (granules
         // 2jj and 2jj+1 of box jb/4) packed as two 16-bit values.

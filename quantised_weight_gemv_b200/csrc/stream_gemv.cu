@@ -151,12 +151,14 @@ __device__ void group_experts(const KernelArgs &a, ExpertGroups &grp)
     __syncwarp();
 }
 
-// Position of a chunk inside a stage: matrix (or expert piece) u, band, k-piece.
+// Position of a chunk inside a stage: matrix (or expert piece) u, band, k-piece,
+// with the current unit's geometry cached in registers.
 struct Cursor {
     int s;        // stage
     int u;        // matrix index (plan: global; otherwise 0 / piece)
     int band, kp;
     int c, c_end; // chunk index within the stage and end of this worker's range
+    int cpb, nbands;
 };
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
@@ -167,7 +169,7 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
 }
 
 template <int FMT, int MODE>
-__global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_constant__ KernelArgs a)
+__global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(const __grid_constant__ KernelArgs a)
 {
     constexpr int D = Fmt<FMT>::kStages;
     constexpr int CB = Fmt<FMT>::kCodeBytes;
@@ -241,14 +243,16 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
     const int w = warp * gridDim.x + blockIdx.x;
     const uint64_t pol = policy_evict_first();
 
-    // Per-unit geometry (matrix, or expert piece in MoE mode).
-    auto unit_mat = [&](int u) -> const MatDesc & { return MOE ? a.mat0 : mats[u]; };
+    // Per-unit geometry (matrix, or expert piece in MoE mode).  Only plan mode
+    // indexes a descriptor array; the other modes have one descriptor.
+    auto unit_mat = [&](int u) -> const MatDesc & { return PLAN ? mats[u] : a.mat0; };
     auto unit_cpb = [&](int u) { return unit_mat(u).cpb; };
-    auto unit_nbands = [&](int u) { return unit_mat(u).nbands; };
     auto unit_chunk_base = [&](int u) {
-        return MOE ? u * a.mat0.nbands * a.mat0.cpb : mats[u].chunk_base;
+        return PLAN ? mats[u].chunk_base : (MOE ? u * a.mat0.nbands * a.mat0.cpb : 0);
     };
-    auto unit_band_base = [&](int u) { return MOE ? u * a.mat0.nbands : mats[u].band_base; };
+    auto unit_band_base = [&](int u) {
+        return PLAN ? mats[u].band_base : (MOE ? u * a.mat0.nbands : 0);
+    };
 
     // Place a cursor at the first chunk of this worker's range in stage s, or
     // at the first later stage where the range is non-empty.  Returns false
@@ -260,15 +264,17 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
                 continue;
             const int c0 = w * st.cpw;
             const int c1 = min(c0 + st.cpw, st.T);
-            int u = MOE ? c0 / (a.mat0.nbands * a.mat0.cpb) : st.mat_begin;
-            if (!MOE)
+            int u = MOE ? c0 / (a.mat0.nbands * a.mat0.cpb) : (PLAN ? st.mat_begin : 0);
+            if (PLAN)
                 while (u + 1 < st.mat_end && mats[u + 1].chunk_base <= c0)
                     u++;
             const int rel = c0 - unit_chunk_base(u);
             cu.s = s;
             cu.u = u;
-            cu.band = rel / unit_cpb(u);
-            cu.kp = rel - cu.band * unit_cpb(u);
+            cu.cpb = unit_mat(u).cpb;
+            cu.nbands = unit_mat(u).nbands;
+            cu.band = rel / cu.cpb;
+            cu.kp = rel - cu.band * cu.cpb;
             cu.c = c0;
             cu.c_end = c1;
             return true;
@@ -278,15 +284,21 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
     };
     auto advance = [&](Cursor &cu) {
         cu.c++;
-        if (++cu.kp == unit_cpb(cu.u)) {
+        if (cu.c == cu.c_end) {
+            seek(cu, cu.s + 1);
+            return;
+        }
+        if (++cu.kp == cu.cpb) {
             cu.kp = 0;
-            if (++cu.band == unit_nbands(cu.u)) {
+            if (++cu.band == cu.nbands) {
                 cu.band = 0;
                 cu.u++;
+                if (PLAN) {
+                    cu.cpb = mats[cu.u].cpb;
+                    cu.nbands = mats[cu.u].nbands;
+                }
             }
         }
-        if (cu.c == cu.c_end)
-            seek(cu, cu.s + 1);
     };
 
     Cursor iss;
@@ -305,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
                 tma_load_3d(cdst, &a.mat0.tm_codes, bar, iss.kp * 128, row, e, pol);
                 tma_load_3d(sdst, &a.mat0.tm_scales, bar, iss.kp * 8, row, e, pol);
             } else {
-                const MatDesc &m = mats[iss.u];
+                const MatDesc &m = unit_mat(iss.u);
 #pragma unroll
                 for (int bx = 0; bx < Fmt<FMT>::kBoxes; bx++)
                     tma_load_2d(cdst + bx * (ROWS * 128), &m.tm_codes, bar,
@@ -364,17 +376,19 @@ __global__ void __launch_bounds__(kThreads, 2) stream_gemv_kernel(const __grid_c
 #pragma unroll
         for (int mt = 0; mt < MT; mt++)
             __stcg(part_at(w, myslot, mt), make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]));
-        __threadfence();
+        // The warp's partial stores happen before lane 0's release increment
+        // (__syncwarp orders them); the last arriver's acquire increment then
+        // makes every partial visible to the whole warp (__syncwarp again).
         __syncwarp();
         const int wf = bs / st.cpw, wl = (be - 1) / st.cpw;
         int *ctr = a.counters + unit_band_base(u) + band;
         int old = 0;
         if (lane == 0)
-            old = atomicAdd(ctr, 1);
+            old = atom_add_acq_rel_gpu(ctr, 1);
         old = __shfl_sync(0xffffffffu, old, 0);
         if (old != wl - wf)
             return;
-        __threadfence();
+        __syncwarp();
         float s4[MT][4];
 #pragma unroll
         for (int mt = 0; mt < MT; mt++)
@@ -565,13 +579,13 @@ int32_t prepare_kernel()
     return BQ_OK;
 }
 
-// CTAs of one launch: two per SM (the kernel's occupancy), capped.
+// CTAs of one launch: BQ_MIN_BLOCKS per SM (the kernel's occupancy), capped.
 int max_ctas()
 {
     const int sms = device_sm_count();
     if (sms <= 0)
         return -1;
-    return std::min(2 * sms, kMaxCtas);
+    return std::min(BQ_MIN_BLOCKS * sms, kMaxCtas);
 }
 
 size_t counters_bytes(long long n) { return align_up((size_t)n * sizeof(int), 256); }
@@ -767,7 +781,7 @@ extern "C" int32_t bq_step_plan(int32_t fmt, const bq_step_mat *mats, int32_t n_
     const int sms = device_sm_count();
     if (sms <= 0)
         return BQ_ERR_CUDA;
-    const int G = std::min(std::min(occ, 2) * sms, kMaxCtas);
+    const int G = std::min(std::min(occ, BQ_MIN_BLOCKS) * sms, kMaxCtas);
     const int wmax = G * kWarps;
 
     std::vector<int> order(n_mats);
