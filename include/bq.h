@@ -132,6 +132,26 @@ BQ_API int32_t bq_gemv_q4(const bq_qmat *W, const uint16_t *x, int32_t B, float 
 BQ_API int32_t bq_gemv_q8(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
                    void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
 
+/* Q4 decode GEMV for callers that cannot allocate device memory: code inside
+ * a framework that owns every device allocation, or a decode loop that must
+ * never call cudaMalloc (it can synchronise the device).  The pages have no
+ * counterpart of this entry point; it exists for such callers only.
+ * Same operation, arguments and results as bq_gemv_q4, without ws/ws_bytes:
+ * the scratch the kernel needs lives in one fixed array inside the library
+ * (about 5.3 MB, reserved on every GPU that loads the library until the
+ * process exits).
+ *   - N must be <= 1048576 rows; larger N returns BQ_ERR_WORKSPACE and
+ *     launches nothing.  Nothing is allocated: no cudaMalloc / cudaFree.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array and clears the part that must start at
+ *     zero (an async memset on `stream`) before its kernel.  Calls that can
+ *     overlap on the GPU (other streams, other host threads) race on it and
+ *     must be serialised by the caller. */
+BQ_API int32_t bq_gemv_q4_noalloc(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
+                                  int32_t *dev_status, void *stream);
+
 /* --------------------------------------------------------- decode step --- */
 
 /* One matrix of a decode step.  All planes and buffers are device memory. */

@@ -56,6 +56,7 @@ _SIGS = {
     "bq_gemv_workspace_bytes": (_sz, [_i32, _i32]),
     "bq_gemv_q4": (_i32, [_QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
     "bq_gemv_q8": (_i32, [_QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
+    "bq_gemv_q4_noalloc": (_i32, [_QP, _vp, _i32, _vp, _vp, _vp]),
     "bq_step_plan_bytes": (_sz, [_i32]),
     "bq_step_plan": (_i32, [_i32, _SMP, _i32, _vp, _sz, _SIP]),
     "bq_step_run": (_i32, [_SIP, _vp, _vp, _sz, _vp, _vp]),

@@ -45,6 +45,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "bq_device.cuh"
@@ -948,4 +949,105 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
             return BQ_ERR_CUDA;
     }
     return BQ_OK;
+}
+
+// ------------------------------------------------- Q4 GEMV without workspace --
+// Some callers cannot hand the library a workspace: code embedded in a host
+// framework that owns every device allocation, or a latency-critical decode
+// loop that must never call cudaMalloc (which can synchronise the device).
+// bq_gemv_q4_noalloc serves them with the scratch the split-band sums need
+// (arrival counters + partial sums) held in one fixed device array below.
+// That array is part of the loaded library: every GPU that loads it keeps
+// kNoAllocScratchBytes reserved until the process exits.
+namespace bq {
+namespace {
+constexpr int kNoAllocMaxCtas = 320;                     // 2560 worker warps at most
+constexpr long long kNoAllocMaxRows = 1LL << 20;         // N limit of this entry point
+constexpr size_t kNoAllocCounterBytes = (size_t)(kNoAllocMaxRows / 16) * sizeof(int);
+constexpr size_t kNoAllocPartialBytes =
+    (size_t)kNoAllocMaxCtas * kWarps * 2 * Fmt<4>::kMT * 32 * sizeof(float4);
+constexpr size_t kNoAllocScratchBytes = kNoAllocCounterBytes + kNoAllocPartialBytes;
+}  // namespace
+}  // namespace bq
+
+static __device__ __align__(256) uint8_t g_bq_noalloc_scratch[bq::kNoAllocScratchBytes];
+
+namespace bq {
+namespace {
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[64];   // device address of the scratch array, per device
+
+// Device address of the scratch array on the current device.  The host-side
+// name g_bq_noalloc_scratch is only a stand-in, never a device address, so it
+// is looked up once per device (with that device current) and cached.
+void *noalloc_scratch(int32_t *err)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        *err = BQ_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_bq_noalloc_scratch) != cudaSuccess || !p) {
+            *err = BQ_ERR_CUDA;
+            return nullptr;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    return g_noalloc_ptr[dev];
+}
+}  // namespace
+}  // namespace bq
+
+extern "C" int32_t bq_gemv_q4_noalloc(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
+                                      int32_t *dev_status, void *stream)
+{
+    int32_t st = check_qmat(W);
+    if (st != BQ_OK)
+        return st;
+    if (!x || !y)
+        return BQ_ERR_NULL;
+    if (B < 1 || B > 8)
+        return BQ_ERR_BATCH;
+    if (!aligned16(x) || !aligned16(y))
+        return BQ_ERR_ALIGN;
+    if (W->N > kNoAllocMaxRows)
+        return BQ_ERR_WORKSPACE;   // more rows than the fixed scratch covers
+    const long long nbands16 = (W->N + 15) / 16;
+    if (nbands16 * ((W->K + kChunkK - 1) / kChunkK) >= (1LL << 31))
+        return BQ_ERR_SHAPE;
+    st = prepare_kernel<4, kModeMatrix>();
+    if (st != BQ_OK)
+        return st;
+    int32_t err = BQ_OK;
+    uint8_t *scratch = static_cast<uint8_t *>(noalloc_scratch(&err));
+    if (!scratch)
+        return err;
+
+    KernelArgs a;
+    memset(&a, 0, sizeof(a));
+    if (!fill_matdesc(4, W, x, B, y, &a.mat0))
+        return BQ_ERR_CUDA;
+    const long long T = (long long)a.mat0.cpb * a.mat0.nbands;
+    const int cap = max_ctas();
+    if (cap < 0)
+        return BQ_ERR_CUDA;
+    const int G = (int)std::min<long long>(std::min(cap, kNoAllocMaxCtas), T);
+    a.wmax = G * kWarps;
+    fill_stage(&a.stage0, 0, 1, T, a.mat0.nbands, a.wmax);
+    a.n_stages = 1;
+    a.counters = reinterpret_cast<int *>(scratch);
+    a.partials = reinterpret_cast<float *>(scratch + kNoAllocCounterBytes);
+    a.status = dev_status;
+    // The array keeps whatever the previous call left; the band counters
+    // must start at zero, so clear them on this call's stream first.
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(a.counters, 0, (size_t)a.mat0.nbands * sizeof(int), s) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    void *args[] = {&a};
+    cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<4, kModeMatrix>, dim3(G),
+                               dim3(kThreads), smem_bytes<4>(), s, args);
+    return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
