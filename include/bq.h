@@ -182,7 +182,8 @@ BQ_API size_t bq_step_plan_bytes(int32_t n_mats);
  * the fixed per-token overhead; "Kernel Fusie": launch overhead matters
  * because decode kernels are short) becomes one launch per token.
  *   fmt        4 or 8 (every matrix of the plan has this format)
- *   mats       host array of n_mats matrices (any order; stable by stage)
+ *   mats       host array of n_mats matrices (any order; stable by stage),
+ *              1 <= n_mats <= 256
  *   plan       device buffer, 64-byte aligned, >= bq_step_plan_bytes(n_mats);
  *              written synchronously (cudaMemcpy) -- do not call during
  *              stream capture

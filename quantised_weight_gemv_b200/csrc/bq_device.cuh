@@ -110,6 +110,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// Pass a value through an opaque volatile asm: anything computed from the
+// result is ordered after every earlier volatile asm (e.g. an mbarrier wait),
+// even when it is itself a non-volatile asm with no memory clobber.
+__device__ __forceinline__ uint32_t launder(uint32_t v)
+{
+    uint32_t r;
+    asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v) : "memory");
+    return r;
+}
+
 // Wait for phase `parity` of an mbarrier, giving up after kWaitCycles.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
 {
@@ -180,12 +190,19 @@ __device__ __forceinline__ uint4 lds128(const uint8_t *p)
     return *reinterpret_cast<const uint4 *>(p);
 }
 
-// 8 bytes of x through the read-only path, kept in L1 (every warp of the SM
-// re-reads the same activations for every band).
+// 8 bytes of x.  COHERENT = false: the read-only path, kept in L1 (every warp
+// of the SM re-reads the same activations for every band) -- valid when
+// nothing in the launch writes x.  COHERENT = true: cached in L2 only, so a
+// value another SM wrote earlier in the same launch (a previous stage's
+// output, after the grid barrier) is never read from a stale L1 line.
+template <bool COHERENT>
 __device__ __forceinline__ uint2 ldg64(const void *p)
 {
     uint2 v;
-    asm("ld.global.nc.L1::evict_last.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    if constexpr (COHERENT)
+        asm volatile("ld.global.cg.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    else
+        asm("ld.global.nc.L1::evict_last.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
     return v;
 }
 
@@ -325,55 +342,115 @@ __device__ __forceinline__ uint32_t pick_u32(const uint4 &v, int i)
 template <int FMT>
 __device__ __forceinline__ void block_offset(uint2 xa, uint2 xb, float (&s)[4])
 {
-    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
     const uint32_t z = zero_point_pair<FMT>();
-    mma16816(s, z, z, z, z, xa.x, xa.y, zero);
-    mma16816(s, z, z, z, z, xb.x, xb.y, s);
+    asm("{\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%4,%4,%4}, {%5,%6}, "
+        "{%9,%9,%9,%9};\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%4,%4,%4}, {%7,%8}, "
+        "{%0,%1,%2,%3};\n\t}"
+        : "=&f"(s[0]), "=&f"(s[1]), "=&f"(s[2]), "=&f"(s[3])
+        : "r"(z), "r"(xa.x), "r"(xa.y), "r"(xb.x), "r"(xb.y), "f"(0.0f));
 }
 
-// One block (32 weights along K) of the chunk for m-tile mt (rows
-// 16*mt + g and 16*mt + g + 8).  `xa` holds x at k..k+3 and `xb` at
-// k+16..k+19 (k = block start + 4t) for batch column g; `sw` is this lane's
-// swizzled offset of block jb in a 128-byte code row; `off` the block's
-// zero-point term from block_offset.
-template <int FMT>
-__device__ __forceinline__ void block_mma(const uint8_t *lane_codes, int jb, int sw, uint2 xa,
-                                          uint2 xb, const float (&off)[4], float dg, float dg8,
-                                          float (&acc)[4])
+// One Q4 block (32 weights along K) for one 16-row m-tile, in PTX so the
+// instruction sequence is exactly: 2 shared loads (rows g, g+8), 4 prmt and
+// 8 mask/shift ops to place the nibbles as fp16 subnormals, 2 mma (low then
+// high nibbles, starting from the zero-point term `off`), 4 fma for the
+// scales.  `addr` is the shared address of row g's 4-byte group.
+__device__ __forceinline__ void block_q4(uint32_t addr, uint2 xa, uint2 xb, const float (&off)[4],
+                                         float dg, float dg8, float (&acc)[4])
 {
-    float c[4];
-    if constexpr (FMT == 4) {
-        const uint8_t *p = lane_codes + sw;
-        const Q4Pairs r0 = dequant_q4(lds32(p));          // row g
-        const Q4Pairs r8 = dequant_q4(lds32(p + 1024));   // row g + 8
-        mma16816(c, r0.lo01, r8.lo01, r0.lo23, r8.lo23, xa.x, xa.y, off);
-#if BQ_Q4_HI_INPLACE
-        const uint32_t xb0 = hmul2u(xb.x, 0x2C002C00u), xb1 = hmul2u(xb.y, 0x2C002C00u);
-        mma16816(c, r0.hi01, r8.hi01, r0.hi23, r8.hi23, xb0, xb1, c);
-#else
-        mma16816(c, r0.hi01, r8.hi01, r0.hi23, r8.hi23, xb.x, xb.y, c);
-#endif
-    } else {
-        // sw holds the offsets of the block's two 16-byte halves (granules
-        // 2jj and 2jj+1 of box jb/4) packed as two 16-bit values.
-        const uint8_t *base = lane_codes + (jb >> 2) * 2048;
-        const int oa = sw & 0xffff, ob = sw >> 16;
-        const Q8Pairs a0 = dequant_q8(lds32(base + oa));
-        const Q8Pairs a8 = dequant_q8(lds32(base + oa + 1024));
-        const Q8Pairs b0 = dequant_q8(lds32(base + ob));
-        const Q8Pairs b8 = dequant_q8(lds32(base + ob + 1024));
-        mma16816(c, a0.p01, a8.p01, a0.p23, a8.p23, xa.x, xa.y, off);
-        mma16816(c, b0.p01, b8.p01, b0.p23, b8.p23, xb.x, xb.y, c);
-    }
-    acc[0] = fmaf(dg, c[0], acc[0]);
-    acc[1] = fmaf(dg, c[1], acc[1]);
-    acc[2] = fmaf(dg8, c[2], acc[2]);
-    acc[3] = fmaf(dg8, c[3], acc[3]);
+    asm("{\n\t"
+        ".reg .b32 w0, w8, p01, p23, q01, q23, a0, a1, a2, a3;\n\t"
+        ".reg .f32 c0, c1, c2, c3;\n\t"
+        "ld.shared.b32 w0, [%4];\n\t"
+        "ld.shared.b32 w8, [%4+1024];\n\t"
+        "prmt.b32 p01, w0, 0, 0x4140;\n\t"
+        "prmt.b32 p23, w0, 0, 0x4342;\n\t"
+        "prmt.b32 q01, w8, 0, 0x4140;\n\t"
+        "prmt.b32 q23, w8, 0, 0x4342;\n\t"
+        "and.b32 a0, p01, 0x000F000F;\n\t"
+        "and.b32 a1, q01, 0x000F000F;\n\t"
+        "and.b32 a2, p23, 0x000F000F;\n\t"
+        "and.b32 a3, q23, 0x000F000F;\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {c0,c1,c2,c3}, {a0,a1,a2,a3}, {%5,%6}, "
+        "{%9,%10,%11,%12};\n\t"
+        "shr.u32 p01, p01, 4;\n\t"
+        "shr.u32 q01, q01, 4;\n\t"
+        "shr.u32 p23, p23, 4;\n\t"
+        "shr.u32 q23, q23, 4;\n\t"
+        "and.b32 a0, p01, 0x000F000F;\n\t"
+        "and.b32 a1, q01, 0x000F000F;\n\t"
+        "and.b32 a2, p23, 0x000F000F;\n\t"
+        "and.b32 a3, q23, 0x000F000F;\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {c0,c1,c2,c3}, {a0,a1,a2,a3}, {%7,%8}, "
+        "{c0,c1,c2,c3};\n\t"
+        "fma.rn.f32 %0, %13, c0, %0;\n\t"
+        "fma.rn.f32 %1, %13, c1, %1;\n\t"
+        "fma.rn.f32 %2, %14, c2, %2;\n\t"
+        "fma.rn.f32 %3, %14, c3, %3;\n\t}"
+        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
+        : "r"(addr), "r"(xa.x), "r"(xa.y), "r"(xb.x), "r"(xb.y), "f"(off[0]), "f"(off[1]),
+          "f"(off[2]), "f"(off[3]), "f"(dg), "f"(dg8));
+}
+
+// One Q8 block for the 16-row m-tile: addr_a / addr_b are row g's 4-byte
+// groups in the block's two 16-element halves.
+__device__ __forceinline__ void block_q8(uint32_t addr_a, uint32_t addr_b, uint2 xa, uint2 xb,
+                                         const float (&off)[4], float dg, float dg8, float (&acc)[4])
+{
+    asm("{\n\t"
+        ".reg .b32 w0, w8, v0, v8, a0, a1, a2, a3;\n\t"
+        ".reg .f32 c0, c1, c2, c3;\n\t"
+        "ld.shared.b32 w0, [%4];\n\t"
+        "ld.shared.b32 w8, [%4+1024];\n\t"
+        "ld.shared.b32 v0, [%5];\n\t"
+        "ld.shared.b32 v8, [%5+1024];\n\t"
+        "xor.b32 w0, w0, 0x80808080;\n\t"
+        "xor.b32 w8, w8, 0x80808080;\n\t"
+        "prmt.b32 a0, w0, 0, 0x4140;\n\t"
+        "prmt.b32 a1, w8, 0, 0x4140;\n\t"
+        "prmt.b32 a2, w0, 0, 0x4342;\n\t"
+        "prmt.b32 a3, w8, 0, 0x4342;\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {c0,c1,c2,c3}, {a0,a1,a2,a3}, {%6,%7}, "
+        "{%10,%11,%12,%13};\n\t"
+        "xor.b32 v0, v0, 0x80808080;\n\t"
+        "xor.b32 v8, v8, 0x80808080;\n\t"
+        "prmt.b32 a0, v0, 0, 0x4140;\n\t"
+        "prmt.b32 a1, v8, 0, 0x4140;\n\t"
+        "prmt.b32 a2, v0, 0, 0x4342;\n\t"
+        "prmt.b32 a3, v8, 0, 0x4342;\n\t"
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {c0,c1,c2,c3}, {a0,a1,a2,a3}, {%8,%9}, "
+        "{c0,c1,c2,c3};\n\t"
+        "fma.rn.f32 %0, %14, c0, %0;\n\t"
+        "fma.rn.f32 %1, %14, c1, %1;\n\t"
+        "fma.rn.f32 %2, %15, c2, %2;\n\t"
+        "fma.rn.f32 %3, %15, c3, %3;\n\t}"
+        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
+        : "r"(addr_a), "r"(addr_b), "r"(xa.x), "r"(xa.y), "r"(xb.x), "r"(xb.y), "f"(off[0]),
+          "f"(off[1]), "f"(off[2]), "f"(off[3]), "f"(dg), "f"(dg8));
+}
+
+// Both halves of an fp16 pair as fp32.
+__device__ __forceinline__ void halves_to_float(uint32_t v, float &lo, float &hi)
+{
+    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "cvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(lo), "=f"(hi) : "r"(v));
+}
+
+__device__ __forceinline__ uint4 lds128_u32(uint32_t addr)
+{
+    uint4 v;
+    asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
 }
 
 // Per-lane swizzled offsets of the 8 blocks of a chunk row (constant for a
 // lane): TMA's 128-byte swizzle XORs the 16-byte granule index with the row
-// index mod 8, and row mod 8 == g for every row this lane reads.
+// index mod 8, and row mod 8 == g for every row this lane reads.  For Q8 the
+// two 16-byte halves of a block are packed as two 16-bit offsets.
 template <int FMT>
 __device__ __forceinline__ void lane_swizzle(int g, int (&sw)[8])
 {
@@ -388,61 +465,79 @@ __device__ __forceinline__ void lane_swizzle(int g, int (&sw)[8])
     }
 }
 
-// A whole chunk: 8 blocks (nblk of them valid) starting at k0 along K, for
-// the chunk's kMT m-tiles.  xrow points at x[column g][0]; a lane whose column
-// is absent (g >= B) reads a valid row instead -- its mma column is garbage
-// and is never stored, which keeps every load unconditional.
-template <int FMT>
-__device__ __forceinline__ void chunk_mma(const uint8_t *codes_s, const uint8_t *scales_s,
-                                          const __half *xrow, int k0, int nblk, int g, int t,
-                                          const int (&sw)[8], float (&acc)[Fmt<FMT>::kMT][4])
+// The x fragments of a chunk: for block jb, xa = x[k..k+3] and xb =
+// x[k+16..k+19] with k = k0 + 32 jb + 4t, for batch column g.  xrow points at
+// x[column g][0]; a lane whose column is absent (g >= B) reads a valid row
+// instead -- its mma column is garbage and is never stored, which keeps
+// every load unconditional.  Only the nblk valid blocks are read.
+template <bool COHERENT>
+__device__ __forceinline__ void chunk_load_x(const __half *xrow, int k0, int nblk, int t,
+                                             uint2 (&xa)[8], uint2 (&xb)[8])
 {
-    constexpr int MT = Fmt<FMT>::kMT;
-    uint4 sc[MT][2];
-#pragma unroll
-    for (int mt = 0; mt < MT; mt++) {
-        sc[mt][0] = lds128(scales_s + (16 * mt + g) * 16);
-        sc[mt][1] = lds128(scales_s + (16 * mt + g + 8) * 16);
-    }
-    const uint8_t *lane_codes = codes_s + g * 128 + 4 * t;
     const __half *xp = xrow + k0 + 4 * t;
     if (nblk == 8) {
-        uint2 xa[8], xb[8];
 #pragma unroll
         for (int jb = 0; jb < 8; jb++) {
-            xa[jb] = ldg64(xp + 32 * jb);
-            xb[jb] = ldg64(xp + 32 * jb + 16);
-        }
-#pragma unroll
-        for (int jb = 0; jb < 8; jb++) {
-            float off[4];
-            block_offset<FMT>(xa[jb], xb[jb], off);
-#pragma unroll
-            for (int mt = 0; mt < MT; mt++) {
-                const uint32_t wg = pick_u32(sc[mt][0], jb >> 1), wg8 = pick_u32(sc[mt][1], jb >> 1);
-                const float dg = (jb & 1) ? half_hi(wg) : half_lo(wg);
-                const float dg8 = (jb & 1) ? half_hi(wg8) : half_lo(wg8);
-                block_mma<FMT>(lane_codes + mt * 2048, jb, sw[jb], xa[jb], xb[jb], off, dg, dg8,
-                               acc[mt]);
-            }
+            xa[jb] = ldg64<COHERENT>(xp + 32 * jb);
+            xb[jb] = ldg64<COHERENT>(xp + 32 * jb + 16);
         }
     } else {
 #pragma unroll
         for (int jb = 0; jb < 8; jb++) {
             if (jb < nblk) {
-                const uint2 xa = ldg64(xp + 32 * jb);
-                const uint2 xb = ldg64(xp + 32 * jb + 16);
-                float off[4];
-                block_offset<FMT>(xa, xb, off);
-#pragma unroll
-                for (int mt = 0; mt < MT; mt++) {
-                    const uint32_t wg = pick_u32(sc[mt][0], jb >> 1), wg8 = pick_u32(sc[mt][1], jb >> 1);
-                    const float dg = (jb & 1) ? half_hi(wg) : half_lo(wg);
-                    const float dg8 = (jb & 1) ? half_hi(wg8) : half_lo(wg8);
-                    block_mma<FMT>(lane_codes + mt * 2048, jb, sw[jb], xa, xb, off, dg, dg8, acc[mt]);
-                }
+                xa[jb] = ldg64<COHERENT>(xp + 32 * jb);
+                xb[jb] = ldg64<COHERENT>(xp + 32 * jb + 16);
+            } else {
+                xa[jb] = xb[jb] = make_uint2(0u, 0u);
             }
         }
+    }
+}
+
+// A whole chunk: 8 blocks (nblk of them valid) for the chunk's kMT m-tiles,
+// with the x fragments already loaded.  codes_s / scales_s are the slot's
+// shared addresses, laundered through the slot's mbarrier wait.
+template <int FMT>
+__device__ __forceinline__ void chunk_mma(uint32_t codes_s, uint32_t scales_s, int nblk, int g,
+                                          int t, const int (&sw)[8], const uint2 (&xa)[8],
+                                          const uint2 (&xb)[8], float (&acc)[Fmt<FMT>::kMT][4])
+{
+    constexpr int MT = Fmt<FMT>::kMT;
+    uint4 sc[MT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; mt++) {
+        sc[mt][0] = lds128_u32(scales_s + (16 * mt + g) * 16);
+        sc[mt][1] = lds128_u32(scales_s + (16 * mt + g + 8) * 16);
+    }
+    const uint32_t lane_codes = codes_s + g * 128 + 4 * t;
+    auto one_block = [&](int jb) {
+        float off[4];
+        block_offset<FMT>(xa[jb], xb[jb], off);
+#pragma unroll
+        for (int mt = 0; mt < MT; mt++) {
+            float d0, d1, e0, e1;
+            halves_to_float(pick_u32(sc[mt][0], jb >> 1), d0, d1);
+            halves_to_float(pick_u32(sc[mt][1], jb >> 1), e0, e1);
+            const float dg = (jb & 1) ? d1 : d0;
+            const float dg8 = (jb & 1) ? e1 : e0;
+            if constexpr (FMT == 4) {
+                block_q4(lane_codes + mt * 2048 + sw[jb], xa[jb], xb[jb], off, dg, dg8, acc[mt]);
+            } else {
+                const uint32_t base = lane_codes + (jb >> 2) * 2048;
+                block_q8(base + (sw[jb] & 0xffff), base + (sw[jb] >> 16), xa[jb], xb[jb], off, dg,
+                         dg8, acc[mt]);
+            }
+        }
+    };
+    if (nblk == 8) {
+#pragma unroll
+        for (int jb = 0; jb < 8; jb++)
+            one_block(jb);
+    } else {
+#pragma unroll
+        for (int jb = 0; jb < 8; jb++)
+            if (jb < nblk)
+                one_block(jb);
     }
 }
 

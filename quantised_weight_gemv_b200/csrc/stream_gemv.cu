@@ -69,6 +69,17 @@ struct alignas(64) MatDesc {
     int band_base;       // first arrival counter of this matrix within its stage
 };
 
+// The per-matrix fields the worker loop reads (everything but the tensor
+// maps), cached in shared memory so cursor moves, band changes and flushes
+// never wait on global memory.
+struct MatInfo {
+    const __half *x;
+    float *y;
+    int N, K, B, cpb, nbands, chunk_base, band_base, pad;
+};
+
+constexpr int kMaxPlanMats = 256;   // plan size limit (shared-memory cache)
+
 struct StageDesc {
     int mat_begin, mat_end;
     int T;               // chunks in the stage
@@ -89,12 +100,12 @@ struct KernelArgs {
     const MatDesc *mats;             // plan mode (device memory)
     const StageDesc *stages;
     int n_stages;
+    int n_mats;
     int wmax;                        // gridDim.x * kWarps
     int *counters;                   // per band of a stage; zero on entry and exit
     float *partials;                 // [wmax][2][kMT][32 lanes] float4
     int *status;                     // device status word or null
-    unsigned *sync;                  // plan mode: [0] arrivals, [32] stage flag, [64] exits
-                                     // (separate 128-byte lines)
+    unsigned *sync;                  // plan mode: [0] arrivals, [64] exits (separate lines)
     // routed experts
     int E, topk, x_per_slot;
     const int *idx;
@@ -184,6 +195,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     extern __shared__ uint8_t smem_raw[];
     __shared__ ExpertGroups grp;
     __shared__ int cta_arrivals;
+    __shared__ int local_ctr[kWarps];   // arrivals of CTA-local split bands
     __shared__ alignas(8) uint64_t stage_bar;
 
     uint8_t *sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -192,15 +204,41 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     uint8_t *codes_ring = sbase + warp * D * CB;
     uint8_t *scales_ring = sbase + kWarps * D * CB + warp * D * SB;
     const uint32_t bars = smem_u32(sbase + kWarps * D * (CB + SB) + warp * D * 8);
-
-    const MatDesc *mats = PLAN ? a.mats : &a.mat0;
-    const StageDesc *stg = PLAN ? a.stages : &a.stage0;
+    // Per-warp partial sums of CTA-local split bands: [warp][slot][mt][lane].
+    float4 *local_part = reinterpret_cast<float4 *>(sbase + kWarps * D * (CB + SB) + kWarps * D * 8);
+    // Descriptor cache: stage table then matrix info (one entry each outside
+    // plan mode).
+    StageDesc *stg = reinterpret_cast<StageDesc *>(local_part + kWarps * 2 * MT * 32);
     const int n_stages = PLAN ? a.n_stages : 1;
+    MatInfo *minfo = reinterpret_cast<MatInfo *>(stg + n_stages);
+    const MatDesc *mats = PLAN ? a.mats : &a.mat0;   // tensor maps stay in global / param space
+    {
+        const int n_m = PLAN ? a.n_mats : 1;
+        for (int i = threadIdx.x; i < n_stages; i += kThreads)
+            stg[i] = PLAN ? a.stages[i] : a.stage0;
+        for (int i = threadIdx.x; i < n_m; i += kThreads) {
+            const MatDesc &m = mats[i];
+            MatInfo mi;
+            mi.x = m.x;
+            mi.y = m.y;
+            mi.N = m.N;
+            mi.K = m.K;
+            mi.B = m.B;
+            mi.cpb = m.cpb;
+            mi.nbands = m.nbands;
+            mi.chunk_base = m.chunk_base;
+            mi.band_base = m.band_base;
+            mi.pad = 0;
+            minfo[i] = mi;
+        }
+    }
 
     if (lane == 0) {
         for (int s = 0; s < D; s++)
             mbar_init(bars + 8 * s, 1);
     }
+    if (threadIdx.x < kWarps)
+        local_ctr[threadIdx.x] = 0;
     if (PLAN && threadIdx.x == 0) {
         cta_arrivals = 0;
         mbar_init(smem_u32(&stage_bar), 1);
@@ -213,7 +251,6 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     // waits for the previous kernel on the stream to complete.
     pdl_wait();
 
-    StageDesc moe_stage;
     if constexpr (MOE) {
         if (warp == 0)
             group_experts(a, grp);
@@ -229,30 +266,36 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                     a.mat0.y[(size_t)i * a.mat0.N + r] = 0.f;
             }
         }
-        moe_stage = a.stage0;
-        moe_stage.nbands = grp.npieces * a.mat0.nbands;
-        moe_stage.T = moe_stage.nbands * a.mat0.cpb;
-        moe_stage.cpw = (moe_stage.T + a.wmax - 1) / a.wmax;
-        if (moe_stage.cpw < 1)
-            moe_stage.cpw = 1;
-        moe_stage.W = (moe_stage.T + moe_stage.cpw - 1) / moe_stage.cpw;
-        stg = &moe_stage;
+        if (threadIdx.x == 0) {
+            StageDesc st = a.stage0;
+            st.nbands = grp.npieces * a.mat0.nbands;
+            st.T = st.nbands * a.mat0.cpb;
+            st.cpw = (st.T + a.wmax - 1) / a.wmax;
+            if (st.cpw < 1)
+                st.cpw = 1;
+            st.W = (st.T + st.cpw - 1) / st.cpw;
+            stg[0] = st;
+        }
+        __syncthreads();
     } else {
         __syncthreads();
     }
 
-    const int w = warp * gridDim.x + blockIdx.x;
+    // Workers are numbered CTA-major, so a band split among consecutive
+    // workers usually lies within one CTA and is summed in shared memory.
+    const int w = blockIdx.x * kWarps + warp;
+    const int cta_first = blockIdx.x * kWarps;
     const uint64_t pol = policy_evict_first();
 
     // Per-unit geometry (matrix, or expert piece in MoE mode).  Only plan mode
     // indexes a descriptor array; the other modes have one descriptor.
-    auto unit_mat = [&](int u) -> const MatDesc & { return PLAN ? mats[u] : a.mat0; };
+    auto unit_mat = [&](int u) -> const MatInfo & { return minfo[PLAN ? u : 0]; };
     auto unit_cpb = [&](int u) { return unit_mat(u).cpb; };
     auto unit_chunk_base = [&](int u) {
-        return PLAN ? mats[u].chunk_base : (MOE ? u * a.mat0.nbands * a.mat0.cpb : 0);
+        return PLAN ? minfo[u].chunk_base : (MOE ? u * a.mat0.nbands * a.mat0.cpb : 0);
     };
     auto unit_band_base = [&](int u) {
-        return PLAN ? mats[u].band_base : (MOE ? u * a.mat0.nbands : 0);
+        return PLAN ? minfo[u].band_base : (MOE ? u * a.mat0.nbands : 0);
     };
 
     // Place a cursor at the first chunk of this worker's range in stage s, or
@@ -267,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             const int c1 = min(c0 + st.cpw, st.T);
             int u = MOE ? c0 / (a.mat0.nbands * a.mat0.cpb) : (PLAN ? st.mat_begin : 0);
             if (PLAN)
-                while (u + 1 < st.mat_end && mats[u + 1].chunk_base <= c0)
+                while (u + 1 < st.mat_end && minfo[u + 1].chunk_base <= c0)
                     u++;
             const int rel = c0 - unit_chunk_base(u);
             cu.s = s;
@@ -295,8 +338,8 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 cu.band = 0;
                 cu.u++;
                 if (PLAN) {
-                    cu.cpb = mats[cu.u].cpb;
-                    cu.nbands = mats[cu.u].nbands;
+                    cu.cpb = minfo[cu.u].cpb;
+                    cu.nbands = minfo[cu.u].nbands;
                 }
             }
         }
@@ -318,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 tma_load_3d(cdst, &a.mat0.tm_codes, bar, iss.kp * 128, row, e, pol);
                 tma_load_3d(sdst, &a.mat0.tm_scales, bar, iss.kp * 8, row, e, pol);
             } else {
-                const MatDesc &m = unit_mat(iss.u);
+                const MatDesc &m = mats[PLAN ? iss.u : 0];
 #pragma unroll
                 for (int bx = 0; bx < Fmt<FMT>::kBoxes; bx++)
                     tma_load_2d(cdst + bx * (ROWS * 128), &m.tm_codes, bar,
@@ -338,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     // Output of one band: acc[mt] holds (row 16mt+g, col 2t), (row 16mt+g,
     // col 2t+1), (row 16mt+g+8, col 2t), (row 16mt+g+8, col 2t+1).
     auto store_band = [&](int u, int band, const float (&v)[MT][4]) {
-        const MatDesc &m = unit_mat(u);
+        const MatInfo &m = unit_mat(u);
 #pragma unroll
         for (int mt = 0; mt < MT; mt++) {
 #pragma unroll
@@ -374,6 +417,48 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             return;
         }
         const int myslot = (c0 >= bs) ? 0 : 1;
+        const int wf = bs / st.cpw, wl = (be - 1) / st.cpw;
+        if (wf >= cta_first && wl < cta_first + kWarps) {
+            // Every worker of the band is a warp of this CTA: exchange the
+            // partials through shared memory.  Each worker stores its partial
+            // and bumps the band's shared counter (slot wf - cta_first, unique
+            // among the CTA's open bands) with CTA-scope release; the last to
+            // arrive acquires, adds the partials in worker order, stores y and
+            // resets the counter.  Nobody waits.
+#pragma unroll
+            for (int mt = 0; mt < MT; mt++)
+                local_part[((warp * 2 + myslot) * MT + mt) * 32 + lane] =
+                    make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]);
+            __syncwarp();
+            int lold = 0;
+            if (lane == 0)
+                asm volatile("atom.acq_rel.cta.shared::cta.add.s32 %0, [%1], 1;"
+                             : "=r"(lold) : "r"(smem_u32(&local_ctr[wf - cta_first])) : "memory");
+            lold = __shfl_sync(0xffffffffu, lold, 0);
+            if (lold != wl - wf)
+                return;
+            __syncwarp();
+            float s4[MT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; mt++)
+                s4[mt][0] = s4[mt][1] = s4[mt][2] = s4[mt][3] = 0.f;
+            for (int v = wf; v <= wl; v++) {
+                const int sl = (v * st.cpw >= bs) ? 0 : 1;
+#pragma unroll
+                for (int mt = 0; mt < MT; mt++) {
+                    const float4 p = local_part[(((v - cta_first) * 2 + sl) * MT + mt) * 32 + lane];
+                    s4[mt][0] += p.x;
+                    s4[mt][1] += p.y;
+                    s4[mt][2] += p.z;
+                    s4[mt][3] += p.w;
+                }
+            }
+            store_band(u, band, s4);
+            if (lane == 0)
+                local_ctr[wf - cta_first] = 0;
+            return;
+        }
+        // The band spans CTAs: partials through the workspace, counted arrivals.
 #pragma unroll
         for (int mt = 0; mt < MT; mt++)
             __stcg(part_at(w, myslot, mt), make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]));
@@ -381,7 +466,6 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
         // (__syncwarp orders them); the last arriver's acquire increment then
         // makes every partial visible to the whole warp (__syncwarp again).
         __syncwarp();
-        const int wf = bs / st.cpw, wl = (be - 1) / st.cpw;
         int *ctr = a.counters + unit_band_base(u) + band;
         int old = 0;
         if (lane == 0)
@@ -412,34 +496,31 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     };
 
     // Grid barrier between stages (plan mode; the launch is cooperative, so
-    // every CTA is resident).  The last warp of a CTA to finish stage s adds
-    // one arrival to the grid counter; the CTA whose arrival completes stage s
-    // publishes s+1 in a separate flag word, which every CTA's last warp polls
-    // (with back-off, so the pollers do not hammer the line the arrivals hit)
-    // before releasing its CTA's warps through a shared mbarrier.  Every wait
-    // is bounded.
+    // every CTA is resident).  Each warp's lane 0 arrives on a CTA counter
+    // with CTA-scope release; the CTA's last warp acquires it, adds one
+    // GPU-scope release arrival to the grid counter (a fire-and-forget
+    // reduction; release is cumulative, so it publishes every warp's y
+    // stores) and polls the counter (acquire, short back-off) until all CTAs
+    // have arrived, then releases its CTA's warps through a shared mbarrier.
+    // Every wait is bounded.
     bool ok = true;
     auto stage_arrive_and_wait = [&](int s) {
         __syncwarp();
         if (lane == 0) {
-            __threadfence();
-            const int old = atomicAdd(&cta_arrivals, 1);
+            int old;
+            asm volatile("atom.acq_rel.cta.shared::cta.add.s32 %0, [%1], 1;"
+                         : "=r"(old) : "r"(smem_u32(&cta_arrivals)) : "memory");
             if (old == kWarps * (s + 1) - 1) {
                 const unsigned target = gridDim.x * (unsigned)(s + 1);
-                if (atomicAdd(&a.sync[0], 1u) == target - 1) {
-                    __threadfence();
-                    atomicExch(&a.sync[32], (unsigned)(s + 1));
-                }
+                asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&a.sync[0]) : "memory");
                 const long long t0 = clock64();
-                unsigned ns = 32;
-                while (ld_acquire_gpu(&a.sync[32]) < (unsigned)(s + 1)) {
+                while (ld_acquire_gpu(&a.sync[0]) < target) {
                     if (clock64() - t0 > kWaitCycles) {
                         if (a.status)
                             atomicOr(a.status, kStatusTimeout);
                         break;
                     }
-                    __nanosleep(ns);
-                    ns = ns < 256 ? 2 * ns : 256;
+                    __nanosleep(32);
                 }
                 asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&stage_bar))
                              : "memory");
@@ -451,7 +532,6 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 atomicOr(a.status, kStatusTimeout);
             ok = false;
         }
-        __threadfence();
     };
 
     Cursor cur;
@@ -471,17 +551,6 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 break;
         }
         while (live && cur.s == s) {
-            if (iss_live && issued < done + D) {
-                __syncwarp();
-                issue_one();
-            }
-            const int slot = done % D;
-            if (!mbar_wait_bounded(bars + 8 * slot, (uint32_t)((done / D) & 1))) {
-                if (lane == 0 && a.status)
-                    atomicOr(a.status, kStatusTimeout);
-                ok = false;
-                break;
-            }
             if (cur.u != acc_u || cur.band != acc_band) {
                 if (acc_u >= 0)
                     flush(s, acc_u, acc_band, acc);
@@ -489,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 for (int mt = 0; mt < MT; mt++)
                     acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
                 if (cur.u != acc_u) {
-                    const MatDesc &m = unit_mat(cur.u);
+                    const MatInfo &m = unit_mat(cur.u);
                     nb32 = m.K / kBlock;
                     if constexpr (MOE) {
                         const int col = min(g, grp.piece_count[cur.u] - 1);
@@ -502,9 +571,28 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 acc_u = cur.u;
                 acc_band = cur.band;
             }
+            // x first (its latency then overlaps the TMA issue and the wait),
+            // then the load of a later chunk into the slot freed last round,
+            // then this chunk's weights.
             const int left = nb32 - cur.kp * 8;
-            chunk_mma<FMT>(codes_ring + slot * CB, scales_ring + slot * SB, xrow,
-                           cur.kp * kChunkK, left < 8 ? left : 8, g, t, sw, acc);
+            const int nblk = left < 8 ? left : 8;
+            uint2 xa[8], xb[8];
+            chunk_load_x<PLAN>(xrow, cur.kp * kChunkK, nblk, t, xa, xb);
+            if (iss_live && issued < done + D) {
+                __syncwarp();
+                issue_one();
+            }
+            const int slot = done % D;
+            if (!mbar_wait_bounded(bars + 8 * slot, (uint32_t)((done / D) & 1))) {
+                if (lane == 0 && a.status)
+                    atomicOr(a.status, kStatusTimeout);
+                ok = false;
+                break;
+            }
+            // Shared addresses of the slot, ordered after its wait (launder).
+            const uint32_t cs = launder(smem_u32(codes_ring + slot * CB));
+            const uint32_t ss = launder(smem_u32(scales_ring + slot * SB));
+            chunk_mma<FMT>(cs, ss, nblk, g, t, sw, xa, xb, acc);
             done++;
             advance(cur);
             live = cur.s < n_stages;
@@ -531,7 +619,6 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             const unsigned old = atomicAdd(&a.sync[64], 1u);
             if (old == gridDim.x - 1) {
                 a.sync[0] = 0;
-                a.sync[32] = 0;
                 a.sync[64] = 0;
                 __threadfence();
             }
@@ -562,6 +649,14 @@ __global__ void moe_combine_kernel(const float *slot_out, const int *idx, const 
 // ------------------------------------------------------------------ host ----
 namespace {
 
+// Dynamic shared memory of a launch: the rings plus the descriptor cache.
+template <int FMT>
+constexpr size_t launch_smem(int n_stages, int n_mats)
+{
+    return (size_t)smem_bytes<FMT>() + (size_t)kWarps * 2 * Fmt<FMT>::kMT * 32 * sizeof(float4) +
+           (size_t)n_stages * sizeof(StageDesc) + (size_t)n_mats * sizeof(MatInfo);
+}
+
 template <int FMT, int MODE>
 int32_t prepare_kernel()
 {
@@ -573,7 +668,9 @@ int32_t prepare_kernel()
         return BQ_OK;
     if (cudaFuncSetAttribute((const void *)stream_gemv_kernel<FMT, MODE>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem_bytes<FMT>()) != cudaSuccess)
+                             (int)launch_smem<FMT>(MODE == kModePlan ? kMaxPlanMats : 1,
+                                                   MODE == kModePlan ? kMaxPlanMats : 1)) !=
+        cudaSuccess)
         return BQ_ERR_CUDA;
     if (dev >= 0 && dev < 64)
         done[dev] = true;
@@ -671,8 +768,8 @@ int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void
     a.status = dev_status;
     void *args[] = {&a};
     cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<FMT, kModeMatrix>, dim3(G),
-                               dim3(kThreads), smem_bytes<FMT>(), static_cast<cudaStream_t>(stream),
-                               args);
+                               dim3(kThreads), launch_smem<FMT>(1, 1),
+                               static_cast<cudaStream_t>(stream), args);
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
@@ -689,6 +786,7 @@ int32_t step_run_impl(const bq_step_info *info, const void *plan, void *ws, int3
     a.stages = reinterpret_cast<const StageDesc *>(pb + info->stages_off);
     a.mats = reinterpret_cast<const MatDesc *>(pb + info->mats_off);
     a.n_stages = info->n_stages;
+    a.n_mats = info->n_mats;
     a.wmax = info->grid * kWarps;
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     a.sync = reinterpret_cast<unsigned *>(wsb);
@@ -699,7 +797,7 @@ int32_t step_run_impl(const bq_step_info *info, const void *plan, void *ws, int3
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info->grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem_bytes<FMT>();
+    cfg.dynamicSmemBytes = launch_smem<FMT>(info->n_stages, info->n_mats);
     cfg.stream = static_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
@@ -749,7 +847,7 @@ extern "C" int32_t bq_step_plan(int32_t fmt, const bq_step_mat *mats, int32_t n_
 {
     if (!mats || !plan || !info)
         return BQ_ERR_NULL;
-    if ((fmt != 4 && fmt != 8) || n_mats < 1)
+    if ((fmt != 4 && fmt != 8) || n_mats < 1 || n_mats > kMaxPlanMats)
         return BQ_ERR_SHAPE;
     if (plan_bytes < bq_step_plan_bytes(n_mats))
         return BQ_ERR_WORKSPACE;
@@ -775,8 +873,11 @@ extern "C" int32_t bq_step_plan(int32_t fmt, const bq_step_mat *mats, int32_t n_
     int occ = 0;
     const void *kfn = fmt == 4 ? (const void *)stream_gemv_kernel<4, kModePlan>
                                : (const void *)stream_gemv_kernel<8, kModePlan>;
+    // (n_stages <= n_mats, so sizing the cache for n_mats stages is an upper bound)
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &occ, kfn, kThreads, fmt == 4 ? smem_bytes<4>() : smem_bytes<8>()) != cudaSuccess ||
+            &occ, kfn, kThreads,
+            fmt == 4 ? launch_smem<4>(n_mats, n_mats) : launch_smem<8>(n_mats, n_mats)) !=
+            cudaSuccess ||
         occ < 1)
         return BQ_ERR_CUDA;
     const int sms = device_sm_count();
@@ -935,7 +1036,7 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
     void *args[] = {&a};
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<4, kModeMoE>, dim3(G),
-                               dim3(kThreads), smem_bytes<4>(), s, args);
+                               dim3(kThreads), launch_smem<4>(1, 1), s, args);
     if (e != cudaSuccess)
         return BQ_ERR_CUDA;
     if (route_w) {
@@ -1048,6 +1149,6 @@ extern "C" int32_t bq_gemv_q4_noalloc(const bq_qmat *W, const uint16_t *x, int32
         return BQ_ERR_CUDA;
     void *args[] = {&a};
     cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<4, kModeMatrix>, dim3(G),
-                               dim3(kThreads), smem_bytes<4>(), s, args);
+                               dim3(kThreads), launch_smem<4>(1, 1), s, args);
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }

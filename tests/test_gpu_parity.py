@@ -290,3 +290,48 @@ def test_step_barrier_orders_dependent_stages():
         assert np.array_equal(y0.cpu().numpy()[0], y0_expect)
         y_ref, absy = oracle.gemv_q4(codes1, scales1, x1_expect)
         check_tol(y1.cpu().numpy(), y_ref, absy)
+
+
+def test_step_reread_buffer_sees_later_writes():
+    """A buffer is read as x by stage 0, overwritten (as y) by stage 1 and read
+    again as x by stage 2, all in one launch: stage 2 must see stage 1's
+    values, not a stale copy cached while stage 0 read it."""
+    import torch
+    N1, K1 = 256, 64
+    r = np.random.default_rng(5)
+    q1 = r.integers(0, 16, size=(N1, K1))
+    codes1 = np.zeros((N1, K1 // 2), dtype=np.uint8)
+    for j in range(K1 // 32):
+        for i in range(16):
+            codes1[:, 16 * j + i] = q1[:, 32 * j + i] | (q1[:, 32 * j + i + 16] << 4)
+    scales1 = np.zeros((N1, 8), dtype=np.uint16)
+    scales1[:, :2] = 0x3C00
+    x1 = np.zeros((1, K1), dtype=np.float16)
+    x1[0, 5] = 1.0
+    y1_expect = (q1[:, 5] - 8).astype(np.float32)               # small integers
+    X = torch.full((1, N1), 0.5, dtype=torch.float32, device=DEV)  # shared buffer
+    K0 = 2 * N1                                                  # its fp16 view
+    before = np.full((1, N1), 0.5, dtype=np.float32).view(np.uint16).reshape(1, K0)
+    after = y1_expect.view(np.uint16).reshape(1, K0)
+    w0 = synth.weights_f32(synth.key(0, 85, 0, 0, synth.KIND_W), 1024, K0)
+    w2 = synth.weights_f32(synth.key(0, 85, 2, 0, synth.KIND_W), 2048, K0)
+    c0, s0 = oracle.quantize_q4(w0)
+    c2, s2 = oracle.quantize_q4(w2)
+    y0 = torch.empty((1, 1024), dtype=torch.float32, device=DEV)
+    y2 = torch.empty((1, 2048), dtype=torch.float32, device=DEV)
+    tc0, ts0, tc1, ts1, tc2, ts2 = dev(c0), dev(s0), dev(codes1), dev(scales1), dev(c2), dev(s2)
+    xt1 = dev(x1.view(np.uint16))
+    plan = bq.StepPlan(4, [(bq.qmat(tc0, ts0, 1024, K0), X.view(torch.int16), y0, 0),
+                           (bq.qmat(tc1, ts1, N1, K1), xt1, X, 1),
+                           (bq.qmat(tc2, ts2, 2048, K0), X.view(torch.int16), y2, 2)], DEV)
+    st = new_status()
+    for _ in range(3):
+        X.fill_(0.5)
+        plan.run(st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        r0, a0 = oracle.gemv_q4(c0, s0, before)
+        r2, a2 = oracle.gemv_q4(c2, s2, after)
+        check_tol(y0.cpu().numpy(), r0, a0)
+        assert np.array_equal(X.cpu().numpy()[0], y1_expect)
+        check_tol(y2.cpu().numpy(), r2, a2)
