@@ -38,6 +38,40 @@ METRIC = "weight-stream HBM GB/s (decode step, algorithmic bytes)"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "source": "fallback"}
 
 
+def kernel_source_hash() -> str:
+    """sha256 over the CUDA sources; a profile's traffic figure is only used
+    while the kernels are byte-identical to the profiled ones."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "quantised_weight_gemv_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload: str, engine: str):
+    """DRAM bytes per launch (read + write) from a committed ncu summary under
+    profiles/: a line `<!-- bench-traffic: workload=... engine=...
+    bytes_per_launch=... source_sha256=... -->`.  None when no summary
+    matches the current kernel sources."""
+    import glob
+    import re
+    cur = kernel_source_hash()
+    for p in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        with open(p) as f:
+            for line in f:
+                m = re.search(r"bench-traffic:(.*?)-->", line)
+                if not m:
+                    continue
+                kv = dict(t.split("=", 1) for t in m.group(1).split() if "=" in t)
+                if (kv.get("workload") == workload and kv.get("engine") == engine
+                        and kv.get("source_sha256") == cur):
+                    return int(float(kv["bytes_per_launch"]))
+    return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -57,6 +91,10 @@ for _f in (4, 8):
     for _b in (1, 2, 4, 8):
         _w = synth.dense_h4096(_f, _b)
         WORKLOADS[_w.name] = _w
+    for _n, _k in synth.SWEEP_SHAPES:
+        for _b in (1, 8):
+            _w = synth.sweep_workload(_f, _n, _k, _b)
+            WORKLOADS[_w.name] = _w
 
 
 def fused_stages(wl: synth.DenseWorkload):
@@ -172,7 +210,7 @@ class DenseStep:
                 y = torch.empty((self.B, Ntot), dtype=torch.float32, device=device)
                 label = "+".join(m.name for m in mats)
                 q = bq.qmat(codes, scales, Ntot, K)
-                self.launches.append((q, x, y, label, layer * len(stages) + s))
+                self.launches.append((q, x, y, label, wl.stage_of(layer, s)))
                 self._keep += [codes, scales]
                 nb = synth.packed_bytes(wl.fmt, Ntot, K) + self.B * K * 2 + self.B * Ntot * 4
                 self.bytes_alg += nb
@@ -186,7 +224,8 @@ class DenseStep:
         self.plan = None
 
     def build_plan(self):
-        """The whole step as one plan (stages in model order), built once."""
+        """The whole step as one plan (stages in model order), built once.
+        (A plan holds at most 256 matrices; larger sets use --engine graph.)"""
         self.plan = self.bq.StepPlan(self.fmt, [(q, x, y, st) for q, x, y, _, st in self.launches],
                                      self.device)
 
@@ -459,7 +498,8 @@ def main():
                                    else "CUDA events around each launch"),
                          "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                          "peak_source": peaks["source"], "unit": "GB/s",
-                         "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                         "frac": round(achieved / peaks["hbm_gbs"], 4),
+                         "traffic": profiled_traffic(wl.name, args.engine),
                          "bytes_per_launch": int(dom_bytes),
                          "launch_us": round(dom_s * 1e6, 3)},
             "cpu_baseline": cpu,

@@ -103,18 +103,16 @@ class DenseWorkload:
     layers: int
     mats: Tuple[Mat, ...]   # per-layer matrices, in model order
     B: int = 1
+    independent: bool = False   # layers are independent copies (one stage for all)
 
     def layer_weights(self) -> int:
         return sum(m.N * m.K for m in self.mats)
 
-    def step_mats(self) -> List[Tuple[int, Mat]]:
-        """(layer, matrix) for a whole decode step, stage by stage in model order."""
+    def stage_of(self, layer: int, stage: int) -> int:
+        """Global stage of a layer's stage: layers run one after another, unless
+        they are independent copies (then every layer shares the stages)."""
         n_st = 1 + max(m.stage for m in self.mats)
-        out = []
-        for l in range(self.layers):
-            for m in self.mats:
-                out.append((l, dataclasses.replace(m, stage=l * n_st + m.stage)))
-        return out
+        return stage if self.independent else layer * n_st + stage
 
 
 def packed_bytes(fmt: int, N: int, K: int) -> int:
@@ -157,6 +155,14 @@ DENSE_H5120 = DenseWorkload(5, "dense64L-h5120-ffn25600-q4", 4, 64, (
 # Matrix-shape sweep (N x K) for achieved bandwidth against matrix size.
 SWEEP_SHAPES = ((512, 512), (1024, 1024), (2048, 2048), (4096, 4096), (5120, 5120),
                 (1024, 5120), (8192, 5120), (25600, 5120), (5120, 25600))
+
+
+def sweep_workload(fmt: int, N: int, K: int, B: int = 1, min_bytes: int = 512 << 20) -> DenseWorkload:
+    """Independent copies of one N x K matrix, enough of them (>= min_bytes,
+    i.e. several times the L2) that no copy is served from L2."""
+    copies = max(2, -(-min_bytes // packed_bytes(fmt, N, K)))
+    return DenseWorkload(6, f"sweep-q{fmt}-{N}x{K}-b{B}", fmt, copies, (Mat("w", N, K, 0),), B,
+                         independent=True)
 
 
 @dataclasses.dataclass(frozen=True)
