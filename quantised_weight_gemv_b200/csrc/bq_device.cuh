@@ -192,15 +192,16 @@ __device__ __forceinline__ uint4 lds128(const uint8_t *p)
 
 // 8 bytes of x.  COHERENT = false: the read-only path, kept in L1 (every warp
 // of the SM re-reads the same activations for every band) -- valid when
-// nothing in the launch writes x.  COHERENT = true: cached in L2 only, so a
-// value another SM wrote earlier in the same launch (a previous stage's
-// output, after the grid barrier) is never read from a stale L1 line.
+// nothing in the launch writes x.  COHERENT = true: an ordinary (weak) load,
+// L1-cached, for x that an earlier stage of the same launch may have written:
+// it is issued after the grid barrier's GPU-scope acquire, which the memory
+// model requires to make those writes visible to it (no stale L1 line).
 template <bool COHERENT>
 __device__ __forceinline__ uint2 ldg64(const void *p)
 {
     uint2 v;
     if constexpr (COHERENT)
-        asm volatile("ld.global.cg.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+        asm volatile("ld.global.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p) : "memory");
     else
         asm("ld.global.nc.L1::evict_last.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
     return v;

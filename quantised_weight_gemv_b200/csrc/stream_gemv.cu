@@ -348,6 +348,23 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     Cursor iss;
     bool iss_live = seek(iss, 0);
     int issued = 0;
+    // Plan mode: the TMA unit must fetch a matrix's tensor maps from global
+    // memory before its first load; prefetch them one load ahead of the issue
+    // cursor so no load waits for a descriptor.
+    int prefetched_u = -1;
+    auto prefetch_maps = [&](int u) {
+        if constexpr (PLAN) {
+            if (lane == 0 && u > prefetched_u && u < a.n_mats) {
+                prefetch_tensormap(&mats[u].tm_codes);
+                prefetch_tensormap(&mats[u].tm_scales);
+                prefetched_u = u;
+            }
+        }
+    };
+    if (iss_live) {
+        prefetch_maps(iss.u);
+        prefetch_maps(iss.u + 1);
+    }
     auto issue_one = [&]() {
         if (lane == 0) {
             const int slot = issued % D;
@@ -372,6 +389,8 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
         issued++;
         advance(iss);
         iss_live = iss.s < n_stages;
+        if (iss_live)
+            prefetch_maps(iss.u);   // the matrix of the next load this warp issues
     };
 
     // Fill the ring.
