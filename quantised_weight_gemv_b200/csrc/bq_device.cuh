@@ -20,11 +20,15 @@
 #include <stdint.h>
 #include <string.h>
 
+#ifndef BQ_WARPS
+#define BQ_WARPS 8          // worker warps per CTA
+#endif
+
 namespace bq {
 
 constexpr int kBlock = 32;          // weights per quantisation block
 constexpr int kChunkK = 256;        // weights along K per chunk
-constexpr int kWarps = 8;           // worker warps per CTA
+constexpr int kWarps = BQ_WARPS;    // worker warps per CTA
 constexpr int kThreads = kWarps * 32;
 
 // Status bits OR-ed into the caller's device status word (1 << bq_status).
@@ -44,9 +48,6 @@ constexpr long long kWaitCycles = 4000000000LL;
 #endif
 #ifndef BQ_MIN_BLOCKS
 #define BQ_MIN_BLOCKS 2     // CTAs per SM the register budget is sized for
-#endif
-#ifndef BQ_Q4_HI_INPLACE
-#define BQ_Q4_HI_INPLACE 0  // 1: high nibbles stay in place (x scaled by 1/16)
 #endif
 
 template <int FMT> struct Fmt;
@@ -177,19 +178,6 @@ __device__ __forceinline__ void pdl_wait()
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// Shared-memory reads through ordinary pointers: the compiler sees them as
-// loads, so it can schedule them freely between the mbarrier waits (whose asm
-// carries a memory clobber) but never across one.
-__device__ __forceinline__ uint32_t lds32(const uint8_t *p)
-{
-    return *reinterpret_cast<const uint32_t *>(p);
-}
-
-__device__ __forceinline__ uint4 lds128(const uint8_t *p)
-{
-    return *reinterpret_cast<const uint4 *>(p);
-}
-
 // 8 bytes of x.  COHERENT = false: the read-only path, kept in L1 (every warp
 // of the SM re-reads the same activations for every band) -- valid when
 // nothing in the launch writes x.  COHERENT = true: an ordinary (weak) load,
@@ -228,27 +216,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
     return d;
 }
 
-__device__ __forceinline__ uint32_t hsub2u(uint32_t a, uint32_t b)
-{
-    uint32_t d;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-__device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b)
-{
-    uint32_t d;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-__device__ __forceinline__ uint32_t hfma2u(uint32_t a, uint32_t b, uint32_t c)
-{
-    uint32_t d;
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-
 // D = A(16x16 f16) * B(16x8 f16) + C, fp32 accumulators.
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1, const float (&c)[4])
@@ -270,46 +237,11 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 //
 // Codes enter the tensor core as fp16 *subnormals*: a 16-bit lane holding the
 // integer u (< 1024) in its low bits and zero elsewhere is exactly u * 2^-24,
-// so masking the code bits into place is the whole conversion.  The format's
-// zero point z (8 for Q4, 128 for the Q8 code biased by +128) is removed by a
-// second mma that starts each block's accumulator at -z * 2^-24 * sum(x)
-// (see block_mma).  Every product is exact; the 2^-24 is undone at the store.
-struct Q4Pairs {
-    uint32_t lo01, lo23, hi01, hi23;   // f16x2 of q * 2^-24, q in [0, 15]
-};
-
-__device__ __forceinline__ Q4Pairs dequant_q4(uint32_t w)
-{
-    // bytes b0..b3 of w hold elements e..e+3 (low nibbles) and e+16..e+19
-    // (high nibbles)
-    const uint32_t p01 = prmt(w, 0u, 0x4140u);    // [b0, 0, b1, 0]
-    const uint32_t p23 = prmt(w, 0u, 0x4342u);    // [b2, 0, b3, 0]
-    Q4Pairs r;
-    r.lo01 = p01 & 0x000F000Fu;
-    r.lo23 = p23 & 0x000F000Fu;
-#if BQ_Q4_HI_INPLACE
-    r.hi01 = p01 & 0x00F000F0u;       // 16 q * 2^-24: paired with x / 16
-    r.hi23 = p23 & 0x00F000F0u;
-#else
-    r.hi01 = (p01 >> 4) & 0x000F000Fu;
-    r.hi23 = (p23 >> 4) & 0x000F000Fu;
-#endif
-    return r;
-}
-
-// Q8: int8 q -> byte u = q ^ 0x80 = q + 128 in [0, 255], as u * 2^-24.
-struct Q8Pairs {
-    uint32_t p01, p23;                 // f16x2 of (q + 128) * 2^-24
-};
-
-__device__ __forceinline__ Q8Pairs dequant_q8(uint32_t w)
-{
-    const uint32_t u = w ^ 0x80808080u;
-    Q8Pairs r;
-    r.p01 = prmt(u, 0u, 0x4140u);
-    r.p23 = prmt(u, 0u, 0x4342u);
-    return r;
-}
+// so masking the code bits into place is the whole conversion (Q4: the two
+// nibbles of a byte, Q8: the byte biased by +128).  The format's zero point z
+// (8 for Q4, 128 for the biased Q8 code) is removed by a second mma that
+// starts each block's accumulator at -z * 2^-24 * sum(x) (block_offset).
+// Every product is exact; the 2^-24 is undone at the store.
 
 // f16x2 of -z * 2^-24 (a subnormal): z = 8 -> 2^-21, z = 128 -> 2^-17.
 template <int FMT>

@@ -11,12 +11,10 @@
 namespace bq {
 
 // Upper bound on CTAs of one streamed launch (2 per SM on up to 256 SMs); it
-// sizes the per-worker partial-sum area of the workspace.
+// sizes the cross-CTA partial-sum area of the workspace.
 constexpr int kMaxCtas = 512;
-constexpr int kMaxWorkers = kMaxCtas * 8;
-// (3 CTAs per SM on up to 170 SMs, or 2 on up to 256, stay within kMaxCtas.)
-// Two partial slots of up to 64 rows x 8 columns fp32 per worker.
-constexpr size_t kPartialBytesPerWorker = 2 * 512 * sizeof(float);
+// Two partial slots of up to 64 rows x 8 columns fp32 per CTA.
+constexpr size_t kPartialBytesPerCta = 2 * 512 * sizeof(float);
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -10,19 +10,22 @@
 //
 // Work decomposition (stream-K over chunks).  A matrix is cut into bands of
 // kRows rows (32 for Q4, 16 for Q8) and a band into chunks of 256 weights
-// along K; chunks are numbered band-major.  Every warp of the grid is an independent worker that owns a
-// ring of shared-memory slots with its own mbarriers; its lane 0 keeps
-// `stages - 1` chunks of TMA loads in flight ahead of the chunk the warp is
-// computing.  Worker w takes chunks [w*cpw, (w+1)*cpw) of a stage, where cpw =
-// ceil(chunks / workers), so every SM streams the same number of bytes
-// whatever the matrix shapes.
+// along K; chunks are numbered band-major.  Every warp of the grid is an
+// independent worker that owns a ring of shared-memory slots with its own
+// mbarriers; its lane 0 keeps TMA loads of the warp's next chunks in flight
+// in every slot but the one being read (in a decode step, in every slot: a
+// slot is refilled as soon as the warp has read it).  Worker w takes chunks
+// [w*cpw, (w+1)*cpw) of a stage, where cpw = ceil(chunks / workers), so every
+// SM streams the same number of bytes whatever the matrix shapes.
 //
 // A band wholly inside one worker's range is written straight to y.  A band
-// cut by range boundaries is summed deterministically: each worker that
-// touched it stores its fp32 partial (kRows rows x 8 columns) in the workspace
-// and bumps the band's arrival counter; the last to arrive adds the partials
-// in worker order, writes y and resets the counter.  No worker waits for
-// another.
+// cut by range boundaries is summed deterministically in two levels: the
+// workers of one CTA that touched it combine their fp32 partials (kRows rows x
+// 8 columns) in shared memory, the last of them to arrive adding them in
+// worker order; if the band continues in other CTAs, that CTA partial goes to
+// the workspace with a counted arrival, and the last CTA to arrive adds the
+// CTA partials in CTA order, writes y and resets the counter.  No worker waits
+// for another.
 //
 // Three modes share that worker loop:
 //  - one matrix (bq_gemv_q4 / _q8): its descriptor is a kernel parameter;
@@ -393,8 +396,10 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             prefetch_maps(iss.u);   // the matrix of the next load this warp issues
     };
 
-    // Fill the ring.
-    while (iss_live && issued < D - 1)
+    // Fill the ring.  Plan mode keeps every slot loading (see the refill
+    // below); the other modes run one slot behind, refilling a slot at the
+    // top of the next chunk, after that chunk's x loads are in flight.
+    while (iss_live && issued < (PLAN ? D : D - 1))
         issue_one();
 
     // Output of one band: acc[mt] holds (row 16mt+g, col 2t), (row 16mt+g,
@@ -422,28 +427,34 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
         }
     };
 
-    // Partials: [worker][slot 0/1][mt][lane] float4.
-    auto part_at = [&](int v, int sl, int mt) {
-        return reinterpret_cast<float4 *>(a.partials) + (((size_t)v * 2 + sl) * MT + mt) * 32 + lane;
+    // Cross-CTA partials: [CTA][slot 0/1][mt][lane] float4.  A CTA has at
+    // most two bands that continue into other CTAs in a stage: the one holding
+    // its first chunk (slot 0) and the one holding its last (slot 1).
+    auto part_at = [&](int c, int sl, int mt) {
+        return reinterpret_cast<float4 *>(a.partials) + (((size_t)c * 2 + sl) * MT + mt) * 32 + lane;
     };
-    auto flush = [&](int s, int u, int band, const float (&acc)[MT][4]) {
+    // Writes the band's finished sum to y when this worker is the last to
+    // contribute; `acc` (this worker's partial) is used as scratch.
+    auto flush = [&](int s, int u, int band, float (&acc)[MT][4]) {
         const StageDesc &st = stg[s];
+        const int cpw = st.cpw;
         const int cpb = unit_cpb(u);
         const int bs = unit_chunk_base(u) + band * cpb, be = bs + cpb;
-        const int c0 = w * st.cpw, c1 = min(c0 + st.cpw, st.T);
+        const int c0 = w * cpw, c1 = min(c0 + cpw, st.T);
         if (bs >= c0 && be <= c1) {
             store_band(u, band, acc);
             return;
         }
-        const int myslot = (c0 >= bs) ? 0 : 1;
-        const int wf = bs / st.cpw, wl = (be - 1) / st.cpw;
-        if (wf >= cta_first && wl < cta_first + kWarps) {
-            // Every worker of the band is a warp of this CTA: exchange the
-            // partials through shared memory.  Each worker stores its partial
-            // and bumps the band's shared counter (slot wf - cta_first, unique
-            // among the CTA's open bands) with CTA-scope release; the last to
-            // arrive acquires, adds the partials in worker order, stores y and
-            // resets the counter.  Nobody waits.
+        // Workers wf..wl share the band; lf..ll of them are warps of this CTA.
+        const int wf = bs / cpw, wl = (be - 1) / cpw;
+        const int lf = max(wf, cta_first), ll = min(wl, cta_first + kWarps - 1);
+        if (ll > lf) {
+            // Level 1, in shared memory: each of the CTA's workers stores its
+            // partial and bumps the band's CTA counter (slot lf - cta_first,
+            // unique among the CTA's open bands) with CTA-scope release; the
+            // last to arrive acquires and adds the partials in worker order.
+            // Nobody waits.
+            const int myslot = (c0 >= bs) ? 0 : 1;
 #pragma unroll
             for (int mt = 0; mt < MT; mt++)
                 local_part[((warp * 2 + myslot) * MT + mt) * 32 + lane] =
@@ -452,35 +463,40 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             int lold = 0;
             if (lane == 0)
                 asm volatile("atom.acq_rel.cta.shared::cta.add.s32 %0, [%1], 1;"
-                             : "=r"(lold) : "r"(smem_u32(&local_ctr[wf - cta_first])) : "memory");
+                             : "=r"(lold) : "r"(smem_u32(&local_ctr[lf - cta_first])) : "memory");
             lold = __shfl_sync(0xffffffffu, lold, 0);
-            if (lold != wl - wf)
+            if (lold != ll - lf)
                 return;
             __syncwarp();
-            float s4[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; mt++)
-                s4[mt][0] = s4[mt][1] = s4[mt][2] = s4[mt][3] = 0.f;
-            for (int v = wf; v <= wl; v++) {
-                const int sl = (v * st.cpw >= bs) ? 0 : 1;
+                acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+            for (int v = lf; v <= ll; v++) {
+                const int sl = (v * cpw >= bs) ? 0 : 1;
 #pragma unroll
                 for (int mt = 0; mt < MT; mt++) {
                     const float4 p = local_part[(((v - cta_first) * 2 + sl) * MT + mt) * 32 + lane];
-                    s4[mt][0] += p.x;
-                    s4[mt][1] += p.y;
-                    s4[mt][2] += p.z;
-                    s4[mt][3] += p.w;
+                    acc[mt][0] += p.x;
+                    acc[mt][1] += p.y;
+                    acc[mt][2] += p.z;
+                    acc[mt][3] += p.w;
                 }
             }
-            store_band(u, band, s4);
             if (lane == 0)
-                local_ctr[wf - cta_first] = 0;
+                local_ctr[lf - cta_first] = 0;
+        }
+        if (wf >= cta_first && wl < cta_first + kWarps) {
+            store_band(u, band, acc);
             return;
         }
-        // The band spans CTAs: partials through the workspace, counted arrivals.
+        // Level 2, the band continues in other CTAs: one partial per CTA
+        // through the workspace and a counted arrival; the last CTA to arrive
+        // adds the partials in CTA order, stores y and resets the counter.
+        const int cf = wf / kWarps, cl = wl / kWarps;
+        const int cslot = (bs <= cta_first * cpw) ? 0 : 1;
 #pragma unroll
         for (int mt = 0; mt < MT; mt++)
-            __stcg(part_at(w, myslot, mt), make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]));
+            __stcg(part_at(blockIdx.x, cslot, mt), make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]));
         // The warp's partial stores happen before lane 0's release increment
         // (__syncwarp orders them); the last arriver's acquire increment then
         // makes every partial visible to the whole warp (__syncwarp again).
@@ -490,26 +506,41 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
         if (lane == 0)
             old = atom_add_acq_rel_gpu(ctr, 1);
         old = __shfl_sync(0xffffffffu, old, 0);
-        if (old != wl - wf)
+        if (old != cl - cf)
             return;
         __syncwarp();
-        float s4[MT][4];
 #pragma unroll
         for (int mt = 0; mt < MT; mt++)
-            s4[mt][0] = s4[mt][1] = s4[mt][2] = s4[mt][3] = 0.f;
-        for (int v = wf; v <= wl; v++) {
-            const int sl = (v * st.cpw >= bs) ? 0 : 1;
+            acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+        // Two CTAs' partials in flight at a time.
+        for (int v = cf; v <= cl; v += 2) {
+            const int v1 = min(v + 1, cl);
+            const int sl0 = (bs <= v * kWarps * cpw) ? 0 : 1;
+            const int sl1 = (bs <= v1 * kWarps * cpw) ? 0 : 1;
+            float4 p0[MT], p1[MT];
 #pragma unroll
             for (int mt = 0; mt < MT; mt++) {
-                const float4 p = (v == w) ? make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3])
-                                          : __ldcg(part_at(v, sl, mt));
-                s4[mt][0] += p.x;
-                s4[mt][1] += p.y;
-                s4[mt][2] += p.z;
-                s4[mt][3] += p.w;
+                p0[mt] = __ldcg(part_at(v, sl0, mt));
+                p1[mt] = __ldcg(part_at(v1, sl1, mt));
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; mt++) {
+                acc[mt][0] += p0[mt].x;
+                acc[mt][1] += p0[mt].y;
+                acc[mt][2] += p0[mt].z;
+                acc[mt][3] += p0[mt].w;
+            }
+            if (v1 > v) {
+#pragma unroll
+                for (int mt = 0; mt < MT; mt++) {
+                    acc[mt][0] += p1[mt].x;
+                    acc[mt][1] += p1[mt].y;
+                    acc[mt][2] += p1[mt].z;
+                    acc[mt][3] += p1[mt].w;
+                }
             }
         }
-        store_band(u, band, s4);
+        store_band(u, band, acc);
         if (lane == 0)
             *ctr = 0;
     };
@@ -591,13 +622,13 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 acc_band = cur.band;
             }
             // x first (its latency then overlaps the TMA issue and the wait),
-            // then the load of a later chunk into the slot freed last round,
-            // then this chunk's weights.
+            // then (outside plan mode) the load of a later chunk into the slot
+            // freed last round, then this chunk's weights.
             const int left = nb32 - cur.kp * 8;
             const int nblk = left < 8 ? left : 8;
             uint2 xa[8], xb[8];
             chunk_load_x<PLAN>(xrow, cur.kp * kChunkK, nblk, t, xa, xb);
-            if (iss_live && issued < done + D) {
+            if (!PLAN && iss_live && issued < done + D) {
                 __syncwarp();
                 issue_one();
             }
@@ -613,6 +644,14 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             const uint32_t ss = launder(smem_u32(scales_ring + slot * SB));
             chunk_mma<FMT>(cs, ss, nblk, g, t, sw, xa, xb, acc);
             done++;
+            // Plan mode: refill the slot just read at once, before any flush
+            // or stage barrier, so the ring always holds the warp's next D
+            // chunks -- across stage boundaries too.  (The __syncwarp orders
+            // every lane's reads of the slot before lane 0 issues the copy.)
+            if (PLAN && iss_live) {
+                __syncwarp();
+                issue_one();
+            }
             advance(cur);
             live = cur.s < n_stages;
         }
@@ -706,7 +745,7 @@ int max_ctas()
 }
 
 size_t counters_bytes(long long n) { return align_up((size_t)n * sizeof(int), 256); }
-constexpr size_t kPartialsBytes = (size_t)kMaxWorkers * kPartialBytesPerWorker;
+constexpr size_t kPartialsBytes = (size_t)kMaxCtas * kPartialBytesPerCta;
 constexpr size_t kSyncBytes = 512;
 
 int rows_of(int fmt) { return fmt == 4 ? Fmt<4>::kRows : Fmt<8>::kRows; }
@@ -1081,11 +1120,11 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
 // kNoAllocScratchBytes reserved until the process exits.
 namespace bq {
 namespace {
-constexpr int kNoAllocMaxCtas = 320;                     // 2560 worker warps at most
+constexpr int kNoAllocMaxCtas = 320;                     // CTAs of one launch at most
 constexpr long long kNoAllocMaxRows = 1LL << 20;         // N limit of this entry point
 constexpr size_t kNoAllocCounterBytes = (size_t)(kNoAllocMaxRows / 16) * sizeof(int);
 constexpr size_t kNoAllocPartialBytes =
-    (size_t)kNoAllocMaxCtas * kWarps * 2 * Fmt<4>::kMT * 32 * sizeof(float4);
+    (size_t)kNoAllocMaxCtas * 2 * Fmt<4>::kMT * 32 * sizeof(float4);
 constexpr size_t kNoAllocScratchBytes = kNoAllocCounterBytes + kNoAllocPartialBytes;
 }  // namespace
 }  // namespace bq
