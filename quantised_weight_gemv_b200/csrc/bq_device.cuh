@@ -399,15 +399,14 @@ __device__ __forceinline__ void lane_swizzle(int g, int (&sw)[8])
 }
 
 // The x fragments of a chunk: for block jb, xa = x[k..k+3] and xb =
-// x[k+16..k+19] with k = k0 + 32 jb + 4t, for batch column g.  xrow points at
-// x[column g][0]; a lane whose column is absent (g >= B) reads a valid row
-// instead -- its mma column is garbage and is never stored, which keeps
+// x[k+16..k+19] with k = k0 + 32 jb + 4t, for batch column g.  `xp` points at
+// x[column g][k0 + 4t]; a lane whose column is absent (g >= B) reads a valid
+// row instead -- its mma column is garbage and is never stored, which keeps
 // every load unconditional.  Only the nblk valid blocks are read.
 template <bool COHERENT>
-__device__ __forceinline__ void chunk_load_x(const __half *xrow, int k0, int nblk, int t,
-                                             uint2 (&xa)[8], uint2 (&xb)[8])
+__device__ __forceinline__ void chunk_load_x(const __half *xp, int nblk, uint2 (&xa)[8],
+                                             uint2 (&xb)[8])
 {
-    const __half *xp = xrow + k0 + 4 * t;
     if (nblk == 8) {
 #pragma unroll
         for (int jb = 0; jb < 8; jb++) {

@@ -348,8 +348,13 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
         }
     };
 
+    // Chunks left in the cursor's current run: consecutive chunks of one
+    // band inside the worker's range.
+    auto run_left = [&](const Cursor &cu) { return min(cu.cpb - cu.kp, cu.c_end - cu.c); };
+
     Cursor iss;
     bool iss_live = seek(iss, 0);
+    int iss_left = iss_live ? run_left(iss) : 0;
     int issued = 0;
     // Plan mode: the TMA unit must fetch a matrix's tensor maps from global
     // memory before its first load; prefetch them one load ahead of the issue
@@ -390,10 +395,17 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             }
         }
         issued++;
+        if (--iss_left > 0) {   // next chunk of the same run
+            iss.kp++;
+            iss.c++;
+            return;
+        }
         advance(iss);
         iss_live = iss.s < n_stages;
-        if (iss_live)
+        if (iss_live) {
+            iss_left = run_left(iss);
             prefetch_maps(iss.u);   // the matrix of the next load this warp issues
+        }
     };
 
     // Fill the ring.  Plan mode keeps every slot loading (see the refill
@@ -621,37 +633,57 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 acc_u = cur.u;
                 acc_band = cur.band;
             }
-            // x first (its latency then overlaps the TMA issue and the wait),
-            // then (outside plan mode) the load of a later chunk into the slot
-            // freed last round, then this chunk's weights.
-            const int left = nb32 - cur.kp * 8;
-            const int nblk = left < 8 ? left : 8;
-            uint2 xa[8], xb[8];
-            chunk_load_x<PLAN>(xrow, cur.kp * kChunkK, nblk, t, xa, xb);
-            if (!PLAN && iss_live && issued < done + D) {
-                __syncwarp();
-                issue_one();
-            }
-            const int slot = done % D;
-            if (!mbar_wait_bounded(bars + 8 * slot, (uint32_t)((done / D) & 1))) {
-                if (lane == 0 && a.status)
-                    atomicOr(a.status, kStatusTimeout);
-                ok = false;
+            // One chunk of the run: x first (its latency then overlaps the
+            // TMA issue and the wait), then (outside plan mode) the load of a
+            // later chunk into the slot freed last round, then this chunk's
+            // weights.  Called with a literal nblk of 8 for full chunks, so
+            // their code has no per-block bounds.
+            auto one_chunk = [&](const __half *xp, int nblk) -> bool {
+                uint2 xa[8], xb[8];
+                chunk_load_x<PLAN>(xp, nblk, xa, xb);
+                if (!PLAN && iss_live && issued < done + D) {
+                    __syncwarp();
+                    issue_one();
+                }
+                const int slot = done % D;
+                if (!mbar_wait_bounded(bars + 8 * slot, (uint32_t)((done / D) & 1))) {
+                    if (lane == 0 && a.status)
+                        atomicOr(a.status, kStatusTimeout);
+                    return false;
+                }
+                // Shared addresses of the slot, ordered after its wait (launder).
+                const uint32_t cs = launder(smem_u32(codes_ring + slot * CB));
+                const uint32_t ss = launder(smem_u32(scales_ring + slot * SB));
+                chunk_mma<FMT>(cs, ss, nblk, g, t, sw, xa, xb, acc);
+                done++;
+                // Plan mode: refill the slot just read at once, before any
+                // flush or stage barrier, so the ring always holds the warp's
+                // next D chunks -- across stage boundaries too.  (The
+                // __syncwarp orders every lane's reads of the slot before lane
+                // 0 issues the copy.)
+                if (PLAN && iss_live) {
+                    __syncwarp();
+                    issue_one();
+                }
+                return true;
+            };
+            // The run: consecutive chunks of this band inside the worker's
+            // range; only the band's last chunk can be partial (K not a
+            // multiple of 256).
+            const int run = run_left(cur);
+            const int tail = nb32 - (cur.cpb - 1) * 8;   // blocks in the band's last chunk
+            const int nfull = (cur.kp + run == cur.cpb && tail < 8) ? run - 1 : run;
+            const __half *xp = xrow + cur.kp * kChunkK + 4 * t;
+            for (int i = 0; i < nfull && ok; i++, xp += kChunkK)
+                ok = one_chunk(xp, 8);
+            if (ok && nfull < run)
+                ok = one_chunk(xp, tail);
+            if (!ok)
                 break;
-            }
-            // Shared addresses of the slot, ordered after its wait (launder).
-            const uint32_t cs = launder(smem_u32(codes_ring + slot * CB));
-            const uint32_t ss = launder(smem_u32(scales_ring + slot * SB));
-            chunk_mma<FMT>(cs, ss, nblk, g, t, sw, xa, xb, acc);
-            done++;
-            // Plan mode: refill the slot just read at once, before any flush
-            // or stage barrier, so the ring always holds the warp's next D
-            // chunks -- across stage boundaries too.  (The __syncwarp orders
-            // every lane's reads of the slot before lane 0 issues the copy.)
-            if (PLAN && iss_live) {
-                __syncwarp();
-                issue_one();
-            }
+            // Step the cursor past the run (its last step may change band,
+            // matrix or stage).
+            cur.c += run - 1;
+            cur.kp += run - 1;
             advance(cur);
             live = cur.s < n_stages;
         }
