@@ -207,7 +207,7 @@ class DenseStep:
                     del w
                 x = synth.activations_f16_torch(synth.key(seed, wl.wid, layer, s, synth.KIND_X),
                                                 (self.B, K), device)
-                y = torch.empty((self.B, Ntot), dtype=torch.float32, device=device)
+                y = (self.B, Ntot)   # allocated below, in one buffer with every other y
                 label = "+".join(m.name for m in mats)
                 q = bq.qmat(codes, scales, Ntot, K)
                 self.launches.append((q, x, y, label, wl.stage_of(layer, s)))
@@ -216,6 +216,26 @@ class DenseStep:
                 self.bytes_alg += nb
                 self.bytes_by_label[label] = self.bytes_by_label.get(label, 0) + nb
                 ws_max = max(ws_max, bq.lib().bq_gemv_workspace_bytes(Ntot, K))
+        # Every x in one device buffer and every y in another (64-byte aligned
+        # slices), so a step's inputs and results each move in one copy.
+        def pack(shapes, dtype, fill=None):
+            esz = torch.empty((), dtype=dtype).element_size()
+            offs, n = [], 0
+            for shp in shapes:
+                offs.append(n)
+                cnt = shp[0] * shp[1]
+                n += -(-cnt * esz // 64) * 64 // esz
+            buf = torch.empty(n, dtype=dtype, device=device)
+            views = [buf[o:o + a * b].view(a, b) for o, (a, b) in zip(offs, shapes)]
+            return buf, views
+        self.x_all, xv = pack([e[1].shape for e in self.launches], torch.float16)
+        self.y_all, yv = pack([e[2] for e in self.launches], torch.float32)
+        self.y_all.zero_()
+        packed = []
+        for (q, x, _, label, stg), xd, yd in zip(self.launches, xv, yv):
+            xd.copy_(x)
+            packed.append((q, xd, yd, label, stg))
+        self.launches = packed
         torch.cuda.synchronize()
         if int(st.item()) != 0:
             raise RuntimeError(f"device quantiser status {int(st.item()):#x}")
@@ -251,7 +271,8 @@ class DenseStep:
         return n
 
     def io_tensors(self):
-        return [e[1] for e in self.launches], [e[2] for e in self.launches]
+        """The step's inputs (every x) and results (every y), each one buffer."""
+        return self.x_all, self.y_all
 
 
 # ---------------------------------------------------------- CPU oracle ----
@@ -439,28 +460,26 @@ def main():
     achieved = dom_bytes / dom_s / 1e9
 
     # end to end: pinned host x -> device, step, y -> pinned host, every step
+    # (one copy each way: every x of the step lives in one buffer, every y in
+    # another)
     xs, ys = step.io_tensors()
-    hx = [x.cpu().pin_memory() for x in xs]
-    hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys]
+    hx = xs.cpu().pin_memory()
+    hy = torch.empty(ys.shape, dtype=ys.dtype).pin_memory()
     e2e_steps = max(1, min(args.steps, 500))
     with torch.cuda.stream(stream):
         for _ in range(3):
-            for h, d in zip(hx, xs):
-                d.copy_(h, non_blocking=True)
+            xs.copy_(hx, non_blocking=True)
             g.replay()
-            for h, d in zip(hy, ys):
-                h.copy_(d, non_blocking=True)
+            hy.copy_(ys, non_blocking=True)
     torch.cuda.synchronize()
     barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         f0.record(stream)
         for _ in range(e2e_steps):
-            for h, d in zip(hx, xs):
-                d.copy_(h, non_blocking=True)
+            xs.copy_(hx, non_blocking=True)
             g.replay()
-            for h, d in zip(hy, ys):
-                h.copy_(d, non_blocking=True)
+            hy.copy_(ys, non_blocking=True)
         f1.record(stream)
     torch.cuda.synchronize()
     t_e2e = f0.elapsed_time(f1) / 1e3
@@ -468,8 +487,8 @@ def main():
         tt = torch.tensor([t_e2e], dtype=torch.float64, device=device)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         t_e2e = float(tt.item())
-    h2d = sum(x.numel() * x.element_size() for x in xs)
-    d2h = sum(y.numel() * y.element_size() for y in ys)
+    h2d = xs.numel() * xs.element_size()
+    d2h = ys.numel() * ys.element_size()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -141,6 +141,13 @@ __device__ __forceinline__ uint64_t policy_evict_first()
     return p;
 }
 
+__device__ __forceinline__ uint64_t policy_evict_normal()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
                                             int x, int y, uint64_t policy)
 {
@@ -237,21 +244,30 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 //
 // Codes enter the tensor core as fp16 *subnormals*: a 16-bit lane holding the
 // integer u (< 1024) in its low bits and zero elsewhere is exactly u * 2^-24,
-// so masking the code bits into place is the whole conversion (Q4: the two
-// nibbles of a byte, Q8: the byte biased by +128).  The format's zero point z
-// (8 for Q4, 128 for the biased Q8 code) is removed by a second mma that
-// starts each block's accumulator at -z * 2^-24 * sum(x) (block_offset).
-// Every product is exact; the 2^-24 is undone at the store.
+// so masking the code bits into place is the whole conversion.  Q8: the byte
+// biased by +128 (u = q + 128).  Q4: both nibbles of a byte are placed at bits
+// 4-7 of their lanes (u = 16 q): the high nibble is already there, the low one
+// gets there by a multiply by 16 -- on the FMA pipe, which leaves the ALU pipe
+// (the busier one) one operation per register instead of two.  Either way the
+// lane is z' + u for a zero point z' = 128 (8 * 16 for Q4), removed by a second
+// mma that starts each block's accumulator at -128 * 2^-24 * sum(x)
+// (block_offset).  Every product is exact; the scale 2^-24 (2^-20 for Q4) is
+// undone at the store.
 
 // f16x2 of -z * 2^-24 (a subnormal): z = 8 -> 2^-21, z = 128 -> 2^-17.
 template <int FMT>
 __host__ __device__ constexpr uint32_t zero_point_pair()
 {
-    return FMT == 4 ? 0x80088008u : 0x80808080u;
+    return 0x80808080u;
 }
 
-// The y of a band is stored as acc * 2^24.
-constexpr float kUnscale = 16777216.0f;
+// The y of a band is stored as acc * 2^20 (Q4: codes enter at 16 * 2^-24) or
+// acc * 2^24 (Q8).
+template <int FMT>
+__host__ __device__ constexpr float unscale()
+{
+    return FMT == 4 ? 1048576.0f : 16777216.0f;
+}
 
 __device__ __forceinline__ float half_lo(uint32_t v)
 {
@@ -286,12 +302,14 @@ __device__ __forceinline__ void block_offset(uint2 xa, uint2 xb, float (&s)[4])
 }
 
 // One Q4 block (32 weights along K) for one 16-row m-tile, in PTX so the
-// instruction sequence is exactly: 2 shared loads (rows g, g+8), 4 prmt and
-// 8 mask/shift ops to place the nibbles as fp16 subnormals, 2 mma (low then
-// high nibbles, starting from the zero-point term `off`), 4 fma for the
-// scales.  `addr` is the shared address of row g's 4-byte group.
+// instruction sequence is exactly: 2 shared loads (rows g, g+8), 4 prmt to
+// spread the 4 code bytes of each row over fp16 lanes, 4 multiplies by 16
+// (`m16` holds 16 in a register, so they stay multiplies) and 8 masks to place
+// each nibble at bits 4-7, 2 mma (low then high nibbles, starting from the
+// zero-point term `off`), 4 fma for the scales.  `addr` is the shared address
+// of row g's 4-byte group.
 __device__ __forceinline__ void block_q4(uint32_t addr, uint2 xa, uint2 xb, const float (&off)[4],
-                                         float dg, float dg8, float (&acc)[4])
+                                         float dg, float dg8, float (&acc)[4], uint32_t m16)
 {
     asm("{\n\t"
         ".reg .b32 w0, w8, p01, p23, q01, q23, a0, a1, a2, a3;\n\t"
@@ -302,20 +320,20 @@ __device__ __forceinline__ void block_q4(uint32_t addr, uint2 xa, uint2 xb, cons
         "prmt.b32 p23, w0, 0, 0x4342;\n\t"
         "prmt.b32 q01, w8, 0, 0x4140;\n\t"
         "prmt.b32 q23, w8, 0, 0x4342;\n\t"
-        "and.b32 a0, p01, 0x000F000F;\n\t"
-        "and.b32 a1, q01, 0x000F000F;\n\t"
-        "and.b32 a2, p23, 0x000F000F;\n\t"
-        "and.b32 a3, q23, 0x000F000F;\n\t"
+        "mul.lo.u32 a0, p01, %15;\n\t"
+        "mul.lo.u32 a1, q01, %15;\n\t"
+        "mul.lo.u32 a2, p23, %15;\n\t"
+        "mul.lo.u32 a3, q23, %15;\n\t"
+        "and.b32 a0, a0, 0x00F000F0;\n\t"
+        "and.b32 a1, a1, 0x00F000F0;\n\t"
+        "and.b32 a2, a2, 0x00F000F0;\n\t"
+        "and.b32 a3, a3, 0x00F000F0;\n\t"
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {c0,c1,c2,c3}, {a0,a1,a2,a3}, {%5,%6}, "
         "{%9,%10,%11,%12};\n\t"
-        "shr.u32 p01, p01, 4;\n\t"
-        "shr.u32 q01, q01, 4;\n\t"
-        "shr.u32 p23, p23, 4;\n\t"
-        "shr.u32 q23, q23, 4;\n\t"
-        "and.b32 a0, p01, 0x000F000F;\n\t"
-        "and.b32 a1, q01, 0x000F000F;\n\t"
-        "and.b32 a2, p23, 0x000F000F;\n\t"
-        "and.b32 a3, q23, 0x000F000F;\n\t"
+        "and.b32 a0, p01, 0x00F000F0;\n\t"
+        "and.b32 a1, q01, 0x00F000F0;\n\t"
+        "and.b32 a2, p23, 0x00F000F0;\n\t"
+        "and.b32 a3, q23, 0x00F000F0;\n\t"
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {c0,c1,c2,c3}, {a0,a1,a2,a3}, {%7,%8}, "
         "{c0,c1,c2,c3};\n\t"
         "fma.rn.f32 %0, %13, c0, %0;\n\t"
@@ -324,9 +342,8 @@ __device__ __forceinline__ void block_q4(uint32_t addr, uint2 xa, uint2 xb, cons
         "fma.rn.f32 %3, %14, c3, %3;\n\t}"
         : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
         : "r"(addr), "r"(xa.x), "r"(xa.y), "r"(xb.x), "r"(xb.y), "f"(off[0]), "f"(off[1]),
-          "f"(off[2]), "f"(off[3]), "f"(dg), "f"(dg8));
+          "f"(off[2]), "f"(off[3]), "f"(dg), "f"(dg8), "r"(m16));
 }
-
 // One Q8 block for the 16-row m-tile: addr_a / addr_b are row g's 4-byte
 // groups in the block's two 16-element halves.
 __device__ __forceinline__ void block_q8(uint32_t addr_a, uint32_t addr_b, uint2 xa, uint2 xb,
@@ -432,7 +449,8 @@ __device__ __forceinline__ void chunk_load_x(const __half *xp, int nblk, uint2 (
 template <int FMT>
 __device__ __forceinline__ void chunk_mma(uint32_t codes_s, uint32_t scales_s, int nblk, int g,
                                           int t, const int (&sw)[8], const uint2 (&xa)[8],
-                                          const uint2 (&xb)[8], float (&acc)[Fmt<FMT>::kMT][4])
+                                          const uint2 (&xb)[8], float (&acc)[Fmt<FMT>::kMT][4],
+                                          uint32_t m16)
 {
     constexpr int MT = Fmt<FMT>::kMT;
     uint4 sc[MT][2];
@@ -453,7 +471,7 @@ __device__ __forceinline__ void chunk_mma(uint32_t codes_s, uint32_t scales_s, i
             const float dg = (jb & 1) ? d1 : d0;
             const float dg8 = (jb & 1) ? e1 : e0;
             if constexpr (FMT == 4) {
-                block_q4(lane_codes + mt * 2048 + sw[jb], xa[jb], xb[jb], off, dg, dg8, acc[mt]);
+                block_q4(lane_codes + mt * 2048 + sw[jb], xa[jb], xb[jb], off, dg, dg8, acc[mt], m16);
             } else {
                 const uint32_t base = lane_codes + (jb >> 2) * 2048;
                 block_q8(base + (sw[jb] & 0xffff), base + (sw[jb] >> 16), xa[jb], xb[jb], off, dg,

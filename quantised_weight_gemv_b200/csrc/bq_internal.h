@@ -22,10 +22,12 @@ inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Number of SMs of the current device (cached per device).  -1 on error.
 int device_sm_count();
 
-// Build a 2-D or 3-D tiled tensor map (no multicast).  Returns false on error.
+// Build a 2-D or 3-D tiled tensor map (no multicast).  `promotion` widens each
+// L2 fill the copies cause.  Returns false on error.
 bool encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank,
                        const void *base, const uint64_t *dims, const uint64_t *strides_bytes,
-                       const uint32_t *box, CUtensorMapSwizzle swizzle);
+                       const uint32_t *box, CUtensorMapSwizzle swizzle,
+                       CUtensorMapL2promotion promotion);
 
 // Launch `kernel` with the programmatic-dependent-launch attribute.
 cudaError_t launch_pdl(const void *kernel, dim3 grid, dim3 block, size_t smem,

@@ -46,7 +46,7 @@ int device_sm_count()
 
 bool encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base,
                        const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
-                       CUtensorMapSwizzle swizzle)
+                       CUtensorMapSwizzle swizzle, CUtensorMapL2promotion promotion)
 {
     std::call_once(g_encode_once, load_encode);
     if (!g_encode)
@@ -60,8 +60,7 @@ bool encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank, co
     for (int i = 0; i < rank - 1; i++)
         gstride[i] = strides_bytes[i];
     CUresult r = g_encode(map, dtype, (cuuint32_t)rank, const_cast<void *>(base), gdim, gstride,
-                          bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promotion,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }

@@ -289,6 +289,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     const int w = blockIdx.x * kWarps + warp;
     const int cta_first = blockIdx.x * kWarps;
     const uint64_t pol = policy_evict_first();
+    const uint64_t pol_s = policy_evict_normal();
 
     // Per-unit geometry (matrix, or expert piece in MoE mode).  Only plan mode
     // indexes a descriptor array; the other modes have one descriptor.
@@ -384,14 +385,14 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             if constexpr (MOE) {
                 const int e = grp.piece_expert[iss.u];
                 tma_load_3d(cdst, &a.mat0.tm_codes, bar, iss.kp * 128, row, e, pol);
-                tma_load_3d(sdst, &a.mat0.tm_scales, bar, iss.kp * 8, row, e, pol);
+                tma_load_3d(sdst, &a.mat0.tm_scales, bar, iss.kp * 8, row, e, (FMT == 4) ? pol : pol_s);
             } else {
                 const MatDesc &m = mats[PLAN ? iss.u : 0];
 #pragma unroll
                 for (int bx = 0; bx < Fmt<FMT>::kBoxes; bx++)
                     tma_load_2d(cdst + bx * (ROWS * 128), &m.tm_codes, bar,
                                 iss.kp * 128 * Fmt<FMT>::kBoxes + bx * 128, row, pol);
-                tma_load_2d(sdst, &m.tm_scales, bar, iss.kp * 8, row, pol);
+                tma_load_2d(sdst, &m.tm_scales, bar, iss.kp * 8, row, (FMT == 4) ? pol : pol_s);
             }
         }
         issued++;
@@ -429,11 +430,11 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 if constexpr (MOE) {
                     if (col < grp.piece_count[u]) {
                         const int slot = grp.sorted_slot[grp.piece_first[u] + col];
-                        m.y[(size_t)slot * m.N + row] = v[mt][q] * kUnscale;
+                        m.y[(size_t)slot * m.N + row] = v[mt][q] * unscale<FMT>();
                     }
                 } else {
                     if (col < m.B)
-                        m.y[(size_t)col * m.N + row] = v[mt][q] * kUnscale;
+                        m.y[(size_t)col * m.N + row] = v[mt][q] * unscale<FMT>();
                 }
             }
         }
@@ -603,6 +604,9 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     int acc_u = -1, acc_band = -1; // band the accumulators belong to
     int sw[8];
     lane_swizzle<FMT>(g, sw);
+    // 16 in a register the compiler cannot see through, so the Q4 nibble
+    // placement multiplies on the FMA pipe instead of shifting on the ALU.
+    const uint32_t m16 = launder(16u);
     const __half *xrow = nullptr;
     int nb32 = 0;
 
@@ -654,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 // Shared addresses of the slot, ordered after its wait (launder).
                 const uint32_t cs = launder(smem_u32(codes_ring + slot * CB));
                 const uint32_t ss = launder(smem_u32(scales_ring + slot * SB));
-                chunk_mma<FMT>(cs, ss, nblk, g, t, sw, xa, xb, acc);
+                chunk_mma<FMT>(cs, ss, nblk, g, t, sw, xa, xb, acc, m16);
                 done++;
                 // Plan mode: refill the slot just read at once, before any
                 // flush or stage barrier, so the ring always holds the warp's
@@ -780,6 +784,12 @@ size_t counters_bytes(long long n) { return align_up((size_t)n * sizeof(int), 25
 constexpr size_t kPartialsBytes = (size_t)kMaxCtas * kPartialBytesPerCta;
 constexpr size_t kSyncBytes = 512;
 
+// L2 fill widths: a code box row is 128 bytes (promote to exactly that); a
+// scale box row is 16 bytes of a longer row, and a wider fill would pull in
+// bytes of the neighbouring row too (measured: ~7% extra DRAM reads at 256 B).
+constexpr CUtensorMapL2promotion kPromoCodes = CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
+constexpr CUtensorMapL2promotion kPromoScales = CU_TENSOR_MAP_L2_PROMOTION_NONE;
+
 int rows_of(int fmt) { return fmt == 4 ? Fmt<4>::kRows : Fmt<8>::kRows; }
 
 bool fill_matdesc(int fmt, const bq_qmat *W, const uint16_t *x, int B, float *y, MatDesc *m)
@@ -793,9 +803,9 @@ bool fill_matdesc(int fmt, const bq_qmat *W, const uint16_t *x, int B, float *y,
     const uint64_t sstr[1] = {(uint64_t)ldS * 2};
     const uint32_t sbox[2] = {8, (uint32_t)R};
     if (!encode_tensor_map(&m->tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, cdims, cstr,
-                           cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                           cbox, CU_TENSOR_MAP_SWIZZLE_128B, kPromoCodes) ||
         !encode_tensor_map(&m->tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, W->scales, sdims, sstr,
-                           sbox, CU_TENSOR_MAP_SWIZZLE_NONE))
+                           sbox, CU_TENSOR_MAP_SWIZZLE_NONE, kPromoScales))
         return false;
     m->x = reinterpret_cast<const __half *>(x);
     m->y = y;
@@ -1098,9 +1108,9 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
     const uint64_t sstr[2] = {(uint64_t)ldS * 2, (uint64_t)scales_stride * 2};
     const uint32_t sbox[3] = {8, (uint32_t)Fmt<4>::kRows, 1};
     if (!encode_tensor_map(&a.mat0.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, Wstack->codes,
-                           cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                           cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B, kPromoCodes) ||
         !encode_tensor_map(&a.mat0.tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, Wstack->scales,
-                           sdims, sstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE))
+                           sdims, sstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE, kPromoScales))
         return BQ_ERR_CUDA;
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     float *slot_buf = reinterpret_cast<float *>(wsb + counters_bytes(nbands * B * topk) + kPartialsBytes);
