@@ -87,6 +87,9 @@ WORKLOADS = {
     synth.SINGLE_Q8.name: synth.SINGLE_Q8,
     synth.DENSE_H5120.name: synth.DENSE_H5120,
 }
+for _b in (1, 8):
+    _w = synth.moe_h2048(_b)
+    WORKLOADS[_w.name] = _w
 for _f in (4, 8):
     for _b in (1, 2, 4, 8):
         _w = synth.dense_h4096(_f, _b)
@@ -275,6 +278,97 @@ class DenseStep:
         return self.x_all, self.y_all
 
 
+class MoEStep:
+    """A routed-expert decode step resident in HBM: per layer, the expert stack of
+    gate|up (2*ffn x hidden) and of down (hidden x ffn), Q4, all E experts of all
+    layers (~16.3 GB for 48 layers of 128 experts).  One step = per layer the
+    gate|up call (per-slot outputs) and the down call (combined with the routing
+    weights); algorithmic bytes count the distinct routed experts only."""
+
+    def __init__(self, wl: synth.MoEWorkload, device, seed: int = 0):
+        import torch
+        from quantised_weight_gemv_b200 import bq
+        self.wl, self.device, self.bq = wl, device, bq
+        self.B, self.fmt = wl.B, 4
+        E, topk, B = wl.E, wl.topk, wl.B
+        (Ng, Kg), (Nd, Kd) = wl.gateup(), wl.down()
+        st = torch.zeros(1, dtype=torch.int32, device=device)
+        self.layers = []
+        self.bytes_alg = 0
+        self.distinct = []
+        self._keep = []
+        ins, outs = [], []
+        for layer in range(wl.layers):
+            idx, r = synth.routing(synth.key(seed, wl.wid, layer, 0, synth.KIND_IDX),
+                                   synth.key(seed, wl.wid, layer, 0, synth.KIND_LOGIT), B, E, topk)
+            stacks = []
+            for mid, (N, K) in ((0, (Ng, Kg)), (1, (Nd, Kd))):
+                ldS = bq.scales_ld(K)
+                codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=device)
+                scales = torch.empty((E, N, ldS), dtype=torch.int16, device=device)
+                w = synth.weights_f32_torch(synth.key(seed, wl.wid, layer, mid, synth.KIND_W),
+                                            E * N, K, device)
+                bq.quantize_dev(4, w, codes.view(E * N, K // 2), scales.view(E * N, ldS), st)
+                del w
+                stacks.append((bq.qmat(codes, scales, N, K), N * K // 2, N * ldS))
+                self._keep += [codes, scales]
+            x = synth.activations_f16_torch(synth.key(seed, wl.wid, layer, 0, synth.KIND_X),
+                                            (B, Kg), device)
+            h = synth.activations_f16_torch(synth.key(seed, wl.wid, layer, 1, synth.KIND_H),
+                                            (B, topk, Kd), device)
+            ins += [x, h]
+            outs += [(B, topk, Ng), (B, Nd)]
+            nd = len(set(idx.ravel().tolist()))
+            self.distinct.append(nd)
+            self.bytes_alg += (nd * (synth.packed_bytes(4, Ng, Kg) + synth.packed_bytes(4, Nd, Kd))
+                               + x.numel() * 2 + h.numel() * 2 + B * topk * Ng * 4 + B * Nd * 4)
+            self.layers.append([stacks, torch.as_tensor(idx, device=device),
+                                torch.as_tensor(r, device=device)])
+        # Every input of the step (x, per-slot h, expert ids, routing weights)
+        # in one byte buffer and every output in another, 64-byte aligned
+        # slices: one copy each way end to end.
+        def pack(tensors):
+            offs, n = [], 0
+            for t in tensors:
+                offs.append(n)
+                n += -(-t.numel() * t.element_size() // 64) * 64
+            buf = torch.zeros(n, dtype=torch.uint8, device=device)
+            views = []
+            for o, t in zip(offs, tensors):
+                v = buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+                v.copy_(t)
+                views.append(v)
+            return buf, views
+        in_t = []
+        for li, L in enumerate(self.layers):
+            in_t += [ins[2 * li], ins[2 * li + 1], L[1], L[2]]
+        self.x_all, iv = pack(in_t)
+        self.y_all, ov = pack([torch.zeros(o, dtype=torch.float32, device=device) for o in outs])
+        for li, L in enumerate(self.layers):
+            x, h, idx, r = iv[4 * li:4 * li + 4]
+            L[1], L[2] = idx, r
+            L += [x, h, ov[2 * li], ov[2 * li + 1]]
+        ws = max(bq.lib().bq_moe_workspace_bytes(Ng, Kg, B, topk, E),
+                 bq.lib().bq_moe_workspace_bytes(Nd, Kd, B, topk, E))
+        self.ws = bq.workspace(ws, device)
+        torch.cuda.synchronize()
+        if int(st.item()) != 0:
+            raise RuntimeError(f"device quantiser status {int(st.item()):#x}")
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.launches_per_step = 3 * wl.layers   # gate|up, down, combine
+
+    def launch(self, stream, only=None):
+        E = self.wl.E
+        for stacks, idx, r, x, h, y_gu, y_dn in self.layers:
+            (qg, cg, sg), (qd, cd, sd) = stacks
+            self.bq.moe_gemv_q4(qg, E, cg, sg, x, False, idx, None, y_gu, self.ws, self.status, stream)
+            self.bq.moe_gemv_q4(qd, E, cd, sd, h, True, idx, r, y_dn, self.ws, self.status, stream)
+        return self.launches_per_step
+
+    def io_tensors(self):
+        return self.x_all, self.y_all
+
+
 # ---------------------------------------------------------- CPU oracle ----
 def oracle_sample(wl: synth.DenseWorkload, seed: int = 0):
     """Packed planes (oracle quantiser) + x for one layer of the workload."""
@@ -293,21 +387,68 @@ def oracle_sample(wl: synth.DenseWorkload, seed: int = 0):
     return mats
 
 
-def time_oracle_once(wl, mats, threads):
+def moe_oracle_sample(wl: synth.MoEWorkload, seed: int = 0):
+    """Layer 0 of a routed-expert workload for the oracle: the same routing as
+    the GPU step, packed stacks (oracle quantiser) holding the routed experts,
+    x and the per-slot h.  Returns (jobs, algorithmic bytes)."""
+    import numpy as np
     import oracle
+    E, topk, B = wl.E, wl.topk, wl.B
+    idx, r = synth.routing(synth.key(seed, wl.wid, 0, 0, synth.KIND_IDX),
+                           synth.key(seed, wl.wid, 0, 0, synth.KIND_LOGIT), B, E, topk)
+    used = sorted(set(idx.ravel().tolist()))
+    jobs, nbytes = [], 0
+    for mid, (N, K) in ((0, wl.gateup()), (1, wl.down())):
+        ldS = (K // 32 + 7) // 8 * 8
+        codes = np.zeros((E, N, K // 2), dtype=np.uint8)
+        scales = np.zeros((E, N, ldS), dtype=np.uint16)
+        for e in used:
+            w = synth.weights_f32(synth.key(seed, wl.wid, 0, mid * 1000 + e, synth.KIND_W), N, K)
+            codes[e], scales[e] = oracle.quantize_q4(w)
+        if mid == 0:
+            x = synth.activations_f16_bits(synth.key(seed, wl.wid, 0, 0, synth.KIND_X), B, K)
+            jobs.append((codes, scales, x, False, idx, None))
+            nbytes += x.size * 2 + B * topk * N * 4
+        else:
+            h = synth.activations_f16_bits(synth.key(seed, wl.wid, 0, 1, synth.KIND_H), B, topk, K)
+            jobs.append((codes, scales, h, True, idx, r))
+            nbytes += h.size * 2 + B * N * 4
+        nbytes += len(used) * synth.packed_bytes(4, N, K)
+    return jobs, nbytes
+
+
+def oracle_job(wl):
+    """(run-once callable, algorithmic bytes, sample label) for the CPU oracle."""
+    import oracle
+    threads = os.cpu_count() or 1
+    if isinstance(wl, synth.MoEWorkload):
+        jobs, nbytes = moe_oracle_sample(wl)
+
+        def run():
+            for codes, scales, x, per_slot, idx, r in jobs:
+                oracle.moe_gemv_q4(codes, scales, x, per_slot, idx, r, nthreads=threads)
+        return run, nbytes
+    mats = oracle_sample(wl)
+    nbytes = sum(m[3] for m in mats)
+
+    def run():
+        for codes, scales, x, _ in mats:
+            (oracle.gemv_q4 if wl.fmt == 4 else oracle.gemv_q8)(codes, scales, x, nthreads=threads)
+    return run, nbytes
+
+
+def time_once(run):
     t0 = time.perf_counter()
-    for codes, scales, x, _ in mats:
-        (oracle.gemv_q4 if wl.fmt == 4 else oracle.gemv_q8)(codes, scales, x, nthreads=threads)
+    run()
     return time.perf_counter() - t0
 
 
 def cpu_baseline(wl, budget_s=10.0):
     threads = os.cpu_count() or 1
-    mats = oracle_sample(wl)
-    nbytes = sum(m[3] for m in mats)
+    run, nbytes = oracle_job(wl)
     reps, total = 0, 0.0
     while total < budget_s or reps == 0:
-        total += time_oracle_once(wl, mats, threads)
+        total += time_once(run)
         reps += 1
     return {"value": round(nbytes * reps / total / 1e9, 4), "unit": "GB/s", "cores": threads,
             "kind": "oracle",
@@ -319,13 +460,12 @@ def run_reference(args, wl, rank):
     if rank != 0:
         return
     threads = os.cpu_count() or 1
-    mats = oracle_sample(wl)
-    nbytes = sum(m[3] for m in mats)
+    run, nbytes = oracle_job(wl)
     for _ in range(args.warmup):
-        time_oracle_once(wl, mats, threads)
+        time_once(run)
     t = 0.0
     for _ in range(args.steps):
-        t += time_oracle_once(wl, mats, threads)
+        t += time_once(run)
     val = nbytes * args.steps / t / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s",
@@ -379,7 +519,12 @@ def main():
         if world > 1:
             dist.barrier()
 
-    step = DenseStep(wl, device)
+    is_moe = isinstance(wl, synth.MoEWorkload)
+    if is_moe:
+        args.engine = "graph"   # one graph of the per-layer expert calls
+        step = MoEStep(wl, device)
+    else:
+        step = DenseStep(wl, device)
     stream = torch.cuda.Stream(device)
     peaks = load_peaks()
 
@@ -430,10 +575,11 @@ def main():
     if int(step.status.item()) != 0:
         raise RuntimeError(f"device status {int(step.status.item()):#x}")
 
-    if args.engine == "step":
-        # the step kernel is the only kernel: one launch per step, timed over
-        # the timed region itself
-        dom = "decode step (all stages)"
+    if args.engine == "step" or is_moe:
+        # the step kernel is the only kernel (one launch per step), or (routed
+        # experts) the expert kernel is every launch but the small combine
+        # kernels: timed over the timed region itself
+        dom = "decode step (all stages)" if not is_moe else "routed-expert step (all launches)"
         dom_s = t_dev / args.steps
         dom_bytes = step.bytes_alg
     else:
@@ -501,18 +647,21 @@ def main():
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": f"q{wl.fmt} weights, f16 x, f16 mma operands, f32 accumulate",
+            "dtype": f"q{step.fmt} weights, f16 x, f16 mma operands, f32 accumulate",
             "data": "synthetic (seeded N(0,0.02) weights, N(0,1) fp16 activations)",
             "config": {"workload": wl.name, "batch": wl.B, "layers": wl.layers,
                        "launches_per_step": n_launch, "bytes_per_step": step.bytes_alg,
-                       "engine": ("one cooperative launch per step (bq_step_run), graph-captured"
+                       "engine": ("cuda-graph of per-layer bq_moe_gemv_q4 calls" if is_moe else
+                                  "one cooperative launch per step (bq_step_run), graph-captured"
                                   if args.engine == "step" else "cuda-graph of per-matrix launches"),
                        "l2": "inputs larger than L2 (no flush)",
                        "parallelism": f"replicas x{world}"},
             "tokens_per_s_equiv": round(world * wl.B / (t_dev / args.steps), 1),
+            **({"distinct_experts_per_layer": round(statistics.mean(step.distinct), 2)}
+               if is_moe else {}),
             "frac_of_measured_hbm": round(value / world / peaks["hbm_gbs"], 4),
             "frac_of_8TBps": round(value / world / 8000.0, 4),
-            "roofline": {"bound": "hbm", "kernel": f"stream_gemv q{wl.fmt} ({dom})",
+            "roofline": {"bound": "hbm", "kernel": f"stream_gemv q{step.fmt} ({dom})",
                          "timed": ("CUDA events over the timed region" if args.engine == "step"
                                    else "CUDA events around each launch"),
                          "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
