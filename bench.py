@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 from quantised_weight_gemv_b200 import synth  # noqa: E402
 
 METRIC = "weight-stream HBM GB/s (decode step, algorithmic bytes)"
+L2_FLUSH_BYTES = 256 << 20   # twice the B200's 126 MB L2
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "source": "fallback"}
 
 
@@ -96,8 +97,8 @@ for _f in (4, 8):
         WORKLOADS[_w.name] = _w
     for _n, _k in synth.SWEEP_SHAPES:
         for _b in (1, 8):
-            _w = synth.sweep_workload(_f, _n, _k, _b)
-            WORKLOADS[_w.name] = _w
+            for _w in (synth.sweep_workload(_f, _n, _k, _b), synth.single_workload(_f, _n, _k, _b)):
+                WORKLOADS[_w.name] = _w
 
 
 def fused_stages(wl: synth.DenseWorkload):
@@ -482,6 +483,24 @@ def run_reference(args, wl, rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------ replicas ----
+def max_over_ranks(t: float, device, world: int) -> float:
+    """The slowest rank's time (every rank takes part; the result is on all)."""
+    if world == 1:
+        return t
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([t], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_gbs(world: int, bytes_per_step: int, steps: int, t: float) -> float:
+    """Whole-job GB/s: every replica streams bytes_per_step per step, timed by the
+    slowest rank."""
+    return world * bytes_per_step * steps / t / 1e9
+
+
 # ---------------------------------------------------------------- main ----
 def main():
     ap = argparse.ArgumentParser()
@@ -490,9 +509,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="bq", choices=["bq", "reference"])
     ap.add_argument("--workload", default=synth.DENSE_H2048.name, choices=sorted(WORKLOADS))
-    ap.add_argument("--engine", default="step", choices=["step", "graph"],
+    ap.add_argument("--engine", default=None, choices=["step", "graph"],
                     help="step: one cooperative launch per token (bq_step_run); "
-                         "graph: a CUDA graph of per-matrix bq_gemv launches")
+                         "graph: a CUDA graph of per-matrix bq_gemv launches.  Default: "
+                         "graph for a single matrix and for routed experts, step otherwise")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -524,6 +544,8 @@ def main():
         args.engine = "graph"   # one graph of the per-layer expert calls
         step = MoEStep(wl, device)
     else:
+        if args.engine is None:   # one matrix: the plain bq_gemv call
+            args.engine = "graph" if wl.layers == 1 and len(wl.mats) == 1 else "step"
         step = DenseStep(wl, device)
     stream = torch.cuda.Stream(device)
     peaks = load_peaks()
@@ -555,23 +577,36 @@ def main():
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
+    # A step smaller than twice the L2 would be served from L2 when replayed:
+    # then every step is timed alone, after an untimed write of a buffer
+    # larger than the L2.
+    flush = None
+    if step.bytes_alg < L2_FLUSH_BYTES:
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_begin = time.time()
+    pairs = []
     with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(args.steps):
-            g.replay()
-        e1.record(stream)
+        if flush is None:
+            e0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            e1.record(stream)
+        else:
+            for _ in range(args.steps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+                pairs.append((a, b))
     torch.cuda.synchronize()
     t_end = time.time()
     barrier()
     torch.cuda.synchronize()
     clocks = sampler.stop(t_begin, t_end)
-    t_dev = e0.elapsed_time(e1) / 1e3
-    if world > 1:
-        tt = torch.tensor([t_dev], dtype=torch.float64, device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_dev = float(tt.item())
+    t_local = (e0.elapsed_time(e1) if flush is None else sum(a.elapsed_time(b) for a, b in pairs)) / 1e3
+    t_dev = max_over_ranks(t_local, device, world)
     if int(step.status.item()) != 0:
         raise RuntimeError(f"device status {int(step.status.item()):#x}")
 
@@ -593,6 +628,8 @@ def main():
                 for q, x, y, label, _ in step.launches:
                     if label != dom:
                         continue
+                    if flush is not None:
+                        flush.zero_()   # a set smaller than the L2: time each call cold
                     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                     a.record(stream)
                     fn(ctypes.byref(q), x.data_ptr(), step.B, y.data_ptr(), step.ws.data_ptr(),
@@ -620,19 +657,26 @@ def main():
     torch.cuda.synchronize()
     barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pairs = []
     with torch.cuda.stream(stream):
-        f0.record(stream)
+        if flush is None:
+            f0.record(stream)
         for _ in range(e2e_steps):
+            if flush is not None:
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
             xs.copy_(hx, non_blocking=True)
             g.replay()
             hy.copy_(ys, non_blocking=True)
-        f1.record(stream)
+            if flush is not None:
+                b.record(stream)
+                pairs.append((a, b))
+        if flush is None:
+            f1.record(stream)
     torch.cuda.synchronize()
-    t_e2e = f0.elapsed_time(f1) / 1e3
-    if world > 1:
-        tt = torch.tensor([t_e2e], dtype=torch.float64, device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_e2e = float(tt.item())
+    t_local = (f0.elapsed_time(f1) if flush is None else sum(a.elapsed_time(b) for a, b in pairs)) / 1e3
+    t_e2e = max_over_ranks(t_local, device, world)
     h2d = xs.numel() * xs.element_size()
     d2h = ys.numel() * ys.element_size()
 
@@ -641,7 +685,7 @@ def main():
         cpu = cpu_baseline(wl)
 
     if rank == 0:
-        value = world * step.bytes_alg * args.steps / t_dev / 1e9
+        value = job_gbs(world, step.bytes_alg, args.steps, t_dev)
         ms = t_dev / args.steps * 1e3
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -654,7 +698,9 @@ def main():
                        "engine": ("cuda-graph of per-layer bq_moe_gemv_q4 calls" if is_moe else
                                   "one cooperative launch per step (bq_step_run), graph-captured"
                                   if args.engine == "step" else "cuda-graph of per-matrix launches"),
-                       "l2": "inputs larger than L2 (no flush)",
+                       "l2": ("inputs larger than L2 (no flush)" if flush is None else
+                              f"L2 flushed before every step ({L2_FLUSH_BYTES >> 20} MB write, untimed); "
+                              "steps timed one by one"),
                        "parallelism": f"replicas x{world}"},
             "tokens_per_s_equiv": round(world * wl.B / (t_dev / args.steps), 1),
             **({"distinct_experts_per_layer": round(statistics.mean(step.distinct), 2)}
@@ -671,7 +717,7 @@ def main():
                          "bytes_per_launch": int(dom_bytes),
                          "launch_us": round(dom_s * 1e6, 3)},
             "cpu_baseline": cpu,
-            "e2e": {"value": round(world * step.bytes_alg * e2e_steps / t_e2e / 1e9, 2),
+            "e2e": {"value": round(job_gbs(world, step.bytes_alg, e2e_steps, t_e2e), 2),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
             "gpu_launches": n_launch * args.steps,

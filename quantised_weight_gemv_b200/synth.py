@@ -157,12 +157,20 @@ SWEEP_SHAPES = ((512, 512), (1024, 1024), (2048, 2048), (4096, 4096), (5120, 512
                 (1024, 5120), (8192, 5120), (25600, 5120), (5120, 25600))
 
 
-def sweep_workload(fmt: int, N: int, K: int, B: int = 1, min_bytes: int = 512 << 20) -> DenseWorkload:
+def sweep_workload(fmt: int, N: int, K: int, B: int = 1, min_bytes: int = 512 << 20,
+                   max_copies: int = 256) -> DenseWorkload:
     """Independent copies of one N x K matrix, enough of them (>= min_bytes,
-    i.e. several times the L2) that no copy is served from L2."""
-    copies = max(2, -(-min_bytes // packed_bytes(fmt, N, K)))
+    i.e. several times the L2) that no copy is served from L2 -- at most
+    max_copies (the matrices one step plan holds); a set that then stays below
+    twice the L2 is timed with the L2 flushed before every step."""
+    copies = min(max_copies, max(2, -(-min_bytes // packed_bytes(fmt, N, K))))
     return DenseWorkload(6, f"sweep-q{fmt}-{N}x{K}-b{B}", fmt, copies, (Mat("w", N, K, 0),), B,
                          independent=True)
+
+
+def single_workload(fmt: int, N: int, K: int, B: int = 1) -> DenseWorkload:
+    """One N x K matrix: a single call (its latency, with the L2 flushed)."""
+    return DenseWorkload(7, f"single-q{fmt}-{N}x{K}-b{B}", fmt, 1, (Mat("w", N, K, 0),), B)
 
 
 @dataclasses.dataclass(frozen=True)
