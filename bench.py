@@ -691,7 +691,9 @@ def main():
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": f"q{step.fmt} weights, f16 x, f16 mma operands, f32 accumulate",
+            "dtype": "f16",
+            "arith": (f"q{step.fmt} codes as exact f16 subnormal mma operands, f16 x, "
+                      "f32 accumulation and scaling"),
             "data": "synthetic (seeded N(0,0.02) weights, N(0,1) fp16 activations)",
             "config": {"workload": wl.name, "batch": wl.B, "layers": wl.layers,
                        "launches_per_step": n_launch, "bytes_per_step": step.bytes_alg,
