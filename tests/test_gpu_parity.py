@@ -193,6 +193,21 @@ def test_moe_out_of_range_index_sets_status_no_trap():
         check_tol(y, y_ref, absy)
 
 
+def test_moe_token_with_no_valid_slot_combines_to_zero():
+    """A token whose every expert id is out of range: its combined row is 0 (the
+    output starts as NaN, so every element must be written), the other tokens
+    are combined normally, and the status flags the bad ids."""
+    N, K, B, topk, E = 96, 512, 3, 3, 6
+    codes, scales, x, _, r = _moe_inputs(E, N, K, B, topk, 13, True)
+    idx = np.array([[0, 5, 2], [-1, 6, 99], [2, 2, 3]], dtype=np.int32)
+    y, st = gpu_moe(codes, scales, x, True, idx, r)
+    assert st == 1 << bq.BQ_ERR_EXPERT_INDEX
+    assert np.all(y[1] == 0.0)
+    y_ref, absy, bad = oracle.moe_gemv_q4(codes, scales, x, True, idx, r)
+    assert bad
+    check_tol(y, y_ref, absy)
+
+
 def test_moe_single_expert_matches_dense():
     N, K, B = 200, 1024, 6
     codes, scales, x, _, _ = _moe_inputs(3, N, K, B, 1, 12, False)
