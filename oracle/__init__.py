@@ -78,6 +78,10 @@ def lib() -> ctypes.CDLL:
                 _c_u8p, _c_u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 ctypes.c_longlong, ctypes.c_longlong, _c_u16p, ctypes.c_int, _c_i32p,
                 _c_f32p, ctypes.c_int, ctypes.c_int, _c_f64p, _c_f64p, ctypes.c_int]
+            L.oracle_silu.restype = ctypes.c_double
+            L.oracle_silu.argtypes = [ctypes.c_double]
+            L.oracle_swiglu_f16.restype = None
+            L.oracle_swiglu_f16.argtypes = [_c_f64p, _c_f64p, ctypes.c_int, _c_u16p]
             _lib = L
         return _lib
 
@@ -212,3 +216,20 @@ def moe_gemv_q4(codes, scales, x_bits, x_per_slot: bool, expert_idx, route_w=Non
     if rc not in (0, 2):
         raise ValueError(f"oracle moe gemv failed ({rc})")
     return y, absy, rc == 2
+
+
+def silu(z: float) -> float:
+    """silu(z) = z / (1 + e^-z) in fp64."""
+    return float(lib().oracle_silu(float(z)))
+
+
+def swiglu_f16(g, u) -> np.ndarray:
+    """fp16 bits of silu(g) * u, evaluated in fp64 and rounded once (ties to
+    even).  g, u: float arrays of the same shape (fp64 sums of the gate and up
+    projections)."""
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    u = np.ascontiguousarray(u, dtype=np.float64)
+    assert g.shape == u.shape
+    h = np.empty(g.shape, dtype=np.uint16)
+    lib().oracle_swiglu_f16(_p(g, _c_f64p), _p(u, _c_f64p), int(g.size), _p(h, _c_u16p))
+    return h

@@ -370,3 +370,26 @@ int oracle_moe_gemv_q4(const uint8_t *codes, const uint16_t *scales, int E, int 
     free(tmp);
     return bad ? 2 : 0;
 }
+
+/*
+ * Feed-forward activation between the fused gate|up projection and the down
+ * projection.  The pages' runtime fuses operator sequences inside
+ * feed-forward blocks (gist.science technical summary, "Methodologie" ->
+ * "Kernel Fusie en Specialisatie"); the activation of the model families they
+ * evaluate (Qwen3, Llama 3.2) is SwiGLU:
+ *
+ *      h[i] = silu(g[i]) * u[i],    silu(z) = z / (1 + e^-z)
+ *
+ * evaluated here in fp64 and rounded once to the nearest fp16 (ties to even),
+ * the type the down projection consumes.
+ */
+double oracle_silu(double z)
+{
+    return z / (1.0 + exp(-z));
+}
+
+void oracle_swiglu_f16(const double *g, const double *u, int n, uint16_t *h)
+{
+    for (int i = 0; i < n; i++)
+        h[i] = oracle_double_to_half(oracle_silu(g[i]) * u[i]);
+}

@@ -9,6 +9,7 @@ plausible slip in the oracle (swapped nibbles, a transposed operand, a dropped
 -8 offset, a wrong rounding rule, a mis-strided scale plane) fails at least
 one of them.
 """
+import math
 from fractions import Fraction
 
 import numpy as np
@@ -346,3 +347,34 @@ def test_moe_out_of_range_index_flags_and_skips():
     np.testing.assert_allclose(y[1], np.float64(np.float32(0.75)) * y1[0], rtol=1e-15)
     per, _, bad = oracle.moe_gemv_q4(codes, scales, x, False, idx, None)
     assert bad and np.all(per[0, 1] == 0) and np.all(per[1, 0] == 0)
+
+
+# ------------------------------------------------------------- SwiGLU ----
+def test_silu_closed_forms():
+    """silu(z) = z * sigmoid(z): sigmoid(0) = 1/2 and sigmoid(ln 3) = 3/4 give
+    exact values; sigmoid(z) + sigmoid(-z) = 1 gives the odd part
+    silu(z) - silu(-z) = z, and sigmoid(z) - sigmoid(-z) = tanh(z/2) the even
+    part silu(z) + silu(-z) = z tanh(z/2) (library tanh, an independent
+    function); large |z| saturates to z and to 0."""
+    assert oracle.silu(0.0) == 0.0
+    assert oracle.silu(math.log(3.0)) == pytest.approx(0.75 * math.log(3.0), rel=1e-15)
+    assert oracle.silu(-math.log(3.0)) == pytest.approx(-0.25 * math.log(3.0), rel=1e-15)
+    for z in (0.1, 0.5, 1.0, 2.5, 7.0, 20.0):
+        assert oracle.silu(z) - oracle.silu(-z) == pytest.approx(z, rel=1e-14)
+        assert oracle.silu(z) + oracle.silu(-z) == pytest.approx(z * math.tanh(z / 2.0), rel=1e-12)
+    assert oracle.silu(40.0) == pytest.approx(40.0, rel=1e-15)
+    assert abs(oracle.silu(-40.0)) < 1e-15
+
+
+def test_swiglu_f16_rounds_the_product_once():
+    """h = fp16(silu(g) * u): with sigmoid(ln 3) = 3/4 and u a power of two the
+    exact value is (3/4) ln 3 * 2^k, whose nearest fp16 numpy's float16 gives;
+    u = 0 gives a zero; silu(+-40) * u saturates to u*40 and to -0."""
+    ln3 = math.log(3.0)
+    g = np.array([ln3, ln3, ln3, -ln3, 0.0, 40.0, -40.0])
+    u = np.array([1.0, 4.0, -0.125, 2.0, 3.0, 0.5, 1.0])
+    h = oracle.swiglu_f16(g, u)
+    want = np.array([0.75 * ln3, 3.0 * ln3, -0.75 * ln3 / 8.0, -0.5 * ln3, 0.0, 20.0, -0.0],
+                    dtype=np.float64).astype(np.float16).view(np.uint16)
+    assert np.array_equal(h[:6], want[:6])
+    assert h[6] == 0x8000        # -40 * sigmoid(-40) = -1.7e-16: rounds to -0
