@@ -152,15 +152,50 @@ BQ_API int32_t bq_gemv_q8(const bq_qmat *W, const uint16_t *x, int32_t B, float 
 BQ_API int32_t bq_gemv_q4_noalloc(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
                                   int32_t *dev_status, void *stream);
 
+/* ------------------------------------------------------------ epilogues --- */
+
+/* What a GEMV writes.
+ *
+ * BQ_EPI_NONE: y is fp32 [B][N], the GEMV result.
+ *
+ * BQ_EPI_SWIGLU: the feed-forward activation fused into the gate|up
+ * projection, so the down projection reads its input straight from this
+ * output.  The pages' runtime fuses operator sequences inside feed-forward
+ * blocks to save global-memory round trips and launches (gist.science
+ * technical summary, "Methodologie" -> "Kernel Fusie en Specialisatie"); the
+ * activation of the families they evaluate (Qwen3, Llama 3.2) is SwiGLU.
+ *   W   the gate and up projections of one block (each F x K) in "SwiGLU pair
+ *       order": N = 2F with F a multiple of 8; rows 16j .. 16j+7 are gate rows
+ *       8j .. 8j+7 and rows 16j+8 .. 16j+15 are up rows 8j .. 8j+7 (each row
+ *       quantised on its own, so the planes of the two projections are just
+ *       interleaved 8 rows at a time).
+ *   y   fp16 bits [B][F]: h[b][i] = silu(g) * u, g and u the GEMV results for
+ *       gate row i and up row i, silu(z) = z / (1 + e^-z), evaluated in fp32
+ *       and rounded to the nearest fp16 -- the input format of the next GEMV. */
+enum { BQ_EPI_NONE = 0, BQ_EPI_SWIGLU = 1 };
+
+/* Q4 or Q8 decode GEMV with an output epilogue.
+ *   fmt        4 or 8
+ *   y          device: fp32 [B][N] (BQ_EPI_NONE) or fp16 bits [B][N/2]
+ *              (BQ_EPI_SWIGLU, N a multiple of 16), 16-byte aligned
+ *   epilogue   BQ_EPI_*; anything else returns BQ_ERR_SHAPE
+ * Other arguments, errors and launch behaviour as bq_gemv_q4. */
+BQ_API int32_t bq_gemv_ex(int32_t fmt, const bq_qmat *W, const uint16_t *x, int32_t B, void *y,
+                          int32_t epilogue, void *ws, size_t ws_bytes, int32_t *dev_status,
+                          void *stream);
+
 /* --------------------------------------------------------- decode step --- */
 
 /* One matrix of a decode step.  All planes and buffers are device memory. */
 typedef struct bq_step_mat {
     bq_qmat W;            /* the quantised matrix (plane layout above) */
     const uint16_t *x;    /* fp16 bits [B][K], 16-byte aligned */
-    float *y;             /* fp32 [B][N], 16-byte aligned, overwritten */
+    void *y;              /* output per `epilogue` (fp32 [B][N] by default), 16-byte
+                             aligned, overwritten */
     int32_t B;            /* 1..8 */
     int32_t stage;        /* >= 0; stages run in increasing order */
+    int32_t epilogue;     /* BQ_EPI_* */
+    int32_t reserved;     /* 0 */
 } bq_step_mat;
 
 /* Host-side description of a built plan (filled by bq_step_plan). */

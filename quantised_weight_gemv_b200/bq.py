@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libbq.so")
 
 BQ_OK, BQ_ERR_NULL, BQ_ERR_SHAPE, BQ_ERR_ALIGN, BQ_ERR_BATCH = 0, 1, 2, 3, 4
 BQ_ERR_EXPERT_INDEX, BQ_ERR_CUDA, BQ_ERR_TIMEOUT, BQ_ERR_WORKSPACE, BQ_ERR_RANGE = 5, 6, 7, 8, 9
+BQ_EPI_NONE, BQ_EPI_SWIGLU = 0, 1
 
 
 class bq_qmat(ctypes.Structure):
@@ -26,7 +27,8 @@ class bq_qmat(ctypes.Structure):
 
 class bq_step_mat(ctypes.Structure):
     _fields_ = [("W", bq_qmat), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p),
-                ("B", ctypes.c_int32), ("stage", ctypes.c_int32)]
+                ("B", ctypes.c_int32), ("stage", ctypes.c_int32),
+                ("epilogue", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class bq_step_info(ctypes.Structure):
@@ -55,6 +57,7 @@ _SIGS = {
     "bq_scales_ld": (_i32, [_i32]),
     "bq_gemv_workspace_bytes": (_sz, [_i32, _i32]),
     "bq_gemv_q4": (_i32, [_QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
+    "bq_gemv_ex": (_i32, [_i32, _QP, _vp, _i32, _vp, _i32, _vp, _sz, _vp, _vp]),
     "bq_gemv_q8": (_i32, [_QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
     "bq_gemv_q4_noalloc": (_i32, [_QP, _vp, _i32, _vp, _vp, _vp]),
     "bq_step_plan_bytes": (_sz, [_i32]),
@@ -139,13 +142,20 @@ def workspace(nbytes: int, device):
     return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)
 
 
-def gemv(fmt: int, W: bq_qmat, x, y, ws, status=None, stream=None) -> None:
-    """y[B, N] (fp32) = deq(W) . x[B, K] (fp16), through bq_gemv_q4 / bq_gemv_q8."""
-    fn = lib().bq_gemv_q4 if fmt == 4 else lib().bq_gemv_q8
+def gemv(fmt: int, W: bq_qmat, x, y, ws, status=None, stream=None, epilogue: int = BQ_EPI_NONE) -> None:
+    """y[B, N] (fp32) = deq(W) . x[B, K] (fp16), through bq_gemv_q4 / bq_gemv_q8;
+    with epilogue BQ_EPI_SWIGLU, y is fp16 [B, N/2] through bq_gemv_ex."""
     B = x.shape[0]
-    rc = fn(ctypes.byref(W), x.data_ptr(), B, y.data_ptr(), ws.data_ptr(),
-            ws.numel() * ws.element_size(), _ptr(status), _stream_ptr(stream))
-    check(f"bq_gemv_q{fmt}", rc)
+    if epilogue == BQ_EPI_NONE:
+        fn = lib().bq_gemv_q4 if fmt == 4 else lib().bq_gemv_q8
+        rc = fn(ctypes.byref(W), x.data_ptr(), B, y.data_ptr(), ws.data_ptr(),
+                ws.numel() * ws.element_size(), _ptr(status), _stream_ptr(stream))
+        check(f"bq_gemv_q{fmt}", rc)
+        return
+    rc = lib().bq_gemv_ex(int(fmt), ctypes.byref(W), x.data_ptr(), B, y.data_ptr(), int(epilogue),
+                          ws.data_ptr(), ws.numel() * ws.element_size(), _ptr(status),
+                          _stream_ptr(stream))
+    check("bq_gemv_ex", rc)
 
 
 def moe_gemv_q4(Wstack: bq_qmat, E: int, codes_stride: int, scales_stride: int, x,
@@ -163,13 +173,17 @@ class StepPlan:
     allocations owned by this object), built once by bq_step_plan."""
 
     def __init__(self, fmt: int, entries, device):
-        """entries: iterable of (bq_qmat, x, y, stage) with device tensors."""
+        """entries: iterable of (bq_qmat, x, y, stage) or (bq_qmat, x, y, stage,
+        epilogue) with device tensors."""
         import torch
         entries = list(entries)
         arr = (bq_step_mat * len(entries))()
         self._refs = []
-        for i, (W, x, y, stage) in enumerate(entries):
-            arr[i] = bq_step_mat(W, x.data_ptr(), y.data_ptr(), int(x.shape[0]), int(stage))
+        for i, e in enumerate(entries):
+            W, x, y, stage = e[:4]
+            epi = e[4] if len(e) > 4 else BQ_EPI_NONE
+            arr[i] = bq_step_mat(W, x.data_ptr(), y.data_ptr(), int(x.shape[0]), int(stage),
+                                 int(epi), 0)
             self._refs += [W, x, y]
         nbytes = lib().bq_step_plan_bytes(len(entries))
         self.plan = torch.empty(nbytes + 64, dtype=torch.uint8, device=device)

@@ -70,6 +70,7 @@ struct alignas(64) MatDesc {
     int nbands;
     int chunk_base;      // first chunk of this matrix within its stage
     int band_base;       // first arrival counter of this matrix within its stage
+    int epi;             // BQ_EPI_*
 };
 
 // The per-matrix fields the worker loop reads (everything but the tensor
@@ -78,7 +79,7 @@ struct alignas(64) MatDesc {
 struct MatInfo {
     const __half *x;
     float *y;
-    int N, K, B, cpb, nbands, chunk_base, band_base, pad;
+    int N, K, B, cpb, nbands, chunk_base, band_base, epi;
 };
 
 constexpr int kMaxPlanMats = 256;   // plan size limit (shared-memory cache)
@@ -231,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             mi.nbands = m.nbands;
             mi.chunk_base = m.chunk_base;
             mi.band_base = m.band_base;
-            mi.pad = 0;
+            mi.epi = m.epi;
             minfo[i] = mi;
         }
     }
@@ -419,6 +420,30 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     // col 2t+1), (row 16mt+g+8, col 2t), (row 16mt+g+8, col 2t+1).
     auto store_band = [&](int u, int band, const float (&v)[MT][4]) {
         const MatInfo &m = unit_mat(u);
+        if (!MOE && m.epi == BQ_EPI_SWIGLU) {
+            // SwiGLU pair order: in each 16-row tile, rows 0-7 are gate rows
+            // and rows 8-15 the up rows of the same 8 outputs, so this lane
+            // holds gate (v[mt][c]) and up (v[mt][2 + c]) of output i for
+            // batch columns 2t + c.  h = silu(g) * u in fp32, stored as fp16.
+            __half *h = reinterpret_cast<__half *>(m.y);
+            const int F = m.N / 2;
+#pragma unroll
+            for (int mt = 0; mt < MT; mt++) {
+                const int i = (band * ROWS + 16 * mt) / 2 + g;
+                if (i >= F)
+                    continue;
+#pragma unroll
+                for (int c = 0; c < 2; c++) {
+                    const int col = 2 * t + c;
+                    if (col >= m.B)
+                        continue;
+                    const float gv = v[mt][c] * unscale<FMT>();
+                    const float uv = v[mt][2 + c] * unscale<FMT>();
+                    h[(size_t)col * F + i] = __float2half_rn(gv / (1.0f + expf(-gv)) * uv);
+                }
+            }
+            return;
+        }
 #pragma unroll
         for (int mt = 0; mt < MT; mt++) {
 #pragma unroll
@@ -816,7 +841,15 @@ bool fill_matdesc(int fmt, const bq_qmat *W, const uint16_t *x, int B, float *y,
     m->nbands = (N + R - 1) / R;
     m->chunk_base = 0;
     m->band_base = 0;
+    m->epi = BQ_EPI_NONE;
     return true;
+}
+
+// An epilogue and the matrix it applies to: SwiGLU needs whole 16-row
+// gate|up tiles.
+bool epilogue_ok(int epi, int N)
+{
+    return epi == BQ_EPI_NONE || (epi == BQ_EPI_SWIGLU && N % 16 == 0);
 }
 
 void fill_stage(StageDesc *st, int mat_begin, int mat_end, long long T, int nbands, int wmax)
@@ -830,12 +863,14 @@ void fill_stage(StageDesc *st, int mat_begin, int mat_end, long long T, int nban
 }
 
 template <int FMT>
-int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void *ws,
-                  size_t ws_bytes, int32_t *dev_status, void *stream)
+int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32_t epi,
+                  void *ws, size_t ws_bytes, int32_t *dev_status, void *stream)
 {
     int32_t st = check_qmat(W);
     if (st != BQ_OK)
         return st;
+    if (!epilogue_ok(epi, W->N))
+        return BQ_ERR_SHAPE;
     if (!x || !y || !ws)
         return BQ_ERR_NULL;
     if (B < 1 || B > 8)
@@ -853,8 +888,9 @@ int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void
 
     KernelArgs a;
     memset(&a, 0, sizeof(a));
-    if (!fill_matdesc(FMT, W, x, B, y, &a.mat0))
+    if (!fill_matdesc(FMT, W, x, B, static_cast<float *>(y), &a.mat0))
         return BQ_ERR_CUDA;
+    a.mat0.epi = epi;
     const long long T = (long long)a.mat0.cpb * a.mat0.nbands;
     const int cap = max_ctas();
     if (cap < 0)
@@ -924,13 +960,24 @@ extern "C" size_t bq_gemv_workspace_bytes(int32_t N, int32_t K)
 extern "C" int32_t bq_gemv_q4(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void *ws,
                               size_t ws_bytes, int32_t *dev_status, void *stream)
 {
-    return gemv_impl<4>(W, x, B, y, ws, ws_bytes, dev_status, stream);
+    return gemv_impl<4>(W, x, B, y, BQ_EPI_NONE, ws, ws_bytes, dev_status, stream);
 }
 
 extern "C" int32_t bq_gemv_q8(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void *ws,
                               size_t ws_bytes, int32_t *dev_status, void *stream)
 {
-    return gemv_impl<8>(W, x, B, y, ws, ws_bytes, dev_status, stream);
+    return gemv_impl<8>(W, x, B, y, BQ_EPI_NONE, ws, ws_bytes, dev_status, stream);
+}
+
+extern "C" int32_t bq_gemv_ex(int32_t fmt, const bq_qmat *W, const uint16_t *x, int32_t B,
+                              void *y, int32_t epilogue, void *ws, size_t ws_bytes,
+                              int32_t *dev_status, void *stream)
+{
+    if (fmt == 4)
+        return gemv_impl<4>(W, x, B, y, epilogue, ws, ws_bytes, dev_status, stream);
+    if (fmt == 8)
+        return gemv_impl<8>(W, x, B, y, epilogue, ws, ws_bytes, dev_status, stream);
+    return BQ_ERR_SHAPE;
 }
 
 // ------------------------------------------------------------ decode step --
@@ -961,7 +1008,7 @@ extern "C" int32_t bq_step_plan(int32_t fmt, const bq_step_mat *mats, int32_t n_
             return BQ_ERR_NULL;
         if (mats[i].B < 1 || mats[i].B > 8)
             return BQ_ERR_BATCH;
-        if (mats[i].stage < 0)
+        if (mats[i].stage < 0 || !epilogue_ok(mats[i].epilogue, mats[i].W.N))
             return BQ_ERR_SHAPE;
         if (!aligned16(mats[i].x) || !aligned16(mats[i].y))
             return BQ_ERR_ALIGN;
@@ -1000,8 +1047,9 @@ extern "C" int32_t bq_step_plan(int32_t fmt, const bq_step_mat *mats, int32_t n_
         long long T = 0, bands = 0;
         while (j < n_mats && mats[order[j]].stage == s) {
             const bq_step_mat &m = mats[order[j]];
-            if (!fill_matdesc(fmt, &m.W, m.x, m.B, m.y, &md[j]))
+            if (!fill_matdesc(fmt, &m.W, m.x, m.B, static_cast<float *>(m.y), &md[j]))
                 return BQ_ERR_CUDA;
+            md[j].epi = m.epilogue;
             md[j].chunk_base = (int)T;
             md[j].band_base = (int)bands;
             T += (long long)md[j].cpb * md[j].nbands;

@@ -3,7 +3,10 @@ path through the C ABI binding, and check the tolerance
 
     |y - y_ref| <= 1e-3 * sum_k |deq(w) x| + 1e-5      (per output element)
 
-against the fp64 oracle."""
+against the fp64 oracle.  For the SwiGLU epilogue, h = silu(g) * u is checked
+against the oracle's fp16 h with that tolerance carried through silu(g) * u
+(|d silu / dz| <= 1.1 everywhere) plus one fp16 unit in the last place for
+the two roundings to fp16."""
 import numpy as np
 
 import oracle
@@ -61,3 +64,29 @@ def oracle_gemv(fmt, codes, scales, x_bits, nthreads=8):
 
 def quantize(fmt, w):
     return oracle.quantize_q4(w) if fmt == 4 else oracle.quantize_q8(w)
+
+
+def pair_order(gate, up):
+    """Rows of the gate and up projections (each [F, ...], F a multiple of 8)
+    interleaved 8 at a time: SwiGLU pair order."""
+    F = gate.shape[0]
+    assert F % 8 == 0 and up.shape == gate.shape
+    g = gate.reshape(F // 8, 8, *gate.shape[1:])
+    u = up.reshape(F // 8, 8, *up.shape[1:])
+    return np.stack([g, u], axis=1).reshape(2 * F, *gate.shape[1:])
+
+
+def check_swiglu(h_bits, g, absg, u, absu):
+    """Assert the SwiGLU output h (fp16 bits [B, F]) against the oracle."""
+    h = np.asarray(h_bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+    h_ref = oracle.swiglu_f16(g, u).view(np.float16).astype(np.float64)
+    assert np.all(np.isfinite(h))
+    tol_g = REL * absg + ABS
+    tol_u = REL * absu + ABS
+    sil = np.array([oracle.silu(z) for z in np.ravel(g)]).reshape(g.shape)
+    bound = 1.1 * np.abs(u) * tol_g + np.abs(sil) * tol_u + tol_g * tol_u \
+        + 2.0 ** -10 * np.abs(h_ref) + 2.0 ** -24
+    err = np.abs(h - h_ref)
+    bad = np.argwhere(err > bound)
+    assert bad.size == 0, f"{len(bad)} h out of tolerance, first {bad[:5].tolist()}"
+    return float(np.max(err / bound)) if err.size else 0.0

@@ -148,6 +148,22 @@ def test_gemv_argument_validation_before_launch(fmt):
     assert _gemv_rc(fmt, ws_bytes=1024) == bq.BQ_ERR_WORKSPACE
 
 
+def test_gemv_ex_epilogue_validation_before_launch():
+    f = bq.lib().bq_gemv_ex
+
+    def rc(fmt=4, N=64, epi=bq.BQ_EPI_SWIGLU):
+        W = bq.bq_qmat(FAKE, FAKE, N, 256)
+        return f(fmt, ctypes.byref(W), FAKE, 1, FAKE, epi, FAKE, 1 << 30, None, None)
+
+    assert rc(fmt=5) == bq.BQ_ERR_SHAPE
+    assert rc(epi=2) == bq.BQ_ERR_SHAPE
+    assert rc(epi=-1) == bq.BQ_ERR_SHAPE
+    assert rc(N=40) == bq.BQ_ERR_SHAPE            # SwiGLU needs whole 16-row gate|up tiles
+    W = bq.bq_qmat(FAKE, FAKE, 64, 256)
+    assert f(4, ctypes.byref(W), None, 1, FAKE, bq.BQ_EPI_SWIGLU, FAKE, 1 << 30, None, None) == bq.BQ_ERR_NULL
+    assert f(8, ctypes.byref(W), FAKE, 9, FAKE, bq.BQ_EPI_SWIGLU, FAKE, 1 << 30, None, None) == bq.BQ_ERR_BATCH
+
+
 def test_moe_argument_validation_before_launch():
     W = bq.bq_qmat(FAKE, FAKE, 64, 256)
     f = bq.lib().bq_moe_gemv_q4
@@ -208,6 +224,12 @@ def test_step_argument_validation_before_launch():
     arr[1].stage = -1
     assert L.bq_step_plan(4, arr, 2, FAKE, nb, ctypes.byref(info)) == bq.BQ_ERR_SHAPE
     arr[1].stage = 1
+    arr[1].epilogue = 3
+    assert L.bq_step_plan(4, arr, 2, FAKE, nb, ctypes.byref(info)) == bq.BQ_ERR_SHAPE
+    arr[1].epilogue = bq.BQ_EPI_SWIGLU
+    arr[1].W.N = 24                                   # not whole 16-row gate|up tiles
+    assert L.bq_step_plan(4, arr, 2, FAKE, nb, ctypes.byref(info)) == bq.BQ_ERR_SHAPE
+    arr[1].W.N = 64
     arr[0].W.K = 40
     assert L.bq_step_plan(4, arr, 2, FAKE, nb, ctypes.byref(info)) == bq.BQ_ERR_SHAPE
     info = bq.bq_step_info(4, 2, 2, 296, 10, 0, 64, 128, 1 << 20)

@@ -1,0 +1,75 @@
+"""The fused feed-forward path: a gate|up GEMV in SwiGLU pair order whose
+epilogue writes h = silu(gate) * up as fp16, and the down GEMV reading h,
+against the oracle (gate / up / down GEMVs in fp64, SwiGLU in fp64 rounded
+once to fp16)."""
+import numpy as np
+import pytest
+
+import oracle
+from quantised_weight_gemv_b200 import bq, synth
+from tests.gpu_helpers import (DEV, check_swiglu, check_tol, dev, new_status, oracle_gemv,
+                               pair_order)
+
+pytestmark = pytest.mark.gpu
+
+
+def _quant(fmt, w):
+    return oracle.quantize_q4(w) if fmt == 4 else oracle.quantize_q8(w)
+
+
+def _ffn_inputs(fmt, F, K, B, seed):
+    wg = synth.weights_f32(synth.key(seed, 82, 0, 0, synth.KIND_W), F, K)
+    wu = synth.weights_f32(synth.key(seed, 82, 0, 1, synth.KIND_W), F, K)
+    (cg, sg), (cu, su) = _quant(fmt, wg), _quant(fmt, wu)
+    x = synth.activations_f16_bits(synth.key(seed, 82, 0, 0, synth.KIND_X), B, K)
+    return cg, sg, cu, su, x
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+@pytest.mark.parametrize("F,K", [(8, 256), (24, 800), (200, 2048), (1024, 512)])
+@pytest.mark.parametrize("B", [1, 3, 8])
+def test_gemv_swiglu_epilogue(fmt, F, K, B):
+    import torch
+    cg, sg, cu, su, x = _ffn_inputs(fmt, F, K, B, 5)
+    codes, scales = pair_order(cg, cu), pair_order(sg, su)
+    N = 2 * F
+    c, s, xt = dev(codes.view(np.uint8)), dev(scales), dev(x)
+    h = torch.full((B, F), float("nan"), dtype=torch.float16, device=DEV)
+    ws = bq.workspace(bq.lib().bq_gemv_workspace_bytes(N, K), DEV)
+    st = new_status()
+    bq.gemv(fmt, bq.qmat(c, s, N, K), xt, h, ws, st, epilogue=bq.BQ_EPI_SWIGLU)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    g, ag = oracle_gemv(fmt, cg, sg, x)
+    u, au = oracle_gemv(fmt, cu, su, x)
+    check_swiglu(h.cpu().numpy().view(np.uint16), g, ag, u, au)
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
+@pytest.mark.parametrize("F,H", [(256, 512), (768, 2048)])
+def test_step_fused_ffn(fmt, F, H):
+    """One feed-forward block as a two-stage plan: gate|up + SwiGLU (stage 0)
+    writes h, down (stage 1) reads it; run twice (the plan is reusable)."""
+    import torch
+    B = 2
+    cg, sg, cu, su, x = _ffn_inputs(fmt, F, H, B, 6)
+    wd = synth.weights_f32(synth.key(6, 82, 0, 2, synth.KIND_W), H, F)
+    cd, sd = _quant(fmt, wd)
+    c1, s1 = dev(pair_order(cg, cu).view(np.uint8)), dev(pair_order(sg, su))
+    c2, s2 = dev(cd.view(np.uint8)), dev(sd)
+    xt = dev(x)
+    h = torch.full((B, F), float("nan"), dtype=torch.float16, device=DEV)
+    y = torch.full((B, H), float("nan"), dtype=torch.float32, device=DEV)
+    plan = bq.StepPlan(fmt, [(bq.qmat(c1, s1, 2 * F, H), xt, h, 0, bq.BQ_EPI_SWIGLU),
+                             (bq.qmat(c2, s2, H, F), h, y, 1)], DEV)
+    st = new_status()
+    for _ in range(2):
+        plan.run(st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        hb = h.cpu().numpy().view(np.uint16)
+        g, ag = oracle_gemv(fmt, cg, sg, x)
+        u, au = oracle_gemv(fmt, cu, su, x)
+        check_swiglu(hb, g, ag, u, au)
+        yr, ar = oracle_gemv(fmt, cd, sd, hb)      # down on the h the GPU produced
+        check_tol(y.cpu().numpy(), yr, ar)
