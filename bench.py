@@ -180,66 +180,120 @@ def phys_gpu_index(local_rank: int) -> int:
 
 # ------------------------------------------------------ device workload ----
 class DenseStep:
-    """All matrices of one decode step resident in HBM, plus x / y buffers."""
+    """All matrices of one decode step resident in HBM, plus x / y buffers.
 
-    def __init__(self, wl: synth.DenseWorkload, device, seed: int = 0):
+    Each layer's feed-forward block is fused: its gate and up projections form
+    one matrix in SwiGLU pair order whose epilogue writes h = silu(gate) * up
+    (fp16), and the down projection reads that h -- so the down stage really
+    depends on the stage before it.  Every other stage reads its own seeded
+    activations."""
+
+    def __init__(self, wl: synth.DenseWorkload, device, seed: int = 0, ffn: bool = True):
         import torch
         from quantised_weight_gemv_b200 import bq
         self.wl, self.device, self.bq = wl, device, bq
         self.B = wl.B
         self.fmt = wl.fmt
-        self.launches = []      # (qmat, x, y, label)
+        self.launches = []      # (qmat, x, y, label, stage, epilogue)
         self.bytes_alg = 0
         self.bytes_by_label = {}
         self._keep = []
         st = torch.zeros(1, dtype=torch.int32, device=device)
         ws_max = 0
         stages = fused_stages(wl)
+        Kc = lambda K: K // 2 if wl.fmt == 4 else K
+        pending = []            # (layer, stage, mats, K, Ntot, codes, scales, x-or-None, out spec)
         for layer in range(wl.layers):
+            h_shape = None
             for s, mats in stages:
                 K = mats[0].K
                 Ntot = sum(m.N for m in mats)
                 ldS = bq.scales_ld(K)
-                codes = torch.empty((Ntot, K // 2 if wl.fmt == 4 else K), dtype=torch.uint8, device=device)
+                names = [m.name for m in mats]
+                swiglu = ffn and names in (["gate", "up"], ["gateup"])
+                codes = torch.empty((Ntot, Kc(K)), dtype=torch.uint8, device=device)
                 scales = torch.empty((Ntot, ldS), dtype=torch.int16, device=device)
-                r0 = 0
-                for mi, m in enumerate(mats):
-                    w = synth.weights_f32_torch(synth.key(seed, wl.wid, layer, wl.mats.index(m),
-                                                          synth.KIND_W), m.N, K, device)
-                    bq.quantize_dev(wl.fmt, w, codes[r0:r0 + m.N], scales[r0:r0 + m.N], st)
-                    r0 += m.N
-                    del w
-                x = synth.activations_f16_torch(synth.key(seed, wl.wid, layer, s, synth.KIND_X),
-                                                (self.B, K), device)
-                y = (self.B, Ntot)   # allocated below, in one buffer with every other y
-                label = "+".join(m.name for m in mats)
-                q = bq.qmat(codes, scales, Ntot, K)
-                self.launches.append((q, x, y, label, wl.stage_of(layer, s)))
+                if swiglu:
+                    # gate rows and up rows, each quantised on its own, then
+                    # interleaved 8 at a time (SwiGLU pair order)
+                    F = Ntot // 2
+                    parts = []
+                    if names == ["gate", "up"]:
+                        for m in mats:
+                            parts.append(synth.weights_f32_torch(
+                                synth.key(seed, wl.wid, layer, wl.mats.index(m), synth.KIND_W),
+                                m.N, K, device))
+                    else:
+                        w = synth.weights_f32_torch(
+                            synth.key(seed, wl.wid, layer, wl.mats.index(mats[0]), synth.KIND_W),
+                            Ntot, K, device)
+                        parts = [w[:F], w[F:]]
+                    cv = codes.view(F // 8, 2, 8, Kc(K))
+                    sv = scales.view(F // 8, 2, 8, ldS)
+                    for half, w in enumerate(parts):
+                        ct = torch.empty((F, Kc(K)), dtype=torch.uint8, device=device)
+                        stt = torch.empty((F, ldS), dtype=torch.int16, device=device)
+                        bq.quantize_dev(wl.fmt, w.contiguous(), ct, stt, st)
+                        cv[:, half].copy_(ct.view(F // 8, 8, Kc(K)))
+                        sv[:, half].copy_(stt.view(F // 8, 8, ldS))
+                    del parts
+                else:
+                    r0 = 0
+                    for m in mats:
+                        w = synth.weights_f32_torch(synth.key(seed, wl.wid, layer, wl.mats.index(m),
+                                                              synth.KIND_W), m.N, K, device)
+                        bq.quantize_dev(wl.fmt, w, codes[r0:r0 + m.N], scales[r0:r0 + m.N], st)
+                        r0 += m.N
+                        del w
+                reads_h = ffn and names == ["down"] and h_shape is not None
+                x = None if reads_h else synth.activations_f16_torch(
+                    synth.key(seed, wl.wid, layer, s, synth.KIND_X), (self.B, K), device)
+                out = ("h", (self.B, Ntot // 2)) if swiglu else ("y", (self.B, Ntot))
+                pending.append((layer, s, "+".join(names), K, Ntot, codes, scales, x, out, reads_h))
+                if swiglu:
+                    h_shape = (self.B, Ntot // 2)
                 self._keep += [codes, scales]
-                nb = synth.packed_bytes(wl.fmt, Ntot, K) + self.B * K * 2 + self.B * Ntot * 4
+                nb = (synth.packed_bytes(wl.fmt, Ntot, K) + self.B * K * 2 +
+                      (self.B * (Ntot // 2) * 2 if swiglu else self.B * Ntot * 4))
                 self.bytes_alg += nb
+                label = "+".join(names)
                 self.bytes_by_label[label] = self.bytes_by_label.get(label, 0) + nb
                 ws_max = max(ws_max, bq.lib().bq_gemv_workspace_bytes(Ntot, K))
-        # Every x in one device buffer and every y in another (64-byte aligned
-        # slices), so a step's inputs and results each move in one copy.
-        def pack(shapes, dtype, fill=None):
+
+        # Every seeded x in one device buffer and every fp32 y in another
+        # (64-byte aligned slices), so a step's inputs and results each move in
+        # one copy; the SwiGLU outputs h live in a third buffer on the device.
+        def pack(shapes, dtype):
             esz = torch.empty((), dtype=dtype).element_size()
             offs, n = [], 0
             for shp in shapes:
                 offs.append(n)
                 cnt = shp[0] * shp[1]
                 n += -(-cnt * esz // 64) * 64 // esz
-            buf = torch.empty(n, dtype=dtype, device=device)
+            buf = torch.zeros(max(n, 1), dtype=dtype, device=device)
             views = [buf[o:o + a * b].view(a, b) for o, (a, b) in zip(offs, shapes)]
             return buf, views
-        self.x_all, xv = pack([e[1].shape for e in self.launches], torch.float16)
-        self.y_all, yv = pack([e[2] for e in self.launches], torch.float32)
-        self.y_all.zero_()
-        packed = []
-        for (q, x, _, label, stg), xd, yd in zip(self.launches, xv, yv):
-            xd.copy_(x)
-            packed.append((q, xd, yd, label, stg))
-        self.launches = packed
+        self.x_all, xv = pack([p[7].shape for p in pending if p[7] is not None], torch.float16)
+        self.y_all, yv = pack([p[8][1] for p in pending if p[8][0] == "y"], torch.float32)
+        self.h_all, hv = pack([p[8][1] for p in pending if p[8][0] == "h"], torch.float16)
+        xi = yi = hi = 0
+        last_h = None
+        for layer, s, label, K, Ntot, codes, scales, x, (kind, shp), reads_h in pending:
+            if reads_h:
+                xd = last_h
+            else:
+                xd = xv[xi]
+                xd.copy_(x)
+                xi += 1
+            if kind == "h":
+                yd, epi = hv[hi], bq.BQ_EPI_SWIGLU
+                hi += 1
+                last_h = yd
+            else:
+                yd, epi = yv[yi], bq.BQ_EPI_NONE
+                yi += 1
+            q = bq.qmat(codes, scales, Ntot, K)
+            self.launches.append((q, xd, yd, label, wl.stage_of(layer, s), epi))
         torch.cuda.synchronize()
         if int(st.item()) != 0:
             raise RuntimeError(f"device quantiser status {int(st.item()):#x}")
@@ -250,7 +304,8 @@ class DenseStep:
     def build_plan(self):
         """The whole step as one plan (stages in model order), built once.
         (A plan holds at most 256 matrices; larger sets use --engine graph.)"""
-        self.plan = self.bq.StepPlan(self.fmt, [(q, x, y, st) for q, x, y, _, st in self.launches],
+        self.plan = self.bq.StepPlan(self.fmt, [(q, x, y, st, epi)
+                                                for q, x, y, _, st, epi in self.launches],
                                      self.device)
 
     def run_step(self, stream):
@@ -258,19 +313,22 @@ class DenseStep:
         self.plan.run(self.status, stream)
         return 1
 
-    def launch(self, stream, only=None):
+    def launch_one(self, entry, stream):
         import ctypes
-        L = self.bq.lib()
-        fn = L.bq_gemv_q4 if self.fmt == 4 else L.bq_gemv_q8
-        sp = stream.cuda_stream
-        wsp, wsb, stp = self.ws.data_ptr(), self.ws.numel(), self.status.data_ptr()
+        q, x, y, label, _, epi = entry
+        rc = self.bq.lib().bq_gemv_ex(self.fmt, ctypes.byref(q), x.data_ptr(), self.B, y.data_ptr(),
+                                      epi, self.ws.data_ptr(), self.ws.numel(),
+                                      self.status.data_ptr(), stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(f"bq_gemv_ex: {self.bq.bq_status_string(rc)}")
+
+    def launch(self, stream, only=None):
+        """The step as per-matrix calls (the graph engine), in model order."""
         n = 0
-        for q, x, y, label, _ in self.launches:
-            if only is not None and label != only:
+        for e in self.launches:
+            if only is not None and e[3] != only:
                 continue
-            rc = fn(ctypes.byref(q), x.data_ptr(), self.B, y.data_ptr(), wsp, wsb, stp, sp)
-            if rc != 0:
-                raise RuntimeError(f"bq_gemv_q{self.fmt}: {self.bq.bq_status_string(rc)}")
+            self.launch_one(e, stream)
             n += 1
         return n
 
@@ -619,21 +677,18 @@ def main():
         dom_bytes = step.bytes_alg
     else:
         # dominant kernel: its launches timed one by one with events on its stream
-        import ctypes
         dom = max(step.bytes_by_label, key=step.bytes_by_label.get)
         durs = []
-        fn = step.bq.lib().bq_gemv_q4 if step.fmt == 4 else step.bq.lib().bq_gemv_q8
         with torch.cuda.stream(stream):
             for _ in range(3):
-                for q, x, y, label, _ in step.launches:
-                    if label != dom:
+                for e in step.launches:
+                    if e[3] != dom:
                         continue
                     if flush is not None:
                         flush.zero_()   # a set smaller than the L2: time each call cold
                     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                     a.record(stream)
-                    fn(ctypes.byref(q), x.data_ptr(), step.B, y.data_ptr(), step.ws.data_ptr(),
-                       step.ws.numel(), step.status.data_ptr(), stream.cuda_stream)
+                    step.launch_one(e, stream)
                     b.record(stream)
                     durs.append((a, b))
         torch.cuda.synchronize()

@@ -4,7 +4,7 @@ device).
 
 The oracle cannot redo multi-GB steps, so each test checks every output row
 of the first and the last layer and a seeded sample of rows of every other
-matrix.  For each checked row the fp32 weights are regenerated from the same
+matrix (for the fused feed-forward stage: of its SwiGLU output h).  For each checked row the fp32 weights are regenerated from the same
 seeded generator, quantised by the oracle, compared bit-for-bit with the
 device-quantised planes the kernel streamed, and multiplied by the oracle in
 fp64 against the same activations.  No oracle input comes from the CUDA path:
@@ -16,7 +16,7 @@ import pytest
 
 import oracle
 from quantised_weight_gemv_b200 import bq, synth
-from tests.gpu_helpers import DEV, check_tol, dev, new_status
+from tests.gpu_helpers import DEV, check_swiglu, check_tol, dev, new_status
 
 pytestmark = pytest.mark.gpu
 
@@ -28,7 +28,29 @@ def _rows_for(layer, layers, N, every, rng):
     return np.sort(rng.choice(N, size=k, replace=False))
 
 
+def _regen_rows(wl, seed, layer, m, rows, K, N_mat):
+    """fp32 rows of matrix m of a layer, regenerated from its seed key on the GPU."""
+    import torch
+    w = synth.weights_f32_torch(synth.key(seed, wl.wid, layer, wl.mats.index(m), synth.KIND_W),
+                                N_mat, K, DEV)
+    out = w[torch.as_tensor(rows, device=DEV)].cpu().numpy()
+    del w
+    return out
+
+
+def _quant(fmt, w):
+    return oracle.quantize_q4(w) if fmt == 4 else oracle.quantize_q8(w)
+
+
+def _gemv(fmt, codes, scales, xb):
+    return (oracle.gemv_q4 if fmt == 4 else oracle.gemv_q8)(codes, scales, xb, nthreads=8)
+
+
 def _check_step(wl, every, seed=0):
+    """Run the decode step once; check sampled rows of every matrix.  The fused
+    feed-forward stage (gate|up in SwiGLU pair order) is checked on its fp16
+    output h against the oracle's SwiGLU of the oracle's gate and up GEMVs;
+    the down stage then reads the h the GPU produced."""
     import torch
     import bench
     step = bench.DenseStep(wl, torch.device(DEV), seed=seed)
@@ -43,28 +65,44 @@ def _check_step(wl, every, seed=0):
     li = 0
     for layer in range(wl.layers):
         for s, group in stages:
-            q, x, y, label, _ = step.launches[li]
+            q, x, y, label, _, epi = step.launches[li]
             li += 1
             codes_d, scales_d = q._refs
+            K = group[0].K
             xb = x.cpu().numpy().view(np.uint16)
+            if epi == bq.BQ_EPI_SWIGLU:
+                F = sum(m.N for m in group) // 2
+                rows = _rows_for(layer, wl.layers, F, every, rng)
+                if len(group) == 2:
+                    wg = _regen_rows(wl, seed, layer, group[0], rows, K, F)
+                    wu = _regen_rows(wl, seed, layer, group[1], rows, K, F)
+                else:
+                    wg = _regen_rows(wl, seed, layer, group[0], rows, K, 2 * F)
+                    wu = _regen_rows(wl, seed, layer, group[0], rows + F, K, 2 * F)
+                (cg, sg), (cu, su) = _quant(wl.fmt, wg), _quant(wl.fmt, wu)
+                rg = torch.as_tensor(16 * (rows // 8) + rows % 8, device=DEV)   # pair order
+                for r_dev, c_ref, s_ref, what in ((rg, cg, sg, "gate"), (rg + 8, cu, su, "up")):
+                    assert np.array_equal(codes_d[r_dev].cpu().numpy(), c_ref.view(np.uint8)), \
+                        f"{label} L{layer}: {what} codes differ"
+                    assert np.array_equal(scales_d[r_dev].cpu().numpy().view(np.uint16), s_ref), \
+                        f"{label} L{layer}: {what} scales differ"
+                g, ag = _gemv(wl.fmt, cg, sg, xb)
+                u, au = _gemv(wl.fmt, cu, su, xb)
+                hb = y.cpu().numpy().view(np.uint16)[:, rows]
+                worst = max(worst, check_swiglu(hb, g, ag, u, au))
+                continue
             yg = y.cpu().numpy()
             r0 = 0
             for m in group:
                 rows = _rows_for(layer, wl.layers, m.N, every, rng)
-                w = synth.weights_f32_torch(synth.key(seed, wl.wid, layer, wl.mats.index(m),
-                                                      synth.KIND_W), m.N, m.K, DEV)
-                wr = w[torch.as_tensor(rows, device=DEV)].cpu().numpy()
-                del w
-                if wl.fmt == 4:
-                    oc, os_ = oracle.quantize_q4(wr)
-                else:
-                    oc, os_ = oracle.quantize_q8(wr)
+                wr = _regen_rows(wl, seed, layer, m, rows, m.K, m.N)
+                oc, os_ = _quant(wl.fmt, wr)
                 sel = torch.as_tensor(rows + r0, device=DEV)
                 gc = codes_d[sel].cpu().numpy()
                 gs = scales_d[sel].cpu().numpy().view(np.uint16)
                 assert np.array_equal(gc, oc.view(np.uint8)), f"{label} L{layer}: codes differ"
                 assert np.array_equal(gs, os_), f"{label} L{layer}: scales differ"
-                yr, ar = (oracle.gemv_q4 if wl.fmt == 4 else oracle.gemv_q8)(oc, os_, xb, nthreads=8)
+                yr, ar = _gemv(wl.fmt, oc, os_, xb)
                 worst = max(worst, check_tol(yg[:, rows + r0], yr, ar))
                 r0 += m.N
     return worst
