@@ -268,6 +268,20 @@ BQ_API int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t codes_st
                        int32_t topk, float *y, void *ws, size_t ws_bytes,
                        int32_t *dev_status, void *stream);
 
+/* bq_moe_gemv_q4 with an output epilogue (see BQ_EPI_*).  With
+ * BQ_EPI_SWIGLU each expert's planes hold its gate and up projections in
+ * SwiGLU pair order (N = 2F, N a multiple of 16), route_w must be NULL, and y
+ * is fp16 bits [B][topk][F]: per slot h = silu(gate) * up of the slot's
+ * expert, the per-slot input (x_per_slot = 1) of the down projection -- the
+ * routed-expert feed-forward block with its activation fused.  An invalid
+ * slot's h is zero.  Anything else as bq_moe_gemv_q4; a bad epilogue, or
+ * SwiGLU with route_w or with N not a multiple of 16, returns BQ_ERR_SHAPE. */
+BQ_API int32_t bq_moe_gemv_ex(const bq_qmat *Wstack, int32_t E, int64_t codes_stride,
+                              int64_t scales_stride, const uint16_t *x, int32_t x_per_slot,
+                              const int32_t *expert_idx, const float *route_w, int32_t B,
+                              int32_t topk, void *y, int32_t epilogue, void *ws, size_t ws_bytes,
+                              int32_t *dev_status, void *stream);
+
 /* ---------------------------------------------- host-side pack / unpack --- */
 /* All host pointers; no CUDA call is made.  Bit-exact by construction. */
 

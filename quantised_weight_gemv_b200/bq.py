@@ -66,6 +66,8 @@ _SIGS = {
     "bq_moe_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "bq_moe_gemv_q4": (_i32, [_QP, _i32, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _i32, _vp,
                               _vp, _sz, _vp, _vp]),
+    "bq_moe_gemv_ex": (_i32, [_QP, _i32, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _i32,
+                              _vp, _sz, _vp, _vp]),
     "bq_quantize_q8": (_i32, [_vp, _i32, _i32, _vp, _vp]),
     "bq_quantize_q4": (_i32, [_vp, _i32, _i32, _vp, _vp]),
     "bq_dequantize_q8": (_i32, [_vp, _vp, _i32, _i32, _vp]),
@@ -159,13 +161,16 @@ def gemv(fmt: int, W: bq_qmat, x, y, ws, status=None, stream=None, epilogue: int
 
 
 def moe_gemv_q4(Wstack: bq_qmat, E: int, codes_stride: int, scales_stride: int, x,
-                x_per_slot: bool, expert_idx, route_w, y, ws, status=None, stream=None) -> None:
+                x_per_slot: bool, expert_idx, route_w, y, ws, status=None, stream=None,
+                epilogue: int = BQ_EPI_NONE) -> None:
+    """Routed-expert Q4 GEMV (bq_moe_gemv_q4); with epilogue BQ_EPI_SWIGLU,
+    per-slot fp16 h (bq_moe_gemv_ex)."""
     B, topk = expert_idx.shape
-    rc = lib().bq_moe_gemv_q4(ctypes.byref(Wstack), int(E), int(codes_stride), int(scales_stride),
+    rc = lib().bq_moe_gemv_ex(ctypes.byref(Wstack), int(E), int(codes_stride), int(scales_stride),
                               x.data_ptr(), 1 if x_per_slot else 0, expert_idx.data_ptr(),
-                              _ptr(route_w), B, topk, y.data_ptr(), ws.data_ptr(),
+                              _ptr(route_w), B, topk, y.data_ptr(), int(epilogue), ws.data_ptr(),
                               ws.numel() * ws.element_size(), _ptr(status), _stream_ptr(stream))
-    check("bq_moe_gemv_q4", rc)
+    check("bq_moe_gemv_ex", rc)
 
 
 class StepPlan:

@@ -266,8 +266,15 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             for (int i = 0; i < a.mat0.B * a.topk; i++) {
                 if (grp.key[i] != 0x7fffffff)
                     continue;
-                for (int r = threadIdx.x; r < a.mat0.N; r += kThreads)
-                    a.mat0.y[(size_t)i * a.mat0.N + r] = 0.f;
+                if (a.mat0.epi == BQ_EPI_SWIGLU) {
+                    __half *h = reinterpret_cast<__half *>(a.mat0.y);
+                    const int F = a.mat0.N / 2;
+                    for (int r = threadIdx.x; r < F; r += kThreads)
+                        h[(size_t)i * F + r] = __float2half_rn(0.0f);
+                } else {
+                    for (int r = threadIdx.x; r < a.mat0.N; r += kThreads)
+                        a.mat0.y[(size_t)i * a.mat0.N + r] = 0.f;
+                }
             }
         }
         if (threadIdx.x == 0) {
@@ -420,11 +427,12 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     // col 2t+1), (row 16mt+g+8, col 2t), (row 16mt+g+8, col 2t+1).
     auto store_band = [&](int u, int band, const float (&v)[MT][4]) {
         const MatInfo &m = unit_mat(u);
-        if (!MOE && m.epi == BQ_EPI_SWIGLU) {
+        if (m.epi == BQ_EPI_SWIGLU) {
             // SwiGLU pair order: in each 16-row tile, rows 0-7 are gate rows
             // and rows 8-15 the up rows of the same 8 outputs, so this lane
             // holds gate (v[mt][c]) and up (v[mt][2 + c]) of output i for
-            // batch columns 2t + c.  h = silu(g) * u in fp32, stored as fp16.
+            // batch column (or expert-piece slot) 2t + c.  h = silu(g) * u in
+            // fp32, stored as fp16.
             __half *h = reinterpret_cast<__half *>(m.y);
             const int F = m.N / 2;
 #pragma unroll
@@ -435,11 +443,19 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
 #pragma unroll
                 for (int c = 0; c < 2; c++) {
                     const int col = 2 * t + c;
-                    if (col >= m.B)
-                        continue;
+                    int out;   // output row of h
+                    if constexpr (MOE) {
+                        if (col >= grp.piece_count[u])
+                            continue;
+                        out = grp.sorted_slot[grp.piece_first[u] + col];
+                    } else {
+                        if (col >= m.B)
+                            continue;
+                        out = col;
+                    }
                     const float gv = v[mt][c] * unscale<FMT>();
                     const float uv = v[mt][2 + c] * unscale<FMT>();
-                    h[(size_t)col * F + i] = __float2half_rn(gv / (1.0f + expf(-gv)) * uv);
+                    h[(size_t)out * F + i] = __float2half_rn(gv / (1.0f + expf(-gv)) * uv);
                 }
             }
             return;
@@ -1123,9 +1139,21 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
                                   int32_t topk, float *y, void *ws, size_t ws_bytes,
                                   int32_t *dev_status, void *stream)
 {
+    return bq_moe_gemv_ex(Wstack, E, codes_stride, scales_stride, x, x_per_slot, expert_idx,
+                          route_w, B, topk, y, BQ_EPI_NONE, ws, ws_bytes, dev_status, stream);
+}
+
+extern "C" int32_t bq_moe_gemv_ex(const bq_qmat *Wstack, int32_t E, int64_t codes_stride,
+                                  int64_t scales_stride, const uint16_t *x, int32_t x_per_slot,
+                                  const int32_t *expert_idx, const float *route_w, int32_t B,
+                                  int32_t topk, void *y, int32_t epilogue, void *ws,
+                                  size_t ws_bytes, int32_t *dev_status, void *stream)
+{
     int32_t st = check_qmat(Wstack);
     if (st != BQ_OK)
         return st;
+    if (!epilogue_ok(epilogue, Wstack->N) || (epilogue == BQ_EPI_SWIGLU && route_w))
+        return BQ_ERR_SHAPE;
     if (!x || !expert_idx || !y || !ws)
         return BQ_ERR_NULL;
     if (B < 1 || B > 8 || B * topk > kMaxSlots)
@@ -1163,7 +1191,8 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     float *slot_buf = reinterpret_cast<float *>(wsb + counters_bytes(nbands * B * topk) + kPartialsBytes);
     a.mat0.x = reinterpret_cast<const __half *>(x);
-    a.mat0.y = route_w ? slot_buf : y;
+    a.mat0.y = route_w ? slot_buf : static_cast<float *>(y);
+    a.mat0.epi = epilogue;
     a.mat0.N = N;
     a.mat0.K = K;
     a.mat0.B = B;
@@ -1190,7 +1219,8 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
     if (route_w) {
         const float *sb = slot_buf;
         int Bv = B, tk = topk, Nv = N, Ev = E;
-        void *cargs[] = {(void *)&sb, (void *)&expert_idx, (void *)&route_w, &Bv, &tk, &Nv, &Ev, &y};
+        float *yc = static_cast<float *>(y);
+        void *cargs[] = {(void *)&sb, (void *)&expert_idx, (void *)&route_w, &Bv, &tk, &Nv, &Ev, &yc};
         int cg = (B * N + 255) / 256;
         cg = std::max(1, std::min(cg, 4 * std::max(1, device_sm_count())));
         e = launch_pdl((const void *)moe_combine_kernel, dim3(cg), dim3(256), 0, s, cargs);

@@ -73,3 +73,52 @@ def test_step_fused_ffn(fmt, F, H):
         check_swiglu(hb, g, ag, u, au)
         yr, ar = oracle_gemv(fmt, cd, sd, hb)      # down on the h the GPU produced
         check_tol(y.cpu().numpy(), yr, ar)
+
+
+def _expert_ffn(E, F, H, seed):
+    """Per expert: gate / up (F x H) and down (H x F) Q4 planes."""
+    cg, sg, cu, su, cd, sd = [], [], [], [], [], []
+    for e in range(E):
+        for lst_c, lst_s, mid, n, k in ((cg, sg, 0, F, H), (cu, su, 1, F, H), (cd, sd, 2, H, F)):
+            c, s = oracle.quantize_q4(synth.weights_f32(synth.key(seed, 83, e, mid, synth.KIND_W), n, k))
+            lst_c.append(c)
+            lst_s.append(s)
+    return [np.stack(a) for a in (cg, sg, cu, su, cd, sd)]
+
+
+@pytest.mark.parametrize("B,topk,E", [(1, 8, 16), (8, 8, 32), (3, 2, 5)])
+def test_moe_expert_ffn_fused(B, topk, E):
+    """Routed-expert feed-forward block: per-slot gate|up with the SwiGLU
+    epilogue writes h [B][topk][F] (fp16), then down reads it per slot and
+    combines with the routing weights.  One slot id is out of range: its h is
+    zero and the status flags it."""
+    import torch
+    F, H = 96, 512
+    cg, sg, cu, su, cd, sd = _expert_ffn(E, F, H, 7)
+    codes_gu = np.stack([pair_order(cg[e], cu[e]) for e in range(E)])
+    scales_gu = np.stack([pair_order(sg[e], su[e]) for e in range(E)])
+    x = synth.activations_f16_bits(synth.key(7, 83, 0, 0, synth.KIND_X), B, H)
+    idx, r = synth.routing(synth.key(7, 83, 0, 0, synth.KIND_IDX),
+                           synth.key(7, 83, 0, 0, synth.KIND_LOGIT), B, E, topk)
+    idx[B - 1, topk - 1] = E + 3
+    ldS_h, ldS_f = scales_gu.shape[2], sd.shape[2]
+    c1, s1, c2, s2 = (dev(codes_gu.view(np.uint8)), dev(scales_gu), dev(cd.view(np.uint8)), dev(sd))
+    xt, it, rt = dev(x), dev(idx), dev(r)
+    h = torch.full((B, topk, F), float("nan"), dtype=torch.float16, device=DEV)
+    y = torch.full((B, H), float("nan"), dtype=torch.float32, device=DEV)
+    ws1 = bq.workspace(bq.lib().bq_moe_workspace_bytes(2 * F, H, B, topk, E), DEV)
+    ws2 = bq.workspace(bq.lib().bq_moe_workspace_bytes(H, F, B, topk, E), DEV)
+    st = new_status()
+    bq.moe_gemv_q4(bq.qmat(c1, s1, 2 * F, H), E, 2 * F * H // 2, 2 * F * ldS_h, xt, False, it,
+                   None, h, ws1, st, epilogue=bq.BQ_EPI_SWIGLU)
+    bq.moe_gemv_q4(bq.qmat(c2, s2, H, F), E, H * F // 2, H * ldS_f, h, True, it, rt, y, ws2, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 1 << bq.BQ_ERR_EXPERT_INDEX
+    hb = h.cpu().numpy().view(np.uint16)
+    assert np.all(hb[B - 1, topk - 1] == 0)
+    g, ag, bad = oracle.moe_gemv_q4(cg, sg, x, False, idx)
+    u, au, _ = oracle.moe_gemv_q4(cu, su, x, False, idx)
+    assert bad
+    check_swiglu(hb, g, ag, u, au)
+    yr, ar, _ = oracle.moe_gemv_q4(cd, sd, hb, True, idx, r)      # down on the GPU's h
+    check_tol(y.cpu().numpy(), yr, ar)
