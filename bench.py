@@ -339,10 +339,12 @@ class DenseStep:
 
 class MoEStep:
     """A routed-expert decode step resident in HBM: per layer, the expert stack of
-    gate|up (2*ffn x hidden) and of down (hidden x ffn), Q4, all E experts of all
-    layers (~16.3 GB for 48 layers of 128 experts).  One step = per layer the
-    gate|up call (per-slot outputs) and the down call (combined with the routing
-    weights); algorithmic bytes count the distinct routed experts only."""
+    gate|up (2*ffn x hidden, SwiGLU pair order) and of down (hidden x ffn), Q4,
+    all E experts of all layers (~16.3 GB for 48 layers of 128 experts).  One
+    step = per layer the gate|up call, whose SwiGLU epilogue writes each routed
+    slot's h (fp16), and the down call reading h per slot, combined with the
+    routing weights -- the expert feed-forward block with its activation fused.
+    Algorithmic bytes count the distinct routed experts only."""
 
     def __init__(self, wl: synth.MoEWorkload, device, seed: int = 0):
         import torch
@@ -351,12 +353,13 @@ class MoEStep:
         self.B, self.fmt = wl.B, 4
         E, topk, B = wl.E, wl.topk, wl.B
         (Ng, Kg), (Nd, Kd) = wl.gateup(), wl.down()
+        F = Ng // 2
         st = torch.zeros(1, dtype=torch.int32, device=device)
         self.layers = []
         self.bytes_alg = 0
         self.distinct = []
         self._keep = []
-        ins, outs = [], []
+        ins = []
         for layer in range(wl.layers):
             idx, r = synth.routing(synth.key(seed, wl.wid, layer, 0, synth.KIND_IDX),
                                    synth.key(seed, wl.wid, layer, 0, synth.KIND_LOGIT), B, E, topk)
@@ -367,25 +370,32 @@ class MoEStep:
                 scales = torch.empty((E, N, ldS), dtype=torch.int16, device=device)
                 w = synth.weights_f32_torch(synth.key(seed, wl.wid, layer, mid, synth.KIND_W),
                                             E * N, K, device)
-                bq.quantize_dev(4, w, codes.view(E * N, K // 2), scales.view(E * N, ldS), st)
+                if mid == 0:
+                    # expert e: rows [0, F) gate, [F, 2F) up; quantised row by
+                    # row, then interleaved 8 rows at a time (SwiGLU pair order)
+                    ct = torch.empty((E * N, K // 2), dtype=torch.uint8, device=device)
+                    stt = torch.empty((E * N, ldS), dtype=torch.int16, device=device)
+                    bq.quantize_dev(4, w, ct, stt, st)
+                    codes.copy_(ct.view(E, 2, F // 8, 8, K // 2).transpose(1, 2).reshape(E, N, K // 2))
+                    scales.copy_(stt.view(E, 2, F // 8, 8, ldS).transpose(1, 2).reshape(E, N, ldS))
+                    del ct, stt
+                else:
+                    bq.quantize_dev(4, w, codes.view(E * N, K // 2), scales.view(E * N, ldS), st)
                 del w
                 stacks.append((bq.qmat(codes, scales, N, K), N * K // 2, N * ldS))
                 self._keep += [codes, scales]
             x = synth.activations_f16_torch(synth.key(seed, wl.wid, layer, 0, synth.KIND_X),
                                             (B, Kg), device)
-            h = synth.activations_f16_torch(synth.key(seed, wl.wid, layer, 1, synth.KIND_H),
-                                            (B, topk, Kd), device)
-            ins += [x, h]
-            outs += [(B, topk, Ng), (B, Nd)]
+            ins.append(x)
             nd = len(set(idx.ravel().tolist()))
             self.distinct.append(nd)
             self.bytes_alg += (nd * (synth.packed_bytes(4, Ng, Kg) + synth.packed_bytes(4, Nd, Kd))
-                               + x.numel() * 2 + h.numel() * 2 + B * topk * Ng * 4 + B * Nd * 4)
+                               + x.numel() * 2 + 2 * (B * topk * F * 2) + B * Nd * 4)
             self.layers.append([stacks, torch.as_tensor(idx, device=device),
                                 torch.as_tensor(r, device=device)])
-        # Every input of the step (x, per-slot h, expert ids, routing weights)
-        # in one byte buffer and every output in another, 64-byte aligned
-        # slices: one copy each way end to end.
+        # Every input of the step (x, expert ids, routing weights) in one byte
+        # buffer and every output in another, 64-byte aligned slices: one copy
+        # each way end to end.  The per-slot h stay on the device.
         def pack(tensors):
             offs, n = [], 0
             for t in tensors:
@@ -400,13 +410,15 @@ class MoEStep:
             return buf, views
         in_t = []
         for li, L in enumerate(self.layers):
-            in_t += [ins[2 * li], ins[2 * li + 1], L[1], L[2]]
+            in_t += [ins[li], L[1], L[2]]
         self.x_all, iv = pack(in_t)
-        self.y_all, ov = pack([torch.zeros(o, dtype=torch.float32, device=device) for o in outs])
+        self.y_all, ov = pack([torch.zeros((B, Nd), dtype=torch.float32, device=device)
+                               for _ in self.layers])
+        self.h_all = torch.zeros((wl.layers, B, topk, F), dtype=torch.float16, device=device)
         for li, L in enumerate(self.layers):
-            x, h, idx, r = iv[4 * li:4 * li + 4]
+            x, idx, r = iv[3 * li:3 * li + 3]
             L[1], L[2] = idx, r
-            L += [x, h, ov[2 * li], ov[2 * li + 1]]
+            L += [x, self.h_all[li], ov[li]]
         ws = max(bq.lib().bq_moe_workspace_bytes(Ng, Kg, B, topk, E),
                  bq.lib().bq_moe_workspace_bytes(Nd, Kd, B, topk, E))
         self.ws = bq.workspace(ws, device)
@@ -418,10 +430,11 @@ class MoEStep:
 
     def launch(self, stream, only=None):
         E = self.wl.E
-        for stacks, idx, r, x, h, y_gu, y_dn in self.layers:
+        for stacks, idx, r, x, h, y in self.layers:
             (qg, cg, sg), (qd, cd, sd) = stacks
-            self.bq.moe_gemv_q4(qg, E, cg, sg, x, False, idx, None, y_gu, self.ws, self.status, stream)
-            self.bq.moe_gemv_q4(qd, E, cd, sd, h, True, idx, r, y_dn, self.ws, self.status, stream)
+            self.bq.moe_gemv_q4(qg, E, cg, sg, x, False, idx, None, h, self.ws, self.status, stream,
+                                epilogue=self.bq.BQ_EPI_SWIGLU)
+            self.bq.moe_gemv_q4(qd, E, cd, sd, h, True, idx, r, y, self.ws, self.status, stream)
         return self.launches_per_step
 
     def io_tensors(self):
@@ -467,11 +480,10 @@ def moe_oracle_sample(wl: synth.MoEWorkload, seed: int = 0):
         if mid == 0:
             x = synth.activations_f16_bits(synth.key(seed, wl.wid, 0, 0, synth.KIND_X), B, K)
             jobs.append((codes, scales, x, False, idx, None))
-            nbytes += x.size * 2 + B * topk * N * 4
+            nbytes += x.size * 2 + B * topk * (N // 2) * 2
         else:
-            h = synth.activations_f16_bits(synth.key(seed, wl.wid, 0, 1, synth.KIND_H), B, topk, K)
-            jobs.append((codes, scales, h, True, idx, r))
-            nbytes += h.size * 2 + B * N * 4
+            jobs.append((codes, scales, None, True, idx, r))   # x = h of the gate|up job
+            nbytes += B * topk * K * 2 + B * N * 4
         nbytes += len(used) * synth.packed_bytes(4, N, K)
     return jobs, nbytes
 
@@ -484,8 +496,13 @@ def oracle_job(wl):
         jobs, nbytes = moe_oracle_sample(wl)
 
         def run():
-            for codes, scales, x, per_slot, idx, r in jobs:
-                oracle.moe_gemv_q4(codes, scales, x, per_slot, idx, r, nthreads=threads)
+            # gate|up per slot, SwiGLU (gate rows first, up rows second), down
+            # per slot on h, combined with the routing weights
+            (cg, sg, x, _, idx, _), (cd, sd, _, _, _, r) = jobs
+            y, _, _ = oracle.moe_gemv_q4(cg, sg, x, False, idx, None, nthreads=threads)
+            F = y.shape[2] // 2
+            h = oracle.swiglu_f16(y[..., :F], y[..., F:])
+            oracle.moe_gemv_q4(cd, sd, h, True, idx, r, nthreads=threads)
         return run, nbytes
     mats = oracle_sample(wl)
     nbytes = sum(m[3] for m in mats)

@@ -16,7 +16,7 @@ import pytest
 
 import oracle
 from quantised_weight_gemv_b200 import bq, synth
-from tests.gpu_helpers import DEV, check_swiglu, check_tol, dev, new_status
+from tests.gpu_helpers import DEV, check_swiglu, check_tol, dev, new_status, pair_order
 
 pytestmark = pytest.mark.gpu
 
@@ -145,49 +145,56 @@ def test_dense64_h5120_step():
 
 @pytest.mark.parametrize("B", [1, 8])
 def test_moe_layer_full(B):
-    """One routed-expert layer: 128 experts, gate|up 1536 x 2048 per expert
-    (per-slot outputs) and down 2048 x 768 (combined with the routing
-    weights), top-8, every output row of every routed slot."""
+    """Layer 0 of the routed-expert decode step, built exactly as the benchmark
+    builds it (128 experts, gate|up 1536 x 2048 per expert in SwiGLU pair
+    order, down 2048 x 768, top-8): per-slot h = silu(gate) * up of every
+    routed slot, and y = down(h) combined with the routing weights, against
+    the oracle on every routed expert."""
+    import dataclasses
     import torch
-    wl = synth.moe_h2048(B)
-    E, topk, layer = wl.E, wl.topk, 0
-    idx, r = synth.routing(synth.key(0, wl.wid, layer, 0, synth.KIND_IDX),
-                           synth.key(0, wl.wid, layer, 0, synth.KIND_LOGIT), B, E, topk)
-    st = new_status()
-    for part, (N, K) in (("gateup", wl.gateup()), ("down", wl.down())):
-        mid = 0 if part == "gateup" else 1
+    import bench
+    wl = dataclasses.replace(synth.moe_h2048(B), layers=1)
+    step = bench.MoEStep(wl, torch.device(DEV))
+    step.launch(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0
+    E, topk, seed = wl.E, wl.topk, 0
+    (Ng, Kg), (Nd, Kd) = wl.gateup(), wl.down()
+    F = Ng // 2
+    stacks, idx_d, r_d, x_d, h_d, y_d = step.layers[0]
+    idx, r = idx_d.cpu().numpy(), r_d.cpu().numpy()
+    used = sorted(set(idx.ravel().tolist()))
+    planes = []
+    for mid, (N, K) in ((0, (Ng, Kg)), (1, (Nd, Kd))):
+        w = synth.weights_f32_torch(synth.key(seed, wl.wid, 0, mid, synth.KIND_W), E * N, K, DEV)
+        rows = np.concatenate([np.arange(e * N, (e + 1) * N) for e in used])
+        wu = w[torch.as_tensor(rows, device=DEV)].cpu().numpy().reshape(len(used), N, K)
+        del w
         ldS = bq.scales_ld(K)
-        codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=DEV)
-        scales = torch.empty((E, N, ldS), dtype=torch.int16, device=DEV)
-        for e in range(E):
-            w = synth.weights_f32_torch(synth.key(0, wl.wid, layer, mid * 1000 + e, synth.KIND_W),
-                                        N, K, DEV)
-            bq.quantize_dev(4, w, codes[e], scales[e], st)
-        if part == "gateup":
-            x = synth.activations_f16_torch(synth.key(0, wl.wid, layer, 0, synth.KIND_X), (B, K), DEV)
-            per_slot, rr = False, None
-            y = torch.empty((B, topk, N), dtype=torch.float32, device=DEV)
-        else:
-            x = synth.activations_f16_torch(synth.key(0, wl.wid, layer, 1, synth.KIND_H),
-                                            (B, topk, K), DEV)
-            per_slot, rr = True, r
-            y = torch.empty((B, N), dtype=torch.float32, device=DEV)
-        ws = bq.workspace(bq.lib().bq_moe_workspace_bytes(N, K, B, topk, E), DEV)
-        it, rt = dev(idx), dev(rr) if rr is not None else None
-        bq.moe_gemv_q4(bq.qmat(codes, scales, N, K), E, N * K // 2, N * ldS, x, per_slot, it, rt,
-                       y, ws, st)
-        torch.cuda.synchronize()
-        assert int(st.item()) == 0
-        used = sorted(set(idx.ravel().tolist()))
-        oc = np.zeros((E, N, K // 2), dtype=np.uint8)
-        os_ = np.zeros((E, N, ldS), dtype=np.uint16)
-        for e in used:
-            w = synth.weights_f32_torch(synth.key(0, wl.wid, layer, mid * 1000 + e, synth.KIND_W),
-                                        N, K, DEV).cpu().numpy()
-            oc[e], os_[e] = oracle.quantize_q4(w)
-            assert np.array_equal(codes[e].cpu().numpy(), oc[e])
-            assert np.array_equal(scales[e].cpu().numpy().view(np.uint16), os_[e])
-        xb = x.cpu().numpy().view(np.uint16)
-        yr, ar, bad = oracle.moe_gemv_q4(oc, os_, xb, per_slot, idx, rr, nthreads=8)
-        assert not bad
-        check_tol(y.cpu().numpy(), yr, ar)
+        codes_d, scales_d = stacks[mid][0]._refs
+        parts = []
+        for half in ((0, F), (F, 2 * F)) if mid == 0 else ((0, N),):
+            c = np.zeros((E, half[1] - half[0], K // 2), dtype=np.uint8)
+            sc = np.zeros((E, half[1] - half[0], ldS), dtype=np.uint16)
+            for j, e in enumerate(used):
+                c[e], sc[e] = oracle.quantize_q4(wu[j, half[0]:half[1]])
+            parts.append((c, sc))
+        for j, e in enumerate(used):        # the device planes are the oracle's, bit for bit
+            if mid == 0:
+                want_c = pair_order(parts[0][0][e], parts[1][0][e])
+                want_s = pair_order(parts[0][1][e], parts[1][1][e])
+            else:
+                want_c, want_s = parts[0][0][e], parts[0][1][e]
+            assert np.array_equal(codes_d[e].cpu().numpy(), want_c), f"expert {e} codes"
+            assert np.array_equal(scales_d[e].cpu().numpy().view(np.uint16), want_s), f"expert {e} scales"
+        planes.append(parts)
+    xb = x_d.cpu().numpy().view(np.uint16)
+    (cg, sg), (cu, su) = planes[0]
+    g, ag, bad = oracle.moe_gemv_q4(cg, sg, xb, False, idx, nthreads=8)
+    u, au, _ = oracle.moe_gemv_q4(cu, su, xb, False, idx, nthreads=8)
+    assert not bad
+    hb = h_d.cpu().numpy().view(np.uint16)
+    check_swiglu(hb, g, ag, u, au)
+    (cd, sd), = planes[1]
+    yr, ar, _ = oracle.moe_gemv_q4(cd, sd, hb, True, idx, r, nthreads=8)
+    check_tol(y_d.cpu().numpy(), yr, ar)
