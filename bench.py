@@ -316,9 +316,11 @@ class DenseStep:
     def launch_one(self, entry, stream):
         import ctypes
         q, x, y, label, _, epi = entry
+        # the step's weights are resident and never written: each launch may
+        # start loading them while the previous one drains
         rc = self.bq.lib().bq_gemv_ex(self.fmt, ctypes.byref(q), x.data_ptr(), self.B, y.data_ptr(),
-                                      epi, self.ws.data_ptr(), self.ws.numel(),
-                                      self.status.data_ptr(), stream.cuda_stream)
+                                      epi, self.bq.BQ_GEMV_STATIC_WEIGHTS, self.ws.data_ptr(),
+                                      self.ws.numel(), self.status.data_ptr(), stream.cuda_stream)
         if rc != 0:
             raise RuntimeError(f"bq_gemv_ex: {self.bq.bq_status_string(rc)}")
 
@@ -585,9 +587,9 @@ def main():
     ap.add_argument("--impl", default="bq", choices=["bq", "reference"])
     ap.add_argument("--workload", default=synth.DENSE_H2048.name, choices=sorted(WORKLOADS))
     ap.add_argument("--engine", default=None, choices=["step", "graph"],
-                    help="step: one cooperative launch per token (bq_step_run); "
-                         "graph: a CUDA graph of per-matrix bq_gemv launches.  Default: "
-                         "graph for a single matrix and for routed experts, step otherwise")
+                    help="graph (default): a CUDA graph of per-matrix bq_gemv_ex launches "
+                         "with static weights; step: one cooperative launch per token "
+                         "(bq_step_run)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -619,8 +621,11 @@ def main():
         args.engine = "graph"   # one graph of the per-layer expert calls
         step = MoEStep(wl, device)
     else:
-        if args.engine is None:   # one matrix: the plain bq_gemv call
-            args.engine = "graph" if wl.layers == 1 and len(wl.mats) == 1 else "step"
+        if args.engine is None:
+            # the chain of per-matrix launches with static weights: each launch
+            # starts loading its weights while the previous one drains, which
+            # measured faster than the one-launch plan's grid barriers
+            args.engine = "graph"
         step = DenseStep(wl, device)
     stream = torch.cuda.Stream(device)
     peaks = load_peaks()
@@ -685,6 +690,7 @@ def main():
     if int(step.status.item()) != 0:
         raise RuntimeError(f"device status {int(step.status.item()):#x}")
 
+    isolated = None
     if args.engine == "step" or is_moe:
         # the step kernel is the only kernel (one launch per step), or (routed
         # experts) the expert kernel is every launch but the small combine
@@ -693,13 +699,19 @@ def main():
         dom_s = t_dev / args.steps
         dom_bytes = step.bytes_alg
     else:
-        # dominant kernel: its launches timed one by one with events on its stream
-        dom = max(step.bytes_by_label, key=step.bytes_by_label.get)
+        # every launch of the step is the same kernel: its average launch over
+        # the timed region (bytes per launch = step bytes / launches)
+        dom = f"average of the {n_launch} launches of a step"
+        dom_s = t_dev / args.steps / n_launch
+        dom_bytes = step.bytes_alg / n_launch
+        # for reference: the largest projection's launch timed alone (no
+        # neighbour to overlap its start with)
+        big = max(step.bytes_by_label, key=step.bytes_by_label.get)
         durs = []
         with torch.cuda.stream(stream):
             for _ in range(3):
                 for e in step.launches:
-                    if e[3] != dom:
+                    if e[3] != big:
                         continue
                     if flush is not None:
                         flush.zero_()   # a set smaller than the L2: time each call cold
@@ -709,9 +721,10 @@ def main():
                     b.record(stream)
                     durs.append((a, b))
         torch.cuda.synchronize()
-        n_dom = sum(1 for l in step.launches if l[3] == dom)
-        dom_s = statistics.mean(a.elapsed_time(b) for a, b in durs) / 1e3
-        dom_bytes = step.bytes_by_label[dom] / n_dom
+        n_big = sum(1 for l in step.launches if l[3] == big)
+        big_s = statistics.mean(a.elapsed_time(b) for a, b in durs) / 1e3
+        isolated = {"launch": big, "us": round(big_s * 1e6, 3),
+                    "GB/s": round(step.bytes_by_label[big] / n_big / big_s / 1e9, 1)}
     achieved = dom_bytes / dom_s / 1e9
 
     # end to end: pinned host x -> device, step, y -> pinned host, every step
@@ -769,9 +782,10 @@ def main():
             "data": "synthetic (seeded N(0,0.02) weights, N(0,1) fp16 activations)",
             "config": {"workload": wl.name, "batch": wl.B, "layers": wl.layers,
                        "launches_per_step": n_launch, "bytes_per_step": step.bytes_alg,
-                       "engine": ("cuda-graph of per-layer bq_moe_gemv_q4 calls" if is_moe else
+                       "engine": ("cuda-graph of per-layer bq_moe_gemv_ex calls" if is_moe else
                                   "one cooperative launch per step (bq_step_run), graph-captured"
-                                  if args.engine == "step" else "cuda-graph of per-matrix launches"),
+                                  if args.engine == "step" else
+                                  "cuda-graph of per-matrix bq_gemv_ex launches, static weights"),
                        "l2": ("inputs larger than L2 (no flush)" if flush is None else
                               f"L2 flushed before every step ({L2_FLUSH_BYTES >> 20} MB write, untimed); "
                               "steps timed one by one"),
@@ -782,14 +796,14 @@ def main():
             "frac_of_measured_hbm": round(value / world / peaks["hbm_gbs"], 4),
             "frac_of_8TBps": round(value / world / 8000.0, 4),
             "roofline": {"bound": "hbm", "kernel": f"stream_gemv q{step.fmt} ({dom})",
-                         "timed": ("CUDA events over the timed region" if args.engine == "step"
-                                   else "CUDA events around each launch"),
+                         "timed": "CUDA events over the timed region",
                          "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                          "peak_source": peaks["source"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4),
                          "traffic": profiled_traffic(wl.name, args.engine),
                          "bytes_per_launch": int(dom_bytes),
-                         "launch_us": round(dom_s * 1e6, 3)},
+                         "launch_us": round(dom_s * 1e6, 3),
+                         **({"isolated_launch": isolated} if isolated else {})},
             "cpu_baseline": cpu,
             "e2e": {"value": round(job_gbs(world, step.bytes_alg, e2e_steps, t_e2e), 2),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -46,8 +46,11 @@
  *   - Workspace: calls that take `ws` need ws_bytes >= the matching
  *     bq_*_workspace_bytes() value.  The workspace must be zero-filled once
  *     (e.g. cudaMemsetAsync) before its first use; every call that completes
- *     leaves its counters at zero again, so one zero-fill suffices.  Two calls
- *     that may run at the same time must not share a workspace.
+ *     leaves all of it zero again (counters and scratch), so one zero-fill
+ *     suffices and calls of any shapes may use one workspace one after
+ *     another on a stream.  Two calls that may run at the same time must not
+ *     share a workspace.  After a call that reported a timeout the workspace
+ *     must be zero-filled again.
  *   - Errors: the return code covers everything the host can check before
  *     launching (null pointers, shapes, alignment, batch range, workspace
  *     size) and launch failures; nothing is launched when it is not BQ_OK.
@@ -174,15 +177,27 @@ BQ_API int32_t bq_gemv_q4_noalloc(const bq_qmat *W, const uint16_t *x, int32_t B
  *       and rounded to the nearest fp16 -- the input format of the next GEMV. */
 enum { BQ_EPI_NONE = 0, BQ_EPI_SWIGLU = 1 };
 
+/* Flags of bq_gemv_ex.
+ *
+ * BQ_GEMV_STATIC_WEIGHTS: the caller guarantees that no kernel still running
+ * on (or before) the stream writes W's planes.  The launch then starts
+ * streaming the weights as soon as its CTAs are resident -- while the
+ * previous kernel on the stream drains (programmatic dependent launch) --
+ * and waits for that kernel only before it reads x or writes y and the
+ * workspace.  In a chain of per-projection launches (a decode step) this
+ * hides each launch's weight latency behind the previous one's tail. */
+enum { BQ_GEMV_STATIC_WEIGHTS = 1 };
+
 /* Q4 or Q8 decode GEMV with an output epilogue.
  *   fmt        4 or 8
  *   y          device: fp32 [B][N] (BQ_EPI_NONE) or fp16 bits [B][N/2]
  *              (BQ_EPI_SWIGLU, N a multiple of 16), 16-byte aligned
  *   epilogue   BQ_EPI_*; anything else returns BQ_ERR_SHAPE
+ *   flags      0 or BQ_GEMV_STATIC_WEIGHTS; other bits return BQ_ERR_SHAPE
  * Other arguments, errors and launch behaviour as bq_gemv_q4. */
 BQ_API int32_t bq_gemv_ex(int32_t fmt, const bq_qmat *W, const uint16_t *x, int32_t B, void *y,
-                          int32_t epilogue, void *ws, size_t ws_bytes, int32_t *dev_status,
-                          void *stream);
+                          int32_t epilogue, int32_t flags, void *ws, size_t ws_bytes,
+                          int32_t *dev_status, void *stream);
 
 /* --------------------------------------------------------- decode step --- */
 

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libbq.so")
 BQ_OK, BQ_ERR_NULL, BQ_ERR_SHAPE, BQ_ERR_ALIGN, BQ_ERR_BATCH = 0, 1, 2, 3, 4
 BQ_ERR_EXPERT_INDEX, BQ_ERR_CUDA, BQ_ERR_TIMEOUT, BQ_ERR_WORKSPACE, BQ_ERR_RANGE = 5, 6, 7, 8, 9
 BQ_EPI_NONE, BQ_EPI_SWIGLU = 0, 1
+BQ_GEMV_STATIC_WEIGHTS = 1
 
 
 class bq_qmat(ctypes.Structure):
@@ -57,7 +58,7 @@ _SIGS = {
     "bq_scales_ld": (_i32, [_i32]),
     "bq_gemv_workspace_bytes": (_sz, [_i32, _i32]),
     "bq_gemv_q4": (_i32, [_QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
-    "bq_gemv_ex": (_i32, [_i32, _QP, _vp, _i32, _vp, _i32, _vp, _sz, _vp, _vp]),
+    "bq_gemv_ex": (_i32, [_i32, _QP, _vp, _i32, _vp, _i32, _i32, _vp, _sz, _vp, _vp]),
     "bq_gemv_q8": (_i32, [_QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
     "bq_gemv_q4_noalloc": (_i32, [_QP, _vp, _i32, _vp, _vp, _vp]),
     "bq_step_plan_bytes": (_sz, [_i32]),
@@ -144,18 +145,20 @@ def workspace(nbytes: int, device):
     return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)
 
 
-def gemv(fmt: int, W: bq_qmat, x, y, ws, status=None, stream=None, epilogue: int = BQ_EPI_NONE) -> None:
+def gemv(fmt: int, W: bq_qmat, x, y, ws, status=None, stream=None, epilogue: int = BQ_EPI_NONE,
+         flags: int = 0) -> None:
     """y[B, N] (fp32) = deq(W) . x[B, K] (fp16), through bq_gemv_q4 / bq_gemv_q8;
-    with epilogue BQ_EPI_SWIGLU, y is fp16 [B, N/2] through bq_gemv_ex."""
+    with an epilogue (BQ_EPI_SWIGLU: y is fp16 [B, N/2]) or flags, through
+    bq_gemv_ex."""
     B = x.shape[0]
-    if epilogue == BQ_EPI_NONE:
+    if epilogue == BQ_EPI_NONE and flags == 0:
         fn = lib().bq_gemv_q4 if fmt == 4 else lib().bq_gemv_q8
         rc = fn(ctypes.byref(W), x.data_ptr(), B, y.data_ptr(), ws.data_ptr(),
                 ws.numel() * ws.element_size(), _ptr(status), _stream_ptr(stream))
         check(f"bq_gemv_q{fmt}", rc)
         return
     rc = lib().bq_gemv_ex(int(fmt), ctypes.byref(W), x.data_ptr(), B, y.data_ptr(), int(epilogue),
-                          ws.data_ptr(), ws.numel() * ws.element_size(), _ptr(status),
+                          int(flags), ws.data_ptr(), ws.numel() * ws.element_size(), _ptr(status),
                           _stream_ptr(stream))
     check("bq_gemv_ex", rc)
 

@@ -109,6 +109,7 @@ struct KernelArgs {
     int *counters;                   // per band of a stage; zero on entry and exit
     float *partials;                 // [wmax][2][kMT][32 lanes] float4
     int *status;                     // device status word or null
+    int prefill;                     // matrix mode: load weights before the PDL wait
     unsigned *sync;                  // plan mode: [0] arrivals, [64] exits (separate lines)
     // routed experts
     int E, topk, x_per_slot;
@@ -252,8 +253,12 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
 
     pdl_launch_dependents();
     // Everything below reads inputs or writes outputs and the workspace, so it
-    // waits for the previous kernel on the stream to complete.
-    pdl_wait();
+    // waits for the previous kernel on the stream to complete -- except, when
+    // the caller declared the weights static, the first weight loads of the
+    // ring (matrix mode), issued before the wait further down.
+    const bool prefill = !MOE && !PLAN && a.prefill;
+    if (!prefill)
+        pdl_wait();
 
     if constexpr (MOE) {
         if (warp == 0)
@@ -419,9 +424,13 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
 
     // Fill the ring.  Plan mode keeps every slot loading (see the refill
     // below); the other modes run one slot behind, refilling a slot at the
-    // top of the next chunk, after that chunk's x loads are in flight.
-    while (iss_live && issued < (PLAN ? D : D - 1))
+    // top of the next chunk, after that chunk's x loads are in flight -- but
+    // fill every slot when the loads run ahead of the wait for the previous
+    // kernel.
+    while (iss_live && issued < ((PLAN || prefill) ? D : D - 1))
         issue_one();
+    if (prefill)
+        pdl_wait();
 
     // Output of one band: acc[mt] holds (row 16mt+g, col 2t), (row 16mt+g,
     // col 2t+1), (row 16mt+g+8, col 2t), (row 16mt+g+8, col 2t+1).
@@ -566,7 +575,10 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
 #pragma unroll
         for (int mt = 0; mt < MT; mt++)
             acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-        // Two CTAs' partials in flight at a time.
+        // Two CTAs' partials in flight at a time.  Each slot is cleared once
+        // read, so the workspace is all-zero again when the launch ends and
+        // any later call, of any shape, can use it.
+        const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int v = cf; v <= cl; v += 2) {
             const int v1 = min(v + 1, cl);
             const int sl0 = (bs <= v * kWarps * cpw) ? 0 : 1;
@@ -576,6 +588,11 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             for (int mt = 0; mt < MT; mt++) {
                 p0[mt] = __ldcg(part_at(v, sl0, mt));
                 p1[mt] = __ldcg(part_at(v1, sl1, mt));
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; mt++) {
+                __stcg(part_at(v, sl0, mt), zero4);
+                __stcg(part_at(v1, sl1, mt), zero4);
             }
 #pragma unroll
             for (int mt = 0; mt < MT; mt++) {
@@ -763,7 +780,8 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
 
 // y[b][n] = sum_s route_w[b][s] * slot_out[b*topk + s][n], in slot order, over
 // the slots whose expert index is valid.
-__global__ void moe_combine_kernel(const float *slot_out, const int *idx, const float *route_w,
+// Each slot value is cleared once read, leaving the workspace all-zero.
+__global__ void moe_combine_kernel(float *slot_out, const int *idx, const float *route_w,
                                    int B, int topk, int N, int E, float *y)
 {
     pdl_launch_dependents();
@@ -772,10 +790,26 @@ __global__ void moe_combine_kernel(const float *slot_out, const int *idx, const 
     for (int o = blockIdx.x * blockDim.x + threadIdx.x; o < total; o += gridDim.x * blockDim.x) {
         const int b = o / N, nn = o - b * N;
         float s = 0.f;
-        for (int k = 0; k < topk; k++) {
-            const int e = idx[b * topk + k];
-            if (e >= 0 && e < E)
-                s = fmaf(route_w[b * topk + k], slot_out[(size_t)(b * topk + k) * N + nn], s);
+        // eight slots' loads in flight, then their stores of zero
+        for (int k0 = 0; k0 < topk; k0 += 8) {
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int k = k0 + j;
+                const int e = k < topk ? idx[b * topk + k] : -1;
+                v[j] = (e >= 0 && e < E) ? slot_out[(size_t)(b * topk + k) * N + nn] : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const int k = k0 + j;
+                if (k < topk) {
+                    const int e = idx[b * topk + k];
+                    if (e >= 0 && e < E) {
+                        s = fmaf(route_w[b * topk + k], v[j], s);
+                        slot_out[(size_t)(b * topk + k) * N + nn] = 0.f;
+                    }
+                }
+            }
         }
         y[o] = s;
     }
@@ -880,12 +914,12 @@ void fill_stage(StageDesc *st, int mat_begin, int mat_end, long long T, int nban
 
 template <int FMT>
 int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32_t epi,
-                  void *ws, size_t ws_bytes, int32_t *dev_status, void *stream)
+                  int32_t flags, void *ws, size_t ws_bytes, int32_t *dev_status, void *stream)
 {
     int32_t st = check_qmat(W);
     if (st != BQ_OK)
         return st;
-    if (!epilogue_ok(epi, W->N))
+    if (!epilogue_ok(epi, W->N) || (flags & ~BQ_GEMV_STATIC_WEIGHTS) != 0)
         return BQ_ERR_SHAPE;
     if (!x || !y || !ws)
         return BQ_ERR_NULL;
@@ -907,6 +941,7 @@ int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32
     if (!fill_matdesc(FMT, W, x, B, static_cast<float *>(y), &a.mat0))
         return BQ_ERR_CUDA;
     a.mat0.epi = epi;
+    a.prefill = (flags & BQ_GEMV_STATIC_WEIGHTS) ? 1 : 0;
     const long long T = (long long)a.mat0.cpb * a.mat0.nbands;
     const int cap = max_ctas();
     if (cap < 0)
@@ -976,23 +1011,23 @@ extern "C" size_t bq_gemv_workspace_bytes(int32_t N, int32_t K)
 extern "C" int32_t bq_gemv_q4(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void *ws,
                               size_t ws_bytes, int32_t *dev_status, void *stream)
 {
-    return gemv_impl<4>(W, x, B, y, BQ_EPI_NONE, ws, ws_bytes, dev_status, stream);
+    return gemv_impl<4>(W, x, B, y, BQ_EPI_NONE, 0, ws, ws_bytes, dev_status, stream);
 }
 
 extern "C" int32_t bq_gemv_q8(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void *ws,
                               size_t ws_bytes, int32_t *dev_status, void *stream)
 {
-    return gemv_impl<8>(W, x, B, y, BQ_EPI_NONE, ws, ws_bytes, dev_status, stream);
+    return gemv_impl<8>(W, x, B, y, BQ_EPI_NONE, 0, ws, ws_bytes, dev_status, stream);
 }
 
 extern "C" int32_t bq_gemv_ex(int32_t fmt, const bq_qmat *W, const uint16_t *x, int32_t B,
-                              void *y, int32_t epilogue, void *ws, size_t ws_bytes,
+                              void *y, int32_t epilogue, int32_t flags, void *ws, size_t ws_bytes,
                               int32_t *dev_status, void *stream)
 {
     if (fmt == 4)
-        return gemv_impl<4>(W, x, B, y, epilogue, ws, ws_bytes, dev_status, stream);
+        return gemv_impl<4>(W, x, B, y, epilogue, flags, ws, ws_bytes, dev_status, stream);
     if (fmt == 8)
-        return gemv_impl<8>(W, x, B, y, epilogue, ws, ws_bytes, dev_status, stream);
+        return gemv_impl<8>(W, x, B, y, epilogue, flags, ws, ws_bytes, dev_status, stream);
     return BQ_ERR_SHAPE;
 }
 
@@ -1217,7 +1252,7 @@ extern "C" int32_t bq_moe_gemv_ex(const bq_qmat *Wstack, int32_t E, int64_t code
     if (e != cudaSuccess)
         return BQ_ERR_CUDA;
     if (route_w) {
-        const float *sb = slot_buf;
+        float *sb = slot_buf;
         int Bv = B, tk = topk, Nv = N, Ev = E;
         float *yc = static_cast<float *>(y);
         void *cargs[] = {(void *)&sb, (void *)&expert_idx, (void *)&route_w, &Bv, &tk, &Nv, &Ev, &yc};

@@ -151,17 +151,19 @@ def test_gemv_argument_validation_before_launch(fmt):
 def test_gemv_ex_epilogue_validation_before_launch():
     f = bq.lib().bq_gemv_ex
 
-    def rc(fmt=4, N=64, epi=bq.BQ_EPI_SWIGLU):
+    def rc(fmt=4, N=64, epi=bq.BQ_EPI_SWIGLU, flags=0):
         W = bq.bq_qmat(FAKE, FAKE, N, 256)
-        return f(fmt, ctypes.byref(W), FAKE, 1, FAKE, epi, FAKE, 1 << 30, None, None)
+        return f(fmt, ctypes.byref(W), FAKE, 1, FAKE, epi, flags, FAKE, 1 << 30, None, None)
 
     assert rc(fmt=5) == bq.BQ_ERR_SHAPE
+    assert rc(flags=2) == bq.BQ_ERR_SHAPE
+    assert rc(flags=bq.BQ_GEMV_STATIC_WEIGHTS, N=40) == bq.BQ_ERR_SHAPE
     assert rc(epi=2) == bq.BQ_ERR_SHAPE
     assert rc(epi=-1) == bq.BQ_ERR_SHAPE
     assert rc(N=40) == bq.BQ_ERR_SHAPE            # SwiGLU needs whole 16-row gate|up tiles
     W = bq.bq_qmat(FAKE, FAKE, 64, 256)
-    assert f(4, ctypes.byref(W), None, 1, FAKE, bq.BQ_EPI_SWIGLU, FAKE, 1 << 30, None, None) == bq.BQ_ERR_NULL
-    assert f(8, ctypes.byref(W), FAKE, 9, FAKE, bq.BQ_EPI_SWIGLU, FAKE, 1 << 30, None, None) == bq.BQ_ERR_BATCH
+    assert f(4, ctypes.byref(W), None, 1, FAKE, bq.BQ_EPI_SWIGLU, 0, FAKE, 1 << 30, None, None) == bq.BQ_ERR_NULL
+    assert f(8, ctypes.byref(W), FAKE, 9, FAKE, bq.BQ_EPI_SWIGLU, 1, FAKE, 1 << 30, None, None) == bq.BQ_ERR_BATCH
 
 
 def test_moe_argument_validation_before_launch():

@@ -46,7 +46,7 @@ def _gemv(fmt, codes, scales, xb):
     return (oracle.gemv_q4 if fmt == 4 else oracle.gemv_q8)(codes, scales, xb, nthreads=8)
 
 
-def _check_step(wl, every, seed=0):
+def _check_step(wl, every, seed=0, engine="step"):
     """Run the decode step once; check sampled rows of every matrix.  The fused
     feed-forward stage (gate|up in SwiGLU pair order) is checked on its fp16
     output h against the oracle's SwiGLU of the oracle's gate and up GEMVs;
@@ -54,11 +54,16 @@ def _check_step(wl, every, seed=0):
     import torch
     import bench
     step = bench.DenseStep(wl, torch.device(DEV), seed=seed)
-    step.build_plan()
-    st = new_status()
-    step.plan.run(st)
-    torch.cuda.synchronize()
-    assert int(st.item()) == 0 and int(step.status.item()) == 0
+    if engine == "step":
+        step.build_plan()
+        st = new_status()
+        step.plan.run(st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+    else:       # the per-matrix launch chain bench.py's graph engine times
+        step.launch(torch.cuda.current_stream())
+        torch.cuda.synchronize()
+    assert int(step.status.item()) == 0
     rng = np.random.default_rng([seed, wl.wid, 12345])
     stages = bench.fused_stages(wl)
     worst = 0.0
@@ -127,15 +132,17 @@ def test_single_q8_2048_all_rows():
     check_tol(y.cpu().numpy(), yr, ar)
 
 
-def test_dense16_h2048_step():
-    """16-layer decoder (hidden 2048, FFN 8192), Q4, batch 1, as one plan."""
-    _check_step(synth.DENSE_H2048, every=16)
+@pytest.mark.parametrize("engine", ["step", "graph"])
+def test_dense16_h2048_step(engine):
+    """16-layer decoder (hidden 2048, FFN 8192), Q4, batch 1: as one plan, and
+    as the chain of per-matrix launches with static weights."""
+    _check_step(synth.DENSE_H2048, every=16, engine=engine)
 
 
 @pytest.mark.parametrize("fmt", [4, 8])
 def test_dense36_h4096_step_batch8(fmt):
-    """36 distinct copies of a hidden-4096 layer, batch 8, as one plan."""
-    _check_step(synth.dense_h4096(fmt, 8), every=128)
+    """36 distinct copies of a hidden-4096 layer, batch 8, as a launch chain."""
+    _check_step(synth.dense_h4096(fmt, 8), every=128, engine="graph")
 
 
 def test_dense64_h5120_step():

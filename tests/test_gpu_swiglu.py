@@ -46,6 +46,39 @@ def test_gemv_swiglu_epilogue(fmt, F, K, B):
 
 
 @pytest.mark.parametrize("fmt", [4, 8])
+def test_launch_chain_fused_ffn_static_weights(fmt):
+    """The feed-forward block as two back-to-back bq_gemv_ex launches with the
+    static-weights flag (each launch loads weights before waiting for the
+    previous one): down must still read the h gate|up wrote.  Three rounds
+    with different inputs, no host sync in between."""
+    import torch
+    F, H, B = 512, 1024, 3
+    cg, sg, cu, su, _ = _ffn_inputs(fmt, F, H, B, 8)
+    wd = synth.weights_f32(synth.key(8, 82, 0, 2, synth.KIND_W), H, F)
+    cd, sd = _quant(fmt, wd)
+    W1 = bq.qmat(dev(pair_order(cg, cu).view(np.uint8)), dev(pair_order(sg, su)), 2 * F, H)
+    W2 = bq.qmat(dev(cd.view(np.uint8)), dev(sd), H, F)
+    ws = bq.workspace(bq.lib().bq_gemv_workspace_bytes(2 * F, max(H, F)) * 2, DEV)
+    st = new_status()
+    xs = [synth.activations_f16_bits(synth.key(8 + r, 82, 1, 0, synth.KIND_X), B, H) for r in range(3)]
+    hs = [torch.full((B, F), float("nan"), dtype=torch.float16, device=DEV) for _ in range(3)]
+    ys = [torch.full((B, H), float("nan"), dtype=torch.float32, device=DEV) for _ in range(3)]
+    for r in range(3):
+        bq.gemv(fmt, W1, dev(xs[r]), hs[r], ws, st, epilogue=bq.BQ_EPI_SWIGLU,
+                flags=bq.BQ_GEMV_STATIC_WEIGHTS)
+        bq.gemv(fmt, W2, hs[r], ys[r], ws, st, flags=bq.BQ_GEMV_STATIC_WEIGHTS)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for r in range(3):
+        g, ag = oracle_gemv(fmt, cg, sg, xs[r])
+        u, au = oracle_gemv(fmt, cu, su, xs[r])
+        hb = hs[r].cpu().numpy().view(np.uint16)
+        check_swiglu(hb, g, ag, u, au)
+        yr, ar = oracle_gemv(fmt, cd, sd, hb)
+        check_tol(ys[r].cpu().numpy(), yr, ar)
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
 @pytest.mark.parametrize("F,H", [(256, 512), (768, 2048)])
 def test_step_fused_ffn(fmt, F, H):
     """One feed-forward block as a two-stage plan: gate|up + SwiGLU (stage 0)
