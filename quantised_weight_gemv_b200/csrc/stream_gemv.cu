@@ -429,21 +429,42 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     // kernel.
     while (iss_live && issued < ((PLAN || prefill) ? D : D - 1))
         issue_one();
+
+    bool ok = true;
+    int sw[8];
+    lane_swizzle<FMT>(g, sw);
+    // 16 in a register the compiler cannot see through, so the Q4 nibble
+    // placement multiplies on the FMA pipe instead of shifting on the ALU.
+    const uint32_t m16 = launder(16u);
     if (prefill)
         pdl_wait();
 
     // Output of one band: acc[mt] holds (row 16mt+g, col 2t), (row 16mt+g,
     // col 2t+1), (row 16mt+g+8, col 2t), (row 16mt+g+8, col 2t+1).
     auto store_band = [&](int u, int band, const float (&v)[MT][4]) {
-        const MatInfo &m = unit_mat(u);
-        if (m.epi == BQ_EPI_SWIGLU) {
+        // The descriptor fields and this lane's two output columns are read
+        // into registers first: the output pointer is a generic one, so
+        // otherwise every store would force shared-memory reloads.
+        const MatInfo &mref = unit_mat(u);
+        const int N = mref.N, epi = mref.epi;
+        float *const y = mref.y;
+        int out[2];                      // output row of batch column (or piece slot) 2t + c; -1: none
+#pragma unroll
+        for (int c = 0; c < 2; c++) {
+            const int col = 2 * t + c;
+            if constexpr (MOE)
+                out[c] = col < grp.piece_count[u] ? grp.sorted_slot[grp.piece_first[u] + col] : -1;
+            else
+                out[c] = col < mref.B ? col : -1;
+        }
+        if (epi == BQ_EPI_SWIGLU) {
             // SwiGLU pair order: in each 16-row tile, rows 0-7 are gate rows
             // and rows 8-15 the up rows of the same 8 outputs, so this lane
             // holds gate (v[mt][c]) and up (v[mt][2 + c]) of output i for
             // batch column (or expert-piece slot) 2t + c.  h = silu(g) * u in
             // fp32, stored as fp16.
-            __half *h = reinterpret_cast<__half *>(m.y);
-            const int F = m.N / 2;
+            __half *const h = reinterpret_cast<__half *>(y);
+            const int F = N / 2;
 #pragma unroll
             for (int mt = 0; mt < MT; mt++) {
                 const int i = (band * ROWS + 16 * mt) / 2 + g;
@@ -451,20 +472,11 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                     continue;
 #pragma unroll
                 for (int c = 0; c < 2; c++) {
-                    const int col = 2 * t + c;
-                    int out;   // output row of h
-                    if constexpr (MOE) {
-                        if (col >= grp.piece_count[u])
-                            continue;
-                        out = grp.sorted_slot[grp.piece_first[u] + col];
-                    } else {
-                        if (col >= m.B)
-                            continue;
-                        out = col;
-                    }
+                    if (out[c] < 0)
+                        continue;
                     const float gv = v[mt][c] * unscale<FMT>();
                     const float uv = v[mt][2 + c] * unscale<FMT>();
-                    h[(size_t)out * F + i] = __float2half_rn(gv / (1.0f + expf(-gv)) * uv);
+                    h[(size_t)out[c] * F + i] = __float2half_rn(gv / (1.0f + expf(-gv)) * uv);
                 }
             }
             return;
@@ -474,18 +486,9 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
 #pragma unroll
             for (int q = 0; q < 4; q++) {
                 const int row = band * ROWS + 16 * mt + g + ((q & 2) ? 8 : 0);
-                const int col = 2 * t + (q & 1);
-                if (row >= m.N)
-                    continue;
-                if constexpr (MOE) {
-                    if (col < grp.piece_count[u]) {
-                        const int slot = grp.sorted_slot[grp.piece_first[u] + col];
-                        m.y[(size_t)slot * m.N + row] = v[mt][q] * unscale<FMT>();
-                    }
-                } else {
-                    if (col < m.B)
-                        m.y[(size_t)col * m.N + row] = v[mt][q] * unscale<FMT>();
-                }
+                const int o = out[q & 1];
+                if (row < N && o >= 0)
+                    y[(size_t)o * N + row] = v[mt][q] * unscale<FMT>();
             }
         }
     };
@@ -624,7 +627,6 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     // stores) and polls the counter (acquire, short back-off) until all CTAs
     // have arrived, then releases its CTA's warps through a shared mbarrier.
     // Every wait is bounded.
-    bool ok = true;
     auto stage_arrive_and_wait = [&](int s) {
         __syncwarp();
         if (lane == 0) {
@@ -660,11 +662,6 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     int done = 0;                  // chunks consumed (ring index)
     float acc[MT][4];
     int acc_u = -1, acc_band = -1; // band the accumulators belong to
-    int sw[8];
-    lane_swizzle<FMT>(g, sw);
-    // 16 in a register the compiler cannot see through, so the Q4 nibble
-    // placement multiplies on the FMA pipe instead of shifting on the ALU.
-    const uint32_t m16 = launder(16u);
     const __half *xrow = nullptr;
     int nb32 = 0;
 

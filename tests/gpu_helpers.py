@@ -29,8 +29,9 @@ def new_status():
     return torch.zeros(1, dtype=torch.int32, device=DEV)
 
 
-def gpu_gemv(fmt, codes, scales, x_bits, ws=None, status=None):
-    """Run bq_gemv_q{fmt} on numpy planes / fp16 bits; returns fp32 [B, N]."""
+def gpu_gemv(fmt, codes, scales, x_bits, ws=None, status=None, flags=0):
+    """Run bq_gemv_q{fmt} (bq_gemv_ex when flags are given) on numpy planes /
+    fp16 bits; returns fp32 [B, N]."""
     import torch
     N = codes.shape[0]
     K = codes.shape[1] * (2 if fmt == 4 else 1)
@@ -40,7 +41,7 @@ def gpu_gemv(fmt, codes, scales, x_bits, ws=None, status=None):
     y = torch.full((B, N), float("nan"), dtype=torch.float32, device=DEV)
     ws = ws if ws is not None else bq.workspace(bq.lib().bq_gemv_workspace_bytes(N, K), DEV)
     st = status if status is not None else new_status()
-    bq.gemv(fmt, bq.qmat(c, s, N, K), x, y, ws, st)
+    bq.gemv(fmt, bq.qmat(c, s, N, K), x, y, ws, st, flags=flags)
     torch.cuda.synchronize()
     assert int(st.item()) == 0, f"device status {int(st.item()):#x}"
     return y.cpu().numpy()

@@ -31,6 +31,22 @@ def test_gemv_parity_small(fmt, N, K, B):
 
 
 @pytest.mark.parametrize("fmt", [4, 8])
+@pytest.mark.parametrize("N,K", SHAPES)
+@pytest.mark.parametrize("B", [1, 3, 8])
+def test_gemv_static_weights_parity(fmt, N, K, B):
+    """With BQ_GEMV_STATIC_WEIGHTS the weight ring fills before the wait on
+    the previous kernel; the arithmetic is the plain call's, so y is the
+    oracle's within tolerance and bit-identical to the plain call's."""
+    w = synth.weights_f32(synth.key(0, 81, N, K, synth.KIND_W), N, K)
+    codes, scales = quantize(fmt, w)
+    x = synth.activations_f16_bits(synth.key(0, 81, N, K, synth.KIND_X), B, K)
+    y = gpu_gemv(fmt, codes, scales, x, flags=bq.BQ_GEMV_STATIC_WEIGHTS)
+    y_ref, absy = oracle_gemv(fmt, codes, scales, x)
+    check_tol(y, y_ref, absy)
+    assert np.array_equal(y, gpu_gemv(fmt, codes, scales, x))
+
+
+@pytest.mark.parametrize("fmt", [4, 8])
 def test_gemv_one_hot_is_correctly_rounded(fmt):
     """x = e_k returns column k of deq(W); the only rounding is fp32's."""
     N, K = 40, 512
