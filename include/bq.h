@@ -185,15 +185,24 @@ enum { BQ_EPI_NONE = 0, BQ_EPI_SWIGLU = 1 };
  * previous kernel on the stream drains (programmatic dependent launch) --
  * and waits for that kernel only before it reads x or writes y and the
  * workspace.  In a chain of per-projection launches (a decode step) this
- * hides each launch's weight latency behind the previous one's tail. */
-enum { BQ_GEMV_STATIC_WEIGHTS = 1 };
+ * hides each launch's weight latency behind the previous one's tail.
+ *
+ * BQ_GEMV_ROWS16 / BQ_GEMV_ROWS32: the work unit's height for Q4 (the rows
+ * of one chunk of 256 weights along K).  Without either flag the library
+ * picks it per call from N, K and the device's SM count: 32-row chunks take
+ * fewer instructions per weight (two 16-row tiles share each x fragment),
+ * 16-row chunks give twice the work units, which pays when a launch is too
+ * small to give every warp a 32-row chunk.  The result is the same up to
+ * fp32 summation order.  Q8 chunks are always 16 rows: ROWS16 is accepted,
+ * ROWS32 returns BQ_ERR_SHAPE, and so does setting both. */
+enum { BQ_GEMV_STATIC_WEIGHTS = 1, BQ_GEMV_ROWS16 = 2, BQ_GEMV_ROWS32 = 4 };
 
 /* Q4 or Q8 decode GEMV with an output epilogue.
  *   fmt        4 or 8
  *   y          device: fp32 [B][N] (BQ_EPI_NONE) or fp16 bits [B][N/2]
  *              (BQ_EPI_SWIGLU, N a multiple of 16), 16-byte aligned
  *   epilogue   BQ_EPI_*; anything else returns BQ_ERR_SHAPE
- *   flags      0 or BQ_GEMV_STATIC_WEIGHTS; other bits return BQ_ERR_SHAPE
+ *   flags      0 or an OR of BQ_GEMV_*; other bits return BQ_ERR_SHAPE
  * Other arguments, errors and launch behaviour as bq_gemv_q4. */
 BQ_API int32_t bq_gemv_ex(int32_t fmt, const bq_qmat *W, const uint16_t *x, int32_t B, void *y,
                           int32_t epilogue, int32_t flags, void *ws, size_t ws_bytes,

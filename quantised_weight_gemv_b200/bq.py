@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libbq.so")
 BQ_OK, BQ_ERR_NULL, BQ_ERR_SHAPE, BQ_ERR_ALIGN, BQ_ERR_BATCH = 0, 1, 2, 3, 4
 BQ_ERR_EXPERT_INDEX, BQ_ERR_CUDA, BQ_ERR_TIMEOUT, BQ_ERR_WORKSPACE, BQ_ERR_RANGE = 5, 6, 7, 8, 9
 BQ_EPI_NONE, BQ_EPI_SWIGLU = 0, 1
-BQ_GEMV_STATIC_WEIGHTS = 1
+BQ_GEMV_STATIC_WEIGHTS, BQ_GEMV_ROWS16, BQ_GEMV_ROWS32 = 1, 2, 4
 
 
 class bq_qmat(ctypes.Structure):

@@ -41,7 +41,7 @@ constexpr long long kWaitCycles = 4000000000LL;
 
 // Tuning knobs (compile-time; the defaults are the measured best on B200).
 #ifndef BQ_Q4_MT
-#define BQ_Q4_MT 2          // 16-row m-tiles per Q4 chunk
+#define BQ_Q4_MT 2          // 16-row m-tiles per Q4 chunk where no geometry is chosen per call
 #endif
 #ifndef BQ_STAGES
 #define BQ_STAGES 2         // ring slots per worker warp
@@ -50,16 +50,26 @@ constexpr long long kWaitCycles = 4000000000LL;
 #define BQ_MIN_BLOCKS 2     // CTAs per SM the register budget is sized for
 #endif
 
-template <int FMT> struct Fmt;
-template <> struct Fmt<4> {
-    static constexpr int kMT = BQ_Q4_MT;                // m-tiles of 16 rows per chunk
+// Chunk geometry of a format: MT m-tiles of 16 rows.  Q4 comes in two: 32-row
+// chunks (MT = 2, two m-tiles share every x fragment: fewer instructions per
+// weight) and 16-row chunks (MT = 1: twice the work units, for launches too
+// small to give every warp a 32-row chunk).  Q8 chunks are 16 rows.
+template <int FMT>
+__host__ __device__ constexpr int default_mt()
+{
+    return FMT == 4 ? BQ_Q4_MT : 1;
+}
+template <int FMT, int MT = default_mt<FMT>()> struct Fmt;
+template <int MT> struct Fmt<4, MT> {
+    static_assert(MT == 1 || MT == 2, "Q4 chunks are 16 or 32 rows");
+    static constexpr int kMT = MT;                      // m-tiles of 16 rows per chunk
     static constexpr int kRows = 16 * kMT;              // rows per chunk / band
     static constexpr int kBoxes = 1;                    // 128-byte-wide code boxes
-    static constexpr int kCodeBytes = kRows * 128;      // 4 KB
+    static constexpr int kCodeBytes = kRows * 128;      // 2 or 4 KB
     static constexpr int kScaleBytes = kRows * 16;      // kRows x 8 fp16
     static constexpr int kStages = BQ_STAGES;
 };
-template <> struct Fmt<8> {
+template <> struct Fmt<8, 1> {
     static constexpr int kMT = 1;
     static constexpr int kRows = 16;
     static constexpr int kBoxes = 2;
@@ -68,11 +78,11 @@ template <> struct Fmt<8> {
     static constexpr int kStages = BQ_STAGES;
 };
 
-template <int FMT>
+template <int FMT, int MT = default_mt<FMT>()>
 constexpr int smem_bytes()
 {
-    return kWarps * Fmt<FMT>::kStages * (Fmt<FMT>::kCodeBytes + Fmt<FMT>::kScaleBytes) +
-           kWarps * Fmt<FMT>::kStages * 8 + 1024;
+    using F = Fmt<FMT, MT>;
+    return kWarps * F::kStages * (F::kCodeBytes + F::kScaleBytes) + kWarps * F::kStages * 8 + 1024;
 }
 
 // ------------------------------------------------------------------ PTX ----
@@ -446,13 +456,11 @@ __device__ __forceinline__ void chunk_load_x(const __half *xp, int nblk, uint2 (
 // A whole chunk: 8 blocks (nblk of them valid) for the chunk's kMT m-tiles,
 // with the x fragments already loaded.  codes_s / scales_s are the slot's
 // shared addresses, laundered through the slot's mbarrier wait.
-template <int FMT>
+template <int FMT, int MT>
 __device__ __forceinline__ void chunk_mma(uint32_t codes_s, uint32_t scales_s, int nblk, int g,
                                           int t, const int (&sw)[8], const uint2 (&xa)[8],
-                                          const uint2 (&xb)[8], float (&acc)[Fmt<FMT>::kMT][4],
-                                          uint32_t m16)
+                                          const uint2 (&xb)[8], float (&acc)[MT][4], uint32_t m16)
 {
-    constexpr int MT = Fmt<FMT>::kMT;
     uint4 sc[MT][2];
 #pragma unroll
     for (int mt = 0; mt < MT; mt++) {

@@ -185,14 +185,15 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
     return v;
 }
 
-template <int FMT, int MODE>
+template <int FMT, int MODE, int MTQ = default_mt<FMT>()>
 __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(const __grid_constant__ KernelArgs a)
 {
-    constexpr int D = Fmt<FMT>::kStages;
-    constexpr int CB = Fmt<FMT>::kCodeBytes;
-    constexpr int SB = Fmt<FMT>::kScaleBytes;
-    constexpr int MT = Fmt<FMT>::kMT;
-    constexpr int ROWS = Fmt<FMT>::kRows;
+    using F = Fmt<FMT, MTQ>;
+    constexpr int D = F::kStages;
+    constexpr int CB = F::kCodeBytes;
+    constexpr int SB = F::kScaleBytes;
+    constexpr int MT = F::kMT;
+    constexpr int ROWS = F::kRows;
     constexpr uint32_t kTx = CB + SB;
     constexpr bool MOE = MODE == kModeMoE;
     constexpr bool PLAN = MODE == kModePlan;
@@ -402,9 +403,9 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             } else {
                 const MatDesc &m = mats[PLAN ? iss.u : 0];
 #pragma unroll
-                for (int bx = 0; bx < Fmt<FMT>::kBoxes; bx++)
+                for (int bx = 0; bx < F::kBoxes; bx++)
                     tma_load_2d(cdst + bx * (ROWS * 128), &m.tm_codes, bar,
-                                iss.kp * 128 * Fmt<FMT>::kBoxes + bx * 128, row, pol);
+                                iss.kp * 128 * F::kBoxes + bx * 128, row, pol);
                 tma_load_2d(sdst, &m.tm_scales, bar, iss.kp * 8, row, (FMT == 4) ? pol : pol_s);
             }
         }
@@ -713,7 +714,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 // Shared addresses of the slot, ordered after its wait (launder).
                 const uint32_t cs = launder(smem_u32(codes_ring + slot * CB));
                 const uint32_t ss = launder(smem_u32(scales_ring + slot * SB));
-                chunk_mma<FMT>(cs, ss, nblk, g, t, sw, xa, xb, acc, m16);
+                chunk_mma<FMT, MT>(cs, ss, nblk, g, t, sw, xa, xb, acc, m16);
                 done++;
                 // Plan mode: refill the slot just read at once, before any
                 // flush or stage barrier, so the ring always holds the warp's
@@ -816,14 +817,14 @@ __global__ void moe_combine_kernel(float *slot_out, const int *idx, const float 
 namespace {
 
 // Dynamic shared memory of a launch: the rings plus the descriptor cache.
-template <int FMT>
+template <int FMT, int MT = default_mt<FMT>()>
 constexpr size_t launch_smem(int n_stages, int n_mats)
 {
-    return (size_t)smem_bytes<FMT>() + (size_t)kWarps * 2 * Fmt<FMT>::kMT * 32 * sizeof(float4) +
+    return (size_t)smem_bytes<FMT, MT>() + (size_t)kWarps * 2 * MT * 32 * sizeof(float4) +
            (size_t)n_stages * sizeof(StageDesc) + (size_t)n_mats * sizeof(MatInfo);
 }
 
-template <int FMT, int MODE>
+template <int FMT, int MODE, int MT = default_mt<FMT>()>
 int32_t prepare_kernel()
 {
     static bool done[64] = {};
@@ -832,10 +833,10 @@ int32_t prepare_kernel()
         return BQ_ERR_CUDA;
     if (dev >= 0 && dev < 64 && done[dev])
         return BQ_OK;
-    if (cudaFuncSetAttribute((const void *)stream_gemv_kernel<FMT, MODE>,
+    if (cudaFuncSetAttribute((const void *)stream_gemv_kernel<FMT, MODE, MT>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)launch_smem<FMT>(MODE == kModePlan ? kMaxPlanMats : 1,
-                                                   MODE == kModePlan ? kMaxPlanMats : 1)) !=
+                             (int)launch_smem<FMT, MT>(MODE == kModePlan ? kMaxPlanMats : 1,
+                                                       MODE == kModePlan ? kMaxPlanMats : 1)) !=
         cudaSuccess)
         return BQ_ERR_CUDA;
     if (dev >= 0 && dev < 64)
@@ -864,9 +865,14 @@ constexpr CUtensorMapL2promotion kPromoScales = CU_TENSOR_MAP_L2_PROMOTION_NONE;
 
 int rows_of(int fmt) { return fmt == 4 ? Fmt<4>::kRows : Fmt<8>::kRows; }
 
-bool fill_matdesc(int fmt, const bq_qmat *W, const uint16_t *x, int B, float *y, MatDesc *m)
+// R: rows per chunk (the band height), rows_of(fmt) unless a launch chose
+// another Q4 geometry.
+bool fill_matdesc(int fmt, const bq_qmat *W, const uint16_t *x, int B, float *y, MatDesc *m,
+                  int R = 0)
 {
-    const int N = W->N, K = W->K, R = rows_of(fmt);
+    if (R == 0)
+        R = rows_of(fmt);
+    const int N = W->N, K = W->K;
     const uint64_t cdims[2] = {(uint64_t)(fmt == 4 ? K / 2 : K), (uint64_t)N};
     const uint64_t cstr[1] = {(uint64_t)(fmt == 4 ? K / 2 : K)};
     const uint32_t cbox[2] = {128, (uint32_t)R};
@@ -909,33 +915,51 @@ void fill_stage(StageDesc *st, int mat_begin, int mat_end, long long T, int nban
     st->nbands = nbands;
 }
 
-template <int FMT>
-int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32_t epi,
-                  int32_t flags, void *ws, size_t ws_bytes, int32_t *dev_status, void *stream)
+// Q4 chunk height for one matrix launch.  A launch lasts as long as its
+// busiest warp: its chunks, each a chain of dependent loads and mma, plus the
+// sum of any band its range shares -- far dearer once some band's workers
+// span CTAs (workspace partials and a GPU-scope arrival instead of shared
+// memory).  32-row chunks take fewer instructions per weight; 16-row chunks
+// halve a warp's unit of work and a band's split.  Both are estimated with a
+// linear model fitted to launch-chain timings of Q4 shapes from 512 x 2048
+// to 51200 x 5120 at B = 1 and 8 on a B200 (per warp: 0.19 per chunk + 1.15
+// per 16-row tile, + 2.68 when a band crosses CTAs, + 0.35 per 16-row chunk
+// at large B; microseconds), and the cheaper is taken.
+int choose_q4_mt(long long N, long long K, int B, int cap_ctas)
 {
-    int32_t st = check_qmat(W);
-    if (st != BQ_OK)
-        return st;
-    if (!epilogue_ok(epi, W->N) || (flags & ~BQ_GEMV_STATIC_WEIGHTS) != 0)
-        return BQ_ERR_SHAPE;
-    if (!x || !y || !ws)
-        return BQ_ERR_NULL;
-    if (B < 1 || B > 8)
-        return BQ_ERR_BATCH;
-    if (!aligned16(x) || !aligned16(y) || !aligned16(ws))
-        return BQ_ERR_ALIGN;
-    if (ws_bytes < bq_gemv_workspace_bytes(W->N, W->K))
-        return BQ_ERR_WORKSPACE;
-    const long long nbands = (W->N + 15) / 16;
-    if (nbands * ((W->K + kChunkK - 1) / kChunkK) >= (1LL << 31))
-        return BQ_ERR_SHAPE;
-    st = prepare_kernel<FMT, kModeMatrix>();
-    if (st != BQ_OK)
-        return st;
+    const long long cpb = (K + kChunkK - 1) / kChunkK;
+    long long best = 0;
+    int best_mt = 2;
+    for (int mt = 2; mt >= 1; mt--) {
+        const long long nbands = (N + 16 * mt - 1) / (16 * mt);
+        const long long T = nbands * cpb;
+        const long long wmax = std::min<long long>(cap_ctas, T) * kWarps;
+        const long long cpw = std::max<long long>(1, (T + wmax - 1) / wmax);
+        // Workers are numbered CTA-major, so CTA j starts at chunk
+        // j * kWarps * cpw: some band crosses a CTA boundary unless every
+        // boundary is a band boundary.
+        const long long cta_chunks = kWarps * cpw;
+        const bool crosses = cta_chunks < T && cta_chunks % cpb != 0;
+        const long long cost = 19 * cpw + 115 * cpw * mt + (crosses ? 268 : 0) +
+                               ((mt == 1 && B > 4) ? 35 * cpw : 0);
+        if (mt == 2 || cost < best) {
+            best = cost;
+            best_mt = mt;
+        }
+    }
+    return best_mt;
+}
 
+template <int FMT, int MT>
+int32_t gemv_launch(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32_t epi,
+                    int32_t flags, void *ws, int32_t *dev_status, void *stream)
+{
+    int32_t st = prepare_kernel<FMT, kModeMatrix, MT>();
+    if (st != BQ_OK)
+        return st;
     KernelArgs a;
     memset(&a, 0, sizeof(a));
-    if (!fill_matdesc(FMT, W, x, B, static_cast<float *>(y), &a.mat0))
+    if (!fill_matdesc(FMT, W, x, B, static_cast<float *>(y), &a.mat0, Fmt<FMT, MT>::kRows))
         return BQ_ERR_CUDA;
     a.mat0.epi = epi;
     a.prefill = (flags & BQ_GEMV_STATIC_WEIGHTS) ? 1 : 0;
@@ -951,10 +975,48 @@ int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32
     a.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + counters_bytes(a.mat0.nbands));
     a.status = dev_status;
     void *args[] = {&a};
-    cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<FMT, kModeMatrix>, dim3(G),
-                               dim3(kThreads), launch_smem<FMT>(1, 1),
+    cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<FMT, kModeMatrix, MT>, dim3(G),
+                               dim3(kThreads), launch_smem<FMT, MT>(1, 1),
                                static_cast<cudaStream_t>(stream), args);
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+template <int FMT>
+int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32_t epi,
+                  int32_t flags, void *ws, size_t ws_bytes, int32_t *dev_status, void *stream)
+{
+    int32_t st = check_qmat(W);
+    if (st != BQ_OK)
+        return st;
+    constexpr int32_t kKnown = BQ_GEMV_STATIC_WEIGHTS | BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32;
+    const int32_t rows = flags & (BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32);
+    if (!epilogue_ok(epi, W->N) || (flags & ~kKnown) != 0 ||
+        rows == (BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32) || (FMT == 8 && rows == BQ_GEMV_ROWS32))
+        return BQ_ERR_SHAPE;
+    if (!x || !y || !ws)
+        return BQ_ERR_NULL;
+    if (B < 1 || B > 8)
+        return BQ_ERR_BATCH;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(ws))
+        return BQ_ERR_ALIGN;
+    if (ws_bytes < bq_gemv_workspace_bytes(W->N, W->K))
+        return BQ_ERR_WORKSPACE;
+    const long long nbands = (W->N + 15) / 16;
+    if (nbands * ((W->K + kChunkK - 1) / kChunkK) >= (1LL << 31))
+        return BQ_ERR_SHAPE;
+    if constexpr (FMT == 8) {
+        return gemv_launch<8, 1>(W, x, B, y, epi, flags, ws, dev_status, stream);
+    } else {
+        int mt = rows == BQ_GEMV_ROWS16 ? 1 : 2;
+        if (rows == 0) {
+            const int cap = max_ctas();
+            if (cap < 0)
+                return BQ_ERR_CUDA;
+            mt = choose_q4_mt(W->N, W->K, B, cap);
+        }
+        return mt == 1 ? gemv_launch<4, 1>(W, x, B, y, epi, flags, ws, dev_status, stream)
+                       : gemv_launch<4, 2>(W, x, B, y, epi, flags, ws, dev_status, stream);
+    }
 }
 
 template <int FMT>

@@ -156,7 +156,9 @@ def test_gemv_ex_epilogue_validation_before_launch():
         return f(fmt, ctypes.byref(W), FAKE, 1, FAKE, epi, flags, FAKE, 1 << 30, None, None)
 
     assert rc(fmt=5) == bq.BQ_ERR_SHAPE
-    assert rc(flags=2) == bq.BQ_ERR_SHAPE
+    assert rc(flags=8) == bq.BQ_ERR_SHAPE           # unknown flag bit
+    assert rc(flags=bq.BQ_GEMV_ROWS16 | bq.BQ_GEMV_ROWS32) == bq.BQ_ERR_SHAPE
+    assert rc(fmt=8, flags=bq.BQ_GEMV_ROWS32) == bq.BQ_ERR_SHAPE   # Q8 chunks are 16 rows
     assert rc(flags=bq.BQ_GEMV_STATIC_WEIGHTS, N=40) == bq.BQ_ERR_SHAPE
     assert rc(epi=2) == bq.BQ_ERR_SHAPE
     assert rc(epi=-1) == bq.BQ_ERR_SHAPE

@@ -30,6 +30,21 @@ def test_gemv_parity_small(fmt, N, K, B):
     check_tol(y, y_ref, absy)
 
 
+@pytest.mark.parametrize("rows", [16, 32])
+@pytest.mark.parametrize("N,K", SHAPES)
+@pytest.mark.parametrize("B", [1, 3, 8])
+def test_q4_chunk_heights_parity(rows, N, K, B):
+    """Q4 with 16-row and with 32-row work units (BQ_GEMV_ROWS16 / ROWS32):
+    both within the oracle's tolerance."""
+    w = synth.weights_f32(synth.key(0, 82, N, K, synth.KIND_W), N, K)
+    codes, scales = quantize(4, w)
+    x = synth.activations_f16_bits(synth.key(0, 82, N, K, synth.KIND_X), B, K)
+    flag = bq.BQ_GEMV_ROWS16 if rows == 16 else bq.BQ_GEMV_ROWS32
+    y = gpu_gemv(4, codes, scales, x, flags=flag)
+    y_ref, absy = oracle_gemv(4, codes, scales, x)
+    check_tol(y, y_ref, absy)
+
+
 @pytest.mark.parametrize("fmt", [4, 8])
 @pytest.mark.parametrize("N,K", SHAPES)
 @pytest.mark.parametrize("B", [1, 3, 8])

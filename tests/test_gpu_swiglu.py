@@ -25,10 +25,13 @@ def _ffn_inputs(fmt, F, K, B, seed):
     return cg, sg, cu, su, x
 
 
-@pytest.mark.parametrize("fmt", [4, 8])
+@pytest.mark.parametrize("fmt,flags", [(4, 0), (4, bq.BQ_GEMV_ROWS16), (4, bq.BQ_GEMV_ROWS32),
+                                       (8, 0)])
 @pytest.mark.parametrize("F,K", [(8, 256), (24, 800), (200, 2048), (1024, 512)])
 @pytest.mark.parametrize("B", [1, 3, 8])
-def test_gemv_swiglu_epilogue(fmt, F, K, B):
+def test_gemv_swiglu_epilogue(fmt, flags, F, K, B):
+    """The SwiGLU epilogue with either Q4 chunk height (a 16-row tile holds 8
+    gate and the same 8 up rows in both)."""
     import torch
     cg, sg, cu, su, x = _ffn_inputs(fmt, F, K, B, 5)
     codes, scales = pair_order(cg, cu), pair_order(sg, su)
@@ -37,7 +40,7 @@ def test_gemv_swiglu_epilogue(fmt, F, K, B):
     h = torch.full((B, F), float("nan"), dtype=torch.float16, device=DEV)
     ws = bq.workspace(bq.lib().bq_gemv_workspace_bytes(N, K), DEV)
     st = new_status()
-    bq.gemv(fmt, bq.qmat(c, s, N, K), xt, h, ws, st, epilogue=bq.BQ_EPI_SWIGLU)
+    bq.gemv(fmt, bq.qmat(c, s, N, K), xt, h, ws, st, epilogue=bq.BQ_EPI_SWIGLU, flags=flags)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     g, ag = oracle_gemv(fmt, cg, sg, x)
