@@ -29,6 +29,7 @@ namespace bq {
 constexpr int kBlock = 32;          // weights per quantisation block
 constexpr int kChunkK = 256;        // weights along K per chunk
 constexpr int kWarps = BQ_WARPS;    // worker warps per CTA
+constexpr int kMaxCluster = 8;      // CTAs of a cluster (portable limit)
 constexpr int kThreads = kWarps * 32;
 
 // Status bits OR-ed into the caller's device status word (1 << bq_status).
@@ -42,6 +43,9 @@ constexpr long long kWaitCycles = 4000000000LL;
 // Tuning knobs (compile-time; the defaults are the measured best on B200).
 #ifndef BQ_Q4_MT
 #define BQ_Q4_MT 2          // 16-row m-tiles per Q4 chunk where no geometry is chosen per call
+#endif
+#ifndef BQ_CLUSTER_SUMS
+#define BQ_CLUSTER_SUMS 1   // matrix mode: cross-CTA band sums through a cluster's shared memory
 #endif
 #ifndef BQ_STAGES
 #define BQ_STAGES 2         // ring slots per worker warp
@@ -121,6 +125,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// The same wait with cluster-scope acquire: for data other CTAs of the
+// cluster stored into this CTA's shared memory (st_async_v4).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Pass a value through an opaque volatile asm: anything computed from the
 // result is ordered after every earlier volatile asm (e.g. an mbarrier wait),
 // even when it is itself a non-volatile asm with no memory clobber.
@@ -138,6 +157,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
         return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kWaitCycles)
+            return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait_cluster(bar, parity)) {
         if (clock64() - t0 > kWaitCycles)
             return false;
     }
@@ -176,6 +205,40 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
         ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z), "l"(policy)
         : "memory");
+}
+
+// ------------------------------------------------------------ clusters ----
+__device__ __forceinline__ uint32_t cluster_nctarank()
+{
+    uint32_t n;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+    return n;
+}
+// Every thread of every CTA of the cluster arrives (release) and waits
+// (acquire): shared-memory state set up before it is visible cluster-wide.
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+                 ::: "memory");
+}
+__device__ __forceinline__ void fence_mbarrier_init_cluster()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// The shared::cluster address of `addr` (a shared::cta address) in the CTA
+// of cluster rank `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+// 16 bytes into another CTA's shared memory; completes 16 bytes of that
+// CTA's mbarrier transaction count.
+__device__ __forceinline__ void st_async_v4(uint32_t remote, float4 v, uint32_t remote_bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(remote), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(remote_bar) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
@@ -404,6 +467,14 @@ __device__ __forceinline__ uint4 lds128_u32(uint32_t addr)
     uint4 v;
     asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float4 lds128_f32(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
     return v;
 }
 

@@ -29,9 +29,10 @@ bool encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank,
                        const uint32_t *box, CUtensorMapSwizzle swizzle,
                        CUtensorMapL2promotion promotion);
 
-// Launch `kernel` with the programmatic-dependent-launch attribute.
+// Launch `kernel` with the programmatic-dependent-launch attribute, as
+// clusters of `cluster` CTAs along x when cluster > 1 (grid.x a multiple).
 cudaError_t launch_pdl(const void *kernel, dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t stream, void **args);
+                       cudaStream_t stream, void **args, int cluster = 1);
 
 // Validation of a plane-layout matrix whose planes are device pointers.
 int32_t check_qmat(const bq_qmat *W);

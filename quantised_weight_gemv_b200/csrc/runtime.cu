@@ -66,18 +66,26 @@ bool encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank, co
 }
 
 cudaError_t launch_pdl(const void *kernel, dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t stream, void **args)
+                       cudaStream_t stream, void **args, int cluster)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    int n = 1;
+    if (cluster > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = (unsigned)cluster;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        n = 2;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = n;
     return cudaLaunchKernelExC(&cfg, kernel, args);
 }
 

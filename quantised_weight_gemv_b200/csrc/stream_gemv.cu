@@ -185,7 +185,7 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
     return v;
 }
 
-template <int FMT, int MODE, int MTQ = default_mt<FMT>()>
+template <int FMT, int MODE, int MTQ = default_mt<FMT>(), bool CL = false>
 __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(const __grid_constant__ KernelArgs a)
 {
     using F = Fmt<FMT, MTQ>;
@@ -203,6 +203,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     __shared__ int cta_arrivals;
     __shared__ int local_ctr[kWarps];   // arrivals of CTA-local split bands
     __shared__ alignas(8) uint64_t stage_bar;
+    __shared__ alignas(8) uint64_t cl_bar;   // CL: cross-CTA partials received
 
     uint8_t *sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -217,6 +218,12 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     StageDesc *stg = reinterpret_cast<StageDesc *>(local_part + kWarps * 2 * MT * 32);
     const int n_stages = PLAN ? a.n_stages : 1;
     MatInfo *minfo = reinterpret_cast<MatInfo *>(stg + n_stages);
+    // CL (matrix mode, launched as clusters whose boundaries are band
+    // boundaries): the partials other CTAs of the cluster send for the band
+    // this CTA finishes, [sender - this CTA - 1][mt][lane] float4, after the
+    // descriptor cache (one matrix).
+    static_assert(!CL || MODE == kModeMatrix, "cluster sums are a matrix-mode path");
+    const uint32_t cl_recv = CL ? (smem_u32(minfo + 1) + 15u) / 16u * 16u : 0u;
     const MatDesc *mats = PLAN ? a.mats : &a.mat0;   // tensor maps stay in global / param space
     {
         const int n_m = PLAN ? a.n_mats : 1;
@@ -248,6 +255,10 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     if (PLAN && threadIdx.x == 0) {
         cta_arrivals = 0;
         mbar_init(smem_u32(&stage_bar), 1);
+    }
+    if (CL && threadIdx.x == 0) {
+        mbar_init(smem_u32(&cl_bar), 1);
+        fence_mbarrier_init_cluster();
     }
     if (lane == 0)
         fence_barrier_init();
@@ -296,6 +307,10 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
         __syncthreads();
     } else {
         __syncthreads();
+        // Every CTA's receive barrier is initialised before any CTA of the
+        // cluster can send to it.
+        if constexpr (CL)
+            cluster_sync_all();
     }
 
     // Workers are numbered CTA-major, so a band split among consecutive
@@ -556,10 +571,57 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             store_band(u, band, acc);
             return;
         }
+        const int cf = wf / kWarps, cl = wl / kWarps;
+        if constexpr (CL) {
+            // Level 2 inside the cluster (the host launches clusters only when
+            // no band crosses one): the band's other CTAs store their partial
+            // straight into the shared memory of its first CTA, which waits
+            // for them, adds all in CTA order and stores y.  Each CTA finishes
+            // at most one such band (its last one) and sends for at most one
+            // (its first one), so one receive area and one mbarrier phase per
+            // launch suffice.
+            const uint32_t C = cluster_nctarank();
+            const uint32_t first_rank = (uint32_t)cf % C;
+            if (blockIdx.x != (unsigned)cf) {
+                const uint32_t slot = cl_recv + ((uint32_t)(blockIdx.x - cf - 1) * MT * 32 + lane) * 16;
+                const uint32_t rbar = mapa_shared(smem_u32(&cl_bar), first_rank);
+#pragma unroll
+                for (int mt = 0; mt < MT; mt++)
+                    st_async_v4(mapa_shared(slot + mt * 512, first_rank),
+                                make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]), rbar);
+                return;
+            }
+            if (lane == 0)
+                mbar_arrive_expect_tx(smem_u32(&cl_bar), (uint32_t)((cl - cf) * MT * 512));
+            if (!__all_sync(0xffffffffu, mbar_wait_cluster_bounded(smem_u32(&cl_bar), 0u))) {
+                if (lane == 0 && a.status)
+                    atomicOr(a.status, kStatusTimeout);
+                return;
+            }
+            float sum[MT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; mt++) {
+                sum[mt][0] = 0.f + acc[mt][0];
+                sum[mt][1] = 0.f + acc[mt][1];
+                sum[mt][2] = 0.f + acc[mt][2];
+                sum[mt][3] = 0.f + acc[mt][3];
+            }
+            for (int v = cf + 1; v <= cl; v++) {
+#pragma unroll
+                for (int mt = 0; mt < MT; mt++) {
+                    const float4 p = lds128_f32(cl_recv + (((uint32_t)(v - cf - 1) * MT + mt) * 32 + lane) * 16);
+                    sum[mt][0] += p.x;
+                    sum[mt][1] += p.y;
+                    sum[mt][2] += p.z;
+                    sum[mt][3] += p.w;
+                }
+            }
+            store_band(u, band, sum);
+            return;
+        }
         // Level 2, the band continues in other CTAs: one partial per CTA
         // through the workspace and a counted arrival; the last CTA to arrive
         // adds the partials in CTA order, stores y and resets the counter.
-        const int cf = wf / kWarps, cl = wl / kWarps;
         const int cslot = (bs <= cta_first * cpw) ? 0 : 1;
 #pragma unroll
         for (int mt = 0; mt < MT; mt++)
@@ -818,13 +880,14 @@ namespace {
 
 // Dynamic shared memory of a launch: the rings plus the descriptor cache.
 template <int FMT, int MT = default_mt<FMT>()>
-constexpr size_t launch_smem(int n_stages, int n_mats)
+constexpr size_t launch_smem(int n_stages, int n_mats, bool cl = false)
 {
     return (size_t)smem_bytes<FMT, MT>() + (size_t)kWarps * 2 * MT * 32 * sizeof(float4) +
-           (size_t)n_stages * sizeof(StageDesc) + (size_t)n_mats * sizeof(MatInfo);
+           (size_t)n_stages * sizeof(StageDesc) + (size_t)n_mats * sizeof(MatInfo) +
+           (cl ? 16 + (size_t)(kMaxCluster - 1) * MT * 32 * sizeof(float4) : 0);
 }
 
-template <int FMT, int MODE, int MT = default_mt<FMT>()>
+template <int FMT, int MODE, int MT = default_mt<FMT>(), bool CL = false>
 int32_t prepare_kernel()
 {
     static bool done[64] = {};
@@ -833,10 +896,10 @@ int32_t prepare_kernel()
         return BQ_ERR_CUDA;
     if (dev >= 0 && dev < 64 && done[dev])
         return BQ_OK;
-    if (cudaFuncSetAttribute((const void *)stream_gemv_kernel<FMT, MODE, MT>,
+    if (cudaFuncSetAttribute((const void *)stream_gemv_kernel<FMT, MODE, MT, CL>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)launch_smem<FMT, MT>(MODE == kModePlan ? kMaxPlanMats : 1,
-                                                       MODE == kModePlan ? kMaxPlanMats : 1)) !=
+                                                       MODE == kModePlan ? kMaxPlanMats : 1, CL)) !=
         cudaSuccess)
         return BQ_ERR_CUDA;
     if (dev >= 0 && dev < 64)
@@ -950,13 +1013,47 @@ int choose_q4_mt(long long N, long long K, int B, int cap_ctas)
     return best_mt;
 }
 
+// Cluster size for a matrix launch whose bands would be summed across CTAs:
+// the smallest C in {2, 4, 8} that makes every cluster boundary a band
+// boundary (C * kWarps * cpw chunks a multiple of the chunks per band), so
+// that every cross-CTA sum stays inside one cluster, and for which the grid
+// (rounded up to a multiple of C, at most `cap` CTAs) divides into clusters.
+// 1 when the launch needs no cross-CTA sums or no such C exists.  *G is
+// rounded up accordingly; the extra CTAs have no chunks (cpw is unchanged:
+// it is 1 whenever G < cap).
+int cluster_for(long long T, long long cpb, long long cpw, int *G, int cap)
+{
+    const long long cta_chunks = kWarps * cpw;
+    if (!(cta_chunks < T && cta_chunks % cpb != 0))
+        return 1;
+    for (int c = 2; c <= kMaxCluster; c *= 2) {
+        const int Gc = (*G + c - 1) / c * c;
+        if (Gc <= cap && (c * cta_chunks) % cpb == 0) {
+            *G = Gc;
+            return c;
+        }
+    }
+    return 1;
+}
+
+template <int FMT, int MT, bool CL>
+int32_t gemv_launch_as(const KernelArgs &a0, int G, int C, void *stream)
+{
+    int32_t st = prepare_kernel<FMT, kModeMatrix, MT, CL>();
+    if (st != BQ_OK)
+        return st;
+    KernelArgs a = a0;
+    void *args[] = {&a};
+    cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<FMT, kModeMatrix, MT, CL>, dim3(G),
+                               dim3(kThreads), launch_smem<FMT, MT>(1, 1, CL),
+                               static_cast<cudaStream_t>(stream), args, C);
+    return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
 template <int FMT, int MT>
 int32_t gemv_launch(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32_t epi,
                     int32_t flags, void *ws, int32_t *dev_status, void *stream)
 {
-    int32_t st = prepare_kernel<FMT, kModeMatrix, MT>();
-    if (st != BQ_OK)
-        return st;
     KernelArgs a;
     memset(&a, 0, sizeof(a));
     if (!fill_matdesc(FMT, W, x, B, static_cast<float *>(y), &a.mat0, Fmt<FMT, MT>::kRows))
@@ -967,18 +1064,30 @@ int32_t gemv_launch(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int
     const int cap = max_ctas();
     if (cap < 0)
         return BQ_ERR_CUDA;
-    const int G = (int)std::min<long long>(cap, T);
+    int G = (int)std::min<long long>(cap, T);
     a.wmax = G * kWarps;
     fill_stage(&a.stage0, 0, 1, T, a.mat0.nbands, a.wmax);
+    const int cpw = a.stage0.cpw;
+    const int C = BQ_CLUSTER_SUMS ? cluster_for(T, a.mat0.cpb, cpw, &G, cap) : 1;
+    if (C > 1) {
+        a.wmax = G * kWarps;
+        fill_stage(&a.stage0, 0, 1, T, a.mat0.nbands, a.wmax);
+        if (a.stage0.cpw != cpw)
+            return BQ_ERR_CUDA;   // cannot happen: cpw is 1 whenever G grew
+    }
     a.n_stages = 1;
     a.counters = static_cast<int *>(ws);
     a.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + counters_bytes(a.mat0.nbands));
     a.status = dev_status;
-    void *args[] = {&a};
-    cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<FMT, kModeMatrix, MT>, dim3(G),
-                               dim3(kThreads), launch_smem<FMT, MT>(1, 1),
-                               static_cast<cudaStream_t>(stream), args);
-    return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+    if (C > 1) {
+        const int32_t st = gemv_launch_as<FMT, MT, true>(a, G, C, stream);
+        if (st == BQ_OK)
+            return st;
+        // The device could not place the clusters: sum across CTAs through
+        // the workspace instead (same results).
+        (void)cudaGetLastError();
+    }
+    return gemv_launch_as<FMT, MT, false>(a, G, 1, stream);
 }
 
 template <int FMT>

@@ -45,6 +45,26 @@ def test_q4_chunk_heights_parity(rows, N, K, B):
     check_tol(y, y_ref, absy)
 
 
+@pytest.mark.parametrize("fmt,N,K,rows", [(4, 2048, 8192, 32), (4, 2000, 8192, 32),
+                                          (4, 4096, 4096, 32), (4, 1024, 16384, 32),
+                                          (4, 2048, 8192, 16), (8, 1024, 8192, 16)])
+@pytest.mark.parametrize("B", [1, 3, 8])
+def test_bands_summed_across_ctas_in_clusters(fmt, N, K, rows, B):
+    """Shapes whose bands are split among several CTAs (each band's chunks
+    outnumber a CTA's warps) with cluster boundaries on band boundaries: the
+    launch runs as clusters of 2, 4 or 8 CTAs and sums each band's CTA
+    partials in the shared memory of its first CTA."""
+    w = synth.weights_f32(synth.key(0, 83, N, K, synth.KIND_W), N, K)
+    codes, scales = quantize(fmt, w)
+    x = synth.activations_f16_bits(synth.key(0, 83, N, K, synth.KIND_X), B, K)
+    flag = bq.BQ_GEMV_ROWS16 if rows == 16 else bq.BQ_GEMV_ROWS32
+    y = gpu_gemv(fmt, codes, scales, x, flags=flag)
+    y_ref, absy = oracle_gemv(fmt, codes, scales, x)
+    check_tol(y, y_ref, absy)
+    # and the same call again: every receive area and barrier starts clean
+    assert np.array_equal(y, gpu_gemv(fmt, codes, scales, x, flags=flag))
+
+
 @pytest.mark.parametrize("fmt", [4, 8])
 @pytest.mark.parametrize("N,K", SHAPES)
 @pytest.mark.parametrize("B", [1, 3, 8])
