@@ -1014,26 +1014,73 @@ int choose_q4_mt(long long N, long long K, int B, int cap_ctas)
 }
 
 // Cluster size for a matrix launch whose bands would be summed across CTAs:
-// the smallest C in {2, 4, 8} that makes every cluster boundary a band
-// boundary (C * kWarps * cpw chunks a multiple of the chunks per band), so
-// that every cross-CTA sum stays inside one cluster, and for which the grid
-// (rounded up to a multiple of C, at most `cap` CTAs) divides into clusters.
-// 1 when the launch needs no cross-CTA sums or no such C exists.  *G is
-// rounded up accordingly; the extra CTAs have no chunks (cpw is unchanged:
-// it is 1 whenever G < cap).
-int cluster_for(long long T, long long cpb, long long cpw, int *G, int cap)
+// the smallest C in {2, 4, 8} that makes every cluster boundary a band boundary
+// (C * kWarps * cpw chunks a multiple of the chunks per band), so that every
+// cross-CTA sum stays inside one cluster.  The grid shrinks to the CTAs that
+// have chunks, rounded up to a multiple of C (no more than `cap`); the
+// chunks per worker stay the same, and the device must hold all those
+// clusters at once (`resident(C)`): a second wave would cost far more than
+// the sums save.  (Clusters of 3, 5, 6 or 7, which the rule would also
+// allow, measured slower than the workspace sums on full-device launches:
+// 5 CTAs at 2 per SM leave SM slots that neither cluster can use.)  1 when
+// the launch needs no cross-CTA sums or no C works.  *G becomes the grid of
+// the chosen C.
+template <class Resident>
+int cluster_for(long long T, long long cpb, long long cpw, int *G, int cap, Resident resident)
 {
     const long long cta_chunks = kWarps * cpw;
     if (!(cta_chunks < T && cta_chunks % cpb != 0))
         return 1;
+    const long long busy = ((T + cpw - 1) / cpw + kWarps - 1) / kWarps;   // CTAs with chunks
     for (int c = 2; c <= kMaxCluster; c *= 2) {
-        const int Gc = (*G + c - 1) / c * c;
-        if (Gc <= cap && (c * cta_chunks) % cpb == 0) {
-            *G = Gc;
+        const long long Gc = (busy + c - 1) / c * c;
+        if (Gc > cap)
+            continue;
+        const long long wmax = Gc * kWarps;
+        if (std::max<long long>(1, (T + wmax - 1) / wmax) != cpw)
+            continue;
+        if ((c * cta_chunks) % cpb == 0 && (long long)resident(c) * c >= Gc) {
+            *G = (int)Gc;
             return c;
         }
     }
     return 1;
+}
+
+// Clusters of C CTAs of the cluster-sum kernel the device holds at once
+// (cached per device and C; 0 if the query fails).
+template <int FMT, int MT>
+int resident_clusters(int C)
+{
+    static int cache[64][kMaxCluster + 1];
+    static bool known[64][kMaxCluster + 1];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || C < 1 || C > kMaxCluster)
+        return 0;
+    if (known[dev][C])
+        return cache[dev][C];
+    int n = 0;
+    if (prepare_kernel<FMT, kModeMatrix, MT, true>() == BQ_OK) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(C * kMaxCtas);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = launch_smem<FMT, MT>(1, 1, true);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, (const void *)stream_gemv_kernel<FMT, kModeMatrix, MT, true>,
+                                           &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();
+            n = 0;
+        }
+    }
+    cache[dev][C] = n;
+    known[dev][C] = true;
+    return n;
 }
 
 template <int FMT, int MT, bool CL>
@@ -1068,12 +1115,14 @@ int32_t gemv_launch(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int
     a.wmax = G * kWarps;
     fill_stage(&a.stage0, 0, 1, T, a.mat0.nbands, a.wmax);
     const int cpw = a.stage0.cpw;
-    const int C = BQ_CLUSTER_SUMS ? cluster_for(T, a.mat0.cpb, cpw, &G, cap) : 1;
+    const int C = BQ_CLUSTER_SUMS ? cluster_for(T, a.mat0.cpb, cpw, &G, cap,
+                                                [](int c) { return resident_clusters<FMT, MT>(c); })
+                                  : 1;
     if (C > 1) {
         a.wmax = G * kWarps;
         fill_stage(&a.stage0, 0, 1, T, a.mat0.nbands, a.wmax);
         if (a.stage0.cpw != cpw)
-            return BQ_ERR_CUDA;   // cannot happen: cpw is 1 whenever G grew
+            return BQ_ERR_CUDA;   // cannot happen: cluster_for keeps cpw
     }
     a.n_stages = 1;
     a.counters = static_cast<int *>(ws);
