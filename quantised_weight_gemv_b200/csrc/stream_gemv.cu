@@ -492,7 +492,10 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                         continue;
                     const float gv = v[mt][c] * unscale<FMT>();
                     const float uv = v[mt][2 + c] * unscale<FMT>();
-                    h[(size_t)out[c] * F + i] = __float2half_rn(gv / (1.0f + expf(-gv)) * uv);
+                    // silu(g) * u with the fast exp and divide (a few fp32
+                    // ulp, far below the fp16 rounding that follows); for g
+                    // below about -88 the divisor is inf and the result 0.
+                    h[(size_t)out[c] * F + i] = __float2half_rn(__fdividef(gv, 1.0f + __expf(-gv)) * uv);
                 }
             }
             return;
@@ -726,6 +729,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     float acc[MT][4];
     int acc_u = -1, acc_band = -1; // band the accumulators belong to
     const __half *xrow = nullptr;
+    int pf_blocks = 0;             // x prefetch: next chunk's blocks, 0 when the rows would crowd L1
     int nb32 = 0;
 
     for (int s = 0; s < n_stages; s++) {
@@ -750,6 +754,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                         xrow = m.x + (size_t)(a.x_per_slot ? sl : sl / a.topk) * m.K;
                     } else {
                         xrow = m.x + (size_t)min(g, m.B - 1) * m.K;
+                        pf_blocks = m.B <= 2 ? 8 : 0;
                     }
                 }
                 acc_u = cur.u;
@@ -760,9 +765,17 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             // later chunk into the slot freed last round, then this chunk's
             // weights.  Called with a literal nblk of 8 for full chunks, so
             // their code has no per-block bounds.
-            auto one_chunk = [&](const __half *xp, int nblk) -> bool {
+            auto one_chunk = [&](const __half *xp, int nblk, int next_nblk) -> bool {
                 uint2 xa[8], xb[8];
                 chunk_load_x<PLAN>(xp, nblk, xa, xb);
+                // The run's next chunk (next_nblk blocks, 0: none): pull its
+                // x into L1 now, so its loads do not wait a full L2 round
+                // trip after this chunk's compute.  Lane t fetches the
+                // 128-byte line t of its row's 512 bytes.  Only for B <= 2:
+                // L1 is what shared memory leaves (~28 KB an SM), and 16
+                // warps' next chunks at B = 8 (64 KB) measured slower.
+                if (2 * t < min(next_nblk, pf_blocks))
+                    prefetch_l1(xp + kChunkK + 60 * t);
                 if (!PLAN && iss_live && issued < done + D) {
                     __syncwarp();
                     issue_one();
@@ -797,9 +810,9 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             const int nfull = (cur.kp + run == cur.cpb && tail < 8) ? run - 1 : run;
             const __half *xp = xrow + cur.kp * kChunkK + 4 * t;
             for (int i = 0; i < nfull && ok; i++, xp += kChunkK)
-                ok = one_chunk(xp, 8);
+                ok = one_chunk(xp, 8, i + 1 < nfull ? 8 : (nfull < run ? tail : 0));
             if (ok && nfull < run)
-                ok = one_chunk(xp, tail);
+                ok = one_chunk(xp, tail, 0);
             if (!ok)
                 break;
             // Step the cursor past the run (its last step may change band,
