@@ -1393,7 +1393,7 @@ extern "C" size_t bq_moe_workspace_bytes(int32_t N, int32_t K, int32_t B, int32_
     if (N < 1 || K < 32 || K % 32 != 0 || B < 1 || B > 8 || topk < 1 || B * topk > kMaxSlots ||
         E < 1 || E > 65535)
         return 0;
-    const long long nbands = (N + Fmt<4>::kRows - 1) / Fmt<4>::kRows;
+    const long long nbands = (N + 15) / 16;   // the finest band height (16-row chunks)
     return counters_bytes(nbands * B * topk) + kPartialsBytes +
            align_up((size_t)B * topk * N * sizeof(float), 256);
 }
@@ -1407,6 +1407,76 @@ extern "C" int32_t bq_moe_gemv_q4(const bq_qmat *Wstack, int32_t E, int64_t code
     return bq_moe_gemv_ex(Wstack, E, codes_stride, scales_stride, x, x_per_slot, expert_idx,
                           route_w, B, topk, y, BQ_EPI_NONE, ws, ws_bytes, dev_status, stream);
 }
+
+namespace bq {
+namespace {
+template <int MT>
+int32_t moe_launch(const bq_qmat *Wstack, int32_t E, int64_t codes_stride, int64_t scales_stride,
+                   const uint16_t *x, int32_t x_per_slot, const int32_t *expert_idx,
+                   const float *route_w, int32_t B, int32_t topk, void *y, int32_t epilogue,
+                   void *ws, int32_t *dev_status, void *stream, int G)
+{
+    constexpr int R = Fmt<4, MT>::kRows;
+    const int N = Wstack->N, K = Wstack->K, ldS = bq_scales_ld(K);
+    const long long nbands = (N + R - 1) / R;
+    const long long cpb = (K + kChunkK - 1) / kChunkK;
+    int32_t st = prepare_kernel<4, kModeMoE, MT>();
+    if (st != BQ_OK)
+        return st;
+
+    KernelArgs a;
+    memset(&a, 0, sizeof(a));
+    const uint64_t cdims[3] = {(uint64_t)(K / 2), (uint64_t)N, (uint64_t)E};
+    const uint64_t cstr[2] = {(uint64_t)(K / 2), (uint64_t)codes_stride};
+    const uint32_t cbox[3] = {128, (uint32_t)R, 1};
+    const uint64_t sdims[3] = {(uint64_t)(K / 32), (uint64_t)N, (uint64_t)E};
+    const uint64_t sstr[2] = {(uint64_t)ldS * 2, (uint64_t)scales_stride * 2};
+    const uint32_t sbox[3] = {8, (uint32_t)R, 1};
+    if (!encode_tensor_map(&a.mat0.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, Wstack->codes,
+                           cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B, kPromoCodes) ||
+        !encode_tensor_map(&a.mat0.tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, Wstack->scales,
+                           sdims, sstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE, kPromoScales))
+        return BQ_ERR_CUDA;
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    float *slot_buf = reinterpret_cast<float *>(wsb + counters_bytes(nbands * B * topk) + kPartialsBytes);
+    a.mat0.x = reinterpret_cast<const __half *>(x);
+    a.mat0.y = route_w ? slot_buf : static_cast<float *>(y);
+    a.mat0.epi = epilogue;
+    a.mat0.N = N;
+    a.mat0.K = K;
+    a.mat0.B = B;
+    a.mat0.cpb = (int)cpb;
+    a.mat0.nbands = (int)nbands;
+    a.wmax = G * kWarps;
+    a.n_stages = 1;
+    a.counters = reinterpret_cast<int *>(wsb);
+    a.partials = reinterpret_cast<float *>(wsb + counters_bytes(nbands * B * topk));
+    a.status = dev_status;
+    a.E = E;
+    a.topk = topk;
+    a.x_per_slot = x_per_slot ? 1 : 0;
+    a.idx = expert_idx;
+    void *args[] = {&a};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<4, kModeMoE, MT>, dim3(G),
+                               dim3(kThreads), launch_smem<4, MT>(1, 1), s, args);
+    if (e != cudaSuccess)
+        return BQ_ERR_CUDA;
+    if (route_w) {
+        float *sb = slot_buf;
+        int Bv = B, tk = topk, Nv = N, Ev = E;
+        float *yc = static_cast<float *>(y);
+        void *cargs[] = {(void *)&sb, (void *)&expert_idx, (void *)&route_w, &Bv, &tk, &Nv, &Ev, &yc};
+        int cg = (B * N + 255) / 256;
+        cg = std::max(1, std::min(cg, 4 * std::max(1, device_sm_count())));
+        e = launch_pdl((const void *)moe_combine_kernel, dim3(cg), dim3(256), 0, s, cargs);
+        if (e != cudaSuccess)
+            return BQ_ERR_CUDA;
+    }
+    return BQ_OK;
+}
+}  // namespace
+}  // namespace bq
 
 extern "C" int32_t bq_moe_gemv_ex(const bq_qmat *Wstack, int32_t E, int64_t codes_stride,
                                   int64_t scales_stride, const uint16_t *x, int32_t x_per_slot,
@@ -1432,68 +1502,23 @@ extern "C" int32_t bq_moe_gemv_ex(const bq_qmat *Wstack, int32_t E, int64_t code
         return BQ_ERR_ALIGN;
     if (ws_bytes < bq_moe_workspace_bytes(N, K, B, topk, E))
         return BQ_ERR_WORKSPACE;
-    const long long nbands = (N + Fmt<4>::kRows - 1) / Fmt<4>::kRows;
     const long long cpb = (K + kChunkK - 1) / kChunkK;
-    if ((long long)B * topk * nbands * cpb >= (1LL << 31))
+    if ((long long)B * topk * ((N + 15) / 16) * cpb >= (1LL << 31))
         return BQ_ERR_SHAPE;
-    st = prepare_kernel<4, kModeMoE>();
-    if (st != BQ_OK)
-        return st;
-
-    KernelArgs a;
-    memset(&a, 0, sizeof(a));
-    const uint64_t cdims[3] = {(uint64_t)(K / 2), (uint64_t)N, (uint64_t)E};
-    const uint64_t cstr[2] = {(uint64_t)(K / 2), (uint64_t)codes_stride};
-    const uint32_t cbox[3] = {128, (uint32_t)Fmt<4>::kRows, 1};
-    const uint64_t sdims[3] = {(uint64_t)(K / 32), (uint64_t)N, (uint64_t)E};
-    const uint64_t sstr[2] = {(uint64_t)ldS * 2, (uint64_t)scales_stride * 2};
-    const uint32_t sbox[3] = {8, (uint32_t)Fmt<4>::kRows, 1};
-    if (!encode_tensor_map(&a.mat0.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, Wstack->codes,
-                           cdims, cstr, cbox, CU_TENSOR_MAP_SWIZZLE_128B, kPromoCodes) ||
-        !encode_tensor_map(&a.mat0.tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, Wstack->scales,
-                           sdims, sstr, sbox, CU_TENSOR_MAP_SWIZZLE_NONE, kPromoScales))
-        return BQ_ERR_CUDA;
-    uint8_t *wsb = static_cast<uint8_t *>(ws);
-    float *slot_buf = reinterpret_cast<float *>(wsb + counters_bytes(nbands * B * topk) + kPartialsBytes);
-    a.mat0.x = reinterpret_cast<const __half *>(x);
-    a.mat0.y = route_w ? slot_buf : static_cast<float *>(y);
-    a.mat0.epi = epilogue;
-    a.mat0.N = N;
-    a.mat0.K = K;
-    a.mat0.B = B;
-    a.mat0.cpb = (int)cpb;
-    a.mat0.nbands = (int)nbands;
     const int G = max_ctas();
     if (G < 0)
         return BQ_ERR_CUDA;
-    a.wmax = G * kWarps;
-    a.n_stages = 1;
-    a.counters = reinterpret_cast<int *>(wsb);
-    a.partials = reinterpret_cast<float *>(wsb + counters_bytes(nbands * B * topk));
-    a.status = dev_status;
-    a.E = E;
-    a.topk = topk;
-    a.x_per_slot = x_per_slot ? 1 : 0;
-    a.idx = expert_idx;
-    void *args[] = {&a};
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<4, kModeMoE>, dim3(G),
-                               dim3(kThreads), launch_smem<4>(1, 1), s, args);
-    if (e != cudaSuccess)
-        return BQ_ERR_CUDA;
-    if (route_w) {
-        float *sb = slot_buf;
-        int Bv = B, tk = topk, Nv = N, Ev = E;
-        float *yc = static_cast<float *>(y);
-        void *cargs[] = {(void *)&sb, (void *)&expert_idx, (void *)&route_w, &Bv, &tk, &Nv, &Ev, &yc};
-        int cg = (B * N + 255) / 256;
-        cg = std::max(1, std::min(cg, 4 * std::max(1, device_sm_count())));
-        e = launch_pdl((const void *)moe_combine_kernel, dim3(cg), dim3(256), 0, s, cargs);
-        if (e != cudaSuccess)
-            return BQ_ERR_CUDA;
-    }
-    return BQ_OK;
+    // Chunk height as for one matrix, over the rows of the routed experts'
+    // pieces (at most B * topk of them, one per distinct expert and up to 8
+    // slots each).
+    const long long pieces = std::min<long long>((long long)B * topk, E);
+    const int mt = choose_q4_mt((long long)N * pieces, K, 1, G);
+    return mt == 1 ? moe_launch<1>(Wstack, E, codes_stride, scales_stride, x, x_per_slot, expert_idx,
+                                   route_w, B, topk, y, epilogue, ws, dev_status, stream, G)
+                   : moe_launch<2>(Wstack, E, codes_stride, scales_stride, x, x_per_slot, expert_idx,
+                                   route_w, B, topk, y, epilogue, ws, dev_status, stream, G);
 }
+
 
 // ------------------------------------------------- Q4 GEMV without workspace --
 // Some callers cannot hand the library a workspace: code embedded in a host
