@@ -197,6 +197,32 @@ enum { BQ_EPI_NONE = 0, BQ_EPI_SWIGLU = 1 };
  * ROWS32 returns BQ_ERR_SHAPE, and so does setting both. */
 enum { BQ_GEMV_STATIC_WEIGHTS = 1, BQ_GEMV_ROWS16 = 2, BQ_GEMV_ROWS32 = 4 };
 
+/* The launch geometry bq_gemv_ex chooses for one matrix (nothing is
+ * launched).  Work is cut into chunks of `rows` rows x 256 weights along K;
+ * a band (the rows of one chunk height) has chunks_per_band of them, and
+ * workers (warps, 8 per CTA) take chunks_per_worker consecutive chunks each.
+ *   sm_count   > 0: computed for a device with that many SMs, assuming it
+ *              holds every cluster grid at once (no device is touched);
+ *              0: the current device, as bq_gemv_ex would launch on it
+ *   out        host pointer, filled on BQ_OK
+ * Arguments fmt, N, K, B, flags as bq_gemv_ex; errors as its validation
+ * (BQ_ERR_SHAPE, BQ_ERR_BATCH, BQ_ERR_NULL), BQ_ERR_CUDA if sm_count is 0
+ * and no device can be queried. */
+typedef struct bq_gemv_geometry {
+    int32_t rows;               /* rows per chunk: 16 or 32 (Q4), 16 (Q8) */
+    int32_t chunks;             /* bands x chunks_per_band */
+    int32_t chunks_per_band;    /* ceil(K / 256) */
+    int32_t chunks_per_worker;
+    int32_t grid;               /* CTAs launched */
+    int32_t cluster;            /* CTAs per thread-block cluster; 1: no clusters */
+    int32_t cross_cta_bands;    /* 1: some band's chunks span CTAs (summed across CTAs:
+                                   inside its cluster when cluster > 1, else through the
+                                   workspace) */
+    int32_t reserved;
+} bq_gemv_geometry;
+BQ_API int32_t bq_gemv_geometry_of(int32_t fmt, int32_t N, int32_t K, int32_t B, int32_t flags,
+                                   int32_t sm_count, bq_gemv_geometry *out);
+
 /* Q4 or Q8 decode GEMV with an output epilogue.
  *   fmt        4 or 8
  *   y          device: fp32 [B][N] (BQ_EPI_NONE) or fp16 bits [B][N/2]

@@ -40,6 +40,12 @@ class bq_step_info(ctypes.Structure):
                 ("ws_bytes", ctypes.c_uint64)]
 
 
+class bq_gemv_geometry(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("rows", "chunks", "chunks_per_band",
+                                               "chunks_per_worker", "grid", "cluster",
+                                               "cross_cta_bands", "reserved")]
+
+
 class BQError(RuntimeError):
     def __init__(self, fn: str, status: int):
         super().__init__(f"{fn}: {bq_status_string(status)} ({status})")
@@ -62,6 +68,7 @@ _SIGS = {
     "bq_gemv_q8": (_i32, [_QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
     "bq_gemv_q4_noalloc": (_i32, [_QP, _vp, _i32, _vp, _vp, _vp]),
     "bq_step_plan_bytes": (_sz, [_i32]),
+    "bq_gemv_geometry_of": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp]),
     "bq_step_plan": (_i32, [_i32, _SMP, _i32, _vp, _sz, _SIP]),
     "bq_step_run": (_i32, [_SIP, _vp, _vp, _sz, _vp, _vp]),
     "bq_moe_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
@@ -133,6 +140,15 @@ def qmat(codes, scales, N: int, K: int) -> bq_qmat:
     m = bq_qmat(codes.data_ptr(), scales.data_ptr(), int(N), int(K))
     m._refs = (codes, scales)
     return m
+
+
+def gemv_geometry(fmt: int, N: int, K: int, B: int, flags: int = 0, sm_count: int = 0) -> dict:
+    """The launch geometry bq_gemv_ex chooses (bq_gemv_geometry_of); with
+    sm_count > 0 computed for such a device without touching one."""
+    g = bq_gemv_geometry()
+    check("bq_gemv_geometry_of",
+          lib().bq_gemv_geometry_of(fmt, N, K, B, flags, sm_count, ctypes.byref(g)))
+    return {n: getattr(g, n) for n, _ in bq_gemv_geometry._fields_ if n != "reserved"}
 
 
 def scales_ld(K: int) -> int:

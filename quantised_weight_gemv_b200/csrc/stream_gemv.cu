@@ -1060,6 +1060,38 @@ int cluster_for(long long T, long long cpb, long long cpw, int *G, int cap, Resi
     return 1;
 }
 
+// Launch geometry of one matrix: chunk height, the stream-K split, the grid
+// and the cluster size.  `cap` is the CTA limit of a launch (2 per SM);
+// `resident(mt, C)` the clusters of C CTAs the device holds at once.
+struct Geometry {
+    int mt;                 // 16-row m-tiles per chunk
+    long long nbands, cpb, T;
+    int cpw, G, C;
+    bool crosses;           // some band's chunks span CTAs (before clusters)
+};
+
+template <class Resident>
+Geometry matrix_geometry(int fmt, long long N, long long K, int B, int32_t rows_flag, int cap,
+                         Resident resident)
+{
+    Geometry g;
+    g.mt = fmt == 8 ? 1
+                    : rows_flag == BQ_GEMV_ROWS16 ? 1
+                    : rows_flag == BQ_GEMV_ROWS32 ? 2 : choose_q4_mt(N, K, B, cap);
+    g.nbands = (N + 16 * g.mt - 1) / (16 * g.mt);
+    g.cpb = (K + kChunkK - 1) / kChunkK;
+    g.T = g.nbands * g.cpb;
+    g.G = (int)std::min<long long>(cap, g.T);
+    const long long wmax = (long long)g.G * kWarps;
+    g.cpw = (int)std::max<long long>(1, (g.T + wmax - 1) / wmax);
+    g.crosses = (long long)kWarps * g.cpw < g.T && ((long long)kWarps * g.cpw) % g.cpb != 0;
+    const int mt = g.mt;
+    g.C = BQ_CLUSTER_SUMS ? cluster_for(g.T, g.cpb, g.cpw, &g.G, cap,
+                                        [&](int c) { return resident(mt, c); })
+                          : 1;
+    return g;
+}
+
 // Clusters of C CTAs of the cluster-sum kernel the device holds at once
 // (cached per device and C; 0 if the query fails).
 template <int FMT, int MT>
@@ -1112,7 +1144,7 @@ int32_t gemv_launch_as(const KernelArgs &a0, int G, int C, void *stream)
 
 template <int FMT, int MT>
 int32_t gemv_launch(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32_t epi,
-                    int32_t flags, void *ws, int32_t *dev_status, void *stream)
+                    int32_t flags, void *ws, int32_t *dev_status, void *stream, const Geometry &geo)
 {
     KernelArgs a;
     memset(&a, 0, sizeof(a));
@@ -1121,22 +1153,11 @@ int32_t gemv_launch(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int
     a.mat0.epi = epi;
     a.prefill = (flags & BQ_GEMV_STATIC_WEIGHTS) ? 1 : 0;
     const long long T = (long long)a.mat0.cpb * a.mat0.nbands;
-    const int cap = max_ctas();
-    if (cap < 0)
-        return BQ_ERR_CUDA;
-    int G = (int)std::min<long long>(cap, T);
+    const int G = geo.G, C = geo.C;
     a.wmax = G * kWarps;
     fill_stage(&a.stage0, 0, 1, T, a.mat0.nbands, a.wmax);
-    const int cpw = a.stage0.cpw;
-    const int C = BQ_CLUSTER_SUMS ? cluster_for(T, a.mat0.cpb, cpw, &G, cap,
-                                                [](int c) { return resident_clusters<FMT, MT>(c); })
-                                  : 1;
-    if (C > 1) {
-        a.wmax = G * kWarps;
-        fill_stage(&a.stage0, 0, 1, T, a.mat0.nbands, a.wmax);
-        if (a.stage0.cpw != cpw)
-            return BQ_ERR_CUDA;   // cannot happen: cluster_for keeps cpw
-    }
+    if (a.stage0.cpw != geo.cpw)
+        return BQ_ERR_CUDA;   // cannot happen: the geometry was computed for this shape
     a.n_stages = 1;
     a.counters = static_cast<int *>(ws);
     a.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + counters_bytes(a.mat0.nbands));
@@ -1175,18 +1196,20 @@ int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32
     const long long nbands = (W->N + 15) / 16;
     if (nbands * ((W->K + kChunkK - 1) / kChunkK) >= (1LL << 31))
         return BQ_ERR_SHAPE;
+    const int cap = max_ctas();
+    if (cap < 0)
+        return BQ_ERR_CUDA;
+    const Geometry geo = matrix_geometry(FMT, W->N, W->K, B, rows, cap, [](int mt, int c) {
+        if constexpr (FMT == 8)
+            return resident_clusters<8, 1>(c);
+        else
+            return mt == 1 ? resident_clusters<4, 1>(c) : resident_clusters<4, 2>(c);
+    });
     if constexpr (FMT == 8) {
-        return gemv_launch<8, 1>(W, x, B, y, epi, flags, ws, dev_status, stream);
+        return gemv_launch<8, 1>(W, x, B, y, epi, flags, ws, dev_status, stream, geo);
     } else {
-        int mt = rows == BQ_GEMV_ROWS16 ? 1 : 2;
-        if (rows == 0) {
-            const int cap = max_ctas();
-            if (cap < 0)
-                return BQ_ERR_CUDA;
-            mt = choose_q4_mt(W->N, W->K, B, cap);
-        }
-        return mt == 1 ? gemv_launch<4, 1>(W, x, B, y, epi, flags, ws, dev_status, stream)
-                       : gemv_launch<4, 2>(W, x, B, y, epi, flags, ws, dev_status, stream);
+        return geo.mt == 1 ? gemv_launch<4, 1>(W, x, B, y, epi, flags, ws, dev_status, stream, geo)
+                           : gemv_launch<4, 2>(W, x, B, y, epi, flags, ws, dev_status, stream, geo);
     }
 }
 
@@ -1236,6 +1259,45 @@ extern "C" size_t bq_gemv_workspace_bytes(int32_t N, int32_t K)
         return 0;
     const long long nbands = (N + 15) / 16;   // the finest band height of any format
     return counters_bytes(nbands) + kPartialsBytes;
+}
+
+extern "C" int32_t bq_gemv_geometry_of(int32_t fmt, int32_t N, int32_t K, int32_t B,
+                                       int32_t flags, int32_t sm_count, bq_gemv_geometry *out)
+{
+    if (!out)
+        return BQ_ERR_NULL;
+    const int32_t rows = flags & (BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32);
+    constexpr int32_t kKnown = BQ_GEMV_STATIC_WEIGHTS | BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32;
+    if ((fmt != 4 && fmt != 8) || N < 1 || K < 32 || K % 32 != 0 || (flags & ~kKnown) != 0 ||
+        rows == (BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32) || (fmt == 8 && rows == BQ_GEMV_ROWS32) ||
+        sm_count < 0)
+        return BQ_ERR_SHAPE;
+    if (B < 1 || B > 8)
+        return BQ_ERR_BATCH;
+    Geometry g;
+    if (sm_count > 0) {
+        // a device of sm_count SMs that holds any cluster grid at once
+        const int cap = std::min(BQ_MIN_BLOCKS * sm_count, kMaxCtas);
+        g = matrix_geometry(fmt, N, K, B, rows, cap, [](int, int) { return kMaxCtas; });
+    } else {
+        const int cap = max_ctas();
+        if (cap < 0)
+            return BQ_ERR_CUDA;
+        g = fmt == 4 ? matrix_geometry(4, N, K, B, rows, cap, [](int mt, int c) {
+                return mt == 1 ? resident_clusters<4, 1>(c) : resident_clusters<4, 2>(c);
+            })
+                     : matrix_geometry(8, N, K, B, rows, cap,
+                                       [](int, int c) { return resident_clusters<8, 1>(c); });
+    }
+    out->rows = 16 * g.mt;
+    out->chunks = (int32_t)g.T;
+    out->chunks_per_band = (int32_t)g.cpb;
+    out->chunks_per_worker = g.cpw;
+    out->grid = g.G;
+    out->cluster = g.C;
+    out->cross_cta_bands = g.crosses ? 1 : 0;
+    out->reserved = 0;
+    return BQ_OK;
 }
 
 extern "C" int32_t bq_gemv_q4(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void *ws,
