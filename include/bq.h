@@ -126,7 +126,11 @@ BQ_API size_t bq_gemv_workspace_bytes(int32_t N, int32_t K);
  *   stream     cudaStream_t
  * The launch carries the programmatic-dependent-launch attribute: its CTAs
  * may become resident while the previous kernel on the stream drains, and
- * they read or write no memory before that kernel has completed. */
+ * they read or write no memory before that kernel has completed.  The work
+ * unit height and whether bands summed across CTAs run as thread-block
+ * clusters are chosen per call from N, K, B and the device
+ * (bq_gemv_geometry_of reports the choice); y is deterministic for a given
+ * device and shape. */
 BQ_API int32_t bq_gemv_q4(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
                    void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
 

@@ -9,8 +9,9 @@
 // keep HBM busy with the packed weight bytes and read each of them once.
 //
 // Work decomposition (stream-K over chunks).  A matrix is cut into bands of
-// kRows rows (32 for Q4, 16 for Q8) and a band into chunks of 256 weights
-// along K; chunks are numbered band-major.  Every warp of the grid is an
+// kRows rows (16 for Q8; 32 or 16 for Q4, chosen per launch by
+// choose_q4_mt) and a band into chunks of 256 weights along K; chunks are
+// numbered band-major.  Every warp of the grid is an
 // independent worker that owns a ring of shared-memory slots with its own
 // mbarriers; its lane 0 keeps TMA loads of the warp's next chunks in flight
 // in every slot but the one being read (in a decode step, in every slot: a
@@ -25,10 +26,16 @@
 // worker order; if the band continues in other CTAs, that CTA partial goes to
 // the workspace with a counted arrival, and the last CTA to arrive adds the
 // CTA partials in CTA order, writes y and resets the counter.  No worker waits
-// for another.
+// for another.  When the launch runs as thread-block clusters whose
+// boundaries are band boundaries (cluster_for), the CTA partials go instead
+// straight into the shared memory of the band's first CTA, which waits for
+// them and adds them in the same order.
 //
 // Three modes share that worker loop:
-//  - one matrix (bq_gemv_q4 / _q8): its descriptor is a kernel parameter;
+//  - one matrix (bq_gemv_q4 / _q8 / _ex): its descriptor is a kernel
+//    parameter; a chain of such launches is a decode step too, each launch
+//    loading its first weights while the previous one drains (programmatic
+//    dependent launch, BQ_GEMV_STATIC_WEIGHTS);
 //  - a decode step (bq_step_run): a plan in device memory lists matrices in
 //    stages; stage s+1 may read what stage s wrote (in a model, the next
 //    projection's input), so the persistent, co-resident grid passes a grid
@@ -38,7 +45,7 @@
 //    and dispatch cost the pages single out for small models (gist.science
 //    technical summary, "Resultaten" and "Kernel Fusie") becomes one launch
 //    per token;
-//  - routed experts (bq_moe_gemv_q4): every CTA sorts the (token, slot) ->
+//  - routed experts (bq_moe_gemv_q4 / _ex): every CTA sorts the (token, slot) ->
 //    expert list (at most 64 entries) in shared memory, which gives the same
 //    grouping on every CTA without a separate kernel; each distinct expert,
 //    cut into pieces of at most 8 routed slots (the mma's N), becomes one
