@@ -21,6 +21,15 @@
  * formats (abstract; technical summary "Belangrijkste Bijdragen").  The
  * definitions used here are the workload definitions that accompany them.
  *
+ * Q6 (a third format of the same family; the pages list formats from Q2 to
+ * FP16 without defining them): 32-element blocks along K, one fp16 scale
+ * d = absmax/31, code q = clamp(round(w/d)+32, 0, 63), weight d*(q-32).  A
+ * row of codes is 3K/4 bytes: first a low-nibble plane laid out exactly as Q4
+ * (block j at byte 16j; byte i holds the low 4 bits of element i, and in its
+ * high nibble those of element i+16), then a 2-bit plane (block j at byte
+ * K/2 + 8j; byte i holds the top 2 bits of elements i, i+8, i+16 and i+24 in
+ * bits 0-1, 2-3, 4-5 and 6-7).
+ *
  * Readings taken where the definition is silent (each is also listed in the
  * design notes of the repository):
  *   - blocks run along K (the reduction axis), consecutive within a row;
@@ -106,8 +115,9 @@ int oracle_scales_ld(int K)
  * scale overflows fp16 or the input holds a non-finite value.
  * ------------------------------------------------------------------------ */
 static int oracle_quantize(const float *w, int N, int K, int levels_half,
-                           int is_q4, uint8_t *codes, uint16_t *scales)
+                           int fmt, uint8_t *codes, uint16_t *scales)
 {
+    const int zero = fmt == 4 ? 8 : (fmt == 6 ? 32 : 0);   /* zero-point code */
     if (N < 1 || K < ORACLE_BLOCK || K % ORACLE_BLOCK)
         return -1;
     int nb = K / ORACLE_BLOCK;
@@ -134,21 +144,31 @@ static int oracle_quantize(const float *w, int N, int K, int levels_half,
             int q[ORACLE_BLOCK];
             for (int i = 0; i < ORACLE_BLOCK; i++) {
                 if (d == 0.0f) {
-                    q[i] = is_q4 ? 8 : 0;
+                    q[i] = zero;
                     continue;
                 }
                 float r = roundf(blk[i] / d);      /* fp32 division, half away */
-                if (is_q4) {
-                    float t = r + 8.0f;
-                    q[i] = t < 0.0f ? 0 : (t > 15.0f ? 15 : (int)t);
+                if (fmt == 4 || fmt == 6) {
+                    float t = r + (float)zero;
+                    float top = (float)(2 * zero - 1);   /* 15 or 63 */
+                    q[i] = t < 0.0f ? 0 : (t > top ? (int)top : (int)t);
                 } else {
                     q[i] = r < -127.0f ? -127 : (r > 127.0f ? 127 : (int)r);
                 }
             }
-            if (is_q4) {
+            if (fmt == 4) {
                 uint8_t *dst = codes + (size_t)n * (K / 2) + (size_t)j * 16;
                 for (int i = 0; i < 16; i++)
                     dst[i] = (uint8_t)(q[i] | (q[i + 16] << 4));
+            } else if (fmt == 6) {
+                uint8_t *row = codes + (size_t)n * (3 * (size_t)K / 4);
+                uint8_t *lo = row + (size_t)j * 16;
+                uint8_t *hi = row + (size_t)K / 2 + (size_t)j * 8;
+                for (int i = 0; i < 16; i++)
+                    lo[i] = (uint8_t)((q[i] & 15) | ((q[i + 16] & 15) << 4));
+                for (int i = 0; i < 8; i++)
+                    hi[i] = (uint8_t)((q[i] >> 4) | ((q[i + 8] >> 4) << 2) |
+                                      ((q[i + 16] >> 4) << 4) | ((q[i + 24] >> 4) << 6));
             } else {
                 int8_t *dst = (int8_t *)codes + (size_t)n * K + (size_t)j * ORACLE_BLOCK;
                 for (int i = 0; i < ORACLE_BLOCK; i++)
@@ -161,12 +181,18 @@ static int oracle_quantize(const float *w, int N, int K, int levels_half,
 
 int oracle_quantize_q8(const float *w, int N, int K, int8_t *codes, uint16_t *scales)
 {
-    return oracle_quantize(w, N, K, 127, 0, (uint8_t *)codes, scales);
+    return oracle_quantize(w, N, K, 127, 8, (uint8_t *)codes, scales);
 }
 
 int oracle_quantize_q4(const float *w, int N, int K, uint8_t *codes, uint16_t *scales)
 {
-    return oracle_quantize(w, N, K, 7, 1, codes, scales);
+    return oracle_quantize(w, N, K, 7, 4, codes, scales);
+}
+
+/* codes: N rows of 3K/4 bytes (see the header) */
+int oracle_quantize_q6(const float *w, int N, int K, uint8_t *codes, uint16_t *scales)
+{
+    return oracle_quantize(w, N, K, 31, 6, codes, scales);
 }
 
 /* ---------------------------------------------------------------------------
@@ -181,6 +207,21 @@ static double deq_q4(const uint8_t *codes, const uint16_t *scales, int K, int ld
     int q = (i < 16) ? (byte & 0x0f) : (byte >> 4);
     double d = oracle_half_to_double(scales[(size_t)n * ldS + j]);
     return d * (double)(q - 8);
+}
+
+static double deq_q6(const uint8_t *codes, const uint16_t *scales, int K, int ldS,
+                     int n, int k)
+{
+    int j = k / ORACLE_BLOCK;
+    int i = k % ORACLE_BLOCK;
+    const uint8_t *row = codes + (size_t)n * (3 * (size_t)K / 4);
+    uint8_t lo_byte = row[(size_t)j * 16 + (i % 16)];
+    uint8_t hi_byte = row[(size_t)K / 2 + (size_t)j * 8 + (i % 8)];
+    int lo = (i < 16) ? (lo_byte & 0x0f) : (lo_byte >> 4);
+    int hi = (hi_byte >> (2 * (i / 8))) & 3;
+    int q = lo | (hi << 4);
+    double d = oracle_half_to_double(scales[(size_t)n * ldS + j]);
+    return d * (double)(q - 32);
 }
 
 static double deq_q8(const int8_t *codes, const uint16_t *scales, int K, int ldS,
@@ -200,6 +241,15 @@ void oracle_dequantize_q4(const uint8_t *codes, const uint16_t *scales, int N, i
             w[(size_t)n * K + k] = deq_q4(codes, scales, K, ldS, n, k);
 }
 
+void oracle_dequantize_q6(const uint8_t *codes, const uint16_t *scales, int N, int K,
+                          double *w)
+{
+    int ldS = oracle_scales_ld(K);
+    for (int n = 0; n < N; n++)
+        for (int k = 0; k < K; k++)
+            w[(size_t)n * K + k] = deq_q6(codes, scales, K, ldS, n, k);
+}
+
 void oracle_dequantize_q8(const int8_t *codes, const uint16_t *scales, int N, int K,
                           double *w)
 {
@@ -216,7 +266,7 @@ void oracle_dequantize_q8(const int8_t *codes, const uint16_t *scales, int N, in
  * output is still one plain sequential sum.
  * ------------------------------------------------------------------------ */
 typedef struct {
-    int fmt;                  /* 4 or 8 */
+    int fmt;                  /* 4, 6 or 8 */
     const void *codes;
     const uint16_t *scales;
     int N, K, ldS;
@@ -232,9 +282,9 @@ static void gemv_rows(const gemv_job *t)
         for (int b = 0; b < t->B; b++) {
             double s = 0.0, sa = 0.0;
             for (int k = 0; k < t->K; k++) {
-                double w = (t->fmt == 4)
-                               ? deq_q4((const uint8_t *)t->codes, t->scales, t->K, t->ldS, n, k)
-                               : deq_q8((const int8_t *)t->codes, t->scales, t->K, t->ldS, n, k);
+                double w = (t->fmt == 4)   ? deq_q4((const uint8_t *)t->codes, t->scales, t->K, t->ldS, n, k)
+                           : (t->fmt == 6) ? deq_q6((const uint8_t *)t->codes, t->scales, t->K, t->ldS, n, k)
+                                           : deq_q8((const int8_t *)t->codes, t->scales, t->K, t->ldS, n, k);
                 double p = w * oracle_half_to_double(t->x[(size_t)b * t->ldx + k]);
                 s += p;
                 sa += fabs(p);
@@ -295,6 +345,12 @@ int oracle_gemv_q4(const uint8_t *codes, const uint16_t *scales, int N, int K,
                    const uint16_t *x, int B, int ldx, double *y, double *absy, int nthreads)
 {
     return oracle_gemv(4, codes, scales, N, K, x, B, ldx, y, absy, nthreads);
+}
+
+int oracle_gemv_q6(const uint8_t *codes, const uint16_t *scales, int N, int K,
+                   const uint16_t *x, int B, int ldx, double *y, double *absy, int nthreads)
+{
+    return oracle_gemv(6, codes, scales, N, K, x, B, ldx, y, absy, nthreads);
 }
 
 int oracle_gemv_q8(const int8_t *codes, const uint16_t *scales, int N, int K,

@@ -50,7 +50,7 @@ def test_double_to_half_vs_numpy_rne():
 def _expect_exact(fmt, N, nb, e, seed):
     """w = d*v with d = 2^-e and one element per block at +-levels."""
     r = np.random.default_rng(seed)
-    lv = 7 if fmt == 4 else 127
+    lv = {4: 7, 6: 31, 8: 127}[fmt]
     v = r.integers(-lv, lv + 1, size=(N, nb, 32))
     pin = r.integers(0, 32, size=(N, nb))
     sgn = r.choice([-1, 1], size=(N, nb))
@@ -78,6 +78,28 @@ def test_quantize_q4_exact_representable(e):
     assert np.array_equal(oracle.dequantize_q4(codes, scales), w.astype(np.float64))
 
 
+def _q6_planes(q):
+    """Q6 code rows [N, nb, 32] -> the packed row [N, 3K/4], from the format
+    text: the low-nibble plane (Q4's layout) then the 2-bit plane."""
+    N, nb, _ = q.shape
+    lo = (q[..., :16] & 15) | ((q[..., 16:] & 15) << 4)
+    h = q >> 4
+    hi = h[..., 0:8] | (h[..., 8:16] << 2) | (h[..., 16:24] << 4) | (h[..., 24:32] << 6)
+    return np.concatenate([lo.reshape(N, nb * 16), hi.reshape(N, nb * 8)], axis=1).astype(np.uint8)
+
+
+@pytest.mark.parametrize("e", [4, 7, 10, 15, 18, 24])
+def test_quantize_q6_exact_representable(e):
+    N, nb = 4, 10                      # K = 320: ldS = 16 (padded from 10)
+    v, w, d = _expect_exact(6, N, nb, e, 300 + e)
+    codes, scales = oracle.quantize_q6(w)
+    assert codes.shape == (N, 3 * 320 // 4) and scales.shape == (N, 16)
+    dbits = ((15 - e) << 10) if e <= 14 else (1 << (24 - e))
+    assert np.all(scales[:, :nb] == dbits) and np.all(scales[:, nb:] == 0)
+    assert np.array_equal(codes, _q6_planes(v + 32))
+    assert np.array_equal(oracle.dequantize_q6(codes, scales), w.astype(np.float64))
+
+
 @pytest.mark.parametrize("e", [4, 7, 10, 16, 24])
 def test_quantize_q8_exact_representable(e):
     N, nb = 3, 8
@@ -97,6 +119,8 @@ def test_quantize_zero_block_and_tiny_scale():
     assert np.all(s4 == 0) and np.all(c4 == 0x88)
     c8, s8 = oracle.quantize_q8(w)
     assert np.all(s8 == 0) and np.all(c8 == 0)
+    c6, s6 = oracle.quantize_q6(w)        # q = 32: low nibbles 0, top bits 2 (0b10)
+    assert np.all(s6 == 0) and np.all(c6[:, :32] == 0) and np.all(c6[:, 32:] == 0xAA)
 
 
 def test_quantize_round_half_away_and_ties():
@@ -131,8 +155,10 @@ def test_quantize_nearest_grid_point():
     w = synth.weights_f32(synth.key(0, 90, 0, 0, 0), 16, 256)
     c4, s4 = oracle.quantize_q4(w)
     c8, s8 = oracle.quantize_q8(w)
-    for fmt, codes, scales, lv in ((4, c4, s4, (-8, 7)), (8, c8, s8, (-127, 127))):
-        deq = oracle.dequantize_q4(codes, scales) if fmt == 4 else oracle.dequantize_q8(codes, scales)
+    c6, s6 = oracle.quantize_q6(w)
+    for fmt, codes, scales, lv in ((4, c4, s4, (-8, 7)), (8, c8, s8, (-127, 127)),
+                                   (6, c6, s6, (-32, 31))):
+        deq = {4: oracle.dequantize_q4, 6: oracle.dequantize_q6, 8: oracle.dequantize_q8}[fmt](codes, scales)
         d = oracle.half_to_double(scales[:, :8]).repeat(32, axis=1)
         grid = np.arange(lv[0], lv[1] + 1)[None, None, :] * d[..., None]
         nearest = np.abs(grid - w.astype(np.float64)[..., None]).min(axis=-1)
@@ -140,7 +166,8 @@ def test_quantize_nearest_grid_point():
 
 
 # ---------------------------------------------------------- golden files ----
-@pytest.mark.parametrize("name,fmt", [("q4_block_worked.txt", 4), ("q8_block_worked.txt", 8)])
+@pytest.mark.parametrize("name,fmt", [("q4_block_worked.txt", 4), ("q8_block_worked.txt", 8),
+                                      ("q6_block_worked.txt", 6)])
 def test_golden_worked_block(name, fmt):
     g = read_golden(name)
     v = np.array([int(t) for t in g["w_over_d"]])
@@ -152,6 +179,11 @@ def test_golden_worked_block(name, fmt):
         assert [int(b) for b in codes[0]] == [int(t, 16) for t in g["packed"]]
         q = [(codes[0, i % 16] >> (4 * (i // 16))) & 15 for i in range(32)]
         y, a = oracle.gemv_q4(codes, scales, x)
+    elif fmt == 6:
+        codes, scales = oracle.quantize_q6(w)
+        assert [int(b) for b in codes[0]] == [int(t, 16) for t in g["packed"]]
+        q = [int(round(v)) + 32 for v in oracle.dequantize_q6(codes, scales)[0] / d]
+        y, a = oracle.gemv_q6(codes, scales, x)
     else:
         codes, scales = oracle.quantize_q8(w)
         q = [int(c) for c in codes[0]]
@@ -184,6 +216,31 @@ def test_q4_nibble_order_exhaustive():
             assert y[0, 0] == c - 8
 
 
+def test_q6_bit_positions_exhaustive():
+    """Every (position, code) of a 1x32 Q6 block: element i's low 4 bits are
+    in the low (i < 16) or high (i >= 16) nibble of byte i mod 16, its top 2
+    bits in bit pair i // 8 of byte K/2 + i mod 8."""
+    one = np.array([0x3C00], dtype=np.uint16)          # fp16 1.0
+    scales = np.zeros((1, 8), dtype=np.uint16)
+    scales[0, 0] = one[0]
+    for p in range(32):
+        xo = np.zeros((1, 32), dtype=np.uint16)
+        xo[0, p] = one[0]
+        for c in range(64):
+            q = [32] * 32
+            q[p] = c
+            lo = [(q[i] & 15) | ((q[i + 16] & 15) << 4) for i in range(16)]
+            hi = [(q[i] >> 4) | ((q[i + 8] >> 4) << 2) | ((q[i + 16] >> 4) << 4) |
+                  ((q[i + 24] >> 4) << 6) for i in range(8)]
+            packed = np.array([lo + hi], dtype=np.uint8)
+            deq = oracle.dequantize_q6(packed, scales)
+            expect = np.zeros((1, 32))
+            expect[0, p] = c - 32
+            assert np.array_equal(deq, expect), (p, c)
+            y, _ = oracle.gemv_q6(packed, scales, xo)
+            assert y[0, 0] == c - 32
+
+
 def test_scale_plane_stride_and_block_index():
     """Scale (n, j) scales exactly block j of row n, with rows ldS apart."""
     N, K = 3, 96                                       # ldS = 8 > K/32 = 3
@@ -200,20 +257,30 @@ def test_scale_plane_stride_and_block_index():
     c8 = np.ones((N, K), dtype=np.int8)
     deq8 = oracle.dequantize_q8(c8, scales)
     assert np.array_equal(deq8, deq)
+    # Q6 code 33 (v = 1): low nibbles 1, top bits 2 in every pair
+    c6 = np.concatenate([np.full((N, K // 2), 0x11, dtype=np.uint8),
+                         np.full((N, K // 4), 0xAA, dtype=np.uint8)], axis=1)
+    assert np.array_equal(oracle.dequantize_q6(c6, scales), deq)
 
 
 # ------------------------------------------------------------------ GEMV ----
 def _rand_planes(fmt, N, K, seed):
     w = synth.weights_f32(synth.key(seed, 91, 0, 0, 0), N, K)
-    return oracle.quantize_q4(w) if fmt == 4 else oracle.quantize_q8(w)
+    return {4: oracle.quantize_q4, 6: oracle.quantize_q6, 8: oracle.quantize_q8}[fmt](w)
 
 
-@pytest.mark.parametrize("fmt", [4, 8])
+_DEQ = {4: lambda c, s: oracle.dequantize_q4(c, s), 6: lambda c, s: oracle.dequantize_q6(c, s),
+        8: lambda c, s: oracle.dequantize_q8(c, s)}
+_GEMV = {4: lambda *a, **k: oracle.gemv_q4(*a, **k), 6: lambda *a, **k: oracle.gemv_q6(*a, **k),
+         8: lambda *a, **k: oracle.gemv_q8(*a, **k)}
+
+
+@pytest.mark.parametrize("fmt", [4, 6, 8])
 def test_gemv_one_hot_returns_columns(fmt):
     N, K = 7, 96
     codes, scales = _rand_planes(fmt, N, K, 1)
-    deq = oracle.dequantize_q4(codes, scales) if fmt == 4 else oracle.dequantize_q8(codes, scales)
-    gemv = oracle.gemv_q4 if fmt == 4 else oracle.gemv_q8
+    deq = _DEQ[fmt](codes, scales)
+    gemv = _GEMV[fmt]
     one = np.float16(1.0).view(np.uint16)
     x = np.zeros((K, K), dtype=np.uint16)
     x[np.arange(K), np.arange(K)] = one                 # B = K one-hot rows, 8 at a time
@@ -222,13 +289,13 @@ def test_gemv_one_hot_returns_columns(fmt):
         assert np.array_equal(y, deq[:, b0:b0 + 8].T)
 
 
-@pytest.mark.parametrize("fmt", [4, 8])
+@pytest.mark.parametrize("fmt", [4, 6, 8])
 def test_gemv_all_ones_returns_row_sums(fmt):
     import math
     N, K = 11, 160
     codes, scales = _rand_planes(fmt, N, K, 2)
-    deq = oracle.dequantize_q4(codes, scales) if fmt == 4 else oracle.dequantize_q8(codes, scales)
-    gemv = oracle.gemv_q4 if fmt == 4 else oracle.gemv_q8
+    deq = _DEQ[fmt](codes, scales)
+    gemv = _GEMV[fmt]
     x = np.full((2, K), np.float16(1.0).view(np.uint16), dtype=np.uint16)
     y, a = gemv(codes, scales, x)
     for n in range(N):
@@ -245,15 +312,19 @@ def _unpack_fraction(fmt, codes, scales, n, k):
     i = k % 32
     byte = int(codes[n, (k // 32) * 16 + i % 16])
     q = byte & 15 if i < 16 else byte >> 4
+    if fmt == 6:
+        K = codes.shape[1] * 4 // 3
+        top = (int(codes[n, K // 2 + (k // 32) * 8 + i % 8]) >> (2 * (i // 8))) & 3
+        return d * ((q | (top << 4)) - 32)
     return d * (q - 8)
 
 
-@pytest.mark.parametrize("fmt", [4, 8])
+@pytest.mark.parametrize("fmt", [4, 6, 8])
 @pytest.mark.parametrize("N,K,B", [(1, 32, 1), (3, 64, 2), (8, 96, 8), (5, 32, 3), (2, 96, 5)])
 def test_gemv_brute_force_exact(fmt, N, K, B):
     codes, scales = _rand_planes(fmt, N, K, 10 * N + K + B)
     x = synth.activations_f16_bits(synth.key(3, 91, N, K, 1), B, K)
-    gemv = oracle.gemv_q4 if fmt == 4 else oracle.gemv_q8
+    gemv = _GEMV[fmt]
     y, a = gemv(codes, scales, x)
     xf = x.view(np.float16)
     for b in range(B):
@@ -266,12 +337,12 @@ def test_gemv_brute_force_exact(fmt, N, K, B):
             assert abs(Fraction(a[b, n]) - exact_abs) <= exact_abs * Fraction(1, 2 ** 50)
 
 
-@pytest.mark.parametrize("fmt", [4, 8])
+@pytest.mark.parametrize("fmt", [4, 6, 8])
 def test_gemv_batch_rows_independent_and_threads(fmt):
     N, K, B = 37, 256, 6
     codes, scales = _rand_planes(fmt, N, K, 5)
     x = synth.activations_f16_bits(synth.key(4, 91, 0, 0, 1), B, K)
-    gemv = oracle.gemv_q4 if fmt == 4 else oracle.gemv_q8
+    gemv = _GEMV[fmt]
     y, a = gemv(codes, scales, x)
     y4, a4 = gemv(codes, scales, x, nthreads=4)
     assert np.array_equal(y, y4) and np.array_equal(a, a4)
