@@ -227,8 +227,9 @@ typedef struct bq_gemv_geometry {
 BQ_API int32_t bq_gemv_geometry_of(int32_t fmt, int32_t N, int32_t K, int32_t B, int32_t flags,
                                    int32_t sm_count, bq_gemv_geometry *out);
 
-/* Q4 or Q8 decode GEMV with an output epilogue.
- *   fmt        4 or 8
+/* Q4, Q6 or Q8 decode GEMV with an output epilogue.
+ *   fmt        4, 6 or 8 (Q6: K a multiple of 64, codes as bq_quantize_q6
+ *              lays them out: rows of 3K/4 bytes, 16-row work units)
  *   y          device: fp32 [B][N] (BQ_EPI_NONE) or fp16 bits [B][N/2]
  *              (BQ_EPI_SWIGLU, N a multiple of 16), 16-byte aligned
  *   epilogue   BQ_EPI_*; anything else returns BQ_ERR_SHAPE
@@ -349,10 +350,22 @@ BQ_API int32_t bq_moe_gemv_ex(const bq_qmat *Wstack, int32_t E, int64_t codes_st
 BQ_API int32_t bq_quantize_q8(const float *w, int32_t N, int32_t K, int8_t *codes, uint16_t *scales);
 BQ_API int32_t bq_quantize_q4(const float *w, int32_t N, int32_t K, uint8_t *codes, uint16_t *scales);
 
+/* Q6, a third format of the family (the pages list formats from Q2 to FP16
+ * without defining them; BaseRT abstract): d = fp16_rne(a / 31),
+ * q = clamp(round-half-away(w / d) + 32, 0, 63), zero-point code 32.  codes:
+ * uint8 [N][3K/4], each row the low-nibble plane (K/2 bytes, Q4's layout:
+ * block j at byte 16j, byte i = low 4 bits of element i | those of element
+ * i+16 << 4) followed by the top-bit plane (K/4 bytes: block j at byte
+ * K/2 + 8j, byte i = top 2 bits of elements i, i+8, i+16, i+24 in bits 0-1,
+ * 2-3, 4-5, 6-7).  Errors as bq_quantize_q4. */
+BQ_API int32_t bq_quantize_q6(const float *w, int32_t N, int32_t K, uint8_t *codes, uint16_t *scales);
+
 /* Dequantise planes into fp32 weights [N][K] (exact: d * q fits fp32). */
 BQ_API int32_t bq_dequantize_q8(const int8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
                          float *w);
 BQ_API int32_t bq_dequantize_q4(const uint8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
+                         float *w);
+BQ_API int32_t bq_dequantize_q6(const uint8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
                          float *w);
 
 /* Planes <-> interleaved blocks.  blocks: N*(K/32) records, row-major over
@@ -377,6 +390,10 @@ BQ_API int32_t bq_blocks_to_planes_q8(const uint8_t *blocks, int32_t N, int32_t 
 BQ_API int32_t bq_quantize_q4_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
                            uint16_t *scales, int32_t *dev_status, void *stream);
 BQ_API int32_t bq_quantize_q8_dev(const float *w, int32_t N, int32_t K, int8_t *codes,
+                           uint16_t *scales, int32_t *dev_status, void *stream);
+/* Q6 on the GPU: K must be a multiple of 64 (rows of 3K/4 bytes stay
+ * 16-byte aligned), else BQ_ERR_SHAPE. */
+BQ_API int32_t bq_quantize_q6_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
                            uint16_t *scales, int32_t *dev_status, void *stream);
 
 #ifdef __cplusplus

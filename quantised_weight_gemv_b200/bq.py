@@ -80,12 +80,15 @@ _SIGS = {
     "bq_quantize_q4": (_i32, [_vp, _i32, _i32, _vp, _vp]),
     "bq_dequantize_q8": (_i32, [_vp, _vp, _i32, _i32, _vp]),
     "bq_dequantize_q4": (_i32, [_vp, _vp, _i32, _i32, _vp]),
+    "bq_quantize_q6": (_i32, [_vp, _i32, _i32, _vp, _vp]),
+    "bq_dequantize_q6": (_i32, [_vp, _vp, _i32, _i32, _vp]),
     "bq_planes_to_blocks_q4": (_i32, [_vp, _vp, _i32, _i32, _vp]),
     "bq_planes_to_blocks_q8": (_i32, [_vp, _vp, _i32, _i32, _vp]),
     "bq_blocks_to_planes_q4": (_i32, [_vp, _i32, _i32, _vp, _vp]),
     "bq_blocks_to_planes_q8": (_i32, [_vp, _i32, _i32, _vp, _vp]),
     "bq_quantize_q4_dev": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "bq_quantize_q8_dev": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "bq_quantize_q6_dev": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
 }
 
 
@@ -164,10 +167,10 @@ def workspace(nbytes: int, device):
 def gemv(fmt: int, W: bq_qmat, x, y, ws, status=None, stream=None, epilogue: int = BQ_EPI_NONE,
          flags: int = 0) -> None:
     """y[B, N] (fp32) = deq(W) . x[B, K] (fp16), through bq_gemv_q4 / bq_gemv_q8;
-    with an epilogue (BQ_EPI_SWIGLU: y is fp16 [B, N/2]) or flags, through
+    Q6, an epilogue (BQ_EPI_SWIGLU: y is fp16 [B, N/2]) or flags go through
     bq_gemv_ex."""
     B = x.shape[0]
-    if epilogue == BQ_EPI_NONE and flags == 0:
+    if epilogue == BQ_EPI_NONE and flags == 0 and fmt in (4, 8):
         fn = lib().bq_gemv_q4 if fmt == 4 else lib().bq_gemv_q8
         rc = fn(ctypes.byref(W), x.data_ptr(), B, y.data_ptr(), ws.data_ptr(),
                 ws.numel() * ws.element_size(), _ptr(status), _stream_ptr(stream))
@@ -226,7 +229,7 @@ class StepPlan:
 
 def quantize_dev(fmt: int, w, codes, scales, status=None, stream=None) -> None:
     N, K = w.shape
-    fn = lib().bq_quantize_q4_dev if fmt == 4 else lib().bq_quantize_q8_dev
+    fn = {4: lib().bq_quantize_q4_dev, 6: lib().bq_quantize_q6_dev, 8: lib().bq_quantize_q8_dev}[fmt]
     check(f"bq_quantize_q{fmt}_dev",
           fn(w.data_ptr(), N, K, codes.data_ptr(), scales.data_ptr(), _ptr(status),
              _stream_ptr(stream)))

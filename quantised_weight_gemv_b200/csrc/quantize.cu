@@ -7,6 +7,10 @@
 // *stored* scale, clamped to [-127, 127] (Q8), or that +8 clamped to [0, 15]
 // (Q4); a block whose fp16 scale is zero gets the zero-point code (0 / 8).
 // Q4 byte i of a block packs element i (low nibble) and element i+16 (high).
+// Q6 (d = a/31, q = round(w/d)+32 clamped to [0, 63], zero-point code 32):
+// a row of codes is 3K/4 bytes -- the low nibbles in Q4's layout (block j at
+// byte 16j), then the top 2 bits (block j at byte K/2 + 8j; byte i holds
+// those of elements i, i+8, i+16, i+24 in bits 0-1, 2-3, 4-5, 6-7).
 // The pages name the Q4 and Q8 formats (BaseRT abstract: eight formats from
 // Q2 to FP16; technical summary "Belangrijkste Bijdragen": evaluation at Q4
 // and Q8) without spelling out their bits; the definition above is the one
@@ -22,11 +26,14 @@
 namespace bq {
 namespace {
 
+// codes_out: the block's code bytes (Q6: its 16 low-nibble bytes, then its
+// 8 top-bit bytes; the caller places them in their planes).
 template <int FMT>
 __host__ __device__ inline void quantize_block(const float *w, uint8_t *codes_out,
                                                uint16_t *scale_out, bool *ok)
 {
-    constexpr float kLevels = FMT == 4 ? 7.0f : 127.0f;
+    constexpr float kLevels = FMT == 4 ? 7.0f : (FMT == 6 ? 31.0f : 127.0f);
+    constexpr int kZero = FMT == 4 ? 8 : (FMT == 6 ? 32 : 0);
     float a = 0.0f;
     bool finite = true;
     for (int i = 0; i < 32; i++) {
@@ -57,7 +64,7 @@ __host__ __device__ inline void quantize_block(const float *w, uint8_t *codes_ou
     int q[32];
     for (int i = 0; i < 32; i++) {
         if (!finite || d == 0.0f) {
-            q[i] = FMT == 4 ? 8 : 0;
+            q[i] = kZero;
             continue;
         }
 #ifdef __CUDA_ARCH__
@@ -65,9 +72,10 @@ __host__ __device__ inline void quantize_block(const float *w, uint8_t *codes_ou
 #else
         const float r = roundf(w[i] / d);
 #endif
-        if (FMT == 4) {
-            const float s = r + 8.0f;
-            q[i] = s < 0.0f ? 0 : (s > 15.0f ? 15 : (int)s);
+        if (FMT == 4 || FMT == 6) {
+            const float s = r + (float)kZero;
+            const float top = (float)(2 * kZero - 1);
+            q[i] = s < 0.0f ? 0 : (s > top ? (int)top : (int)s);
         } else {
             q[i] = r < -127.0f ? -127 : (r > 127.0f ? 127 : (int)r);
         }
@@ -75,10 +83,23 @@ __host__ __device__ inline void quantize_block(const float *w, uint8_t *codes_ou
     if (FMT == 4) {
         for (int i = 0; i < 16; i++)
             codes_out[i] = (uint8_t)(q[i] | (q[i + 16] << 4));
+    } else if (FMT == 6) {
+        for (int i = 0; i < 16; i++)
+            codes_out[i] = (uint8_t)((q[i] & 15) | ((q[i + 16] & 15) << 4));
+        for (int i = 0; i < 8; i++)
+            codes_out[16 + i] = (uint8_t)((q[i] >> 4) | ((q[i + 8] >> 4) << 2) |
+                                          ((q[i + 16] >> 4) << 4) | ((q[i + 24] >> 4) << 6));
     } else {
         for (int i = 0; i < 32; i++)
             codes_out[i] = (uint8_t)(int8_t)q[i];
     }
+}
+
+// Where a block's code bytes go: Q6 splits them over its two planes.
+template <int FMT>
+__host__ __device__ inline size_t row_code_bytes(int K)
+{
+    return FMT == 4 ? (size_t)K / 2 : (FMT == 6 ? 3 * (size_t)K / 4 : (size_t)K);
 }
 
 template <int FMT>
@@ -89,16 +110,22 @@ int32_t quantize_host(const float *w, int32_t N, int32_t K, uint8_t *codes, uint
     if (N < 1 || K < 32 || K % 32 != 0)
         return BQ_ERR_SHAPE;
     const int nb = K / 32, ldS = bq_scales_ld(K);
-    const size_t row_bytes = FMT == 4 ? (size_t)K / 2 : (size_t)K;
+    const size_t row_bytes = row_code_bytes<FMT>(K);
     const size_t blk_bytes = FMT == 4 ? 16 : 32;
     for (int n = 0; n < N; n++) {
         for (int j = nb; j < ldS; j++)
             scales[(size_t)n * ldS + j] = 0;
         for (int j = 0; j < nb; j++) {
             bool ok = true;
+            uint8_t *row = codes + (size_t)n * row_bytes;
+            uint8_t buf[32];
             quantize_block<FMT>(w + (size_t)n * K + (size_t)j * 32,
-                                codes + (size_t)n * row_bytes + (size_t)j * blk_bytes,
+                                FMT == 6 ? buf : row + (size_t)j * blk_bytes,
                                 scales + (size_t)n * ldS + j, &ok);
+            if (FMT == 6) {
+                memcpy(row + (size_t)j * 16, buf, 16);
+                memcpy(row + (size_t)K / 2 + (size_t)j * 8, buf + 16, 8);
+            }
             if (!ok)
                 return BQ_ERR_RANGE;
         }
@@ -113,7 +140,7 @@ __global__ void quantize_kernel(const float *__restrict__ w, int N, int K, uint8
 {
     const int nb = K / 32, ldS = (nb + 7) / 8 * 8;
     const long long total = (long long)N * nb;
-    const size_t row_bytes = FMT == 4 ? (size_t)K / 2 : (size_t)K;
+    const size_t row_bytes = row_code_bytes<FMT>(K);
     const size_t blk_bytes = FMT == 4 ? 16 : 32;
     for (long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x; b < total;
          b += (long long)gridDim.x * blockDim.x) {
@@ -134,12 +161,19 @@ __global__ void quantize_kernel(const float *__restrict__ w, int N, int K, uint8
         quantize_block<FMT>(v, out, &sc, &ok);
         if (!ok && status)
             atomicOr(status, kStatusRange);
-        uint4 *dst = reinterpret_cast<uint4 *>(codes + (size_t)n * row_bytes + (size_t)j * blk_bytes);
         uint32_t wv[8];
         memcpy(wv, out, sizeof(wv));
-        dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-        if (FMT == 8)
-            dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+        if (FMT == 6) {
+            // (K % 64 == 0: rows of 3K/4 bytes keep both planes aligned)
+            uint8_t *row = codes + (size_t)n * row_bytes;
+            *reinterpret_cast<uint4 *>(row + (size_t)j * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            *reinterpret_cast<uint2 *>(row + (size_t)K / 2 + (size_t)j * 8) = make_uint2(wv[4], wv[5]);
+        } else {
+            uint4 *dst = reinterpret_cast<uint4 *>(codes + (size_t)n * row_bytes + (size_t)j * blk_bytes);
+            dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            if (FMT == 8)
+                dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+        }
         scales[(size_t)n * ldS + j] = sc;
         if (j == nb - 1)
             for (int p = nb; p < ldS; p++)
@@ -153,7 +187,7 @@ int32_t quantize_dev(const float *w, int32_t N, int32_t K, void *codes, uint16_t
 {
     if (!w || !codes || !scales)
         return BQ_ERR_NULL;
-    if (N < 1 || K < 32 || K % 32 != 0)
+    if (N < 1 || K < 32 || K % 32 != 0 || (FMT == 6 && K % 64 != 0))
         return BQ_ERR_SHAPE;
     if (!aligned16(w) || !aligned16(codes) || !aligned16(scales))
         return BQ_ERR_ALIGN;
@@ -185,6 +219,12 @@ int32_t dequantize_host(const void *codes, const uint16_t *scales, int32_t N, in
             if (FMT == 4) {
                 const uint8_t byte = c[(size_t)n * (K / 2) + (k / 32) * 16 + (k % 16)];
                 q = ((k % 32) < 16 ? (byte & 15) : (byte >> 4)) - 8;
+            } else if (FMT == 6) {
+                const uint8_t *row = c + (size_t)n * (3 * (size_t)K / 4);
+                const uint8_t lo = row[(k / 32) * 16 + (k % 16)];
+                const uint8_t hi = row[(size_t)K / 2 + (k / 32) * 8 + (k % 8)];
+                q = (((k % 32) < 16 ? (lo & 15) : (lo >> 4)) | (((hi >> (2 * ((k % 32) / 8))) & 3) << 4)) -
+                    32;
             } else {
                 q = (int8_t)c[(size_t)n * K + k];
             }
@@ -282,6 +322,21 @@ extern "C" int32_t bq_blocks_to_planes_q8(const uint8_t *blocks, int32_t N, int3
                                           int8_t *codes, uint16_t *scales)
 {
     return blocks_to_planes<8>(blocks, N, K, codes, scales);
+}
+extern "C" int32_t bq_quantize_q6(const float *w, int32_t N, int32_t K, uint8_t *codes,
+                                  uint16_t *scales)
+{
+    return quantize_host<6>(w, N, K, codes, scales);
+}
+extern "C" int32_t bq_dequantize_q6(const uint8_t *codes, const uint16_t *scales, int32_t N,
+                                    int32_t K, float *w)
+{
+    return dequantize_host<6>(codes, scales, N, K, w);
+}
+extern "C" int32_t bq_quantize_q6_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
+                                      uint16_t *scales, int32_t *dev_status, void *stream)
+{
+    return quantize_dev<6>(w, N, K, codes, scales, dev_status, stream);
 }
 extern "C" int32_t bq_quantize_q4_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
                                       uint16_t *scales, int32_t *dev_status, void *stream)

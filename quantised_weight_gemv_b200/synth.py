@@ -117,7 +117,7 @@ class DenseWorkload:
 
 def packed_bytes(fmt: int, N: int, K: int) -> int:
     """Algorithmic bytes of one packed matrix: codes + scales (no padding)."""
-    codes = N * K // 2 if fmt == 4 else N * K
+    codes = {4: N * K // 2, 6: 3 * N * K // 4, 8: N * K}[fmt]
     return codes + N * (K // 32) * 2
 
 
@@ -132,6 +132,11 @@ DENSE_H2048 = DenseWorkload(2, "dense16L-h2048-ffn8192-q4", 4, 16, (
     Mat("gate", 8192, 2048, 2), Mat("up", 8192, 2048, 2),
     Mat("down", 2048, 8192, 3),
 ))
+
+
+def dense_h2048(fmt: int) -> DenseWorkload:
+    """The 16-layer hidden-2048 decoder in another format (Q6 or Q8)."""
+    return DenseWorkload(8, f"dense16L-h2048-ffn8192-q{fmt}", fmt, 16, DENSE_H2048.mats)
 
 
 def dense_h4096(fmt: int, B: int) -> DenseWorkload:

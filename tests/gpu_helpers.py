@@ -34,7 +34,7 @@ def gpu_gemv(fmt, codes, scales, x_bits, ws=None, status=None, flags=0):
     fp16 bits; returns fp32 [B, N]."""
     import torch
     N = codes.shape[0]
-    K = codes.shape[1] * (2 if fmt == 4 else 1)
+    K = {4: codes.shape[1] * 2, 6: codes.shape[1] * 4 // 3, 8: codes.shape[1]}[fmt]
     x_bits = np.atleast_2d(x_bits)
     B = x_bits.shape[0]
     c, s, x = dev(codes.view(np.uint8)), dev(scales), dev(x_bits)
@@ -60,11 +60,12 @@ def check_tol(y, y_ref, absy):
 
 
 def oracle_gemv(fmt, codes, scales, x_bits, nthreads=8):
-    return (oracle.gemv_q4 if fmt == 4 else oracle.gemv_q8)(codes, scales, x_bits, nthreads=nthreads)
+    fn = {4: oracle.gemv_q4, 6: oracle.gemv_q6, 8: oracle.gemv_q8}[fmt]
+    return fn(codes, scales, x_bits, nthreads=nthreads)
 
 
 def quantize(fmt, w):
-    return oracle.quantize_q4(w) if fmt == 4 else oracle.quantize_q8(w)
+    return {4: oracle.quantize_q4, 6: oracle.quantize_q6, 8: oracle.quantize_q8}[fmt](w)
 
 
 def pair_order(gate, up):

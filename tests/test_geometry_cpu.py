@@ -37,14 +37,16 @@ SHAPES = [(1, 32), (16, 256), (40, 2048), (777, 3072), (2048, 2048), (3072, 2048
 
 @pytest.mark.parametrize("sm_count", [148, 132, 100])
 @pytest.mark.parametrize("fmt,flags", [(4, 0), (4, bq.BQ_GEMV_ROWS16), (4, bq.BQ_GEMV_ROWS32),
-                                       (8, 0), (4, bq.BQ_GEMV_STATIC_WEIGHTS)])
+                                       (8, 0), (4, bq.BQ_GEMV_STATIC_WEIGHTS), (6, 0)])
 @pytest.mark.parametrize("B", [1, 8])
 def test_geometry_matches_brute_force(sm_count, fmt, flags, B):
     cap = min(2 * sm_count, 512)
     for N, K in SHAPES:
+        if fmt == 6 and K % 64:
+            continue
         g = bq.gemv_geometry(fmt, N, K, B, flags, sm_count=sm_count)
         rows = g["rows"]
-        if fmt == 8 or flags == bq.BQ_GEMV_ROWS16:
+        if fmt != 4 or flags == bq.BQ_GEMV_ROWS16:
             assert rows == 16
         elif flags == bq.BQ_GEMV_ROWS32:
             assert rows == 32

@@ -39,11 +39,12 @@ def _regen_rows(wl, seed, layer, m, rows, K, N_mat):
 
 
 def _quant(fmt, w):
-    return oracle.quantize_q4(w) if fmt == 4 else oracle.quantize_q8(w)
+    return {4: oracle.quantize_q4, 6: oracle.quantize_q6, 8: oracle.quantize_q8}[fmt](w)
 
 
 def _gemv(fmt, codes, scales, xb):
-    return (oracle.gemv_q4 if fmt == 4 else oracle.gemv_q8)(codes, scales, xb, nthreads=8)
+    fn = {4: oracle.gemv_q4, 6: oracle.gemv_q6, 8: oracle.gemv_q8}[fmt]
+    return fn(codes, scales, xb, nthreads=8)
 
 
 def _check_step(wl, every, seed=0, engine="step"):
@@ -137,6 +138,11 @@ def test_dense16_h2048_step(engine):
     """16-layer decoder (hidden 2048, FFN 8192), Q4, batch 1: as one plan, and
     as the chain of per-matrix launches with static weights."""
     _check_step(synth.DENSE_H2048, every=16, engine=engine)
+
+
+def test_dense16_h2048_q6_chain():
+    """The 16-layer hidden-2048 decoder in Q6, as the launch chain."""
+    _check_step(synth.dense_h2048(6), every=16, engine="graph")
 
 
 @pytest.mark.parametrize("fmt", [4, 8])
