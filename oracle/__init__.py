@@ -61,6 +61,10 @@ def lib() -> ctypes.CDLL:
             L.oracle_scales_ld.argtypes = [ctypes.c_int]
             L.oracle_quantize_q4.restype = ctypes.c_int
             L.oracle_quantize_q4.argtypes = [_c_f32p, ctypes.c_int, ctypes.c_int, _c_u8p, _c_u16p]
+            L.oracle_quantize_q5.restype = ctypes.c_int
+            L.oracle_quantize_q5.argtypes = [_c_f32p, ctypes.c_int, ctypes.c_int, _c_u8p, _c_u16p]
+            L.oracle_dequantize_q5.restype = None
+            L.oracle_dequantize_q5.argtypes = [_c_u8p, _c_u16p, ctypes.c_int, ctypes.c_int, _c_f64p]
             L.oracle_quantize_q6.restype = ctypes.c_int
             L.oracle_quantize_q6.argtypes = [_c_f32p, ctypes.c_int, ctypes.c_int, _c_u8p, _c_u16p]
             L.oracle_dequantize_q6.restype = None
@@ -75,6 +79,8 @@ def lib() -> ctypes.CDLL:
                          ctypes.c_int, ctypes.c_int, _c_f64p, _c_f64p, ctypes.c_int]
             L.oracle_gemv_q4.restype = ctypes.c_int
             L.oracle_gemv_q4.argtypes = gemv_args
+            L.oracle_gemv_q5.restype = ctypes.c_int
+            L.oracle_gemv_q5.argtypes = gemv_args
             L.oracle_gemv_q6.restype = ctypes.c_int
             L.oracle_gemv_q6.argtypes = gemv_args
             L.oracle_gemv_q8.restype = ctypes.c_int
@@ -129,6 +135,19 @@ def quantize_q4(w: np.ndarray):
     return codes, scales
 
 
+def quantize_q5(w: np.ndarray):
+    """fp32 [N, K] -> (codes uint8 [N, 5K/8]: low-nibble plane then 1-bit
+    plane, scales fp16-bits uint16 [N, ldS])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    codes = np.zeros((N, 5 * K // 8), dtype=np.uint8)
+    scales = np.zeros((N, scales_ld(K)), dtype=np.uint16)
+    rc = lib().oracle_quantize_q5(_p(w, _c_f32p), N, K, _p(codes, _c_u8p), _p(scales, _c_u16p))
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_q5 failed ({rc})")
+    return codes, scales
+
+
 def quantize_q6(w: np.ndarray):
     """fp32 [N, K] -> (codes uint8 [N, 3K/4]: low-nibble plane then 2-bit
     plane, scales fp16-bits uint16 [N, ldS])."""
@@ -161,6 +180,16 @@ def dequantize_q4(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     assert scales.shape == (N, scales_ld(K))
     out = np.zeros((N, K), dtype=np.float64)
     lib().oracle_dequantize_q4(_p(codes, _c_u8p), _p(scales, _c_u16p), N, K, _p(out, _c_f64p))
+    return out
+
+
+def dequantize_q5(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    N, K = codes.shape[0], codes.shape[1] * 8 // 5
+    assert scales.shape == (N, scales_ld(K))
+    out = np.zeros((N, K), dtype=np.float64)
+    lib().oracle_dequantize_q5(_p(codes, _c_u8p), _p(scales, _c_u16p), N, K, _p(out, _c_f64p))
     return out
 
 
@@ -205,6 +234,12 @@ def gemv_q4(codes, scales, x_bits, nthreads: int = 1):
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint16)
     return _gemv(lib().oracle_gemv_q4, codes, scales, codes.shape[1] * 2, x_bits, nthreads)
+
+
+def gemv_q5(codes, scales, x_bits, nthreads: int = 1):
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    return _gemv(lib().oracle_gemv_q5, codes, scales, codes.shape[1] * 8 // 5, x_bits, nthreads)
 
 
 def gemv_q6(codes, scales, x_bits, nthreads: int = 1):

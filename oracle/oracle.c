@@ -30,6 +30,11 @@
  * K/2 + 8j; byte i holds the top 2 bits of elements i, i+8, i+16 and i+24 in
  * bits 0-1, 2-3, 4-5 and 6-7).
  *
+ * Q5 (the same construction with one top bit): d = absmax/15, q =
+ * clamp(round(w/d)+16, 0, 31), weight d*(q-16); a row of codes is 5K/8 bytes:
+ * the low-nibble plane as Q4, then a 1-bit plane (block j at byte K/2 + 4j;
+ * byte i (0..3) holds the top bit of element i + 4p in bit p, p = 0..7).
+ *
  * Readings taken where the definition is silent (each is also listed in the
  * design notes of the repository):
  *   - blocks run along K (the reduction axis), consecutive within a row;
@@ -117,7 +122,7 @@ int oracle_scales_ld(int K)
 static int oracle_quantize(const float *w, int N, int K, int levels_half,
                            int fmt, uint8_t *codes, uint16_t *scales)
 {
-    const int zero = fmt == 4 ? 8 : (fmt == 6 ? 32 : 0);   /* zero-point code */
+    const int zero = fmt == 4 ? 8 : (fmt == 5 ? 16 : (fmt == 6 ? 32 : 0));   /* zero-point code */
     if (N < 1 || K < ORACLE_BLOCK || K % ORACLE_BLOCK)
         return -1;
     int nb = K / ORACLE_BLOCK;
@@ -148,9 +153,9 @@ static int oracle_quantize(const float *w, int N, int K, int levels_half,
                     continue;
                 }
                 float r = roundf(blk[i] / d);      /* fp32 division, half away */
-                if (fmt == 4 || fmt == 6) {
+                if (fmt != 8) {
                     float t = r + (float)zero;
-                    float top = (float)(2 * zero - 1);   /* 15 or 63 */
+                    float top = (float)(2 * zero - 1);   /* 15, 31 or 63 */
                     q[i] = t < 0.0f ? 0 : (t > top ? (int)top : (int)t);
                 } else {
                     q[i] = r < -127.0f ? -127 : (r > 127.0f ? 127 : (int)r);
@@ -160,6 +165,18 @@ static int oracle_quantize(const float *w, int N, int K, int levels_half,
                 uint8_t *dst = codes + (size_t)n * (K / 2) + (size_t)j * 16;
                 for (int i = 0; i < 16; i++)
                     dst[i] = (uint8_t)(q[i] | (q[i + 16] << 4));
+            } else if (fmt == 5) {
+                uint8_t *row = codes + (size_t)n * (5 * (size_t)K / 8);
+                uint8_t *lo = row + (size_t)j * 16;
+                uint8_t *hi = row + (size_t)K / 2 + (size_t)j * 4;
+                for (int i = 0; i < 16; i++)
+                    lo[i] = (uint8_t)((q[i] & 15) | ((q[i + 16] & 15) << 4));
+                for (int i = 0; i < 4; i++) {
+                    int b = 0;
+                    for (int p = 0; p < 8; p++)
+                        b |= (q[i + 4 * p] >> 4) << p;
+                    hi[i] = (uint8_t)b;
+                }
             } else if (fmt == 6) {
                 uint8_t *row = codes + (size_t)n * (3 * (size_t)K / 4);
                 uint8_t *lo = row + (size_t)j * 16;
@@ -189,6 +206,12 @@ int oracle_quantize_q4(const float *w, int N, int K, uint8_t *codes, uint16_t *s
     return oracle_quantize(w, N, K, 7, 4, codes, scales);
 }
 
+/* codes: N rows of 5K/8 bytes (see the header) */
+int oracle_quantize_q5(const float *w, int N, int K, uint8_t *codes, uint16_t *scales)
+{
+    return oracle_quantize(w, N, K, 15, 5, codes, scales);
+}
+
 /* codes: N rows of 3K/4 bytes (see the header) */
 int oracle_quantize_q6(const float *w, int N, int K, uint8_t *codes, uint16_t *scales)
 {
@@ -207,6 +230,21 @@ static double deq_q4(const uint8_t *codes, const uint16_t *scales, int K, int ld
     int q = (i < 16) ? (byte & 0x0f) : (byte >> 4);
     double d = oracle_half_to_double(scales[(size_t)n * ldS + j]);
     return d * (double)(q - 8);
+}
+
+static double deq_q5(const uint8_t *codes, const uint16_t *scales, int K, int ldS,
+                     int n, int k)
+{
+    int j = k / ORACLE_BLOCK;
+    int i = k % ORACLE_BLOCK;
+    const uint8_t *row = codes + (size_t)n * (5 * (size_t)K / 8);
+    uint8_t lo_byte = row[(size_t)j * 16 + (i % 16)];
+    uint8_t hi_byte = row[(size_t)K / 2 + (size_t)j * 4 + (i % 4)];
+    int lo = (i < 16) ? (lo_byte & 0x0f) : (lo_byte >> 4);
+    int hi = (hi_byte >> (i / 4)) & 1;
+    int q = lo | (hi << 4);
+    double d = oracle_half_to_double(scales[(size_t)n * ldS + j]);
+    return d * (double)(q - 16);
 }
 
 static double deq_q6(const uint8_t *codes, const uint16_t *scales, int K, int ldS,
@@ -241,6 +279,15 @@ void oracle_dequantize_q4(const uint8_t *codes, const uint16_t *scales, int N, i
             w[(size_t)n * K + k] = deq_q4(codes, scales, K, ldS, n, k);
 }
 
+void oracle_dequantize_q5(const uint8_t *codes, const uint16_t *scales, int N, int K,
+                          double *w)
+{
+    int ldS = oracle_scales_ld(K);
+    for (int n = 0; n < N; n++)
+        for (int k = 0; k < K; k++)
+            w[(size_t)n * K + k] = deq_q5(codes, scales, K, ldS, n, k);
+}
+
 void oracle_dequantize_q6(const uint8_t *codes, const uint16_t *scales, int N, int K,
                           double *w)
 {
@@ -266,7 +313,7 @@ void oracle_dequantize_q8(const int8_t *codes, const uint16_t *scales, int N, in
  * output is still one plain sequential sum.
  * ------------------------------------------------------------------------ */
 typedef struct {
-    int fmt;                  /* 4, 6 or 8 */
+    int fmt;                  /* 4, 5, 6 or 8 */
     const void *codes;
     const uint16_t *scales;
     int N, K, ldS;
@@ -283,6 +330,7 @@ static void gemv_rows(const gemv_job *t)
             double s = 0.0, sa = 0.0;
             for (int k = 0; k < t->K; k++) {
                 double w = (t->fmt == 4)   ? deq_q4((const uint8_t *)t->codes, t->scales, t->K, t->ldS, n, k)
+                           : (t->fmt == 5) ? deq_q5((const uint8_t *)t->codes, t->scales, t->K, t->ldS, n, k)
                            : (t->fmt == 6) ? deq_q6((const uint8_t *)t->codes, t->scales, t->K, t->ldS, n, k)
                                            : deq_q8((const int8_t *)t->codes, t->scales, t->K, t->ldS, n, k);
                 double p = w * oracle_half_to_double(t->x[(size_t)b * t->ldx + k]);
@@ -345,6 +393,12 @@ int oracle_gemv_q4(const uint8_t *codes, const uint16_t *scales, int N, int K,
                    const uint16_t *x, int B, int ldx, double *y, double *absy, int nthreads)
 {
     return oracle_gemv(4, codes, scales, N, K, x, B, ldx, y, absy, nthreads);
+}
+
+int oracle_gemv_q5(const uint8_t *codes, const uint16_t *scales, int N, int K,
+                   const uint16_t *x, int B, int ldx, double *y, double *absy, int nthreads)
+{
+    return oracle_gemv(5, codes, scales, N, K, x, B, ldx, y, absy, nthreads);
 }
 
 int oracle_gemv_q6(const uint8_t *codes, const uint16_t *scales, int N, int K,

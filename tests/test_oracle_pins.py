@@ -50,7 +50,7 @@ def test_double_to_half_vs_numpy_rne():
 def _expect_exact(fmt, N, nb, e, seed):
     """w = d*v with d = 2^-e and one element per block at +-levels."""
     r = np.random.default_rng(seed)
-    lv = {4: 7, 6: 31, 8: 127}[fmt]
+    lv = {4: 7, 5: 15, 6: 31, 8: 127}[fmt]
     v = r.integers(-lv, lv + 1, size=(N, nb, 32))
     pin = r.integers(0, 32, size=(N, nb))
     sgn = r.choice([-1, 1], size=(N, nb))
@@ -88,6 +88,30 @@ def _q6_planes(q):
     return np.concatenate([lo.reshape(N, nb * 16), hi.reshape(N, nb * 8)], axis=1).astype(np.uint8)
 
 
+def _q5_planes(q):
+    """Q5 code rows [N, nb, 32] -> the packed row [N, 5K/8], from the format
+    text: the low-nibble plane then the 1-bit plane."""
+    N, nb, _ = q.shape
+    lo = (q[..., :16] & 15) | ((q[..., 16:] & 15) << 4)
+    top = (q >> 4).reshape(N, nb, 8, 4)        # [.., p, i] = element i + 4p
+    hi = np.zeros((N, nb, 4), dtype=np.int64)
+    for p in range(8):
+        hi |= top[:, :, p, :] << p
+    return np.concatenate([lo.reshape(N, nb * 16), hi.reshape(N, nb * 4)], axis=1).astype(np.uint8)
+
+
+@pytest.mark.parametrize("e", [4, 7, 10, 15, 18, 24])
+def test_quantize_q5_exact_representable(e):
+    N, nb = 4, 12                      # K = 384: ldS = 16 (padded from 12)
+    v, w, d = _expect_exact(5, N, nb, e, 500 + e)
+    codes, scales = oracle.quantize_q5(w)
+    assert codes.shape == (N, 5 * 384 // 8) and scales.shape == (N, 16)
+    dbits = ((15 - e) << 10) if e <= 14 else (1 << (24 - e))
+    assert np.all(scales[:, :nb] == dbits) and np.all(scales[:, nb:] == 0)
+    assert np.array_equal(codes, _q5_planes(v + 16))
+    assert np.array_equal(oracle.dequantize_q5(codes, scales), w.astype(np.float64))
+
+
 @pytest.mark.parametrize("e", [4, 7, 10, 15, 18, 24])
 def test_quantize_q6_exact_representable(e):
     N, nb = 4, 10                      # K = 320: ldS = 16 (padded from 10)
@@ -121,6 +145,8 @@ def test_quantize_zero_block_and_tiny_scale():
     assert np.all(s8 == 0) and np.all(c8 == 0)
     c6, s6 = oracle.quantize_q6(w)        # q = 32: low nibbles 0, top bits 2 (0b10)
     assert np.all(s6 == 0) and np.all(c6[:, :32] == 0) and np.all(c6[:, 32:] == 0xAA)
+    c5, s5 = oracle.quantize_q5(w)        # q = 16: low nibbles 0, every top bit 1
+    assert np.all(s5 == 0) and np.all(c5[:, :32] == 0) and np.all(c5[:, 32:] == 0xFF)
 
 
 def test_quantize_round_half_away_and_ties():
@@ -156,9 +182,11 @@ def test_quantize_nearest_grid_point():
     c4, s4 = oracle.quantize_q4(w)
     c8, s8 = oracle.quantize_q8(w)
     c6, s6 = oracle.quantize_q6(w)
+    c5, s5 = oracle.quantize_q5(w)
     for fmt, codes, scales, lv in ((4, c4, s4, (-8, 7)), (8, c8, s8, (-127, 127)),
-                                   (6, c6, s6, (-32, 31))):
-        deq = {4: oracle.dequantize_q4, 6: oracle.dequantize_q6, 8: oracle.dequantize_q8}[fmt](codes, scales)
+                                   (6, c6, s6, (-32, 31)), (5, c5, s5, (-16, 15))):
+        deq = {4: oracle.dequantize_q4, 5: oracle.dequantize_q5, 6: oracle.dequantize_q6,
+               8: oracle.dequantize_q8}[fmt](codes, scales)
         d = oracle.half_to_double(scales[:, :8]).repeat(32, axis=1)
         grid = np.arange(lv[0], lv[1] + 1)[None, None, :] * d[..., None]
         nearest = np.abs(grid - w.astype(np.float64)[..., None]).min(axis=-1)
@@ -167,7 +195,7 @@ def test_quantize_nearest_grid_point():
 
 # ---------------------------------------------------------- golden files ----
 @pytest.mark.parametrize("name,fmt", [("q4_block_worked.txt", 4), ("q8_block_worked.txt", 8),
-                                      ("q6_block_worked.txt", 6)])
+                                      ("q6_block_worked.txt", 6), ("q5_block_worked.txt", 5)])
 def test_golden_worked_block(name, fmt):
     g = read_golden(name)
     v = np.array([int(t) for t in g["w_over_d"]])
@@ -179,11 +207,14 @@ def test_golden_worked_block(name, fmt):
         assert [int(b) for b in codes[0]] == [int(t, 16) for t in g["packed"]]
         q = [(codes[0, i % 16] >> (4 * (i // 16))) & 15 for i in range(32)]
         y, a = oracle.gemv_q4(codes, scales, x)
-    elif fmt == 6:
-        codes, scales = oracle.quantize_q6(w)
+    elif fmt in (5, 6):
+        quant, deq, gemv = ((oracle.quantize_q5, oracle.dequantize_q5, oracle.gemv_q5) if fmt == 5
+                            else (oracle.quantize_q6, oracle.dequantize_q6, oracle.gemv_q6))
+        codes, scales = quant(w)
         assert [int(b) for b in codes[0]] == [int(t, 16) for t in g["packed"]]
-        q = [int(round(v)) + 32 for v in oracle.dequantize_q6(codes, scales)[0] / d]
-        y, a = oracle.gemv_q6(codes, scales, x)
+        zero = 16 if fmt == 5 else 32
+        q = [int(round(v)) + zero for v in deq(codes, scales)[0] / d]
+        y, a = gemv(codes, scales, x)
     else:
         codes, scales = oracle.quantize_q8(w)
         q = [int(c) for c in codes[0]]
@@ -241,6 +272,29 @@ def test_q6_bit_positions_exhaustive():
             assert y[0, 0] == c - 32
 
 
+def test_q5_bit_positions_exhaustive():
+    """Every (position, code) of a 1x32 Q5 block: element i's low 4 bits as
+    Q4's, its top bit in bit i // 4 of byte K/2 + i mod 4."""
+    one = np.array([0x3C00], dtype=np.uint16)          # fp16 1.0
+    scales = np.zeros((1, 8), dtype=np.uint16)
+    scales[0, 0] = one[0]
+    for p in range(32):
+        xo = np.zeros((1, 32), dtype=np.uint16)
+        xo[0, p] = one[0]
+        for c in range(32):
+            q = [16] * 32
+            q[p] = c
+            lo = [(q[i] & 15) | ((q[i + 16] & 15) << 4) for i in range(16)]
+            hi = [sum((q[i + 4 * b] >> 4) << b for b in range(8)) for i in range(4)]
+            packed = np.array([lo + hi], dtype=np.uint8)
+            deq = oracle.dequantize_q5(packed, scales)
+            expect = np.zeros((1, 32))
+            expect[0, p] = c - 16
+            assert np.array_equal(deq, expect), (p, c)
+            y, _ = oracle.gemv_q5(packed, scales, xo)
+            assert y[0, 0] == c - 16
+
+
 def test_scale_plane_stride_and_block_index():
     """Scale (n, j) scales exactly block j of row n, with rows ldS apart."""
     N, K = 3, 96                                       # ldS = 8 > K/32 = 3
@@ -261,21 +315,26 @@ def test_scale_plane_stride_and_block_index():
     c6 = np.concatenate([np.full((N, K // 2), 0x11, dtype=np.uint8),
                          np.full((N, K // 4), 0xAA, dtype=np.uint8)], axis=1)
     assert np.array_equal(oracle.dequantize_q6(c6, scales), deq)
+    # Q5 code 17 (v = 1): low nibbles 1, every top bit 1
+    c5 = np.concatenate([np.full((N, K // 2), 0x11, dtype=np.uint8),
+                         np.full((N, K // 8), 0xFF, dtype=np.uint8)], axis=1)
+    assert np.array_equal(oracle.dequantize_q5(c5, scales), deq)
 
 
 # ------------------------------------------------------------------ GEMV ----
 def _rand_planes(fmt, N, K, seed):
     w = synth.weights_f32(synth.key(seed, 91, 0, 0, 0), N, K)
-    return {4: oracle.quantize_q4, 6: oracle.quantize_q6, 8: oracle.quantize_q8}[fmt](w)
+    return {4: oracle.quantize_q4, 5: oracle.quantize_q5, 6: oracle.quantize_q6,
+            8: oracle.quantize_q8}[fmt](w)
 
 
-_DEQ = {4: lambda c, s: oracle.dequantize_q4(c, s), 6: lambda c, s: oracle.dequantize_q6(c, s),
-        8: lambda c, s: oracle.dequantize_q8(c, s)}
-_GEMV = {4: lambda *a, **k: oracle.gemv_q4(*a, **k), 6: lambda *a, **k: oracle.gemv_q6(*a, **k),
-         8: lambda *a, **k: oracle.gemv_q8(*a, **k)}
+_DEQ = {4: lambda c, s: oracle.dequantize_q4(c, s), 5: lambda c, s: oracle.dequantize_q5(c, s),
+        6: lambda c, s: oracle.dequantize_q6(c, s), 8: lambda c, s: oracle.dequantize_q8(c, s)}
+_GEMV = {4: lambda *a, **k: oracle.gemv_q4(*a, **k), 5: lambda *a, **k: oracle.gemv_q5(*a, **k),
+         6: lambda *a, **k: oracle.gemv_q6(*a, **k), 8: lambda *a, **k: oracle.gemv_q8(*a, **k)}
 
 
-@pytest.mark.parametrize("fmt", [4, 6, 8])
+@pytest.mark.parametrize("fmt", [4, 5, 6, 8])
 def test_gemv_one_hot_returns_columns(fmt):
     N, K = 7, 96
     codes, scales = _rand_planes(fmt, N, K, 1)
@@ -289,7 +348,7 @@ def test_gemv_one_hot_returns_columns(fmt):
         assert np.array_equal(y, deq[:, b0:b0 + 8].T)
 
 
-@pytest.mark.parametrize("fmt", [4, 6, 8])
+@pytest.mark.parametrize("fmt", [4, 5, 6, 8])
 def test_gemv_all_ones_returns_row_sums(fmt):
     import math
     N, K = 11, 160
@@ -316,10 +375,14 @@ def _unpack_fraction(fmt, codes, scales, n, k):
         K = codes.shape[1] * 4 // 3
         top = (int(codes[n, K // 2 + (k // 32) * 8 + i % 8]) >> (2 * (i // 8))) & 3
         return d * ((q | (top << 4)) - 32)
+    if fmt == 5:
+        K = codes.shape[1] * 8 // 5
+        top = (int(codes[n, K // 2 + (k // 32) * 4 + i % 4]) >> (i // 4)) & 1
+        return d * ((q | (top << 4)) - 16)
     return d * (q - 8)
 
 
-@pytest.mark.parametrize("fmt", [4, 6, 8])
+@pytest.mark.parametrize("fmt", [4, 5, 6, 8])
 @pytest.mark.parametrize("N,K,B", [(1, 32, 1), (3, 64, 2), (8, 96, 8), (5, 32, 3), (2, 96, 5)])
 def test_gemv_brute_force_exact(fmt, N, K, B):
     codes, scales = _rand_planes(fmt, N, K, 10 * N + K + B)
@@ -337,7 +400,7 @@ def test_gemv_brute_force_exact(fmt, N, K, B):
             assert abs(Fraction(a[b, n]) - exact_abs) <= exact_abs * Fraction(1, 2 ** 50)
 
 
-@pytest.mark.parametrize("fmt", [4, 6, 8])
+@pytest.mark.parametrize("fmt", [4, 5, 6, 8])
 def test_gemv_batch_rows_independent_and_threads(fmt):
     N, K, B = 37, 256, 6
     codes, scales = _rand_planes(fmt, N, K, 5)
