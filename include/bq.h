@@ -227,9 +227,10 @@ typedef struct bq_gemv_geometry {
 BQ_API int32_t bq_gemv_geometry_of(int32_t fmt, int32_t N, int32_t K, int32_t B, int32_t flags,
                                    int32_t sm_count, bq_gemv_geometry *out);
 
-/* Q4, Q6 or Q8 decode GEMV with an output epilogue.
- *   fmt        4, 6 or 8 (Q6: K a multiple of 64, codes as bq_quantize_q6
- *              lays them out: rows of 3K/4 bytes, 16-row work units)
+/* Q4, Q5, Q6 or Q8 decode GEMV with an output epilogue.
+ *   fmt        4, 5, 6 or 8 (Q6: K a multiple of 64, codes as bq_quantize_q6
+ *              lays them out, rows of 3K/4 bytes; Q5: K a multiple of 128,
+ *              as bq_quantize_q5, rows of 5K/8 bytes; both 16-row work units)
  *   y          device: fp32 [B][N] (BQ_EPI_NONE) or fp16 bits [B][N/2]
  *              (BQ_EPI_SWIGLU, N a multiple of 16), 16-byte aligned
  *   epilogue   BQ_EPI_*; anything else returns BQ_ERR_SHAPE
@@ -360,12 +361,21 @@ BQ_API int32_t bq_quantize_q4(const float *w, int32_t N, int32_t K, uint8_t *cod
  * 2-3, 4-5, 6-7).  Errors as bq_quantize_q4. */
 BQ_API int32_t bq_quantize_q6(const float *w, int32_t N, int32_t K, uint8_t *codes, uint16_t *scales);
 
+/* Q5, the same construction with one top bit: d = fp16_rne(a / 15),
+ * q = clamp(round-half-away(w / d) + 16, 0, 31), zero-point code 16.  codes:
+ * uint8 [N][5K/8], each row the low-nibble plane (K/2 bytes, as Q4) followed
+ * by the top-bit plane (K/8 bytes: block j at byte K/2 + 4j, byte i = 0..3
+ * holds the top bit of element i + 4p in bit p, p = 0..7). */
+BQ_API int32_t bq_quantize_q5(const float *w, int32_t N, int32_t K, uint8_t *codes, uint16_t *scales);
+
 /* Dequantise planes into fp32 weights [N][K] (exact: d * q fits fp32). */
 BQ_API int32_t bq_dequantize_q8(const int8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
                          float *w);
 BQ_API int32_t bq_dequantize_q4(const uint8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
                          float *w);
 BQ_API int32_t bq_dequantize_q6(const uint8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
+                         float *w);
+BQ_API int32_t bq_dequantize_q5(const uint8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
                          float *w);
 
 /* Planes <-> interleaved blocks.  blocks: N*(K/32) records, row-major over
@@ -394,6 +404,10 @@ BQ_API int32_t bq_quantize_q8_dev(const float *w, int32_t N, int32_t K, int8_t *
 /* Q6 on the GPU: K must be a multiple of 64 (rows of 3K/4 bytes stay
  * 16-byte aligned), else BQ_ERR_SHAPE. */
 BQ_API int32_t bq_quantize_q6_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
+                           uint16_t *scales, int32_t *dev_status, void *stream);
+/* Q5 on the GPU: K must be a multiple of 128 (rows of 5K/8 bytes stay
+ * 16-byte aligned), else BQ_ERR_SHAPE. */
+BQ_API int32_t bq_quantize_q5_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
                            uint16_t *scales, int32_t *dev_status, void *stream);
 
 #ifdef __cplusplus

@@ -73,26 +73,39 @@ template <int MT> struct Fmt<4, MT> {
     static constexpr int kRows = 16 * kMT;              // rows per chunk / band
     static constexpr int kBoxes = 1;                    // 128-byte-wide code boxes
     static constexpr int kCodeBytes = kRows * 128;      // 2 or 4 KB
+    static constexpr int kCodeLoad = kCodeBytes;        // code bytes one chunk's loads bring
     static constexpr int kScaleBytes = kRows * 16;      // kRows x 8 fp16
     static constexpr int kStages = BQ_STAGES;
 };
-template <> struct Fmt<6, 1> {
+// Q5 likewise, with a 32-byte top-bit box: 2.5 KB of codes per chunk, in a
+// 3 KB slot (slots stay 1024-byte aligned, as the 128-byte swizzle of the
+// low-nibble box assumes).
+template <int FMT> struct FmtTop {
     static constexpr int kMT = 1;
     static constexpr int kRows = 16;
     static constexpr int kBoxes = 1;                    // + the top-bit box
-    static constexpr int kLoBytes = kRows * 128;        // 2 KB
-    static constexpr int kCodeBytes = kLoBytes + kRows * 64;   // 3 KB
+    static constexpr int kTopRow = FMT == 6 ? 64 : 32;  // top-bit bytes per row and chunk
+    static constexpr int kCodeLoad = kRows * 128 + kRows * kTopRow;
+    static constexpr int kCodeBytes = 3072;             // slot stride
     static constexpr int kScaleBytes = kRows * 16;
     static constexpr int kStages = BQ_STAGES;
 };
+template <> struct Fmt<6, 1> : FmtTop<6> {};
+template <> struct Fmt<5, 1> : FmtTop<5> {};
 template <> struct Fmt<8, 1> {
     static constexpr int kMT = 1;
     static constexpr int kRows = 16;
     static constexpr int kBoxes = 2;
     static constexpr int kCodeBytes = 2 * kRows * 128;  // 4 KB
+    static constexpr int kCodeLoad = kCodeBytes;
     static constexpr int kScaleBytes = kRows * 16;
     static constexpr int kStages = BQ_STAGES;
 };
+static_assert(Fmt<5, 1>::kCodeLoad <= Fmt<5, 1>::kCodeBytes &&
+                  Fmt<6, 1>::kCodeLoad <= Fmt<6, 1>::kCodeBytes && Fmt<4, 2>::kCodeBytes % 1024 == 0 &&
+                  Fmt<5, 1>::kCodeBytes % 1024 == 0 && Fmt<6, 1>::kCodeBytes % 1024 == 0 &&
+                  Fmt<8, 1>::kCodeBytes % 1024 == 0,
+              "code slots hold a chunk and stay 1024-byte aligned");
 
 template <int FMT, int MT = default_mt<FMT>()>
 constexpr int smem_bytes()
@@ -345,12 +358,12 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // (block_offset).  Every product is exact; the scale 2^-24 (2^-20 for Q4) is
 // undone at the store.
 
-// f16x2 of -z' * 2^-24 (a subnormal): z' = 128 (Q4: 8 * 16; Q8: 128) or
-// 512 (Q6: 32 * 16).
+// f16x2 of -z' * 2^-24 (a subnormal): z' = 128 (Q4: 8 * 16; Q8: 128), 256
+// (Q5: 16 * 16) or 512 (Q6: 32 * 16).
 template <int FMT>
 __host__ __device__ constexpr uint32_t zero_point_pair()
 {
-    return FMT == 6 ? 0x82008200u : 0x80808080u;
+    return FMT == 6 ? 0x82008200u : (FMT == 5 ? 0x81008100u : 0x80808080u);
 }
 
 // The y of a band is stored as acc * 2^20 (Q4 and Q6: codes enter at
@@ -436,25 +449,32 @@ __device__ __forceinline__ void block_q4(uint32_t addr, uint2 xa, uint2 xb, cons
         : "r"(addr), "r"(xa.x), "r"(xa.y), "r"(xb.x), "r"(xb.y), "f"(off[0]), "f"(off[1]),
           "f"(off[2]), "f"(off[3]), "f"(dg), "f"(dg8), "r"(m16));
 }
-// One Q6 block for a 16-row m-tile: Q4's nibble placement (u = 16 * low 4
-// bits at bits 4-7) plus the top 2 bits of each code at bits 8-9, so a lane
-// holds u = 16 q exactly (q < 64, u < 1024).  `addr` is row g's 4-byte group
-// of low nibbles (as block_q4); `addr_hi` row g's 4-byte group of top bits:
-// byte i of it holds element 4(t%2)+i's pairs, pair t/2 for elements 4t..4t+3
-// and pair t/2 + 2 for elements 4t+16..4t+19.  `mh1` / `mh2` = 2^(8 - 2(t/2))
-// / 2^(4 - 2(t/2)) move those pairs to bits 8-9 (multiplies, on the FMA
-// pipe).  Row g+8 is 1024 bytes (low plane) / 512 bytes (top plane) on.
-__device__ __forceinline__ void block_q6(uint32_t addr, uint32_t addr_hi, uint2 xa, uint2 xb,
-                                         const float (&off)[4], float dg, float dg8,
-                                         float (&acc)[4], uint32_t m16, uint32_t mh1, uint32_t mh2)
+// One Q6 or Q5 block for a 16-row m-tile: Q4's nibble placement (u = 16 *
+// low 4 bits at bits 4-7) plus the top bits of each code at bits 8-9 (Q6: 2
+// bits) or bit 8 (Q5: 1), so a lane holds u = 16 q exactly (q < 64, u <
+// 1024).  `addr` is row g's 4-byte group of low nibbles (as block_q4);
+// `addr_hi` row g's 4-byte group of top bits, whose byte i serves elements
+// 4t+i and 4t+16+i: Q6 -- byte i of the group at 4(t%2) holds pairs of
+// elements 4(t%2)+i+8p, pair t/2 for 4t+i and t/2+2 for 4t+16+i; Q5 -- byte
+// i of the block's 4 bytes holds bits of elements i+4p, bit t for 4t+i and
+// t+4 for 4t+16+i.  `mh1` / `mh2` (Q6: 2^(8-2(t/2)), 2^(4-2(t/2)); Q5:
+// 2^(8-t), 2^(4-t)) move those bits to bit 8 (multiplies, on the FMA pipe).
+// Row g+8 is 1024 bytes on in the low plane, 8 top rows on in the top plane.
+template <int FMT>
+__device__ __forceinline__ void block_qtop(uint32_t addr, uint32_t addr_hi, uint2 xa, uint2 xb,
+                                           const float (&off)[4], float dg, float dg8,
+                                           float (&acc)[4], uint32_t m16, uint32_t mh1,
+                                           uint32_t mh2)
 {
+    constexpr uint32_t kTopMask = FMT == 6 ? 0x03000300u : 0x01000100u;
+    constexpr int kTop8 = 8 * Fmt<FMT, 1>::kTopRow;   // row g+8 in the top plane
     asm("{\n\t"
         ".reg .b32 w0, w8, h0, h8, p01, p23, q01, q23, e01, e23, f01, f23, a0, a1, a2, a3, t0, t1, t2, t3;\n\t"
         ".reg .f32 c0, c1, c2, c3;\n\t"
         "ld.shared.b32 w0, [%4];\n\t"
         "ld.shared.b32 w8, [%4+1024];\n\t"
         "ld.shared.b32 h0, [%5];\n\t"
-        "ld.shared.b32 h8, [%5+512];\n\t"
+        "ld.shared.b32 h8, [%5+%19];\n\t"
         "prmt.b32 p01, w0, 0, 0x4140;\n\t"
         "prmt.b32 p23, w0, 0, 0x4342;\n\t"
         "prmt.b32 q01, w8, 0, 0x4140;\n\t"
@@ -472,10 +492,10 @@ __device__ __forceinline__ void block_q6(uint32_t addr, uint32_t addr_hi, uint2 
         "mul.lo.u32 t1, f01, %17;\n\t"
         "mul.lo.u32 t2, e23, %17;\n\t"
         "mul.lo.u32 t3, f23, %17;\n\t"
-        "and.b32 t0, t0, 0x03000300;\n\t"
-        "and.b32 t1, t1, 0x03000300;\n\t"
-        "and.b32 t2, t2, 0x03000300;\n\t"
-        "and.b32 t3, t3, 0x03000300;\n\t"
+        "and.b32 t0, t0, %20;\n\t"
+        "and.b32 t1, t1, %20;\n\t"
+        "and.b32 t2, t2, %20;\n\t"
+        "and.b32 t3, t3, %20;\n\t"
         "lop3.b32 a0, a0, 0x00F000F0, t0, 0xEA;\n\t"
         "lop3.b32 a1, a1, 0x00F000F0, t1, 0xEA;\n\t"
         "lop3.b32 a2, a2, 0x00F000F0, t2, 0xEA;\n\t"
@@ -487,10 +507,10 @@ __device__ __forceinline__ void block_q6(uint32_t addr, uint32_t addr_hi, uint2 
         "mul.lo.u32 t1, f01, %18;\n\t"
         "mul.lo.u32 t2, e23, %18;\n\t"
         "mul.lo.u32 t3, f23, %18;\n\t"
-        "and.b32 t0, t0, 0x03000300;\n\t"
-        "and.b32 t1, t1, 0x03000300;\n\t"
-        "and.b32 t2, t2, 0x03000300;\n\t"
-        "and.b32 t3, t3, 0x03000300;\n\t"
+        "and.b32 t0, t0, %20;\n\t"
+        "and.b32 t1, t1, %20;\n\t"
+        "and.b32 t2, t2, %20;\n\t"
+        "and.b32 t3, t3, %20;\n\t"
         "lop3.b32 a0, p01, 0x00F000F0, t0, 0xEA;\n\t"
         "lop3.b32 a1, q01, 0x00F000F0, t1, 0xEA;\n\t"
         "lop3.b32 a2, p23, 0x00F000F0, t2, 0xEA;\n\t"
@@ -503,7 +523,8 @@ __device__ __forceinline__ void block_q6(uint32_t addr, uint32_t addr_hi, uint2 
         "fma.rn.f32 %3, %15, c3, %3;\n\t}"
         : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
         : "r"(addr), "r"(addr_hi), "r"(xa.x), "r"(xa.y), "r"(xb.x), "r"(xb.y), "f"(off[0]),
-          "f"(off[1]), "f"(off[2]), "f"(off[3]), "f"(dg), "f"(dg8), "r"(m16), "r"(mh1), "r"(mh2));
+          "f"(off[1]), "f"(off[2]), "f"(off[3]), "f"(dg), "f"(dg8), "r"(m16), "r"(mh1), "r"(mh2),
+          "n"(kTop8), "n"(kTopMask));
 }
 
 // One Q8 block for the 16-row m-tile: addr_a / addr_b are row g's 4-byte
@@ -576,7 +597,7 @@ __device__ __forceinline__ void lane_swizzle(int g, int (&sw)[8])
 {
 #pragma unroll
     for (int jb = 0; jb < 8; jb++) {
-        if constexpr (FMT == 4 || FMT == 6) {   // (Q6: its low-nibble plane)
+        if constexpr (FMT == 4 || FMT == 5 || FMT == 6) {   // (Q5, Q6: the low-nibble plane)
             sw[jb] = ((jb ^ g) & 7) << 4;
         } else {
             const int jj = jb & 3;
@@ -628,10 +649,12 @@ __device__ __forceinline__ void chunk_mma(uint32_t codes_s, uint32_t scales_s, i
         sc[mt][1] = lds128_u32(scales_s + (16 * mt + g + 8) * 16);
     }
     const uint32_t lane_codes = codes_s + g * 128 + 4 * t;
-    // Q6: this lane's top-bit group (rows 64 bytes apart, after the 16 rows of
-    // low nibbles) and the multipliers that move its pairs to bits 8-9.
-    const uint32_t lane_hi = codes_s + 16 * 128 + g * 64 + 4 * (t & 1);
-    const uint32_t mh1 = 1u << (8 - 2 * (t >> 1)), mh2 = 1u << (4 - 2 * (t >> 1));
+    // Q6 / Q5: this lane's top-bit group (after the 16 rows of low nibbles;
+    // rows 64 / 32 bytes apart) and the multipliers that move its bits to 8.
+    const uint32_t lane_hi = FMT == 6 ? codes_s + 16 * 128 + g * 64 + 4 * (t & 1)
+                                      : codes_s + 16 * 128 + g * 32;
+    const uint32_t mh1 = FMT == 6 ? 1u << (8 - 2 * (t >> 1)) : 1u << (8 - t);
+    const uint32_t mh2 = FMT == 6 ? 1u << (4 - 2 * (t >> 1)) : 1u << (4 - t);
     auto one_block = [&](int jb) {
         float off[4];
         block_offset<FMT>(xa[jb], xb[jb], off);
@@ -644,9 +667,9 @@ __device__ __forceinline__ void chunk_mma(uint32_t codes_s, uint32_t scales_s, i
             const float dg8 = (jb & 1) ? e1 : e0;
             if constexpr (FMT == 4) {
                 block_q4(lane_codes + mt * 2048 + sw[jb], xa[jb], xb[jb], off, dg, dg8, acc[mt], m16);
-            } else if constexpr (FMT == 6) {
-                block_q6(lane_codes + sw[jb], lane_hi + 8 * jb, xa[jb], xb[jb], off, dg, dg8, acc[mt],
-                         m16, mh1, mh2);
+            } else if constexpr (FMT == 6 || FMT == 5) {
+                block_qtop<FMT>(lane_codes + sw[jb], lane_hi + (FMT == 6 ? 8 : 4) * jb, xa[jb],
+                                xb[jb], off, dg, dg8, acc[mt], m16, mh1, mh2);
             } else {
                 const uint32_t base = lane_codes + (jb >> 2) * 2048;
                 block_q8(base + (sw[jb] & 0xffff), base + (sw[jb] >> 16), xa[jb], xb[jb], off, dg,

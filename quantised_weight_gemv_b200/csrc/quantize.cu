@@ -11,6 +11,10 @@
 // a row of codes is 3K/4 bytes -- the low nibbles in Q4's layout (block j at
 // byte 16j), then the top 2 bits (block j at byte K/2 + 8j; byte i holds
 // those of elements i, i+8, i+16, i+24 in bits 0-1, 2-3, 4-5, 6-7).
+// Q5 (d = a/15, q = round(w/d)+16 clamped to [0, 31], zero-point code 16):
+// rows of 5K/8 bytes -- the low nibbles as Q4, then one top bit per element
+// (block j at byte K/2 + 4j; byte i = 0..3 holds that of element i + 4p in
+// bit p).
 // The pages name the Q4 and Q8 formats (BaseRT abstract: eight formats from
 // Q2 to FP16; technical summary "Belangrijkste Bijdragen": evaluation at Q4
 // and Q8) without spelling out their bits; the definition above is the one
@@ -32,8 +36,8 @@ template <int FMT>
 __host__ __device__ inline void quantize_block(const float *w, uint8_t *codes_out,
                                                uint16_t *scale_out, bool *ok)
 {
-    constexpr float kLevels = FMT == 4 ? 7.0f : (FMT == 6 ? 31.0f : 127.0f);
-    constexpr int kZero = FMT == 4 ? 8 : (FMT == 6 ? 32 : 0);
+    constexpr float kLevels = FMT == 4 ? 7.0f : (FMT == 5 ? 15.0f : (FMT == 6 ? 31.0f : 127.0f));
+    constexpr int kZero = FMT == 4 ? 8 : (FMT == 5 ? 16 : (FMT == 6 ? 32 : 0));
     float a = 0.0f;
     bool finite = true;
     for (int i = 0; i < 32; i++) {
@@ -72,7 +76,7 @@ __host__ __device__ inline void quantize_block(const float *w, uint8_t *codes_ou
 #else
         const float r = roundf(w[i] / d);
 #endif
-        if (FMT == 4 || FMT == 6) {
+        if (FMT != 8) {
             const float s = r + (float)kZero;
             const float top = (float)(2 * kZero - 1);
             q[i] = s < 0.0f ? 0 : (s > top ? (int)top : (int)s);
@@ -83,6 +87,15 @@ __host__ __device__ inline void quantize_block(const float *w, uint8_t *codes_ou
     if (FMT == 4) {
         for (int i = 0; i < 16; i++)
             codes_out[i] = (uint8_t)(q[i] | (q[i + 16] << 4));
+    } else if (FMT == 5) {
+        for (int i = 0; i < 16; i++)
+            codes_out[i] = (uint8_t)((q[i] & 15) | ((q[i + 16] & 15) << 4));
+        for (int i = 0; i < 4; i++) {
+            int b = 0;
+            for (int p = 0; p < 8; p++)
+                b |= (q[i + 4 * p] >> 4) << p;
+            codes_out[16 + i] = (uint8_t)b;
+        }
     } else if (FMT == 6) {
         for (int i = 0; i < 16; i++)
             codes_out[i] = (uint8_t)((q[i] & 15) | ((q[i + 16] & 15) << 4));
@@ -99,7 +112,8 @@ __host__ __device__ inline void quantize_block(const float *w, uint8_t *codes_ou
 template <int FMT>
 __host__ __device__ inline size_t row_code_bytes(int K)
 {
-    return FMT == 4 ? (size_t)K / 2 : (FMT == 6 ? 3 * (size_t)K / 4 : (size_t)K);
+    return FMT == 4 ? (size_t)K / 2
+                    : (FMT == 5 ? 5 * (size_t)K / 8 : (FMT == 6 ? 3 * (size_t)K / 4 : (size_t)K));
 }
 
 template <int FMT>
@@ -119,12 +133,14 @@ int32_t quantize_host(const float *w, int32_t N, int32_t K, uint8_t *codes, uint
             bool ok = true;
             uint8_t *row = codes + (size_t)n * row_bytes;
             uint8_t buf[32];
+            constexpr bool kPlanes = FMT == 5 || FMT == 6;    // codes split over two planes
+            constexpr int kTop = FMT == 5 ? 4 : 8;            // top-plane bytes per block
             quantize_block<FMT>(w + (size_t)n * K + (size_t)j * 32,
-                                FMT == 6 ? buf : row + (size_t)j * blk_bytes,
+                                kPlanes ? buf : row + (size_t)j * blk_bytes,
                                 scales + (size_t)n * ldS + j, &ok);
-            if (FMT == 6) {
+            if (kPlanes) {
                 memcpy(row + (size_t)j * 16, buf, 16);
-                memcpy(row + (size_t)K / 2 + (size_t)j * 8, buf + 16, 8);
+                memcpy(row + (size_t)K / 2 + (size_t)j * kTop, buf + 16, kTop);
             }
             if (!ok)
                 return BQ_ERR_RANGE;
@@ -163,11 +179,14 @@ __global__ void quantize_kernel(const float *__restrict__ w, int N, int K, uint8
             atomicOr(status, kStatusRange);
         uint32_t wv[8];
         memcpy(wv, out, sizeof(wv));
-        if (FMT == 6) {
-            // (K % 64 == 0: rows of 3K/4 bytes keep both planes aligned)
+        if (FMT == 5 || FMT == 6) {
+            // (Q6: K % 64 == 0, Q5: K % 128 == 0: rows keep both planes aligned)
             uint8_t *row = codes + (size_t)n * row_bytes;
             *reinterpret_cast<uint4 *>(row + (size_t)j * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-            *reinterpret_cast<uint2 *>(row + (size_t)K / 2 + (size_t)j * 8) = make_uint2(wv[4], wv[5]);
+            if (FMT == 6)
+                *reinterpret_cast<uint2 *>(row + (size_t)K / 2 + (size_t)j * 8) = make_uint2(wv[4], wv[5]);
+            else
+                *reinterpret_cast<uint32_t *>(row + (size_t)K / 2 + (size_t)j * 4) = wv[4];
         } else {
             uint4 *dst = reinterpret_cast<uint4 *>(codes + (size_t)n * row_bytes + (size_t)j * blk_bytes);
             dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
@@ -187,7 +206,7 @@ int32_t quantize_dev(const float *w, int32_t N, int32_t K, void *codes, uint16_t
 {
     if (!w || !codes || !scales)
         return BQ_ERR_NULL;
-    if (N < 1 || K < 32 || K % 32 != 0 || (FMT == 6 && K % 64 != 0))
+    if (N < 1 || K < 32 || K % 32 != 0 || (FMT == 6 && K % 64 != 0) || (FMT == 5 && K % 128 != 0))
         return BQ_ERR_SHAPE;
     if (!aligned16(w) || !aligned16(codes) || !aligned16(scales))
         return BQ_ERR_ALIGN;
@@ -219,6 +238,11 @@ int32_t dequantize_host(const void *codes, const uint16_t *scales, int32_t N, in
             if (FMT == 4) {
                 const uint8_t byte = c[(size_t)n * (K / 2) + (k / 32) * 16 + (k % 16)];
                 q = ((k % 32) < 16 ? (byte & 15) : (byte >> 4)) - 8;
+            } else if (FMT == 5) {
+                const uint8_t *row = c + (size_t)n * (5 * (size_t)K / 8);
+                const uint8_t lo = row[(k / 32) * 16 + (k % 16)];
+                const uint8_t hi = row[(size_t)K / 2 + (k / 32) * 4 + (k % 4)];
+                q = (((k % 32) < 16 ? (lo & 15) : (lo >> 4)) | (((hi >> ((k % 32) / 4)) & 1) << 4)) - 16;
             } else if (FMT == 6) {
                 const uint8_t *row = c + (size_t)n * (3 * (size_t)K / 4);
                 const uint8_t lo = row[(k / 32) * 16 + (k % 16)];
@@ -322,6 +346,21 @@ extern "C" int32_t bq_blocks_to_planes_q8(const uint8_t *blocks, int32_t N, int3
                                           int8_t *codes, uint16_t *scales)
 {
     return blocks_to_planes<8>(blocks, N, K, codes, scales);
+}
+extern "C" int32_t bq_quantize_q5(const float *w, int32_t N, int32_t K, uint8_t *codes,
+                                  uint16_t *scales)
+{
+    return quantize_host<5>(w, N, K, codes, scales);
+}
+extern "C" int32_t bq_dequantize_q5(const uint8_t *codes, const uint16_t *scales, int32_t N,
+                                    int32_t K, float *w)
+{
+    return dequantize_host<5>(codes, scales, N, K, w);
+}
+extern "C" int32_t bq_quantize_q5_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
+                                      uint16_t *scales, int32_t *dev_status, void *stream)
+{
+    return quantize_dev<5>(w, N, K, codes, scales, dev_status, stream);
 }
 extern "C" int32_t bq_quantize_q6(const float *w, int32_t N, int32_t K, uint8_t *codes,
                                   uint16_t *scales)

@@ -121,7 +121,7 @@ struct KernelArgs {
     // routed experts
     int E, topk, x_per_slot;
     const int *idx;
-    // Q6 (matrix mode): the top-bit plane of mat0's codes
+    // Q5 / Q6 (matrix mode): the top-bit plane of mat0's codes
     alignas(64) CUtensorMap tm_codes_hi;
 };
 
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     constexpr int SB = F::kScaleBytes;
     constexpr int MT = F::kMT;
     constexpr int ROWS = F::kRows;
-    constexpr uint32_t kTx = CB + SB;
+    constexpr uint32_t kTx = F::kCodeLoad + SB;   // bytes one chunk's loads bring
     constexpr bool MOE = MODE == kModeMoE;
     constexpr bool PLAN = MODE == kModePlan;
 
@@ -430,8 +430,8 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 for (int bx = 0; bx < F::kBoxes; bx++)
                     tma_load_2d(cdst + bx * (ROWS * 128), &m.tm_codes, bar,
                                 iss.kp * 128 * F::kBoxes + bx * 128, row, pol);
-                if constexpr (FMT == 6)
-                    tma_load_2d(cdst + ROWS * 128, &a.tm_codes_hi, bar, iss.kp * 64, row, pol);
+                if constexpr (FMT == 5 || FMT == 6)
+                    tma_load_2d(cdst + ROWS * 128, &a.tm_codes_hi, bar, iss.kp * F::kTopRow, row, pol);
                 tma_load_2d(sdst, &m.tm_scales, bar, iss.kp * 8, row, (FMT == 4) ? pol : pol_s);
             }
         }
@@ -950,7 +950,7 @@ constexpr size_t kSyncBytes = 512;
 constexpr CUtensorMapL2promotion kPromoCodes = CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
 constexpr CUtensorMapL2promotion kPromoScales = CU_TENSOR_MAP_L2_PROMOTION_NONE;
 
-int rows_of(int fmt) { return fmt == 4 ? Fmt<4>::kRows : (fmt == 6 ? Fmt<6>::kRows : Fmt<8>::kRows); }
+int rows_of(int fmt) { return fmt == 4 ? Fmt<4>::kRows : Fmt<8>::kRows; }   // (Q5, Q6: 16 as Q8)
 
 // R: rows per chunk (the band height), rows_of(fmt) unless a launch chose
 // another Q4 geometry.
@@ -960,9 +960,12 @@ bool fill_matdesc(int fmt, const bq_qmat *W, const uint16_t *x, int B, float *y,
     if (R == 0)
         R = rows_of(fmt);
     const int N = W->N, K = W->K;
-    // Q6: the low-nibble plane, the first K/2 bytes of each 3K/4-byte row
+    // Q5 / Q6: the low-nibble plane, the first K/2 bytes of each 5K/8- or
+    // 3K/4-byte row
     const uint64_t cdims[2] = {(uint64_t)(fmt == 8 ? K : K / 2), (uint64_t)N};
-    const uint64_t cstr[1] = {(uint64_t)(fmt == 4 ? K / 2 : (fmt == 6 ? 3 * K / 4 : K))};
+    const uint64_t cstr[1] = {(uint64_t)(fmt == 4   ? K / 2
+                                         : fmt == 5 ? 5 * K / 8
+                                         : fmt == 6 ? 3 * K / 4 : K)};
     const uint32_t cbox[2] = {128, (uint32_t)R};
     const int ldS = bq_scales_ld(K);
     const uint64_t sdims[2] = {(uint64_t)(K / 32), (uint64_t)N};
@@ -1162,12 +1165,13 @@ int32_t gemv_launch(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int
     memset(&a, 0, sizeof(a));
     if (!fill_matdesc(FMT, W, x, B, static_cast<float *>(y), &a.mat0, Fmt<FMT, MT>::kRows))
         return BQ_ERR_CUDA;
-    if constexpr (FMT == 6) {
-        // the top-bit plane: the last K/4 bytes of each 3K/4-byte row
+    if constexpr (FMT == 5 || FMT == 6) {
+        // the top-bit plane: the last K/8 (Q5) or K/4 (Q6) bytes of each row
         const int N = W->N, K = W->K;
-        const uint64_t hdims[2] = {(uint64_t)(K / 4), (uint64_t)N};
-        const uint64_t hstr[1] = {(uint64_t)(3 * K / 4)};
-        const uint32_t hbox[2] = {64, (uint32_t)Fmt<6>::kRows};
+        const int top = FMT == 6 ? K / 4 : K / 8;
+        const uint64_t hdims[2] = {(uint64_t)top, (uint64_t)N};
+        const uint64_t hstr[1] = {(uint64_t)(K / 2 + top)};
+        const uint32_t hbox[2] = {(uint32_t)Fmt<FMT>::kTopRow, (uint32_t)Fmt<FMT>::kRows};
         if (!encode_tensor_map(&a.tm_codes_hi, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                                static_cast<const uint8_t *>(W->codes) + K / 2, hdims, hstr, hbox,
                                CU_TENSOR_MAP_SWIZZLE_NONE, kPromoCodes))
@@ -1207,7 +1211,7 @@ int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32
     const int32_t rows = flags & (BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32);
     if (!epilogue_ok(epi, W->N) || (flags & ~kKnown) != 0 ||
         rows == (BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32) || (FMT != 4 && rows == BQ_GEMV_ROWS32) ||
-        (FMT == 6 && W->K % 64 != 0))
+        (FMT == 6 && W->K % 64 != 0) || (FMT == 5 && W->K % 128 != 0))
         return BQ_ERR_SHAPE;
     if (!x || !y || !ws)
         return BQ_ERR_NULL;
@@ -1292,8 +1296,8 @@ extern "C" int32_t bq_gemv_geometry_of(int32_t fmt, int32_t N, int32_t K, int32_
         return BQ_ERR_NULL;
     const int32_t rows = flags & (BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32);
     constexpr int32_t kKnown = BQ_GEMV_STATIC_WEIGHTS | BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32;
-    if ((fmt != 4 && fmt != 6 && fmt != 8) || N < 1 || K < 32 || K % 32 != 0 ||
-        (fmt == 6 && K % 64 != 0) || (flags & ~kKnown) != 0 ||
+    if ((fmt != 4 && fmt != 5 && fmt != 6 && fmt != 8) || N < 1 || K < 32 || K % 32 != 0 ||
+        (fmt == 6 && K % 64 != 0) || (fmt == 5 && K % 128 != 0) || (flags & ~kKnown) != 0 ||
         rows == (BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32) || (fmt != 4 && rows == BQ_GEMV_ROWS32) ||
         sm_count < 0)
         return BQ_ERR_SHAPE;
@@ -1313,6 +1317,8 @@ extern "C" int32_t bq_gemv_geometry_of(int32_t fmt, int32_t N, int32_t K, int32_
             })
             : fmt == 6 ? matrix_geometry(6, N, K, B, rows, cap,
                                          [](int, int c) { return resident_clusters<6, 1>(c); })
+            : fmt == 5 ? matrix_geometry(5, N, K, B, rows, cap,
+                                         [](int, int c) { return resident_clusters<5, 1>(c); })
                        : matrix_geometry(8, N, K, B, rows, cap,
                                          [](int, int c) { return resident_clusters<8, 1>(c); });
     }
@@ -1347,6 +1353,8 @@ extern "C" int32_t bq_gemv_ex(int32_t fmt, const bq_qmat *W, const uint16_t *x, 
         return gemv_impl<4>(W, x, B, y, epilogue, flags, ws, ws_bytes, dev_status, stream);
     if (fmt == 6)
         return gemv_impl<6>(W, x, B, y, epilogue, flags, ws, ws_bytes, dev_status, stream);
+    if (fmt == 5)
+        return gemv_impl<5>(W, x, B, y, epilogue, flags, ws, ws_bytes, dev_status, stream);
     if (fmt == 8)
         return gemv_impl<8>(W, x, B, y, epilogue, flags, ws, ws_bytes, dev_status, stream);
     return BQ_ERR_SHAPE;

@@ -37,12 +37,13 @@ SHAPES = [(1, 32), (16, 256), (40, 2048), (777, 3072), (2048, 2048), (3072, 2048
 
 @pytest.mark.parametrize("sm_count", [148, 132, 100])
 @pytest.mark.parametrize("fmt,flags", [(4, 0), (4, bq.BQ_GEMV_ROWS16), (4, bq.BQ_GEMV_ROWS32),
-                                       (8, 0), (4, bq.BQ_GEMV_STATIC_WEIGHTS), (6, 0)])
+                                       (8, 0), (4, bq.BQ_GEMV_STATIC_WEIGHTS), (6, 0),
+                                       (5, 0)])
 @pytest.mark.parametrize("B", [1, 8])
 def test_geometry_matches_brute_force(sm_count, fmt, flags, B):
     cap = min(2 * sm_count, 512)
     for N, K in SHAPES:
-        if fmt == 6 and K % 64:
+        if (fmt == 6 and K % 64) or (fmt == 5 and K % 128):
             continue
         g = bq.gemv_geometry(fmt, N, K, B, flags, sm_count=sm_count)
         rows = g["rows"]
@@ -89,7 +90,9 @@ def test_geometry_validation():
     call = lambda fmt, N, K, B, flags, sm: bq.lib().bq_gemv_geometry_of(
         fmt, N, K, B, flags, sm, ctypes.byref(out))
     assert f(4, 64, 256, 1, 0, 148) == bq.BQ_ERR_NULL
-    assert call(5, 64, 256, 1, 0, 148) == bq.BQ_ERR_SHAPE
+    assert call(7, 64, 256, 1, 0, 148) == bq.BQ_ERR_SHAPE
+    assert call(5, 64, 192, 1, 0, 148) == bq.BQ_ERR_SHAPE          # Q5: K % 128
+    assert call(6, 64, 96, 1, 0, 148) == bq.BQ_ERR_SHAPE           # Q6: K % 64
     assert call(4, 64, 48, 1, 0, 148) == bq.BQ_ERR_SHAPE
     assert call(4, 0, 256, 1, 0, 148) == bq.BQ_ERR_SHAPE
     assert call(4, 64, 256, 0, 0, 148) == bq.BQ_ERR_BATCH
