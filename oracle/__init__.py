@@ -61,6 +61,13 @@ def lib() -> ctypes.CDLL:
             L.oracle_scales_ld.argtypes = [ctypes.c_int]
             L.oracle_quantize_q4.restype = ctypes.c_int
             L.oracle_quantize_q4.argtypes = [_c_f32p, ctypes.c_int, ctypes.c_int, _c_u8p, _c_u16p]
+            for f in ("q2", "q3"):
+                getattr(L, f"oracle_quantize_{f}").restype = ctypes.c_int
+                getattr(L, f"oracle_quantize_{f}").argtypes = [
+                    _c_f32p, ctypes.c_int, ctypes.c_int, _c_u8p, _c_u16p]
+                getattr(L, f"oracle_dequantize_{f}").restype = None
+                getattr(L, f"oracle_dequantize_{f}").argtypes = [
+                    _c_u8p, _c_u16p, ctypes.c_int, ctypes.c_int, _c_f64p]
             L.oracle_quantize_q5.restype = ctypes.c_int
             L.oracle_quantize_q5.argtypes = [_c_f32p, ctypes.c_int, ctypes.c_int, _c_u8p, _c_u16p]
             L.oracle_dequantize_q5.restype = None
@@ -79,6 +86,10 @@ def lib() -> ctypes.CDLL:
                          ctypes.c_int, ctypes.c_int, _c_f64p, _c_f64p, ctypes.c_int]
             L.oracle_gemv_q4.restype = ctypes.c_int
             L.oracle_gemv_q4.argtypes = gemv_args
+            L.oracle_gemv_q2.restype = ctypes.c_int
+            L.oracle_gemv_q2.argtypes = gemv_args
+            L.oracle_gemv_q3.restype = ctypes.c_int
+            L.oracle_gemv_q3.argtypes = gemv_args
             L.oracle_gemv_q5.restype = ctypes.c_int
             L.oracle_gemv_q5.argtypes = gemv_args
             L.oracle_gemv_q6.restype = ctypes.c_int
@@ -135,6 +146,32 @@ def quantize_q4(w: np.ndarray):
     return codes, scales
 
 
+def quantize_q2(w: np.ndarray):
+    """fp32 [N, K] -> (codes uint8 [N, K/4]: the 2-bit plane, scales
+    fp16-bits uint16 [N, ldS])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    codes = np.zeros((N, K // 4), dtype=np.uint8)
+    scales = np.zeros((N, scales_ld(K)), dtype=np.uint16)
+    rc = lib().oracle_quantize_q2(_p(w, _c_f32p), N, K, _p(codes, _c_u8p), _p(scales, _c_u16p))
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_q2 failed ({rc})")
+    return codes, scales
+
+
+def quantize_q3(w: np.ndarray):
+    """fp32 [N, K] -> (codes uint8 [N, 3K/8]: 2-bit plane then 1-bit plane,
+    scales fp16-bits uint16 [N, ldS])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    codes = np.zeros((N, 3 * K // 8), dtype=np.uint8)
+    scales = np.zeros((N, scales_ld(K)), dtype=np.uint16)
+    rc = lib().oracle_quantize_q3(_p(w, _c_f32p), N, K, _p(codes, _c_u8p), _p(scales, _c_u16p))
+    if rc != 0:
+        raise ValueError(f"oracle_quantize_q3 failed ({rc})")
+    return codes, scales
+
+
 def quantize_q5(w: np.ndarray):
     """fp32 [N, K] -> (codes uint8 [N, 5K/8]: low-nibble plane then 1-bit
     plane, scales fp16-bits uint16 [N, ldS])."""
@@ -180,6 +217,26 @@ def dequantize_q4(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     assert scales.shape == (N, scales_ld(K))
     out = np.zeros((N, K), dtype=np.float64)
     lib().oracle_dequantize_q4(_p(codes, _c_u8p), _p(scales, _c_u16p), N, K, _p(out, _c_f64p))
+    return out
+
+
+def dequantize_q2(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    N, K = codes.shape[0], codes.shape[1] * 4
+    assert scales.shape == (N, scales_ld(K))
+    out = np.zeros((N, K), dtype=np.float64)
+    lib().oracle_dequantize_q2(_p(codes, _c_u8p), _p(scales, _c_u16p), N, K, _p(out, _c_f64p))
+    return out
+
+
+def dequantize_q3(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    N, K = codes.shape[0], codes.shape[1] * 8 // 3
+    assert scales.shape == (N, scales_ld(K))
+    out = np.zeros((N, K), dtype=np.float64)
+    lib().oracle_dequantize_q3(_p(codes, _c_u8p), _p(scales, _c_u16p), N, K, _p(out, _c_f64p))
     return out
 
 
@@ -234,6 +291,18 @@ def gemv_q4(codes, scales, x_bits, nthreads: int = 1):
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint16)
     return _gemv(lib().oracle_gemv_q4, codes, scales, codes.shape[1] * 2, x_bits, nthreads)
+
+
+def gemv_q2(codes, scales, x_bits, nthreads: int = 1):
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    return _gemv(lib().oracle_gemv_q2, codes, scales, codes.shape[1] * 4, x_bits, nthreads)
+
+
+def gemv_q3(codes, scales, x_bits, nthreads: int = 1):
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    return _gemv(lib().oracle_gemv_q3, codes, scales, codes.shape[1] * 8 // 3, x_bits, nthreads)
 
 
 def gemv_q5(codes, scales, x_bits, nthreads: int = 1):

@@ -35,6 +35,18 @@
  * the low-nibble plane as Q4, then a 1-bit plane (block j at byte K/2 + 4j;
  * byte i (0..3) holds the top bit of element i + 4p in bit p, p = 0..7).
  *
+ * Q3 (the 3-bit member): d = absmax/3, q = clamp(round(w/d)+4, 0, 7), weight
+ * d*(q-4); a row of codes is 3K/8 bytes: a 2-bit plane holding the low 2 bits
+ * of each code (block j at byte 8j; byte i holds elements i, i+8, i+16 and
+ * i+24 in bits 0-1, 2-3, 4-5 and 6-7, the layout of Q6's top plane), then a
+ * 1-bit plane holding bit 2 (block j at byte K/4 + 4j; byte i (0..3) holds
+ * element i + 4p in bit p, the layout of Q5's top plane).
+ *
+ * Q2 (the 2-bit member): d = absmax/1, q = clamp(round(w/d)+2, 0, 3), weight
+ * d*(q-2); a row of codes is K/4 bytes, the 2-bit plane alone (laid out as
+ * Q3's).  The quantiser never emits code 0 (|w/d| <= 1), but the format and
+ * its dequantisation define it.
+ *
  * Readings taken where the definition is silent (each is also listed in the
  * design notes of the repository):
  *   - blocks run along K (the reduction axis), consecutive within a row;
@@ -122,7 +134,8 @@ int oracle_scales_ld(int K)
 static int oracle_quantize(const float *w, int N, int K, int levels_half,
                            int fmt, uint8_t *codes, uint16_t *scales)
 {
-    const int zero = fmt == 4 ? 8 : (fmt == 5 ? 16 : (fmt == 6 ? 32 : 0));   /* zero-point code */
+    /* zero-point code: 2, 4, 16, 32 or 8 for Q2, Q3, Q5, Q6 or Q4; Q8 has none */
+    const int zero = fmt == 2 ? 2 : fmt == 3 ? 4 : fmt == 4 ? 8 : fmt == 5 ? 16 : fmt == 6 ? 32 : 0;
     if (N < 1 || K < ORACLE_BLOCK || K % ORACLE_BLOCK)
         return -1;
     int nb = K / ORACLE_BLOCK;
@@ -155,7 +168,7 @@ static int oracle_quantize(const float *w, int N, int K, int levels_half,
                 float r = roundf(blk[i] / d);      /* fp32 division, half away */
                 if (fmt != 8) {
                     float t = r + (float)zero;
-                    float top = (float)(2 * zero - 1);   /* 15, 31 or 63 */
+                    float top = (float)(2 * zero - 1);   /* 3, 7, 15, 31 or 63 */
                     q[i] = t < 0.0f ? 0 : (t > top ? (int)top : (int)t);
                 } else {
                     q[i] = r < -127.0f ? -127 : (r > 127.0f ? 127 : (int)r);
@@ -176,6 +189,21 @@ static int oracle_quantize(const float *w, int N, int K, int levels_half,
                     for (int p = 0; p < 8; p++)
                         b |= (q[i + 4 * p] >> 4) << p;
                     hi[i] = (uint8_t)b;
+                }
+            } else if (fmt == 2 || fmt == 3) {
+                uint8_t *row = codes + (size_t)n * (fmt == 2 ? (size_t)K / 4 : 3 * (size_t)K / 8);
+                uint8_t *lo = row + (size_t)j * 8;
+                for (int i = 0; i < 8; i++)
+                    lo[i] = (uint8_t)((q[i] & 3) | ((q[i + 8] & 3) << 2) |
+                                      ((q[i + 16] & 3) << 4) | ((q[i + 24] & 3) << 6));
+                if (fmt == 3) {
+                    uint8_t *hi = row + (size_t)K / 4 + (size_t)j * 4;
+                    for (int i = 0; i < 4; i++) {
+                        int b = 0;
+                        for (int p = 0; p < 8; p++)
+                            b |= (q[i + 4 * p] >> 2) << p;
+                        hi[i] = (uint8_t)b;
+                    }
                 }
             } else if (fmt == 6) {
                 uint8_t *row = codes + (size_t)n * (3 * (size_t)K / 4);
@@ -206,6 +234,18 @@ int oracle_quantize_q4(const float *w, int N, int K, uint8_t *codes, uint16_t *s
     return oracle_quantize(w, N, K, 7, 4, codes, scales);
 }
 
+/* codes: N rows of K/4 bytes (see the header) */
+int oracle_quantize_q2(const float *w, int N, int K, uint8_t *codes, uint16_t *scales)
+{
+    return oracle_quantize(w, N, K, 1, 2, codes, scales);
+}
+
+/* codes: N rows of 3K/8 bytes (see the header) */
+int oracle_quantize_q3(const float *w, int N, int K, uint8_t *codes, uint16_t *scales)
+{
+    return oracle_quantize(w, N, K, 3, 3, codes, scales);
+}
+
 /* codes: N rows of 5K/8 bytes (see the header) */
 int oracle_quantize_q5(const float *w, int N, int K, uint8_t *codes, uint16_t *scales)
 {
@@ -230,6 +270,32 @@ static double deq_q4(const uint8_t *codes, const uint16_t *scales, int K, int ld
     int q = (i < 16) ? (byte & 0x0f) : (byte >> 4);
     double d = oracle_half_to_double(scales[(size_t)n * ldS + j]);
     return d * (double)(q - 8);
+}
+
+static double deq_q2(const uint8_t *codes, const uint16_t *scales, int K, int ldS,
+                     int n, int k)
+{
+    int j = k / ORACLE_BLOCK;
+    int i = k % ORACLE_BLOCK;
+    uint8_t byte = codes[(size_t)n * ((size_t)K / 4) + (size_t)j * 8 + (i % 8)];
+    int q = (byte >> (2 * (i / 8))) & 3;
+    double d = oracle_half_to_double(scales[(size_t)n * ldS + j]);
+    return d * (double)(q - 2);
+}
+
+static double deq_q3(const uint8_t *codes, const uint16_t *scales, int K, int ldS,
+                     int n, int k)
+{
+    int j = k / ORACLE_BLOCK;
+    int i = k % ORACLE_BLOCK;
+    const uint8_t *row = codes + (size_t)n * (3 * (size_t)K / 8);
+    uint8_t lo_byte = row[(size_t)j * 8 + (i % 8)];
+    uint8_t hi_byte = row[(size_t)K / 4 + (size_t)j * 4 + (i % 4)];
+    int lo = (lo_byte >> (2 * (i / 8))) & 3;
+    int hi = (hi_byte >> (i / 4)) & 1;
+    int q = lo | (hi << 2);
+    double d = oracle_half_to_double(scales[(size_t)n * ldS + j]);
+    return d * (double)(q - 4);
 }
 
 static double deq_q5(const uint8_t *codes, const uint16_t *scales, int K, int ldS,
@@ -279,6 +345,24 @@ void oracle_dequantize_q4(const uint8_t *codes, const uint16_t *scales, int N, i
             w[(size_t)n * K + k] = deq_q4(codes, scales, K, ldS, n, k);
 }
 
+void oracle_dequantize_q2(const uint8_t *codes, const uint16_t *scales, int N, int K,
+                          double *w)
+{
+    int ldS = oracle_scales_ld(K);
+    for (int n = 0; n < N; n++)
+        for (int k = 0; k < K; k++)
+            w[(size_t)n * K + k] = deq_q2(codes, scales, K, ldS, n, k);
+}
+
+void oracle_dequantize_q3(const uint8_t *codes, const uint16_t *scales, int N, int K,
+                          double *w)
+{
+    int ldS = oracle_scales_ld(K);
+    for (int n = 0; n < N; n++)
+        for (int k = 0; k < K; k++)
+            w[(size_t)n * K + k] = deq_q3(codes, scales, K, ldS, n, k);
+}
+
 void oracle_dequantize_q5(const uint8_t *codes, const uint16_t *scales, int N, int K,
                           double *w)
 {
@@ -313,7 +397,7 @@ void oracle_dequantize_q8(const int8_t *codes, const uint16_t *scales, int N, in
  * output is still one plain sequential sum.
  * ------------------------------------------------------------------------ */
 typedef struct {
-    int fmt;                  /* 4, 5, 6 or 8 */
+    int fmt;                  /* 2, 3, 4, 5, 6 or 8 */
     const void *codes;
     const uint16_t *scales;
     int N, K, ldS;
@@ -329,7 +413,9 @@ static void gemv_rows(const gemv_job *t)
         for (int b = 0; b < t->B; b++) {
             double s = 0.0, sa = 0.0;
             for (int k = 0; k < t->K; k++) {
-                double w = (t->fmt == 4)   ? deq_q4((const uint8_t *)t->codes, t->scales, t->K, t->ldS, n, k)
+                double w = (t->fmt == 2)   ? deq_q2((const uint8_t *)t->codes, t->scales, t->K, t->ldS, n, k)
+                           : (t->fmt == 3) ? deq_q3((const uint8_t *)t->codes, t->scales, t->K, t->ldS, n, k)
+                           : (t->fmt == 4) ? deq_q4((const uint8_t *)t->codes, t->scales, t->K, t->ldS, n, k)
                            : (t->fmt == 5) ? deq_q5((const uint8_t *)t->codes, t->scales, t->K, t->ldS, n, k)
                            : (t->fmt == 6) ? deq_q6((const uint8_t *)t->codes, t->scales, t->K, t->ldS, n, k)
                                            : deq_q8((const int8_t *)t->codes, t->scales, t->K, t->ldS, n, k);
@@ -393,6 +479,18 @@ int oracle_gemv_q4(const uint8_t *codes, const uint16_t *scales, int N, int K,
                    const uint16_t *x, int B, int ldx, double *y, double *absy, int nthreads)
 {
     return oracle_gemv(4, codes, scales, N, K, x, B, ldx, y, absy, nthreads);
+}
+
+int oracle_gemv_q2(const uint8_t *codes, const uint16_t *scales, int N, int K,
+                   const uint16_t *x, int B, int ldx, double *y, double *absy, int nthreads)
+{
+    return oracle_gemv(2, codes, scales, N, K, x, B, ldx, y, absy, nthreads);
+}
+
+int oracle_gemv_q3(const uint8_t *codes, const uint16_t *scales, int N, int K,
+                   const uint16_t *x, int B, int ldx, double *y, double *absy, int nthreads)
+{
+    return oracle_gemv(3, codes, scales, N, K, x, B, ldx, y, absy, nthreads);
 }
 
 int oracle_gemv_q5(const uint8_t *codes, const uint16_t *scales, int N, int K,

@@ -50,7 +50,7 @@ def test_double_to_half_vs_numpy_rne():
 def _expect_exact(fmt, N, nb, e, seed):
     """w = d*v with d = 2^-e and one element per block at +-levels."""
     r = np.random.default_rng(seed)
-    lv = {4: 7, 5: 15, 6: 31, 8: 127}[fmt]
+    lv = {2: 1, 3: 3, 4: 7, 5: 15, 6: 31, 8: 127}[fmt]
     v = r.integers(-lv, lv + 1, size=(N, nb, 32))
     pin = r.integers(0, 32, size=(N, nb))
     sgn = r.choice([-1, 1], size=(N, nb))
@@ -100,6 +100,55 @@ def _q5_planes(q):
     return np.concatenate([lo.reshape(N, nb * 16), hi.reshape(N, nb * 4)], axis=1).astype(np.uint8)
 
 
+def _two_bit_plane(q):
+    """[N, nb, 32] -> [N, nb, 8]: byte i holds bits 0-1 of elements i, i+8,
+    i+16, i+24 in bits 0-1, 2-3, 4-5, 6-7."""
+    q = q & 3
+    return q[..., 0:8] | (q[..., 8:16] << 2) | (q[..., 16:24] << 4) | (q[..., 24:32] << 6)
+
+
+def _q2_planes(q):
+    """Q2 code rows [N, nb, 32] -> the packed row [N, K/4], from the format text."""
+    N, nb, _ = q.shape
+    return _two_bit_plane(q).reshape(N, nb * 8).astype(np.uint8)
+
+
+def _q3_planes(q):
+    """Q3 code rows [N, nb, 32] -> the packed row [N, 3K/8], from the format
+    text: the 2-bit plane of the low bits, then the 1-bit plane of bit 2."""
+    N, nb, _ = q.shape
+    top = (q >> 2).reshape(N, nb, 8, 4)        # [.., p, i] = element i + 4p
+    hi = np.zeros((N, nb, 4), dtype=np.int64)
+    for p in range(8):
+        hi |= top[:, :, p, :] << p
+    return np.concatenate([_two_bit_plane(q).reshape(N, nb * 8), hi.reshape(N, nb * 4)],
+                          axis=1).astype(np.uint8)
+
+
+@pytest.mark.parametrize("e", [4, 7, 10, 15, 18, 24])
+def test_quantize_q2_exact_representable(e):
+    N, nb = 4, 10                      # K = 320: ldS = 16 (padded from 10)
+    v, w, d = _expect_exact(2, N, nb, e, 700 + e)
+    codes, scales = oracle.quantize_q2(w)
+    assert codes.shape == (N, 320 // 4) and scales.shape == (N, 16)
+    dbits = ((15 - e) << 10) if e <= 14 else (1 << (24 - e))
+    assert np.all(scales[:, :nb] == dbits) and np.all(scales[:, nb:] == 0)
+    assert np.array_equal(codes, _q2_planes(v + 2))
+    assert np.array_equal(oracle.dequantize_q2(codes, scales), w.astype(np.float64))
+
+
+@pytest.mark.parametrize("e", [4, 7, 10, 15, 18, 24])
+def test_quantize_q3_exact_representable(e):
+    N, nb = 4, 12                      # K = 384: ldS = 16 (padded from 12)
+    v, w, d = _expect_exact(3, N, nb, e, 600 + e)
+    codes, scales = oracle.quantize_q3(w)
+    assert codes.shape == (N, 3 * 384 // 8) and scales.shape == (N, 16)
+    dbits = ((15 - e) << 10) if e <= 14 else (1 << (24 - e))
+    assert np.all(scales[:, :nb] == dbits) and np.all(scales[:, nb:] == 0)
+    assert np.array_equal(codes, _q3_planes(v + 4))
+    assert np.array_equal(oracle.dequantize_q3(codes, scales), w.astype(np.float64))
+
+
 @pytest.mark.parametrize("e", [4, 7, 10, 15, 18, 24])
 def test_quantize_q5_exact_representable(e):
     N, nb = 4, 12                      # K = 384: ldS = 16 (padded from 12)
@@ -147,6 +196,10 @@ def test_quantize_zero_block_and_tiny_scale():
     assert np.all(s6 == 0) and np.all(c6[:, :32] == 0) and np.all(c6[:, 32:] == 0xAA)
     c5, s5 = oracle.quantize_q5(w)        # q = 16: low nibbles 0, every top bit 1
     assert np.all(s5 == 0) and np.all(c5[:, :32] == 0) and np.all(c5[:, 32:] == 0xFF)
+    c3, s3 = oracle.quantize_q3(w)        # q = 4: low 2 bits 0, every bit 2 set
+    assert np.all(s3 == 0) and np.all(c3[:, :16] == 0) and np.all(c3[:, 16:] == 0xFF)
+    c2, s2 = oracle.quantize_q2(w)        # q = 2: every 2-bit field 0b10
+    assert np.all(s2 == 0) and np.all(c2 == 0xAA)
 
 
 def test_quantize_round_half_away_and_ties():
@@ -183,9 +236,13 @@ def test_quantize_nearest_grid_point():
     c8, s8 = oracle.quantize_q8(w)
     c6, s6 = oracle.quantize_q6(w)
     c5, s5 = oracle.quantize_q5(w)
+    c3, s3 = oracle.quantize_q3(w)
+    c2, s2 = oracle.quantize_q2(w)
     for fmt, codes, scales, lv in ((4, c4, s4, (-8, 7)), (8, c8, s8, (-127, 127)),
-                                   (6, c6, s6, (-32, 31)), (5, c5, s5, (-16, 15))):
-        deq = {4: oracle.dequantize_q4, 5: oracle.dequantize_q5, 6: oracle.dequantize_q6,
+                                   (6, c6, s6, (-32, 31)), (5, c5, s5, (-16, 15)),
+                                   (3, c3, s3, (-4, 3)), (2, c2, s2, (-2, 1))):
+        deq = {2: oracle.dequantize_q2, 3: oracle.dequantize_q3, 4: oracle.dequantize_q4,
+               5: oracle.dequantize_q5, 6: oracle.dequantize_q6,
                8: oracle.dequantize_q8}[fmt](codes, scales)
         d = oracle.half_to_double(scales[:, :8]).repeat(32, axis=1)
         grid = np.arange(lv[0], lv[1] + 1)[None, None, :] * d[..., None]
@@ -195,7 +252,8 @@ def test_quantize_nearest_grid_point():
 
 # ---------------------------------------------------------- golden files ----
 @pytest.mark.parametrize("name,fmt", [("q4_block_worked.txt", 4), ("q8_block_worked.txt", 8),
-                                      ("q6_block_worked.txt", 6), ("q5_block_worked.txt", 5)])
+                                      ("q6_block_worked.txt", 6), ("q5_block_worked.txt", 5),
+                                      ("q3_block_worked.txt", 3), ("q2_block_worked.txt", 2)])
 def test_golden_worked_block(name, fmt):
     g = read_golden(name)
     v = np.array([int(t) for t in g["w_over_d"]])
@@ -207,12 +265,15 @@ def test_golden_worked_block(name, fmt):
         assert [int(b) for b in codes[0]] == [int(t, 16) for t in g["packed"]]
         q = [(codes[0, i % 16] >> (4 * (i // 16))) & 15 for i in range(32)]
         y, a = oracle.gemv_q4(codes, scales, x)
-    elif fmt in (5, 6):
-        quant, deq, gemv = ((oracle.quantize_q5, oracle.dequantize_q5, oracle.gemv_q5) if fmt == 5
-                            else (oracle.quantize_q6, oracle.dequantize_q6, oracle.gemv_q6))
+    elif fmt in (2, 3, 5, 6):
+        quant, deq, gemv = {
+            2: (oracle.quantize_q2, oracle.dequantize_q2, oracle.gemv_q2),
+            3: (oracle.quantize_q3, oracle.dequantize_q3, oracle.gemv_q3),
+            5: (oracle.quantize_q5, oracle.dequantize_q5, oracle.gemv_q5),
+            6: (oracle.quantize_q6, oracle.dequantize_q6, oracle.gemv_q6)}[fmt]
         codes, scales = quant(w)
         assert [int(b) for b in codes[0]] == [int(t, 16) for t in g["packed"]]
-        zero = 16 if fmt == 5 else 32
+        zero = {2: 2, 3: 4, 5: 16, 6: 32}[fmt]
         q = [int(round(v)) + zero for v in deq(codes, scales)[0] / d]
         y, a = gemv(codes, scales, x)
     else:
@@ -295,6 +356,52 @@ def test_q5_bit_positions_exhaustive():
             assert y[0, 0] == c - 16
 
 
+def test_q3_bit_positions_exhaustive():
+    """Every (position, code) of a 1x32 Q3 block: element i's low 2 bits in
+    bit pair i // 8 of byte i mod 8, its bit 2 in bit i // 4 of byte K/4 + i mod 4."""
+    one = np.array([0x3C00], dtype=np.uint16)          # fp16 1.0
+    scales = np.zeros((1, 8), dtype=np.uint16)
+    scales[0, 0] = one[0]
+    for p in range(32):
+        xo = np.zeros((1, 32), dtype=np.uint16)
+        xo[0, p] = one[0]
+        for c in range(8):
+            q = [4] * 32
+            q[p] = c
+            lo = [(q[i] & 3) | ((q[i + 8] & 3) << 2) | ((q[i + 16] & 3) << 4) |
+                  ((q[i + 24] & 3) << 6) for i in range(8)]
+            hi = [sum((q[i + 4 * b] >> 2) << b for b in range(8)) for i in range(4)]
+            packed = np.array([lo + hi], dtype=np.uint8)
+            deq = oracle.dequantize_q3(packed, scales)
+            expect = np.zeros((1, 32))
+            expect[0, p] = c - 4
+            assert np.array_equal(deq, expect), (p, c)
+            y, _ = oracle.gemv_q3(packed, scales, xo)
+            assert y[0, 0] == c - 4
+
+
+def test_q2_bit_positions_exhaustive():
+    """Every (position, code) of a 1x32 Q2 block: element i in bit pair
+    i // 8 of byte i mod 8."""
+    one = np.array([0x3C00], dtype=np.uint16)          # fp16 1.0
+    scales = np.zeros((1, 8), dtype=np.uint16)
+    scales[0, 0] = one[0]
+    for p in range(32):
+        xo = np.zeros((1, 32), dtype=np.uint16)
+        xo[0, p] = one[0]
+        for c in range(4):
+            q = [2] * 32
+            q[p] = c
+            packed = np.array([[q[i] | (q[i + 8] << 2) | (q[i + 16] << 4) | (q[i + 24] << 6)
+                                for i in range(8)]], dtype=np.uint8)
+            deq = oracle.dequantize_q2(packed, scales)
+            expect = np.zeros((1, 32))
+            expect[0, p] = c - 2
+            assert np.array_equal(deq, expect), (p, c)
+            y, _ = oracle.gemv_q2(packed, scales, xo)
+            assert y[0, 0] == c - 2
+
+
 def test_scale_plane_stride_and_block_index():
     """Scale (n, j) scales exactly block j of row n, with rows ldS apart."""
     N, K = 3, 96                                       # ldS = 8 > K/32 = 3
@@ -319,22 +426,31 @@ def test_scale_plane_stride_and_block_index():
     c5 = np.concatenate([np.full((N, K // 2), 0x11, dtype=np.uint8),
                          np.full((N, K // 8), 0xFF, dtype=np.uint8)], axis=1)
     assert np.array_equal(oracle.dequantize_q5(c5, scales), deq)
+    # Q3 code 5 (v = 1): low 2 bits 1 in every pair, every bit 2 set
+    c3 = np.concatenate([np.full((N, K // 4), 0x55, dtype=np.uint8),
+                         np.full((N, K // 8), 0xFF, dtype=np.uint8)], axis=1)
+    assert np.array_equal(oracle.dequantize_q3(c3, scales), deq)
+    # Q2 code 3 (v = 1) in every pair
+    assert np.array_equal(oracle.dequantize_q2(np.full((N, K // 4), 0xFF, dtype=np.uint8),
+                                               scales), deq)
 
 
 # ------------------------------------------------------------------ GEMV ----
 def _rand_planes(fmt, N, K, seed):
     w = synth.weights_f32(synth.key(seed, 91, 0, 0, 0), N, K)
-    return {4: oracle.quantize_q4, 5: oracle.quantize_q5, 6: oracle.quantize_q6,
-            8: oracle.quantize_q8}[fmt](w)
+    return {2: oracle.quantize_q2, 3: oracle.quantize_q3, 4: oracle.quantize_q4,
+            5: oracle.quantize_q5, 6: oracle.quantize_q6, 8: oracle.quantize_q8}[fmt](w)
 
 
-_DEQ = {4: lambda c, s: oracle.dequantize_q4(c, s), 5: lambda c, s: oracle.dequantize_q5(c, s),
+_DEQ = {2: lambda c, s: oracle.dequantize_q2(c, s), 3: lambda c, s: oracle.dequantize_q3(c, s),
+        4: lambda c, s: oracle.dequantize_q4(c, s), 5: lambda c, s: oracle.dequantize_q5(c, s),
         6: lambda c, s: oracle.dequantize_q6(c, s), 8: lambda c, s: oracle.dequantize_q8(c, s)}
-_GEMV = {4: lambda *a, **k: oracle.gemv_q4(*a, **k), 5: lambda *a, **k: oracle.gemv_q5(*a, **k),
+_GEMV = {2: lambda *a, **k: oracle.gemv_q2(*a, **k), 3: lambda *a, **k: oracle.gemv_q3(*a, **k),
+         4: lambda *a, **k: oracle.gemv_q4(*a, **k), 5: lambda *a, **k: oracle.gemv_q5(*a, **k),
          6: lambda *a, **k: oracle.gemv_q6(*a, **k), 8: lambda *a, **k: oracle.gemv_q8(*a, **k)}
 
 
-@pytest.mark.parametrize("fmt", [4, 5, 6, 8])
+@pytest.mark.parametrize("fmt", [2, 3, 4, 5, 6, 8])
 def test_gemv_one_hot_returns_columns(fmt):
     N, K = 7, 96
     codes, scales = _rand_planes(fmt, N, K, 1)
@@ -348,7 +464,7 @@ def test_gemv_one_hot_returns_columns(fmt):
         assert np.array_equal(y, deq[:, b0:b0 + 8].T)
 
 
-@pytest.mark.parametrize("fmt", [4, 5, 6, 8])
+@pytest.mark.parametrize("fmt", [2, 3, 4, 5, 6, 8])
 def test_gemv_all_ones_returns_row_sums(fmt):
     import math
     N, K = 11, 160
@@ -369,6 +485,13 @@ def _unpack_fraction(fmt, codes, scales, n, k):
     if fmt == 8:
         return d * int(codes[n, k])
     i = k % 32
+    if fmt in (2, 3):
+        lo = (int(codes[n, (k // 32) * 8 + i % 8]) >> (2 * (i // 8))) & 3
+        if fmt == 2:
+            return d * (lo - 2)
+        K = codes.shape[1] * 8 // 3
+        top = (int(codes[n, K // 4 + (k // 32) * 4 + i % 4]) >> (i // 4)) & 1
+        return d * ((lo | (top << 2)) - 4)
     byte = int(codes[n, (k // 32) * 16 + i % 16])
     q = byte & 15 if i < 16 else byte >> 4
     if fmt == 6:
@@ -382,7 +505,7 @@ def _unpack_fraction(fmt, codes, scales, n, k):
     return d * (q - 8)
 
 
-@pytest.mark.parametrize("fmt", [4, 5, 6, 8])
+@pytest.mark.parametrize("fmt", [2, 3, 4, 5, 6, 8])
 @pytest.mark.parametrize("N,K,B", [(1, 32, 1), (3, 64, 2), (8, 96, 8), (5, 32, 3), (2, 96, 5)])
 def test_gemv_brute_force_exact(fmt, N, K, B):
     codes, scales = _rand_planes(fmt, N, K, 10 * N + K + B)
@@ -400,7 +523,7 @@ def test_gemv_brute_force_exact(fmt, N, K, B):
             assert abs(Fraction(a[b, n]) - exact_abs) <= exact_abs * Fraction(1, 2 ** 50)
 
 
-@pytest.mark.parametrize("fmt", [4, 5, 6, 8])
+@pytest.mark.parametrize("fmt", [2, 3, 4, 5, 6, 8])
 def test_gemv_batch_rows_independent_and_threads(fmt):
     N, K, B = 37, 256, 6
     codes, scales = _rand_planes(fmt, N, K, 5)
