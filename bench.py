@@ -85,6 +85,8 @@ def load_peaks():
 
 WORKLOADS = {
     synth.DENSE_H2048.name: synth.DENSE_H2048,
+    synth.dense_h2048(2).name: synth.dense_h2048(2),
+    synth.dense_h2048(3).name: synth.dense_h2048(3),
     synth.dense_h2048(5).name: synth.dense_h2048(5),
     synth.dense_h2048(6).name: synth.dense_h2048(6),
     synth.dense_h2048(8).name: synth.dense_h2048(8),
@@ -94,7 +96,7 @@ WORKLOADS = {
 for _b in (1, 8):
     _w = synth.moe_h2048(_b)
     WORKLOADS[_w.name] = _w
-for _f in (4, 5, 6, 8):
+for _f in (2, 3, 4, 5, 6, 8):
     for _b in (1, 2, 4, 8):
         _w = synth.dense_h4096(_f, _b)
         WORKLOADS[_w.name] = _w
@@ -204,7 +206,8 @@ class DenseStep:
         st = torch.zeros(1, dtype=torch.int32, device=device)
         ws_max = 0
         stages = fused_stages(wl)
-        Kc = lambda K: {4: K // 2, 5: 5 * K // 8, 6: 3 * K // 4, 8: K}[wl.fmt]   # code bytes per row
+        Kc = lambda K: {2: K // 4, 3: 3 * K // 8, 4: K // 2, 5: 5 * K // 8, 6: 3 * K // 4,
+                        8: K}[wl.fmt]   # code bytes per row
         pending = []            # (layer, stage, mats, K, Ntot, codes, scales, x-or-None, out spec)
         for layer in range(wl.layers):
             h_shape = None
@@ -457,7 +460,8 @@ def oracle_sample(wl: synth.DenseWorkload, seed: int = 0):
         parts = [synth.weights_f32(synth.key(seed, wl.wid, 0, wl.mats.index(m), synth.KIND_W), m.N, K)
                  for m in group]
         w = np.concatenate(parts, axis=0)
-        codes, scales = {4: oracle.quantize_q4, 5: oracle.quantize_q5, 6: oracle.quantize_q6,
+        codes, scales = {2: oracle.quantize_q2, 3: oracle.quantize_q3, 4: oracle.quantize_q4,
+                         5: oracle.quantize_q5, 6: oracle.quantize_q6,
                          8: oracle.quantize_q8}[wl.fmt](w)
         x = synth.activations_f16_bits(synth.key(seed, wl.wid, 0, s, synth.KIND_X), wl.B, K)
         nbytes = synth.packed_bytes(wl.fmt, w.shape[0], K) + wl.B * K * 2 + wl.B * w.shape[0] * 4
@@ -515,8 +519,8 @@ def oracle_job(wl):
 
     def run():
         for codes, scales, x, _ in mats:
-            {4: oracle.gemv_q4, 5: oracle.gemv_q5, 6: oracle.gemv_q6,
-             8: oracle.gemv_q8}[wl.fmt](codes, scales, x, nthreads=threads)
+            {2: oracle.gemv_q2, 3: oracle.gemv_q3, 4: oracle.gemv_q4, 5: oracle.gemv_q5,
+             6: oracle.gemv_q6, 8: oracle.gemv_q8}[wl.fmt](codes, scales, x, nthreads=threads)
     return run, nbytes
 
 

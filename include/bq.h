@@ -213,7 +213,7 @@ enum { BQ_GEMV_STATIC_WEIGHTS = 1, BQ_GEMV_ROWS16 = 2, BQ_GEMV_ROWS32 = 4 };
  * (BQ_ERR_SHAPE, BQ_ERR_BATCH, BQ_ERR_NULL), BQ_ERR_CUDA if sm_count is 0
  * and no device can be queried. */
 typedef struct bq_gemv_geometry {
-    int32_t rows;               /* rows per chunk: 16 or 32 (Q4), 16 (Q8) */
+    int32_t rows;               /* rows per chunk: 16 or 32 (Q4), 16 (other formats) */
     int32_t chunks;             /* bands x chunks_per_band */
     int32_t chunks_per_band;    /* ceil(K / 256) */
     int32_t chunks_per_worker;
@@ -227,10 +227,13 @@ typedef struct bq_gemv_geometry {
 BQ_API int32_t bq_gemv_geometry_of(int32_t fmt, int32_t N, int32_t K, int32_t B, int32_t flags,
                                    int32_t sm_count, bq_gemv_geometry *out);
 
-/* Q4, Q5, Q6 or Q8 decode GEMV with an output epilogue.
- *   fmt        4, 5, 6 or 8 (Q6: K a multiple of 64, codes as bq_quantize_q6
- *              lays them out, rows of 3K/4 bytes; Q5: K a multiple of 128,
- *              as bq_quantize_q5, rows of 5K/8 bytes; both 16-row work units)
+/* Q2, Q3, Q4, Q5, Q6 or Q8 decode GEMV with an output epilogue.
+ *   fmt        2, 3, 4, 5, 6 or 8 (Q6: K a multiple of 64, codes as
+ *              bq_quantize_q6 lays them out, rows of 3K/4 bytes; Q5: K a
+ *              multiple of 128, as bq_quantize_q5, rows of 5K/8 bytes; Q3: K a
+ *              multiple of 128, as bq_quantize_q3, rows of 3K/8 bytes; Q2: K a
+ *              multiple of 64, as bq_quantize_q2, rows of K/4 bytes; all four
+ *              in 16-row work units)
  *   y          device: fp32 [B][N] (BQ_EPI_NONE) or fp16 bits [B][N/2]
  *              (BQ_EPI_SWIGLU, N a multiple of 16), 16-byte aligned
  *   epilogue   BQ_EPI_*; anything else returns BQ_ERR_SHAPE
@@ -368,6 +371,19 @@ BQ_API int32_t bq_quantize_q6(const float *w, int32_t N, int32_t K, uint8_t *cod
  * holds the top bit of element i + 4p in bit p, p = 0..7). */
 BQ_API int32_t bq_quantize_q5(const float *w, int32_t N, int32_t K, uint8_t *codes, uint16_t *scales);
 
+/* Q3, the 3-bit member: d = fp16_rne(a / 3), q = clamp(round-half-away(w / d)
+ * + 4, 0, 7), zero-point code 4.  codes: uint8 [N][3K/8], each row a 2-bit
+ * plane of the low 2 bits (K/4 bytes: block j at byte 8j, byte i = those of
+ * elements i, i+8, i+16, i+24 in bits 0-1, 2-3, 4-5, 6-7) followed by a
+ * 1-bit plane of bit 2 (K/8 bytes: block j at byte K/4 + 4j, byte i = 0..3
+ * holds that of element i + 4p in bit p). */
+BQ_API int32_t bq_quantize_q3(const float *w, int32_t N, int32_t K, uint8_t *codes, uint16_t *scales);
+
+/* Q2, the 2-bit member: d = fp16_rne(a / 1), q = clamp(round-half-away(w / d)
+ * + 2, 0, 3), zero-point code 2 (the quantiser emits codes 1..3; code 0 is
+ * -2d).  codes: uint8 [N][K/4], the 2-bit plane alone (laid out as Q3's). */
+BQ_API int32_t bq_quantize_q2(const float *w, int32_t N, int32_t K, uint8_t *codes, uint16_t *scales);
+
 /* Dequantise planes into fp32 weights [N][K] (exact: d * q fits fp32). */
 BQ_API int32_t bq_dequantize_q8(const int8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
                          float *w);
@@ -376,6 +392,10 @@ BQ_API int32_t bq_dequantize_q4(const uint8_t *codes, const uint16_t *scales, in
 BQ_API int32_t bq_dequantize_q6(const uint8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
                          float *w);
 BQ_API int32_t bq_dequantize_q5(const uint8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
+                         float *w);
+BQ_API int32_t bq_dequantize_q3(const uint8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
+                         float *w);
+BQ_API int32_t bq_dequantize_q2(const uint8_t *codes, const uint16_t *scales, int32_t N, int32_t K,
                          float *w);
 
 /* Planes <-> interleaved blocks.  blocks: N*(K/32) records, row-major over
@@ -408,6 +428,13 @@ BQ_API int32_t bq_quantize_q6_dev(const float *w, int32_t N, int32_t K, uint8_t 
 /* Q5 on the GPU: K must be a multiple of 128 (rows of 5K/8 bytes stay
  * 16-byte aligned), else BQ_ERR_SHAPE. */
 BQ_API int32_t bq_quantize_q5_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
+                           uint16_t *scales, int32_t *dev_status, void *stream);
+/* Q3 on the GPU: K must be a multiple of 128 (rows of 3K/8 bytes keep both
+ * planes aligned for the block stores), else BQ_ERR_SHAPE. */
+BQ_API int32_t bq_quantize_q3_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
+                           uint16_t *scales, int32_t *dev_status, void *stream);
+/* Q2 on the GPU: any K that is a multiple of 32. */
+BQ_API int32_t bq_quantize_q2_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
                            uint16_t *scales, int32_t *dev_status, void *stream);
 
 #ifdef __cplusplus

@@ -80,6 +80,10 @@ _SIGS = {
     "bq_quantize_q4": (_i32, [_vp, _i32, _i32, _vp, _vp]),
     "bq_dequantize_q8": (_i32, [_vp, _vp, _i32, _i32, _vp]),
     "bq_dequantize_q4": (_i32, [_vp, _vp, _i32, _i32, _vp]),
+    "bq_quantize_q2": (_i32, [_vp, _i32, _i32, _vp, _vp]),
+    "bq_quantize_q3": (_i32, [_vp, _i32, _i32, _vp, _vp]),
+    "bq_dequantize_q2": (_i32, [_vp, _vp, _i32, _i32, _vp]),
+    "bq_dequantize_q3": (_i32, [_vp, _vp, _i32, _i32, _vp]),
     "bq_quantize_q6": (_i32, [_vp, _i32, _i32, _vp, _vp]),
     "bq_quantize_q5": (_i32, [_vp, _i32, _i32, _vp, _vp]),
     "bq_dequantize_q5": (_i32, [_vp, _vp, _i32, _i32, _vp]),
@@ -90,6 +94,8 @@ _SIGS = {
     "bq_blocks_to_planes_q8": (_i32, [_vp, _i32, _i32, _vp, _vp]),
     "bq_quantize_q4_dev": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "bq_quantize_q8_dev": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "bq_quantize_q2_dev": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "bq_quantize_q3_dev": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "bq_quantize_q6_dev": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     "bq_quantize_q5_dev": (_i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
 }
@@ -173,7 +179,7 @@ def gemv(fmt: int, W: bq_qmat, x, y, ws, status=None, stream=None, epilogue: int
     Q6, an epilogue (BQ_EPI_SWIGLU: y is fp16 [B, N/2]) or flags go through
     bq_gemv_ex."""
     B = x.shape[0]
-    if epilogue == BQ_EPI_NONE and flags == 0 and fmt in (4, 8):   # (Q5, Q6: bq_gemv_ex)
+    if epilogue == BQ_EPI_NONE and flags == 0 and fmt in (4, 8):   # (Q2, Q3, Q5, Q6: bq_gemv_ex)
         fn = lib().bq_gemv_q4 if fmt == 4 else lib().bq_gemv_q8
         rc = fn(ctypes.byref(W), x.data_ptr(), B, y.data_ptr(), ws.data_ptr(),
                 ws.numel() * ws.element_size(), _ptr(status), _stream_ptr(stream))
@@ -232,8 +238,8 @@ class StepPlan:
 
 def quantize_dev(fmt: int, w, codes, scales, status=None, stream=None) -> None:
     N, K = w.shape
-    fn = {4: lib().bq_quantize_q4_dev, 5: lib().bq_quantize_q5_dev, 6: lib().bq_quantize_q6_dev,
-          8: lib().bq_quantize_q8_dev}[fmt]
+    fn = {2: lib().bq_quantize_q2_dev, 3: lib().bq_quantize_q3_dev, 4: lib().bq_quantize_q4_dev,
+          5: lib().bq_quantize_q5_dev, 6: lib().bq_quantize_q6_dev, 8: lib().bq_quantize_q8_dev}[fmt]
     check(f"bq_quantize_q{fmt}_dev",
           fn(w.data_ptr(), N, K, codes.data_ptr(), scales.data_ptr(), _ptr(status),
              _stream_ptr(stream)))

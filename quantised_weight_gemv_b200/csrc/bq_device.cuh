@@ -71,7 +71,8 @@ template <int MT> struct Fmt<4, MT> {
     static_assert(MT == 1 || MT == 2, "Q4 chunks are 16 or 32 rows");
     static constexpr int kMT = MT;                      // m-tiles of 16 rows per chunk
     static constexpr int kRows = 16 * kMT;              // rows per chunk / band
-    static constexpr int kBoxes = 1;                    // 128-byte-wide code boxes
+    static constexpr int kBoxes = 1;                    // code boxes of the first plane
+    static constexpr int kLoRow = 128;                  // bytes per row of one such box
     static constexpr int kCodeBytes = kRows * 128;      // 2 or 4 KB
     static constexpr int kCodeLoad = kCodeBytes;        // code bytes one chunk's loads bring
     static constexpr int kScaleBytes = kRows * 16;      // kRows x 8 fp16
@@ -84,6 +85,7 @@ template <int FMT> struct FmtTop {
     static constexpr int kMT = 1;
     static constexpr int kRows = 16;
     static constexpr int kBoxes = 1;                    // + the top-bit box
+    static constexpr int kLoRow = 128;
     static constexpr int kTopRow = FMT == 6 ? 64 : 32;  // top-bit bytes per row and chunk
     static constexpr int kCodeLoad = kRows * 128 + kRows * kTopRow;
     static constexpr int kCodeBytes = 3072;             // slot stride
@@ -92,10 +94,27 @@ template <int FMT> struct FmtTop {
 };
 template <> struct Fmt<6, 1> : FmtTop<6> {};
 template <> struct Fmt<5, 1> : FmtTop<5> {};
+// Q2 / Q3 chunks: 16 rows x 256 weights, the 2-bit plane as one 64-byte box
+// (64-byte swizzle: slots 512-byte aligned) and, for Q3, the 1-bit plane as
+// one 32-byte box after it (no swizzle): 1 KB / 1.5 KB of codes per chunk.
+template <int FMT> struct FmtLow2 {
+    static constexpr int kMT = 1;
+    static constexpr int kRows = 16;
+    static constexpr int kBoxes = 1;                    // (+ the top-bit box for Q3)
+    static constexpr int kLoRow = 64;
+    static constexpr int kTopRow = FMT == 3 ? 32 : 0;
+    static constexpr int kCodeLoad = kRows * (kLoRow + kTopRow);
+    static constexpr int kCodeBytes = kCodeLoad;        // slot stride: 1024 or 1536
+    static constexpr int kScaleBytes = kRows * 16;
+    static constexpr int kStages = BQ_STAGES;
+};
+template <> struct Fmt<2, 1> : FmtLow2<2> {};
+template <> struct Fmt<3, 1> : FmtLow2<3> {};
 template <> struct Fmt<8, 1> {
     static constexpr int kMT = 1;
     static constexpr int kRows = 16;
     static constexpr int kBoxes = 2;
+    static constexpr int kLoRow = 128;
     static constexpr int kCodeBytes = 2 * kRows * 128;  // 4 KB
     static constexpr int kCodeLoad = kCodeBytes;
     static constexpr int kScaleBytes = kRows * 16;
@@ -106,6 +125,8 @@ static_assert(Fmt<5, 1>::kCodeLoad <= Fmt<5, 1>::kCodeBytes &&
                   Fmt<5, 1>::kCodeBytes % 1024 == 0 && Fmt<6, 1>::kCodeBytes % 1024 == 0 &&
                   Fmt<8, 1>::kCodeBytes % 1024 == 0,
               "code slots hold a chunk and stay 1024-byte aligned");
+static_assert(Fmt<2, 1>::kCodeBytes % 512 == 0 && Fmt<3, 1>::kCodeBytes % 512 == 0,
+              "Q2 / Q3 code slots stay 512-byte aligned (the 64-byte swizzle's period)");
 
 template <int FMT, int MT = default_mt<FMT>()>
 constexpr int smem_bytes()
@@ -358,20 +379,21 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // (block_offset).  Every product is exact; the scale 2^-24 (2^-20 for Q4) is
 // undone at the store.
 
-// f16x2 of -z' * 2^-24 (a subnormal): z' = 128 (Q4: 8 * 16; Q8: 128), 256
-// (Q5: 16 * 16) or 512 (Q6: 32 * 16).
+// f16x2 of -z' * 2^-24: z' = 128 (Q4: 8 * 16; Q8: 128), 256 (Q5: 16 * 16),
+// 512 (Q6: 32 * 16; Q2: 2 * 256) or 1024 (Q3: 4 * 256, the smallest normal).
 template <int FMT>
 __host__ __device__ constexpr uint32_t zero_point_pair()
 {
-    return FMT == 6 ? 0x82008200u : (FMT == 5 ? 0x81008100u : 0x80808080u);
+    return FMT == 3 ? 0x84008400u
+                    : (FMT == 6 || FMT == 2 ? 0x82008200u : (FMT == 5 ? 0x81008100u : 0x80808080u));
 }
 
-// The y of a band is stored as acc * 2^20 (Q4 and Q6: codes enter at
-// 16 * 2^-24) or acc * 2^24 (Q8).
+// The y of a band is stored as acc * 2^20 (Q4, Q5, Q6: codes enter at
+// 16 * 2^-24), acc * 2^16 (Q2, Q3: at 256 * 2^-24) or acc * 2^24 (Q8).
 template <int FMT>
 __host__ __device__ constexpr float unscale()
 {
-    return FMT == 8 ? 16777216.0f : 1048576.0f;
+    return FMT == 8 ? 16777216.0f : (FMT == 2 || FMT == 3 ? 65536.0f : 1048576.0f);
 }
 
 __device__ __forceinline__ float half_lo(uint32_t v)
@@ -527,6 +549,129 @@ __device__ __forceinline__ void block_qtop(uint32_t addr, uint32_t addr_hi, uint
           "n"(kTop8), "n"(kTopMask));
 }
 
+// One Q2 or Q3 block for a 16-row m-tile.  `addr` is row g's 4-byte group of
+// the 2-bit plane at byte 4(t%2) of the block: its byte i holds elements
+// 4(t%2)+i+8p in bit pair p, which puts element 4t+i in pair t/2 and element
+// 4t+16+i in pair t/2+2.  After the bytes are spread over fp16 lanes, the
+// multipliers mh1 = 2^(8-2(t/2)) and mh2 = 2^(4-2(t/2)) move those pairs to
+// bits 8-9 (u = 256 * low 2 bits).  Q3 adds bit 2 of each code from
+// `addr_hi`, row g's 4 bytes of the 1-bit plane (Q5's layout: bit t of byte
+// i for element 4t+i, bit t+4 for 4t+16+i), moved to bit 10 by mh3 =
+// 2^(10-t) and mh4 = 2^(6-t).  So a lane holds u = 256 q (q < 8, u < 2048):
+// an fp16 subnormal, or from u = 1024 on a normal of the lowest binade,
+// which is still exactly u * 2^-24.  Row g+8 is 8 rows on: 512 bytes in the
+// 2-bit box, 256 in the 1-bit box.  The multiplies run on the FMA pipe.
+template <int FMT>
+__device__ __forceinline__ void block_q23(uint32_t addr, uint32_t addr_hi, uint2 xa, uint2 xb,
+                                          const float (&off)[4], float dg, float dg8,
+                                          float (&acc)[4], uint32_t mh1, uint32_t mh2,
+                                          uint32_t mh3, uint32_t mh4)
+{
+    if constexpr (FMT == 2) {
+        asm("{\n\t"
+            ".reg .b32 w0, w8, p01, p23, q01, q23, a0, a1, a2, a3;\n\t"
+            ".reg .f32 c0, c1, c2, c3;\n\t"
+            "ld.shared.b32 w0, [%4];\n\t"
+            "ld.shared.b32 w8, [%4+512];\n\t"
+            "prmt.b32 p01, w0, 0, 0x4140;\n\t"
+            "prmt.b32 p23, w0, 0, 0x4342;\n\t"
+            "prmt.b32 q01, w8, 0, 0x4140;\n\t"
+            "prmt.b32 q23, w8, 0, 0x4342;\n\t"
+            "mul.lo.u32 a0, p01, %15;\n\t"
+            "mul.lo.u32 a1, q01, %15;\n\t"
+            "mul.lo.u32 a2, p23, %15;\n\t"
+            "mul.lo.u32 a3, q23, %15;\n\t"
+            "and.b32 a0, a0, 0x03000300;\n\t"
+            "and.b32 a1, a1, 0x03000300;\n\t"
+            "and.b32 a2, a2, 0x03000300;\n\t"
+            "and.b32 a3, a3, 0x03000300;\n\t"
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {c0,c1,c2,c3}, {a0,a1,a2,a3}, {%5,%6}, "
+            "{%9,%10,%11,%12};\n\t"
+            "mul.lo.u32 a0, p01, %16;\n\t"
+            "mul.lo.u32 a1, q01, %16;\n\t"
+            "mul.lo.u32 a2, p23, %16;\n\t"
+            "mul.lo.u32 a3, q23, %16;\n\t"
+            "and.b32 a0, a0, 0x03000300;\n\t"
+            "and.b32 a1, a1, 0x03000300;\n\t"
+            "and.b32 a2, a2, 0x03000300;\n\t"
+            "and.b32 a3, a3, 0x03000300;\n\t"
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {c0,c1,c2,c3}, {a0,a1,a2,a3}, {%7,%8}, "
+            "{c0,c1,c2,c3};\n\t"
+            "fma.rn.f32 %0, %13, c0, %0;\n\t"
+            "fma.rn.f32 %1, %13, c1, %1;\n\t"
+            "fma.rn.f32 %2, %14, c2, %2;\n\t"
+            "fma.rn.f32 %3, %14, c3, %3;\n\t}"
+            : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
+            : "r"(addr), "r"(xa.x), "r"(xa.y), "r"(xb.x), "r"(xb.y), "f"(off[0]), "f"(off[1]),
+              "f"(off[2]), "f"(off[3]), "f"(dg), "f"(dg8), "r"(mh1), "r"(mh2));
+        (void)addr_hi;
+        (void)mh3;
+        (void)mh4;
+    } else {
+        asm("{\n\t"
+            ".reg .b32 w0, w8, h0, h8, p01, p23, q01, q23, e01, e23, f01, f23, a0, a1, a2, a3, t0, t1, t2, t3;\n\t"
+            ".reg .f32 c0, c1, c2, c3;\n\t"
+            "ld.shared.b32 w0, [%4];\n\t"
+            "ld.shared.b32 w8, [%4+512];\n\t"
+            "ld.shared.b32 h0, [%5];\n\t"
+            "ld.shared.b32 h8, [%5+256];\n\t"
+            "prmt.b32 p01, w0, 0, 0x4140;\n\t"
+            "prmt.b32 p23, w0, 0, 0x4342;\n\t"
+            "prmt.b32 q01, w8, 0, 0x4140;\n\t"
+            "prmt.b32 q23, w8, 0, 0x4342;\n\t"
+            "prmt.b32 e01, h0, 0, 0x4140;\n\t"
+            "prmt.b32 e23, h0, 0, 0x4342;\n\t"
+            "prmt.b32 f01, h8, 0, 0x4140;\n\t"
+            "prmt.b32 f23, h8, 0, 0x4342;\n\t"
+            // elements 4t..4t+3: pair t/2 at bits 8-9 | bit t of the 1-bit group at bit 10
+            "mul.lo.u32 a0, p01, %15;\n\t"
+            "mul.lo.u32 a1, q01, %15;\n\t"
+            "mul.lo.u32 a2, p23, %15;\n\t"
+            "mul.lo.u32 a3, q23, %15;\n\t"
+            "mul.lo.u32 t0, e01, %17;\n\t"
+            "mul.lo.u32 t1, f01, %17;\n\t"
+            "mul.lo.u32 t2, e23, %17;\n\t"
+            "mul.lo.u32 t3, f23, %17;\n\t"
+            "and.b32 t0, t0, 0x04000400;\n\t"
+            "and.b32 t1, t1, 0x04000400;\n\t"
+            "and.b32 t2, t2, 0x04000400;\n\t"
+            "and.b32 t3, t3, 0x04000400;\n\t"
+            "lop3.b32 a0, a0, 0x03000300, t0, 0xEA;\n\t"
+            "lop3.b32 a1, a1, 0x03000300, t1, 0xEA;\n\t"
+            "lop3.b32 a2, a2, 0x03000300, t2, 0xEA;\n\t"
+            "lop3.b32 a3, a3, 0x03000300, t3, 0xEA;\n\t"
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {c0,c1,c2,c3}, {a0,a1,a2,a3}, {%6,%7}, "
+            "{%10,%11,%12,%13};\n\t"
+            // elements 4t+16..4t+19: pair t/2+2 | bit t+4
+            "mul.lo.u32 a0, p01, %16;\n\t"
+            "mul.lo.u32 a1, q01, %16;\n\t"
+            "mul.lo.u32 a2, p23, %16;\n\t"
+            "mul.lo.u32 a3, q23, %16;\n\t"
+            "mul.lo.u32 t0, e01, %18;\n\t"
+            "mul.lo.u32 t1, f01, %18;\n\t"
+            "mul.lo.u32 t2, e23, %18;\n\t"
+            "mul.lo.u32 t3, f23, %18;\n\t"
+            "and.b32 t0, t0, 0x04000400;\n\t"
+            "and.b32 t1, t1, 0x04000400;\n\t"
+            "and.b32 t2, t2, 0x04000400;\n\t"
+            "and.b32 t3, t3, 0x04000400;\n\t"
+            "lop3.b32 a0, a0, 0x03000300, t0, 0xEA;\n\t"
+            "lop3.b32 a1, a1, 0x03000300, t1, 0xEA;\n\t"
+            "lop3.b32 a2, a2, 0x03000300, t2, 0xEA;\n\t"
+            "lop3.b32 a3, a3, 0x03000300, t3, 0xEA;\n\t"
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {c0,c1,c2,c3}, {a0,a1,a2,a3}, {%8,%9}, "
+            "{c0,c1,c2,c3};\n\t"
+            "fma.rn.f32 %0, %14, c0, %0;\n\t"
+            "fma.rn.f32 %1, %14, c1, %1;\n\t"
+            "fma.rn.f32 %2, %19, c2, %2;\n\t"
+            "fma.rn.f32 %3, %19, c3, %3;\n\t}"
+            : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
+            : "r"(addr), "r"(addr_hi), "r"(xa.x), "r"(xa.y), "r"(xb.x), "r"(xb.y), "f"(off[0]),
+              "f"(off[1]), "f"(off[2]), "f"(off[3]), "f"(dg), "r"(mh1), "r"(mh2), "r"(mh3),
+              "r"(mh4), "f"(dg8));
+    }
+}
+
 // One Q8 block for the 16-row m-tile: addr_a / addr_b are row g's 4-byte
 // groups in the block's two 16-element halves.
 __device__ __forceinline__ void block_q8(uint32_t addr_a, uint32_t addr_b, uint2 xa, uint2 xb,
@@ -591,13 +736,18 @@ __device__ __forceinline__ float4 lds128_f32(uint32_t addr)
 // Per-lane swizzled offsets of the 8 blocks of a chunk row (constant for a
 // lane): TMA's 128-byte swizzle XORs the 16-byte granule index with the row
 // index mod 8, and row mod 8 == g for every row this lane reads.  For Q8 the
-// two 16-byte halves of a block are packed as two 16-bit offsets.
+// two 16-byte halves of a block are packed as two 16-bit offsets.  Q2 / Q3's
+// 2-bit plane has 64-byte rows under the 64-byte swizzle: a block is 8
+// bytes, half of a 16-byte granule, and the granule index (0..3) is XORed
+// with bits 7-8 of the offset, (row / 2) mod 4 -- the same for rows g and g+8.
 template <int FMT>
 __device__ __forceinline__ void lane_swizzle(int g, int (&sw)[8])
 {
 #pragma unroll
     for (int jb = 0; jb < 8; jb++) {
-        if constexpr (FMT == 4 || FMT == 5 || FMT == 6) {   // (Q5, Q6: the low-nibble plane)
+        if constexpr (FMT == 2 || FMT == 3) {
+            sw[jb] = ((((jb >> 1) ^ (g >> 1)) & 3) << 4) | ((jb & 1) << 3);
+        } else if constexpr (FMT == 4 || FMT == 5 || FMT == 6) {   // (Q5, Q6: the low-nibble plane)
             sw[jb] = ((jb ^ g) & 7) << 4;
         } else {
             const int jj = jb & 3;
@@ -648,13 +798,17 @@ __device__ __forceinline__ void chunk_mma(uint32_t codes_s, uint32_t scales_s, i
         sc[mt][0] = lds128_u32(scales_s + (16 * mt + g) * 16);
         sc[mt][1] = lds128_u32(scales_s + (16 * mt + g + 8) * 16);
     }
-    const uint32_t lane_codes = codes_s + g * 128 + 4 * t;
-    // Q6 / Q5: this lane's top-bit group (after the 16 rows of low nibbles;
-    // rows 64 / 32 bytes apart) and the multipliers that move its bits to 8.
-    const uint32_t lane_hi = FMT == 6 ? codes_s + 16 * 128 + g * 64 + 4 * (t & 1)
-                                      : codes_s + 16 * 128 + g * 32;
-    const uint32_t mh1 = FMT == 6 ? 1u << (8 - 2 * (t >> 1)) : 1u << (8 - t);
-    const uint32_t mh2 = FMT == 6 ? 1u << (4 - 2 * (t >> 1)) : 1u << (4 - t);
+    constexpr bool kLow2 = FMT == 2 || FMT == 3;     // first plane: 2-bit, 64-byte rows
+    const uint32_t lane_codes = kLow2 ? codes_s + g * 64 + 4 * (t & 1) : codes_s + g * 128 + 4 * t;
+    // Q6 / Q5 / Q3: this lane's top-bit group (after the 16 rows of the first
+    // plane; rows 64 / 32 / 32 bytes apart) and the multipliers that move its
+    // bits into place.
+    const uint32_t lane_hi = FMT == 6   ? codes_s + 16 * 128 + g * 64 + 4 * (t & 1)
+                             : FMT == 3 ? codes_s + 16 * 64 + g * 32
+                                        : codes_s + 16 * 128 + g * 32;
+    const uint32_t mh1 = FMT == 6 || kLow2 ? 1u << (8 - 2 * (t >> 1)) : 1u << (8 - t);
+    const uint32_t mh2 = FMT == 6 || kLow2 ? 1u << (4 - 2 * (t >> 1)) : 1u << (4 - t);
+    const uint32_t mh3 = 1u << (10 - t), mh4 = 1u << (6 - t);    // Q3: bit 2 of a code -> bit 10
     auto one_block = [&](int jb) {
         float off[4];
         block_offset<FMT>(xa[jb], xb[jb], off);
@@ -667,6 +821,9 @@ __device__ __forceinline__ void chunk_mma(uint32_t codes_s, uint32_t scales_s, i
             const float dg8 = (jb & 1) ? e1 : e0;
             if constexpr (FMT == 4) {
                 block_q4(lane_codes + mt * 2048 + sw[jb], xa[jb], xb[jb], off, dg, dg8, acc[mt], m16);
+            } else if constexpr (kLow2) {
+                block_q23<FMT>(lane_codes + sw[jb], lane_hi + 4 * jb, xa[jb], xb[jb], off, dg, dg8,
+                               acc[mt], mh1, mh2, mh3, mh4);
             } else if constexpr (FMT == 6 || FMT == 5) {
                 block_qtop<FMT>(lane_codes + sw[jb], lane_hi + (FMT == 6 ? 8 : 4) * jb, xa[jb],
                                 xb[jb], off, dg, dg8, acc[mt], m16, mh1, mh2);

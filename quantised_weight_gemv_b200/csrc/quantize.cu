@@ -15,6 +15,12 @@
 // rows of 5K/8 bytes -- the low nibbles as Q4, then one top bit per element
 // (block j at byte K/2 + 4j; byte i = 0..3 holds that of element i + 4p in
 // bit p).
+// Q3 (d = a/3, q = round(w/d)+4 clamped to [0, 7], zero-point code 4): rows
+// of 3K/8 bytes -- the low 2 bits of each code (block j at byte 8j; byte i
+// holds those of elements i, i+8, i+16, i+24 in bits 0-1, 2-3, 4-5, 6-7),
+// then bit 2 (block j at byte K/4 + 4j; byte i = 0..3 holds that of element
+// i + 4p in bit p).  Q2 (d = a/1, q = round(w/d)+2 clamped to [0, 3], zero-
+// point code 2): rows of K/4 bytes, the 2-bit plane alone.
 // The pages name the Q4 and Q8 formats (BaseRT abstract: eight formats from
 // Q2 to FP16; technical summary "Belangrijkste Bijdragen": evaluation at Q4
 // and Q8) without spelling out their bits; the definition above is the one
@@ -30,14 +36,33 @@
 namespace bq {
 namespace {
 
-// codes_out: the block's code bytes (Q6: its 16 low-nibble bytes, then its
-// 8 top-bit bytes; the caller places them in their planes).
+// Bytes of a block in a row's first plane (Q2/Q3: the 2-bit plane; Q4-Q6:
+// the low-nibble plane; Q8: the codes) and in its second plane (the top bits
+// of Q3, Q5, Q6; none otherwise).
+template <int FMT>
+__host__ __device__ constexpr int lo_block_bytes()
+{
+    return FMT == 2 || FMT == 3 ? 8 : (FMT == 8 ? 32 : 16);
+}
+template <int FMT>
+__host__ __device__ constexpr int top_block_bytes()
+{
+    return FMT == 6 ? 8 : (FMT == 5 || FMT == 3 ? 4 : 0);
+}
+
+// codes_out: the block's code bytes (first its first-plane bytes, then its
+// top-bit bytes; the caller places them in their planes).
 template <int FMT>
 __host__ __device__ inline void quantize_block(const float *w, uint8_t *codes_out,
                                                uint16_t *scale_out, bool *ok)
 {
-    constexpr float kLevels = FMT == 4 ? 7.0f : (FMT == 5 ? 15.0f : (FMT == 6 ? 31.0f : 127.0f));
-    constexpr int kZero = FMT == 4 ? 8 : (FMT == 5 ? 16 : (FMT == 6 ? 32 : 0));
+    constexpr float kLevels = FMT == 2   ? 1.0f
+                              : FMT == 3 ? 3.0f
+                              : FMT == 4 ? 7.0f
+                              : FMT == 5 ? 15.0f
+                              : FMT == 6 ? 31.0f
+                                         : 127.0f;
+    constexpr int kZero = FMT == 2 ? 2 : FMT == 3 ? 4 : FMT == 4 ? 8 : FMT == 5 ? 16 : FMT == 6 ? 32 : 0;
     float a = 0.0f;
     bool finite = true;
     for (int i = 0; i < 32; i++) {
@@ -84,7 +109,18 @@ __host__ __device__ inline void quantize_block(const float *w, uint8_t *codes_ou
             q[i] = r < -127.0f ? -127 : (r > 127.0f ? 127 : (int)r);
         }
     }
-    if (FMT == 4) {
+    if (FMT == 2 || FMT == 3) {
+        for (int i = 0; i < 8; i++)
+            codes_out[i] = (uint8_t)((q[i] & 3) | ((q[i + 8] & 3) << 2) | ((q[i + 16] & 3) << 4) |
+                                     ((q[i + 24] & 3) << 6));
+        if (FMT == 3)
+            for (int i = 0; i < 4; i++) {
+                int b = 0;
+                for (int p = 0; p < 8; p++)
+                    b |= (q[i + 4 * p] >> 2) << p;
+                codes_out[8 + i] = (uint8_t)b;
+            }
+    } else if (FMT == 4) {
         for (int i = 0; i < 16; i++)
             codes_out[i] = (uint8_t)(q[i] | (q[i + 16] << 4));
     } else if (FMT == 5) {
@@ -108,12 +144,11 @@ __host__ __device__ inline void quantize_block(const float *w, uint8_t *codes_ou
     }
 }
 
-// Where a block's code bytes go: Q6 splits them over its two planes.
+// Code bytes of a row: both planes.
 template <int FMT>
 __host__ __device__ inline size_t row_code_bytes(int K)
 {
-    return FMT == 4 ? (size_t)K / 2
-                    : (FMT == 5 ? 5 * (size_t)K / 8 : (FMT == 6 ? 3 * (size_t)K / 4 : (size_t)K));
+    return (size_t)(K / 32) * (lo_block_bytes<FMT>() + top_block_bytes<FMT>());
 }
 
 template <int FMT>
@@ -125,7 +160,8 @@ int32_t quantize_host(const float *w, int32_t N, int32_t K, uint8_t *codes, uint
         return BQ_ERR_SHAPE;
     const int nb = K / 32, ldS = bq_scales_ld(K);
     const size_t row_bytes = row_code_bytes<FMT>(K);
-    const size_t blk_bytes = FMT == 4 ? 16 : 32;
+    constexpr int kLo = lo_block_bytes<FMT>(), kTop = top_block_bytes<FMT>();
+    const size_t lo_row = (size_t)nb * kLo;            // the top plane starts here
     for (int n = 0; n < N; n++) {
         for (int j = nb; j < ldS; j++)
             scales[(size_t)n * ldS + j] = 0;
@@ -133,15 +169,11 @@ int32_t quantize_host(const float *w, int32_t N, int32_t K, uint8_t *codes, uint
             bool ok = true;
             uint8_t *row = codes + (size_t)n * row_bytes;
             uint8_t buf[32];
-            constexpr bool kPlanes = FMT == 5 || FMT == 6;    // codes split over two planes
-            constexpr int kTop = FMT == 5 ? 4 : 8;            // top-plane bytes per block
-            quantize_block<FMT>(w + (size_t)n * K + (size_t)j * 32,
-                                kPlanes ? buf : row + (size_t)j * blk_bytes,
+            quantize_block<FMT>(w + (size_t)n * K + (size_t)j * 32, buf,
                                 scales + (size_t)n * ldS + j, &ok);
-            if (kPlanes) {
-                memcpy(row + (size_t)j * 16, buf, 16);
-                memcpy(row + (size_t)K / 2 + (size_t)j * kTop, buf + 16, kTop);
-            }
+            memcpy(row + (size_t)j * kLo, buf, kLo);
+            if (kTop > 0)
+                memcpy(row + lo_row + (size_t)j * kTop, buf + kLo, kTop);
             if (!ok)
                 return BQ_ERR_RANGE;
         }
@@ -157,7 +189,7 @@ __global__ void quantize_kernel(const float *__restrict__ w, int N, int K, uint8
     const int nb = K / 32, ldS = (nb + 7) / 8 * 8;
     const long long total = (long long)N * nb;
     const size_t row_bytes = row_code_bytes<FMT>(K);
-    const size_t blk_bytes = FMT == 4 ? 16 : 32;
+    const size_t blk_bytes = lo_block_bytes<FMT>();
     for (long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x; b < total;
          b += (long long)gridDim.x * blockDim.x) {
         const int n = (int)(b / nb), j = (int)(b - (long long)n * nb);
@@ -179,7 +211,13 @@ __global__ void quantize_kernel(const float *__restrict__ w, int N, int K, uint8
             atomicOr(status, kStatusRange);
         uint32_t wv[8];
         memcpy(wv, out, sizeof(wv));
-        if (FMT == 5 || FMT == 6) {
+        if (FMT == 2 || FMT == 3) {
+            // (Q3: K % 128 == 0: rows keep both planes aligned)
+            uint8_t *row = codes + (size_t)n * row_bytes;
+            *reinterpret_cast<uint2 *>(row + (size_t)j * 8) = make_uint2(wv[0], wv[1]);
+            if (FMT == 3)
+                *reinterpret_cast<uint32_t *>(row + (size_t)K / 4 + (size_t)j * 4) = wv[2];
+        } else if (FMT == 5 || FMT == 6) {
             // (Q6: K % 64 == 0, Q5: K % 128 == 0: rows keep both planes aligned)
             uint8_t *row = codes + (size_t)n * row_bytes;
             *reinterpret_cast<uint4 *>(row + (size_t)j * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
@@ -206,7 +244,8 @@ int32_t quantize_dev(const float *w, int32_t N, int32_t K, void *codes, uint16_t
 {
     if (!w || !codes || !scales)
         return BQ_ERR_NULL;
-    if (N < 1 || K < 32 || K % 32 != 0 || (FMT == 6 && K % 64 != 0) || (FMT == 5 && K % 128 != 0))
+    if (N < 1 || K < 32 || K % 32 != 0 || (FMT == 6 && K % 64 != 0) ||
+        ((FMT == 5 || FMT == 3) && K % 128 != 0))
         return BQ_ERR_SHAPE;
     if (!aligned16(w) || !aligned16(codes) || !aligned16(scales))
         return BQ_ERR_ALIGN;
@@ -235,7 +274,16 @@ int32_t dequantize_host(const void *codes, const uint16_t *scales, int32_t N, in
         for (int k = 0; k < K; k++) {
             const float d = __half2float(__ushort_as_half(scales[(size_t)n * ldS + k / 32]));
             int q;
-            if (FMT == 4) {
+            if (FMT == 2 || FMT == 3) {
+                const uint8_t *row = c + (size_t)n * row_code_bytes<FMT>(K);
+                const uint8_t lo = row[(k / 32) * 8 + (k % 8)];
+                q = (lo >> (2 * ((k % 32) / 8))) & 3;
+                if (FMT == 3) {
+                    const uint8_t hi = row[(size_t)K / 4 + (k / 32) * 4 + (k % 4)];
+                    q |= ((hi >> ((k % 32) / 4)) & 1) << 2;
+                }
+                q -= FMT == 3 ? 4 : 2;
+            } else if (FMT == 4) {
                 const uint8_t byte = c[(size_t)n * (K / 2) + (k / 32) * 16 + (k % 16)];
                 q = ((k % 32) < 16 ? (byte & 15) : (byte >> 4)) - 8;
             } else if (FMT == 5) {
@@ -346,6 +394,36 @@ extern "C" int32_t bq_blocks_to_planes_q8(const uint8_t *blocks, int32_t N, int3
                                           int8_t *codes, uint16_t *scales)
 {
     return blocks_to_planes<8>(blocks, N, K, codes, scales);
+}
+extern "C" int32_t bq_quantize_q2(const float *w, int32_t N, int32_t K, uint8_t *codes,
+                                  uint16_t *scales)
+{
+    return quantize_host<2>(w, N, K, codes, scales);
+}
+extern "C" int32_t bq_dequantize_q2(const uint8_t *codes, const uint16_t *scales, int32_t N,
+                                    int32_t K, float *w)
+{
+    return dequantize_host<2>(codes, scales, N, K, w);
+}
+extern "C" int32_t bq_quantize_q2_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
+                                      uint16_t *scales, int32_t *dev_status, void *stream)
+{
+    return quantize_dev<2>(w, N, K, codes, scales, dev_status, stream);
+}
+extern "C" int32_t bq_quantize_q3(const float *w, int32_t N, int32_t K, uint8_t *codes,
+                                  uint16_t *scales)
+{
+    return quantize_host<3>(w, N, K, codes, scales);
+}
+extern "C" int32_t bq_dequantize_q3(const uint8_t *codes, const uint16_t *scales, int32_t N,
+                                    int32_t K, float *w)
+{
+    return dequantize_host<3>(codes, scales, N, K, w);
+}
+extern "C" int32_t bq_quantize_q3_dev(const float *w, int32_t N, int32_t K, uint8_t *codes,
+                                      uint16_t *scales, int32_t *dev_status, void *stream)
+{
+    return quantize_dev<3>(w, N, K, codes, scales, dev_status, stream);
 }
 extern "C" int32_t bq_quantize_q5(const float *w, int32_t N, int32_t K, uint8_t *codes,
                                   uint16_t *scales)

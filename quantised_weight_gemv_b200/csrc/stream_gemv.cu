@@ -121,7 +121,7 @@ struct KernelArgs {
     // routed experts
     int E, topk, x_per_slot;
     const int *idx;
-    // Q5 / Q6 (matrix mode): the top-bit plane of mat0's codes
+    // Q3 / Q5 / Q6 (matrix mode): the top-bit plane of mat0's codes
     alignas(64) CUtensorMap tm_codes_hi;
 };
 
@@ -428,10 +428,11 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 const MatDesc &m = mats[PLAN ? iss.u : 0];
 #pragma unroll
                 for (int bx = 0; bx < F::kBoxes; bx++)
-                    tma_load_2d(cdst + bx * (ROWS * 128), &m.tm_codes, bar,
-                                iss.kp * 128 * F::kBoxes + bx * 128, row, pol);
-                if constexpr (FMT == 5 || FMT == 6)
-                    tma_load_2d(cdst + ROWS * 128, &a.tm_codes_hi, bar, iss.kp * F::kTopRow, row, pol);
+                    tma_load_2d(cdst + bx * (ROWS * F::kLoRow), &m.tm_codes, bar,
+                                iss.kp * F::kLoRow * F::kBoxes + bx * F::kLoRow, row, pol);
+                if constexpr (FMT == 3 || FMT == 5 || FMT == 6)
+                    tma_load_2d(cdst + ROWS * F::kLoRow, &a.tm_codes_hi, bar, iss.kp * F::kTopRow,
+                                row, pol);
                 tma_load_2d(sdst, &m.tm_scales, bar, iss.kp * 8, row, (FMT == 4) ? pol : pol_s);
             }
         }
@@ -950,7 +951,7 @@ constexpr size_t kSyncBytes = 512;
 constexpr CUtensorMapL2promotion kPromoCodes = CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
 constexpr CUtensorMapL2promotion kPromoScales = CU_TENSOR_MAP_L2_PROMOTION_NONE;
 
-int rows_of(int fmt) { return fmt == 4 ? Fmt<4>::kRows : Fmt<8>::kRows; }   // (Q5, Q6: 16 as Q8)
+int rows_of(int fmt) { return fmt == 4 ? Fmt<4>::kRows : Fmt<8>::kRows; }   // (Q2-Q6: 16 as Q8)
 
 // R: rows per chunk (the band height), rows_of(fmt) unless a launch chose
 // another Q4 geometry.
@@ -960,19 +961,25 @@ bool fill_matdesc(int fmt, const bq_qmat *W, const uint16_t *x, int B, float *y,
     if (R == 0)
         R = rows_of(fmt);
     const int N = W->N, K = W->K;
-    // Q5 / Q6: the low-nibble plane, the first K/2 bytes of each 5K/8- or
-    // 3K/4-byte row
-    const uint64_t cdims[2] = {(uint64_t)(fmt == 8 ? K : K / 2), (uint64_t)N};
-    const uint64_t cstr[1] = {(uint64_t)(fmt == 4   ? K / 2
+    // The first plane of each row: Q5 / Q6 the low-nibble plane, the first
+    // K/2 bytes of each 5K/8- or 3K/4-byte row; Q3 the 2-bit plane, the first
+    // K/4 bytes of each 3K/8-byte row (Q2: all of a K/4-byte row), in 64-byte
+    // boxes under the 64-byte swizzle.
+    const bool low2 = fmt == 2 || fmt == 3;
+    const uint64_t cdims[2] = {(uint64_t)(fmt == 8 ? K : low2 ? K / 4 : K / 2), (uint64_t)N};
+    const uint64_t cstr[1] = {(uint64_t)(fmt == 2   ? K / 4
+                                         : fmt == 3 ? 3 * K / 8
+                                         : fmt == 4 ? K / 2
                                          : fmt == 5 ? 5 * K / 8
                                          : fmt == 6 ? 3 * K / 4 : K)};
-    const uint32_t cbox[2] = {128, (uint32_t)R};
+    const uint32_t cbox[2] = {low2 ? 64u : 128u, (uint32_t)R};
     const int ldS = bq_scales_ld(K);
     const uint64_t sdims[2] = {(uint64_t)(K / 32), (uint64_t)N};
     const uint64_t sstr[1] = {(uint64_t)ldS * 2};
     const uint32_t sbox[2] = {8, (uint32_t)R};
     if (!encode_tensor_map(&m->tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, cdims, cstr,
-                           cbox, CU_TENSOR_MAP_SWIZZLE_128B, kPromoCodes) ||
+                           cbox, low2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                           kPromoCodes) ||
         !encode_tensor_map(&m->tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, W->scales, sdims, sstr,
                            sbox, CU_TENSOR_MAP_SWIZZLE_NONE, kPromoScales))
         return false;
@@ -1165,15 +1172,17 @@ int32_t gemv_launch(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int
     memset(&a, 0, sizeof(a));
     if (!fill_matdesc(FMT, W, x, B, static_cast<float *>(y), &a.mat0, Fmt<FMT, MT>::kRows))
         return BQ_ERR_CUDA;
-    if constexpr (FMT == 5 || FMT == 6) {
-        // the top-bit plane: the last K/8 (Q5) or K/4 (Q6) bytes of each row
+    if constexpr (FMT == 3 || FMT == 5 || FMT == 6) {
+        // the top-bit plane: the last K/8 (Q3, Q5) or K/4 (Q6) bytes of each
+        // row, after a first plane of K/4 (Q3) or K/2 bytes
         const int N = W->N, K = W->K;
+        const int first = FMT == 3 ? K / 4 : K / 2;
         const int top = FMT == 6 ? K / 4 : K / 8;
         const uint64_t hdims[2] = {(uint64_t)top, (uint64_t)N};
-        const uint64_t hstr[1] = {(uint64_t)(K / 2 + top)};
+        const uint64_t hstr[1] = {(uint64_t)(first + top)};
         const uint32_t hbox[2] = {(uint32_t)Fmt<FMT>::kTopRow, (uint32_t)Fmt<FMT>::kRows};
         if (!encode_tensor_map(&a.tm_codes_hi, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
-                               static_cast<const uint8_t *>(W->codes) + K / 2, hdims, hstr, hbox,
+                               static_cast<const uint8_t *>(W->codes) + first, hdims, hstr, hbox,
                                CU_TENSOR_MAP_SWIZZLE_NONE, kPromoCodes))
             return BQ_ERR_CUDA;
     }
@@ -1211,7 +1220,7 @@ int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32
     const int32_t rows = flags & (BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32);
     if (!epilogue_ok(epi, W->N) || (flags & ~kKnown) != 0 ||
         rows == (BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32) || (FMT != 4 && rows == BQ_GEMV_ROWS32) ||
-        (FMT == 6 && W->K % 64 != 0) || (FMT == 5 && W->K % 128 != 0))
+        ((FMT == 6 || FMT == 2) && W->K % 64 != 0) || ((FMT == 5 || FMT == 3) && W->K % 128 != 0))
         return BQ_ERR_SHAPE;
     if (!x || !y || !ws)
         return BQ_ERR_NULL;
@@ -1296,8 +1305,9 @@ extern "C" int32_t bq_gemv_geometry_of(int32_t fmt, int32_t N, int32_t K, int32_
         return BQ_ERR_NULL;
     const int32_t rows = flags & (BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32);
     constexpr int32_t kKnown = BQ_GEMV_STATIC_WEIGHTS | BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32;
-    if ((fmt != 4 && fmt != 5 && fmt != 6 && fmt != 8) || N < 1 || K < 32 || K % 32 != 0 ||
-        (fmt == 6 && K % 64 != 0) || (fmt == 5 && K % 128 != 0) || (flags & ~kKnown) != 0 ||
+    if (fmt < 2 || fmt > 8 || fmt == 7 || N < 1 || K < 32 || K % 32 != 0 ||
+        ((fmt == 6 || fmt == 2) && K % 64 != 0) || ((fmt == 5 || fmt == 3) && K % 128 != 0) ||
+        (flags & ~kKnown) != 0 ||
         rows == (BQ_GEMV_ROWS16 | BQ_GEMV_ROWS32) || (fmt != 4 && rows == BQ_GEMV_ROWS32) ||
         sm_count < 0)
         return BQ_ERR_SHAPE;
@@ -1319,6 +1329,10 @@ extern "C" int32_t bq_gemv_geometry_of(int32_t fmt, int32_t N, int32_t K, int32_
                                          [](int, int c) { return resident_clusters<6, 1>(c); })
             : fmt == 5 ? matrix_geometry(5, N, K, B, rows, cap,
                                          [](int, int c) { return resident_clusters<5, 1>(c); })
+            : fmt == 3 ? matrix_geometry(3, N, K, B, rows, cap,
+                                         [](int, int c) { return resident_clusters<3, 1>(c); })
+            : fmt == 2 ? matrix_geometry(2, N, K, B, rows, cap,
+                                         [](int, int c) { return resident_clusters<2, 1>(c); })
                        : matrix_geometry(8, N, K, B, rows, cap,
                                          [](int, int c) { return resident_clusters<8, 1>(c); });
     }
@@ -1355,6 +1369,10 @@ extern "C" int32_t bq_gemv_ex(int32_t fmt, const bq_qmat *W, const uint16_t *x, 
         return gemv_impl<6>(W, x, B, y, epilogue, flags, ws, ws_bytes, dev_status, stream);
     if (fmt == 5)
         return gemv_impl<5>(W, x, B, y, epilogue, flags, ws, ws_bytes, dev_status, stream);
+    if (fmt == 3)
+        return gemv_impl<3>(W, x, B, y, epilogue, flags, ws, ws_bytes, dev_status, stream);
+    if (fmt == 2)
+        return gemv_impl<2>(W, x, B, y, epilogue, flags, ws, ws_bytes, dev_status, stream);
     if (fmt == 8)
         return gemv_impl<8>(W, x, B, y, epilogue, flags, ws, ws_bytes, dev_status, stream);
     return BQ_ERR_SHAPE;

@@ -99,7 +99,7 @@ class Mat:
 class DenseWorkload:
     wid: int            # workload id, part of every seed key
     name: str
-    fmt: int            # 4 or 8
+    fmt: int            # 2, 3, 4, 5, 6 or 8
     layers: int
     mats: Tuple[Mat, ...]   # per-layer matrices, in model order
     B: int = 1
@@ -117,7 +117,8 @@ class DenseWorkload:
 
 def packed_bytes(fmt: int, N: int, K: int) -> int:
     """Algorithmic bytes of one packed matrix: codes + scales (no padding)."""
-    codes = {4: N * K // 2, 5: 5 * N * K // 8, 6: 3 * N * K // 4, 8: N * K}[fmt]
+    codes = {2: N * K // 4, 3: 3 * N * K // 8, 4: N * K // 2, 5: 5 * N * K // 8,
+             6: 3 * N * K // 4, 8: N * K}[fmt]
     return codes + N * (K // 32) * 2
 
 
@@ -135,7 +136,7 @@ DENSE_H2048 = DenseWorkload(2, "dense16L-h2048-ffn8192-q4", 4, 16, (
 
 
 def dense_h2048(fmt: int) -> DenseWorkload:
-    """The 16-layer hidden-2048 decoder in another format (Q5, Q6 or Q8)."""
+    """The 16-layer hidden-2048 decoder in another format (Q2, Q3, Q5, Q6 or Q8)."""
     return DenseWorkload(8, f"dense16L-h2048-ffn8192-q{fmt}", fmt, 16, DENSE_H2048.mats)
 
 

@@ -34,8 +34,8 @@ def gpu_gemv(fmt, codes, scales, x_bits, ws=None, status=None, flags=0):
     fp16 bits; returns fp32 [B, N]."""
     import torch
     N = codes.shape[0]
-    K = {4: codes.shape[1] * 2, 5: codes.shape[1] * 8 // 5, 6: codes.shape[1] * 4 // 3,
-         8: codes.shape[1]}[fmt]
+    K = {2: codes.shape[1] * 4, 3: codes.shape[1] * 8 // 3, 4: codes.shape[1] * 2,
+         5: codes.shape[1] * 8 // 5, 6: codes.shape[1] * 4 // 3, 8: codes.shape[1]}[fmt]
     x_bits = np.atleast_2d(x_bits)
     B = x_bits.shape[0]
     c, s, x = dev(codes.view(np.uint8)), dev(scales), dev(x_bits)
@@ -61,13 +61,14 @@ def check_tol(y, y_ref, absy):
 
 
 def oracle_gemv(fmt, codes, scales, x_bits, nthreads=8):
-    fn = {4: oracle.gemv_q4, 5: oracle.gemv_q5, 6: oracle.gemv_q6, 8: oracle.gemv_q8}[fmt]
+    fn = {2: oracle.gemv_q2, 3: oracle.gemv_q3, 4: oracle.gemv_q4, 5: oracle.gemv_q5,
+          6: oracle.gemv_q6, 8: oracle.gemv_q8}[fmt]
     return fn(codes, scales, x_bits, nthreads=nthreads)
 
 
 def quantize(fmt, w):
-    return {4: oracle.quantize_q4, 5: oracle.quantize_q5, 6: oracle.quantize_q6,
-            8: oracle.quantize_q8}[fmt](w)
+    return {2: oracle.quantize_q2, 3: oracle.quantize_q3, 4: oracle.quantize_q4,
+            5: oracle.quantize_q5, 6: oracle.quantize_q6, 8: oracle.quantize_q8}[fmt](w)
 
 
 def pair_order(gate, up):

@@ -39,17 +39,18 @@ def test_status_strings_and_scales_ld():
     assert bq.scales_ld(33) == 0 and bq.scales_ld(0) == 0
 
 
-_ORQ = {4: lambda w: oracle.quantize_q4(w), 5: lambda w: oracle.quantize_q5(w),
+_ORQ = {2: lambda w: oracle.quantize_q2(w), 3: lambda w: oracle.quantize_q3(w),
+        4: lambda w: oracle.quantize_q4(w), 5: lambda w: oracle.quantize_q5(w),
         6: lambda w: oracle.quantize_q6(w), 8: lambda w: oracle.quantize_q8(w)}
 
 
 def _host_quantize(fmt, w):
     N, K = w.shape
-    width = {4: K // 2, 5: 5 * K // 8, 6: 3 * K // 4, 8: K}[fmt]
+    width = {2: K // 4, 3: 3 * K // 8, 4: K // 2, 5: 5 * K // 8, 6: 3 * K // 4, 8: K}[fmt]
     codes = np.zeros((N, width), dtype=np.int8 if fmt == 8 else np.uint8)
     scales = np.zeros((N, bq.scales_ld(K)), dtype=np.uint16)
-    fn = {4: bq.lib().bq_quantize_q4, 5: bq.lib().bq_quantize_q5, 6: bq.lib().bq_quantize_q6,
-          8: bq.lib().bq_quantize_q8}[fmt]
+    fn = {2: bq.lib().bq_quantize_q2, 3: bq.lib().bq_quantize_q3, 4: bq.lib().bq_quantize_q4,
+          5: bq.lib().bq_quantize_q5, 6: bq.lib().bq_quantize_q6, 8: bq.lib().bq_quantize_q8}[fmt]
     rc = fn(w.ctypes.data, N, K, codes.ctypes.data, scales.ctypes.data)
     return rc, codes, scales
 
@@ -67,7 +68,7 @@ def _edge_weights():
     return w
 
 
-@pytest.mark.parametrize("fmt", [4, 5, 6, 8])
+@pytest.mark.parametrize("fmt", [2, 3, 4, 5, 6, 8])
 def test_host_quantiser_bit_exact_vs_oracle(fmt):
     w = _edge_weights()
     rc, codes, scales = _host_quantize(fmt, w)
@@ -77,7 +78,7 @@ def test_host_quantiser_bit_exact_vs_oracle(fmt):
     assert np.array_equal(scales, os_)
 
 
-@pytest.mark.parametrize("fmt", [4, 5, 6, 8])
+@pytest.mark.parametrize("fmt", [2, 3, 4, 5, 6, 8])
 def test_host_quantiser_rejects_out_of_range(fmt):
     w = np.zeros((1, 32), dtype=np.float32)
     w[0, 3] = np.nan
@@ -86,16 +87,16 @@ def test_host_quantiser_rejects_out_of_range(fmt):
     assert _host_quantize(fmt, w)[0] == bq.BQ_ERR_RANGE
 
 
-@pytest.mark.parametrize("fmt", [4, 5, 6, 8])
+@pytest.mark.parametrize("fmt", [2, 3, 4, 5, 6, 8])
 def test_host_dequantize_matches_oracle(fmt):
     w = synth.weights_f32(synth.key(1, 93, 0, 0, 0), 9, 128)
     codes, scales = _ORQ[fmt](w)
     out = np.zeros(w.shape, dtype=np.float32)
-    fn = {4: bq.lib().bq_dequantize_q4, 5: bq.lib().bq_dequantize_q5, 6: bq.lib().bq_dequantize_q6,
-          8: bq.lib().bq_dequantize_q8}[fmt]
+    fn = {2: bq.lib().bq_dequantize_q2, 3: bq.lib().bq_dequantize_q3, 4: bq.lib().bq_dequantize_q4,
+          5: bq.lib().bq_dequantize_q5, 6: bq.lib().bq_dequantize_q6, 8: bq.lib().bq_dequantize_q8}[fmt]
     assert fn(codes.ctypes.data, scales.ctypes.data, 9, 128, out.ctypes.data) == 0
-    ref = {4: oracle.dequantize_q4, 5: oracle.dequantize_q5, 6: oracle.dequantize_q6,
-           8: oracle.dequantize_q8}[fmt](codes, scales)
+    ref = {2: oracle.dequantize_q2, 3: oracle.dequantize_q3, 4: oracle.dequantize_q4,
+           5: oracle.dequantize_q5, 6: oracle.dequantize_q6, 8: oracle.dequantize_q8}[fmt](codes, scales)
     assert np.array_equal(out.astype(np.float64), ref)
 
 
@@ -164,7 +165,8 @@ def test_gemv_ex_epilogue_validation_before_launch():
         return f(fmt, ctypes.byref(W), FAKE, 1, FAKE, epi, flags, FAKE, 1 << 30, None, None)
 
     assert rc(fmt=7) == bq.BQ_ERR_SHAPE
-    assert rc(fmt=3) == bq.BQ_ERR_SHAPE
+    assert rc(fmt=1) == bq.BQ_ERR_SHAPE
+    assert rc(fmt=9) == bq.BQ_ERR_SHAPE
     assert rc(flags=8) == bq.BQ_ERR_SHAPE           # unknown flag bit
     assert rc(flags=bq.BQ_GEMV_ROWS16 | bq.BQ_GEMV_ROWS32) == bq.BQ_ERR_SHAPE
     assert rc(fmt=8, flags=bq.BQ_GEMV_ROWS32) == bq.BQ_ERR_SHAPE   # Q8 chunks are 16 rows
@@ -176,6 +178,14 @@ def test_gemv_ex_epilogue_validation_before_launch():
     assert f(5, ctypes.byref(W5), FAKE, 1, FAKE, bq.BQ_EPI_NONE, 0, FAKE, 1 << 30, None,
              None) == bq.BQ_ERR_SHAPE
     assert rc(fmt=5, flags=bq.BQ_GEMV_ROWS32) == bq.BQ_ERR_SHAPE
+    W2 = bq.bq_qmat(FAKE, FAKE, 64, 96)                            # Q2 needs K % 64 == 0
+    assert f(2, ctypes.byref(W2), FAKE, 1, FAKE, bq.BQ_EPI_NONE, 0, FAKE, 1 << 30, None,
+             None) == bq.BQ_ERR_SHAPE
+    W3 = bq.bq_qmat(FAKE, FAKE, 64, 192)                           # Q3 needs K % 128 == 0
+    assert f(3, ctypes.byref(W3), FAKE, 1, FAKE, bq.BQ_EPI_NONE, 0, FAKE, 1 << 30, None,
+             None) == bq.BQ_ERR_SHAPE
+    assert rc(fmt=3, flags=bq.BQ_GEMV_ROWS32) == bq.BQ_ERR_SHAPE
+    assert rc(fmt=2, flags=bq.BQ_GEMV_ROWS32) == bq.BQ_ERR_SHAPE
     assert rc(flags=bq.BQ_GEMV_STATIC_WEIGHTS, N=40) == bq.BQ_ERR_SHAPE
     assert rc(epi=2) == bq.BQ_ERR_SHAPE
     assert rc(epi=-1) == bq.BQ_ERR_SHAPE
@@ -207,6 +217,8 @@ def test_moe_argument_validation_before_launch():
 
 
 def test_device_quantiser_argument_validation():
+    assert bq.lib().bq_quantize_q3_dev(FAKE, 4, 192, FAKE, FAKE, None, None) == bq.BQ_ERR_SHAPE
+    assert bq.lib().bq_quantize_q2_dev(FAKE, 4, 60, FAKE, FAKE, None, None) == bq.BQ_ERR_SHAPE
     f = bq.lib().bq_quantize_q4_dev
     assert f(None, 4, 64, FAKE, FAKE, None, None) == bq.BQ_ERR_NULL
     assert f(FAKE, 4, 60, FAKE, FAKE, None, None) == bq.BQ_ERR_SHAPE

@@ -38,12 +38,12 @@ SHAPES = [(1, 32), (16, 256), (40, 2048), (777, 3072), (2048, 2048), (3072, 2048
 @pytest.mark.parametrize("sm_count", [148, 132, 100])
 @pytest.mark.parametrize("fmt,flags", [(4, 0), (4, bq.BQ_GEMV_ROWS16), (4, bq.BQ_GEMV_ROWS32),
                                        (8, 0), (4, bq.BQ_GEMV_STATIC_WEIGHTS), (6, 0),
-                                       (5, 0)])
+                                       (5, 0), (3, 0), (2, 0)])
 @pytest.mark.parametrize("B", [1, 8])
 def test_geometry_matches_brute_force(sm_count, fmt, flags, B):
     cap = min(2 * sm_count, 512)
     for N, K in SHAPES:
-        if (fmt == 6 and K % 64) or (fmt == 5 and K % 128):
+        if (fmt in (2, 6) and K % 64) or (fmt in (3, 5) and K % 128):
             continue
         g = bq.gemv_geometry(fmt, N, K, B, flags, sm_count=sm_count)
         rows = g["rows"]
@@ -93,6 +93,11 @@ def test_geometry_validation():
     assert call(7, 64, 256, 1, 0, 148) == bq.BQ_ERR_SHAPE
     assert call(5, 64, 192, 1, 0, 148) == bq.BQ_ERR_SHAPE          # Q5: K % 128
     assert call(6, 64, 96, 1, 0, 148) == bq.BQ_ERR_SHAPE           # Q6: K % 64
+    assert call(3, 64, 192, 1, 0, 148) == bq.BQ_ERR_SHAPE          # Q3: K % 128
+    assert call(2, 64, 96, 1, 0, 148) == bq.BQ_ERR_SHAPE           # Q2: K % 64
+    assert call(1, 64, 256, 1, 0, 148) == bq.BQ_ERR_SHAPE
+    assert call(3, 64, 256, 1, 0, 148) == bq.BQ_OK and out.rows == 16
+    assert call(2, 64, 256, 1, bq.BQ_GEMV_ROWS32, 148) == bq.BQ_ERR_SHAPE
     assert call(4, 64, 48, 1, 0, 148) == bq.BQ_ERR_SHAPE
     assert call(4, 0, 256, 1, 0, 148) == bq.BQ_ERR_SHAPE
     assert call(4, 64, 256, 0, 0, 148) == bq.BQ_ERR_BATCH

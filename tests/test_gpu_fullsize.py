@@ -39,12 +39,13 @@ def _regen_rows(wl, seed, layer, m, rows, K, N_mat):
 
 
 def _quant(fmt, w):
-    return {4: oracle.quantize_q4, 5: oracle.quantize_q5, 6: oracle.quantize_q6,
-            8: oracle.quantize_q8}[fmt](w)
+    return {2: oracle.quantize_q2, 3: oracle.quantize_q3, 4: oracle.quantize_q4,
+            5: oracle.quantize_q5, 6: oracle.quantize_q6, 8: oracle.quantize_q8}[fmt](w)
 
 
 def _gemv(fmt, codes, scales, xb):
-    fn = {4: oracle.gemv_q4, 5: oracle.gemv_q5, 6: oracle.gemv_q6, 8: oracle.gemv_q8}[fmt]
+    fn = {2: oracle.gemv_q2, 3: oracle.gemv_q3, 4: oracle.gemv_q4, 5: oracle.gemv_q5,
+          6: oracle.gemv_q6, 8: oracle.gemv_q8}[fmt]
     return fn(codes, scales, xb, nthreads=8)
 
 
@@ -141,9 +142,9 @@ def test_dense16_h2048_step(engine):
     _check_step(synth.DENSE_H2048, every=16, engine=engine)
 
 
-@pytest.mark.parametrize("fmt", [6, 5])
-def test_dense16_h2048_q5_q6_chain(fmt):
-    """The 16-layer hidden-2048 decoder in Q6 and in Q5, as the launch chain."""
+@pytest.mark.parametrize("fmt", [6, 5, 3, 2])
+def test_dense16_h2048_other_formats_chain(fmt):
+    """The 16-layer hidden-2048 decoder in Q6, Q5, Q3 and Q2, as the launch chain."""
     _check_step(synth.dense_h2048(fmt), every=16, engine="graph")
 
 
