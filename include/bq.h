@@ -197,7 +197,7 @@ enum { BQ_EPI_NONE = 0, BQ_EPI_SWIGLU = 1 };
  * fewer instructions per weight (two 16-row tiles share each x fragment),
  * 16-row chunks give twice the work units, which pays when a launch is too
  * small to give every warp a 32-row chunk.  The result is the same up to
- * fp32 summation order.  Q8 chunks are always 16 rows: ROWS16 is accepted,
+ * fp32 summation order.  Chunks of the other formats are always 16 rows: ROWS16 is accepted,
  * ROWS32 returns BQ_ERR_SHAPE, and so does setting both. */
 enum { BQ_GEMV_STATIC_WEIGHTS = 1, BQ_GEMV_ROWS16 = 2, BQ_GEMV_ROWS32 = 4 };
 

@@ -1,18 +1,21 @@
 // bq_device.cuh -- device building blocks of the streamed block-quantised GEMV
 // for sm_100a: PTX wrappers (mbarrier, TMA tensor loads, mma.sync,
-// programmatic dependent launch), in-register Q4/Q8 dequantisation and the
-// per-chunk dot product.
+// programmatic dependent launch), in-register dequantisation of every format
+// and the per-chunk dot product.
 //
-// Work unit ("chunk"): kRows weight rows (32 for Q4, 16 for Q8) x 256 weights
-// along K (8 blocks of 32).  A chunk's codes arrive in shared memory through
-// one (Q4: 32 rows x 128 bytes) or two (Q8: 16 rows x 128 bytes each) 2-D TMA
-// boxes with the 128-byte swizzle, its scales through one kRows x 8 fp16 box.  A warp reads them with 32-bit shared loads that
-// the swizzle makes bank-conflict free, turns each 4-byte group into fp16
-// pairs in registers (exact: see "dequant" below), and forms the block's
-// partial dot products with m16n8k16 mma.sync (fp16 in, fp32 accumulate): M = 16 weight rows (a Q4 chunk is two such m-tiles that
-// share every x fragment), N = the batch (B <= 8), K = 16 elements of one
-// block.  Each block's partial sum is scaled by its fp32-converted scale once
-// (y += d * sum((q - z) x)), so the only roundings are fp32 ones.
+// Work unit ("chunk"): kRows weight rows (32 or 16 for Q4, 16 for the other
+// formats) x 256 weights along K (8 blocks of 32).  A Q4 / Q8 chunk's codes
+// arrive in shared memory through one (Q4: kRows x 128 bytes) or two (Q8: 16
+// rows x 128 bytes each) 2-D TMA boxes with the 128-byte swizzle (the other
+// formats: see their traits below), its scales through one kRows x 8 fp16
+// box.  A warp reads them with 32-bit shared loads that the swizzle makes
+// bank-conflict free, turns each 4-byte group into fp16 pairs in registers
+// (exact: see "dequant" below), and forms the block's partial dot products
+// with m16n8k16 mma.sync (fp16 in, fp32 accumulate): M = 16 weight rows (a
+// 32-row Q4 chunk is two such m-tiles that share every x fragment), N = the
+// batch (B <= 8), K = 16 elements of one block.  Each block's partial sum is
+// scaled by its fp32-converted scale once (y += d * sum((q - z) x)), so the
+// only roundings are fp32 ones.
 #pragma once
 
 #include <cuda.h>
@@ -57,7 +60,7 @@ constexpr long long kWaitCycles = 4000000000LL;
 // Chunk geometry of a format: MT m-tiles of 16 rows.  Q4 comes in two: 32-row
 // chunks (MT = 2, two m-tiles share every x fragment: fewer instructions per
 // weight) and 16-row chunks (MT = 1: twice the work units, for launches too
-// small to give every warp a 32-row chunk).  Q8 chunks are 16 rows.
+// small to give every warp a 32-row chunk).  Q8, Q2, Q3, Q5 and Q6 chunks are 16 rows.
 template <int FMT>
 __host__ __device__ constexpr int default_mt()
 {

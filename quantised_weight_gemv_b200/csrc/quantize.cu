@@ -1,5 +1,5 @@
 // quantize.cu -- block quantisers (host and device) and plane <-> block
-// conversions for the Q4 / Q8 formats.
+// conversions for the Q2-Q6 and Q8 formats (plane <-> block for Q4 / Q8).
 //
 // Per 32-weight block along K: a = max|w| (fp32); d = fp16 round-to-nearest-
 // even of a/127 (Q8) or a/7 (Q4), computed as an IEEE fp32 division; codes

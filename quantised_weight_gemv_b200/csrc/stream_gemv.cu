@@ -1,5 +1,6 @@
 // stream_gemv.cu -- the streamed decode GEMV over block-quantised weights
-// (dense Q4/Q8, whole decode steps, grouped routed-expert Q4), sm_100a.
+// (dense Q2-Q6 and Q8, whole decode steps in Q4/Q8, grouped routed-expert
+// Q4), sm_100a.
 //
 // The decode step is a GEMV per quantisation format with the dequantisation
 // inside the inner loop (BaseRT, gist.science technical summary,
@@ -9,7 +10,7 @@
 // keep HBM busy with the packed weight bytes and read each of them once.
 //
 // Work decomposition (stream-K over chunks).  A matrix is cut into bands of
-// kRows rows (16 for Q8; 32 or 16 for Q4, chosen per launch by
+// kRows rows (16 for Q8, Q2, Q3, Q5, Q6; 32 or 16 for Q4, chosen per launch by
 // choose_q4_mt) and a band into chunks of 256 weights along K; chunks are
 // numbered band-major.  Every warp of the grid is an
 // independent worker that owns a ring of shared-memory slots with its own
@@ -54,6 +55,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -915,11 +917,13 @@ constexpr size_t launch_smem(int n_stages, int n_mats, bool cl = false)
 template <int FMT, int MODE, int MT = default_mt<FMT>(), bool CL = false>
 int32_t prepare_kernel()
 {
-    static bool done[64] = {};
+    // Per device: the attribute is set once.  Atomic, since host threads may
+    // launch concurrently (two of them setting it twice is harmless).
+    static std::atomic<bool> done[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
         return BQ_ERR_CUDA;
-    if (dev >= 0 && dev < 64 && done[dev])
+    if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire))
         return BQ_OK;
     if (cudaFuncSetAttribute((const void *)stream_gemv_kernel<FMT, MODE, MT, CL>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -928,7 +932,7 @@ int32_t prepare_kernel()
         cudaSuccess)
         return BQ_ERR_CUDA;
     if (dev >= 0 && dev < 64)
-        done[dev] = true;
+        done[dev].store(true, std::memory_order_release);
     return BQ_OK;
 }
 
@@ -1115,17 +1119,18 @@ Geometry matrix_geometry(int fmt, long long N, long long K, int B, int32_t rows_
 }
 
 // Clusters of C CTAs of the cluster-sum kernel the device holds at once
-// (cached per device and C; 0 if the query fails).
+// (cached per device and C as n + 1, 0 meaning not yet queried; atomic, since
+// host threads may launch concurrently; 0 if the query fails).
 template <int FMT, int MT>
 int resident_clusters(int C)
 {
-    static int cache[64][kMaxCluster + 1];
-    static bool known[64][kMaxCluster + 1];
+    static std::atomic<int> cache[64][kMaxCluster + 1];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || C < 1 || C > kMaxCluster)
         return 0;
-    if (known[dev][C])
-        return cache[dev][C];
+    const int known = cache[dev][C].load(std::memory_order_acquire);
+    if (known > 0)
+        return known - 1;
     int n = 0;
     if (prepare_kernel<FMT, kModeMatrix, MT, true>() == BQ_OK) {
         cudaLaunchConfig_t cfg = {};
@@ -1145,8 +1150,7 @@ int resident_clusters(int C)
             n = 0;
         }
     }
-    cache[dev][C] = n;
-    known[dev][C] = true;
+    cache[dev][C].store(n + 1, std::memory_order_release);
     return n;
 }
 
