@@ -1,0 +1,46 @@
+"""The benchmark's reference arm (the fp64 oracle timed on the host cores)
+runs without a GPU.  This checks that its JSON line keeps the contract the
+driver reads: the same metric, unit and direction as the GPU arm, a bounded
+sample stated in `cpu_baseline`, and an `e2e` object with no host<->device
+bytes (the oracle never touches a device)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _reference_line(*extra):
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                        "--warmup", "0", *extra], cwd=ROOT, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+def test_reference_arm_json_contract():
+    import bench
+    d = _reference_line()
+    assert d["impl"] == "reference"
+    assert d["metric"] == bench.METRIC and d["unit"] == "GB/s"
+    assert d["higher_is_better"] is True and d["n_gpus"] == 1 and d["steps"] == 1
+    assert d["warmup"] >= 3                          # warm-up is never below three steps
+    assert d["value"] > 0 and d["ms_per_step"] > 0
+    assert d["config"]["workload"] == "dense16L-h2048-ffn8192-q4"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
+    assert "layer 0" in cb["sample"]
+    e = d["e2e"]
+    assert e["value"] == d["value"] and e["unit"] == d["unit"]
+    assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+@pytest.mark.parametrize("workload", ["dense16L-h2048-ffn8192-q3", "dense16L-h2048-ffn8192-q2"])
+def test_reference_arm_other_formats(workload):
+    d = _reference_line("--workload", workload)
+    assert d["config"]["workload"] == workload and d["value"] > 0
