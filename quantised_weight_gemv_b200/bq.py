@@ -144,6 +144,40 @@ def _stream_ptr(stream) -> int:
     return s.cuda_stream
 
 
+_ROW_BYTES = {2: lambda K: K // 4, 3: lambda K: 3 * K // 8, 4: lambda K: K // 2,
+              5: lambda K: 5 * K // 8, 6: lambda K: 3 * K // 4, 8: lambda K: K}
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def _on_device(fn: str, **tensors) -> None:
+    """The C library takes raw device pointers and cannot tell a host
+    pointer from a device one: refuse host tensors before any launch."""
+    for name, t in tensors.items():
+        if t is not None and not t.is_cuda:
+            raise ValueError(f"{fn}: {name} must be a CUDA tensor (got device {t.device})")
+
+
+def _check_planes(fn: str, fmt: int, W: bq_qmat) -> None:
+    """Device planes behind a bq_qmat made by qmat(): on the GPU and large
+    enough for N rows of the format (the kernel reads them through TMA maps
+    built from N and K alone)."""
+    refs = getattr(W, "_refs", None)
+    if refs is None:
+        return
+    codes, scales = refs
+    _on_device(fn, codes=codes, scales=scales)
+    if fmt in _ROW_BYTES and W.K % 32 == 0:
+        if _nbytes(codes) < W.N * _ROW_BYTES[fmt](W.K):
+            raise ValueError(f"{fn}: codes hold {_nbytes(codes)} bytes, "
+                             f"{W.N} rows of Q{fmt} need {W.N * _ROW_BYTES[fmt](W.K)}")
+        if _nbytes(scales) < W.N * scales_ld(W.K) * 2:
+            raise ValueError(f"{fn}: scales hold {_nbytes(scales)} bytes, "
+                             f"need {W.N * scales_ld(W.K) * 2}")
+
+
 def qmat(codes, scales, N: int, K: int) -> bq_qmat:
     """bq_qmat over two tensors (device planes for GEMV, host for pack calls).
 
@@ -178,7 +212,15 @@ def gemv(fmt: int, W: bq_qmat, x, y, ws, status=None, stream=None, epilogue: int
     """y[B, N] (fp32) = deq(W) . x[B, K] (fp16), through bq_gemv_q4 / bq_gemv_q8;
     Q6, an epilogue (BQ_EPI_SWIGLU: y is fp16 [B, N/2]) or flags go through
     bq_gemv_ex."""
+    _on_device("gemv", x=x, y=y, ws=ws, status=status)
+    _check_planes("gemv", fmt, W)
+    if x.dim() != 2 or x.shape[1] != W.K or x.element_size() != 2 or not x.is_contiguous():
+        raise ValueError(f"gemv: x must be a contiguous [B, {W.K}] tensor of fp16 bits, got "
+                         f"{tuple(x.shape)} {x.dtype}")
     B = x.shape[0]
+    need = B * W.N * (4 if epilogue == BQ_EPI_NONE else 1)      # fp32 [B][N] or fp16 [B][N/2]
+    if not y.is_contiguous() or _nbytes(y) < need:
+        raise ValueError(f"gemv: y must be contiguous with at least {need} bytes")
     if epilogue == BQ_EPI_NONE and flags == 0 and fmt in (4, 8):   # (Q2, Q3, Q5, Q6: bq_gemv_ex)
         fn = lib().bq_gemv_q4 if fmt == 4 else lib().bq_gemv_q8
         rc = fn(ctypes.byref(W), x.data_ptr(), B, y.data_ptr(), ws.data_ptr(),
@@ -196,6 +238,11 @@ def moe_gemv_q4(Wstack: bq_qmat, E: int, codes_stride: int, scales_stride: int, 
                 epilogue: int = BQ_EPI_NONE) -> None:
     """Routed-expert Q4 GEMV (bq_moe_gemv_q4); with epilogue BQ_EPI_SWIGLU,
     per-slot fp16 h (bq_moe_gemv_ex)."""
+    _on_device("moe_gemv_q4", x=x, expert_idx=expert_idx, route_w=route_w, y=y, ws=ws,
+               status=status)
+    refs = getattr(Wstack, "_refs", None)
+    if refs is not None:
+        _on_device("moe_gemv_q4", codes=refs[0], scales=refs[1])
     B, topk = expert_idx.shape
     rc = lib().bq_moe_gemv_ex(ctypes.byref(Wstack), int(E), int(codes_stride), int(scales_stride),
                               x.data_ptr(), 1 if x_per_slot else 0, expert_idx.data_ptr(),
@@ -218,6 +265,8 @@ class StepPlan:
         for i, e in enumerate(entries):
             W, x, y, stage = e[:4]
             epi = e[4] if len(e) > 4 else BQ_EPI_NONE
+            _on_device("StepPlan", x=x, y=y)
+            _check_planes("StepPlan", fmt, W)
             arr[i] = bq_step_mat(W, x.data_ptr(), y.data_ptr(), int(x.shape[0]), int(stage),
                                  int(epi), 0)
             self._refs += [W, x, y]
@@ -237,7 +286,14 @@ class StepPlan:
 
 
 def quantize_dev(fmt: int, w, codes, scales, status=None, stream=None) -> None:
+    _on_device("quantize_dev", w=w, codes=codes, scales=scales, status=status)
     N, K = w.shape
+    if (w.element_size() != 4 or not w.is_contiguous() or not codes.is_contiguous()
+            or not scales.is_contiguous()):
+        raise ValueError("quantize_dev: w must be contiguous fp32 [N, K]; codes and scales contiguous")
+    if fmt in _ROW_BYTES and K % 32 == 0 and (_nbytes(codes) < N * _ROW_BYTES[fmt](K)
+                                              or _nbytes(scales) < N * scales_ld(K) * 2):
+        raise ValueError(f"quantize_dev: planes too small for {N} rows of Q{fmt} with K = {K}")
     fn = {2: lib().bq_quantize_q2_dev, 3: lib().bq_quantize_q3_dev, 4: lib().bq_quantize_q4_dev,
           5: lib().bq_quantize_q5_dev, 6: lib().bq_quantize_q6_dev, 8: lib().bq_quantize_q8_dev}[fmt]
     check(f"bq_quantize_q{fmt}_dev",
