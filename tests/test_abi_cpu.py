@@ -238,6 +238,20 @@ def test_product_path_has_no_oracle_or_fallback():
                 assert "oracle.c" not in src and "liboracle" not in src, fn
 
 
+def test_oracle_shares_nothing_with_the_library():
+    """The oracle is plain C over the C standard library: it includes no header
+    of the package or the CUDA toolkit, and its Python wrapper imports nothing
+    from the package."""
+    import re
+    with open(os.path.join(ROOT, "oracle", "oracle.c")) as f:
+        src = f.read()
+    includes = re.findall(r'#include\s*[<"]([^>"]+)[>"]', src)
+    assert set(includes) <= {"math.h", "pthread.h", "stdint.h", "stdlib.h", "string.h"}, includes
+    with open(os.path.join(ROOT, "oracle", "__init__.py")) as f:
+        py = f.read()
+    assert "quantised_weight_gemv_b200" not in py and "libbq" not in py
+
+
 def test_step_argument_validation_before_launch():
     L = bq.lib()
     assert L.bq_step_plan_bytes(0) == 0 and L.bq_step_plan_bytes(3) > 3 * 320
