@@ -22,6 +22,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -498,8 +499,11 @@ def moe_oracle_sample(wl: synth.MoEWorkload, seed: int = 0):
     return jobs, nbytes
 
 
-def oracle_job(wl):
-    """(run-once callable, algorithmic bytes, sample label) for the CPU oracle."""
+def oracle_job(wl, frac: float = 1.0):
+    """(run-once callable, algorithmic bytes) for the CPU oracle: layer 0 of the
+    workload, or (dense workloads, frac < 1) a frac share of every matrix's rows
+    per call, taken from a few row ranges spread over the matrix that successive
+    calls cycle through."""
     import oracle
     threads = os.cpu_count() or 1
     if isinstance(wl, synth.MoEWorkload):
@@ -515,12 +519,31 @@ def oracle_job(wl):
             oracle.moe_gemv_q4(cd, sd, h, True, idx, r, nthreads=threads)
         return run, nbytes
     mats = oracle_sample(wl)
-    nbytes = sum(m[3] for m in mats)
+    gemv = {2: oracle.gemv_q2, 3: oracle.gemv_q3, 4: oracle.gemv_q4, 5: oracle.gemv_q5,
+            6: oracle.gemv_q6, 8: oracle.gemv_q8}[wl.fmt]
+    if frac >= 1.0:
+        nbytes = sum(m[3] for m in mats)
+
+        def run():
+            for codes, scales, x, _ in mats:
+                gemv(codes, scales, x, nthreads=threads)
+        return run, nbytes
+    n_slices = min(8, int(math.ceil(1.0 / frac)))
+    sliced, nbytes = [], 0
+    for codes, scales, x, _ in mats:
+        N, K = codes.shape[0], x.shape[1]
+        n = min(N, max(16, int(round(N * frac))))
+        starts = [i * (N - n) // max(1, n_slices - 1) for i in range(n_slices)]
+        sliced.append([(codes[r:r + n].copy(), scales[r:r + n].copy(), x) for r in starts])
+        nbytes += synth.packed_bytes(wl.fmt, n, K) + wl.B * K * 2 + wl.B * n * 4
+    turn = [0]
 
     def run():
-        for codes, scales, x, _ in mats:
-            {2: oracle.gemv_q2, 3: oracle.gemv_q3, 4: oracle.gemv_q4, 5: oracle.gemv_q5,
-             6: oracle.gemv_q6, 8: oracle.gemv_q8}[wl.fmt](codes, scales, x, nthreads=threads)
+        i = turn[0] % n_slices
+        turn[0] += 1
+        for sl in sliced:
+            codes, scales, x = sl[i]
+            gemv(codes, scales, x, nthreads=threads)
     return run, nbytes
 
 
@@ -544,10 +567,22 @@ def cpu_baseline(wl, budget_s=10.0):
 
 
 def run_reference(args, wl, rank):
+    """The oracle on the host cores, on this workload's config and metric.  A
+    step is layer 0; when steps + warm-up of whole layers would overrun the
+    time budget, a step is the same share of every matrix's rows instead,
+    sized so the run fits (at least 1/256 of the rows and 16 rows a matrix)."""
     if rank != 0:
         return
     threads = os.cpu_count() or 1
     run, nbytes = oracle_job(wl)
+    t_layer = time_once(run)                       # a calibration pass (untimed)
+    frac, sample = 1.0, f"layer 0 of {wl.layers} per step ({nbytes/1e6:.1f} MB)"
+    budget = (args.steps + args.warmup) * t_layer
+    if budget > args.ref_budget_s and not isinstance(wl, synth.MoEWorkload):
+        frac = max(args.ref_budget_s / budget, 1.0 / 256)
+        run, nbytes = oracle_job(wl, frac)
+        sample = (f"{frac:.4f} of the rows of every matrix of layer 0 of {wl.layers} per step "
+                  f"({nbytes/1e6:.2f} MB), cycling over row ranges")
     for _ in range(args.warmup):
         time_once(run)
     t = 0.0
@@ -560,9 +595,9 @@ def run_reference(args, wl, rank):
         "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "batch": wl.B, "layers": wl.layers,
-                   "sample": "one layer per step"},
+                   "sample": "one layer per step" if frac >= 1.0 else "a share of one layer per step"},
         "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-                         "sample": f"layer 0 of {wl.layers} per step ({nbytes/1e6:.1f} MB)"},
+                         "sample": sample},
         "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -600,6 +635,8 @@ def main():
                          "with static weights; step: one cooperative launch per token "
                          "(bq_step_run)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget-s", type=float, default=90.0,
+                    help="--impl reference: seconds of oracle work the steps and warm-up may take")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     wl = WORKLOADS[args.workload]

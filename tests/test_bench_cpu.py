@@ -44,3 +44,14 @@ def test_reference_arm_json_contract():
 def test_reference_arm_other_formats(workload):
     d = _reference_line("--workload", workload)
     assert d["config"]["workload"] == workload and d["value"] > 0
+
+
+def test_reference_arm_shrinks_its_step_to_the_time_budget():
+    """Steps + warm-up of whole layers that would overrun the budget make each
+    step a share of every matrix's rows instead; the line says which share."""
+    d = _reference_line("--steps", "400", "--ref-budget-s", "2")
+    assert d["steps"] == 400 and d["value"] > 0
+    assert d["config"]["sample"] == "a share of one layer per step"
+    assert "of the rows of every matrix of layer 0" in d["cpu_baseline"]["sample"]
+    assert d["ms_per_step"] * 403 < 30e3        # the 2 s budget, with slack for a loaded host
+
