@@ -523,6 +523,26 @@ def test_gemv_brute_force_exact(fmt, N, K, B):
             assert abs(Fraction(a[b, n]) - exact_abs) <= exact_abs * Fraction(1, 2 ** 50)
 
 
+@pytest.mark.parametrize("fmt", [4, 8])
+@pytest.mark.parametrize("B", [16, 32])
+def test_gemv_brute_force_exact_wide_batch(fmt, B):
+    """Batches beyond the GEMV's 8 (the size of a speculative-decoding
+    verification batch): the oracle has no batch limit and stays exact."""
+    N, K = 3, 64
+    codes, scales = _rand_planes(fmt, N, K, 900 + B)
+    x = synth.activations_f16_bits(synth.key(5, 91, B, K, 1), B, K)
+    y, a = _GEMV[fmt](codes, scales, x)
+    xf = x.view(np.float16)
+    for b in range(B):
+        for n in range(N):
+            terms = [_unpack_fraction(fmt, codes, scales, n, k) * Fraction(xf[b, k].item())
+                     for k in range(K)]
+            exact = sum(terms)
+            exact_abs = sum(abs(t) for t in terms)
+            assert abs(Fraction(y[b, n]) - exact) <= exact_abs * Fraction(1, 2 ** 50)
+            assert abs(Fraction(a[b, n]) - exact_abs) <= exact_abs * Fraction(1, 2 ** 50)
+
+
 @pytest.mark.parametrize("fmt", [2, 3, 4, 5, 6, 8])
 def test_gemv_batch_rows_independent_and_threads(fmt):
     N, K, B = 37, 256, 6
