@@ -145,8 +145,12 @@ BQ_API int32_t bq_gemv_q8(const bq_qmat *W, const uint16_t *x, int32_t B, float 
  * counterpart of this entry point; it exists for such callers only.
  * Same operation, arguments and results as bq_gemv_q4, without ws/ws_bytes:
  * the scratch the kernel needs lives in one fixed array inside the library
- * (about 5.3 MB, reserved on every GPU that loads the library until the
- * process exits).
+ * (917,504 bytes, about 0.9 MB: 65,536 band counters plus cross-CTA partial
+ * sums for up to 320 CTAs; reserved on every GPU that loads the library until
+ * the process exits).
+ *   - Always 32-row work units (bq_gemv_q4 chooses 16 or 32 rows per call);
+ *     at most 320 CTAs.  Results are within the same tolerance as
+ *     bq_gemv_q4's, but not necessarily bit-identical to them.
  *   - N must be <= 1048576 rows; larger N returns BQ_ERR_WORKSPACE and
  *     launches nothing.  Nothing is allocated: no cudaMalloc / cudaFree.
  *   - The first call on a device looks up the array's device address (once
@@ -158,6 +162,15 @@ BQ_API int32_t bq_gemv_q8(const bq_qmat *W, const uint16_t *x, int32_t B, float 
  *     must be serialised by the caller. */
 BQ_API int32_t bq_gemv_q4_noalloc(const bq_qmat *W, const uint16_t *x, int32_t B, float *y,
                                   int32_t *dev_status, void *stream);
+
+/* Where bq_gemv_q4_noalloc's fixed scratch array lives on the current device:
+ * *dev_ptr its device address, *bytes its size (917,504).  Allocates and
+ * launches nothing.  For tests and tools that inspect the array, or clear or
+ * poison it to check that a call does not depend on what an earlier one left
+ * there.  Same once-per-device address lookup as the first
+ * bq_gemv_q4_noalloc call.  BQ_ERR_NULL if an argument is NULL, BQ_ERR_CUDA
+ * if the lookup fails. */
+BQ_API int32_t bq_gemv_q4_noalloc_scratch(void **dev_ptr, size_t *bytes);
 
 /* ------------------------------------------------------------ epilogues --- */
 
@@ -293,6 +306,33 @@ BQ_API int32_t bq_step_plan(int32_t fmt, const bq_step_mat *mats, int32_t n_mats
  *           (left zero-filled on completion) */
 BQ_API int32_t bq_step_run(const bq_step_info *info, const void *plan, void *ws, size_t ws_bytes,
                            int32_t *dev_status, void *stream);
+
+/* Bounded waits of a plan run.  Every wait in the library's kernels gives up
+ * after a bounded number of SM clock cycles and reports the bit
+ * 1 << BQ_ERR_TIMEOUT in *dev_status instead of hanging; the device never
+ * traps.
+ *   wait_cycles     cycles a grid-barrier wait may last (0 or above 4e9:
+ *                   the default, 4e9, about 2 s at 1.9 GHz)
+ *   extra_arrivals  arrivals each grid barrier waits for beyond the grid's
+ *                   own (0 in normal use; at most 1024).  A value > 0 asks
+ *                   for arrivals that no CTA makes: every CTA's first barrier
+ *                   then runs out after wait_cycles, reports the timeout and
+ *                   stops (it drains its own copies in flight and exits).  It
+ *                   exists so that the timeout path can be exercised without
+ *                   a fault or a missing CTA.
+ * After a run that reported BQ_ERR_TIMEOUT the workspace must be zero-filled
+ * again before the next run; the outputs of the stages after the failed
+ * barrier are not written. */
+typedef struct bq_step_wait {
+    int64_t wait_cycles;
+    int32_t extra_arrivals, reserved;
+} bq_step_wait;
+
+/* bq_step_run with explicit bounded-wait options (wait may be NULL: the
+ * defaults, as bq_step_run).  BQ_ERR_SHAPE on a negative option. */
+BQ_API int32_t bq_step_run_ex(const bq_step_info *info, const void *plan, void *ws,
+                              size_t ws_bytes, const bq_step_wait *wait, int32_t *dev_status,
+                              void *stream);
 
 /* ------------------------------------------------------ routed experts --- */
 

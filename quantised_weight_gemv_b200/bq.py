@@ -40,6 +40,11 @@ class bq_step_info(ctypes.Structure):
                 ("ws_bytes", ctypes.c_uint64)]
 
 
+class bq_step_wait(ctypes.Structure):
+    _fields_ = [("wait_cycles", ctypes.c_int64), ("extra_arrivals", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
 class bq_gemv_geometry(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("rows", "chunks", "chunks_per_band",
                                                "chunks_per_worker", "grid", "cluster",
@@ -67,10 +72,12 @@ _SIGS = {
     "bq_gemv_ex": (_i32, [_i32, _QP, _vp, _i32, _vp, _i32, _i32, _vp, _sz, _vp, _vp]),
     "bq_gemv_q8": (_i32, [_QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
     "bq_gemv_q4_noalloc": (_i32, [_QP, _vp, _i32, _vp, _vp, _vp]),
+    "bq_gemv_q4_noalloc_scratch": (_i32, [ctypes.POINTER(_vp), ctypes.POINTER(_sz)]),
     "bq_step_plan_bytes": (_sz, [_i32]),
     "bq_gemv_geometry_of": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp]),
     "bq_step_plan": (_i32, [_i32, _SMP, _i32, _vp, _sz, _SIP]),
     "bq_step_run": (_i32, [_SIP, _vp, _vp, _sz, _vp, _vp]),
+    "bq_step_run_ex": (_i32, [_SIP, _vp, _vp, _sz, ctypes.POINTER(bq_step_wait), _vp, _vp]),
     "bq_moe_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "bq_moe_gemv_q4": (_i32, [_QP, _i32, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _i32, _vp,
                               _vp, _sz, _vp, _vp]),
@@ -279,10 +286,20 @@ class StepPlan:
                                                  nbytes, ctypes.byref(self.info)))
         self.ws = workspace(self.info.ws_bytes, device)
 
-    def run(self, status=None, stream=None) -> None:
-        check("bq_step_run", lib().bq_step_run(ctypes.byref(self.info), self.plan_ptr,
-                                               self.ws.data_ptr(), self.ws.numel(), _ptr(status),
-                                               _stream_ptr(stream)))
+    def run(self, status=None, stream=None, wait_cycles: int | None = None,
+            extra_arrivals: int = 0) -> None:
+        """One step.  wait_cycles / extra_arrivals: bounded-wait options
+        (bq_step_run_ex); None / 0 are the defaults."""
+        if wait_cycles is None and extra_arrivals == 0:
+            check("bq_step_run", lib().bq_step_run(ctypes.byref(self.info), self.plan_ptr,
+                                                   self.ws.data_ptr(), self.ws.numel(),
+                                                   _ptr(status), _stream_ptr(stream)))
+            return
+        w = bq_step_wait(int(wait_cycles or 0), int(extra_arrivals), 0)
+        check("bq_step_run_ex", lib().bq_step_run_ex(ctypes.byref(self.info), self.plan_ptr,
+                                                     self.ws.data_ptr(), self.ws.numel(),
+                                                     ctypes.byref(w), _ptr(status),
+                                                     _stream_ptr(stream)))
 
 
 def quantize_dev(fmt: int, w, codes, scales, status=None, stream=None) -> None:

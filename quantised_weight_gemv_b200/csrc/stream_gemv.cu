@@ -116,10 +116,12 @@ struct KernelArgs {
     int n_mats;
     int wmax;                        // gridDim.x * kWarps
     int *counters;                   // per band of a stage; zero on entry and exit
-    float *partials;                 // [wmax][2][kMT][32 lanes] float4
+    float *partials;                 // [CTA][slot 0/1][kMT][32 lanes] float4 (cross-CTA band sums)
     int *status;                     // device status word or null
     int prefill;                     // matrix mode: load weights before the PDL wait
     unsigned *sync;                  // plan mode: [0] arrivals, [64] exits (separate lines)
+    long long wait_cycles;           // plan mode: limit of a grid-barrier wait (SM cycles)
+    int extra_arrivals;              // plan mode: arrivals a barrier waits for beyond the grid's
     // routed experts
     int E, topk, x_per_slot;
     const int *idx;
@@ -214,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     __shared__ int cta_arrivals;
     __shared__ int local_ctr[kWarps];   // arrivals of CTA-local split bands
     __shared__ alignas(8) uint64_t stage_bar;
+    __shared__ int stage_failed;        // PLAN: a grid-barrier wait ran out
     __shared__ alignas(8) uint64_t cl_bar;   // CL: cross-CTA partials received
 
     uint8_t *sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -265,6 +268,7 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
         local_ctr[threadIdx.x] = 0;
     if (PLAN && threadIdx.x == 0) {
         cta_arrivals = 0;
+        stage_failed = 0;
         mbar_init(smem_u32(&stage_bar), 1);
     }
     if (CL && threadIdx.x == 0) {
@@ -706,7 +710,11 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
     // reduction; release is cumulative, so it publishes every warp's y
     // stores) and polls the counter (acquire, short back-off) until all CTAs
     // have arrived, then releases its CTA's warps through a shared mbarrier.
-    // Every wait is bounded.
+    // Every wait is bounded: the grid poll by a.wait_cycles, after which it
+    // reports BQ_ERR_TIMEOUT, marks the CTA's barrier failed and still
+    // releases the CTA's warps, which then stop (drain their copies, exit).
+    // a.extra_arrivals > 0 asks for arrivals no CTA makes: the way a test
+    // makes the expiry path run without a fault or a missing CTA.
     auto stage_arrive_and_wait = [&](int s) {
         __syncwarp();
         if (lane == 0) {
@@ -714,17 +722,20 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
             asm volatile("atom.acq_rel.cta.shared::cta.add.s32 %0, [%1], 1;"
                          : "=r"(old) : "r"(smem_u32(&cta_arrivals)) : "memory");
             if (old == kWarps * (s + 1) - 1) {
-                const unsigned target = gridDim.x * (unsigned)(s + 1);
+                const unsigned target = (gridDim.x + (unsigned)a.extra_arrivals) * (unsigned)(s + 1);
                 asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&a.sync[0]) : "memory");
                 const long long t0 = clock64();
                 while (ld_acquire_gpu(&a.sync[0]) < target) {
-                    if (clock64() - t0 > kWaitCycles) {
+                    if (clock64() - t0 > a.wait_cycles) {
                         if (a.status)
                             atomicOr(a.status, kStatusTimeout);
+                        stage_failed = 1;
                         break;
                     }
                     __nanosleep(32);
                 }
+                // (the mbarrier arrive releases the stage_failed store to
+                // the CTA's warps, whose wait acquires it)
                 asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&stage_bar))
                              : "memory");
             }
@@ -735,6 +746,8 @@ __global__ void __launch_bounds__(kThreads, BQ_MIN_BLOCKS) stream_gemv_kernel(co
                 atomicOr(a.status, kStatusTimeout);
             ok = false;
         }
+        if (*(volatile int *)&stage_failed)
+            ok = false;
     };
 
     Cursor cur;
@@ -1256,7 +1269,7 @@ int32_t gemv_impl(const bq_qmat *W, const uint16_t *x, int32_t B, void *y, int32
 
 template <int FMT>
 int32_t step_run_impl(const bq_step_info *info, const void *plan, void *ws, int32_t *dev_status,
-                      void *stream)
+                      void *stream, long long wait_cycles, int extra_arrivals)
 {
     int32_t st = prepare_kernel<FMT, kModePlan>();
     if (st != BQ_OK)
@@ -1274,6 +1287,8 @@ int32_t step_run_impl(const bq_step_info *info, const void *plan, void *ws, int3
     a.counters = reinterpret_cast<int *>(wsb + kSyncBytes);
     a.partials = reinterpret_cast<float *>(wsb + kSyncBytes + counters_bytes(info->max_stage_bands));
     a.status = dev_status;
+    a.wait_cycles = wait_cycles;
+    a.extra_arrivals = extra_arrivals;
     void *args[] = {&a};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(info->grid);
@@ -1493,8 +1508,9 @@ extern "C" int32_t bq_step_plan(int32_t fmt, const bq_step_mat *mats, int32_t n_
     return BQ_OK;
 }
 
-extern "C" int32_t bq_step_run(const bq_step_info *info, const void *plan, void *ws,
-                               size_t ws_bytes, int32_t *dev_status, void *stream)
+extern "C" int32_t bq_step_run_ex(const bq_step_info *info, const void *plan, void *ws,
+                                  size_t ws_bytes, const bq_step_wait *wait, int32_t *dev_status,
+                                  void *stream)
 {
     if (!info || !plan || !ws)
         return BQ_ERR_NULL;
@@ -1504,8 +1520,23 @@ extern "C" int32_t bq_step_run(const bq_step_info *info, const void *plan, void 
         return BQ_ERR_ALIGN;
     if (ws_bytes < info->ws_bytes)
         return BQ_ERR_WORKSPACE;
-    return info->fmt == 4 ? step_run_impl<4>(info, plan, ws, dev_status, stream)
-                          : step_run_impl<8>(info, plan, ws, dev_status, stream);
+    long long cycles = kWaitCycles;
+    int extra = 0;
+    if (wait) {
+        if (wait->wait_cycles < 0 || wait->extra_arrivals < 0 || wait->extra_arrivals > 1024)
+            return BQ_ERR_SHAPE;
+        if (wait->wait_cycles > 0)
+            cycles = std::min<long long>(wait->wait_cycles, kWaitCycles);   // (the warps' own limit)
+        extra = wait->extra_arrivals;
+    }
+    return info->fmt == 4 ? step_run_impl<4>(info, plan, ws, dev_status, stream, cycles, extra)
+                          : step_run_impl<8>(info, plan, ws, dev_status, stream, cycles, extra);
+}
+
+extern "C" int32_t bq_step_run(const bq_step_info *info, const void *plan, void *ws,
+                               size_t ws_bytes, int32_t *dev_status, void *stream)
+{
+    return bq_step_run_ex(info, plan, ws, ws_bytes, nullptr, dev_status, stream);
 }
 
 // ------------------------------------------------------- routed experts --
@@ -1657,6 +1688,8 @@ constexpr size_t kNoAllocCounterBytes = (size_t)(kNoAllocMaxRows / 16) * sizeof(
 constexpr size_t kNoAllocPartialBytes =
     (size_t)kNoAllocMaxCtas * 2 * Fmt<4>::kMT * 32 * sizeof(float4);
 constexpr size_t kNoAllocScratchBytes = kNoAllocCounterBytes + kNoAllocPartialBytes;
+// The size the header states (262,144 bytes of counters + 655,360 of partials).
+static_assert(kNoAllocScratchBytes == 917504, "the documented size of the no-allocation scratch");
 }  // namespace
 }  // namespace bq
 
@@ -1740,4 +1773,17 @@ extern "C" int32_t bq_gemv_q4_noalloc(const bq_qmat *W, const uint16_t *x, int32
     cudaError_t e = launch_pdl((const void *)stream_gemv_kernel<4, kModeMatrix>, dim3(G),
                                dim3(kThreads), launch_smem<4>(1, 1), s, args);
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+extern "C" int32_t bq_gemv_q4_noalloc_scratch(void **dev_ptr, size_t *bytes)
+{
+    if (!dev_ptr || !bytes)
+        return BQ_ERR_NULL;
+    int32_t err = BQ_OK;
+    void *p = noalloc_scratch(&err);
+    if (!p)
+        return err;
+    *dev_ptr = p;
+    *bytes = kNoAllocScratchBytes;
+    return BQ_OK;
 }

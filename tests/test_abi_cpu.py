@@ -283,3 +283,17 @@ def test_step_argument_validation_before_launch():
     assert L.bq_step_run(None, FAKE, FAKE, 1 << 20, None, None) == bq.BQ_ERR_NULL
     assert L.bq_step_run(ctypes.byref(info), FAKE, FAKE, 1024, None, None) == bq.BQ_ERR_WORKSPACE
     assert L.bq_step_run(ctypes.byref(info), FAKE + 16, FAKE, 1 << 20, None, None) == bq.BQ_ERR_ALIGN
+
+
+def test_step_run_ex_rejects_negative_options():
+    """Host-side checks of the bounded-wait options: nothing is launched."""
+    import ctypes
+    info = bq.bq_step_info()
+    info.fmt, info.n_stages, info.grid = 4, 1, 1
+    w = bq.bq_step_wait(-1, 0, 0)
+    fake = 0x7f0000000000
+    assert bq.lib().bq_step_run_ex(ctypes.byref(info), fake, fake, 1 << 30, ctypes.byref(w),
+                                   None, None) == bq.BQ_ERR_SHAPE
+    w = bq.bq_step_wait(0, -1, 0)
+    assert bq.lib().bq_step_run_ex(ctypes.byref(info), fake, fake, 1 << 30, ctypes.byref(w),
+                                   None, None) == bq.BQ_ERR_SHAPE

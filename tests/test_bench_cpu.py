@@ -24,6 +24,7 @@ def _reference_line(*extra):
 
 
 def test_reference_arm_json_contract():
+    """The default workload: the 64-layer hidden-5120 decoder."""
     import bench
     d = _reference_line()
     assert d["impl"] == "reference"
@@ -31,7 +32,7 @@ def test_reference_arm_json_contract():
     assert d["higher_is_better"] is True and d["n_gpus"] == 1 and d["steps"] == 1
     assert d["warmup"] >= 3                          # warm-up is never below three steps
     assert d["value"] > 0 and d["ms_per_step"] > 0
-    assert d["config"]["workload"] == "dense16L-h2048-ffn8192-q4"
+    assert d["config"]["workload"] == "dense64L-h5120-ffn25600-q4"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
     assert "layer 0" in cb["sample"]
@@ -40,7 +41,8 @@ def test_reference_arm_json_contract():
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
 
 
-@pytest.mark.parametrize("workload", ["dense16L-h2048-ffn8192-q3", "dense16L-h2048-ffn8192-q2"])
+@pytest.mark.parametrize("workload", ["dense16L-h2048-ffn8192-q4", "dense16L-h2048-ffn8192-q3",
+                                      "dense16L-h2048-ffn8192-q2"])
 def test_reference_arm_other_formats(workload):
     d = _reference_line("--workload", workload)
     assert d["config"]["workload"] == workload and d["value"] > 0
@@ -49,9 +51,25 @@ def test_reference_arm_other_formats(workload):
 def test_reference_arm_shrinks_its_step_to_the_time_budget():
     """Steps + warm-up of whole layers that would overrun the budget make each
     step a share of every matrix's rows instead; the line says which share."""
-    d = _reference_line("--steps", "400", "--ref-budget-s", "2")
+    d = _reference_line("--steps", "400", "--ref-budget-s", "2", "--workload",
+                        "dense16L-h2048-ffn8192-q4")
     assert d["steps"] == 400 and d["value"] > 0
     assert d["config"]["sample"] == "a share of one layer per step"
     assert "of the rows of every matrix of layer 0" in d["cpu_baseline"]["sample"]
-    assert d["ms_per_step"] * 403 < 30e3        # the 2 s budget, with slack for a loaded host
+    share = d["config"]["rows_share"]
+    assert 0 < share < 1
+    # ms_per_step is a whole layer's time; the share of it timed per step fits
+    # the 2 s budget (with slack for a loaded host)
+    assert d["ms_per_step"] * share * 403 < 30e3
+    # the rate is the same whether the layer or its share is counted
+    layer_mb = 34.3
+    assert abs(layer_mb * 1e6 / (d["ms_per_step"] / 1e3) / 1e9 - d["value"]) < 0.2 * d["value"]
+
+
+def test_default_workload_is_the_largest_single_gpu_decoder():
+    import bench
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    assert 'default=synth.DENSE_H5120.name' in src
+    wl = bench.WORKLOADS["dense64L-h5120-ffn25600-q4"]
+    assert wl.layers == 64 and wl.B == 1
 

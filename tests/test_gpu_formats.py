@@ -30,7 +30,7 @@ _DEQ = {2: oracle.dequantize_q2, 3: oracle.dequantize_q3, 5: oracle.dequantize_q
 
 
 @pytest.mark.parametrize("fmt,N,K", CASES)
-@pytest.mark.parametrize("B", [1, 3, 8])
+@pytest.mark.parametrize("B", [1, 3, 4, 8])
 @pytest.mark.parametrize("flags", [0, bq.BQ_GEMV_STATIC_WEIGHTS])
 def test_gemv_parity(fmt, N, K, B, flags):
     w = synth.weights_f32(synth.key(fmt, 84, N, K, synth.KIND_W), N, K)
@@ -76,7 +76,7 @@ def test_device_quantiser_bit_exact(fmt):
 
 
 @pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("F,K,B", [(8, 256, 1), (200, 2048, 3), (1024, 512, 8)])
+@pytest.mark.parametrize("F,K,B", [(8, 256, 1), (200, 2048, 3), (512, 1024, 4), (1024, 512, 8)])
 def test_swiglu_epilogue(fmt, F, K, B):
     import torch
     wg = synth.weights_f32(synth.key(1, 87, F, K, synth.KIND_W), F, K)

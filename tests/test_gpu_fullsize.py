@@ -49,24 +49,39 @@ def _gemv(fmt, codes, scales, xb):
     return fn(codes, scales, xb, nthreads=8)
 
 
-def _check_step(wl, every, seed=0, engine="step"):
-    """Run the decode step once; check sampled rows of every matrix.  The fused
-    feed-forward stage (gate|up in SwiGLU pair order) is checked on its fp16
-    output h against the oracle's SwiGLU of the oracle's gate and up GEMVs;
-    the down stage then reads the h the GPU produced."""
+def _check_step(wl, every, seed=0, engines=("step",)):
+    """Run the decode step once per engine; check sampled rows of every
+    matrix after each.  The fused feed-forward stage (gate|up in SwiGLU pair
+    order) is checked on its fp16 output h against the oracle's SwiGLU of the
+    oracle's gate and up GEMVs; the down stage then reads the h the GPU
+    produced.  Every output buffer is filled with NaN before each engine runs,
+    so each engine must write every output itself.  engines: "step" (one plan,
+    a single cooperative launch) and/or "graph" (the per-matrix launch chain
+    with static weights that bench.py times)."""
     import torch
     import bench
     step = bench.DenseStep(wl, torch.device(DEV), seed=seed)
-    if engine == "step":
-        step.build_plan()
-        st = new_status()
-        step.plan.run(st)
-        torch.cuda.synchronize()
-        assert int(st.item()) == 0
-    else:       # the per-matrix launch chain bench.py's graph engine times
-        step.launch(torch.cuda.current_stream())
-        torch.cuda.synchronize()
-    assert int(step.status.item()) == 0
+    worst = 0.0
+    for engine in engines:
+        step.y_all.fill_(float("nan"))
+        step.h_all.fill_(float("nan"))
+        if engine == "step":
+            step.build_plan()
+            st = new_status()
+            step.plan.run(st)
+            torch.cuda.synchronize()
+            assert int(st.item()) == 0
+        else:       # the per-matrix launch chain bench.py's graph engine times
+            step.launch(torch.cuda.current_stream())
+            torch.cuda.synchronize()
+        assert int(step.status.item()) == 0
+        worst = max(worst, _check_outputs(wl, step, every, seed))
+    return worst
+
+
+def _check_outputs(wl, step, every, seed):
+    import torch
+    import bench
     rng = np.random.default_rng([seed, wl.wid, 12345])
     stages = bench.fused_stages(wl)
     worst = 0.0
@@ -135,54 +150,67 @@ def test_single_q8_2048_all_rows():
     check_tol(y.cpu().numpy(), yr, ar)
 
 
-@pytest.mark.parametrize("engine", ["step", "graph"])
-def test_dense16_h2048_step(engine):
-    """16-layer decoder (hidden 2048, FFN 8192), Q4, batch 1: as one plan, and
-    as the chain of per-matrix launches with static weights."""
-    _check_step(synth.DENSE_H2048, every=16, engine=engine)
+def test_dense16_h2048_step_every_row():
+    """16-layer decoder (hidden 2048, FFN 8192), Q4, batch 1: every output row
+    of every layer, as one plan and as the chain of per-matrix launches with
+    static weights."""
+    _check_step(synth.DENSE_H2048, every=1, engines=("step", "graph"))
 
 
 @pytest.mark.parametrize("fmt", [6, 5, 3, 2])
 def test_dense16_h2048_other_formats_chain(fmt):
     """The 16-layer hidden-2048 decoder in Q6, Q5, Q3 and Q2, as the launch chain."""
-    _check_step(synth.dense_h2048(fmt), every=16, engine="graph")
+    _check_step(synth.dense_h2048(fmt), every=16, engines=("graph",))
 
 
 @pytest.mark.parametrize("fmt", [4, 8])
-def test_dense36_h4096_step_batch8(fmt):
-    """36 distinct copies of a hidden-4096 layer, batch 8, as a launch chain."""
-    _check_step(synth.dense_h4096(fmt, 8), every=128, engine="graph")
+@pytest.mark.parametrize("B", [1, 2, 4, 8])
+def test_dense36_h4096_step(fmt, B):
+    """36 distinct copies of a hidden-4096 layer at batch 1, 2, 4 and 8, in Q4
+    and Q8, as the launch chain: every row of the first and last layer, 1/128
+    of the rows of every other matrix."""
+    _check_step(synth.dense_h4096(fmt, B), every=128, engines=("graph",))
 
 
 def test_dense64_h5120_step():
-    """64-layer decoder (hidden 5120, FFN 25600, ~16 GB Q4), batch 1, as one plan."""
-    _check_step(synth.DENSE_H5120, every=1024)
+    """64-layer decoder (hidden 5120, FFN 25600, ~16 GB Q4), batch 1: as the
+    launch chain bench.py times, and as one plan."""
+    _check_step(synth.DENSE_H5120, every=1024, engines=("graph", "step"))
 
 
-@pytest.mark.parametrize("B", [1, 8])
-def test_moe_layer_full(B):
-    """Layer 0 of the routed-expert decode step, built exactly as the benchmark
-    builds it (128 experts, gate|up 1536 x 2048 per expert in SwiGLU pair
-    order, down 2048 x 768, top-8): per-slot h = silu(gate) * up of every
-    routed slot, and y = down(h) combined with the routing weights, against
-    the oracle on every routed expert."""
-    import dataclasses
+@pytest.mark.parametrize("B,layers", [(1, None), (8, (0, 47))])
+def test_moe_step_full(B, layers):
+    """The routed-expert decode step built exactly as the benchmark builds it
+    (48 layers of 128 experts, gate|up 1536 x 2048 per expert in SwiGLU pair
+    order, down 2048 x 768, top-8), run once as the benchmark's launch
+    sequence: per-slot h = silu(gate) * up of every routed slot, and y =
+    down(h) combined with the routing weights, against the oracle on every
+    routed expert -- of all 48 layers at batch 1, of the first and last layer
+    at batch 8 (52 distinct experts a layer)."""
     import torch
     import bench
-    wl = dataclasses.replace(synth.moe_h2048(B), layers=1)
+    wl = synth.moe_h2048(B)
     step = bench.MoEStep(wl, torch.device(DEV))
+    step.h_all.fill_(float("nan"))
+    step.y_all.fill_(0xFF)               # NaN bit patterns in every fp32 output
     step.launch(torch.cuda.current_stream())
     torch.cuda.synchronize()
     assert int(step.status.item()) == 0
-    E, topk, seed = wl.E, wl.topk, 0
+    for layer in (range(wl.layers) if layers is None else layers):
+        _check_moe_layer(wl, step, layer)
+
+
+def _check_moe_layer(wl, step, layer, seed=0):
+    import torch
+    E, topk = wl.E, wl.topk
     (Ng, Kg), (Nd, Kd) = wl.gateup(), wl.down()
     F = Ng // 2
-    stacks, idx_d, r_d, x_d, h_d, y_d = step.layers[0]
+    stacks, idx_d, r_d, x_d, h_d, y_d = step.layers[layer]
     idx, r = idx_d.cpu().numpy(), r_d.cpu().numpy()
     used = sorted(set(idx.ravel().tolist()))
     planes = []
     for mid, (N, K) in ((0, (Ng, Kg)), (1, (Nd, Kd))):
-        w = synth.weights_f32_torch(synth.key(seed, wl.wid, 0, mid, synth.KIND_W), E * N, K, DEV)
+        w = synth.weights_f32_torch(synth.key(seed, wl.wid, layer, mid, synth.KIND_W), E * N, K, DEV)
         rows = np.concatenate([np.arange(e * N, (e + 1) * N) for e in used])
         wu = w[torch.as_tensor(rows, device=DEV)].cpu().numpy().reshape(len(used), N, K)
         del w
@@ -201,8 +229,9 @@ def test_moe_layer_full(B):
                 want_s = pair_order(parts[0][1][e], parts[1][1][e])
             else:
                 want_c, want_s = parts[0][0][e], parts[0][1][e]
-            assert np.array_equal(codes_d[e].cpu().numpy(), want_c), f"expert {e} codes"
-            assert np.array_equal(scales_d[e].cpu().numpy().view(np.uint16), want_s), f"expert {e} scales"
+            assert np.array_equal(codes_d[e].cpu().numpy(), want_c), f"L{layer} expert {e} codes"
+            assert np.array_equal(scales_d[e].cpu().numpy().view(np.uint16), want_s), \
+                f"L{layer} expert {e} scales"
         planes.append(parts)
     xb = x_d.cpu().numpy().view(np.uint16)
     (cg, sg), (cu, su) = planes[0]

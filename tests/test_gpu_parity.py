@@ -20,7 +20,7 @@ SHAPES = [(1, 32), (15, 32), (16, 256), (17, 288), (33, 800), (100, 2048), (257,
 
 @pytest.mark.parametrize("fmt", [4, 8])
 @pytest.mark.parametrize("N,K", SHAPES)
-@pytest.mark.parametrize("B", [1, 2, 3, 8])
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_gemv_parity_small(fmt, N, K, B):
     w = synth.weights_f32(synth.key(0, 80, N, K, synth.KIND_W), N, K)
     codes, scales = quantize(fmt, w)
@@ -32,7 +32,7 @@ def test_gemv_parity_small(fmt, N, K, B):
 
 @pytest.mark.parametrize("rows", [16, 32])
 @pytest.mark.parametrize("N,K", SHAPES)
-@pytest.mark.parametrize("B", [1, 3, 8])
+@pytest.mark.parametrize("B", [1, 3, 4, 8])
 def test_q4_chunk_heights_parity(rows, N, K, B):
     """Q4 with 16-row and with 32-row work units (BQ_GEMV_ROWS16 / ROWS32):
     both within the oracle's tolerance."""
@@ -50,7 +50,7 @@ def test_q4_chunk_heights_parity(rows, N, K, B):
                                           (4, 2048, 8192, 16), (8, 1024, 8192, 16),
                                           (4, 1024, 5120, 32), (4, 1024, 1536, 32),
                                           (4, 1000, 1792, 32), (8, 512, 2560, 16)])
-@pytest.mark.parametrize("B", [1, 3, 8])
+@pytest.mark.parametrize("B", [1, 3, 4, 8])
 def test_bands_summed_across_ctas_in_clusters(fmt, N, K, rows, B):
     """Shapes whose bands are split among several CTAs (each band's chunks
     outnumber a CTA's warps) with cluster boundaries on band boundaries: the
@@ -71,7 +71,7 @@ def test_bands_summed_across_ctas_in_clusters(fmt, N, K, rows, B):
 
 @pytest.mark.parametrize("fmt", [4, 8])
 @pytest.mark.parametrize("N,K", SHAPES)
-@pytest.mark.parametrize("B", [1, 3, 8])
+@pytest.mark.parametrize("B", [1, 3, 4, 8])
 def test_gemv_static_weights_parity(fmt, N, K, B):
     """With BQ_GEMV_STATIC_WEIGHTS the weight ring fills before the wait on
     the previous kernel; the arithmetic is the plain call's, so y is the
@@ -227,7 +227,8 @@ def gpu_moe(codes, scales, x, x_per_slot, idx, r):
     return y.cpu().numpy(), int(st.item())
 
 
-@pytest.mark.parametrize("B,topk,E", [(1, 8, 32), (8, 8, 32), (3, 4, 5), (8, 2, 1)])
+@pytest.mark.parametrize("B,topk,E", [(1, 8, 32), (4, 8, 32), (8, 8, 32), (3, 4, 5), (8, 2, 1),
+                                      (4, 2, 6)])
 @pytest.mark.parametrize("x_per_slot", [False, True])
 @pytest.mark.parametrize("combine", [False, True])
 def test_moe_parity(B, topk, E, x_per_slot, combine):

@@ -28,7 +28,7 @@ def _ffn_inputs(fmt, F, K, B, seed):
 @pytest.mark.parametrize("fmt,flags", [(4, 0), (4, bq.BQ_GEMV_ROWS16), (4, bq.BQ_GEMV_ROWS32),
                                        (8, 0)])
 @pytest.mark.parametrize("F,K", [(8, 256), (24, 800), (200, 2048), (1024, 512)])
-@pytest.mark.parametrize("B", [1, 3, 8])
+@pytest.mark.parametrize("B", [1, 3, 4, 8])
 def test_gemv_swiglu_epilogue(fmt, flags, F, K, B):
     """The SwiGLU epilogue with either Q4 chunk height (a 16-row tile holds 8
     gate and the same 8 up rows in both)."""
@@ -122,7 +122,7 @@ def _expert_ffn(E, F, H, seed):
     return [np.stack(a) for a in (cg, sg, cu, su, cd, sd)]
 
 
-@pytest.mark.parametrize("B,topk,E", [(1, 8, 16), (8, 8, 32), (3, 2, 5)])
+@pytest.mark.parametrize("B,topk,E", [(1, 8, 16), (4, 8, 16), (8, 8, 32), (3, 2, 5)])
 def test_moe_expert_ffn_fused(B, topk, E):
     """Routed-expert feed-forward block: per-slot gate|up with the SwiGLU
     epilogue writes h [B][topk][F] (fp16), then down reads it per slot and

@@ -250,6 +250,47 @@ def test_quantize_nearest_grid_point():
         assert np.all(np.abs(deq - w) <= nearest + 1e-18)
 
 
+@pytest.mark.parametrize("fmt,levels,zero", [(4, 7, 8), (8, 127, 0), (6, 31, 32), (5, 15, 16),
+                                             (3, 3, 4), (2, 1, 2)])
+def test_quantize_scale_and_codes_recomputed_in_numpy(fmt, levels, zero):
+    """Random blocks (N(0, 0.02) rows scaled over six decades, some with
+    outliers): the oracle's stored fp16 scale bits equal
+    fp16(fp32(absmax) / fp32(levels)) computed by numpy's IEEE fp32 divide and
+    nearest-even fp16 conversion, and every dequantised weight equals
+    d * (q - zero) with q = clamp(round_half_away(fp32(w) / fp32(d)) + zero)
+    -- the quotient an IEEE fp32 division by the *stored* scale.  Dividing by
+    the unrounded fp32 scale instead changes codes on random blocks and fails
+    here.  (Dividing in fp64 gives the same codes: the stored scale has 11
+    significant bits, so (k + 1/2) * d is an fp32 number and no fp32 quotient
+    of an fp32 w can round onto a tie the exact quotient misses.)"""
+    rng = np.random.default_rng([fmt, 4242])
+    N, K = 96, 512
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    w *= (10.0 ** rng.uniform(-4, 2, size=(N, 1))).astype(np.float32)
+    out = rng.random((N, K)) < 0.01
+    w[out] *= np.float32(9.0)
+    quant = {2: oracle.quantize_q2, 3: oracle.quantize_q3, 4: oracle.quantize_q4,
+             5: oracle.quantize_q5, 6: oracle.quantize_q6, 8: oracle.quantize_q8}[fmt]
+    deq = {2: oracle.dequantize_q2, 3: oracle.dequantize_q3, 4: oracle.dequantize_q4,
+           5: oracle.dequantize_q5, 6: oracle.dequantize_q6, 8: oracle.dequantize_q8}[fmt]
+    codes, scales = quant(w)
+    blocks = w.reshape(N, K // 32, 32)
+    amax = np.abs(blocks).max(axis=2).astype(np.float32)
+    d16 = (amax / np.float32(levels)).astype(np.float16)          # fp32 divide, RNE to fp16
+    assert np.array_equal(scales[:, :K // 32], d16.view(np.uint16))
+    d32 = d16.astype(np.float32)
+    q = np.zeros(blocks.shape, dtype=np.float64)
+    nz = d32 != 0
+    quot = (blocks / np.where(nz, d32, np.float32(1))[..., None]).astype(np.float32)
+    r = np.sign(quot) * np.floor(np.abs(quot.astype(np.float64)) + 0.5)   # half away from zero
+    lo, hi = (-127, 127) if fmt == 8 else (0, 2 * zero - 1)
+    q = np.clip(r + zero, lo, hi)
+    q = np.where(nz[..., None], q, zero)
+    want = (d32.astype(np.float64)[..., None] * (q - zero)).reshape(N, K)
+    got = deq(codes, scales)
+    assert np.array_equal(got, want)
+
+
 # ---------------------------------------------------------- golden files ----
 @pytest.mark.parametrize("name,fmt", [("q4_block_worked.txt", 4), ("q8_block_worked.txt", 8),
                                       ("q6_block_worked.txt", 6), ("q5_block_worked.txt", 5),
