@@ -105,6 +105,10 @@ def lib() -> ctypes.CDLL:
             L.oracle_silu.argtypes = [ctypes.c_double]
             L.oracle_swiglu_f16.restype = None
             L.oracle_swiglu_f16.argtypes = [_c_f64p, _c_f64p, ctypes.c_int, _c_u16p]
+            L.oracle_attn_decode_q8.restype = ctypes.c_int
+            L.oracle_attn_decode_q8.argtypes = [
+                _c_i8p, _c_u16p, _c_i8p, _c_u16p, _c_u16p, _c_i32p, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, _c_f64p, _c_f64p]
             _lib = L
         return _lib
 
@@ -372,3 +376,32 @@ def swiglu_f16(g, u) -> np.ndarray:
     h = np.empty(g.shape, dtype=np.uint16)
     lib().oracle_swiglu_f16(_p(g, _c_f64p), _p(u, _c_f64p), int(g.size), _p(h, _c_u16p))
     return h
+
+
+def attn_decode_q8(k_codes, k_scales, vt_codes, v_scales, q_bits, lens, scale: float):
+    """Decode attention over a Q8 KV cache (fp64).
+
+    k_codes int8 [B, Hkv, Tmax, D]; k_scales uint16 [B, Hkv, Tmax, D/32];
+    vt_codes int8 [B, Hkv, D, Tmax] (values transposed); v_scales uint16
+    [B, Hkv, Tmax, D/32]; q_bits uint16 [B, Hkv*G, D]; lens int32 [B].
+    Returns (o, abso, had_empty) with o, abso float64 [B, Hkv*G, D]."""
+    k_codes = np.ascontiguousarray(k_codes, dtype=np.int8)
+    k_scales = np.ascontiguousarray(k_scales, dtype=np.uint16)
+    vt_codes = np.ascontiguousarray(vt_codes, dtype=np.int8)
+    v_scales = np.ascontiguousarray(v_scales, dtype=np.uint16)
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    lens = np.ascontiguousarray(lens, dtype=np.int32)
+    B, Hkv, Tmax, D = k_codes.shape
+    H = q_bits.shape[1]
+    assert H % Hkv == 0 and q_bits.shape == (B, H, D) and lens.shape == (B,)
+    assert k_scales.shape == (B, Hkv, Tmax, D // 32) and v_scales.shape == k_scales.shape
+    assert vt_codes.shape == (B, Hkv, D, Tmax)
+    o = np.zeros((B, H, D), dtype=np.float64)
+    abso = np.zeros_like(o)
+    rc = lib().oracle_attn_decode_q8(
+        _p(k_codes, _c_i8p), _p(k_scales, _c_u16p), _p(vt_codes, _c_i8p), _p(v_scales, _c_u16p),
+        _p(q_bits, _c_u16p), _p(lens, _c_i32p), B, Hkv, H // Hkv, D, Tmax, float(scale),
+        _p(o, _c_f64p), _p(abso, _c_f64p))
+    if rc not in (0, 2):
+        raise ValueError(f"oracle attention failed ({rc})")
+    return o, abso, rc == 2

@@ -601,3 +601,106 @@ void oracle_swiglu_f16(const double *g, const double *u, int n, uint16_t *h)
     for (int i = 0; i < n; i++)
         h[i] = oracle_double_to_half(oracle_silu(g[i]) * u[i]);
 }
+
+/* ---------------------------------------------------------------------------
+ * Decode attention over a block-quantised KV cache.  The pages' runtime keeps
+ * its KV cache preallocated for the whole decode loop (gist.science technical
+ * summary, "Methodologie" -> "Zero-Allocation Decode Loop"), and at decode
+ * runs a specialised decode-attention kernel beside the GEMV (romaanj.github.io
+ * review of the M5 follow-up paper, "Method").  One new token per sequence
+ * attends to the positions t < lens[b] of its cache:
+ *
+ *      s_t  = scale * sum_d q[d] * K[t][d]
+ *      p_t  = exp(s_t - max_u s_u) / sum_u exp(s_u - max_u s_u)
+ *      o[d] = sum_t p_t * V[t][d]
+ *
+ * with K[t][d] = dK(t, d/32) * k(t, d) and V[t][d] = dV(t, d/32) * v(d, t):
+ * the cache rows are Q8 blocks of 32 along the head dimension (fp16 scale
+ * d = absmax/127, int8 codes -- the Q8 format of the weights, applied to each
+ * position's key and value vectors).  Query head i of a sequence uses KV head
+ * i / G (grouped-query attention).  Everything is evaluated in fp64.
+ *
+ * Layouts (all row-major):
+ *   k_codes   int8  [B][Hkv][Tmax][D]          key codes, one row per position
+ *   k_scales  fp16  [B][Hkv][Tmax][D/32]
+ *   vt_codes  int8  [B][Hkv][D][Tmax]          value codes transposed: row d
+ *                                              holds component d of every
+ *                                              position
+ *   v_scales  fp16  [B][Hkv][Tmax][D/32]       scale of position t's block j
+ *   q         fp16  [B][Hkv*G][D]
+ *   lens      int32 [B]                        0 <= lens[b] <= Tmax
+ *   o, abso   fp64  [B][Hkv*G][D]              abso[d] = sum_t p_t |V[t][d]|
+ * A sequence with lens[b] == 0 attends to nothing: its outputs are zero and
+ * the return value has bit 1 set.  Positions t >= lens[b] are never read.
+ * ------------------------------------------------------------------------ */
+int oracle_attn_decode_q8(const int8_t *k_codes, const uint16_t *k_scales,
+                          const int8_t *vt_codes, const uint16_t *v_scales, const uint16_t *q,
+                          const int32_t *lens, int B, int Hkv, int G, int D, int Tmax,
+                          double scale, double *o, double *abso)
+{
+    if (B < 1 || Hkv < 1 || G < 1 || D < ORACLE_BLOCK || D % ORACLE_BLOCK || Tmax < 1)
+        return -1;
+    const int nb = D / ORACLE_BLOCK, H = Hkv * G;
+    int empty = 0;
+    double *s = (double *)malloc(sizeof(double) * (size_t)Tmax);
+    double *qd = (double *)malloc(sizeof(double) * (size_t)D);
+    if (!s || !qd) {
+        free(s);
+        free(qd);
+        return -3;
+    }
+    for (int b = 0; b < B; b++) {
+        const int L = lens[b];
+        if (L < 0 || L > Tmax) {
+            free(s);
+            free(qd);
+            return -1;
+        }
+        for (int i = 0; i < H; i++) {
+            const int h = i / G;
+            const size_t kv = (size_t)b * Hkv + h;
+            double *oo = o + ((size_t)b * H + i) * D;
+            double *aa = abso + ((size_t)b * H + i) * D;
+            for (int d = 0; d < D; d++)
+                oo[d] = aa[d] = 0.0;
+            if (L == 0) {
+                empty = 1;
+                continue;
+            }
+            for (int d = 0; d < D; d++)
+                qd[d] = oracle_half_to_double(q[((size_t)b * H + i) * D + d]);
+            /* scores */
+            double m = -INFINITY;
+            for (int t = 0; t < L; t++) {
+                const int8_t *kr = k_codes + (kv * Tmax + t) * D;
+                const uint16_t *ksr = k_scales + (kv * Tmax + t) * nb;
+                double acc = 0.0;
+                for (int d = 0; d < D; d++)
+                    acc += qd[d] * (oracle_half_to_double(ksr[d / ORACLE_BLOCK]) * (double)kr[d]);
+                s[t] = scale * acc;
+                if (s[t] > m)
+                    m = s[t];
+            }
+            /* softmax weights */
+            double l = 0.0;
+            for (int t = 0; t < L; t++) {
+                s[t] = exp(s[t] - m);
+                l += s[t];
+            }
+            /* o = sum_t p_t V[t] */
+            for (int t = 0; t < L; t++) {
+                const double p = s[t] / l;
+                const uint16_t *vsr = v_scales + (kv * Tmax + t) * nb;
+                for (int d = 0; d < D; d++) {
+                    const double v = oracle_half_to_double(vsr[d / ORACLE_BLOCK]) *
+                                     (double)vt_codes[(kv * D + d) * Tmax + t];
+                    oo[d] += p * v;
+                    aa[d] += p * fabs(v);
+                }
+            }
+        }
+    }
+    free(s);
+    free(qd);
+    return empty ? 2 : 0;
+}
