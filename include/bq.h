@@ -334,6 +334,44 @@ BQ_API int32_t bq_step_run_ex(const bq_step_info *info, const void *plan, void *
                               size_t ws_bytes, const bq_step_wait *wait, int32_t *dev_status,
                               void *stream);
 
+/* ---------------------------------------- batched verification GEMM --- */
+
+/* Bytes of workspace bq_verify_gemm needs (tile arrival counters + per-CTA
+ * partial sums).  0 on a bad shape. */
+BQ_API size_t bq_verify_workspace_bytes(int32_t N, int32_t K, int32_t B);
+
+/* Batched verification GEMM: y[b][n] = sum_k d(n,k/32) * (q(n,k) - z) * x[b][k]
+ * for a batch of B = 1..32 activation rows -- the step that checks a batch
+ * of drafted tokens in speculative decoding, which the pages name as the way
+ * past decode's bandwidth ceiling: its matrix products are compute-shaped
+ * and suit the tensor cores (romaanj.github.io review of the M5 follow-up
+ * paper, "Future work").  Same operation as the decode GEMV at a wider
+ * batch, on the 5th-generation tensor cores (tcgen05.mma, fp32 accumulators
+ * in tensor memory), one CTA per SM.
+ *   fmt      4 or 8 (the Q4 / Q8 planes of bq_gemv_q4 / bq_gemv_q8)
+ *   W        device planes, N x K, K a multiple of 32
+ *   x        device fp16 bits [B][K], 16-byte aligned
+ *   B        1..32 (else BQ_ERR_BATCH); the MMA's N is 16 for B <= 16 and
+ *            32 above (absent rows read as zero and are never stored)
+ *   y        device fp32 [B][N], overwritten
+ *   ws       device workspace >= bq_verify_workspace_bytes, zero-filled
+ *            before first use and left zero-filled by every call that
+ *            completes (calls of any shape may share one); not shared with
+ *            calls that may run at the same time
+ *   dev_status, stream as bq_gemv_q4 (a bounded wait that runs out sets the
+ *            bit 1 << BQ_ERR_TIMEOUT; the workspace must then be zero-filled
+ *            again)
+ * Rounding: each weight d (q - z) enters the tensor core rounded once to
+ * fp16 (times a per-row power of two that keeps every value in fp16's normal
+ * range, undone exactly afterwards): |y - y_exact| <= 2^-11 sum_k |w x| plus
+ * fp32 accumulation -- inside the decode tolerance 1e-3 sum_k |w x| + 1e-5,
+ * but not bit-identical to bq_gemv_q4 / _q8 (whose codes enter exactly).
+ * Deterministic for a given device and shape (split tiles are summed in a
+ * fixed order). */
+BQ_API int32_t bq_verify_gemm(int32_t fmt, const bq_qmat *W, const uint16_t *x, int32_t B,
+                              float *y, void *ws, size_t ws_bytes, int32_t *dev_status,
+                              void *stream);
+
 /* ------------------------------------------------------ routed experts --- */
 
 /* Bytes of workspace bq_moe_gemv_q4 needs.  0 on a bad shape. */

@@ -79,6 +79,8 @@ _SIGS = {
     "bq_step_run": (_i32, [_SIP, _vp, _vp, _sz, _vp, _vp]),
     "bq_step_run_ex": (_i32, [_SIP, _vp, _vp, _sz, ctypes.POINTER(bq_step_wait), _vp, _vp]),
     "bq_moe_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
+    "bq_verify_workspace_bytes": (_sz, [_i32, _i32, _i32]),
+    "bq_verify_gemm": (_i32, [_i32, _QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
     "bq_moe_gemv_q4": (_i32, [_QP, _i32, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _i32, _vp,
                               _vp, _sz, _vp, _vp]),
     "bq_moe_gemv_ex": (_i32, [_QP, _i32, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _i32,
@@ -238,6 +240,23 @@ def gemv(fmt: int, W: bq_qmat, x, y, ws, status=None, stream=None, epilogue: int
                           int(flags), ws.data_ptr(), ws.numel() * ws.element_size(), _ptr(status),
                           _stream_ptr(stream))
     check("bq_gemv_ex", rc)
+
+
+def verify_gemm(fmt: int, W: bq_qmat, x, y, ws, status=None, stream=None) -> None:
+    """y[B, N] (fp32) = deq(W) . x[B, K] (fp16) for a verification batch of
+    B = 1..32 rows, through bq_verify_gemm (Q4 or Q8; tensor cores)."""
+    _on_device("verify_gemm", x=x, y=y, ws=ws, status=status)
+    _check_planes("verify_gemm", fmt, W)
+    if x.dim() != 2 or x.shape[1] != W.K or x.element_size() != 2 or not x.is_contiguous():
+        raise ValueError(f"verify_gemm: x must be a contiguous [B, {W.K}] tensor of fp16 bits, got "
+                         f"{tuple(x.shape)} {x.dtype}")
+    B = x.shape[0]
+    if not y.is_contiguous() or _nbytes(y) < B * W.N * 4:
+        raise ValueError(f"verify_gemm: y must be contiguous with at least {B * W.N * 4} bytes")
+    check("bq_verify_gemm", lib().bq_verify_gemm(int(fmt), ctypes.byref(W), x.data_ptr(), B,
+                                                 y.data_ptr(), ws.data_ptr(),
+                                                 ws.numel() * ws.element_size(), _ptr(status),
+                                                 _stream_ptr(stream)))
 
 
 def moe_gemv_q4(Wstack: bq_qmat, E: int, codes_stride: int, scales_stride: int, x,

@@ -1,0 +1,781 @@
+// verify_gemm.cu -- the batched-verification GEMM over block-quantised
+// weights (Q4 / Q8, batch 1..32) on the 5th-generation tensor cores (sm_100a).
+//
+// The pages name speculative decoding as the way past the decode bandwidth
+// ceiling: the drafted tokens are checked in one batched verification step
+// whose matrix products are compute-shaped and suit the tensor-core path
+// (romaanj.github.io review of the M5 follow-up paper, "Future work").  Such a
+// step multiplies the same packed weights by a small batch of activation
+// vectors, B = 8..32: y[b][n] = sum_k deq(W)[n][k] x[b][k], with
+// deq(W) = d (q - z) per 32-weight block, the decode GEMV's operation at a
+// wider batch.  At B = 32 a Q4 weight carries 64 flop for 0.5625 bytes, so the
+// legacy mma.sync path of the decode GEMV (whose per-column tiles grow with B)
+// would be bound by its tensor pipe long before HBM; tcgen05.mma with the
+// batch as the MMA's N dimension does the whole batch in one instruction.
+//
+// Tile: 128 weight rows x all B columns, accumulated in tensor memory (TMEM:
+// 128 lanes = rows, NB = 16 or 32 fp32 columns = batch).  Work unit: one
+// tile x 256 weights of K.  Units are numbered tile-major (K fastest) and
+// split into one contiguous range per CTA (one CTA per SM, stream-K), so every
+// SM streams the same number of weight bytes; a tile whose units span several
+// CTAs is summed deterministically through the workspace (last arriver adds
+// the CTA partials in CTA order).
+//
+// Warp roles (16 warps):
+//   warp 0      TMA of the packed codes (128-byte swizzle) and the scales of a
+//               unit into a 3-slot (Q8: 2-slot) ring;
+//   warp 1      allocates TMEM, and one thread issues the MMAs: per 64-weight
+//               sub-stage, 4 x tcgen05.mma (M 128, N NB, K 16, fp16 inputs,
+//               fp32 accumulation) from shared-memory descriptors, then
+//               tcgen05.commit to free the sub-stage's slots;
+//   warp 2      TMA of the activations x (K-major, 128-byte swizzle: the
+//               layout the MMA's B descriptor reads, rows >= B zero-filled);
+//   warps 4-7   epilogue: tcgen05.ld of the accumulator, one thread per row;
+//   warps 8-15  dequantisation: one thread per (row, block) of a sub-stage
+//               turns 16 (Q8: 32) code bytes and the block's fp16 scale into
+//               32 fp16 weights d (q - z) 2^s and stores them into the MMA's A
+//               tile (K-major, 128-byte swizzle).
+//
+// Rounding.  The decode GEMV keeps codes exact and scales each block's sum;
+// a tile accumulated over many blocks cannot, so the A tile holds each weight
+// rounded once to fp16: relative error <= 2^-11, inside the decode tolerance
+// (1e-3 * sum |w x|).  To keep that bound for any scale, each row's values are
+// multiplied by a power of two 2^s chosen from the largest scale of the row in
+// the CTA's K range (the largest |d (q - z)| 2^s lies in [2^14, 2^15)), and
+// the epilogue multiplies by 2^-s: no overflow, and subnormal fp16 only for
+// blocks 2^28 times smaller than the row's largest.
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+
+#include "bq_device.cuh"
+#include "bq_internal.h"
+
+namespace bq {
+namespace vg {
+
+constexpr int kThreads = 512;
+constexpr int TM = 128;                 // rows per tile (MMA M)
+constexpr int kUnitK = 256;             // weights of K per unit
+constexpr int kSubK = 64;               // weights of K per sub-stage (one 128-byte swizzle row of fp16)
+constexpr int AS = 4;                   // A / x sub-stage slots
+constexpr int kShiftRing = 4;           // row shifts of the last 4 segments
+constexpr int kMaxCtas = 512;
+constexpr int kABytes = TM * kSubK * 2; // 16 KB
+constexpr int kScaleBytes = TM * 16;    // 8 fp16 per row per unit
+constexpr int kDequantWarp0 = 8;
+constexpr int kEpiWarp0 = 4;
+
+template <int FMT> struct VFmt;
+template <> struct VFmt<4> {
+    static constexpr int kCodeBytes = TM * 128;   // one 128 x 128-byte box
+    static constexpr int kCS = 3;
+};
+template <> struct VFmt<8> {
+    static constexpr int kCodeBytes = TM * 256;   // two 128 x 128-byte boxes
+    static constexpr int kCS = 2;
+};
+
+template <int FMT, int NB>
+constexpr size_t smem_bytes()
+{
+    return 1024 + (size_t)VFmt<FMT>::kCS * VFmt<FMT>::kCodeBytes + (size_t)AS * kABytes +
+           (size_t)AS * NB * 128 + (size_t)VFmt<FMT>::kCS * kScaleBytes + 1024;
+}
+
+// Per-tile partial sums through the workspace: [CTA][slot 0 / 1][TM][32] fp32.
+constexpr size_t kPartBytesPerCta = 2 * TM * 32 * sizeof(float);
+
+struct Args {
+    CUtensorMap tm_codes;    // Q4: (K/2, N) bytes; Q8: (K, N) bytes; box 128 x 128, SW128
+    CUtensorMap tm_scales;   // (K/32, N) u16, box 8 x 128
+    CUtensorMap tm_x;        // (K, B) f16, box 64 x NB, SW128
+    const uint16_t *scales;  // the scale plane (pre-pass reads it directly)
+    float *y;                // [B][N]
+    int N, K, B, ldS;
+    int ntiles, KU, U, G;    // tiles, units per tile, units, CTAs
+    int *counters;           // [ntiles], zero on entry and exit
+    float *partials;         // [G][2][TM][32]
+    int *status;
+};
+
+// ----------------------------------------------------------- tcgen05 ----
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (fp16 x fp16 -> fp32).
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive (once) on an mbarrier when every tcgen05 operation this thread
+// issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte
+// swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart (stride
+// dimension offset), start address 16-byte granular; descriptor version 1,
+// layout type 2 (SWIZZLE_128B).  The leading-dimension offset is unused by
+// swizzled K-major layouts (set to 1).
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// 32 lanes x N consecutive fp32 columns of TMEM into registers (this warp's
+// lane quarter).
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]);
+template <>
+__device__ __forceinline__ void tmem_ld<32>(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+        "%30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; i++)
+        v[i] = __uint_as_float(r[i]);
+}
+template <>
+__device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, float (&v)[16])
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; i++)
+        v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ uint32_t hadd2_u(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+// fp16 pairs: 0x6400 | byte is the fp16 value 1024 + byte, exactly.
+constexpr uint32_t kMagic = 0x64646464u;
+constexpr uint32_t kNeg1032 = 0xE408E408u;   // -1032 (Q4: 1024 + zero point 8)
+constexpr uint32_t kNeg72 = 0xD480D480u;     // -72   (Q4 high nibble: 64 + 8)
+constexpr uint32_t kSixteenth = 0x2C002C00u; // 1/16
+constexpr uint32_t kNeg1152 = 0xE480E480u;   // -1152 (Q8: 1024 + 128)
+
+// Q4: the 32 weights of one block (16 code bytes; byte i holds element i in
+// its low and element i + 16 in its high nibble) as fp16 (q - 8) * ds,
+// written to four 16-byte granules of the row (elements 0-7, 8-15, 16-23,
+// 24-31).  (1024 + nibble) - 1032 and (1024 + 16 nibble) / 16 - 72 are exact;
+// the product by ds is the one rounding.
+__device__ __forceinline__ void dequant_q4_block(uint4 c, uint32_t ds2, uint32_t row_addr, int g0,
+                                                 int rsw)
+{
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    uint32_t lo[8], hi[8];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const uint32_t p0 = prmt(w[i], kMagic, 0x4140);   // bytes 4i, 4i+1
+        const uint32_t p1 = prmt(w[i], kMagic, 0x4342);   // bytes 4i+2, 4i+3
+        lo[2 * i] = hmul2_u(hadd2_u(p0 & 0xFF0FFF0Fu, kNeg1032), ds2);
+        lo[2 * i + 1] = hmul2_u(hadd2_u(p1 & 0xFF0FFF0Fu, kNeg1032), ds2);
+        hi[2 * i] = hmul2_u(hfma2_u(p0 & 0xFFF0FFF0u, kSixteenth, kNeg72), ds2);
+        hi[2 * i + 1] = hmul2_u(hfma2_u(p1 & 0xFFF0FFF0u, kSixteenth, kNeg72), ds2);
+    }
+    sts128(row_addr + (((g0 + 0) ^ rsw) << 4), lo[0], lo[1], lo[2], lo[3]);
+    sts128(row_addr + (((g0 + 1) ^ rsw) << 4), lo[4], lo[5], lo[6], lo[7]);
+    sts128(row_addr + (((g0 + 2) ^ rsw) << 4), hi[0], hi[1], hi[2], hi[3]);
+    sts128(row_addr + (((g0 + 3) ^ rsw) << 4), hi[4], hi[5], hi[6], hi[7]);
+}
+
+// Q8: 16 signed code bytes (elements e .. e+15) as fp16 q * ds into two
+// granules: (byte ^ 0x80) = q + 128, (1024 + q + 128) - 1152 = q exactly.
+__device__ __forceinline__ void dequant_q8_half(uint4 c, uint32_t ds2, uint32_t row_addr, int g,
+                                                int rsw)
+{
+    const uint32_t w[4] = {c.x ^ 0x80808080u, c.y ^ 0x80808080u, c.z ^ 0x80808080u, c.w ^ 0x80808080u};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        o[2 * i] = hmul2_u(hadd2_u(prmt(w[i], kMagic, 0x4140), kNeg1152), ds2);
+        o[2 * i + 1] = hmul2_u(hadd2_u(prmt(w[i], kMagic, 0x4342), kNeg1152), ds2);
+    }
+    sts128(row_addr + (((g + 0) ^ rsw) << 4), o[0], o[1], o[2], o[3]);
+    sts128(row_addr + (((g + 1) ^ rsw) << 4), o[4], o[5], o[6], o[7]);
+}
+
+// The CTA owning unit x under the balanced split of U units over G CTAs
+// (CTA c owns [floor(c U / G), floor((c + 1) U / G))).
+__device__ __forceinline__ int owner_of(long long x, int U, int G)
+{
+    return (int)(((x + 1) * G - 1) / U);
+}
+
+template <int FMT, int NB>
+__global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_constant__ Args a)
+{
+    using VF = VFmt<FMT>;
+    constexpr int CS = VF::kCS;
+    constexpr int CB = VF::kCodeBytes;
+    constexpr int XB = NB * 128;   // x bytes per sub-stage
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ alignas(8) uint64_t bar_cfull[CS], bar_cempty[CS], bar_afull[AS], bar_aempty[AS],
+        bar_xfull[AS], bar_accfull[2], bar_accempty[2], bar_shift[kShiftRing],
+        bar_shift_free[kShiftRing], bar_done,
+        bar_epi_a, bar_epi_b;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int shift_s[kShiftRing][TM];
+    __shared__ int epi_old;
+    __shared__ int abort_s;
+
+    uint8_t *sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t codes_s = smem_u32(sbase);
+    const uint32_t a_s = codes_s + CS * CB;
+    const uint32_t x_s = a_s + AS * kABytes;
+    const uint32_t sc_s = x_s + AS * XB;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cta = blockIdx.x;
+    const int u0 = (int)((long long)cta * a.U / a.G), u1 = (int)((long long)(cta + 1) * a.U / a.G);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < CS; i++) {
+            mbar_init(smem_u32(&bar_cfull[i]), 1);
+            mbar_init(smem_u32(&bar_cempty[i]), 8);          // the 8 dequant warps
+        }
+        for (int i = 0; i < AS; i++) {
+            mbar_init(smem_u32(&bar_afull[i]), 8);           // the 8 dequant warps
+            mbar_init(smem_u32(&bar_aempty[i]), 1);          // tcgen05.commit
+            mbar_init(smem_u32(&bar_xfull[i]), 1);
+        }
+        for (int i = 0; i < 2; i++) {
+            mbar_init(smem_u32(&bar_accfull[i]), 1);         // tcgen05.commit
+            mbar_init(smem_u32(&bar_accempty[i]), 4);        // the 4 epilogue warps
+        }
+        for (int i = 0; i < kShiftRing; i++) {
+            mbar_init(smem_u32(&bar_shift[i]), 8);           // the 8 dequant warps
+            mbar_init(smem_u32(&bar_shift_free[i]), 4);      // the 4 epilogue warps
+        }
+        mbar_init(smem_u32(&bar_done), 1);
+        mbar_init(smem_u32(&bar_epi_a), 128);                // the epilogue's split-tile handshake
+        mbar_init(smem_u32(&bar_epi_b), 1);
+        abort_s = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&tmem_base_s), 2 * 32);          // two accumulators of up to 32 columns
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+    // Programmatic dependent launch: let the next kernel on the stream get
+    // scheduled, and touch no global memory before the previous one has
+    // completed.
+    pdl_launch_dependents();
+    pdl_wait();
+
+    // Failure path: a bounded wait ran out -- report, and make every role stop.
+    auto fail = [&]() {
+        if (a.status)
+            atomicOr(a.status, kStatusTimeout);
+        *(volatile int *)&abort_s = 1;
+    };
+    auto aborted = [&]() { return *(volatile int *)&abort_s != 0; };
+    auto wait = [&](uint64_t &bar, uint32_t parity) -> bool {
+        if (mbar_wait_bounded(smem_u32(&bar), parity))
+            return true;
+        fail();
+        return false;
+    };
+    // Sub-stages of unit u (the last unit of a row may be short).
+    auto nsub = [&](int u) {
+        const int ku = u % a.KU;
+        return min(kUnitK / kSubK, (a.K - ku * kUnitK + kSubK - 1) / kSubK);
+    };
+
+    if (warp == 0) {
+        // ---------------------------------------------- codes + scales TMA --
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            int n = 0;
+            for (int u = u0; u < u1 && !aborted(); u++, n++) {
+                const int slot = n % CS;
+                if (!wait(bar_cempty[slot], ((n / CS) & 1) ^ 1))
+                    break;
+                const int tile = u / a.KU, ku = u % a.KU;
+                const uint32_t bar = smem_u32(&bar_cfull[slot]);
+                mbar_arrive_expect_tx(bar, CB + kScaleBytes);
+                if constexpr (FMT == 4) {
+                    tma_load_2d(codes_s + slot * CB, &a.tm_codes, bar, ku * 128, tile * TM, pol);
+                } else {
+                    tma_load_2d(codes_s + slot * CB, &a.tm_codes, bar, ku * 256, tile * TM, pol);
+                    tma_load_2d(codes_s + slot * CB + TM * 128, &a.tm_codes, bar, ku * 256 + 128,
+                                tile * TM, pol);
+                }
+                tma_load_2d(sc_s + slot * kScaleBytes, &a.tm_scales, bar, ku * 8, tile * TM, pol);
+            }
+            // Drain: every load issued lands before the CTA may exit.
+            for (int j = max(0, n - CS); j < n; j++)
+                (void)mbar_wait_bounded(smem_u32(&bar_cfull[j % CS]), (j / CS) & 1);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------- x TMA ----
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_normal();
+            int i = 0;
+            for (int u = u0; u < u1 && !aborted(); u++) {
+                const int ku = u % a.KU, ns = nsub(u);
+                bool ok = true;
+                for (int j = 0; j < ns; j++, i++) {
+                    const int slot = i % AS;
+                    if (!wait(bar_aempty[slot], ((i / AS) & 1) ^ 1)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bar = smem_u32(&bar_xfull[slot]);
+                    mbar_arrive_expect_tx(bar, XB);
+                    tma_load_2d(x_s + slot * XB, &a.tm_x, bar, ku * kUnitK + j * kSubK, 0, pol);
+                }
+                if (!ok)
+                    break;
+            }
+            for (int j = max(0, i - AS); j < i; j++)
+                (void)mbar_wait_bounded(smem_u32(&bar_xfull[j % AS]), (j / AS) & 1);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA ----
+        if (lane == 0) {
+            constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(NB >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
+            int i = 0, seg = 0;
+            int u = u0;
+            bool ok = true;
+            while (u < u1 && ok) {
+                const int tile = u / a.KU;
+                const int uend = min(u1, (tile + 1) * a.KU);
+                const int buf = seg & 1;
+                if (!wait(bar_accempty[buf], ((seg >> 1) & 1) ^ 1))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(buf * 32);
+                bool first = true;
+                for (; u < uend && ok; u++) {
+                    const int ns = nsub(u);
+                    for (int j = 0; j < ns; j++, i++) {
+                        const int slot = i % AS;
+                        if (!wait(bar_afull[slot], (i / AS) & 1) || !wait(bar_xfull[slot], (i / AS) & 1)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t ad = desc_k_sw128(a_s + slot * kABytes);
+                        const uint64_t bd = desc_k_sw128(x_s + slot * XB);
+#pragma unroll
+                        for (int kk = 0; kk < kSubK / 16; kk++) {
+                            // K step of 16 fp16 = 32 bytes along the swizzled row
+                            umma_f16(d_tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
+                                     (first && kk == 0) ? 0u : 1u);
+                        }
+                        first = false;
+                        umma_commit(smem_u32(&bar_aempty[slot]));
+                    }
+                }
+                if (!ok)
+                    break;
+                umma_commit(smem_u32(&bar_accfull[buf]));
+                seg++;
+            }
+            // Every MMA issued has completed before TMEM is freed.
+            umma_commit(smem_u32(&bar_done));
+            (void)mbar_wait_bounded(smem_u32(&bar_done), 0);
+        }
+    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+        // ----------------------------------------------------- epilogue ----
+        // (Warp w reads TMEM lanes 32 (w % 4) .. + 31: warps 4-7 cover all.)
+        // Every cross-warp step here is an mbarrier with a bounded wait, so a
+        // role that gave up on a timeout cannot leave the others blocked.
+        const int q = warp - kEpiWarp0;          // TMEM lanes 32q .. 32q + 31
+        const int r = 32 * q + lane;             // row within the tile
+        int seg = 0, nsplit = 0;
+        for (int u = u0; u < u1; seg++) {
+            const int tile = u / a.KU;
+            u = min(u1, (tile + 1) * a.KU);
+            const int buf = seg & 1;
+            if (!wait(bar_shift[seg % kShiftRing], (seg / kShiftRing) & 1))
+                break;
+            const int sh = shift_s[seg % kShiftRing][r];
+            __syncwarp();
+            if (lane == 0)                                 // the slot may take a later segment's shifts
+                mbar_arrive(smem_u32(&bar_shift_free[seg % kShiftRing]));
+            if (!wait(bar_accfull[buf], (seg >> 1) & 1))
+                break;
+            tc_fence_after();
+            float v[NB];
+            tmem_ld<NB>(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * 32), v);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&bar_accempty[buf]));
+            // undo the row's power-of-two prescale (exact)
+            const float unsc = __int_as_float((127 - sh) << 23);
+#pragma unroll
+            for (int b = 0; b < NB; b++)
+                v[b] *= unsc;
+            const int row = tile * TM + r;
+            const long long tu0 = (long long)tile * a.KU;
+            const int cf = owner_of(tu0, a.U, a.G), cl = owner_of(tu0 + a.KU - 1, a.U, a.G);
+            if (cf == cl) {
+                if (row < a.N) {
+#pragma unroll
+                    for (int b = 0; b < NB; b++)
+                        if (b < a.B)
+                            a.y[(size_t)b * a.N + row] = v[b];
+                }
+                continue;
+            }
+            // Tile split across CTAs: this CTA's partial to its slot (0: the
+            // tile of its first unit, 1: of its last), a counted arrival; the
+            // last CTA adds all partials in CTA order and resets the counter.
+            const int my_slot = (tile == u0 / a.KU) ? 0 : 1;
+            float4 *dst = reinterpret_cast<float4 *>(a.partials + (((size_t)cta * 2 + my_slot) * TM + r) * 32);
+#pragma unroll
+            for (int b4 = 0; b4 < NB / 4; b4++)
+                __stcg(dst + b4, make_float4(v[4 * b4], v[4 * b4 + 1], v[4 * b4 + 2], v[4 * b4 + 3]));
+            __threadfence();
+            mbar_arrive(smem_u32(&bar_epi_a));
+            if (r == 0) {
+                if (!wait(bar_epi_a, nsplit & 1))
+                    break;
+                epi_old = atom_add_acq_rel_gpu(a.counters + tile, 1);
+                mbar_arrive(smem_u32(&bar_epi_b));
+            }
+            if (!wait(bar_epi_b, nsplit & 1))
+                break;
+            nsplit++;
+            if (epi_old != cl - cf)
+                continue;
+            __threadfence();
+#pragma unroll
+            for (int b = 0; b < NB; b++)
+                v[b] = 0.f;
+            for (int c = cf; c <= cl; c++) {
+                const int cu0 = (int)((long long)c * a.U / a.G);
+                const int sl = (tile == cu0 / a.KU) ? 0 : 1;
+                float4 *src = reinterpret_cast<float4 *>(a.partials + (((size_t)c * 2 + sl) * TM + r) * 32);
+#pragma unroll
+                for (int b4 = 0; b4 < NB / 4; b4++) {
+                    const float4 p = __ldcg(src + b4);
+                    // cleared once read: the workspace is all-zero again when
+                    // the call ends, so calls of any shape may share it
+                    __stcg(src + b4, make_float4(0.f, 0.f, 0.f, 0.f));
+                    v[4 * b4] += p.x;
+                    v[4 * b4 + 1] += p.y;
+                    v[4 * b4 + 2] += p.z;
+                    v[4 * b4 + 3] += p.w;
+                }
+            }
+            if (row < a.N) {
+#pragma unroll
+                for (int b = 0; b < NB; b++)
+                    if (b < a.B)
+                        a.y[(size_t)b * a.N + row] = v[b];
+            }
+            if (r == 0)
+                a.counters[tile] = 0;
+        }
+    } else if (warp >= kDequantWarp0) {
+        // ------------------------------------------------ dequantisation ----
+        // Thread pair (2r, 2r+1) of a warp serves row r: block h = t & 1 of
+        // each 64-weight sub-stage.  Both halves of a row sit in one warp, so
+        // the row's scale maximum is one shuffle (no CTA barrier).
+        const int t = threadIdx.x - kDequantWarp0 * 32;   // 0 .. 255
+        const int r = t >> 1, h = t & 1;                   // row, block of the sub-stage
+        const int rsw = r & 7;                             // the 128-byte swizzle's XOR
+        int i = 0, n = 0, seg = 0;
+        bool ok = true;
+        for (int u = u0; u < u1 && ok; seg++) {
+            const int tile = u / a.KU;
+            const int uend = min(u1, (tile + 1) * a.KU);
+            const int row = tile * TM + r;
+            // Row shift for this segment: the largest scale of the row over
+            // the segment's units (the bytes the ring is about to bring in;
+            // read here directly, 16 bytes a unit).
+            unsigned m = 0;
+            if (row < a.N) {
+                const uint16_t *srow = a.scales + (size_t)row * a.ldS;
+                for (int uu = u + h; uu < uend; uu += 2) {
+                    const uint4 s8 = __ldg(reinterpret_cast<const uint4 *>(srow + (size_t)(uu % a.KU) * 8));
+                    const uint32_t sv[4] = {s8.x, s8.y, s8.z, s8.w};
+#pragma unroll
+                    for (int k = 0; k < 4; k++)
+                        m = max(m, max(sv[k] & 0x7FFFu, (sv[k] >> 16) & 0x7FFFu));
+                }
+            }
+            m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = min(m, 0x7BFFu);                               // largest finite fp16
+            int s = 0;
+            {
+                // the largest |d (q - z)| (8 dmax for Q4, 127 dmax for Q8)
+                // times 2^s lands in [2^14, 2^15)
+                const float dmax = __half2float(__ushort_as_half((unsigned short)m));
+                const float top = dmax * (FMT == 4 ? 8.0f : 127.0f);
+                if (top > 0.f)
+                    s = 141 - ((__float_as_int(top) >> 23) & 0xFF);
+            }
+            // (the slot's previous segment, seg - 4, must have been read)
+            if (!wait(bar_shift_free[seg % kShiftRing], ((seg / kShiftRing) & 1) ^ 1))
+                break;
+            if (h == 0)
+                shift_s[seg % kShiftRing][r] = s;
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&bar_shift[seg % kShiftRing]));
+            const float two_s = __int_as_float((127 + s) << 23);
+            for (; u < uend && ok; u++, n++) {
+                const int cslot = n % CS;
+                if (!wait(bar_cfull[cslot], (n / CS) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t crow = codes_s + cslot * CB + r * 128;
+                const uint32_t srow_s = sc_s + cslot * kScaleBytes + r * 16;
+                const int ns = nsub(u);
+                for (int j = 0; j < ns; j++, i++) {
+                    const int slot = i % AS;
+                    if (!wait(bar_aempty[slot], ((i / AS) & 1) ^ 1)) {
+                        ok = false;
+                        break;
+                    }
+                    const int blk = 2 * j + h;                        // block of the unit (0..7)
+                    unsigned short dbits;
+                    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(dbits) : "r"(srow_s + 2 * blk));
+                    const float ds = __half2float(__ushort_as_half(dbits)) * two_s;
+                    const __half2 ds2h = __float2half2_rn(ds);
+                    uint32_t ds2;
+                    memcpy(&ds2, &ds2h, 4);
+                    const uint32_t arow = a_s + slot * kABytes + r * 128;
+                    if constexpr (FMT == 4) {
+                        const uint4 c = lds128_u32(crow + ((blk ^ rsw) << 4));
+                        dequant_q4_block(c, ds2, arow, 4 * h, rsw);
+                    } else {
+                        const uint32_t box = crow + (blk >> 2) * (TM * 128);
+                        const int g = 2 * (blk & 3);
+                        const uint4 c0 = lds128_u32(box + ((g ^ rsw) << 4));
+                        const uint4 c1 = lds128_u32(box + (((g + 1) ^ rsw) << 4));
+                        dequant_q8_half(c0, ds2, arow, 4 * h, rsw);
+                        dequant_q8_half(c1, ds2, arow, 4 * h + 2, rsw);
+                    }
+                    fence_proxy_async_smem();     // generic-proxy stores -> the MMA's async-proxy reads
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(smem_u32(&bar_afull[slot]));
+                }
+                if (!ok)
+                    break;
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(smem_u32(&bar_cempty[cslot]));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        tmem_dealloc(tmem, 2 * 32);
+}
+
+}  // namespace vg
+
+namespace {
+
+template <int FMT, int NB>
+int32_t verify_prepare()
+{
+    static std::atomic<bool> done[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire))
+        return BQ_OK;
+    if (cudaFuncSetAttribute((const void *)vg::verify_gemm_kernel<FMT, NB>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)vg::smem_bytes<FMT, NB>()) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    if (dev >= 0 && dev < 64)
+        done[dev].store(true, std::memory_order_release);
+    return BQ_OK;
+}
+
+struct VGeometry {
+    int ntiles, KU, U, G;
+};
+
+VGeometry verify_geometry(long long N, long long K, int sms)
+{
+    VGeometry g;
+    g.ntiles = (int)((N + vg::TM - 1) / vg::TM);
+    g.KU = (int)((K + vg::kUnitK - 1) / vg::kUnitK);
+    g.U = g.ntiles * g.KU;
+    g.G = std::min(std::min(sms, vg::kMaxCtas), g.U);
+    return g;
+}
+
+template <int FMT, int NB>
+int32_t verify_launch(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, void *ws,
+                      int32_t *dev_status, void *stream, const VGeometry &geo)
+{
+    int32_t st = verify_prepare<FMT, NB>();
+    if (st != BQ_OK)
+        return st;
+    vg::Args a;
+    memset(&a, 0, sizeof(a));
+    const int N = W->N, K = W->K;
+    const uint64_t cdims[2] = {(uint64_t)(FMT == 4 ? K / 2 : K), (uint64_t)N};
+    const uint64_t cstr[1] = {(uint64_t)(FMT == 4 ? K / 2 : K)};
+    const uint32_t cbox[2] = {128u, (uint32_t)vg::TM};
+    const int ldS = bq_scales_ld(K);
+    const uint64_t sdims[2] = {(uint64_t)(K / 32), (uint64_t)N};
+    const uint64_t sstr[1] = {(uint64_t)ldS * 2};
+    const uint32_t sbox[2] = {8u, (uint32_t)vg::TM};
+    const uint64_t xdims[2] = {(uint64_t)K, (uint64_t)B};
+    const uint64_t xstr[1] = {(uint64_t)K * 2};
+    const uint32_t xbox[2] = {(uint32_t)vg::kSubK, (uint32_t)NB};
+    if (!encode_tensor_map(&a.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, cdims, cstr, cbox,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
+        !encode_tensor_map(&a.tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, W->scales, sdims, sstr,
+                           sbox, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
+        !encode_tensor_map(&a.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, xdims, xstr, xbox,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
+        return BQ_ERR_CUDA;
+    a.scales = W->scales;
+    a.y = y;
+    a.N = N;
+    a.K = K;
+    a.B = B;
+    a.ldS = ldS;
+    a.ntiles = geo.ntiles;
+    a.KU = geo.KU;
+    a.U = geo.U;
+    a.G = geo.G;
+    a.counters = static_cast<int *>(ws);
+    a.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) +
+                                           align_up((size_t)geo.ntiles * sizeof(int), 256));
+    a.status = dev_status;
+    void *args[] = {&a};
+    cudaError_t e = launch_pdl((const void *)vg::verify_gemm_kernel<FMT, NB>, dim3(geo.G),
+                               dim3(vg::kThreads), vg::smem_bytes<FMT, NB>(),
+                               static_cast<cudaStream_t>(stream), args);
+    return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace bq
+
+using namespace bq;
+
+extern "C" size_t bq_verify_workspace_bytes(int32_t N, int32_t K, int32_t B)
+{
+    if (N < 1 || K < 32 || K % 32 != 0 || B < 1 || B > 32)
+        return 0;
+    const long long ntiles = ((long long)N + vg::TM - 1) / vg::TM;
+    return align_up((size_t)ntiles * sizeof(int), 256) + (size_t)vg::kMaxCtas * vg::kPartBytesPerCta;
+}
+
+extern "C" int32_t bq_verify_gemm(int32_t fmt, const bq_qmat *W, const uint16_t *x, int32_t B,
+                                  float *y, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                  void *stream)
+{
+    int32_t st = check_qmat(W);
+    if (st != BQ_OK)
+        return st;
+    if (fmt != 4 && fmt != 8)
+        return BQ_ERR_SHAPE;
+    if (!x || !y || !ws)
+        return BQ_ERR_NULL;
+    if (B < 1 || B > 32)
+        return BQ_ERR_BATCH;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(ws))
+        return BQ_ERR_ALIGN;
+    if (ws_bytes < bq_verify_workspace_bytes(W->N, W->K, B))
+        return BQ_ERR_WORKSPACE;
+    const int sms = device_sm_count();
+    if (sms <= 0)
+        return BQ_ERR_CUDA;
+    const VGeometry geo = verify_geometry(W->N, W->K, sms);
+    if ((long long)geo.ntiles * geo.KU >= (1LL << 31) / 2)
+        return BQ_ERR_SHAPE;
+    if (fmt == 4)
+        return B <= 16 ? verify_launch<4, 16>(W, x, B, y, ws, dev_status, stream, geo)
+                       : verify_launch<4, 32>(W, x, B, y, ws, dev_status, stream, geo);
+    return B <= 16 ? verify_launch<8, 16>(W, x, B, y, ws, dev_status, stream, geo)
+                   : verify_launch<8, 32>(W, x, B, y, ws, dev_status, stream, geo);
+}
