@@ -79,7 +79,8 @@ def load_peaks():
     try:
         with open(p) as f:
             d = json.load(f)
-        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d.get("bf16_tflops", 0)) or None,
+                "source": "measured"}
     except Exception:
         return dict(PEAKS_FALLBACK)
 
@@ -97,6 +98,15 @@ WORKLOADS = {
 for _b in (1, 8):
     _w = synth.moe_h2048(_b)
     WORKLOADS[_w.name] = _w
+for _w in (synth.attn_h5120(1, 4096), synth.attn_h5120(8, 4096), synth.attn_h5120(1, 32768),
+           synth.attn_h2048(8, 8192)):
+    WORKLOADS[_w.name] = _w
+for _f in (4, 8):
+    for _b in (16, 32):
+        for _w in (synth.verify_h4096(_f, _b),
+                   synth.verify_sweep_workload(_f, 24576, 4096, _b),
+                   synth.verify_sweep_workload(_f, 4096, 12288, _b)):
+            WORKLOADS[_w.name] = _w
 for _f in (2, 3, 4, 5, 6, 8):
     for _b in (1, 2, 4, 8):
         _w = synth.dense_h4096(_f, _b)
@@ -247,6 +257,7 @@ class DenseStep:
     def __init__(self, wl: synth.DenseWorkload, device, seed: int = 0, ffn: bool = True):
         import torch
         from quantised_weight_gemv_b200 import bq
+        ffn = ffn and not wl.verify      # a verification step: every matrix has its own x
         self.wl, self.device, self.bq = wl, device, bq
         self.B = wl.B
         self.fmt = wl.fmt
@@ -315,7 +326,8 @@ class DenseStep:
                 self.bytes_alg += nb
                 label = "+".join(names)
                 self.bytes_by_label[label] = self.bytes_by_label.get(label, 0) + nb
-                ws_max = max(ws_max, bq.lib().bq_gemv_workspace_bytes(Ntot, K))
+                ws_max = max(ws_max, bq.lib().bq_verify_workspace_bytes(Ntot, K, self.B)
+                             if wl.verify else bq.lib().bq_gemv_workspace_bytes(Ntot, K))
 
         # Every seeded x in one device buffer and every fp32 y in another
         # (64-byte aligned slices), so a step's inputs and results each move in
@@ -373,6 +385,13 @@ class DenseStep:
     def launch_one(self, entry, stream):
         import ctypes
         q, x, y, label, _, epi = entry
+        if self.wl.verify:
+            rc = self.bq.lib().bq_verify_gemm(self.fmt, ctypes.byref(q), x.data_ptr(), self.B,
+                                              y.data_ptr(), self.ws.data_ptr(), self.ws.numel(),
+                                              self.status.data_ptr(), stream.cuda_stream)
+            if rc != 0:
+                raise RuntimeError(f"bq_verify_gemm: {self.bq.bq_status_string(rc)}")
+            return
         # the step's weights are resident and never written: each launch may
         # start loading them while the previous one drains
         rc = self.bq.lib().bq_gemv_ex(self.fmt, ctypes.byref(q), x.data_ptr(), self.B, y.data_ptr(),
@@ -500,6 +519,76 @@ class MoEStep:
         return self.x_all, self.y_all
 
 
+class AttnStep:
+    """Decode attention of every layer over a Q8 KV cache resident in HBM:
+    per layer the keys (position-major) and values (transposed) of every
+    (sequence, KV head), Tmax positions each, quantised on the device from
+    seeded N(0, 1) values, plus the layer's queries.  One step = one
+    bq_attn_decode_q8 call per layer.  Algorithmic bytes: the cache bytes of
+    the valid positions (codes + scales of keys and values) + q + o."""
+
+    def __init__(self, wl: synth.AttnWorkload, device, seed: int = 0):
+        import torch
+        from quantised_weight_gemv_b200 import bq
+        self.wl, self.device, self.bq = wl, device, bq
+        self.B, self.fmt = wl.B, 8
+        B, Hkv, G, T, D = wl.B, wl.Hkv, wl.G, wl.Tmax, wl.D
+        rows = B * Hkv * T
+        st = torch.zeros(1, dtype=torch.int32, device=device)
+        lens = wl.lens(seed)
+        self.lens_host = lens
+        self.layers, self._keep = [], []
+        qs = []
+        for layer in range(wl.layers):
+            planes = []
+            for kind in (synth.KIND_KEY, synth.KIND_VAL):
+                g = torch.Generator(device=device)
+                g.manual_seed(synth.torch_seed(synth.key(seed, wl.wid, layer, 0, kind)))
+                f = torch.randn((rows, D), generator=g, dtype=torch.float32, device=device)
+                codes = torch.empty((rows, D), dtype=torch.uint8, device=device)
+                sc = torch.empty((rows, bq.scales_ld(D)), dtype=torch.int16, device=device)
+                bq.quantize_dev(8, f, codes, sc, st)
+                del f
+                sc4 = sc[:, :D // 32].contiguous().view(B, Hkv, T, D // 32)
+                c4 = codes.view(B, Hkv, T, D)
+                if kind == synth.KIND_VAL:
+                    c4 = c4.transpose(2, 3).contiguous()          # [B, Hkv, D, T]
+                planes += [c4, sc4]
+            kv = bq.kv_cache(*planes)
+            self._keep += planes
+            q = synth.activations_f16_torch(synth.key(seed, wl.wid, layer, 0, synth.KIND_X),
+                                            (B, Hkv * G, D), device)
+            qs.append(q)
+            self.layers.append(kv)
+        torch.cuda.synchronize()
+        if int(st.item()) != 0:
+            raise RuntimeError(f"device quantiser status {int(st.item()):#x}")
+        # every query of the step in one buffer, every output in another
+        qn = B * Hkv * G * D
+        self.x_all = torch.empty((wl.layers, qn), dtype=torch.float16, device=device)
+        for li, q in enumerate(qs):
+            self.x_all[li].copy_(q.view(-1))
+        self.y_all = torch.zeros((wl.layers, B, Hkv * G, D), dtype=torch.float32, device=device)
+        self.lens = torch.as_tensor(lens, device=device)
+        self.ws = bq.workspace(bq.lib().bq_attn_workspace_bytes(B, Hkv), device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        L = int(sum(min(max(int(v), 0), T) for v in lens))       # valid positions of a layer
+        self.bytes_alg = wl.layers * (L * Hkv * 2 * (D + 2 * (D // 32)) + qn * 2 + qn * 4)
+        self.launches_per_step = wl.layers
+        self.scale = 1.0 / math.sqrt(D)
+
+    def launch(self, stream, only=None):
+        wl = self.wl
+        for li, kv in enumerate(self.layers):
+            q = self.x_all[li].view(wl.B, wl.Hkv * wl.G, wl.D)
+            self.bq.attn_decode_q8(kv, q, self.lens, wl.G, self.scale, self.y_all[li], self.ws,
+                                   self.status, stream)
+        return self.launches_per_step
+
+    def io_tensors(self):
+        return self.x_all, self.y_all
+
+
 # ---------------------------------------------------------- CPU oracle ----
 _SAMPLES = {}
 
@@ -559,6 +648,35 @@ def moe_oracle_sample(wl: synth.MoEWorkload, seed: int = 0):
     return jobs, nbytes
 
 
+def attn_oracle_job(wl, seed: int = 0):
+    """Layer 0 of an attention workload for the oracle: the same seeded keys,
+    values (quantised by the oracle's Q8 quantiser), queries and lengths.
+    (The oracle's attention is single-threaded.)"""
+    import numpy as np
+    import oracle
+    if ("attn", wl.name, seed) not in _SAMPLES:
+        B, Hkv, G, T, D = wl.B, wl.Hkv, wl.G, wl.Tmax, wl.D
+        rows = B * Hkv * T
+        planes = []
+        for kind in (synth.KIND_KEY, synth.KIND_VAL):
+            f = synth.kv_values_f32(synth.key(seed, wl.wid, 0, 0, kind), rows, D)
+            c, sc = oracle.quantize_q8(f)
+            c = c.reshape(B, Hkv, T, D)
+            if kind == synth.KIND_VAL:
+                c = np.ascontiguousarray(c.transpose(0, 1, 3, 2))
+            planes += [c, np.ascontiguousarray(sc[:, :D // 32]).reshape(B, Hkv, T, D // 32)]
+        q = synth.activations_f16_bits(synth.key(seed, wl.wid, 0, 0, synth.KIND_X), B, Hkv * G, D)
+        _SAMPLES[("attn", wl.name, seed)] = (planes, q, wl.lens(seed))
+    planes, q, lens = _SAMPLES[("attn", wl.name, seed)]
+    L = int(sum(min(max(int(v), 0), wl.Tmax) for v in lens))
+    qn = wl.B * wl.Hkv * wl.G * wl.D
+    nbytes = L * wl.Hkv * 2 * (wl.D + 2 * (wl.D // 32)) + qn * 2 + qn * 4
+
+    def run():
+        oracle.attn_decode_q8(*planes, q, lens, 1.0 / math.sqrt(wl.D))
+    return run, nbytes
+
+
 def oracle_job(wl, frac: float = 1.0, threads: int | None = None):
     """(run-once callable, algorithmic bytes) for the CPU oracle: layer 0 of the
     workload, or (dense workloads, frac < 1) a frac share of every matrix's rows
@@ -566,6 +684,8 @@ def oracle_job(wl, frac: float = 1.0, threads: int | None = None):
     calls cycle through."""
     import oracle
     threads = threads or os.cpu_count() or 1
+    if isinstance(wl, synth.AttnWorkload):
+        return attn_oracle_job(wl)
     if isinstance(wl, synth.MoEWorkload):
         jobs, nbytes = moe_oracle_sample(wl)
 
@@ -623,7 +743,7 @@ def cpu_baseline(wl, budget_s=10.0):
         frac = 1.0
         run, nbytes = oracle_job(wl, threads=threads)
         t1 = time_once(run)
-        if t1 > budget_s and not isinstance(wl, synth.MoEWorkload):
+        if t1 > budget_s and not isinstance(wl, (synth.MoEWorkload, synth.AttnWorkload)):
             frac = max(budget_s / (2 * t1), 1.0 / 256)
             run, nbytes = oracle_job(wl, frac, threads=threads)
         reps, total = 0, 0.0
@@ -653,7 +773,7 @@ def run_reference(args, wl, rank):
     t_layer = time_once(run)                       # a calibration pass (untimed)
     frac, sample = 1.0, f"layer 0 of {wl.layers} per step ({nbytes/1e6:.1f} MB)"
     budget = (args.steps + args.warmup) * t_layer
-    if budget > args.ref_budget_s and not isinstance(wl, synth.MoEWorkload):
+    if budget > args.ref_budget_s and not isinstance(wl, (synth.MoEWorkload, synth.AttnWorkload)):
         frac = max(args.ref_budget_s / budget, 1.0 / 256)
         run, nbytes = oracle_job(wl, frac)
         sample = (f"{frac:.4f} of the rows of every matrix of layer 0 of {wl.layers} per step "
@@ -744,14 +864,19 @@ def main():
             dist.barrier()
 
     is_moe = isinstance(wl, synth.MoEWorkload)
-    if is_moe:
+    is_attn = isinstance(wl, synth.AttnWorkload)
+    if is_attn:
+        args.engine = "graph"   # one graph of the per-layer attention calls
+        step = AttnStep(wl, device)
+    elif is_moe:
         args.engine = "graph"   # one graph of the per-layer expert calls
         step = MoEStep(wl, device)
     else:
-        if args.engine is None:
+        if args.engine is None or wl.verify:
             # the chain of per-matrix launches with static weights: each launch
             # starts loading its weights while the previous one drains, which
-            # measured faster than the one-launch plan's grid barriers
+            # measured faster than the one-launch plan's grid barriers (a
+            # verification step has no plan form)
             args.engine = "graph"
         step = DenseStep(wl, device)
     stream = torch.cuda.Stream(device)
@@ -820,7 +945,12 @@ def main():
         raise RuntimeError(f"device status {int(step.status.item()):#x}")
 
     isolated = None
-    if args.engine == "step" or is_moe:
+    if is_attn:
+        # every launch is the attention kernel: its average launch
+        dom = f"average of the {n_launch} per-layer launches of a step"
+        dom_s = t_dev / args.steps / n_launch
+        dom_bytes = step.bytes_alg / n_launch
+    elif args.engine == "step" or is_moe:
         # the step kernel is the only kernel (one launch per step), or (routed
         # experts) the expert kernel is every launch but the small combine
         # kernels: timed over the timed region itself
@@ -855,6 +985,16 @@ def main():
         isolated = {"launch": big, "us": round(big_s * 1e6, 3),
                     "GB/s": round(step.bytes_by_label[big] / n_big / big_s / 1e9, 1)}
     achieved = dom_bytes / dom_s / 1e9
+    # the verification GEMM's tensor-core rate beside its HBM rate (2 B N K
+    # flop a matrix; the dense f16 peak equals the measured bf16 one)
+    verify = not is_moe and not is_attn and wl.verify
+    tensor = None
+    if verify:
+        flops = 2.0 * wl.B * wl.layers * wl.layer_weights()
+        tf = flops / (t_dev / args.steps) / 1e12
+        tensor = {"achieved_tflops": round(tf, 1), "peak_tflops": peaks.get("bf16_tflops"),
+                  "peak_source": "measured bf16 dense (f16 runs at the same rate)",
+                  "frac": round(tf / peaks["bf16_tflops"], 4) if peaks.get("bf16_tflops") else None}
 
     # end to end: pinned host x -> device, step, y -> pinned host, every step
     # (one copy each way: every x of the step lives in one buffer, every y in
@@ -906,14 +1046,20 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f16",
-            "arith": (f"q{step.fmt} codes as exact f16 subnormal mma operands, f16 x, "
+            "arith": ("q8 KV codes as exact f16 subnormal mma operands, f16 q, f32 scores and "
+                      "online softmax, p*dV*2^s rounded once to f16" if is_attn else
+                      f"q{step.fmt} weights as f16 d(q-z)2^s (one rounding) in tcgen05 mma, f16 x, "
+                      "f32 accumulation in tensor memory" if verify else
+                      f"q{step.fmt} codes as exact f16 subnormal mma operands, f16 x, "
                       "f32 accumulation and scaling"),
             "data": "synthetic (seeded N(0,0.02) weights, N(0,1) fp16 activations)",
             "config": {"workload": wl.name, "batch": wl.B, "layers": wl.layers,
                        "launches_per_step": n_launch, "bytes_per_step": step.bytes_alg,
-                       "engine": ("cuda-graph of per-layer bq_moe_gemv_ex calls" if is_moe else
+                       "engine": ("cuda-graph of per-layer bq_attn_decode_q8 calls" if is_attn else
+                                  "cuda-graph of per-layer bq_moe_gemv_ex calls" if is_moe else
                                   "one cooperative launch per step (bq_step_run), graph-captured"
                                   if args.engine == "step" else
+                                  "cuda-graph of per-matrix bq_verify_gemm launches" if verify else
                                   "cuda-graph of per-matrix bq_gemv_ex launches, static weights"),
                        "l2": ("inputs larger than L2 (no flush)" if flush is None else
                               f"L2 flushed before every step ({L2_FLUSH_BYTES >> 20} MB write, untimed); "
@@ -924,7 +1070,10 @@ def main():
                if is_moe else {}),
             "frac_of_measured_hbm": round(value / world / peaks["hbm_gbs"], 4),
             "frac_of_8TBps": round(value / world / 8000.0, 4),
-            "roofline": {"bound": "hbm", "kernel": f"stream_gemv q{step.fmt} ({dom})",
+            "roofline": {"bound": "hbm",
+                         "kernel": (f"attn_decode q8 KV ({dom})" if is_attn else
+                                    f"verify_gemm q{step.fmt} ({dom})" if verify else
+                                    f"stream_gemv q{step.fmt} ({dom})"),
                          "timed": "CUDA events over the timed region",
                          "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                          "peak_source": peaks["source"], "unit": "GB/s",
@@ -932,7 +1081,8 @@ def main():
                          "traffic": profiled_traffic(wl.name, args.engine),
                          "bytes_per_launch": int(dom_bytes),
                          "launch_us": round(dom_s * 1e6, 3),
-                         **({"isolated_launch": isolated} if isolated else {})},
+                         **({"isolated_launch": isolated} if isolated else {}),
+                         **({"tensor": tensor} if tensor else {})},
             "cpu_baseline": cpu,
             "e2e": {"value": round(job_gbs(world, step.bytes_alg, e2e_steps, t_e2e), 2),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -372,6 +372,60 @@ BQ_API int32_t bq_verify_gemm(int32_t fmt, const bq_qmat *W, const uint16_t *x, 
                               float *y, void *ws, size_t ws_bytes, int32_t *dev_status,
                               void *stream);
 
+/* ----------------------------------- decode attention over a Q8 KV cache --- */
+
+/* A preallocated KV cache of Tmax positions per (sequence, KV head), keys and
+ * values block-quantised in the Q8 format of the weights (32-element blocks
+ * along the head dimension, fp16 scale = absmax/127, int8 codes).  Device
+ * pointers, 16-byte aligned; caller-owned.
+ *   k_codes   int8 [B][Hkv][Tmax][D]    one row of D codes per position
+ *   k_scales  fp16 [B][Hkv][Tmax][D/32]
+ *   vt_codes  int8 [B][Hkv][D][Tmax]    values transposed: row d holds
+ *                                       component d of every position (a new
+ *                                       token writes one byte in each of the D
+ *                                       rows)
+ *   v_scales  fp16 [B][Hkv][Tmax][D/32] scale of position t's block j */
+typedef struct bq_kv_cache {
+    const int8_t *k_codes;
+    const uint16_t *k_scales;
+    const int8_t *vt_codes;
+    const uint16_t *v_scales;
+    int32_t D, Tmax;
+} bq_kv_cache;
+
+/* Bytes of workspace bq_attn_decode_q8 needs (arrival counters per sequence
+ * and head + per-CTA partial results).  0 on a bad shape. */
+BQ_API size_t bq_attn_workspace_bytes(int32_t B, int32_t Hkv);
+
+/* Decode attention: for each sequence b and query head i (KV head h = i / G),
+ *   s_t = scale * sum_d q[b][i][d] K[t][d],  p = softmax over t < lens[b],
+ *   o[b][i][d] = sum_t p_t V[t][d],
+ * with K and V dequantised from the cache (d * code).  The KV cache is kept
+ * preallocated for the whole decode loop (gist.science technical summary,
+ * "Methodologie" -> "Zero-Allocation Decode Loop"), and decode attention is
+ * the other memory-bound kernel of the decode step beside the GEMV
+ * (romaanj.github.io review of the M5 follow-up paper, "Method").
+ *   kv      the cache; D must be 128, Tmax a multiple of 128
+ *   q       device fp16 bits [B][Hkv*G][D]
+ *   lens    device int32 [B]: positions 0 .. lens[b]-1 are attended to
+ *           (clamped to [0, Tmax]; a sequence with none gets o = 0); nothing
+ *           past lens[b] is read into the result
+ *   B, Hkv  sequences, KV heads; G query heads per KV head, 1..8
+ *   scale   softmax scale (typically 1/sqrt(D))
+ *   o       device fp32 [B][Hkv*G][D], overwritten
+ *   ws      device workspace >= bq_attn_workspace_bytes(B, Hkv), zero-filled
+ *           before first use, left zero-filled by every call that completes
+ *   dev_status, stream as bq_gemv_q4
+ * Both products run on tensor cores with the cache codes as exact fp16
+ * operands; the softmax weights times the value scales enter rounded once to
+ * fp16 (relative 2^-11), so |o - o_exact| <= ~2^-11 sum_t p_t |V[t][d]| plus
+ * fp32 accumulation and exp2 approximation error.  Deterministic for a given
+ * device and shape.  BQ_ERR_SHAPE for D != 128, Tmax not a multiple of 128,
+ * or G outside 1..8. */
+BQ_API int32_t bq_attn_decode_q8(const bq_kv_cache *kv, const uint16_t *q, const int32_t *lens,
+                                 int32_t B, int32_t Hkv, int32_t G, float scale, float *o,
+                                 void *ws, size_t ws_bytes, int32_t *dev_status, void *stream);
+
 /* ------------------------------------------------------ routed experts --- */
 
 /* Bytes of workspace bq_moe_gemv_q4 needs.  0 on a bad shape. */

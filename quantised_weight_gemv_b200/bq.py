@@ -45,6 +45,12 @@ class bq_step_wait(ctypes.Structure):
                 ("reserved", ctypes.c_int32)]
 
 
+class bq_kv_cache(ctypes.Structure):
+    _fields_ = [("k_codes", ctypes.c_void_p), ("k_scales", ctypes.c_void_p),
+                ("vt_codes", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
+                ("D", ctypes.c_int32), ("Tmax", ctypes.c_int32)]
+
+
 class bq_gemv_geometry(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("rows", "chunks", "chunks_per_band",
                                                "chunks_per_worker", "grid", "cluster",
@@ -80,6 +86,9 @@ _SIGS = {
     "bq_step_run_ex": (_i32, [_SIP, _vp, _vp, _sz, ctypes.POINTER(bq_step_wait), _vp, _vp]),
     "bq_moe_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "bq_verify_workspace_bytes": (_sz, [_i32, _i32, _i32]),
+    "bq_attn_workspace_bytes": (_sz, [_i32, _i32]),
+    "bq_attn_decode_q8": (_i32, [ctypes.POINTER(bq_kv_cache), _vp, _vp, _i32, _i32, _i32,
+                                 ctypes.c_float, _vp, _vp, _sz, _vp, _vp]),
     "bq_verify_gemm": (_i32, [_i32, _QP, _vp, _i32, _vp, _vp, _sz, _vp, _vp]),
     "bq_moe_gemv_q4": (_i32, [_QP, _i32, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _i32, _vp,
                               _vp, _sz, _vp, _vp]),
@@ -257,6 +266,43 @@ def verify_gemm(fmt: int, W: bq_qmat, x, y, ws, status=None, stream=None) -> Non
                                                  y.data_ptr(), ws.data_ptr(),
                                                  ws.numel() * ws.element_size(), _ptr(status),
                                                  _stream_ptr(stream)))
+
+
+def kv_cache(k_codes, k_scales, vt_codes, v_scales) -> bq_kv_cache:
+    """A bq_kv_cache over device tensors: k_codes int8 [B, Hkv, Tmax, D],
+    k_scales fp16 bits [B, Hkv, Tmax, D/32], vt_codes int8 [B, Hkv, D, Tmax],
+    v_scales fp16 bits [B, Hkv, Tmax, D/32] (the tensors stay owned by the
+    caller; the struct keeps references)."""
+    _on_device("kv_cache", k_codes=k_codes, k_scales=k_scales, vt_codes=vt_codes, v_scales=v_scales)
+    B, Hkv, Tmax, D = k_codes.shape
+    if (tuple(vt_codes.shape) != (B, Hkv, D, Tmax) or tuple(k_scales.shape) != (B, Hkv, Tmax, D // 32)
+            or tuple(v_scales.shape) != (B, Hkv, Tmax, D // 32)
+            or any(not t.is_contiguous() for t in (k_codes, k_scales, vt_codes, v_scales))
+            or k_codes.element_size() != 1 or vt_codes.element_size() != 1
+            or k_scales.element_size() != 2 or v_scales.element_size() != 2):
+        raise ValueError("kv_cache: shapes/dtypes/contiguity do not match the cache layout")
+    kv = bq_kv_cache(k_codes.data_ptr(), k_scales.data_ptr(), vt_codes.data_ptr(),
+                     v_scales.data_ptr(), int(D), int(Tmax))
+    kv._refs = (k_codes, k_scales, vt_codes, v_scales)
+    kv.B, kv.Hkv = int(B), int(Hkv)
+    return kv
+
+
+def attn_decode_q8(kv: bq_kv_cache, q, lens, G: int, scale: float, o, ws, status=None,
+                   stream=None) -> None:
+    """o[B, Hkv*G, D] (fp32) = softmax(scale q K^T) V over the Q8 cache, per
+    sequence over its first lens[b] positions (bq_attn_decode_q8)."""
+    _on_device("attn_decode_q8", q=q, lens=lens, o=o, ws=ws, status=status)
+    B, Hkv = kv.B, kv.Hkv
+    if tuple(q.shape) != (B, Hkv * G, kv.D) or q.element_size() != 2 or not q.is_contiguous():
+        raise ValueError(f"attn_decode_q8: q must be contiguous fp16 bits [{B}, {Hkv * G}, {kv.D}]")
+    if lens.numel() != B or lens.element_size() != 4 or not lens.is_contiguous():
+        raise ValueError(f"attn_decode_q8: lens must be int32 [{B}]")
+    if not o.is_contiguous() or _nbytes(o) < B * Hkv * G * kv.D * 4:
+        raise ValueError("attn_decode_q8: o too small")
+    check("bq_attn_decode_q8", lib().bq_attn_decode_q8(
+        ctypes.byref(kv), q.data_ptr(), lens.data_ptr(), B, Hkv, int(G), float(scale), o.data_ptr(),
+        ws.data_ptr(), ws.numel() * ws.element_size(), _ptr(status), _stream_ptr(stream)))
 
 
 def moe_gemv_q4(Wstack: bq_qmat, E: int, codes_stride: int, scales_stride: int, x,

@@ -712,12 +712,17 @@ __device__ __forceinline__ void block_q8(uint32_t addr_a, uint32_t addr_b, uint2
           "f"(off[1]), "f"(off[2]), "f"(off[3]), "f"(dg), "f"(dg8));
 }
 
-// Both halves of an fp16 pair as fp32.
-__device__ __forceinline__ void halves_to_float(uint32_t v, float &lo, float &hi)
+// One half of an fp16 pair as fp32 (HI: the upper half).  One asm per half,
+// so a block converts only the scale it uses.
+template <bool HI>
+__device__ __forceinline__ float half_of_pair(uint32_t v)
 {
-    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
-        "cvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
-        : "=f"(lo), "=f"(hi) : "r"(v));
+    float f;
+    if constexpr (HI)
+        asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, h;\n\t}" : "=f"(f) : "r"(v));
+    else
+        asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, l;\n\t}" : "=f"(f) : "r"(v));
+    return f;
 }
 
 __device__ __forceinline__ uint4 lds128_u32(uint32_t addr)
@@ -817,11 +822,9 @@ __device__ __forceinline__ void chunk_mma(uint32_t codes_s, uint32_t scales_s, i
         block_offset<FMT>(xa[jb], xb[jb], off);
 #pragma unroll
         for (int mt = 0; mt < MT; mt++) {
-            float d0, d1, e0, e1;
-            halves_to_float(pick_u32(sc[mt][0], jb >> 1), d0, d1);
-            halves_to_float(pick_u32(sc[mt][1], jb >> 1), e0, e1);
-            const float dg = (jb & 1) ? d1 : d0;
-            const float dg8 = (jb & 1) ? e1 : e0;
+            const uint32_t s0 = pick_u32(sc[mt][0], jb >> 1), s8 = pick_u32(sc[mt][1], jb >> 1);
+            const float dg = (jb & 1) ? half_of_pair<true>(s0) : half_of_pair<false>(s0);
+            const float dg8 = (jb & 1) ? half_of_pair<true>(s8) : half_of_pair<false>(s8);
             if constexpr (FMT == 4) {
                 block_q4(lane_codes + mt * 2048 + sw[jb], xa[jb], xb[jb], off, dg, dg8, acc[mt], m16);
             } else if constexpr (kLow2) {

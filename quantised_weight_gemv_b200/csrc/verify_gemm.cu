@@ -22,14 +22,15 @@
 // the CTA partials in CTA order).
 //
 // Warp roles (16 warps):
-//   warp 0      TMA of the packed codes (128-byte swizzle) and the scales of a
-//               unit into a 3-slot (Q8: 2-slot) ring;
+//   warp 0      TMA of a unit's packed codes (128-byte swizzle), scales and
+//               activations x (K-major, 128-byte swizzle: the layout the
+//               MMA's B descriptor reads; rows >= B zero-filled) into a 3-slot
+//               (Q8: 2-slot) ring, so x arrives units ahead of its MMAs;
 //   warp 1      allocates TMEM, and one thread issues the MMAs: per 64-weight
 //               sub-stage, 4 x tcgen05.mma (M 128, N NB, K 16, fp16 inputs,
 //               fp32 accumulation) from shared-memory descriptors, then
-//               tcgen05.commit to free the sub-stage's slots;
-//   warp 2      TMA of the activations x (K-major, 128-byte swizzle: the
-//               layout the MMA's B descriptor reads, rows >= B zero-filled);
+//               tcgen05.commit to free the sub-stage's A slot (and after a
+//               unit's last one, the unit's ring slot);
 //   warps 4-7   epilogue: tcgen05.ld of the accumulator, one thread per row;
 //   warps 8-15  dequantisation: one thread per (row, block) of a sub-stage
 //               turns 16 (Q8: 32) code bytes and the block's fp16 scale into
@@ -78,11 +79,18 @@ template <> struct VFmt<8> {
     static constexpr int kCS = 2;
 };
 
+// A unit's ring slot: codes, then x (4 sub-tiles of NB rows x 64 fp16), then
+// scales.
+template <int FMT, int NB>
+__host__ __device__ constexpr int slot_bytes()
+{
+    return VFmt<FMT>::kCodeBytes + 4 * NB * 128 + kScaleBytes;
+}
+
 template <int FMT, int NB>
 constexpr size_t smem_bytes()
 {
-    return 1024 + (size_t)VFmt<FMT>::kCS * VFmt<FMT>::kCodeBytes + (size_t)AS * kABytes +
-           (size_t)AS * NB * 128 + (size_t)VFmt<FMT>::kCS * kScaleBytes + 1024;
+    return 1024 + (size_t)VFmt<FMT>::kCS * slot_bytes<FMT, NB>() + (size_t)AS * kABytes + 1024;
 }
 
 // Per-tile partial sums through the workspace: [CTA][slot 0 / 1][TM][32] fp32.
@@ -285,9 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
     constexpr int CS = VF::kCS;
     constexpr int CB = VF::kCodeBytes;
     constexpr int XB = NB * 128;   // x bytes per sub-stage
+    constexpr int SLOT = slot_bytes<FMT, NB>();
     extern __shared__ uint8_t smem_raw[];
     __shared__ alignas(8) uint64_t bar_cfull[CS], bar_cempty[CS], bar_afull[AS], bar_aempty[AS],
-        bar_xfull[AS], bar_accfull[2], bar_accempty[2], bar_shift[kShiftRing],
+        bar_accfull[2], bar_accempty[2], bar_shift[kShiftRing],
         bar_shift_free[kShiftRing], bar_done,
         bar_epi_a, bar_epi_b;
     __shared__ uint32_t tmem_base_s;
@@ -296,10 +305,9 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
     __shared__ int abort_s;
 
     uint8_t *sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const uint32_t codes_s = smem_u32(sbase);
-    const uint32_t a_s = codes_s + CS * CB;
-    const uint32_t x_s = a_s + AS * kABytes;
-    const uint32_t sc_s = x_s + AS * XB;
+    const uint32_t ring_s = smem_u32(sbase);                 // CS unit slots (1024-aligned)
+    const uint32_t a_s = ring_s + CS * SLOT;                 // AS A tiles
+    static_assert(SLOT % 1024 == 0, "unit slots keep the 1024-byte alignment of the swizzled boxes");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cta = blockIdx.x;
     const int u0 = (int)((long long)cta * a.U / a.G), u1 = (int)((long long)(cta + 1) * a.U / a.G);
@@ -307,12 +315,11 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
     if (threadIdx.x == 0) {
         for (int i = 0; i < CS; i++) {
             mbar_init(smem_u32(&bar_cfull[i]), 1);
-            mbar_init(smem_u32(&bar_cempty[i]), 8);          // the 8 dequant warps
+            mbar_init(smem_u32(&bar_cempty[i]), 9);          // the 8 dequant warps + the MMAs' commit
         }
         for (int i = 0; i < AS; i++) {
             mbar_init(smem_u32(&bar_afull[i]), 8);           // the 8 dequant warps
             mbar_init(smem_u32(&bar_aempty[i]), 1);          // tcgen05.commit
-            mbar_init(smem_u32(&bar_xfull[i]), 1);
         }
         for (int i = 0; i < 2; i++) {
             mbar_init(smem_u32(&bar_accfull[i]), 1);         // tcgen05.commit
@@ -365,6 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
         // ---------------------------------------------- codes + scales TMA --
         if (lane == 0) {
             const uint64_t pol = policy_evict_first();
+            const uint64_t pol_x = policy_evict_normal();
             int n = 0;
             for (int u = u0; u < u1 && !aborted(); u++, n++) {
                 const int slot = n % CS;
@@ -372,49 +380,28 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                     break;
                 const int tile = u / a.KU, ku = u % a.KU;
                 const uint32_t bar = smem_u32(&bar_cfull[slot]);
-                mbar_arrive_expect_tx(bar, CB + kScaleBytes);
+                const uint32_t dst = ring_s + slot * SLOT;
+                mbar_arrive_expect_tx(bar, SLOT);
                 if constexpr (FMT == 4) {
-                    tma_load_2d(codes_s + slot * CB, &a.tm_codes, bar, ku * 128, tile * TM, pol);
+                    tma_load_2d(dst, &a.tm_codes, bar, ku * 128, tile * TM, pol);
                 } else {
-                    tma_load_2d(codes_s + slot * CB, &a.tm_codes, bar, ku * 256, tile * TM, pol);
-                    tma_load_2d(codes_s + slot * CB + TM * 128, &a.tm_codes, bar, ku * 256 + 128,
-                                tile * TM, pol);
+                    tma_load_2d(dst, &a.tm_codes, bar, ku * 256, tile * TM, pol);
+                    tma_load_2d(dst + TM * 128, &a.tm_codes, bar, ku * 256 + 128, tile * TM, pol);
                 }
-                tma_load_2d(sc_s + slot * kScaleBytes, &a.tm_scales, bar, ku * 8, tile * TM, pol);
+#pragma unroll
+                for (int j = 0; j < 4; j++)     // x: the unit's four 64-wide sub-tiles (L2-resident)
+                    tma_load_2d(dst + CB + j * XB, &a.tm_x, bar, ku * kUnitK + j * kSubK, 0, pol_x);
+                tma_load_2d(dst + CB + 4 * XB, &a.tm_scales, bar, ku * 8, tile * TM, pol);
             }
             // Drain: every load issued lands before the CTA may exit.
             for (int j = max(0, n - CS); j < n; j++)
                 (void)mbar_wait_bounded(smem_u32(&bar_cfull[j % CS]), (j / CS) & 1);
         }
-    } else if (warp == 2) {
-        // ------------------------------------------------------- x TMA ----
-        if (lane == 0) {
-            const uint64_t pol = policy_evict_normal();
-            int i = 0;
-            for (int u = u0; u < u1 && !aborted(); u++) {
-                const int ku = u % a.KU, ns = nsub(u);
-                bool ok = true;
-                for (int j = 0; j < ns; j++, i++) {
-                    const int slot = i % AS;
-                    if (!wait(bar_aempty[slot], ((i / AS) & 1) ^ 1)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t bar = smem_u32(&bar_xfull[slot]);
-                    mbar_arrive_expect_tx(bar, XB);
-                    tma_load_2d(x_s + slot * XB, &a.tm_x, bar, ku * kUnitK + j * kSubK, 0, pol);
-                }
-                if (!ok)
-                    break;
-            }
-            for (int j = max(0, i - AS); j < i; j++)
-                (void)mbar_wait_bounded(smem_u32(&bar_xfull[j % AS]), (j / AS) & 1);
-        }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA ----
         if (lane == 0) {
             constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(NB >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
-            int i = 0, seg = 0;
+            int i = 0, seg = 0, nu = 0;
             int u = u0;
             bool ok = true;
             while (u < u1 && ok) {
@@ -426,17 +413,22 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(buf * 32);
                 bool first = true;
-                for (; u < uend && ok; u++) {
+                for (; u < uend && ok; u++, nu++) {
                     const int ns = nsub(u);
+                    const int cslot = nu % CS;
+                    if (!wait(bar_cfull[cslot], (nu / CS) & 1)) {     // this unit's x has landed
+                        ok = false;
+                        break;
+                    }
                     for (int j = 0; j < ns; j++, i++) {
                         const int slot = i % AS;
-                        if (!wait(bar_afull[slot], (i / AS) & 1) || !wait(bar_xfull[slot], (i / AS) & 1)) {
+                        if (!wait(bar_afull[slot], (i / AS) & 1)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         const uint64_t ad = desc_k_sw128(a_s + slot * kABytes);
-                        const uint64_t bd = desc_k_sw128(x_s + slot * XB);
+                        const uint64_t bd = desc_k_sw128(ring_s + cslot * SLOT + CB + j * XB);
 #pragma unroll
                         for (int kk = 0; kk < kSubK / 16; kk++) {
                             // K step of 16 fp16 = 32 bytes along the swizzled row
@@ -446,6 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                         first = false;
                         umma_commit(smem_u32(&bar_aempty[slot]));
                     }
+                    if (ok)     // the unit's x is read once these MMAs complete
+                        umma_commit(smem_u32(&bar_cempty[cslot]));
                 }
                 if (!ok)
                     break;
@@ -604,8 +598,8 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                     ok = false;
                     break;
                 }
-                const uint32_t crow = codes_s + cslot * CB + r * 128;
-                const uint32_t srow_s = sc_s + cslot * kScaleBytes + r * 16;
+                const uint32_t crow = ring_s + cslot * SLOT + r * 128;
+                const uint32_t srow_s = ring_s + cslot * SLOT + CB + 4 * XB + r * 16;
                 const int ns = nsub(u);
                 for (int j = 0; j < ns; j++, i++) {
                     const int slot = i % AS;

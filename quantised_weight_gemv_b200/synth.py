@@ -7,7 +7,9 @@ their inputs from it.
 
 Distributions (stated with the workloads): weights w ~ N(0, 0.02) (0.02 is the
 standard deviation) drawn in fp32; activations x ~ N(0, 1) drawn in fp32 and
-rounded to fp16 (nearest-even); routed-expert indices drawn uniformly without
+rounded to fp16 (nearest-even); cached keys and values of decode attention
+~ N(0, 1) in fp32 (quantised into the cache per position); routed-expert
+indices drawn uniformly without
 replacement per token; routing weights are a softmax (fp64, stored as fp32) of
 N(0, 1) logits.  Every stream is keyed by
 ``(seed, workload id, layer, matrix id, kind)``.
@@ -24,7 +26,7 @@ from typing import List, Optional, Sequence, Tuple
 
 import numpy as np
 
-KIND_W, KIND_X, KIND_IDX, KIND_LOGIT, KIND_H = 0, 1, 2, 3, 4
+KIND_W, KIND_X, KIND_IDX, KIND_LOGIT, KIND_H, KIND_KEY, KIND_VAL, KIND_LEN = 0, 1, 2, 3, 4, 5, 6, 7
 W_STD = 0.02
 
 
@@ -46,6 +48,16 @@ def torch_seed(k: Sequence[int]) -> int:
 def weights_f32(k: Sequence[int], N: int, K: int) -> np.ndarray:
     """fp32 [N, K], N(0, 0.02)."""
     return (rng(k).standard_normal((N, K), dtype=np.float32) * np.float32(W_STD)).astype(np.float32)
+
+
+def kv_values_f32(k: Sequence[int], *shape: int) -> np.ndarray:
+    """fp32 N(0, 1) keys or values of a KV cache (before quantisation)."""
+    return rng(k).standard_normal(shape, dtype=np.float32)
+
+
+def seq_lens(k: Sequence[int], B: int, Tmax: int) -> np.ndarray:
+    """int32 [B] sequence lengths drawn uniformly from 1 .. Tmax."""
+    return rng(k).integers(1, Tmax + 1, size=B).astype(np.int32)
 
 
 def activations_f16_bits(k: Sequence[int], *shape: int) -> np.ndarray:
@@ -104,6 +116,7 @@ class DenseWorkload:
     mats: Tuple[Mat, ...]   # per-layer matrices, in model order
     B: int = 1
     independent: bool = False   # layers are independent copies (one stage for all)
+    verify: bool = False        # a batched-verification step (bq_verify_gemm per matrix)
 
     def layer_weights(self) -> int:
         return sum(m.N * m.K for m in self.mats)
@@ -149,6 +162,14 @@ def dense_h4096(fmt: int, B: int) -> DenseWorkload:
     ), B)
 
 
+def verify_h4096(fmt: int, B: int) -> DenseWorkload:
+    """The hidden-4096 layer's matrices (36 distinct copies) as a batched
+    verification step of B = 16 or 32 drafted tokens: every matrix through the
+    tensor-core GEMM, each with its own seeded batch of activations."""
+    return DenseWorkload(9, f"verify36L-h4096-ffn12288-q{fmt}-b{B}", fmt, 36,
+                         dense_h4096(fmt, B).mats, B, verify=True)
+
+
 # 64-layer dense decoder, hidden 5120, FFN 25600, Q4, batch 1 (~16 GB packed).
 # Attention shapes: q, o 5120 x 5120; k, v 1024 x 5120 (8 KV heads x 128).
 DENSE_H5120 = DenseWorkload(5, "dense64L-h5120-ffn25600-q4", 4, 64, (
@@ -172,6 +193,14 @@ def sweep_workload(fmt: int, N: int, K: int, B: int = 1, min_bytes: int = 512 <<
     copies = min(max_copies, max(2, -(-min_bytes // packed_bytes(fmt, N, K))))
     return DenseWorkload(6, f"sweep-q{fmt}-{N}x{K}-b{B}", fmt, copies, (Mat("w", N, K, 0),), B,
                          independent=True)
+
+
+def verify_sweep_workload(fmt: int, N: int, K: int, B: int, min_bytes: int = 512 << 20) -> DenseWorkload:
+    """Independent copies of one N x K matrix (>= min_bytes of packed weights)
+    through the batched-verification GEMM: its steady-state rate."""
+    copies = min(256, max(2, -(-min_bytes // packed_bytes(fmt, N, K))))
+    return DenseWorkload(10, f"verify-sweep-q{fmt}-{N}x{K}-b{B}", fmt, copies, (Mat("w", N, K, 0),),
+                         B, independent=True, verify=True)
 
 
 def single_workload(fmt: int, N: int, K: int, B: int = 1) -> DenseWorkload:
@@ -201,3 +230,37 @@ def moe_h2048(B: int) -> MoEWorkload:
     """48 layers, hidden 2048, 128 experts (gate/up 768 x 2048, down 2048 x 768),
     top-8 routing."""
     return MoEWorkload(4, f"moe48L-e128-top8-h2048-b{B}", 48, 128, 8, 2048, 768, B)
+
+
+@dataclasses.dataclass(frozen=True)
+class AttnWorkload:
+    """Decode attention of every layer of a decoder over a Q8 KV cache of
+    Tmax positions per (sequence, KV head), head dimension 128.  lens None:
+    every sequence is full (Tmax positions); else lengths drawn uniformly
+    from 1 .. Tmax (seq_lens)."""
+    wid: int
+    name: str
+    layers: int
+    B: int
+    Hkv: int
+    G: int
+    Tmax: int
+    full: bool = True
+    D: int = 128
+
+    def lens(self, seed: int = 0) -> np.ndarray:
+        if self.full:
+            return np.full(self.B, self.Tmax, dtype=np.int32)
+        return seq_lens(key(seed, self.wid, 0, 0, KIND_LEN), self.B, self.Tmax)
+
+
+def attn_h5120(B: int, Tmax: int) -> AttnWorkload:
+    """The 64-layer hidden-5120 decoder's attention (40 query heads on 8 KV
+    heads), every sequence at Tmax positions."""
+    return AttnWorkload(11, f"attn64L-kv8-g5-t{Tmax}-b{B}", 64, B, 8, 5, Tmax)
+
+
+def attn_h2048(B: int, Tmax: int) -> AttnWorkload:
+    """The 16-layer hidden-2048 decoder's attention (16 query heads on 4 KV
+    heads), sequence lengths drawn uniformly from 1 .. Tmax."""
+    return AttnWorkload(12, f"attn16L-kv4-g4-t{Tmax}-b{B}-mixed", 16, B, 4, 4, Tmax, full=False)

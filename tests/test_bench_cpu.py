@@ -73,3 +73,11 @@ def test_default_workload_is_the_largest_single_gpu_decoder():
     wl = bench.WORKLOADS["dense64L-h5120-ffn25600-q4"]
     assert wl.layers == 64 and wl.B == 1
 
+
+
+def test_reference_arm_attention_workload():
+    """The oracle arm on a decode-attention workload: layer 0's attention over
+    the Q8 cache (the same seeded keys, values, queries and lengths)."""
+    d = _reference_line("--workload", "attn16L-kv4-g4-t8192-b8-mixed", "--steps", "1")
+    assert d["config"]["workload"] == "attn16L-kv4-g4-t8192-b8-mixed" and d["value"] > 0
+    assert "layer 0" in d["cpu_baseline"]["sample"]

@@ -172,6 +172,15 @@ def test_dense36_h4096_step(fmt, B):
     _check_step(synth.dense_h4096(fmt, B), every=128, engines=("graph",))
 
 
+@pytest.mark.parametrize("fmt", [4, 8])
+@pytest.mark.parametrize("B", [16, 32])
+def test_verify36_h4096_step(fmt, B):
+    """The hidden-4096 layer's matrices (36 distinct copies) as a batched
+    verification step at B = 16 and 32 through the tensor-core GEMM: every row
+    of the first and last layer, 1/128 of the rows of every other matrix."""
+    _check_step(synth.verify_h4096(fmt, B), every=128, engines=("graph",))
+
+
 def test_dense64_h5120_step():
     """64-layer decoder (hidden 5120, FFN 25600, ~16 GB Q4), batch 1: as the
     launch chain bench.py times, and as one plan."""
