@@ -489,23 +489,54 @@ __global__ void __launch_bounds__(kThreads, 2) attn_decode_kernel(const __grid_c
                 break;
             if (merge_old == cl - cf) {
                 __threadfence();
+                // The partial of CTA c of this sequence: slot 0 if the sequence
+                // holds c's first unit, else slot 1.  Every CTA after cf starts
+                // inside the sequence, so only cf can hold it in slot 1 (when
+                // cf's range starts in an earlier sequence): one division here,
+                // none per partial.
+                const int cf_slot = (int)((long long)cf * a.U / a.nctas) < sq * a.tps ? 1 : 0;
+                auto part = [&](int c) {
+                    return a.partials + ((size_t)c * 2 + (c == cf ? cf_slot : 0)) * kPartFloats;
+                };
+                // Loads are issued in batches (8, then 4 CTAs at a time) so a
+                // merge of many partials costs a few L2 round trips, not one
+                // per partial; the sums still run in CTA order.
                 float M = -INFINITY;
-                for (int c = cf; c <= cl; c++) {
-                    const int sl = (sq == (int)((long long)c * a.U / a.nctas) / a.tps) ? 0 : 1;
-                    M = fmaxf(M, __ldcg(a.partials + ((size_t)c * 2 + sl) * kPartFloats + j));
+                for (int c0 = cf; c0 <= cl; c0 += 8) {
+                    float mv[8];
+#pragma unroll
+                    for (int k = 0; k < 8; k++)
+                        mv[k] = c0 + k <= cl ? __ldcg(part(c0 + k) + j) : -INFINITY;
+#pragma unroll
+                    for (int k = 0; k < 8; k++)
+                        M = fmaxf(M, mv[k]);
                 }
                 float Ls = 0.f, os[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int c = cf; c <= cl; c++) {
-                    const int sl = (sq == (int)((long long)c * a.U / a.nctas) / a.tps) ? 0 : 1;
-                    const float *pc = a.partials + ((size_t)c * 2 + sl) * kPartFloats;
-                    const float mc = __ldcg(pc + j);
-                    const float f = mc == -INFINITY ? 0.f : ex2(mc - M);
-                    Ls += f * __ldcg(pc + kMaxG + j);
-                    const float4 oc = __ldcg(reinterpret_cast<const float4 *>(pc + 2 * kMaxG + j * D + d4));
-                    os[0] += f * oc.x;
-                    os[1] += f * oc.y;
-                    os[2] += f * oc.z;
-                    os[3] += f * oc.w;
+                for (int c0 = cf; c0 <= cl; c0 += 4) {
+                    float mc[4], lc[4];
+                    float4 oc[4];
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        if (c0 + k <= cl) {
+                            const float *pc = part(c0 + k);
+                            mc[k] = __ldcg(pc + j);
+                            lc[k] = __ldcg(pc + kMaxG + j);
+                            oc[k] = __ldcg(reinterpret_cast<const float4 *>(pc + 2 * kMaxG + j * D + d4));
+                        } else {
+                            mc[k] = -INFINITY;
+                            lc[k] = 0.f;
+                            oc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                    }
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        const float f = mc[k] == -INFINITY ? 0.f : ex2(mc[k] - M);
+                        Ls += f * lc[k];
+                        os[0] += f * oc[k].x;
+                        os[1] += f * oc[k].y;
+                        os[2] += f * oc[k].z;
+                        os[3] += f * oc[k].w;
+                    }
                 }
                 if (j < a.G) {
                     const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
@@ -516,8 +547,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_decode_kernel(const __grid_c
                 if (!sync_compute())
                     break;
                 for (int c = cf; c <= cl; c++) {
-                    const int sl = (sq == (int)((long long)c * a.U / a.nctas) / a.tps) ? 0 : 1;
-                    float *pc = a.partials + ((size_t)c * 2 + sl) * kPartFloats;
+                    float *pc = part(c);
                     __stcg(reinterpret_cast<float4 *>(pc + 2 * kMaxG + j * D + d4), make_float4(0.f, 0.f, 0.f, 0.f));
                     if ((i & 31) == 0) {
                         __stcg(pc + j, 0.f);

@@ -199,9 +199,31 @@ __device__ __forceinline__ uint32_t launder(uint32_t v)
     return r;
 }
 
+// Non-blocking test of phase `parity` of an mbarrier.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+#ifndef BQ_WAIT_TEST_FIRST
+#define BQ_WAIT_TEST_FIRST 1
+#endif
+
 // Wait for phase `parity` of an mbarrier, giving up after kWaitCycles.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
 {
+#if BQ_WAIT_TEST_FIRST
+    if (mbar_test_wait(bar, parity))
+        return true;
+#endif
     if (mbar_try_wait(bar, parity))
         return true;
     const long long t0 = clock64();

@@ -24,19 +24,27 @@
 // Warp roles (16 warps):
 //   warp 0      TMA of a unit's packed codes (128-byte swizzle), scales and
 //               activations x (K-major, 128-byte swizzle: the layout the
-//               MMA's B descriptor reads; rows >= B zero-filled) into a 3-slot
-//               (Q8: 2-slot) ring, so x arrives units ahead of its MMAs;
-//   warp 1      allocates TMEM, and one thread issues the MMAs: per 64-weight
-//               sub-stage, 4 x tcgen05.mma (M 128, N NB, K 16, fp16 inputs,
-//               fp32 accumulation) from shared-memory descriptors, then
-//               tcgen05.commit to free the sub-stage's A slot (and after a
-//               unit's last one, the unit's ring slot);
+//               MMA's B descriptor reads; rows >= B zero-filled) into a ring
+//               of 4-6 unit slots, so x arrives units ahead of its MMAs;
+//   warp 1      allocates TMEM (512 columns: two accumulators and a ring of
+//               6 dequantised A sub-stages), and one thread issues the MMAs:
+//               per 128-weight sub-stage, 8 x tcgen05.mma (M 128, N NB, K 16,
+//               fp16 in, fp32 accumulation) with A read from TMEM and x from a
+//               shared-memory descriptor, then tcgen05.commit to free the A
+//               slot (after a unit's last one, also the unit's ring slot);
 //   warps 4-7   epilogue: tcgen05.ld of the accumulator, one thread per row;
-//   warps 8-15  dequantisation: one thread per (row, block) of a sub-stage
-//               turns 16 (Q8: 32) code bytes and the block's fp16 scale into
-//               32 fp16 weights d (q - z) 2^s and stores them into the MMA's A
-//               tile (K-major, 128-byte swizzle).
-//
+//   warps 8-15  dequantisation: warp w serves TMEM lanes 32 (w % 4) .. + 31
+//               (rows) and one half of each sub-stage; a thread turns two
+//               blocks of its row (32 or 64 code bytes and two fp16 scales)
+//               into 64 fp16 weights d (q - z) 2^s and writes them as 32 TMEM
+//               columns with tcgen05.st.
+// A lives in TMEM, not shared memory: a 128 x 16 fp16 A operand is 4 KB, and
+// reading it from shared memory for every K16 step (plus writing it there
+// first) would need more shared-memory bandwidth than the Q4 stream leaves.
+// Measured (one CTA per SM): a dependent tcgen05.mma of M 128 x N 32 x K 16
+// issues about every 71 cycles, so the MMA side caps a Q4 verification step
+// near 0.7 of HBM; a deeper split into more dequant warps measured slower.
+
 // Rounding.  The decode GEMV keeps codes exact and scales each block's sum;
 // a tile accumulated over many blocks cannot, so the A tile holds each weight
 // rounded once to fp16: relative error <= 2^-11, inside the decode tolerance
@@ -57,14 +65,22 @@
 namespace bq {
 namespace vg {
 
-constexpr int kThreads = 512;
+#ifndef BQ_VERIFY_DQ_GROUPS
+#define BQ_VERIFY_DQ_GROUPS 1
+#endif
+constexpr int kDqGroups = BQ_VERIFY_DQ_GROUPS;   // dequant warp groups (8 warps each), alternate sub-stages
+constexpr int kThreads = (8 + 8 * kDqGroups) * 32;
 constexpr int TM = 128;                 // rows per tile (MMA M)
 constexpr int kUnitK = 256;             // weights of K per unit
-constexpr int kSubK = 64;               // weights of K per sub-stage (one 128-byte swizzle row of fp16)
-constexpr int AS = 4;                   // A / x sub-stage slots
+constexpr int kSubK = 128;              // weights of K per sub-stage (one hand-off to the MMA thread)
+constexpr int kXK = 64;                 // weights of K per x tile (one 128-byte swizzle row of fp16)
+constexpr int AS = 6;                   // A sub-stage slots in tensor memory (3 units)
+constexpr int kAccCols = 64;            // TMEM columns of the two accumulators (up to 32 each)
+constexpr int kACols = kSubK / 2;       // TMEM columns of one A sub-stage (two fp16 a column)
+constexpr int kTmemCols = 512;
+static_assert(kAccCols + AS * kACols <= kTmemCols, "accumulators and the A ring fit in TMEM");
 constexpr int kShiftRing = 4;           // row shifts of the last 4 segments
 constexpr int kMaxCtas = 512;
-constexpr int kABytes = TM * kSubK * 2; // 16 KB
 constexpr int kScaleBytes = TM * 16;    // 8 fp16 per row per unit
 constexpr int kDequantWarp0 = 8;
 constexpr int kEpiWarp0 = 4;
@@ -72,11 +88,9 @@ constexpr int kEpiWarp0 = 4;
 template <int FMT> struct VFmt;
 template <> struct VFmt<4> {
     static constexpr int kCodeBytes = TM * 128;   // one 128 x 128-byte box
-    static constexpr int kCS = 3;
 };
 template <> struct VFmt<8> {
     static constexpr int kCodeBytes = TM * 256;   // two 128 x 128-byte boxes
-    static constexpr int kCS = 2;
 };
 
 // A unit's ring slot: codes, then x (4 sub-tiles of NB rows x 64 fp16), then
@@ -87,10 +101,17 @@ __host__ __device__ constexpr int slot_bytes()
     return VFmt<FMT>::kCodeBytes + 4 * NB * 128 + kScaleBytes;
 }
 
+// Unit slots of the ring: as many as ~200 KB of shared memory holds (4 to 6).
+template <int FMT, int NB>
+__host__ __device__ constexpr int ring_slots()
+{
+    return (200 * 1024) / slot_bytes<FMT, NB>() < 6 ? (200 * 1024) / slot_bytes<FMT, NB>() : 6;
+}
+
 template <int FMT, int NB>
 constexpr size_t smem_bytes()
 {
-    return 1024 + (size_t)VFmt<FMT>::kCS * slot_bytes<FMT, NB>() + (size_t)AS * kABytes + 1024;
+    return 1024 + (size_t)ring_slots<FMT, NB>() * slot_bytes<FMT, NB>() + 1024;
 }
 
 // Per-tile partial sums through the workspace: [CTA][slot 0 / 1][TM][32] fp32.
@@ -199,6 +220,48 @@ __device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, float (&v)[16])
         v[i] = __uint_as_float(r[i]);
 }
 
+// 16 consecutive 32-bit TMEM columns of this thread's lane (32x32b shape: a
+// warp writes its 32 lanes), then wait until the warp's stores are done.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+          "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+          "r"(v[15])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+        "%29, %30, %31, %32};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+          "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+          "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+          "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+          "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16: A's row m is TMEM lane m,
+// its K elements two to a 32-bit column.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -225,11 +288,6 @@ __device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c)
     asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
     return d;
 }
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
-{
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
-}
 
 // fp16 pairs: 0x6400 | byte is the fp16 value 1024 + byte, exactly.
 constexpr uint32_t kMagic = 0x64646464u;
@@ -239,44 +297,35 @@ constexpr uint32_t kSixteenth = 0x2C002C00u; // 1/16
 constexpr uint32_t kNeg1152 = 0xE480E480u;   // -1152 (Q8: 1024 + 128)
 
 // Q4: the 32 weights of one block (16 code bytes; byte i holds element i in
-// its low and element i + 16 in its high nibble) as fp16 (q - 8) * ds,
-// written to four 16-byte granules of the row (elements 0-7, 8-15, 16-23,
-// 24-31).  (1024 + nibble) - 1032 and (1024 + 16 nibble) / 16 - 72 are exact;
-// the product by ds is the one rounding.
-__device__ __forceinline__ void dequant_q4_block(uint4 c, uint32_t ds2, uint32_t row_addr, int g0,
-                                                 int rsw)
+// its low and element i + 16 in its high nibble) as fp16 (q - 8) * ds, two a
+// register in element order: o[c] = elements (2c, 2c + 1).  (1024 + nibble)
+// - 1032 and (1024 + 16 nibble) / 16 - 72 are exact; the product by ds is the
+// one rounding.
+__device__ __forceinline__ void dequant_q4_block(uint4 c, uint32_t ds2, uint32_t (&o)[16])
 {
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-    uint32_t lo[8], hi[8];
 #pragma unroll
     for (int i = 0; i < 4; i++) {
         const uint32_t p0 = prmt(w[i], kMagic, 0x4140);   // bytes 4i, 4i+1
         const uint32_t p1 = prmt(w[i], kMagic, 0x4342);   // bytes 4i+2, 4i+3
-        lo[2 * i] = hmul2_u(hadd2_u(p0 & 0xFF0FFF0Fu, kNeg1032), ds2);
-        lo[2 * i + 1] = hmul2_u(hadd2_u(p1 & 0xFF0FFF0Fu, kNeg1032), ds2);
-        hi[2 * i] = hmul2_u(hfma2_u(p0 & 0xFFF0FFF0u, kSixteenth, kNeg72), ds2);
-        hi[2 * i + 1] = hmul2_u(hfma2_u(p1 & 0xFFF0FFF0u, kSixteenth, kNeg72), ds2);
+        o[2 * i] = hmul2_u(hadd2_u(p0 & 0xFF0FFF0Fu, kNeg1032), ds2);              // elements 4i, 4i+1
+        o[2 * i + 1] = hmul2_u(hadd2_u(p1 & 0xFF0FFF0Fu, kNeg1032), ds2);          // 4i+2, 4i+3
+        o[8 + 2 * i] = hmul2_u(hfma2_u(p0 & 0xFFF0FFF0u, kSixteenth, kNeg72), ds2);     // 16+4i, +1
+        o[8 + 2 * i + 1] = hmul2_u(hfma2_u(p1 & 0xFFF0FFF0u, kSixteenth, kNeg72), ds2); // 16+4i+2, +3
     }
-    sts128(row_addr + (((g0 + 0) ^ rsw) << 4), lo[0], lo[1], lo[2], lo[3]);
-    sts128(row_addr + (((g0 + 1) ^ rsw) << 4), lo[4], lo[5], lo[6], lo[7]);
-    sts128(row_addr + (((g0 + 2) ^ rsw) << 4), hi[0], hi[1], hi[2], hi[3]);
-    sts128(row_addr + (((g0 + 3) ^ rsw) << 4), hi[4], hi[5], hi[6], hi[7]);
 }
 
-// Q8: 16 signed code bytes (elements e .. e+15) as fp16 q * ds into two
-// granules: (byte ^ 0x80) = q + 128, (1024 + q + 128) - 1152 = q exactly.
-__device__ __forceinline__ void dequant_q8_half(uint4 c, uint32_t ds2, uint32_t row_addr, int g,
-                                                int rsw)
+// Q8: 16 signed code bytes (elements e .. e+15) as fp16 q * ds into o[0..7]
+// in element order: (byte ^ 0x80) = q + 128, (1024 + q + 128) - 1152 = q
+// exactly.
+__device__ __forceinline__ void dequant_q8_half(uint4 c, uint32_t ds2, uint32_t *o)
 {
     const uint32_t w[4] = {c.x ^ 0x80808080u, c.y ^ 0x80808080u, c.z ^ 0x80808080u, c.w ^ 0x80808080u};
-    uint32_t o[8];
 #pragma unroll
     for (int i = 0; i < 4; i++) {
         o[2 * i] = hmul2_u(hadd2_u(prmt(w[i], kMagic, 0x4140), kNeg1152), ds2);
         o[2 * i + 1] = hmul2_u(hadd2_u(prmt(w[i], kMagic, 0x4342), kNeg1152), ds2);
     }
-    sts128(row_addr + (((g + 0) ^ rsw) << 4), o[0], o[1], o[2], o[3]);
-    sts128(row_addr + (((g + 1) ^ rsw) << 4), o[4], o[5], o[6], o[7]);
 }
 
 // The CTA owning unit x under the balanced split of U units over G CTAs
@@ -290,7 +339,7 @@ template <int FMT, int NB>
 __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_constant__ Args a)
 {
     using VF = VFmt<FMT>;
-    constexpr int CS = VF::kCS;
+    constexpr int CS = ring_slots<FMT, NB>();
     constexpr int CB = VF::kCodeBytes;
     constexpr int XB = NB * 128;   // x bytes per sub-stage
     constexpr int SLOT = slot_bytes<FMT, NB>();
@@ -306,7 +355,6 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
 
     uint8_t *sbase = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t ring_s = smem_u32(sbase);                 // CS unit slots (1024-aligned)
-    const uint32_t a_s = ring_s + CS * SLOT;                 // AS A tiles
     static_assert(SLOT % 1024 == 0, "unit slots keep the 1024-byte alignment of the swizzled boxes");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cta = blockIdx.x;
@@ -315,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
     if (threadIdx.x == 0) {
         for (int i = 0; i < CS; i++) {
             mbar_init(smem_u32(&bar_cfull[i]), 1);
-            mbar_init(smem_u32(&bar_cempty[i]), 9);          // the 8 dequant warps + the MMAs' commit
+            mbar_init(smem_u32(&bar_cempty[i]), 8 * kDqGroups + 1);   // every dequant warp + the MMAs' commit
         }
         for (int i = 0; i < AS; i++) {
             mbar_init(smem_u32(&bar_afull[i]), 8);           // the 8 dequant warps
@@ -326,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
             mbar_init(smem_u32(&bar_accempty[i]), 4);        // the 4 epilogue warps
         }
         for (int i = 0; i < kShiftRing; i++) {
-            mbar_init(smem_u32(&bar_shift[i]), 8);           // the 8 dequant warps
+            mbar_init(smem_u32(&bar_shift[i]), 4);           // the 4 dequant warps of block 0
             mbar_init(smem_u32(&bar_shift_free[i]), 4);      // the 4 epilogue warps
         }
         mbar_init(smem_u32(&bar_done), 1);
@@ -336,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(&tmem_base_s), 2 * 32);          // two accumulators of up to 32 columns
+        tmem_alloc(smem_u32(&tmem_base_s), kTmemCols);       // accumulators + the A ring (1 CTA / SM)
         tmem_relinquish();
     }
     tc_fence_before();
@@ -390,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                 }
 #pragma unroll
                 for (int j = 0; j < 4; j++)     // x: the unit's four 64-wide sub-tiles (L2-resident)
-                    tma_load_2d(dst + CB + j * XB, &a.tm_x, bar, ku * kUnitK + j * kSubK, 0, pol_x);
+                    tma_load_2d(dst + CB + j * XB, &a.tm_x, bar, ku * kUnitK + j * kXK, 0, pol_x);
                 tma_load_2d(dst + CB + 4 * XB, &a.tm_scales, bar, ku * 8, tile * TM, pol);
             }
             // Drain: every load issued lands before the CTA may exit.
@@ -427,13 +475,14 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                             break;
                         }
                         tc_fence_after();
-                        const uint64_t ad = desc_k_sw128(a_s + slot * kABytes);
-                        const uint64_t bd = desc_k_sw128(ring_s + cslot * SLOT + CB + j * XB);
+                        const uint32_t at = tmem + (uint32_t)(kAccCols + slot * kACols);
 #pragma unroll
                         for (int kk = 0; kk < kSubK / 16; kk++) {
-                            // K step of 16 fp16 = 32 bytes along the swizzled row
-                            umma_f16(d_tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
-                                     (first && kk == 0) ? 0u : 1u);
+                            // K step of 16: 8 TMEM columns of A; x tile 2 j + kk / 4, 32
+                            // bytes a step along its swizzled rows
+                            const uint64_t bd = desc_k_sw128(ring_s + cslot * SLOT + CB + (2 * j + kk / 4) * XB);
+                            umma_f16_ts(d_tmem, at + (uint32_t)(8 * kk), bd + (uint64_t)(2 * (kk % 4)), idesc,
+                                        (first && kk == 0) ? 0u : 1u);
                         }
                         first = false;
                         umma_commit(smem_u32(&bar_aempty[slot]));
@@ -546,12 +595,15 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
         }
     } else if (warp >= kDequantWarp0) {
         // ------------------------------------------------ dequantisation ----
-        // Thread pair (2r, 2r+1) of a warp serves row r: block h = t & 1 of
-        // each 64-weight sub-stage.  Both halves of a row sit in one warp, so
-        // the row's scale maximum is one shuffle (no CTA barrier).
-        const int t = threadIdx.x - kDequantWarp0 * 32;   // 0 .. 255
-        const int r = t >> 1, h = t & 1;                   // row, block of the sub-stage
+        // Warp w writes TMEM lanes 32 (w % 4) .. + 31, so warp w serves rows
+        // r = 32 (w % 4) + lane, block h = (w - 8) / 4 of each 64-weight
+        // sub-stage: a thread turns its (row, block) into 32 fp16 weights and
+        // stores them as 16 TMEM columns of its lane.
+        const int q = warp & 3, h = ((warp - kDequantWarp0) >> 2) & 1;
+        const int grp = (warp - kDequantWarp0) >> 3;       // takes the sub-stages i with i % kDqGroups == grp
+        const int r = 32 * q + lane;                       // row within the tile
         const int rsw = r & 7;                             // the 128-byte swizzle's XOR
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
         int i = 0, n = 0, seg = 0;
         bool ok = true;
         for (int u = u0; u < u1 && ok; seg++) {
@@ -560,19 +612,26 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
             const int row = tile * TM + r;
             // Row shift for this segment: the largest scale of the row over
             // the segment's units (the bytes the ring is about to bring in;
-            // read here directly, 16 bytes a unit).
+            // read here directly, 16 bytes a unit, four units' loads at a time).
             unsigned m = 0;
             if (row < a.N) {
                 const uint16_t *srow = a.scales + (size_t)row * a.ldS;
-                for (int uu = u + h; uu < uend; uu += 2) {
-                    const uint4 s8 = __ldg(reinterpret_cast<const uint4 *>(srow + (size_t)(uu % a.KU) * 8));
-                    const uint32_t sv[4] = {s8.x, s8.y, s8.z, s8.w};
+                for (int u4 = u; u4 < uend; u4 += 4) {
+                    uint4 s8[4];
 #pragma unroll
                     for (int k = 0; k < 4; k++)
-                        m = max(m, max(sv[k] & 0x7FFFu, (sv[k] >> 16) & 0x7FFFu));
+                        s8[k] = u4 + k < uend
+                                    ? __ldg(reinterpret_cast<const uint4 *>(srow + (size_t)((u4 + k) % a.KU) * 8))
+                                    : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        const uint32_t sv[4] = {s8[k].x, s8[k].y, s8[k].z, s8[k].w};
+#pragma unroll
+                        for (int e = 0; e < 4; e++)
+                            m = max(m, max(sv[e] & 0x7FFFu, (sv[e] >> 16) & 0x7FFFu));
+                    }
                 }
             }
-            m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
             m = min(m, 0x7BFFu);                               // largest finite fp16
             int s = 0;
             {
@@ -583,14 +642,15 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                 if (top > 0.f)
                     s = 141 - ((__float_as_int(top) >> 23) & 0xFF);
             }
-            // (the slot's previous segment, seg - 4, must have been read)
-            if (!wait(bar_shift_free[seg % kShiftRing], ((seg / kShiftRing) & 1) ^ 1))
-                break;
-            if (h == 0)
+            if (h == 0 && grp == 0) {
+                // (the slot's previous segment, seg - 4, must have been read)
+                if (!wait(bar_shift_free[seg % kShiftRing], ((seg / kShiftRing) & 1) ^ 1))
+                    break;
                 shift_s[seg % kShiftRing][r] = s;
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(smem_u32(&bar_shift[seg % kShiftRing]));
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(smem_u32(&bar_shift[seg % kShiftRing]));
+            }
             const float two_s = __int_as_float((127 + s) << 23);
             for (; u < uend && ok; u++, n++) {
                 const int cslot = n % CS;
@@ -602,31 +662,41 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                 const uint32_t srow_s = ring_s + cslot * SLOT + CB + 4 * XB + r * 16;
                 const int ns = nsub(u);
                 for (int j = 0; j < ns; j++, i++) {
+                    if (i % kDqGroups != grp)
+                        continue;
                     const int slot = i % AS;
                     if (!wait(bar_aempty[slot], ((i / AS) & 1) ^ 1)) {
                         ok = false;
                         break;
                     }
-                    const int blk = 2 * j + h;                        // block of the unit (0..7)
-                    unsigned short dbits;
-                    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(dbits) : "r"(srow_s + 2 * blk));
-                    const float ds = __half2float(__ushort_as_half(dbits)) * two_s;
-                    const __half2 ds2h = __float2half2_rn(ds);
-                    uint32_t ds2;
-                    memcpy(&ds2, &ds2h, 4);
-                    const uint32_t arow = a_s + slot * kABytes + r * 128;
-                    if constexpr (FMT == 4) {
-                        const uint4 c = lds128_u32(crow + ((blk ^ rsw) << 4));
-                        dequant_q4_block(c, ds2, arow, 4 * h, rsw);
-                    } else {
-                        const uint32_t box = crow + (blk >> 2) * (TM * 128);
-                        const int g = 2 * (blk & 3);
-                        const uint4 c0 = lds128_u32(box + ((g ^ rsw) << 4));
-                        const uint4 c1 = lds128_u32(box + (((g + 1) ^ rsw) << 4));
-                        dequant_q8_half(c0, ds2, arow, 4 * h, rsw);
-                        dequant_q8_half(c1, ds2, arow, 4 * h + 2, rsw);
+                    tc_fence_after();
+                    // this thread's two blocks of the sub-stage: 4 j + 2 h and
+                    // 4 j + 2 h + 1 (64 consecutive weights, 32 TMEM columns)
+                    uint32_t o[32];
+#pragma unroll
+                    for (int e = 0; e < 2; e++) {
+                        const int blk = 4 * j + 2 * h + e;               // block of the unit (0..7)
+                        unsigned short dbits;
+                        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(dbits) : "r"(srow_s + 2 * blk));
+                        const float ds = __half2float(__ushort_as_half(dbits)) * two_s;
+                        const __half2 ds2h = __float2half2_rn(ds);
+                        uint32_t ds2;
+                        memcpy(&ds2, &ds2h, 4);
+                        uint32_t (&oe)[16] = *reinterpret_cast<uint32_t (*)[16]>(o + 16 * e);
+                        if constexpr (FMT == 4) {
+                            const uint4 c = lds128_u32(crow + ((blk ^ rsw) << 4));
+                            dequant_q4_block(c, ds2, oe);
+                        } else {
+                            const uint32_t box = crow + (blk >> 2) * (TM * 128);
+                            const int g = 2 * (blk & 3);
+                            const uint4 c0 = lds128_u32(box + ((g ^ rsw) << 4));
+                            const uint4 c1 = lds128_u32(box + (((g + 1) ^ rsw) << 4));
+                            dequant_q8_half(c0, ds2, oe);
+                            dequant_q8_half(c1, ds2, oe + 8);
+                        }
                     }
-                    fence_proxy_async_smem();     // generic-proxy stores -> the MMA's async-proxy reads
+                    tmem_st32(lane_base + (uint32_t)(kAccCols + slot * kACols + 32 * h), o);
+                    tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
                         mbar_arrive(smem_u32(&bar_afull[slot]));
@@ -644,7 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
     __syncthreads();
     tc_fence_after();
     if (warp == 1)
-        tmem_dealloc(tmem, 2 * 32);
+        tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace vg
@@ -702,7 +772,7 @@ int32_t verify_launch(const bq_qmat *W, const uint16_t *x, int32_t B, float *y, 
     const uint32_t sbox[2] = {8u, (uint32_t)vg::TM};
     const uint64_t xdims[2] = {(uint64_t)K, (uint64_t)B};
     const uint64_t xstr[1] = {(uint64_t)K * 2};
-    const uint32_t xbox[2] = {(uint32_t)vg::kSubK, (uint32_t)NB};
+    const uint32_t xbox[2] = {(uint32_t)vg::kXK, (uint32_t)NB};
     if (!encode_tensor_map(&a.tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, W->codes, cdims, cstr, cbox,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
         !encode_tensor_map(&a.tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, W->scales, sdims, sstr,
