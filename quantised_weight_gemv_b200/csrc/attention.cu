@@ -498,25 +498,15 @@ __global__ void __launch_bounds__(kThreads, 2) attn_decode_kernel(const __grid_c
                 auto part = [&](int c) {
                     return a.partials + ((size_t)c * 2 + (c == cf ? cf_slot : 0)) * kPartFloats;
                 };
-                // Loads are issued in batches (8, then 4 CTAs at a time) so a
-                // merge of many partials costs a few L2 round trips, not one
-                // per partial; the sums still run in CTA order.
-                float M = -INFINITY;
+                // One pass over the partials in CTA order, 8 at a time (their loads
+                // in flight together), keeping a running maximum: a merge of
+                // many partials costs a few L2 round trips, not one per partial.
+                float M = -INFINITY, Ls = 0.f, os[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int c0 = cf; c0 <= cl; c0 += 8) {
-                    float mv[8];
+                    float mc[8], lc[8];
+                    float4 oc[8];
 #pragma unroll
-                    for (int k = 0; k < 8; k++)
-                        mv[k] = c0 + k <= cl ? __ldcg(part(c0 + k) + j) : -INFINITY;
-#pragma unroll
-                    for (int k = 0; k < 8; k++)
-                        M = fmaxf(M, mv[k]);
-                }
-                float Ls = 0.f, os[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int c0 = cf; c0 <= cl; c0 += 4) {
-                    float mc[4], lc[4];
-                    float4 oc[4];
-#pragma unroll
-                    for (int k = 0; k < 4; k++) {
+                    for (int k = 0; k < 8; k++) {
                         if (c0 + k <= cl) {
                             const float *pc = part(c0 + k);
                             mc[k] = __ldcg(pc + j);
@@ -528,15 +518,28 @@ __global__ void __launch_bounds__(kThreads, 2) attn_decode_kernel(const __grid_c
                             oc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
                         }
                     }
+                    float Mb = M;
 #pragma unroll
-                    for (int k = 0; k < 4; k++) {
-                        const float f = mc[k] == -INFINITY ? 0.f : ex2(mc[k] - M);
+                    for (int k = 0; k < 8; k++)
+                        Mb = fmaxf(Mb, mc[k]);
+                    if (Mb == -INFINITY)
+                        continue;                        // nothing valid so far
+                    const float fr = M == -INFINITY ? 0.f : ex2(M - Mb);   // rescale what was summed
+                    Ls *= fr;
+                    os[0] *= fr;
+                    os[1] *= fr;
+                    os[2] *= fr;
+                    os[3] *= fr;
+#pragma unroll
+                    for (int k = 0; k < 8; k++) {
+                        const float f = mc[k] == -INFINITY ? 0.f : ex2(mc[k] - Mb);
                         Ls += f * lc[k];
                         os[0] += f * oc[k].x;
                         os[1] += f * oc[k].y;
                         os[2] += f * oc[k].z;
                         os[3] += f * oc[k].w;
                     }
+                    M = Mb;
                 }
                 if (j < a.G) {
                     const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
