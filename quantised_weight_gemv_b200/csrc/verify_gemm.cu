@@ -28,22 +28,27 @@
 //               of 4-6 unit slots, so x arrives units ahead of its MMAs;
 //   warp 1      allocates TMEM (512 columns: two accumulators and a ring of
 //               6 dequantised A sub-stages), and one thread issues the MMAs:
-//               per 128-weight sub-stage, 8 x tcgen05.mma (M 128, N NB, K 16,
-//               fp16 in, fp32 accumulation) with A read from TMEM and x from a
-//               shared-memory descriptor, then tcgen05.commit to free the A
-//               slot (after a unit's last one, also the unit's ring slot);
+//               per unit one wait (every dequant warp has stored the unit's
+//               A), then per 128-weight sub-stage 8 x tcgen05.mma (M 128, N
+//               NB, K 16, fp16 in, fp32 accumulation) with A read from TMEM
+//               and x from a shared-memory descriptor, and tcgen05.commit to
+//               free the A slot (after a unit's last one, also its ring slot);
+//   warps 2-3   row shifts (below) of each segment, a few segments ahead;
 //   warps 4-7   epilogue: tcgen05.ld of the accumulator, one thread per row;
 //   warps 8-15  dequantisation: warp w serves TMEM lanes 32 (w % 4) .. + 31
 //               (rows) and one half of each sub-stage; a thread turns two
 //               blocks of its row (32 or 64 code bytes and two fp16 scales)
 //               into 64 fp16 weights d (q - z) 2^s and writes them as 32 TMEM
-//               columns with tcgen05.st.
+//               columns with tcgen05.st.  At the start they also compute the
+//               first two segments' row shifts, one row each.
 // A lives in TMEM, not shared memory: a 128 x 16 fp16 A operand is 4 KB, and
 // reading it from shared memory for every K16 step (plus writing it there
 // first) would need more shared-memory bandwidth than the Q4 stream leaves.
-// Measured (one CTA per SM): a dependent tcgen05.mma of M 128 x N 32 x K 16
-// issues about every 71 cycles, so the MMA side caps a Q4 verification step
-// near 0.7 of HBM; a deeper split into more dequant warps measured slower.
+// Measured on B200: a tcgen05.mma of M 128 x N <= 64 x K 16 takes a fixed
+// ~70-130 cycles of the tensor pipe whatever N (N = 256 takes ~130), so the
+// MMA side caps a Q4 verification step near 0.5 of HBM; an mbarrier wait in
+// the issuing thread stalls the pipe for its whole latency (the MMA queue is
+// short), hence one wait per 16 MMAs.
 
 // Rounding.  The decode GEMV keeps codes exact and scales each block's sum;
 // a tile accumulated over many blocks cannot, so the A tile holds each weight
@@ -262,6 +267,12 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
+__device__ __forceinline__ int ld_acquire_gpu_int(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -344,9 +355,9 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
     constexpr int XB = NB * 128;   // x bytes per sub-stage
     constexpr int SLOT = slot_bytes<FMT, NB>();
     extern __shared__ uint8_t smem_raw[];
-    __shared__ alignas(8) uint64_t bar_cfull[CS], bar_cempty[CS], bar_afull[AS], bar_aempty[AS],
+    __shared__ alignas(8) uint64_t bar_cfull[CS], bar_cempty[CS], bar_ufull[AS], bar_aempty[AS],
         bar_accfull[2], bar_accempty[2], bar_shift[kShiftRing],
-        bar_shift_free[kShiftRing], bar_done,
+        bar_shift_free[kShiftRing], bar_done, bar_pre,
         bar_epi_a, bar_epi_b;
     __shared__ uint32_t tmem_base_s;
     __shared__ int shift_s[kShiftRing][TM];
@@ -366,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
             mbar_init(smem_u32(&bar_cempty[i]), 8 * kDqGroups + 1);   // every dequant warp + the MMAs' commit
         }
         for (int i = 0; i < AS; i++) {
-            mbar_init(smem_u32(&bar_afull[i]), 8);           // the 8 dequant warps
+            mbar_init(smem_u32(&bar_ufull[i]), 8 * kDqGroups);   // every dequant warp, once a unit
             mbar_init(smem_u32(&bar_aempty[i]), 1);          // tcgen05.commit
         }
         for (int i = 0; i < 2; i++) {
@@ -374,10 +385,11 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
             mbar_init(smem_u32(&bar_accempty[i]), 4);        // the 4 epilogue warps
         }
         for (int i = 0; i < kShiftRing; i++) {
-            mbar_init(smem_u32(&bar_shift[i]), 4);           // the 4 dequant warps of block 0
-            mbar_init(smem_u32(&bar_shift_free[i]), 4);      // the 4 epilogue warps
+            mbar_init(smem_u32(&bar_shift[i]), 2);           // the row-shift warps 2-3
+            mbar_init(smem_u32(&bar_shift_free[i]), 4 + 8 * kDqGroups);   // epilogue + dequant warps
         }
         mbar_init(smem_u32(&bar_done), 1);
+        mbar_init(smem_u32(&bar_pre), 8 * kDqGroups);        // dequant warps: first two segments' shifts
         mbar_init(smem_u32(&bar_epi_a), 128);                // the epilogue's split-tile handshake
         mbar_init(smem_u32(&bar_epi_b), 1);
         abort_s = 0;
@@ -416,6 +428,44 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
         return min(kUnitK / kSubK, (a.K - ku * kUnitK + kSubK - 1) / kSubK);
     };
 
+    // Largest |scale| (fp16 bits without the sign) of one row of a tile
+    // over n units from ub (16 bytes a unit), sixteen loads in flight.
+    auto row_scale_max = [&](int tile, int ub, int n, int r) -> unsigned {
+        const int row = tile * TM + r;
+        unsigned m = 0u;
+        if (row >= a.N)
+            return m;
+        const uint16_t *srow = a.scales + (size_t)row * a.ldS;
+        for (int k0 = 0; k0 < n; k0 += 16) {
+            uint4 v[16];
+#pragma unroll
+            for (int k = 0; k < 16; k++)
+                v[k] = k0 + k < n ? __ldg(reinterpret_cast<const uint4 *>(srow + (size_t)((ub + k0 + k) % a.KU) * 8))
+                                  : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int k = 0; k < 16; k++) {
+                const uint32_t sv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+                for (int e = 0; e < 4; e++)
+                    m = max(m, max(sv[e] & 0x7FFFu, (sv[e] >> 16) & 0x7FFFu));
+            }
+        }
+        return m;
+    };
+    // The row shift s for a row whose largest scale has fp16 bits m: the
+    // largest |d (q - z)| (8 dmax for Q4, 127 dmax for Q8) times 2^s lands
+    // in [2^14, 2^15).
+    auto shift_of = [](unsigned m) -> int {
+        m = min(m, 0x7BFFu);                                  // largest finite fp16
+        const float top = __half2float(__ushort_as_half((unsigned short)m)) * (FMT == 4 ? 8.0f : 127.0f);
+        return top > 0.f ? 141 - ((__float_as_int(top) >> 23) & 0xFF) : 0;
+    };
+    // The CTA's first two segments: tile t0 from u0 (n0 units), then the
+    // start of tile t0 + 1 (n1 units, 0 if none).
+    const int pre_t0 = u0 / a.KU;
+    const int pre_e0 = min(u1, (pre_t0 + 1) * a.KU);
+    const int pre_n1 = pre_e0 < u1 ? min(u1, (pre_t0 + 2) * a.KU) - pre_e0 : 0;
+
     if (warp == 0) {
         // ---------------------------------------------- codes + scales TMA --
         if (lane == 0) {
@@ -423,6 +473,10 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
             const uint64_t pol_x = policy_evict_normal();
             int n = 0;
             for (int u = u0; u < u1 && !aborted(); u++, n++) {
+                // after the first unit, let the first segments' scale reads
+                // land before the weight stream takes the memory system
+                if (n == 1 && !wait(bar_pre, 0))
+                    break;
                 const int slot = n % CS;
                 if (!wait(bar_cempty[slot], ((n / CS) & 1) ^ 1))
                     break;
@@ -464,17 +518,19 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                 for (; u < uend && ok; u++, nu++) {
                     const int ns = nsub(u);
                     const int cslot = nu % CS;
-                    if (!wait(bar_cfull[cslot], (nu / CS) & 1)) {     // this unit's x has landed
+                    // One wait a unit: every dequant warp has stored the unit's A
+                    // (all its sub-stages).  They arrive only after seeing the
+                    // unit's loads land, so x is in place too.  (A wait in this
+                    // thread stalls the tensor pipe for its whole latency: the
+                    // MMA queue is short.)  The dequant runs at most AS
+                    // sub-stages, so at most AS units, ahead: AS barriers.
+                    if (!wait(bar_ufull[nu % AS], (nu / AS) & 1)) {
                         ok = false;
                         break;
                     }
+                    tc_fence_after();
                     for (int j = 0; j < ns; j++, i++) {
                         const int slot = i % AS;
-                        if (!wait(bar_afull[slot], (i / AS) & 1)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
                         const uint32_t at = tmem + (uint32_t)(kAccCols + slot * kACols);
 #pragma unroll
                         for (int kk = 0; kk < kSubK / 16; kk++) {
@@ -499,6 +555,36 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
             umma_commit(smem_u32(&bar_done));
             (void)mbar_wait_bounded(smem_u32(&bar_done), 0);
         }
+    } else if (warp == 2 || warp == 3) {
+        // --------------------------------------------------- row shifts ----
+        // Each segment's row shifts, up to kShiftRing segments ahead of the
+        // dequantisation.  The first two segments' shifts are computed by the
+        // dequantisation warps at the start (they have nothing else to do
+        // then; one row and segment a thread); warps 2-3 publish them, then
+        // compute the later segments' (thread t: rows t and t + 64).
+        const int t = threadIdx.x - 64;
+        bool ok = wait(bar_pre, 0);
+        if (ok && lane == 0) {
+            mbar_arrive(smem_u32(&bar_shift[0]));
+            if (pre_n1 > 0)
+                mbar_arrive(smem_u32(&bar_shift[1]));
+        }
+        int seg = 2;
+        for (int u = pre_e0 + pre_n1; u < u1 && ok; seg++) {
+            const int tile = u / a.KU;
+            const int uend = min(u1, (tile + 1) * a.KU);
+            const unsigned m0 = row_scale_max(tile, u, uend - u, t);
+            const unsigned m1 = row_scale_max(tile, u, uend - u, t + 64);
+            // (the slot's segment seg - kShiftRing must have been read)
+            if (!wait(bar_shift_free[seg % kShiftRing], ((seg / kShiftRing) & 1) ^ 1))
+                break;
+            shift_s[seg % kShiftRing][t] = shift_of(m0);
+            shift_s[seg % kShiftRing][t + 64] = shift_of(m1);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&bar_shift[seg % kShiftRing]));
+            u = uend;
+        }
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
         // ----------------------------------------------------- epilogue ----
         // (Warp w reads TMEM lanes 32 (w % 4) .. + 31: warps 4-7 cover all.)
@@ -506,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
         // role that gave up on a timeout cannot leave the others blocked.
         const int q = warp - kEpiWarp0;          // TMEM lanes 32q .. 32q + 31
         const int r = 32 * q + lane;             // row within the tile
-        int seg = 0, nsplit = 0;
+        int seg = 0, nsplit = 0, nepa = 0, nepb = 0;   // split tiles; phases of the handshake barriers
         for (int u = u0; u < u1; seg++) {
             const int tile = u / a.KU;
             u = min(u1, (tile + 1) * a.KU);
@@ -543,52 +629,94 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                 }
                 continue;
             }
-            // Tile split across CTAs: this CTA's partial to its slot (0: the
-            // tile of its first unit, 1: of its last), a counted arrival; the
-            // last CTA adds all partials in CTA order and resets the counter.
-            const int my_slot = (tile == u0 / a.KU) ? 0 : 1;
-            float4 *dst = reinterpret_cast<float4 *>(a.partials + (((size_t)cta * 2 + my_slot) * TM + r) * 32);
-#pragma unroll
-            for (int b4 = 0; b4 < NB / 4; b4++)
-                __stcg(dst + b4, make_float4(v[4 * b4], v[4 * b4 + 1], v[4 * b4 + 2], v[4 * b4 + 3]));
-            __threadfence();
-            mbar_arrive(smem_u32(&bar_epi_a));
+            // Tile split across CTAs (cf .. cl).  Whichever CTA completes the
+            // tile last adds every part in CTA order (its own from registers),
+            // so the sum does not depend on which CTA that is.  It usually
+            // knows at once: the CTA holding the tile's first units reaches
+            // them at the end of its range, after the others (which did theirs
+            // at the start of theirs) have published.  So first an acquire
+            // load of the tile's arrival count; only if some part is still
+            // missing does this CTA publish its partial (slot 0: the tile of
+            // its first unit, 1: of its last) and count its arrival, the
+            // arrival that completes the count doing the sum.
+            // Handshake (all bounded mbarriers): epi_b (1 arrival: thread 0
+            // has put a count in epi_old) and epi_a (128: every thread is done
+            // with epi_old, or has stored its partial).  Thread 0 writes
+            // epi_old only after an epi_a phase, so neither barrier gets more
+            // than one phase ahead of a waiter.
+            const int others = cl - cf;
             if (r == 0) {
-                if (!wait(bar_epi_a, nsplit & 1))
+                if (nsplit > 0 && !wait(bar_epi_a, nepa++ & 1))
                     break;
-                epi_old = atom_add_acq_rel_gpu(a.counters + tile, 1);
+                epi_old = ld_acquire_gpu_int(a.counters + tile);
                 mbar_arrive(smem_u32(&bar_epi_b));
             }
-            if (!wait(bar_epi_b, nsplit & 1))
+            if (!wait(bar_epi_b, nepb++ & 1))
                 break;
+            int seen = epi_old;
             nsplit++;
-            if (epi_old != cl - cf)
+            bool published = false;
+            const int my_slot = (tile == u0 / a.KU) ? 0 : 1;
+            if (seen != others) {
+                float4 *dst = reinterpret_cast<float4 *>(a.partials + (((size_t)cta * 2 + my_slot) * TM + r) * 32);
+#pragma unroll
+                for (int b4 = 0; b4 < NB / 4; b4++)
+                    __stcg(dst + b4, make_float4(v[4 * b4], v[4 * b4 + 1], v[4 * b4 + 2], v[4 * b4 + 3]));
+                __threadfence();
+                mbar_arrive(smem_u32(&bar_epi_a));
+                if (r == 0) {
+                    if (!wait(bar_epi_a, nepa++ & 1))
+                        break;
+                    epi_old = atom_add_acq_rel_gpu(a.counters + tile, 1);
+                    mbar_arrive(smem_u32(&bar_epi_b));
+                }
+                if (!wait(bar_epi_b, nepb++ & 1))
+                    break;
+                seen = epi_old;
+                published = true;
+            }
+            mbar_arrive(smem_u32(&bar_epi_a));      // done with epi_old
+            if (seen != others)
                 continue;
-            __threadfence();
+            float t[NB];
 #pragma unroll
             for (int b = 0; b < NB; b++)
-                v[b] = 0.f;
+                t[b] = 0.f;
             for (int c = cf; c <= cl; c++) {
                 const int cu0 = (int)((long long)c * a.U / a.G);
                 const int sl = (tile == cu0 / a.KU) ? 0 : 1;
                 float4 *src = reinterpret_cast<float4 *>(a.partials + (((size_t)c * 2 + sl) * TM + r) * 32);
+                if (c == cta) {
+#pragma unroll
+                    for (int b = 0; b < NB; b++)
+                        t[b] += v[b];
+                    if (published) {
+#pragma unroll
+                        for (int b4 = 0; b4 < NB / 4; b4++)
+                            __stcg(src + b4, make_float4(0.f, 0.f, 0.f, 0.f));
+                    }
+                    continue;
+                }
+                float4 pv[NB / 4];
+#pragma unroll
+                for (int b4 = 0; b4 < NB / 4; b4++)
+                    pv[b4] = __ldcg(src + b4);
+                // cleared once read: the workspace is all-zero again when the
+                // call ends, so calls of any shape may share it
 #pragma unroll
                 for (int b4 = 0; b4 < NB / 4; b4++) {
-                    const float4 p = __ldcg(src + b4);
-                    // cleared once read: the workspace is all-zero again when
-                    // the call ends, so calls of any shape may share it
                     __stcg(src + b4, make_float4(0.f, 0.f, 0.f, 0.f));
-                    v[4 * b4] += p.x;
-                    v[4 * b4 + 1] += p.y;
-                    v[4 * b4 + 2] += p.z;
-                    v[4 * b4 + 3] += p.w;
+                    t[4 * b4] += pv[b4].x;
+                    t[4 * b4 + 1] += pv[b4].y;
+                    t[4 * b4 + 2] += pv[b4].z;
+                    t[4 * b4 + 3] += pv[b4].w;
                 }
             }
             if (row < a.N) {
 #pragma unroll
                 for (int b = 0; b < NB; b++)
                     if (b < a.B)
-                        a.y[(size_t)b * a.N + row] = v[b];
+                        a.y[(size_t)b * a.N + row] = t[b];
             }
             if (r == 0)
                 a.counters[tile] = 0;
@@ -604,53 +732,29 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
         const int r = 32 * q + lane;                       // row within the tile
         const int rsw = r & 7;                             // the 128-byte swizzle's XOR
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+        {
+            // the first two segments' row shifts: thread (j, row) of 256
+            const int tid = threadIdx.x - 32 * kDequantWarp0;
+            const int j = tid >> 7, rr = tid & (TM - 1);
+            if (tid < 2 * TM && (j == 0 || pre_n1 > 0))
+                shift_s[j][rr] = shift_of(j == 0 ? row_scale_max(pre_t0, u0, pre_e0 - u0, rr)
+                                                 : row_scale_max(pre_t0 + 1, pre_e0, pre_n1, rr));
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&bar_pre));
+        }
         int i = 0, n = 0, seg = 0;
         bool ok = true;
         for (int u = u0; u < u1 && ok; seg++) {
             const int tile = u / a.KU;
             const int uend = min(u1, (tile + 1) * a.KU);
-            const int row = tile * TM + r;
-            // Row shift for this segment: the largest scale of the row over
-            // the segment's units (the bytes the ring is about to bring in;
-            // read here directly, 16 bytes a unit, four units' loads at a time).
-            unsigned m = 0;
-            if (row < a.N) {
-                const uint16_t *srow = a.scales + (size_t)row * a.ldS;
-                for (int u4 = u; u4 < uend; u4 += 4) {
-                    uint4 s8[4];
-#pragma unroll
-                    for (int k = 0; k < 4; k++)
-                        s8[k] = u4 + k < uend
-                                    ? __ldg(reinterpret_cast<const uint4 *>(srow + (size_t)((u4 + k) % a.KU) * 8))
-                                    : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                    for (int k = 0; k < 4; k++) {
-                        const uint32_t sv[4] = {s8[k].x, s8[k].y, s8[k].z, s8[k].w};
-#pragma unroll
-                        for (int e = 0; e < 4; e++)
-                            m = max(m, max(sv[e] & 0x7FFFu, (sv[e] >> 16) & 0x7FFFu));
-                    }
-                }
-            }
-            m = min(m, 0x7BFFu);                               // largest finite fp16
-            int s = 0;
-            {
-                // the largest |d (q - z)| (8 dmax for Q4, 127 dmax for Q8)
-                // times 2^s lands in [2^14, 2^15)
-                const float dmax = __half2float(__ushort_as_half((unsigned short)m));
-                const float top = dmax * (FMT == 4 ? 8.0f : 127.0f);
-                if (top > 0.f)
-                    s = 141 - ((__float_as_int(top) >> 23) & 0xFF);
-            }
-            if (h == 0 && grp == 0) {
-                // (the slot's previous segment, seg - 4, must have been read)
-                if (!wait(bar_shift_free[seg % kShiftRing], ((seg / kShiftRing) & 1) ^ 1))
-                    break;
-                shift_s[seg % kShiftRing][r] = s;
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(smem_u32(&bar_shift[seg % kShiftRing]));
-            }
+            // This segment's row shift (warps 2-3 computed it ahead).
+            if (!wait(bar_shift[seg % kShiftRing], (seg / kShiftRing) & 1))
+                break;
+            const int s = shift_s[seg % kShiftRing][r];
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&bar_shift_free[seg % kShiftRing]));
             const float two_s = __int_as_float((127 + s) << 23);
             for (; u < uend && ok; u++, n++) {
                 const int cslot = n % CS;
@@ -696,16 +800,15 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                         }
                     }
                     tmem_st32(lane_base + (uint32_t)(kAccCols + slot * kACols + 32 * h), o);
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(smem_u32(&bar_afull[slot]));
                 }
                 if (!ok)
                     break;
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0)
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(&bar_ufull[n % AS]));
                     mbar_arrive(smem_u32(&bar_cempty[cslot]));
+                }
             }
         }
     }
