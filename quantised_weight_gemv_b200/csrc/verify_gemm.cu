@@ -460,11 +460,25 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
         const float top = __half2float(__ushort_as_half((unsigned short)m)) * (FMT == 4 ? 8.0f : 127.0f);
         return top > 0.f ? 141 - ((__float_as_int(top) >> 23) & 0xFF) : 0;
     };
-    // The CTA's first two segments: tile t0 from u0 (n0 units), then the
-    // start of tile t0 + 1 (n1 units, 0 if none).
-    const int pre_t0 = u0 / a.KU;
-    const int pre_e0 = min(u1, (pre_t0 + 1) * a.KU);
-    const int pre_n1 = pre_e0 < u1 ? min(u1, (pre_t0 + 2) * a.KU) - pre_e0 : 0;
+    // The CTA's segments (its units of one tile each) in processing order.
+    // A range that ends inside a tile shares that tile with the next CTA,
+    // which does the tile's other units at the start of its range; doing
+    // this CTA's part first too lets the tile's cross-CTA sum happen early,
+    // under later units, instead of at the end of both CTAs.  So the last
+    // segment goes first when it is a partial tile; the others keep order.
+    const int seg_t0 = u0 / a.KU;
+    const int seg_n = (u1 - 1) / a.KU - seg_t0 + 1;
+    const bool seg_rot = seg_n > 1 && u1 % a.KU != 0;
+    auto seg_range = [&](int k, int &us, int &ue) {
+        const int t = seg_t0 + (seg_rot ? (k == 0 ? seg_n - 1 : k - 1) : k);
+        us = max(u0, t * a.KU);
+        ue = min(u1, (t + 1) * a.KU);
+    };
+    // The first two segments (the second empty if there is none).
+    int pre_s0, pre_e0, pre_s1 = 0, pre_e1 = 0;
+    seg_range(0, pre_s0, pre_e0);
+    if (seg_n > 1)
+        seg_range(1, pre_s1, pre_e1);
 
     if (warp == 0) {
         // ---------------------------------------------- codes + scales TMA --
@@ -472,14 +486,22 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
             const uint64_t pol = policy_evict_first();
             const uint64_t pol_x = policy_evict_normal();
             int n = 0;
-            for (int u = u0; u < u1 && !aborted(); u++, n++) {
+            bool go = true;
+            for (int k = 0; k < seg_n && go; k++) {
+              int us, ue;
+              seg_range(k, us, ue);
+              for (int u = us; u < ue; u++, n++) {
                 // after the first unit, let the first segments' scale reads
                 // land before the weight stream takes the memory system
-                if (n == 1 && !wait(bar_pre, 0))
+                if (aborted() || (n == 1 && !wait(bar_pre, 0))) {
+                    go = false;
                     break;
+                }
                 const int slot = n % CS;
-                if (!wait(bar_cempty[slot], ((n / CS) & 1) ^ 1))
+                if (!wait(bar_cempty[slot], ((n / CS) & 1) ^ 1)) {
+                    go = false;
                     break;
+                }
                 const int tile = u / a.KU, ku = u % a.KU;
                 const uint32_t bar = smem_u32(&bar_cfull[slot]);
                 const uint32_t dst = ring_s + slot * SLOT;
@@ -494,6 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                 for (int j = 0; j < 4; j++)     // x: the unit's four 64-wide sub-tiles (L2-resident)
                     tma_load_2d(dst + CB + j * XB, &a.tm_x, bar, ku * kUnitK + j * kXK, 0, pol_x);
                 tma_load_2d(dst + CB + 4 * XB, &a.tm_scales, bar, ku * 8, tile * TM, pol);
+              }
             }
             // Drain: every load issued lands before the CTA may exit.
             for (int j = max(0, n - CS); j < n; j++)
@@ -503,19 +526,18 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
         // ---------------------------------------------------------- MMA ----
         if (lane == 0) {
             constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(NB >> 3) << 17) | ((uint32_t)(TM >> 4) << 24);
-            int i = 0, seg = 0, nu = 0;
-            int u = u0;
+            int i = 0, nu = 0;
             bool ok = true;
-            while (u < u1 && ok) {
-                const int tile = u / a.KU;
-                const int uend = min(u1, (tile + 1) * a.KU);
+            for (int seg = 0; seg < seg_n && ok; seg++) {
+                int us, uend;
+                seg_range(seg, us, uend);
                 const int buf = seg & 1;
                 if (!wait(bar_accempty[buf], ((seg >> 1) & 1) ^ 1))
                     break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(buf * 32);
                 bool first = true;
-                for (; u < uend && ok; u++, nu++) {
+                for (int u = us; u < uend && ok; u++, nu++) {
                     const int ns = nsub(u);
                     const int cslot = nu % CS;
                     // One wait a unit: every dequant warp has stored the unit's A
@@ -549,7 +571,6 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                 if (!ok)
                     break;
                 umma_commit(smem_u32(&bar_accfull[buf]));
-                seg++;
             }
             // Every MMA issued has completed before TMEM is freed.
             umma_commit(smem_u32(&bar_done));
@@ -566,13 +587,13 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
         bool ok = wait(bar_pre, 0);
         if (ok && lane == 0) {
             mbar_arrive(smem_u32(&bar_shift[0]));
-            if (pre_n1 > 0)
+            if (seg_n > 1)
                 mbar_arrive(smem_u32(&bar_shift[1]));
         }
-        int seg = 2;
-        for (int u = pre_e0 + pre_n1; u < u1 && ok; seg++) {
+        for (int seg = 2; seg < seg_n && ok; seg++) {
+            int u, uend;
+            seg_range(seg, u, uend);
             const int tile = u / a.KU;
-            const int uend = min(u1, (tile + 1) * a.KU);
             const unsigned m0 = row_scale_max(tile, u, uend - u, t);
             const unsigned m1 = row_scale_max(tile, u, uend - u, t + 64);
             // (the slot's segment seg - kShiftRing must have been read)
@@ -583,7 +604,6 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(smem_u32(&bar_shift[seg % kShiftRing]));
-            u = uend;
         }
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
         // ----------------------------------------------------- epilogue ----
@@ -592,10 +612,11 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
         // role that gave up on a timeout cannot leave the others blocked.
         const int q = warp - kEpiWarp0;          // TMEM lanes 32q .. 32q + 31
         const int r = 32 * q + lane;             // row within the tile
-        int seg = 0, nsplit = 0, nepa = 0, nepb = 0;   // split tiles; phases of the handshake barriers
-        for (int u = u0; u < u1; seg++) {
-            const int tile = u / a.KU;
-            u = min(u1, (tile + 1) * a.KU);
+        int nsplit = 0, nepa = 0, nepb = 0;   // split tiles; phases of the handshake barriers
+        for (int seg = 0; seg < seg_n; seg++) {
+            int us, ue;
+            seg_range(seg, us, ue);
+            const int tile = us / a.KU;
             const int buf = seg & 1;
             if (!wait(bar_shift[seg % kShiftRing], (seg / kShiftRing) & 1))
                 break;
@@ -736,18 +757,18 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
             // the first two segments' row shifts: thread (j, row) of 256
             const int tid = threadIdx.x - 32 * kDequantWarp0;
             const int j = tid >> 7, rr = tid & (TM - 1);
-            if (tid < 2 * TM && (j == 0 || pre_n1 > 0))
-                shift_s[j][rr] = shift_of(j == 0 ? row_scale_max(pre_t0, u0, pre_e0 - u0, rr)
-                                                 : row_scale_max(pre_t0 + 1, pre_e0, pre_n1, rr));
+            if (tid < 2 * TM && (j == 0 || seg_n > 1))
+                shift_s[j][rr] = shift_of(j == 0 ? row_scale_max(pre_s0 / a.KU, pre_s0, pre_e0 - pre_s0, rr)
+                                                 : row_scale_max(pre_s1 / a.KU, pre_s1, pre_e1 - pre_s1, rr));
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(smem_u32(&bar_pre));
         }
-        int i = 0, n = 0, seg = 0;
+        int i = 0, n = 0;
         bool ok = true;
-        for (int u = u0; u < u1 && ok; seg++) {
-            const int tile = u / a.KU;
-            const int uend = min(u1, (tile + 1) * a.KU);
+        for (int seg = 0; seg < seg_n && ok; seg++) {
+            int u, uend;
+            seg_range(seg, u, uend);
             // This segment's row shift (warps 2-3 computed it ahead).
             if (!wait(bar_shift[seg % kShiftRing], (seg / kShiftRing) & 1))
                 break;
