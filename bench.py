@@ -40,27 +40,34 @@ L2_FLUSH_BYTES = 256 << 20   # twice the B200's 126 MB L2
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
-    """sha256 over the CUDA sources; a profile's traffic figure is only used
-    while the kernels are byte-identical to the profiled ones."""
+def kernel_source_hash(unit: str = "stream_gemv.cu") -> str:
+    """sha256 over the sources one kernel is built from: its translation unit
+    under csrc/ plus every shared header (csrc/*.cuh, csrc/*.h, include/bq.h).
+    A profile's traffic figure is only used while these are byte-identical to
+    the profiled ones."""
     import glob
     import hashlib
+    csrc = os.path.join(ROOT, "quantised_weight_gemv_b200", "csrc")
+    files = [os.path.join(csrc, unit)] + sorted(glob.glob(os.path.join(csrc, "*.cuh")) +
+                                                glob.glob(os.path.join(csrc, "*.h")))
+    files.append(os.path.join(ROOT, "include", "bq.h"))
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "quantised_weight_gemv_b200", "csrc", "*"))):
+    for p in files:
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode())
             h.update(f.read())
     return h.hexdigest()
 
 
-def profiled_traffic(workload: str, engine: str):
+def profiled_traffic(workload: str, engine: str, unit: str = "stream_gemv.cu"):
     """DRAM bytes per launch (read + write) from a committed ncu summary under
     profiles/: a line `<!-- bench-traffic: workload=... engine=...
-    bytes_per_launch=... source_sha256=... -->`.  None when no summary
-    matches the current kernel sources."""
+    bytes_per_launch=... source_sha256=... -->`, the hash being
+    kernel_source_hash(unit) of the profiled kernel.  None when no summary
+    matches the current sources."""
     import glob
     import re
-    cur = kernel_source_hash()
+    cur = kernel_source_hash(unit)
     for p in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         with open(p) as f:
             for line in f:
@@ -99,7 +106,7 @@ for _b in (1, 8):
     _w = synth.moe_h2048(_b)
     WORKLOADS[_w.name] = _w
 for _w in (synth.attn_h5120(1, 4096), synth.attn_h5120(8, 4096), synth.attn_h5120(1, 32768),
-           synth.attn_h2048(8, 8192)):
+           synth.attn_h5120(1, 32768, layers=4), synth.attn_h2048(8, 8192)):
     WORKLOADS[_w.name] = _w
 for _f in (4, 8):
     for _b in (16, 32):
@@ -1078,7 +1085,9 @@ def main():
                          "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                          "peak_source": peaks["source"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4),
-                         "traffic": profiled_traffic(wl.name, args.engine),
+                         "traffic": profiled_traffic(wl.name, args.engine,
+                                                     "attention.cu" if is_attn else
+                                                     "verify_gemm.cu" if verify else "stream_gemv.cu"),
                          "bytes_per_launch": int(dom_bytes),
                          "launch_us": round(dom_s * 1e6, 3),
                          **({"isolated_launch": isolated} if isolated else {}),

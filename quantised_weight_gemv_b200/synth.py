@@ -254,10 +254,11 @@ class AttnWorkload:
         return seq_lens(key(seed, self.wid, 0, 0, KIND_LEN), self.B, self.Tmax)
 
 
-def attn_h5120(B: int, Tmax: int) -> AttnWorkload:
-    """The 64-layer hidden-5120 decoder's attention (40 query heads on 8 KV
-    heads), every sequence at Tmax positions."""
-    return AttnWorkload(11, f"attn64L-kv8-g5-t{Tmax}-b{B}", 64, B, 8, 5, Tmax)
+def attn_h5120(B: int, Tmax: int, layers: int = 64) -> AttnWorkload:
+    """The hidden-5120 decoder's attention (40 query heads on 8 KV heads),
+    every sequence at Tmax positions: all 64 layers, or the first `layers`
+    (a cache small enough for a many-pass profile)."""
+    return AttnWorkload(11, f"attn{layers}L-kv8-g5-t{Tmax}-b{B}", layers, B, 8, 5, Tmax)
 
 
 def attn_h2048(B: int, Tmax: int) -> AttnWorkload:
