@@ -660,7 +660,13 @@ extern "C" int32_t bq_attn_decode_q8(const bq_kv_cache *kv, const uint16_t *q, c
     a.Tmax = kv->Tmax;
     a.tps = kv->Tmax / at::TP;
     a.U = B * Hkv * a.tps;
-    a.nctas = std::min(std::min(a.U, 2 * sms), at::kMaxCtas);
+    // CTAs: two per SM when there are units enough.  Below that, one unit
+    // a CTA is not the fastest: a sequence's many CTA partials then cost
+    // more to merge than a second unit costs to compute, so such launches
+    // give every CTA two units (a sequence of one or two units is then one
+    // CTA's, with nothing to merge).
+    const int full = std::min(2 * sms, at::kMaxCtas);
+    a.nctas = a.U > full ? full : std::max(B * Hkv, (a.U + 1) / 2);
     a.s2_scale = scale * 1.4426950408889634f * 16777216.0f;
     a.counters = static_cast<int *>(ws);
     a.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) +
