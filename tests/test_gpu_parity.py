@@ -284,6 +284,32 @@ def test_moe_token_with_no_valid_slot_combines_to_zero():
     check_tol(y, y_ref, absy)
 
 
+@pytest.mark.parametrize("B", [1, 2])
+def test_moe_small_batch_combine(B):
+    """Combined outputs at batch 1-2: a token listing one expert twice, a token
+    with no valid slot (its row must be written as 0: the output starts NaN),
+    and the workspace all-zero again afterwards."""
+    import torch
+    N, K, topk, E = 96, 512, 4, 6
+    codes, scales, x, _, r = _moe_inputs(E, N, K, B, topk, 17 + B, False)
+    rows = [[5, 5, 0, 3], [-1, 6, 99, -2]][:B]
+    idx = np.array(rows, dtype=np.int32)
+    c, s = dev(codes), dev(scales)
+    y = torch.full((B, N), float("nan"), dtype=torch.float32, device=DEV)
+    ws = bq.workspace(bq.lib().bq_moe_workspace_bytes(N, K, B, topk, E), DEV)
+    st = new_status()
+    bq.moe_gemv_q4(bq.qmat(c, s, N, K), E, N * K // 2, N * scales.shape[2], dev(x), False,
+                   dev(idx), dev(r), y, ws, st)
+    torch.cuda.synchronize()
+    yn = y.cpu().numpy()
+    y_ref, absy, bad = oracle.moe_gemv_q4(codes, scales, x, False, idx, r)
+    assert int(st.item()) == (1 << bq.BQ_ERR_EXPERT_INDEX if bad else 0)
+    if B == 2:
+        assert np.all(yn[1] == 0.0)
+    check_tol(yn, y_ref, absy)
+    assert int(torch.count_nonzero(ws).item()) == 0
+
+
 def test_moe_single_expert_matches_dense():
     N, K, B = 200, 1024, 6
     codes, scales, x, _, _ = _moe_inputs(3, N, K, B, 1, 12, False)
