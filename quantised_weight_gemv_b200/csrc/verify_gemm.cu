@@ -225,20 +225,9 @@ __device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, float (&v)[16])
         v[i] = __uint_as_float(r[i]);
 }
 
-// 16 consecutive 32-bit TMEM columns of this thread's lane (32x32b shape: a
-// warp writes its 32 lanes), then wait until the warp's stores are done.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-        "%11, %12, %13, %14, %15, %16};"
-        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
-          "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-          "r"(v[15])
-        : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
+// 32 consecutive 32-bit TMEM columns of this thread's lane (32x32b shape: a
+// warp writes its 32 lanes); asynchronous: tmem_wait_st() waits for the
+// warp's stores.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
 {
     asm volatile(
@@ -251,6 +240,9 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
           "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
           "r"(v[29]), "r"(v[30]), "r"(v[31])
         : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st()
+{
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
@@ -624,8 +616,8 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
             __syncwarp();
             if (lane == 0)                                 // the slot may take a later segment's shifts
                 mbar_arrive(smem_u32(&bar_shift_free[seg % kShiftRing]));
-            if (!wait(bar_accfull[buf], (seg >> 1) & 1))
-                break;
+            if (!__all_sync(0xffffffffu, wait(bar_accfull[buf], (seg >> 1) & 1)))
+                break;                                     // (warp-uniform: tmem_ld is warp-collective)
             tc_fence_after();
             float v[NB];
             tmem_ld<NB>(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * 32), v);
@@ -779,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
             const float two_s = __int_as_float((127 + s) << 23);
             for (; u < uend && ok; u++, n++) {
                 const int cslot = n % CS;
-                if (!wait(bar_cfull[cslot], (n / CS) & 1)) {
+                if (!__all_sync(0xffffffffu, wait(bar_cfull[cslot], (n / CS) & 1))) {
                     ok = false;
                     break;
                 }
@@ -790,7 +782,9 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                     if (i % kDqGroups != grp)
                         continue;
                     const int slot = i % AS;
-                    if (!wait(bar_aempty[slot], ((i / AS) & 1) ^ 1)) {
+                    // (warp-uniform outcome: the TMEM stores and their wait are
+                    // warp-collective)
+                    if (!__all_sync(0xffffffffu, wait(bar_aempty[slot], ((i / AS) & 1) ^ 1))) {
                         ok = false;
                         break;
                     }
@@ -822,6 +816,10 @@ __global__ void __launch_bounds__(kThreads, 1) verify_gemm_kernel(const __grid_c
                     }
                     tmem_st32(lane_base + (uint32_t)(kAccCols + slot * kACols + 32 * h), o);
                 }
+                // one wait for the unit's stores (they overlap the next
+                // sub-stage's dequantisation; also on the way out, so none is
+                // in flight when the columns are freed), then the hand-off
+                tmem_wait_st();
                 if (!ok)
                     break;
                 tc_fence_before();
