@@ -297,3 +297,58 @@ def test_step_run_ex_rejects_negative_options():
     w = bq.bq_step_wait(0, -1, 0)
     assert bq.lib().bq_step_run_ex(ctypes.byref(info), fake, fake, 1 << 30, ctypes.byref(w),
                                    None, None) == bq.BQ_ERR_SHAPE
+
+
+def test_verify_and_attention_workspace_sizes():
+    f = bq.lib().bq_verify_workspace_bytes
+    assert f(0, 256, 8) == 0 and f(128, 48, 8) == 0 and f(128, 256, 0) == 0 and f(128, 256, 33) == 0
+    a, b = f(128, 4096, 32), f(24576, 4096, 32)
+    assert 0 < a < b
+    g = bq.lib().bq_attn_workspace_bytes
+    assert g(0, 8) == 0 and g(1, 0) == 0
+    assert 0 < g(1, 8) <= g(8, 8)
+
+
+def _verify_rc(fmt=4, W=None, x=FAKE, B=16, y=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    W = W if W is not None else bq.bq_qmat(FAKE, FAKE, 256, 512)
+    return bq.lib().bq_verify_gemm(fmt, ctypes.byref(W), x, B, y, ws, ws_bytes, None, None)
+
+
+def test_verify_gemm_argument_validation_before_launch():
+    """Every host-detectable error of bq_verify_gemm is returned before any
+    device call (fake pointers are never dereferenced)."""
+    assert bq.lib().bq_verify_gemm(4, None, FAKE, 16, FAKE, FAKE, 1 << 30, None, None) == bq.BQ_ERR_NULL
+    assert _verify_rc(W=bq.bq_qmat(None, FAKE, 256, 512)) == bq.BQ_ERR_NULL
+    assert _verify_rc(fmt=5) == bq.BQ_ERR_SHAPE                  # Q4 or Q8 only
+    assert _verify_rc(W=bq.bq_qmat(FAKE, FAKE, 256, 48)) == bq.BQ_ERR_SHAPE
+    assert _verify_rc(x=None) == bq.BQ_ERR_NULL
+    assert _verify_rc(ws=None) == bq.BQ_ERR_NULL
+    assert _verify_rc(B=0) == bq.BQ_ERR_BATCH
+    assert _verify_rc(B=33) == bq.BQ_ERR_BATCH
+    assert _verify_rc(y=FAKE + 4) == bq.BQ_ERR_ALIGN
+    assert _verify_rc(ws_bytes=1024) == bq.BQ_ERR_WORKSPACE
+
+
+def _attn_rc(kv=None, q=FAKE, lens=FAKE, B=2, Hkv=4, G=5, scale=0.088, o=FAKE, ws=FAKE,
+             ws_bytes=1 << 30):
+    kv = kv if kv is not None else bq.bq_kv_cache(FAKE, FAKE, FAKE, FAKE, 128, 1024)
+    return bq.lib().bq_attn_decode_q8(ctypes.byref(kv), q, lens, B, Hkv, G, scale, o, ws, ws_bytes,
+                                      None, None)
+
+
+def test_attention_argument_validation_before_launch():
+    """Every host-detectable error of bq_attn_decode_q8 is returned before any
+    device call: null planes, a head dimension other than 128, a cache length
+    that is not a multiple of 128 positions, G outside 1..8, a NaN scale, the
+    batch, 16-byte alignment and the workspace size."""
+    assert bq.lib().bq_attn_decode_q8(None, FAKE, FAKE, 2, 4, 5, 0.1, FAKE, FAKE, 1 << 30,
+                                      None, None) == bq.BQ_ERR_NULL
+    assert _attn_rc(kv=bq.bq_kv_cache(FAKE, None, FAKE, FAKE, 128, 1024)) == bq.BQ_ERR_NULL
+    assert _attn_rc(lens=None) == bq.BQ_ERR_NULL
+    assert _attn_rc(kv=bq.bq_kv_cache(FAKE, FAKE, FAKE, FAKE, 64, 1024)) == bq.BQ_ERR_SHAPE
+    assert _attn_rc(kv=bq.bq_kv_cache(FAKE, FAKE, FAKE, FAKE, 128, 1000)) == bq.BQ_ERR_SHAPE
+    assert _attn_rc(G=0) == bq.BQ_ERR_SHAPE and _attn_rc(G=9) == bq.BQ_ERR_SHAPE
+    assert _attn_rc(scale=float("nan")) == bq.BQ_ERR_SHAPE
+    assert _attn_rc(B=0) == bq.BQ_ERR_BATCH
+    assert _attn_rc(q=FAKE + 2) == bq.BQ_ERR_ALIGN
+    assert _attn_rc(ws_bytes=16) == bq.BQ_ERR_WORKSPACE
