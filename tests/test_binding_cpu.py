@@ -93,3 +93,52 @@ def test_moe_and_step_plan_refuse_host_tensors():
     with pytest.raises(ValueError, match="x must be a CUDA tensor"):
         bq.StepPlan(4, [(bq.qmat(c2, s2, N, K), torch.zeros((1, K), dtype=torch.float16),
                          _Dev(torch.zeros((1, N), dtype=torch.float32)), 0)], "cuda:0")
+
+
+def test_verify_gemm_refuses_host_tensors_and_wrong_shapes():
+    N, K, B = 256, 512, 16
+    c, s = _planes(4, N, K)
+    W = bq.qmat(c, s, N, K)
+    ws = _Dev(torch.zeros(1 << 20, dtype=torch.uint8))
+    y = _Dev(torch.zeros((B, N), dtype=torch.float32))
+    with pytest.raises(ValueError, match="x must be a CUDA tensor"):
+        bq.verify_gemm(4, W, torch.zeros((B, K), dtype=torch.float16), y, ws)
+    with pytest.raises(ValueError, match="x must be a contiguous"):
+        bq.verify_gemm(4, W, _Dev(torch.zeros((B, K + 32), dtype=torch.float16)), y, ws)
+    with pytest.raises(ValueError, match="y must be contiguous"):
+        bq.verify_gemm(4, W, _Dev(torch.zeros((B, K), dtype=torch.float16)),
+                       _Dev(torch.zeros((B, N - 1), dtype=torch.float32)), ws)
+    small = bq.qmat(*_planes(4, N, K, rows=N - 1), N, K)            # planes short of N rows
+    with pytest.raises(ValueError):
+        bq.verify_gemm(4, small, _Dev(torch.zeros((B, K), dtype=torch.float16)), y, ws)
+
+
+def _cache(B, Hkv, T, D=128):
+    return (_Dev(torch.zeros((B, Hkv, T, D), dtype=torch.int8)),
+            _Dev(torch.zeros((B, Hkv, T, D // 32), dtype=torch.int16)),
+            _Dev(torch.zeros((B, Hkv, D, T), dtype=torch.int8)),
+            _Dev(torch.zeros((B, Hkv, T, D // 32), dtype=torch.int16)))
+
+
+def test_attention_refuses_host_tensors_and_wrong_shapes():
+    B, Hkv, G, T, D = 2, 4, 5, 256, 128
+    kc, ks, vt, vs = _cache(B, Hkv, T)
+    with pytest.raises(ValueError, match="k_codes must be a CUDA tensor"):
+        bq.kv_cache(torch.zeros((B, Hkv, T, D), dtype=torch.int8), ks, vt, vs)
+    with pytest.raises(ValueError, match="do not match the cache layout"):
+        bq.kv_cache(kc, ks, _Dev(torch.zeros((B, Hkv, T, D), dtype=torch.int8)), vs)   # not transposed
+    kv = bq.kv_cache(kc, ks, vt, vs)
+    q = _Dev(torch.zeros((B, Hkv * G, D), dtype=torch.float16))
+    lens = _Dev(torch.zeros(B, dtype=torch.int32))
+    o = _Dev(torch.zeros((B, Hkv * G, D), dtype=torch.float32))
+    ws = _Dev(torch.zeros(1 << 20, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="q must be a CUDA tensor"):
+        bq.attn_decode_q8(kv, torch.zeros((B, Hkv * G, D), dtype=torch.float16), lens, G, 0.1, o, ws)
+    with pytest.raises(ValueError, match="q must be contiguous"):
+        bq.attn_decode_q8(kv, _Dev(torch.zeros((B, Hkv * (G + 1), D), dtype=torch.float16)), lens, G,
+                          0.1, o, ws)
+    with pytest.raises(ValueError, match="lens must be int32"):
+        bq.attn_decode_q8(kv, q, _Dev(torch.zeros(B, dtype=torch.int64)), G, 0.1, o, ws)
+    with pytest.raises(ValueError, match="o too small"):
+        bq.attn_decode_q8(kv, q, lens, G, 0.1, _Dev(torch.zeros((B, Hkv * G, D - 1),
+                                                               dtype=torch.float32)), ws)
