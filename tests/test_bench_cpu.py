@@ -81,3 +81,32 @@ def test_reference_arm_attention_workload():
     d = _reference_line("--workload", "attn16L-kv4-g4-t8192-b8-mixed", "--steps", "1")
     assert d["config"]["workload"] == "attn16L-kv4-g4-t8192-b8-mixed" and d["value"] > 0
     assert "layer 0" in d["cpu_baseline"]["sample"]
+
+
+def test_profile_traffic_markers_match_the_current_sources():
+    """Each `bench-traffic` marker under profiles/ (the DRAM bytes a bench line
+    reports as `roofline.traffic`) names a benchmark workload, the graph
+    engine, a positive byte count, and the hash of the kernel sources it was
+    captured on; every marker is for the current sources (a summary of an
+    earlier revision carries none), and the default workload has one."""
+    import glob
+    import re
+    import bench
+    found = {}
+    for p in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for line in open(p):
+            m = re.search(r"bench-traffic:(.*?)-->", line)
+            if not m:
+                continue
+            kv = dict(t.split("=", 1) for t in m.group(1).split() if "=" in t)
+            wl = kv["workload"]
+            assert wl in bench.WORKLOADS, (p, wl)
+            assert kv["engine"] == "graph", p
+            assert int(kv["bytes_per_launch"]) > 0, p
+            unit = ("attention.cu" if wl.startswith("attn") else
+                    "verify_gemm.cu" if wl.startswith("verify") else "stream_gemv.cu")
+            assert kv["source_sha256"] == bench.kernel_source_hash(unit), \
+                f"{os.path.basename(p)}: {unit} changed since this traffic was captured"
+            assert bench.profiled_traffic(wl, "graph", unit) == int(kv["bytes_per_launch"])
+            found[wl] = int(kv["bytes_per_launch"])
+    assert "dense64L-h5120-ffn25600-q4" in found
