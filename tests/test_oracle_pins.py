@@ -327,6 +327,61 @@ def test_golden_worked_block(name, fmt):
     assert a[0, 0] == float(g["abs_sum"][0])
 
 
+def _pack_from_format_text(fmt, q):
+    """The block layouts as each fixture's header states them, written out
+    independently of the oracle: 32 codes of one block -> its bytes."""
+    def plane2(vals):            # byte i: elements i, i+8, i+16, i+24 in bits 0-1 .. 6-7
+        return [vals[i] | vals[i + 8] << 2 | vals[i + 16] << 4 | vals[i + 24] << 6
+                for i in range(8)]
+
+    def nibbles(vals):           # byte i: element i low, element i+16 high
+        return [vals[i] | vals[i + 16] << 4 for i in range(16)]
+
+    def plane1(bits):            # byte i: element i + 4p in bit p
+        return [sum(bits[i + 4 * p] << p for p in range(8)) for i in range(4)]
+
+    if fmt == 2:
+        return plane2(q)
+    if fmt == 3:
+        return plane2([c & 3 for c in q]) + plane1([c >> 2 for c in q])
+    if fmt == 4:
+        return nibbles(q)
+    if fmt == 5:
+        return nibbles([c & 15 for c in q]) + plane1([c >> 4 for c in q])
+    if fmt == 6:
+        return nibbles([c & 15 for c in q]) + plane2([c >> 4 for c in q])
+    raise ValueError(fmt)
+
+
+@pytest.mark.parametrize("name,fmt", [("q2_block_worked.txt", 2), ("q3_block_worked.txt", 3),
+                                      ("q4_block_worked.txt", 4), ("q5_block_worked.txt", 5),
+                                      ("q6_block_worked.txt", 6), ("q8_block_worked.txt", 8)])
+def test_golden_worked_block_is_self_consistent(name, fmt):
+    """Each hand-derived fixture agrees with itself, without the oracle: the
+    codes are w/d plus the format's zero point, the largest |w/d| equals the
+    format's level count (so absmax / levels is the stated power of two), the
+    scale bits are that power of two in fp16, the packed bytes follow the
+    layout stated in the header, and y and sum |w x| are the exact sums."""
+    from fractions import Fraction
+    g = read_golden(name)
+    levels, zero = {2: (1, 2), 3: (3, 4), 4: (7, 8), 5: (15, 16), 6: (31, 32), 8: (127, 0)}[fmt]
+    v = [int(t) for t in g["w_over_d"]]
+    assert len(v) == 32 and int(g["N"][0]) == 1 and int(g["K"][0]) == 32
+    assert max(abs(t) for t in v) == levels and all(-levels - (fmt != 8) <= t <= levels for t in v)
+    q = [t + zero for t in v]
+    assert q == [int(t) for t in g["codes"]]
+    e = int(g["d_log2"][0])
+    assert -14 <= e <= 15 and int(g["scale_bits"][0], 16) == (e + 15) << 10   # normal fp16 2^e
+    if fmt != 8:
+        assert _pack_from_format_text(fmt, q) == [int(t, 16) for t in g["packed"]]
+        assert len(g["packed"]) == {2: 8, 3: 12, 4: 16, 5: 20, 6: 24}[fmt]
+    x = [Fraction(float(np.float16(t))) for t in g["x"]]
+    assert all(float(np.float16(t)) == float(t) for t in g["x"])             # x exact in fp16
+    d = Fraction(2) ** e
+    assert Fraction(g["y"][0]) == d * sum(vi * xi for vi, xi in zip(v, x))
+    assert Fraction(g["abs_sum"][0]) == d * sum(abs(vi * xi) for vi, xi in zip(v, x))
+
+
 # ---------------------------------------------------------- nibble order ----
 def test_q4_nibble_order_exhaustive():
     """Every (position, code) of a 1x32 block: element i < 16 lives in the low
