@@ -80,7 +80,8 @@ _SIGS = {
     "bq_gemv_q4_noalloc": (_i32, [_QP, _vp, _i32, _vp, _vp, _vp]),
     "bq_gemv_q4_noalloc_scratch": (_i32, [ctypes.POINTER(_vp), ctypes.POINTER(_sz)]),
     "bq_step_plan_bytes": (_sz, [_i32]),
-    "bq_gemv_geometry_of": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _vp]),
+    "bq_gemv_geometry_of": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32,
+                                    ctypes.POINTER(bq_gemv_geometry)]),
     "bq_step_plan": (_i32, [_i32, _SMP, _i32, _vp, _sz, _SIP]),
     "bq_step_run": (_i32, [_SIP, _vp, _vp, _sz, _vp, _vp]),
     "bq_step_run_ex": (_i32, [_SIP, _vp, _vp, _sz, ctypes.POINTER(bq_step_wait), _vp, _vp]),

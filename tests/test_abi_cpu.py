@@ -352,3 +352,94 @@ def test_attention_argument_validation_before_launch():
     assert _attn_rc(B=0) == bq.BQ_ERR_BATCH
     assert _attn_rc(q=FAKE + 2) == bq.BQ_ERR_ALIGN
     assert _attn_rc(ws_bytes=16) == bq.BQ_ERR_WORKSPACE
+
+
+def _prototypes():
+    """name -> (return type, [parameter types]) for every BQ_API function of
+    include/bq.h, comments removed and `const` dropped."""
+    with open(os.path.join(ROOT, "include", "bq.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    out = {}
+    for ret, name, params in re.findall(r"BQ_API\s+([^;(]*?)\b(bq_\w+)\s*\(([^)]*)\)\s*;", src):
+        def norm(t):
+            t = re.sub(r"\bconst\b", " ", t)
+            t = re.sub(r"\s*\*", " *", t)
+            return " ".join(t.split())
+        types = []
+        for p in params.split(","):
+            p = norm(p)
+            # drop the parameter name: the last identifier after the type
+            m = re.match(r"^(.*?)(\w+)$", p)
+            assert m, (name, p)
+            types.append(norm(m.group(1)))
+        out[name] = (norm(ret), types)
+    return out
+
+
+def _ctype_of(c):
+    scalars = {"int32_t": ctypes.c_int32, "int64_t": ctypes.c_int64, "uint64_t": ctypes.c_uint64,
+               "size_t": ctypes.c_size_t, "float": ctypes.c_float}
+    if c in scalars:
+        return scalars[c]
+    if c == "char *":
+        return ctypes.c_char_p
+    if c == "void * *":
+        return ctypes.POINTER(ctypes.c_void_p)
+    if c == "size_t *":
+        return ctypes.POINTER(ctypes.c_size_t)
+    m = re.match(r"^(bq_\w+) \*$", c)
+    if m:
+        return ctypes.POINTER(getattr(bq, m.group(1)))
+    assert c.endswith("*"), c
+    return ctypes.c_void_p
+
+
+def test_binding_signatures_match_the_header():
+    """Every ctypes signature the binding declares has the header's parameter
+    count, scalar widths and pointer kinds (a struct pointer as that struct),
+    so an argument can neither shift nor be truncated."""
+    protos = _prototypes()
+    assert set(protos) == set(_declared())
+    assert set(bq._SIGS) == set(protos), set(bq._SIGS) ^ set(protos)
+    for name, (ret, params) in protos.items():
+        res, args = bq._SIGS[name]
+        assert res == _ctype_of(ret), (name, ret, res)
+        assert len(args) == len(params), (name, params, args)
+        for i, (c, a) in enumerate(zip(params, args)):
+            assert a == _ctype_of(c), (name, i, c, a)
+
+
+def test_binding_structs_match_the_header_layout(tmp_path):
+    """Size and field offsets of every structure the binding mirrors, as gcc
+    lays them out from include/bq.h."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc") or shutil.which("cc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    structs = [bq.bq_qmat, bq.bq_step_mat, bq.bq_step_info, bq.bq_step_wait, bq.bq_kv_cache,
+               bq.bq_gemv_geometry]
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "bq.h"', "int main(void) {"]
+    for s in structs:
+        n = s.__name__
+        lines.append(f'printf("{n} sizeof %zu\\n", sizeof({n}));')
+        for f, _ in s._fields_:
+            lines.append(f'printf("{n} {f} %zu\\n", offsetof({n}, {f}));')
+    lines += ["return 0;", "}"]
+    c = tmp_path / "layout.c"
+    c.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([gcc, "-std=c11", "-I", os.path.join(ROOT, "include"), str(c), "-o", str(exe)],
+                   check=True, capture_output=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n"):
+        if line:
+            n, f, v = line.split()
+            got[(n, f)] = int(v)
+    for s in structs:
+        n = s.__name__
+        assert got[(n, "sizeof")] == ctypes.sizeof(s), n
+        for f, _ in s._fields_:
+            assert got[(n, f)] == getattr(s, f).offset, (n, f)
