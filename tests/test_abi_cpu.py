@@ -238,6 +238,18 @@ def test_product_path_has_no_oracle_or_fallback():
                 assert "oracle.c" not in src and "liboracle" not in src, fn
 
 
+def test_binding_raises_when_the_library_is_missing(monkeypatch, tmp_path):
+    """No fallback: with libbq.so absent, loading it and every wrapper raise."""
+    monkeypatch.setattr(bq, "_lib", None)
+    monkeypatch.setattr(bq, "LIB_PATH", str(tmp_path / "libbq.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        bq.lib()
+    with pytest.raises(RuntimeError, match="missing"):
+        bq.bq_scales_ld(256)
+    with pytest.raises(RuntimeError, match="missing"):
+        bq.lib().bq_gemv_workspace_bytes(64, 256)
+
+
 def test_oracle_shares_nothing_with_the_library():
     """The oracle is plain C over the C standard library: it includes no header
     of the package or the CUDA toolkit, and its Python wrapper imports nothing
