@@ -42,7 +42,8 @@ def test_double_to_half_vs_numpy_rne():
     ])
     vals = np.concatenate([vals, -vals])
     ours = oracle.double_to_half(vals)
-    ref = vals.astype(np.float16).view(np.uint16)
+    with np.errstate(over="ignore"):          # overflow to inf is one of the cases checked
+        ref = vals.astype(np.float16).view(np.uint16)
     assert np.array_equal(ours, ref)
 
 
