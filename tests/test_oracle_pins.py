@@ -329,29 +329,13 @@ def test_golden_worked_block(name, fmt):
 
 
 def _pack_from_format_text(fmt, q):
-    """The block layouts as each fixture's header states them, written out
-    independently of the oracle: 32 codes of one block -> its bytes."""
-    def plane2(vals):            # byte i: elements i, i+8, i+16, i+24 in bits 0-1 .. 6-7
-        return [vals[i] | vals[i + 8] << 2 | vals[i + 16] << 4 | vals[i + 24] << 6
-                for i in range(8)]
-
-    def nibbles(vals):           # byte i: element i low, element i+16 high
-        return [vals[i] | vals[i + 16] << 4 for i in range(16)]
-
-    def plane1(bits):            # byte i: element i + 4p in bit p
-        return [sum(bits[i + 4 * p] << p for p in range(8)) for i in range(4)]
-
-    if fmt == 2:
-        return plane2(q)
-    if fmt == 3:
-        return plane2([c & 3 for c in q]) + plane1([c >> 2 for c in q])
+    """32 codes of one block -> its bytes, by the plane packers above (written
+    from the format text, independent of the oracle)."""
+    b = np.array(q, dtype=np.int64).reshape(1, 1, 32)
     if fmt == 4:
-        return nibbles(q)
-    if fmt == 5:
-        return nibbles([c & 15 for c in q]) + plane1([c >> 4 for c in q])
-    if fmt == 6:
-        return nibbles([c & 15 for c in q]) + plane2([c >> 4 for c in q])
-    raise ValueError(fmt)
+        return [int(c) for c in (b[0, 0, :16] | (b[0, 0, 16:] << 4))]
+    pack = {2: _q2_planes, 3: _q3_planes, 5: _q5_planes, 6: _q6_planes}[fmt]
+    return [int(c) for c in pack(b)[0]]
 
 
 @pytest.mark.parametrize("name,fmt", [("q2_block_worked.txt", 2), ("q3_block_worked.txt", 3),
