@@ -1,12 +1,16 @@
 """Decode-step benchmark of the block-quantised weight GEMV on B200.
 
 One step = one decode token through the whole weight stream of the workload:
-every layer's projections in model order (q|k|v, o, gate|up, down), each a Q4
-GEMV with dequantisation in the inner loop.  Default workload: 16-layer dense
-decoder, hidden 2048, FFN 8192, Q4, batch 1 (547 MB of packed weights per step,
-> L2, so no L2 flush is needed).  Weights and activations are synthetic
-(seeded N(0, 0.02) weights, N(0, 1) fp16 activations), generated and quantised
-on the device.
+every layer's projections in model order (q|k|v, o, gate|up with the SwiGLU
+epilogue, down), each a GEMV with dequantisation in the inner loop, launched as
+one CUDA graph of dependent launches.  Default workload: 64-layer dense decoder,
+hidden 5120, FFN 25600, Q4, batch 1 (16.4 GB of packed weights per step, far
+above the L2, so no flush is needed).  Other workloads (--workload): the
+16-layer hidden-2048 and 36-layer hidden-4096 decoders in every format and
+batch, matrix-shape sweeps, routed experts, the batched-verification step on
+the tensor cores, and decode attention over a Q8 KV cache.  Weights and
+activations are synthetic (seeded N(0, 0.02) weights, N(0, 1) fp16
+activations), generated and quantised on the device.
 
 Prints ONE JSON line (rank 0).  `value` = algorithmic bytes (packed codes +
 scales + x + y) of all ranks per second of the slowest rank; tokens/s-equiv =
