@@ -110,3 +110,14 @@ def test_profile_traffic_markers_match_the_current_sources():
             assert bench.profiled_traffic(wl, "graph", unit) == int(kv["bytes_per_launch"])
             found[wl] = int(kv["bytes_per_launch"])
     assert "dense64L-h5120-ffn25600-q4" in found
+
+
+@pytest.mark.parametrize("workload", ["moe48L-e128-top8-h2048-b1", "moe48L-e128-top8-h2048-b8"])
+def test_reference_arm_routed_experts(workload):
+    """The oracle arm on the routed-expert workload: layer 0's routed experts
+    (gate|up with SwiGLU, then down combined in slot order) per step."""
+    d = _reference_line("--workload", workload)
+    assert d["config"]["workload"] == workload and d["value"] > 0
+    assert d["config"]["sample"] == "one layer per step"
+    assert "layer 0" in d["cpu_baseline"]["sample"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0
